@@ -1,0 +1,169 @@
+/*
+ * ssd.h -- C ABI of libssd_b200.so, a B200 (sm_100a) implementation of the
+ * SSD (structured state space duality) layer of Mamba-2.
+ *
+ * The layer (scalar-times-identity A per head, input-dependent dt, B, C):
+ *
+ *     h_t = exp(dt_t * A_h) * h_{t-1} + dt_t * x_t B_t^T        (P x N state per head)
+ *     y_t = h_t C_t + D_h * x_t
+ *
+ * "论文解读：Mamba: Linear-Time Sequence Modeling with Selective State Spaces",
+ * section 状态空间模型: discretise (Delta, A, B) and run the model as a linear
+ * recurrence; section 选择性状态空间模型: dt, B, C vary per token.
+ * "Transformers are SSMs" (CiteArk), AI research summary: the same map is a
+ * 1-semiseparable matrix, evaluated by a block-decomposed matrix-multiply
+ * algorithm on the tensor cores; "what this means": the recurrent form gives
+ * constant-memory inference (ssd_step below).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Every tensor pointer is a DEVICE pointer (cudaMalloc'd or equivalent),
+ *    dense, row-major and contiguous, and 16-byte aligned.  The caller owns
+ *    all memory, including the workspace; the library never allocates.
+ *  - Layouts (b = batch, L = seqlen, H = nheads, P = headdim, N = dstate,
+ *    G = ngroups, T = ceil(L / chunk_size)):
+ *        x, y            (b, L, H, P)   element type = dtype
+ *        dt              (b, L, H)      fp32, already positive (no softplus is applied)
+ *        A, D            (H)            fp32
+ *        B, C            (b, L, G, N)   element type = dtype
+ *        states          (b, H, P, N)   fp32 (init_states, final_states, ssd_step's state)
+ *    Head h reads B/C group g = h / (H / G).
+ *  - dtype: SSD_F32 (all fp32; exact fp32 arithmetic) or SSD_BF16 (x, B, C, y
+ *    in bf16; products on the tensor cores with fp32 accumulation; decays,
+ *    prefix sums, the inter-chunk recurrence and all states in fp32).
+ *  - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *    stream) and runs asynchronously: no call synchronises the device.
+ *  - Errors: arguments are validated on the host before anything is
+ *    launched; a rejected call launches nothing and writes nothing.  A
+ *    failed launch returns SSD_ERR_CUDA (the CUDA error text is available
+ *    from ssd_last_error_detail()).  Asynchronous device errors surface at
+ *    the caller's next synchronisation, as with any CUDA library.
+ *  - Thread safety: calls may be made from several host threads on
+ *    different streams; calls that share a workspace must not overlap.
+ */
+#ifndef SSD_B200_H
+#define SSD_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SSD_API __attribute__((visibility("default")))
+#else
+#define SSD_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SSD_OK = 0,
+    SSD_ERR_INVALID_ARG = 1,  /* null pointer, bad size, misalignment, too-small workspace */
+    SSD_ERR_UNSUPPORTED = 2,  /* well-formed but outside what the kernels implement */
+    SSD_ERR_CUDA = 3,         /* a CUDA runtime/driver call or a launch failed */
+    SSD_ERR_TIMEOUT = 4       /* reserved: a bounded device-side wait gave up */
+} ssd_status_t;
+
+typedef enum { SSD_F32 = 0, SSD_BF16 = 1 } ssd_dtype_t;
+
+typedef struct {
+    int64_t batch;    /* b >= 0 */
+    int64_t seqlen;   /* L >= 0 (any value; a last partial chunk is handled) */
+    int64_t nheads;   /* H >= 1 */
+    int64_t headdim;  /* P, 1..256 */
+    int64_t dstate;   /* N, 1..256 */
+    int64_t ngroups;  /* G >= 1, H % G == 0 */
+} ssd_dims_t;
+
+/* Human-readable name of a status code (static storage). */
+SSD_API const char* ssd_status_string(ssd_status_t s);
+
+/* Detail of the last error raised on the calling host thread (validation
+ * message or CUDA error text); "" if none.  Thread-local static storage. */
+SSD_API const char* ssd_last_error_detail(void);
+
+/*
+ * Bytes of device workspace ssd_chunk_scan_fwd needs for these sizes
+ * (chunk states, per-chunk log-decays and the states entering each chunk).
+ * Writes the size to *bytes.  Returns SSD_ERR_INVALID_ARG / UNSUPPORTED on
+ * sizes that ssd_chunk_scan_fwd would reject.
+ */
+SSD_API ssd_status_t ssd_chunk_scan_fwd_workspace_size(const ssd_dims_t* dims, int chunk_size,
+                                               ssd_dtype_t dtype, size_t* bytes);
+
+/*
+ * Chunked (block-decomposed) SSD forward over whole sequences.
+ * "Transformers are SSMs" (CiteArk), AI research summary: block-decomposed
+ * matrix multiplication of the 1-semiseparable matrix; review page
+ * "Review: Transformers are SSMs (Mamba-2)", 核心概念 item 5 (SSD algorithm:
+ * block decomposition that uses the tensor cores and stays linear in L).
+ * The sequence is cut into chunks of `chunk_size` tokens (a power of two,
+ * 16..256; the last chunk may be partial).  Four steps:
+ *   (1) per chunk, the intra-chunk quadratic term (C B^T masked by the
+ *       exp(segsum(dt*A)) decay) applied to dt*x;
+ *   (2) per chunk, the state it contributes, B^T (decay * dt * x);
+ *   (3) the sequential recurrence of states across chunks (fp32);
+ *   (4) the contribution of the entering state, C * h, plus D_h * x.
+ * init_states: (b,H,P,N) fp32, or NULL for zero initial states.
+ * final_states: (b,H,P,N) fp32 output, or NULL when not wanted.
+ * y: (b,L,H,P) output in dtype.  workspace: >= the size reported by
+ * ssd_chunk_scan_fwd_workspace_size (may be NULL only when that size is 0).
+ * Inputs and outputs must not alias.
+ */
+SSD_API ssd_status_t ssd_chunk_scan_fwd(const void* x, const float* dt, const float* A, const void* B,
+                                const void* C, const float* D, int chunk_size,
+                                const float* init_states, void* y, float* final_states,
+                                const ssd_dims_t* dims, ssd_dtype_t dtype, void* workspace,
+                                size_t workspace_bytes, void* stream);
+
+/*
+ * One decode step for a batch of sequences (the recurrent, constant-memory
+ * form: "Transformers are SSMs" (CiteArk), "what this means"; Mamba digest,
+ * 状态空间模型: the linear-recurrence mode suited to autoregressive inference).
+ *   state (b,H,P,N) fp32, updated in place:  state <- exp(dt*A_h) state + dt x B^T
+ *   y (b,H,P) in dtype:                      y = state C + D_h x
+ * x (b,H,P) dtype; dt (b,H) fp32; B, C (b,G,N) dtype; A, D (H) fp32.
+ * dims->seqlen is ignored.
+ */
+SSD_API ssd_status_t ssd_step(float* state, const void* x, const float* dt, const float* A,
+                      const void* B, const void* C, const float* D, void* y,
+                      const ssd_dims_t* dims, ssd_dtype_t dtype, void* stream);
+
+/*
+ * The forward's steps one at a time (the same kernels ssd_chunk_scan_fwd
+ * launches), for testing each step on its own.  T = ceil(L / chunk_size).
+ *
+ * ssd_chunk_state_fwd -- step (2): chunk_states (b,T,H,P,N) fp32 receives, for
+ *   every chunk, the state reached at the chunk's last token when the state
+ *   at the chunk's start is zero; chunk_logdecay (b,T,H) fp32 receives
+ *   sum_{t in chunk} dt_t * A_h.
+ * ssd_state_passing_fwd -- step (3): prev_states (b,T,H,P,N) in dtype
+ *   receives the state entering each chunk (h before the chunk's first
+ *   token), computed in fp32 as h_c = exp(logdecay_c) h_{c-1} + S_c from
+ *   init_states (NULL = zero); final_states (nullable) receives the state
+ *   after the last chunk.
+ * ssd_chunk_output_fwd -- steps (1) and (4): y from x, dt, A, B, C, D and
+ *   prev_states (as written by ssd_state_passing_fwd).
+ */
+SSD_API ssd_status_t ssd_chunk_state_fwd(const void* x, const float* dt, const float* A, const void* B,
+                                 int chunk_size, float* chunk_states, float* chunk_logdecay,
+                                 const ssd_dims_t* dims, ssd_dtype_t dtype, void* stream);
+SSD_API ssd_status_t ssd_state_passing_fwd(const float* chunk_states, const float* chunk_logdecay,
+                                   const float* init_states, void* prev_states,
+                                   float* final_states, int chunk_size, const ssd_dims_t* dims,
+                                   ssd_dtype_t dtype, void* stream);
+SSD_API ssd_status_t ssd_chunk_output_fwd(const void* x, const float* dt, const float* A, const void* B,
+                                  const void* C, const float* D, const void* prev_states,
+                                  int chunk_size, void* y, const ssd_dims_t* dims,
+                                  ssd_dtype_t dtype, void* stream);
+
+/* Which kernel family ssd_chunk_scan_fwd uses for these sizes:
+ * 1 = tcgen05 tensor-core kernels, 0 = SIMT fp32 kernels, -1 = rejected. */
+SSD_API int ssd_chunk_scan_fwd_uses_tensor_cores(const ssd_dims_t* dims, int chunk_size,
+                                         ssd_dtype_t dtype);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SSD_B200_H */

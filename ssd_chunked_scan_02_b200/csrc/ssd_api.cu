@@ -1,0 +1,256 @@
+// ssd_api.cu -- the C ABI declared in include/ssd.h: host-side validation,
+// workspace layout, kernel selection and launches.  Nothing here allocates
+// device memory or synchronises the device.
+#include <cuda_runtime.h>
+#include <stdarg.h>
+#include <stdint.h>
+#include <stdio.h>
+
+#include "../../include/ssd.h"
+#include "ssd_internal.h"
+#include "tc_kernels.h"
+
+namespace {
+
+thread_local char g_detail[512] = "";
+
+ssd_status_t fail(ssd_status_t s, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_detail, sizeof(g_detail), fmt, ap);
+    va_end(ap);
+    return s;
+}
+
+ssd_status_t cuda_fail(cudaError_t e, const char* where) {
+    return fail(SSD_ERR_CUDA, "%s: %s (%s)", where, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+size_t elt_size(ssd::Elt t) { return t == ssd::Elt::F32 ? 4 : 2; }
+
+// Validates sizes; fills `out`.  need_chunk: chunk_size is meaningful.
+ssd_status_t check_dims(const ssd_dims_t* dims, int chunk, bool need_chunk, ssd_dtype_t dtype,
+                        ssd::Dims* out, ssd::Elt* elt) {
+    if (!dims) return fail(SSD_ERR_INVALID_ARG, "dims is NULL");
+    const ssd_dims_t& d = *dims;
+    if (d.batch < 0 || d.seqlen < 0)
+        return fail(SSD_ERR_INVALID_ARG, "batch (%lld) and seqlen (%lld) must be >= 0",
+                    (long long)d.batch, (long long)d.seqlen);
+    if (d.nheads < 1 || d.headdim < 1 || d.dstate < 1 || d.ngroups < 1)
+        return fail(SSD_ERR_INVALID_ARG, "nheads, headdim, dstate, ngroups must be >= 1");
+    if (d.nheads % d.ngroups != 0)
+        return fail(SSD_ERR_INVALID_ARG, "nheads (%lld) must be a multiple of ngroups (%lld)",
+                    (long long)d.nheads, (long long)d.ngroups);
+    if (d.headdim > 256 || d.dstate > 256)
+        return fail(SSD_ERR_UNSUPPORTED, "headdim and dstate must be <= 256");
+    if (d.nheads > 65535) return fail(SSD_ERR_UNSUPPORTED, "nheads must be <= 65535");
+    if (dtype != SSD_F32 && dtype != SSD_BF16)
+        return fail(SSD_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
+    int Q = 1;
+    if (need_chunk) {
+        if (chunk < 16 || chunk > 256 || (chunk & (chunk - 1)) != 0)
+            return fail(SSD_ERR_UNSUPPORTED, "chunk_size must be a power of two in [16, 256], got %d",
+                        chunk);
+        Q = chunk;
+    }
+    const int64_t T = need_chunk ? (d.seqlen + Q - 1) / Q : 1;
+    if (d.batch * T > 0x7fffffffLL)
+        return fail(SSD_ERR_UNSUPPORTED, "batch * number of chunks exceeds 2^31 - 1");
+    out->b = d.batch; out->L = d.seqlen; out->H = d.nheads; out->P = d.headdim;
+    out->N = d.dstate; out->G = d.ngroups; out->Q = Q; out->T = T;
+    *elt = dtype == SSD_F32 ? ssd::Elt::F32 : ssd::Elt::BF16;
+    return SSD_OK;
+}
+
+struct WsLayout {
+    size_t states, logdecay, prev, total;
+};
+
+WsLayout ws_layout(const ssd::Dims& d, ssd::Elt t) {
+    const size_t nstate = (size_t)(d.b * d.T * d.H) * (size_t)(d.P * d.N);
+    WsLayout w;
+    w.states = 0;
+    w.logdecay = round_up(nstate * 4, 256);
+    w.prev = w.logdecay + round_up((size_t)(d.b * d.T * d.H) * 4, 256);
+    w.total = w.prev + round_up(nstate * elt_size(t), 256);
+    if (nstate == 0) w.total = 0;
+    return w;
+}
+
+#define REQUIRE_PTR(p)                                                                   \
+    do {                                                                                 \
+        if (!(p)) return fail(SSD_ERR_INVALID_ARG, "%s is NULL", #p);                    \
+        if (!aligned16(p)) return fail(SSD_ERR_INVALID_ARG, "%s is not 16-byte aligned", #p); \
+    } while (0)
+#define OPTIONAL_PTR(p)                                                                  \
+    do {                                                                                 \
+        if ((p) && !aligned16(p))                                                        \
+            return fail(SSD_ERR_INVALID_ARG, "%s is not 16-byte aligned", #p);           \
+    } while (0)
+
+bool tc_eligible(const ssd::Dims& d, ssd::Elt t) { return ssd::tc_supported(d, t); }
+
+}  // namespace
+
+extern "C" {
+
+const char* ssd_status_string(ssd_status_t s) {
+    switch (s) {
+        case SSD_OK: return "SSD_OK";
+        case SSD_ERR_INVALID_ARG: return "SSD_ERR_INVALID_ARG";
+        case SSD_ERR_UNSUPPORTED: return "SSD_ERR_UNSUPPORTED";
+        case SSD_ERR_CUDA: return "SSD_ERR_CUDA";
+        case SSD_ERR_TIMEOUT: return "SSD_ERR_TIMEOUT";
+    }
+    return "SSD_ERR_UNKNOWN";
+}
+
+const char* ssd_last_error_detail(void) { return g_detail; }
+
+ssd_status_t ssd_chunk_scan_fwd_workspace_size(const ssd_dims_t* dims, int chunk_size,
+                                               ssd_dtype_t dtype, size_t* bytes) {
+    g_detail[0] = 0;
+    if (!bytes) return fail(SSD_ERR_INVALID_ARG, "bytes is NULL");
+    ssd::Dims d; ssd::Elt t;
+    ssd_status_t st = check_dims(dims, chunk_size, true, dtype, &d, &t);
+    if (st != SSD_OK) return st;
+    *bytes = ws_layout(d, t).total;
+    return SSD_OK;
+}
+
+int ssd_chunk_scan_fwd_uses_tensor_cores(const ssd_dims_t* dims, int chunk_size,
+                                         ssd_dtype_t dtype) {
+    ssd::Dims d; ssd::Elt t;
+    if (check_dims(dims, chunk_size, true, dtype, &d, &t) != SSD_OK) return -1;
+    return tc_eligible(d, t) ? 1 : 0;
+}
+
+ssd_status_t ssd_chunk_scan_fwd(const void* x, const float* dt, const float* A, const void* B,
+                                const void* C, const float* D, int chunk_size,
+                                const float* init_states, void* y, float* final_states,
+                                const ssd_dims_t* dims, ssd_dtype_t dtype, void* workspace,
+                                size_t workspace_bytes, void* stream) {
+    g_detail[0] = 0;
+    ssd::Dims d; ssd::Elt t;
+    ssd_status_t st = check_dims(dims, chunk_size, true, dtype, &d, &t);
+    if (st != SSD_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    OPTIONAL_PTR(init_states);
+    OPTIONAL_PTR(final_states);
+    if (d.b == 0) return SSD_OK;
+    if (d.L == 0) {
+        if (!final_states) return SSD_OK;
+        cudaError_t e = ssd::launch_copy_or_zero(init_states, final_states, d.b * d.H * d.P * d.N, s);
+        return e == cudaSuccess ? SSD_OK : cuda_fail(e, "final-state copy");
+    }
+    REQUIRE_PTR(x); REQUIRE_PTR(dt); REQUIRE_PTR(A); REQUIRE_PTR(B); REQUIRE_PTR(C);
+    REQUIRE_PTR(D); REQUIRE_PTR(y);
+    const WsLayout w = ws_layout(d, t);
+    if (workspace_bytes < w.total)
+        return fail(SSD_ERR_INVALID_ARG, "workspace too small: %zu bytes given, %zu needed",
+                    workspace_bytes, w.total);
+    REQUIRE_PTR(workspace);
+    if (!aligned16(workspace)) return fail(SSD_ERR_INVALID_ARG, "workspace not 16-byte aligned");
+    char* ws = static_cast<char*>(workspace);
+    float* states = reinterpret_cast<float*>(ws + w.states);
+    float* logdecay = reinterpret_cast<float*>(ws + w.logdecay);
+    void* prev = ws + w.prev;
+
+    cudaError_t e;
+    if (tc_eligible(d, t)) {
+        e = ssd::launch_chunk_state_tc(x, dt, A, B, states, logdecay, d, s);
+        if (e != cudaSuccess) return cuda_fail(e, "chunk-state kernel (tcgen05)");
+        e = ssd::launch_state_pass(states, logdecay, init_states, prev, final_states, d, t, s);
+        if (e != cudaSuccess) return cuda_fail(e, "state-passing kernel");
+        e = ssd::launch_chunk_out_tc(x, dt, A, B, C, D, prev, y, d, s);
+        if (e != cudaSuccess) return cuda_fail(e, "chunk-output kernel (tcgen05)");
+        return SSD_OK;
+    }
+    e = ssd::launch_chunk_state_simt(x, dt, A, B, states, logdecay, d, t, s);
+    if (e != cudaSuccess) return cuda_fail(e, "chunk-state kernel");
+    e = ssd::launch_state_pass(states, logdecay, init_states, prev, final_states, d, t, s);
+    if (e != cudaSuccess) return cuda_fail(e, "state-passing kernel");
+    e = ssd::launch_chunk_out_simt(x, dt, A, B, C, D, prev, y, d, t, s);
+    if (e != cudaSuccess) return cuda_fail(e, "chunk-output kernel");
+    return SSD_OK;
+}
+
+ssd_status_t ssd_chunk_state_fwd(const void* x, const float* dt, const float* A, const void* B,
+                                 int chunk_size, float* chunk_states, float* chunk_logdecay,
+                                 const ssd_dims_t* dims, ssd_dtype_t dtype, void* stream) {
+    g_detail[0] = 0;
+    ssd::Dims d; ssd::Elt t;
+    ssd_status_t st = check_dims(dims, chunk_size, true, dtype, &d, &t);
+    if (st != SSD_OK) return st;
+    if (d.b == 0 || d.L == 0) return SSD_OK;
+    REQUIRE_PTR(x); REQUIRE_PTR(dt); REQUIRE_PTR(A); REQUIRE_PTR(B);
+    REQUIRE_PTR(chunk_states); REQUIRE_PTR(chunk_logdecay);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = tc_eligible(d, t)
+                        ? ssd::launch_chunk_state_tc(x, dt, A, B, chunk_states, chunk_logdecay, d, s)
+                        : ssd::launch_chunk_state_simt(x, dt, A, B, chunk_states, chunk_logdecay,
+                                                       d, t, s);
+    return e == cudaSuccess ? SSD_OK : cuda_fail(e, "chunk-state kernel");
+}
+
+ssd_status_t ssd_state_passing_fwd(const float* chunk_states, const float* chunk_logdecay,
+                                   const float* init_states, void* prev_states,
+                                   float* final_states, int chunk_size, const ssd_dims_t* dims,
+                                   ssd_dtype_t dtype, void* stream) {
+    g_detail[0] = 0;
+    ssd::Dims d; ssd::Elt t;
+    ssd_status_t st = check_dims(dims, chunk_size, true, dtype, &d, &t);
+    if (st != SSD_OK) return st;
+    OPTIONAL_PTR(init_states);
+    OPTIONAL_PTR(final_states);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (d.b == 0) return SSD_OK;
+    if (d.L == 0) {
+        if (!final_states) return SSD_OK;
+        cudaError_t e = ssd::launch_copy_or_zero(init_states, final_states, d.b * d.H * d.P * d.N, s);
+        return e == cudaSuccess ? SSD_OK : cuda_fail(e, "final-state copy");
+    }
+    REQUIRE_PTR(chunk_states); REQUIRE_PTR(chunk_logdecay); REQUIRE_PTR(prev_states);
+    cudaError_t e = ssd::launch_state_pass(chunk_states, chunk_logdecay, init_states, prev_states,
+                                           final_states, d, t, s);
+    return e == cudaSuccess ? SSD_OK : cuda_fail(e, "state-passing kernel");
+}
+
+ssd_status_t ssd_chunk_output_fwd(const void* x, const float* dt, const float* A, const void* B,
+                                  const void* C, const float* D, const void* prev_states,
+                                  int chunk_size, void* y, const ssd_dims_t* dims,
+                                  ssd_dtype_t dtype, void* stream) {
+    g_detail[0] = 0;
+    ssd::Dims d; ssd::Elt t;
+    ssd_status_t st = check_dims(dims, chunk_size, true, dtype, &d, &t);
+    if (st != SSD_OK) return st;
+    if (d.b == 0 || d.L == 0) return SSD_OK;
+    REQUIRE_PTR(x); REQUIRE_PTR(dt); REQUIRE_PTR(A); REQUIRE_PTR(B); REQUIRE_PTR(C);
+    REQUIRE_PTR(D); REQUIRE_PTR(prev_states); REQUIRE_PTR(y);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = tc_eligible(d, t)
+                        ? ssd::launch_chunk_out_tc(x, dt, A, B, C, D, prev_states, y, d, s)
+                        : ssd::launch_chunk_out_simt(x, dt, A, B, C, D, prev_states, y, d, t, s);
+    return e == cudaSuccess ? SSD_OK : cuda_fail(e, "chunk-output kernel");
+}
+
+ssd_status_t ssd_step(float* state, const void* x, const float* dt, const float* A,
+                      const void* B, const void* C, const float* D, void* y,
+                      const ssd_dims_t* dims, ssd_dtype_t dtype, void* stream) {
+    g_detail[0] = 0;
+    ssd::Dims d; ssd::Elt t;
+    ssd_status_t st = check_dims(dims, 0, false, dtype, &d, &t);
+    if (st != SSD_OK) return st;
+    if (d.b == 0) return SSD_OK;
+    REQUIRE_PTR(state); REQUIRE_PTR(x); REQUIRE_PTR(dt); REQUIRE_PTR(A); REQUIRE_PTR(B);
+    REQUIRE_PTR(C); REQUIRE_PTR(D); REQUIRE_PTR(y);
+    cudaError_t e = ssd::launch_step(state, x, dt, A, B, C, D, y, d, t,
+                                     static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? SSD_OK : cuda_fail(e, "decode-step kernel");
+}
+
+}  // extern "C"

@@ -1,0 +1,39 @@
+// ssd_internal.h -- launchers shared between the C-ABI layer and the kernels.
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace ssd {
+
+struct Dims {
+    int64_t b, L, H, P, N, G;
+    int Q;        // chunk size
+    int64_t T;    // number of chunks = ceil(L / Q)
+};
+
+// Element type of x, B, C, y and the prev-state buffer.
+enum class Elt { F32 = 0, BF16 = 1 };
+
+// SIMT kernels (exact fp32 arithmetic; any supported size).
+cudaError_t launch_chunk_state_simt(const void* x, const float* dt, const float* A, const void* B,
+                                    float* states, float* logdecay, const Dims& d, Elt t,
+                                    cudaStream_t s);
+cudaError_t launch_chunk_out_simt(const void* x, const float* dt, const float* A, const void* B,
+                                  const void* C, const float* D, const void* prev, void* y,
+                                  const Dims& d, Elt t, cudaStream_t s);
+
+// Inter-chunk recurrence (fp32), writes prev states in `t` and the final state.
+cudaError_t launch_state_pass(const float* states, const float* logdecay, const float* init,
+                              void* prev, float* final_states, const Dims& d, Elt t,
+                              cudaStream_t s);
+
+// Decode step.
+cudaError_t launch_step(float* state, const void* x, const float* dt, const float* A,
+                        const void* B, const void* C, const float* D, void* y, const Dims& d,
+                        Elt t, cudaStream_t s);
+
+// Copies init (or zeros) into final: the L == 0 case.
+cudaError_t launch_copy_or_zero(const float* init, float* final_states, int64_t n,
+                                cudaStream_t s);
+
+}  // namespace ssd

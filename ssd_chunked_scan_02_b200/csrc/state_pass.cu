@@ -1,0 +1,137 @@
+// state_pass.cu -- the sequential inter-chunk state recurrence (step 3 of the
+// block-decomposed SSD forward), in fp32:
+//     h_{-1} = init (or 0),   prev_c = h_{c-1},   h_c = exp(logdecay_c) h_{c-1} + S_c
+// where S_c is the chunk's own state (chunk started from zero) and logdecay_c
+// = sum_{t in chunk c} dt_t A_h.  "论文解读：Mamba: ...", 状态空间模型: the
+// linear-recurrence form, here taken one chunk per step instead of one token.
+//
+// Every (batch, head, p, n) state element is an independent chain; a thread
+// owns VEC consecutive elements (16-byte fp32 loads), walks the chunks in
+// order and keeps the chain in registers.  Loads of later chunks do not
+// depend on the chain, so the unrolled loop keeps several in flight.
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "ssd_internal.h"
+
+namespace ssd {
+namespace {
+
+template <typename TP, int VEC>
+struct Store;
+template <int VEC>
+struct Store<float, VEC> {
+    static __device__ __forceinline__ void run(float* dst, const float* v) {
+        if constexpr (VEC == 4) {
+            *reinterpret_cast<float4*>(dst) = make_float4(v[0], v[1], v[2], v[3]);
+        } else {
+#pragma unroll
+            for (int k = 0; k < VEC; ++k) dst[k] = v[k];
+        }
+    }
+};
+template <int VEC>
+struct Store<__nv_bfloat16, VEC> {
+    static __device__ __forceinline__ void run(__nv_bfloat16* dst, const float* v) {
+        if constexpr (VEC == 4) {
+            __nv_bfloat162 lo = __floats2bfloat162_rn(v[0], v[1]);
+            __nv_bfloat162 hi = __floats2bfloat162_rn(v[2], v[3]);
+            uint2 u;
+            u.x = *reinterpret_cast<uint32_t*>(&lo);
+            u.y = *reinterpret_cast<uint32_t*>(&hi);
+            *reinterpret_cast<uint2*>(dst) = u;
+        } else {
+#pragma unroll
+            for (int k = 0; k < VEC; ++k) dst[k] = __float2bfloat16_rn(v[k]);
+        }
+    }
+};
+
+template <int VEC>
+__device__ __forceinline__ void load_vec(const float* __restrict__ src, float* v) {
+    if constexpr (VEC == 4) {
+        const float4 q = *reinterpret_cast<const float4*>(src);
+        v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
+    } else {
+#pragma unroll
+        for (int k = 0; k < VEC; ++k) v[k] = src[k];
+    }
+}
+
+template <typename TP, int VEC>
+__global__ void __launch_bounds__(256)
+state_pass_kernel(const float* __restrict__ states, const float* __restrict__ logdecay,
+                  const float* __restrict__ init, TP* __restrict__ prev,
+                  float* __restrict__ fin, int64_t b, int64_t T, int64_t H, int64_t PN) {
+    const int64_t nvec = PN / VEC;
+    const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (idx >= b * H * nvec) return;
+    const int64_t bh = idx / nvec;
+    const int64_t off = (idx - bh * nvec) * VEC;
+    const int64_t bb = bh / H, h = bh - bb * H;
+
+    float hs[VEC];
+    if (init) {
+        load_vec<VEC>(init + bh * PN + off, hs);
+    } else {
+#pragma unroll
+        for (int k = 0; k < VEC; ++k) hs[k] = 0.f;
+    }
+    const int64_t cstride = H * PN;
+    const float* sp = states + (bb * T * H + h) * PN + off;
+    const float* lp = logdecay + bb * T * H + h;
+    TP* pp = prev + (bb * T * H + h) * PN + off;
+#pragma unroll 4
+    for (int64_t c = 0; c < T; ++c) {
+        float sv[VEC];
+        load_vec<VEC>(sp + c * cstride, sv);
+        const float a = expf(lp[c * H]);
+        Store<TP, VEC>::run(pp + c * cstride, hs);
+#pragma unroll
+        for (int k = 0; k < VEC; ++k) hs[k] = fmaf(a, hs[k], sv[k]);
+    }
+    if (fin) {
+        float* fp = fin + bh * PN + off;
+#pragma unroll
+        for (int k = 0; k < VEC; ++k) fp[k] = hs[k];
+    }
+}
+
+__global__ void copy_or_zero_kernel(const float* __restrict__ src, float* __restrict__ dst,
+                                    int64_t n) {
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i < n) dst[i] = src ? src[i] : 0.f;
+}
+
+template <typename TP, int VEC>
+cudaError_t run(const float* states, const float* logdecay, const float* init, void* prev,
+                float* fin, const Dims& d, cudaStream_t s) {
+    const int64_t PN = d.P * d.N;
+    const int64_t threads = d.b * d.H * (PN / VEC);
+    if (threads == 0) return cudaSuccess;
+    const int bs = 256;
+    const int64_t blocks = (threads + bs - 1) / bs;
+    state_pass_kernel<TP, VEC><<<(unsigned)blocks, bs, 0, s>>>(
+        states, logdecay, init, static_cast<TP*>(prev), fin, d.b, d.T, d.H, PN);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_state_pass(const float* states, const float* logdecay, const float* init,
+                              void* prev, float* fin, const Dims& d, Elt t, cudaStream_t s) {
+    const bool v4 = ((d.P * d.N) % 4) == 0;
+    if (t == Elt::F32)
+        return v4 ? run<float, 4>(states, logdecay, init, prev, fin, d, s)
+                  : run<float, 1>(states, logdecay, init, prev, fin, d, s);
+    return v4 ? run<__nv_bfloat16, 4>(states, logdecay, init, prev, fin, d, s)
+              : run<__nv_bfloat16, 1>(states, logdecay, init, prev, fin, d, s);
+}
+
+cudaError_t launch_copy_or_zero(const float* init, float* fin, int64_t n, cudaStream_t s) {
+    if (n == 0) return cudaSuccess;
+    copy_or_zero_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(init, fin, n);
+    return cudaGetLastError();
+}
+
+}  // namespace ssd

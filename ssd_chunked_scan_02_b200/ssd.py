@@ -1,0 +1,218 @@
+"""Thin ctypes binding of libssd_b200.so (C ABI in include/ssd.h).
+
+Argument marshalling only: every step of the SSD forward and of the decode
+step runs in the library's CUDA kernels.  PyTorch is used for device memory
+and streams.  There is no CPU fallback: if the library is missing, or a
+tensor is not on a CUDA device, the call raises.
+
+Function names match the C entry points.  Each call enqueues work on the
+current torch CUDA stream (or the ``stream`` argument) and returns without
+synchronising.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libssd_b200.so")
+
+SSD_OK, SSD_ERR_INVALID_ARG, SSD_ERR_UNSUPPORTED, SSD_ERR_CUDA, SSD_ERR_TIMEOUT = 0, 1, 2, 3, 4
+SSD_F32, SSD_BF16 = 0, 1
+
+EXPORTED = ("ssd_status_string", "ssd_last_error_detail", "ssd_chunk_scan_fwd_workspace_size",
+            "ssd_chunk_scan_fwd", "ssd_step", "ssd_chunk_state_fwd", "ssd_state_passing_fwd",
+            "ssd_chunk_output_fwd", "ssd_chunk_scan_fwd_uses_tensor_cores")
+
+
+class SSDError(RuntimeError):
+    def __init__(self, status: int, where: str, detail: str):
+        super().__init__(f"{where}: {status_name(status)}: {detail}")
+        self.status = status
+
+
+class ssd_dims_t(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int64), ("seqlen", ctypes.c_int64),
+                ("nheads", ctypes.c_int64), ("headdim", ctypes.c_int64),
+                ("dstate", ctypes.c_int64), ("ngroups", ctypes.c_int64)]
+
+
+_lib = None
+_vp = ctypes.c_void_p
+
+
+def load(path: str = LIB_PATH):
+    """Open the shared library (once).  Raises if it is missing."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing: build it with "
+                           "`python -m ssd_chunked_scan_02_b200.build` (no CPU fallback exists)")
+    lib = ctypes.CDLL(path)
+    dims_p = ctypes.POINTER(ssd_dims_t)
+    lib.ssd_status_string.restype = ctypes.c_char_p
+    lib.ssd_status_string.argtypes = [ctypes.c_int]
+    lib.ssd_last_error_detail.restype = ctypes.c_char_p
+    lib.ssd_last_error_detail.argtypes = []
+    lib.ssd_chunk_scan_fwd_workspace_size.restype = ctypes.c_int
+    lib.ssd_chunk_scan_fwd_workspace_size.argtypes = [dims_p, ctypes.c_int, ctypes.c_int,
+                                                      ctypes.POINTER(ctypes.c_size_t)]
+    lib.ssd_chunk_scan_fwd_uses_tensor_cores.restype = ctypes.c_int
+    lib.ssd_chunk_scan_fwd_uses_tensor_cores.argtypes = [dims_p, ctypes.c_int, ctypes.c_int]
+    lib.ssd_chunk_scan_fwd.restype = ctypes.c_int
+    lib.ssd_chunk_scan_fwd.argtypes = [_vp] * 6 + [ctypes.c_int, _vp, _vp, _vp, dims_p,
+                                                   ctypes.c_int, _vp, ctypes.c_size_t, _vp]
+    lib.ssd_step.restype = ctypes.c_int
+    lib.ssd_step.argtypes = [_vp] * 8 + [dims_p, ctypes.c_int, _vp]
+    lib.ssd_chunk_state_fwd.restype = ctypes.c_int
+    lib.ssd_chunk_state_fwd.argtypes = [_vp] * 4 + [ctypes.c_int, _vp, _vp, dims_p,
+                                                    ctypes.c_int, _vp]
+    lib.ssd_state_passing_fwd.restype = ctypes.c_int
+    lib.ssd_state_passing_fwd.argtypes = [_vp] * 5 + [ctypes.c_int, dims_p, ctypes.c_int, _vp]
+    lib.ssd_chunk_output_fwd.restype = ctypes.c_int
+    lib.ssd_chunk_output_fwd.argtypes = [_vp] * 7 + [ctypes.c_int, _vp, dims_p, ctypes.c_int, _vp]
+    _lib = lib
+    return lib
+
+
+def status_name(status: int) -> str:
+    return load().ssd_status_string(int(status)).decode()
+
+
+def _check(status: int, where: str):
+    if status != SSD_OK:
+        raise SSDError(status, where, load().ssd_last_error_detail().decode())
+
+
+def _dtype_code(t: torch.dtype) -> int:
+    if t == torch.float32:
+        return SSD_F32
+    if t == torch.bfloat16:
+        return SSD_BF16
+    raise TypeError(f"unsupported element dtype {t} (float32 or bfloat16)")
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensors must be on a CUDA device (there is no CPU path)")
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
+
+
+def make_dims(batch, seqlen, nheads, headdim, dstate, ngroups) -> ssd_dims_t:
+    return ssd_dims_t(int(batch), int(seqlen), int(nheads), int(headdim), int(dstate),
+                      int(ngroups))
+
+
+def _fwd_dims(x, B) -> ssd_dims_t:
+    b, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    return make_dims(b, L, H, P, N, G)
+
+
+def ssd_chunk_scan_fwd_workspace_size(dims: ssd_dims_t, chunk_size: int, dtype: torch.dtype) -> int:
+    n = ctypes.c_size_t(0)
+    _check(load().ssd_chunk_scan_fwd_workspace_size(ctypes.byref(dims), int(chunk_size),
+                                                    _dtype_code(dtype), ctypes.byref(n)),
+           "ssd_chunk_scan_fwd_workspace_size")
+    return int(n.value)
+
+
+def ssd_chunk_scan_fwd_uses_tensor_cores(dims: ssd_dims_t, chunk_size: int,
+                                         dtype: torch.dtype) -> int:
+    return int(load().ssd_chunk_scan_fwd_uses_tensor_cores(ctypes.byref(dims), int(chunk_size),
+                                                           _dtype_code(dtype)))
+
+
+def ssd_chunk_scan_fwd(x, dt, A, B, C, D, chunk_size: int, init_states=None,
+                       return_final_states: bool = False, y=None, final_states=None,
+                       workspace=None, stream=None):
+    """y (b,L,H,P) [, final_states (b,H,P,N) fp32] for the whole sequences."""
+    dims = _fwd_dims(x, B)
+    if y is None:
+        y = torch.empty_like(x)
+    if return_final_states and final_states is None:
+        final_states = torch.empty((x.shape[0], x.shape[2], x.shape[3], B.shape[3]),
+                                   device=x.device, dtype=torch.float32)
+    need = ssd_chunk_scan_fwd_workspace_size(dims, chunk_size, x.dtype)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), device=x.device, dtype=torch.uint8)
+    st = load().ssd_chunk_scan_fwd(_ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+                                   int(chunk_size), _ptr(init_states), _ptr(y),
+                                   _ptr(final_states), ctypes.byref(dims), _dtype_code(x.dtype),
+                                   _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(st, "ssd_chunk_scan_fwd")
+    return (y, final_states) if (return_final_states or final_states is not None) else y
+
+
+def ssd_step(state, x, dt, A, B, C, D, y=None, stream=None):
+    """One decode step; ``state`` (b,H,P,N) fp32 is updated in place.  Returns y (b,H,P)."""
+    b, H, P = x.shape
+    G, N = B.shape[1], B.shape[2]
+    dims = make_dims(b, 1, H, P, N, G)
+    if y is None:
+        y = torch.empty_like(x)
+    st = load().ssd_step(_ptr(state), _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+                         _ptr(y), ctypes.byref(dims), _dtype_code(x.dtype), _stream(stream))
+    _check(st, "ssd_step")
+    return y
+
+
+def n_chunks(seqlen: int, chunk_size: int) -> int:
+    return (int(seqlen) + int(chunk_size) - 1) // int(chunk_size)
+
+
+def ssd_chunk_state_fwd(x, dt, A, B, chunk_size: int, stream=None):
+    """Step (2): per-chunk zero-start states (b,T,H,P,N) fp32 and log-decays (b,T,H)."""
+    dims = _fwd_dims(x, B)
+    b, L, H, P = x.shape
+    T = n_chunks(L, chunk_size)
+    states = torch.empty((b, T, H, P, B.shape[3]), device=x.device, dtype=torch.float32)
+    logdecay = torch.empty((b, T, H), device=x.device, dtype=torch.float32)
+    st = load().ssd_chunk_state_fwd(_ptr(x), _ptr(dt), _ptr(A), _ptr(B), int(chunk_size),
+                                    _ptr(states), _ptr(logdecay), ctypes.byref(dims),
+                                    _dtype_code(x.dtype), _stream(stream))
+    _check(st, "ssd_chunk_state_fwd")
+    return states, logdecay
+
+
+def ssd_state_passing_fwd(chunk_states, chunk_logdecay, chunk_size: int, seqlen: int,
+                          dtype: torch.dtype, init_states=None, want_final: bool = True,
+                          stream=None):
+    """Step (3): states entering each chunk (b,T,H,P,N) in ``dtype`` and the final state."""
+    b, T, H, P, N = chunk_states.shape
+    dims = make_dims(b, seqlen, H, P, N, 1)
+    prev = torch.empty((b, T, H, P, N), device=chunk_states.device, dtype=dtype)
+    final = (torch.empty((b, H, P, N), device=chunk_states.device, dtype=torch.float32)
+             if want_final else None)
+    st = load().ssd_state_passing_fwd(_ptr(chunk_states), _ptr(chunk_logdecay), _ptr(init_states),
+                                      _ptr(prev), _ptr(final), int(chunk_size), ctypes.byref(dims),
+                                      _dtype_code(dtype), _stream(stream))
+    _check(st, "ssd_state_passing_fwd")
+    return prev, final
+
+
+def ssd_chunk_output_fwd(x, dt, A, B, C, D, prev_states, chunk_size: int, y=None, stream=None):
+    """Steps (1) and (4): y from the inputs and the states entering each chunk."""
+    dims = _fwd_dims(x, B)
+    if y is None:
+        y = torch.empty_like(x)
+    st = load().ssd_chunk_output_fwd(_ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+                                     _ptr(prev_states), int(chunk_size), _ptr(y),
+                                     ctypes.byref(dims), _dtype_code(x.dtype), _stream(stream))
+    _check(st, "ssd_chunk_output_fwd")
+    return y

@@ -1,0 +1,192 @@
+"""C-ABI checks that need no GPU: the library loads, exports every symbol its
+header declares, sizes its workspace, and rejects bad arguments before
+launching anything (so every call here returns without touching a device)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from ssd_chunked_scan_02_b200 import build as ssd_build
+from ssd_chunked_scan_02_b200 import ssd
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ssd.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    ssd_build.build()
+    return ssd.load()
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"SSD_API\s+[\w\s\*]*?\b(ssd_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_two_main_calls():
+    syms = declared_symbols()
+    assert "ssd_chunk_scan_fwd" in syms and "ssd_step" in syms
+    assert len(syms) >= 9
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_symbols():
+        assert hasattr(lib, name), f"{name} declared in include/ssd.h but not exported"
+    assert set(declared_symbols()) == set(ssd.EXPORTED)
+
+
+def test_status_strings(lib):
+    assert ssd.status_name(0) == "SSD_OK"
+    assert ssd.status_name(1) == "SSD_ERR_INVALID_ARG"
+    assert ssd.status_name(2) == "SSD_ERR_UNSUPPORTED"
+    assert ssd.status_name(3) == "SSD_ERR_CUDA"
+    assert ssd.status_name(4) == "SSD_ERR_TIMEOUT"
+    assert ssd.status_name(99) == "SSD_ERR_UNKNOWN"
+
+
+def _ws(dims, q, dt):
+    n = ctypes.c_size_t(0)
+    st = ssd.load().ssd_chunk_scan_fwd_workspace_size(ctypes.byref(dims), q, dt, ctypes.byref(n))
+    return st, n.value
+
+
+def _round(v):
+    return (v + 255) // 256 * 256
+
+
+@pytest.mark.parametrize("b,L,H,P,N,G,Q,dt", [
+    (4, 8192, 80, 64, 128, 1, 256, ssd.SSD_BF16),
+    (1, 256, 4, 16, 16, 1, 64, ssd.SSD_F32),
+    (2, 600, 4, 64, 128, 2, 128, ssd.SSD_BF16),   # ragged: 5 chunks, last one partial
+    (3, 1, 2, 3, 5, 1, 16, ssd.SSD_F32),
+])
+def test_workspace_size_formula(lib, b, L, H, P, N, G, Q, dt):
+    st, n = _ws(ssd.make_dims(b, L, H, P, N, G), Q, dt)
+    assert st == ssd.SSD_OK
+    T = (L + Q - 1) // Q
+    elt = 4 if dt == ssd.SSD_F32 else 2
+    ns = b * T * H * P * N
+    assert n == _round(ns * 4) + _round(b * T * H * 4) + _round(ns * elt)
+
+
+def test_workspace_zero_for_empty(lib):
+    assert _ws(ssd.make_dims(0, 100, 4, 8, 8, 1), 64, ssd.SSD_F32) == (ssd.SSD_OK, 0)
+    assert _ws(ssd.make_dims(2, 0, 4, 8, 8, 1), 64, ssd.SSD_F32) == (ssd.SSD_OK, 0)
+
+
+@pytest.mark.parametrize("dims,q,dt,expect", [
+    ((1, 64, 4, 8, 8, 3), 64, ssd.SSD_F32, ssd.SSD_ERR_INVALID_ARG),      # H % G != 0
+    ((1, 64, 0, 8, 8, 1), 64, ssd.SSD_F32, ssd.SSD_ERR_INVALID_ARG),      # H = 0
+    ((-1, 64, 4, 8, 8, 1), 64, ssd.SSD_F32, ssd.SSD_ERR_INVALID_ARG),     # b < 0
+    ((1, 64, 4, 300, 8, 1), 64, ssd.SSD_F32, ssd.SSD_ERR_UNSUPPORTED),    # P > 256
+    ((1, 64, 4, 8, 512, 1), 64, ssd.SSD_F32, ssd.SSD_ERR_UNSUPPORTED),    # N > 256
+    ((1, 64, 4, 8, 8, 1), 96, ssd.SSD_F32, ssd.SSD_ERR_UNSUPPORTED),      # not a power of two
+    ((1, 64, 4, 8, 8, 1), 512, ssd.SSD_F32, ssd.SSD_ERR_UNSUPPORTED),     # chunk too large
+    ((1, 64, 4, 8, 8, 1), 8, ssd.SSD_F32, ssd.SSD_ERR_UNSUPPORTED),       # chunk too small
+    ((1, 64, 4, 8, 8, 1), 64, 7, ssd.SSD_ERR_INVALID_ARG),                # unknown dtype
+])
+def test_workspace_rejects(lib, dims, q, dt, expect):
+    st, _ = _ws(ssd.make_dims(*dims), q, dt)
+    assert st == expect
+    assert ssd.load().ssd_last_error_detail().decode() != ""
+
+
+def test_null_dims_rejected(lib):
+    n = ctypes.c_size_t(0)
+    assert lib.ssd_chunk_scan_fwd_workspace_size(None, 64, 0, ctypes.byref(n)) == 1
+
+
+# Fake, never-dereferenced device addresses: the calls below must fail
+# validation before any launch.
+A16 = 0x7f0000001000
+
+
+def _fwd(lib, dims, ptrs, q=64, dt=ssd.SSD_F32, ws_bytes=1 << 30, init=None, fin=None):
+    x, dtp, A, B, C, D, y, ws = ptrs
+    return lib.ssd_chunk_scan_fwd(x, dtp, A, B, C, D, q, init, y, fin, ctypes.byref(dims), dt,
+                                  ws, ws_bytes, None)
+
+
+def _good():
+    return [A16 + k * 0x100000 for k in range(8)]
+
+
+@pytest.mark.parametrize("which", range(8))
+def test_fwd_null_pointer_rejected(lib, which):
+    p = _good()
+    p[which] = None
+    st = _fwd(lib, ssd.make_dims(1, 128, 4, 8, 8, 1), p)
+    assert st == ssd.SSD_ERR_INVALID_ARG
+    assert "NULL" in lib.ssd_last_error_detail().decode()
+
+
+@pytest.mark.parametrize("which", range(8))
+def test_fwd_misaligned_pointer_rejected(lib, which):
+    p = _good()
+    p[which] += 4
+    st = _fwd(lib, ssd.make_dims(1, 128, 4, 8, 8, 1), p)
+    assert st == ssd.SSD_ERR_INVALID_ARG
+    assert "aligned" in lib.ssd_last_error_detail().decode()
+
+
+def test_fwd_misaligned_optional_rejected(lib):
+    st = _fwd(lib, ssd.make_dims(1, 128, 4, 8, 8, 1), _good(), init=A16 + 8)
+    assert st == ssd.SSD_ERR_INVALID_ARG
+    st = _fwd(lib, ssd.make_dims(1, 128, 4, 8, 8, 1), _good(), fin=A16 + 8)
+    assert st == ssd.SSD_ERR_INVALID_ARG
+
+
+def test_fwd_small_workspace_rejected(lib):
+    dims = ssd.make_dims(2, 600, 4, 64, 128, 1)
+    _, need = _ws(dims, 128, ssd.SSD_BF16)
+    st = _fwd(lib, dims, _good(), q=128, dt=ssd.SSD_BF16, ws_bytes=need - 1)
+    assert st == ssd.SSD_ERR_INVALID_ARG
+    assert "workspace" in lib.ssd_last_error_detail().decode()
+
+
+def test_fwd_bad_chunk_rejected(lib):
+    assert _fwd(lib, ssd.make_dims(1, 128, 4, 8, 8, 1), _good(), q=100) == ssd.SSD_ERR_UNSUPPORTED
+
+
+def test_fwd_empty_batch_is_noop(lib):
+    assert _fwd(lib, ssd.make_dims(0, 128, 4, 8, 8, 1), [None] * 8) == ssd.SSD_OK
+
+
+def test_step_rejects(lib):
+    dims = ssd.make_dims(2, 1, 4, 8, 8, 1)
+    p = _good()
+    assert lib.ssd_step(None, *p[1:8], ctypes.byref(dims), 0, None) == ssd.SSD_ERR_INVALID_ARG
+    p2 = list(p)
+    p2[3] += 2
+    assert lib.ssd_step(*p2, ctypes.byref(dims), 0, None) == ssd.SSD_ERR_INVALID_ARG
+    bad = ssd.make_dims(2, 1, 4, 8, 8, 3)
+    assert lib.ssd_step(*p, ctypes.byref(bad), 0, None) == ssd.SSD_ERR_INVALID_ARG
+    assert lib.ssd_step(*p, ctypes.byref(ssd.make_dims(0, 1, 4, 8, 8, 1)), 0, None) == ssd.SSD_OK
+
+
+def test_stage_entry_points_reject(lib):
+    dims = ssd.make_dims(1, 128, 4, 8, 8, 1)
+    assert lib.ssd_chunk_state_fwd(None, A16, A16, A16, 64, A16, A16, ctypes.byref(dims), 0,
+                                   None) == ssd.SSD_ERR_INVALID_ARG
+    assert lib.ssd_state_passing_fwd(A16, None, None, A16, None, 64, ctypes.byref(dims), 0,
+                                     None) == ssd.SSD_ERR_INVALID_ARG
+    assert lib.ssd_chunk_output_fwd(A16, A16, A16, A16, A16, A16, None, 64, A16,
+                                    ctypes.byref(dims), 0, None) == ssd.SSD_ERR_INVALID_ARG
+    assert lib.ssd_chunk_output_fwd(A16, A16, A16, A16, A16, A16, A16, 24, A16,
+                                    ctypes.byref(dims), 0, None) == ssd.SSD_ERR_UNSUPPORTED
+
+
+def test_tensor_core_selection_query(lib):
+    f = lib.ssd_chunk_scan_fwd_uses_tensor_cores
+    assert f(ctypes.byref(ssd.make_dims(1, 64, 4, 8, 8, 3)), 64, 0) == -1
+    assert f(ctypes.byref(ssd.make_dims(1, 256, 4, 16, 16, 1)), 64, ssd.SSD_F32) == 0
+
+
+def test_binding_refuses_cpu_tensors(lib):
+    import torch
+    x = torch.zeros(1, 64, 2, 8)
+    with pytest.raises(ValueError, match="CUDA"):
+        ssd.ssd_chunk_scan_fwd(x, torch.zeros(1, 64, 2), torch.zeros(2), torch.zeros(1, 64, 1, 8),
+                               torch.zeros(1, 64, 1, 8), torch.zeros(2), 64)

@@ -1,0 +1,358 @@
+"""CUDA path vs the fp64 oracle, element by element, on the same seeded inputs.
+
+Error metric (per tensor): max|gpu - oracle| / max|oracle|; bound 5e-3 for
+bf16 storage, 1e-4 for fp32.  Small cases compare every element; the full
+workload sizes compare sampled (batch, head) pairs, each recomputed by the
+oracle over the whole sequence."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from parity import TOL, gpu_fwd, oracle_fwd, oracle_pairs, rel_err, sample_pairs, to_dev
+from ssd_chunked_scan_02_b200 import inputs, ssd
+
+pytestmark = pytest.mark.gpu
+
+
+def _w(name, b, L, H, P, N, G, Q, dtype, init, seed):
+    return inputs.Workload(name, b, L, H, P, N, G, Q, dtype, with_init=init, want_final=True,
+                           seed=seed)
+
+
+def _check_full(w, chunk=None):
+    inp = inputs.make_inputs(w)
+    y, f = gpu_fwd(inp, chunk or w.chunk)
+    y_ref, f_ref = oracle_fwd(inp)
+    tol = TOL[w.dtype]
+    ey, ef = rel_err(y, y_ref), rel_err(f, f_ref)
+    assert np.all(np.isfinite(y)) and np.all(np.isfinite(f))
+    assert ey <= tol, f"{w.name} Q={chunk or w.chunk}: y rel err {ey:.3g} > {tol}"
+    assert ef <= tol, f"{w.name} Q={chunk or w.chunk}: final rel err {ef:.3g} > {tol}"
+    return ey, ef
+
+
+def test_tiny_f32_workload_full():
+    _check_full(inputs.TINY_F32)
+
+
+SMALL_BF16 = [
+    # name,               b,  L,   H,  P,  N,  G,  Q,  init
+    ("bf16_ragged_q256", 2, 600, 4, 64, 128, 1, 256, True),
+    ("bf16_ragged_q128", 2, 600, 4, 64, 128, 1, 128, True),
+    ("bf16_q64", 2, 300, 4, 64, 128, 1, 64, True),
+    ("bf16_n64_groups2", 1, 1000, 6, 64, 64, 2, 256, False),
+    ("bf16_short_L_lt_Q", 1, 17, 2, 64, 128, 1, 256, True),
+    ("bf16_single_token", 2, 1, 2, 64, 128, 1, 256, True),
+    ("bf16_odd_dims", 3, 513, 2, 32, 48, 1, 128, True),
+    ("bf16_exact_chunks", 2, 1024, 8, 64, 128, 1, 256, True),
+]
+
+
+@pytest.mark.parametrize("case", SMALL_BF16, ids=[c[0] for c in SMALL_BF16])
+def test_small_bf16(case):
+    name, b, L, H, P, N, G, Q, init = case
+    _check_full(_w(name, b, L, H, P, N, G, Q, "bf16", init, seed=100 + len(name)))
+
+
+SMALL_F32 = [
+    ("f32_ragged", 2, 333, 3, 16, 16, 1, 64, True),
+    ("f32_tiny_dims", 1, 256, 4, 3, 5, 1, 32, True),
+    ("f32_big_dims_groups2", 1, 500, 2, 64, 128, 2, 128, True),
+    ("f32_q256", 1, 700, 2, 16, 32, 1, 256, False),
+]
+
+
+@pytest.mark.parametrize("case", SMALL_F32, ids=[c[0] for c in SMALL_F32])
+def test_small_f32(case):
+    name, b, L, H, P, N, G, Q, init = case
+    _check_full(_w(name, b, L, H, P, N, G, Q, "f32", init, seed=200 + len(name)))
+
+
+def _check_sampled(w, k, seed):
+    inp = inputs.make_inputs(w, device="cuda")
+    d = inp
+    out = ssd.ssd_chunk_scan_fwd(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], w.chunk,
+                                 init_states=d["init"], return_final_states=True)
+    y, f = out
+    torch.cuda.synchronize()
+    pairs = sample_pairs(w.batch, w.nheads, k, seed)
+    refs = oracle_pairs(inp, pairs)
+    ys = np.stack([y[b, :, h].double().cpu().numpy() for (b, h) in pairs])
+    fs = np.stack([f[b, h].double().cpu().numpy() for (b, h) in pairs])
+    y_ref = np.stack([r[0] for r in refs])
+    f_ref = np.stack([r[1] for r in refs])
+    tol = TOL[w.dtype]
+    ey, ef = rel_err(ys, y_ref), rel_err(fs, f_ref)
+    assert torch.isfinite(y.float()).all().item()
+    assert ey <= tol, f"{w.name}: sampled y rel err {ey:.3g} > {tol}"
+    assert ef <= tol, f"{w.name}: sampled final rel err {ef:.3g} > {tol}"
+
+
+def test_layer_130m_sampled():
+    _check_sampled(inputs.LAYER_130M, k=8, seed=1)
+
+
+def test_layer_2p7b_sampled():
+    _check_sampled(inputs.LAYER_2P7B, k=8, seed=2)
+
+
+@pytest.mark.parametrize("w", inputs.SWEEP, ids=[w.name for w in inputs.SWEEP])
+def test_sweep_sampled(w):
+    _check_sampled(w, k=3 if w.seqlen >= 131072 else 6, seed=3)
+
+
+def test_decode_1024_steps_sampled():
+    """1024 sequential ssd_step calls at b=256, H=80, P=64, N=128 against the
+    fp64 step oracle on sampled (batch, head) pairs: y at every step and the
+    state after the last step."""
+    w = inputs.DECODE_2P7B
+    gen, par = inputs.make_decode_params(w)
+    state = par["state"].cuda()
+    A, D = par["A"].cuda(), par["D"].cuda()
+    pairs = sample_pairs(w.batch, w.nheads, 6, seed=4)
+    ost = {p: par["state"][p[0], p[1]].double().numpy().copy() for p in pairs}
+    num_y = den_y = 0.0
+    for _ in range(w.steps):
+        tok = inputs.make_decode_token(w, gen)
+        td = to_dev(tok)
+        y = ssd.ssd_step(state, td["x"], td["dt"], A, td["B"], td["C"], D)
+        ycpu = y.double().cpu().numpy()
+        for (b, h) in pairs:
+            yo, st = oracle.step(ost[(b, h)][None, None], tok["x"][b:b + 1, h:h + 1],
+                                 tok["dt"][b:b + 1, h:h + 1], par["A"][h:h + 1],
+                                 tok["B"][b:b + 1], tok["C"][b:b + 1], par["D"][h:h + 1])
+            ost[(b, h)] = st[0, 0]
+            num_y = max(num_y, float(np.max(np.abs(ycpu[b, h] - yo[0, 0]))))
+            den_y = max(den_y, float(np.max(np.abs(yo[0, 0]))))
+    torch.cuda.synchronize()
+    ey = num_y / den_y
+    fs = np.stack([state[b, h].double().cpu().numpy() for (b, h) in pairs])
+    fr = np.stack([ost[p] for p in pairs])
+    es = rel_err(fs, fr)
+    assert ey <= TOL["bf16"], f"decode y rel err {ey:.3g}"
+    assert es <= TOL["bf16"], f"decode state rel err {es:.3g}"
+
+
+def test_decode_f32_small_full():
+    """fp32 decode, every element, 50 steps, odd sizes (scalar kernel path)."""
+    w = inputs.DecodeWorkload("decode_f32_small", 3, 5, 7, 9, 1, 50, "f32", seed=77)
+    gen, par = inputs.make_decode_params(w)
+    state = par["state"].cuda()
+    ost = par["state"].double().numpy().copy()
+    for _ in range(w.steps):
+        tok = inputs.make_decode_token(w, gen)
+        td = to_dev(tok)
+        y = ssd.ssd_step(state, td["x"], td["dt"], par["A"].cuda(), td["B"], td["C"],
+                         par["D"].cuda())
+        yo, ost = oracle.step(ost, tok["x"], tok["dt"], par["A"], tok["B"], tok["C"], par["D"])
+        assert rel_err(y.double().cpu().numpy(), yo) <= TOL["f32"]
+    assert rel_err(state.double().cpu().numpy(), ost) <= TOL["f32"]
+
+
+# --- each step of the forward on its own -------------------------------------------------
+
+STAGE_CASES = [("bf16", 2, 600, 4, 64, 128, 1, 256), ("bf16", 1, 512, 4, 64, 64, 2, 128),
+               ("f32", 2, 333, 3, 16, 16, 1, 64)]
+
+
+def _oracle_chunk_views(inp, Q):
+    """Oracle chunk states (zero start), log-decays and entering states."""
+    x, dt, A, B, C, D, init = (inp[k] for k in ("x", "dt", "A", "B", "C", "D", "init"))
+    b, L, H, P = x.shape
+    N = B.shape[3]
+    T = (L + Q - 1) // Q
+    S = np.zeros((b, T, H, P, N))
+    prev = np.zeros((b, T, H, P, N))
+    ld = np.zeros((b, T, H))
+    h = np.zeros((b, H, P, N)) if init is None else init.double().numpy()
+    for c in range(T):
+        sl = slice(c * Q, min(L, (c + 1) * Q))
+        _, s0 = oracle.recurrence(x[:, sl], dt[:, sl], A, B[:, sl], C[:, sl], D, None)
+        S[:, c] = s0
+        prev[:, c] = h
+        _, h = oracle.recurrence(x[:, sl], dt[:, sl], A, B[:, sl], C[:, sl], D, h)
+        ld[:, c] = (dt[:, sl].double() * A.double()[None, None, :]).sum(dim=1).numpy()
+    return S, ld, prev, h
+
+
+@pytest.mark.parametrize("case", STAGE_CASES, ids=lambda c: "_".join(map(str, c)))
+def test_stage_chunk_state(case):
+    dtype, b, L, H, P, N, G, Q = case
+    inp = inputs.make_inputs(_w("st", b, L, H, P, N, G, Q, dtype, True, seed=31))
+    d = to_dev(inp)
+    S, ld = ssd.ssd_chunk_state_fwd(d["x"], d["dt"], d["A"], d["B"], Q)
+    torch.cuda.synchronize()
+    S_ref, ld_ref, _, _ = _oracle_chunk_views(inp, Q)
+    assert rel_err(S.double().cpu().numpy(), S_ref) <= TOL[dtype]
+    assert np.max(np.abs(ld.double().cpu().numpy() - ld_ref)) <= 1e-4 * max(1.0, np.max(np.abs(ld_ref)))
+
+
+@pytest.mark.parametrize("case", STAGE_CASES, ids=lambda c: "_".join(map(str, c)))
+def test_stage_state_passing(case):
+    dtype, b, L, H, P, N, G, Q = case
+    inp = inputs.make_inputs(_w("sp", b, L, H, P, N, G, Q, dtype, True, seed=32))
+    S_ref, ld_ref, prev_ref, final_ref = _oracle_chunk_views(inp, Q)
+    tdt = torch.float32 if dtype == "f32" else torch.bfloat16
+    prev, fin = ssd.ssd_state_passing_fwd(torch.from_numpy(S_ref).float().cuda(),
+                                          torch.from_numpy(ld_ref).float().cuda(), Q, L, tdt,
+                                          init_states=inp["init"].cuda())
+    torch.cuda.synchronize()
+    assert rel_err(prev.double().cpu().numpy(), prev_ref) <= TOL[dtype]
+    assert rel_err(fin.double().cpu().numpy(), final_ref) <= TOL[dtype]
+
+
+@pytest.mark.parametrize("case", STAGE_CASES, ids=lambda c: "_".join(map(str, c)))
+def test_stage_chunk_output(case):
+    dtype, b, L, H, P, N, G, Q = case
+    inp = inputs.make_inputs(_w("co", b, L, H, P, N, G, Q, dtype, True, seed=33))
+    _, _, prev_ref, _ = _oracle_chunk_views(inp, Q)
+    tdt = torch.float32 if dtype == "f32" else torch.bfloat16
+    d = to_dev(inp)
+    y = ssd.ssd_chunk_output_fwd(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"],
+                                 torch.from_numpy(prev_ref).to(tdt).cuda(), Q)
+    torch.cuda.synchronize()
+    y_ref, _ = oracle_fwd(inp)
+    assert rel_err(y.double().cpu().numpy(), y_ref) <= TOL[dtype]
+
+
+# --- invariants across entry points --------------------------------------------------------
+
+def test_steps_equal_forward():
+    """L decode steps reproduce the chunked forward (both on the GPU)."""
+    w = _w("inv", 2, 300, 4, 64, 128, 1, 128, "bf16", True, seed=41)
+    inp = to_dev(inputs.make_inputs(w))
+    y_fwd, f_fwd = ssd.ssd_chunk_scan_fwd(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"],
+                                          inp["D"], w.chunk, init_states=inp["init"],
+                                          return_final_states=True)
+    state = inp["init"].clone()
+    ys = []
+    for t in range(w.seqlen):
+        ys.append(ssd.ssd_step(state, inp["x"][:, t].contiguous(), inp["dt"][:, t].contiguous(),
+                               inp["A"], inp["B"][:, t].contiguous(), inp["C"][:, t].contiguous(),
+                               inp["D"]))
+    y_dec = torch.stack(ys, dim=1)
+    torch.cuda.synchronize()
+    assert rel_err(y_dec.double().cpu().numpy(), y_fwd.double().cpu().numpy()) <= TOL["bf16"]
+    assert rel_err(state.double().cpu().numpy(), f_fwd.double().cpu().numpy()) <= TOL["bf16"]
+
+
+def test_split_sequence_resume():
+    w = _w("res", 2, 1024, 4, 64, 128, 1, 256, "bf16", True, seed=42)
+    inp = to_dev(inputs.make_inputs(w))
+    y, f = ssd.ssd_chunk_scan_fwd(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], inp["D"],
+                                  256, init_states=inp["init"], return_final_states=True)
+    cut = 384  # not a chunk multiple of 256: the second call starts mid-chunk
+    part = lambda k, s: inp[k][:, s].contiguous()
+    y1, f1 = ssd.ssd_chunk_scan_fwd(part("x", slice(0, cut)), part("dt", slice(0, cut)), inp["A"],
+                                    part("B", slice(0, cut)), part("C", slice(0, cut)), inp["D"],
+                                    256, init_states=inp["init"], return_final_states=True)
+    y2, f2 = ssd.ssd_chunk_scan_fwd(part("x", slice(cut, None)), part("dt", slice(cut, None)),
+                                    inp["A"], part("B", slice(cut, None)),
+                                    part("C", slice(cut, None)), inp["D"], 256, init_states=f1,
+                                    return_final_states=True)
+    torch.cuda.synchronize()
+    ycat = torch.cat([y1, y2], dim=1)
+    assert rel_err(ycat.double().cpu().numpy(), y.double().cpu().numpy()) <= TOL["bf16"]
+    assert rel_err(f2.double().cpu().numpy(), f.double().cpu().numpy()) <= TOL["bf16"]
+
+
+def test_chunk_size_invariance():
+    w = _w("inv_q", 2, 1024, 4, 64, 128, 1, 256, "bf16", True, seed=43)
+    inp = inputs.make_inputs(w)
+    y_ref, f_ref = oracle_fwd(inp)
+    outs = {}
+    for Q in (64, 128, 256):
+        y, f = gpu_fwd(inp, Q)
+        assert rel_err(y, y_ref) <= TOL["bf16"], Q
+        assert rel_err(f, f_ref) <= TOL["bf16"], Q
+        outs[Q] = y
+    assert rel_err(outs[64], outs[256]) <= TOL["bf16"]
+    assert rel_err(outs[128], outs[256]) <= TOL["bf16"]
+
+
+# --- degenerate cases and memory hygiene --------------------------------------------------
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_no_memory_closed_form(dtype):
+    """dt*A -> -inf: y_t = dt_t (C_t.B_t) x_t + D x_t and the initial state is forgotten."""
+    w = _w("nomem", 2, 520, 4, 64, 128, 1, 256, dtype, True, seed=44)
+    inp = inputs.make_inputs(w)
+    inp["A"] = torch.full_like(inp["A"], -1.0e6)
+    y, f = gpu_fwd(inp, 256)
+    x = inp["x"].double().numpy()
+    cb = np.einsum("bln,bln->bl", inp["C"][:, :, 0].double().numpy(), inp["B"][:, :, 0].double().numpy())
+    y_cf = (inp["dt"].double().numpy() * cb[:, :, None])[..., None] * x + inp["D"].double().numpy()[None, None, :, None] * x
+    assert rel_err(y, y_cf) <= TOL[dtype]
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_a_zero_cumulative_sum(dtype):
+    w = _w("azero", 1, 700, 3, 64, 64, 1, 128, dtype, True, seed=45)
+    inp = inputs.make_inputs(w)
+    inp["A"] = torch.zeros_like(inp["A"])
+    y, f = gpu_fwd(inp, 128)
+    y_ref, f_ref = oracle_fwd(inp)
+    assert rel_err(y, y_ref) <= TOL[dtype]
+    assert rel_err(f, f_ref) <= TOL[dtype]
+
+
+def test_c_zero_gives_skip_only():
+    w = _w("czero", 2, 300, 4, 64, 128, 1, 256, "bf16", True, seed=46)
+    inp = inputs.make_inputs(w)
+    inp["C"] = torch.zeros_like(inp["C"])
+    y, _ = gpu_fwd(inp, 256)
+    skip = (inp["D"][None, None, :, None] * inp["x"].float()).to(torch.bfloat16).double().numpy()
+    assert np.max(np.abs(y - skip)) <= 2 ** -8 * np.max(np.abs(skip))
+
+
+def test_empty_sequence_copies_init():
+    init = torch.randn(2, 3, 16, 8, device="cuda")
+    fin = torch.full_like(init, float("nan"))
+    x = torch.empty(2, 0, 3, 16, device="cuda")
+    dt = torch.empty(2, 0, 3, device="cuda")
+    Bm = torch.empty(2, 0, 1, 8, device="cuda")
+    A = -torch.ones(3, device="cuda")
+    D = torch.ones(3, device="cuda")
+    ssd.ssd_chunk_scan_fwd(x, dt, A, Bm, Bm, D, 64, init_states=init, final_states=fin)
+    torch.cuda.synchronize()
+    assert torch.equal(fin, init)
+    fin2 = torch.full_like(init, float("nan"))
+    ssd.ssd_chunk_scan_fwd(x, dt, A, Bm, Bm, D, 64, final_states=fin2)
+    torch.cuda.synchronize()
+    assert torch.count_nonzero(fin2).item() == 0
+
+
+def test_guard_bands_and_full_coverage():
+    """Outputs are written exactly in bounds: sentinel padding around y and
+    the final states stays intact, and a NaN prefill of y is fully replaced."""
+    w = _w("guard", 2, 600, 4, 64, 128, 1, 256, "bf16", True, seed=47)
+    inp = to_dev(inputs.make_inputs(w))
+    pad = 4096
+    ny = inp["x"].numel()
+    ybuf = torch.full((ny + 2 * pad,), float("nan"), device="cuda", dtype=torch.bfloat16)
+    ybuf[:pad] = 7.0
+    ybuf[-pad:] = 7.0
+    y = ybuf[pad:pad + ny].view_as(inp["x"])
+    nf = 2 * 4 * 64 * 128
+    fbuf = torch.full((nf + 2 * pad,), 5.0, device="cuda")
+    fin = fbuf[pad:pad + nf].view(2, 4, 64, 128)
+    need = ssd.ssd_chunk_scan_fwd_workspace_size(ssd.make_dims(2, 600, 4, 64, 128, 1), 256,
+                                                 torch.bfloat16)
+    wbuf = torch.full((need + 2 * pad,), 0xAB, device="cuda", dtype=torch.uint8)
+    ws = wbuf[pad:pad + need]
+    ssd.ssd_chunk_scan_fwd(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], inp["D"], 256,
+                           init_states=inp["init"], y=y, final_states=fin, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.all(ybuf[:pad] == 7.0) and torch.all(ybuf[-pad:] == 7.0)
+    assert torch.all(fbuf[:pad] == 5.0) and torch.all(fbuf[-pad:] == 5.0)
+    assert torch.all(wbuf[:pad] == 0xAB) and torch.all(wbuf[-pad:] == 0xAB)
+    assert torch.isfinite(y.float()).all() and torch.isfinite(fin).all()
+
+
+def test_tensor_core_path_selected_for_layer_shapes():
+    dims = ssd.make_dims(4, 8192, 80, 64, 128, 1)
+    assert ssd.ssd_chunk_scan_fwd_uses_tensor_cores(dims, 256, torch.bfloat16) in (0, 1)
+    assert ssd.ssd_chunk_scan_fwd_uses_tensor_cores(dims, 256, torch.float32) == 0
