@@ -1,0 +1,475 @@
+"""Benchmark of the SSD layer on B200.
+
+A step is one chunked forward (all four steps of the block-decomposed
+algorithm: chunk states, inter-chunk recurrence, intra-chunk masked C B^T
+term and entering-state term + D skip) over the 2.7B-layer workload
+(batch 4, L 8192, H 80, P 64, N 128, G 1, chunk 256, bf16 x/B/C, fp32 dt/A/D,
+random initial states, final states returned), with inputs resident in HBM.
+The decode step (batch 256, H 80, P 64, N 128) is timed in the same run and
+reported under "decode".
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+With N > 1 (launched by torchrun) every rank runs the same per-GPU workload
+(weak scaling; the layer shards over batch and heads with no exchange) and
+rank 0 prints one JSON line with the max-over-ranks device time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "SSD fwd tokens/s and TFLOP/s (% bf16 TC peak) at 2.7B-layer shape; decode GB/s"
+UNIT = "tokens/s"
+L2_FLUSH_BYTES = 512 << 20
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return {"hbm_gbs": j["hbm_gbs"], "bf16_tflops": j["bf16_tflops"],
+                "bf16_tflops_sustained": j.get("bf16_tflops_sustained", j["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+# ---------------------------------------------------------------- workload model
+def fwd_model(w):
+    """Algorithmic FLOPs and minimum HBM bytes of one chunked forward."""
+    b, L, H, P, N, G, Q = w.batch, w.seqlen, w.nheads, w.headdim, w.dstate, w.ngroups, w.chunk
+    sx = 2 if w.dtype == "bf16" else 4
+    # causal half of the diagonal blocks, C B^T once per group, states in and out
+    f_alg = 2 * b * L * (G * N * (Q + 1) / 2 + H * P * (Q + 1) / 2 + 2 * H * N * P)
+    f_dense = 2 * b * L * (G * N * Q + H * P * Q + 2 * H * N * P)
+    n_state = b * H * P * N
+    bytes_min = (b * L * (2 * H * P * sx + 2 * G * N * sx + 4 * H)
+                 + 4 * n_state * (int(w.with_init) + int(w.want_final)))
+    return f_alg, f_dense, bytes_min
+
+
+def kernel_bytes(w):
+    """Bytes each kernel of the three-kernel forward must move (its inputs
+    and outputs, each once)."""
+    b, L, H, P, N, G, Q = w.batch, w.seqlen, w.nheads, w.headdim, w.dstate, w.ngroups, w.chunk
+    sx = 2 if w.dtype == "bf16" else 4
+    T = (L + Q - 1) // Q
+    ns = b * T * H * P * N
+    x = b * L * H * P * sx
+    bc = b * L * G * N * sx
+    dt = b * L * H * 4
+    init = 4 * b * H * P * N * int(w.with_init)
+    fin = 4 * b * H * P * N * int(w.want_final)
+    return {
+        "chunk_state": x + bc + dt + 4 * ns + 4 * b * T * H,
+        "state_pass": 4 * ns + 4 * b * T * H + sx * ns + init + fin,
+        "chunk_out": 2 * x + 2 * bc + dt + sx * ns,
+    }
+
+
+KERNEL_SOURCES = {
+    "chunk_state": ["chunk_state_tc.cu", "chunk_simt.cu"],
+    "state_pass": ["state_pass.cu"],
+    "chunk_out": ["chunk_out_tc.cu", "chunk_simt.cu"],
+    "decode": ["decode.cu"],
+}
+
+
+def source_sha(kernel: str) -> str:
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES[kernel]:
+        p = os.path.join(ROOT, "ssd_chunked_scan_02_b200", "csrc", f)
+        if os.path.exists(p):
+            h.update(open(p, "rb").read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(kernel: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current source of that kernel; else None."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        j = json.load(f)
+    e = j.get(kernel)
+    if not e or e.get("workload") != workload or e.get("source_sha") != source_sha(kernel):
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"ssd_bench_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [s.strip() for s in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        try:
+            os.remove(self.path)
+        except OSError:
+            pass
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[k] for r in rows for k in range(4) if r[5 + k] == "Active"})
+        loaded = [s for s in sm if mx and s > 0.5 * max(mx)] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ---------------------------------------------------------------- distributed plumbing
+def dist_setup(n):
+    import torch
+    if n <= 1:
+        return 0, 1, 0
+    import torch.distributed as dist
+    rank = int(os.environ["RANK"])
+    world = int(os.environ["WORLD_SIZE"])
+    local = int(os.environ.get("LOCAL_RANK", rank))
+    torch.cuda.set_device(local)
+    import datetime
+    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                            device_id=torch.device("cuda", local))
+    return rank, world, local
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world <= 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], device="cuda", dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ---------------------------------------------------------------- CPU oracle baseline
+def cpu_oracle_sample(w, inp_cpu, seconds_budget: float = 12.0):
+    """Time the fp64 oracle on a bounded sample of the workload: batch
+    element 0 (all heads, the whole sequence), repeated for about
+    ``seconds_budget`` seconds.  Returns
+    (tokens/s scaled to the full layer, description, cores)."""
+    import oracle
+    cores = os.cpu_count() or 1
+    heads = w.nheads
+    sl = {
+        "x": inp_cpu["x"][0:1, :, :heads], "dt": inp_cpu["dt"][0:1, :, :heads],
+        "A": inp_cpu["A"][:heads], "B": inp_cpu["B"][0:1], "C": inp_cpu["C"][0:1],
+        "D": inp_cpu["D"][:heads],
+        "init": inp_cpu["init"][0:1, :heads] if inp_cpu.get("init") is not None else None,
+    }
+    args = [oracle._f64(sl[k]) for k in ("x", "dt", "A", "B", "C", "D")]
+    init = oracle._f64(sl["init"]) if sl["init"] is not None else None
+    t0 = time.perf_counter()
+    reps = 0
+    while True:
+        oracle.recurrence(*args, init, threads=cores)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el > seconds_budget or reps >= 1000:
+            break
+    per = el / reps
+    # the sample covers heads/H of one batch element's tokens
+    frac = heads / w.nheads
+    tok_s = w.seqlen * frac / per
+    desc = (f"fp64 oracle recurrence over batch 0, heads 0..{heads - 1} of {w.nheads}, "
+            f"L={w.seqlen} ({reps} reps, {per:.3f} s each); tokens/s scaled by heads")
+    return tok_s, desc, cores
+
+
+# ---------------------------------------------------------------- reference arm
+def run_reference(args):
+    """The reference arm here is the fp64 CPU oracle, timed as it stands."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import torch
+    from ssd_chunked_scan_02_b200 import inputs
+    w = inputs.LAYER_2P7B
+    inp = inputs.make_inputs(w)
+    times = []
+    cores = os.cpu_count() or 1
+    desc = None
+    for i in range(args.warmup + args.steps):
+        tok_s, desc, cores = cpu_oracle_sample(w, inp, seconds_budget=3.0)
+        if i >= args.warmup:
+            times.append(tok_s)
+    value = statistics.mean(times)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * w.tokens / value, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "batch": w.batch, "seqlen": w.seqlen, "nheads": w.nheads,
+                   "headdim": w.headdim, "dstate": w.dstate, "ngroups": w.ngroups,
+                   "chunk": w.chunk, "l2": "n/a (CPU)"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+    return 0
+
+
+# ---------------------------------------------------------------- GPU arm
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--decode-steps", type=int, default=50)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    import torch
+    from ssd_chunked_scan_02_b200 import inputs, ssd
+
+    rank, world, local = dist_setup(args.gpus)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(dev)
+    pk = peaks()
+
+    w = inputs.LAYER_2P7B
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(w.seed + 1000 * rank)
+    inp = inputs.make_inputs(w, device=dev, gen=gen)
+    x, dt, A, Bm, Cm, D, init = (inp[k] for k in ("x", "dt", "A", "B", "C", "D", "init"))
+    y = torch.empty_like(x)
+    fin = torch.empty((w.batch, w.nheads, w.headdim, w.dstate), device=dev, dtype=torch.float32)
+    dims = ssd.make_dims(w.batch, w.seqlen, w.nheads, w.headdim, w.dstate, w.ngroups)
+    need = ssd.ssd_chunk_scan_fwd_workspace_size(dims, w.chunk, x.dtype)
+    ws = torch.empty(need, device=dev, dtype=torch.uint8)
+    flush = torch.empty(L2_FLUSH_BYTES, device=dev, dtype=torch.uint8)
+    uses_tc = ssd.ssd_chunk_scan_fwd_uses_tensor_cores(dims, w.chunk, x.dtype) == 1
+
+    def fwd():
+        ssd.ssd_chunk_scan_fwd(x, dt, A, Bm, Cm, D, w.chunk, init_states=init, y=y,
+                               final_states=fin, workspace=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        fwd()
+    torch.cuda.synchronize(dev)
+
+    sampler = ClockSampler(local) if rank == 0 else None
+    if sampler:
+        sampler.start()
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    for s, e in evs:
+        flush.zero_()                      # L2 flush between timed steps (not timed)
+        s.record(stream)
+        fwd()
+        e.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    step_ms = [s.elapsed_time(e) for s, e in evs]
+    total_ms = max_over_ranks(sum(step_ms), world)
+    clocks = sampler.stop() if sampler else None
+    ms_per_step = total_ms / args.steps
+
+    # ---- per-kernel times (same stream, CUDA events between the three launches)
+    T = (w.seqlen + w.chunk - 1) // w.chunk
+    S_buf = torch.empty((w.batch, T, w.nheads, w.headdim, w.dstate), device=dev,
+                        dtype=torch.float32)
+    ld_buf = torch.empty((w.batch, T, w.nheads), device=dev, dtype=torch.float32)
+    prev_buf = torch.empty((w.batch, T, w.nheads, w.headdim, w.dstate), device=dev,
+                           dtype=x.dtype)
+    lib = ssd.load()
+    import ctypes
+    sp = ctypes.c_void_p(stream.cuda_stream)
+    P = lambda t: ctypes.c_void_p(t.data_ptr()) if t is not None else None
+    kt = {"chunk_state": [], "state_pass": [], "chunk_out": []}
+    reps = max(5, args.steps // 2)
+    for r in range(reps + 2):
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        flush.zero_()
+        ev[0].record(stream)
+        lib.ssd_chunk_state_fwd(P(x), P(dt), P(A), P(Bm), w.chunk, P(S_buf), P(ld_buf),
+                                ctypes.byref(dims), ssd.SSD_BF16, sp)
+        ev[1].record(stream)
+        lib.ssd_state_passing_fwd(P(S_buf), P(ld_buf), P(init), P(prev_buf), P(fin), w.chunk,
+                                  ctypes.byref(dims), ssd.SSD_BF16, sp)
+        ev[2].record(stream)
+        lib.ssd_chunk_output_fwd(P(x), P(dt), P(A), P(Bm), P(Cm), P(D), P(prev_buf), w.chunk,
+                                 P(y), ctypes.byref(dims), ssd.SSD_BF16, sp)
+        ev[3].record(stream)
+        torch.cuda.synchronize(dev)
+        if r >= 2:
+            kt["chunk_state"].append(ev[0].elapsed_time(ev[1]))
+            kt["state_pass"].append(ev[1].elapsed_time(ev[2]))
+            kt["chunk_out"].append(ev[2].elapsed_time(ev[3]))
+    kmean = {k: statistics.mean(v) for k, v in kt.items()}
+    dom = max(kmean, key=kmean.get)
+    kb = kernel_bytes(w)
+    dom_gbs = kb[dom] / (kmean[dom] * 1e-3) / 1e9
+
+    # ---- decode step (b=256, H=80, P=64, N=128), state resident
+    dw = inputs.DECODE_2P7B
+    dgen = torch.Generator(device=dev)
+    dgen.manual_seed(dw.seed + 1000 * rank)
+    _, dpar = inputs.make_decode_params(dw, device=dev, gen=dgen)
+    toks = [inputs.make_decode_token(dw, dgen, device=dev) for _ in range(4)]
+    dstate = dpar["state"]
+    ydec = torch.empty((dw.batch, dw.nheads, dw.headdim), device=dev, dtype=torch.bfloat16)
+
+    def dstep(i):
+        t = toks[i % len(toks)]
+        ssd.ssd_step(dstate, t["x"], t["dt"], dpar["A"], t["B"], t["C"], dpar["D"], y=ydec,
+                     stream=stream)
+    for i in range(5):
+        dstep(i)
+    torch.cuda.synchronize(dev)
+    dms = []
+    for i in range(args.decode_steps):
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        flush.zero_()
+        s.record(stream)
+        dstep(i)
+        e.record(stream)
+        dms.append((s, e))
+    torch.cuda.synchronize(dev)
+    dec_ms = statistics.mean([s.elapsed_time(e) for s, e in dms])
+    dec_bytes = (2 * 4 * dw.batch * dw.nheads * dw.headdim * dw.dstate
+                 + dw.batch * dw.nheads * (2 * dw.headdim * 2 + 4)
+                 + 2 * 2 * dw.batch * dw.ngroups * dw.dstate)
+    dec_gbs = dec_bytes / (dec_ms * 1e-3) / 1e9
+
+    # ---- end to end through the C ABI with host buffers (pinned), copies timed
+    host = {k: (v.cpu().pin_memory() if v is not None else None) for k, v in inp.items()}
+    y_host = torch.empty(y.shape, dtype=y.dtype, pin_memory=True)
+    f_host = torch.empty(fin.shape, dtype=fin.dtype, pin_memory=True)
+    h2d = sum(v.numel() * v.element_size() for k, v in host.items()
+              if v is not None and k not in ("A", "D")) + A.numel() * 4 + D.numel() * 4
+    d2h = y.numel() * y.element_size() + fin.numel() * 4
+
+    def e2e_step():
+        for k in ("x", "dt", "B", "C", "init", "A", "D"):
+            if host[k] is not None:
+                inp[k].copy_(host[k], non_blocking=True)
+        fwd()
+        y_host.copy_(y, non_blocking=True)
+        f_host.copy_(fin, non_blocking=True)
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    e2e_steps = max(3, args.steps // 4)
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(s.elapsed_time(e), world) / e2e_steps
+
+    # ---- CPU oracle baseline (rank 0, N = 1 only)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        inp_cpu = {k: (v.cpu() if v is not None else None) for k, v in inp.items()}
+        tok_s, desc, cores = cpu_oracle_sample(w, inp_cpu)
+        cpu = {"value": tok_s, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc}
+
+    if rank == 0:
+        f_alg, f_dense, bytes_min = fwd_model(w)
+        t = ms_per_step * 1e-3
+        tok_s = world * w.tokens / t
+        t_roof = max(bytes_min / (pk["hbm_gbs"] * 1e9), f_dense / (pk["bf16_tflops"] * 1e12))
+        bound = "hbm"
+        peak_gbs = pk["hbm_gbs"]
+        line = {
+            "metric": METRIC, "value": tok_s, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": w.name, "batch": w.batch, "seqlen": w.seqlen,
+                       "nheads": w.nheads, "headdim": w.headdim, "dstate": w.dstate,
+                       "ngroups": w.ngroups, "chunk": w.chunk, "init_states": True,
+                       "final_states": True, "tensor_cores": uses_tc,
+                       "l2": "flushed (512 MiB write) before every timed step; inputs > L2"},
+            "tflops": {"alg": f_alg / t / 1e12, "dense": f_dense / t / 1e12,
+                       "pct_bf16_peak_dense": 100 * f_dense / t / 1e12 / pk["bf16_tflops"],
+                       "pct_bf16_peak_alg": 100 * f_alg / t / 1e12 / pk["bf16_tflops"],
+                       "peak_tflops": pk["bf16_tflops"], "peak_source": pk["source"]},
+            "roofline": {"bound": bound, "kernel": dom, "achieved": dom_gbs, "peak": peak_gbs,
+                         "unit": "GB/s", "frac": dom_gbs / peak_gbs,
+                         "traffic": traffic_for(dom, w.name),
+                         "alg_bytes_per_launch": kb[dom], "ms_per_launch": kmean[dom],
+                         "peak_source": pk["source"]},
+            "roofline_step": {"bound": "hbm", "bytes_min": bytes_min,
+                              "achieved_gbs": bytes_min / t / 1e9,
+                              "t_min_ms": 1e3 * t_roof, "frac": t_roof / t},
+            "kernels_ms": kmean,
+            "decode": {"workload": dw.name, "ms_per_step": dec_ms, "gbs": dec_gbs,
+                       "frac_hbm": dec_gbs / peak_gbs, "bytes_per_step": dec_bytes},
+            "e2e": {"value": world * w.tokens / (e2e_ms * 1e-3), "unit": UNIT,
+                    "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "cpu_baseline": cpu,
+            "gpu_launches": 3 * args.steps,
+            "clocks": clocks,
+        }
+        print(json.dumps(line))
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())
