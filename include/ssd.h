@@ -158,6 +158,31 @@ SSD_API ssd_status_t ssd_chunk_output_fwd(const void* x, const float* dt, const 
                                   int chunk_size, void* y, const ssd_dims_t* dims,
                                   ssd_dtype_t dtype, void* stream);
 
+/*
+ * ssd_chunk_scan_fwd for callers that cannot allocate device memory (a plugin
+ * inside a host runtime that owns the device heap and offers no allocator,
+ * or a latency-critical path that cannot afford the device-wide
+ * synchronisation of cudaMalloc/cudaFree).  The pages describe no
+ * counterpart: this is a library convenience, not part of the method.
+ * Same arguments and result as ssd_chunk_scan_fwd, without the workspace:
+ * the scratch comes from one fixed device array of SSD_NOALLOC_SCRATCH_BYTES
+ * inside the library, resident on every GPU that loads the library until
+ * the process exits.  Sizes whose workspace (ssd_chunk_scan_fwd_workspace_size)
+ * exceeds that return SSD_ERR_UNSUPPORTED with a message.  The first call
+ * on each device looks up the array's device address (cudaGetSymbolAddress)
+ * with that device current; make it before any stream capture.  Nothing is
+ * allocated or freed.  All calls share the array and it keeps the last
+ * call's contents (every byte read is rewritten first within a call, so no
+ * clearing is needed), so calls that overlap on the GPU race: serialise them.
+ */
+#define SSD_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+SSD_API ssd_status_t ssd_chunk_scan_fwd_noalloc(const void* x, const float* dt, const float* A,
+                                                const void* B, const void* C, const float* D,
+                                                int chunk_size, const float* init_states,
+                                                void* y, float* final_states,
+                                                const ssd_dims_t* dims, ssd_dtype_t dtype,
+                                                void* stream);
+
 /* Which kernel family ssd_chunk_scan_fwd uses for these sizes:
  * 1 = tcgen05 tensor-core kernels, 0 = SIMT fp32 kernels, -1 = rejected. */
 SSD_API int ssd_chunk_scan_fwd_uses_tensor_cores(const ssd_dims_t* dims, int chunk_size,

@@ -96,6 +96,16 @@ bool tc_eligible(const ssd::Dims& d, ssd::Elt t) { return ssd::tc_supported(d, t
 
 }  // namespace
 
+namespace ssd {
+// Records a message for ssd_last_error_detail() on this host thread.
+void set_error_detail(const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_detail, sizeof(g_detail), fmt, ap);
+    va_end(ap);
+}
+}  // namespace ssd
+
 extern "C" {
 
 const char* ssd_status_string(ssd_status_t s) {

@@ -24,7 +24,8 @@ SSD_F32, SSD_BF16 = 0, 1
 
 EXPORTED = ("ssd_status_string", "ssd_last_error_detail", "ssd_chunk_scan_fwd_workspace_size",
             "ssd_chunk_scan_fwd", "ssd_step", "ssd_chunk_state_fwd", "ssd_state_passing_fwd",
-            "ssd_chunk_output_fwd", "ssd_chunk_scan_fwd_uses_tensor_cores")
+            "ssd_chunk_output_fwd", "ssd_chunk_scan_fwd_uses_tensor_cores",
+            "ssd_chunk_scan_fwd_noalloc")
 
 
 class SSDError(RuntimeError):
@@ -65,6 +66,9 @@ def load(path: str = LIB_PATH):
     lib.ssd_chunk_scan_fwd.restype = ctypes.c_int
     lib.ssd_chunk_scan_fwd.argtypes = [_vp] * 6 + [ctypes.c_int, _vp, _vp, _vp, dims_p,
                                                    ctypes.c_int, _vp, ctypes.c_size_t, _vp]
+    lib.ssd_chunk_scan_fwd_noalloc.restype = ctypes.c_int
+    lib.ssd_chunk_scan_fwd_noalloc.argtypes = [_vp] * 6 + [ctypes.c_int, _vp, _vp, _vp, dims_p,
+                                                           ctypes.c_int, _vp]
     lib.ssd_step.restype = ctypes.c_int
     lib.ssd_step.argtypes = [_vp] * 8 + [dims_p, ctypes.c_int, _vp]
     lib.ssd_chunk_state_fwd.restype = ctypes.c_int
@@ -157,6 +161,30 @@ def ssd_chunk_scan_fwd(x, dt, A, B, C, D, chunk_size: int, init_states=None,
                                    _ptr(workspace), workspace.numel(), _stream(stream))
     _check(st, "ssd_chunk_scan_fwd")
     return (y, final_states) if (return_final_states or final_states is not None) else y
+
+
+def ssd_chunk_scan_fwd_noalloc(x, dt, A, B, C, D, chunk_size: int, init_states=None,
+                               return_final_states: bool = False, y=None, final_states=None,
+                               stream=None):
+    """ssd_chunk_scan_fwd without a caller workspace: the library's built-in
+    scratch array (SSD_NOALLOC_SCRATCH_BYTES) is used instead.  For callers
+    that cannot allocate device memory; calls that overlap on the GPU race on
+    that array."""
+    dims = _fwd_dims(x, B)
+    if y is None:
+        y = torch.empty_like(x)
+    if return_final_states and final_states is None:
+        final_states = torch.empty((x.shape[0], x.shape[2], x.shape[3], B.shape[3]),
+                                   device=x.device, dtype=torch.float32)
+    st = load().ssd_chunk_scan_fwd_noalloc(_ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+                                           int(chunk_size), _ptr(init_states), _ptr(y),
+                                           _ptr(final_states), ctypes.byref(dims),
+                                           _dtype_code(x.dtype), _stream(stream))
+    _check(st, "ssd_chunk_scan_fwd_noalloc")
+    return (y, final_states) if (return_final_states or final_states is not None) else y
+
+
+NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
 
 
 def ssd_step(state, x, dt, A, B, C, D, y=None, stream=None):
