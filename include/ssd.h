@@ -183,6 +183,15 @@ SSD_API ssd_status_t ssd_chunk_scan_fwd_noalloc(const void* x, const float* dt, 
                                                 const ssd_dims_t* dims, ssd_dtype_t dtype,
                                                 void* stream);
 
+/*
+ * Reports, and clears, a device-side wait that gave up in an earlier call on
+ * the current device: the tensor-core kernels bound every wait, and one that
+ * runs out records SSD_ERR_TIMEOUT in a device status word and ends the
+ * kernel cleanly (its outputs are then incomplete).  Synchronises `stream`.
+ * Returns SSD_OK if no wait gave up, SSD_ERR_TIMEOUT if one did.
+ */
+SSD_API ssd_status_t ssd_poll_device_status(void* stream);
+
 /* Which kernel family ssd_chunk_scan_fwd uses for these sizes:
  * 1 = tcgen05 tensor-core kernels, 0 = SIMT fp32 kernels, -1 = rejected. */
 SSD_API int ssd_chunk_scan_fwd_uses_tensor_cores(const ssd_dims_t* dims, int chunk_size,

@@ -5,11 +5,8 @@
 // for autoregressive inference.
 //
 // The step is pure HBM streaming: every fp32 state element is read once and
-// written once, with two flops per byte.  A warp owns kRows consecutive
-// state rows (one row = the N-vector of one (batch, head, p)), each lane
-// moves 16-byte pieces, and all rows' loads are issued before any arithmetic
-// so each warp keeps kRows * 512 bytes in flight.  Loads and stores use the
-// streaming cache hints (the state is touched once per step).
+// written once, with two flops per byte.  Loads and stores of the state use
+// the streaming cache hints (it is touched once per step).
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -18,7 +15,6 @@
 namespace ssd {
 namespace {
 
-constexpr int kRows = 4;
 constexpr int kThreads = 256;
 
 template <typename T>
@@ -37,67 +33,66 @@ __device__ __forceinline__ void load4<__nv_bfloat16>(const __nv_bfloat16* p, flo
     v[0] = a.x; v[1] = a.y; v[2] = b.x; v[3] = b.y;
 }
 
-// N % 4 == 0 and N <= 128 * kMaxPieces: each lane handles up to kMaxPieces
-// 4-element pieces of each row.
-constexpr int kMaxPieces = 2;
-
-template <typename T>
+// One 256-thread block per (batch, head): the head's P x N fp32 state is
+// P * N / 4 float4 items; thread t owns items t, t + 256, ... so each warp
+// covers whole rows (NV = N / 4 lanes per row, NV a power of two <= 32) and
+// always the same four state columns, whose B and C values it loads once.
+// dt, A, D and the head's x row are loaded once per block; eight state items
+// per thread are loaded before any arithmetic.
+template <typename T, int NV>
 __global__ void __launch_bounds__(kThreads)
-step_kernel_v4(float* __restrict__ state, const T* __restrict__ x, const float* __restrict__ dt,
+step_kernel_bh(float* __restrict__ state, const T* __restrict__ x, const float* __restrict__ dt,
                const float* __restrict__ A, const T* __restrict__ Bm, const T* __restrict__ Cm,
-               const float* __restrict__ Dv, T* __restrict__ y, int64_t b, int64_t H, int64_t P,
-               int64_t N, int64_t G) {
-    const int lane = threadIdx.x & 31;
-    const int64_t warp = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5;
-    const int64_t nwarps = ((int64_t)gridDim.x * kThreads) >> 5;
-    const int64_t rows = b * H * P;
-    const int64_t hpg = H / G;
+               const float* __restrict__ Dv, T* __restrict__ y, int64_t H, int64_t P,
+               int64_t G) {
+    constexpr int N = NV * 4;
+    constexpr int kBatch = 8;
+    __shared__ float s_x[256];
+    const int tid = threadIdx.x;
+    const int64_t bh = blockIdx.x;
+    const int64_t bb = bh / H, h = bh - bb * H, g = h / (H / G);
+    for (int p = tid; p < P; p += kThreads) s_x[p] = to_f32(x[bh * P + p]);
+    const float dtv = dt[bh];
+    const float a = expf(dtv * A[h]);
+    const float Dh = Dv[h];
+    const int n4 = tid % NV;
+    float bv[4], cv[4];
+    load4<T>(Bm + (bb * G + g) * N + n4 * 4, bv);
+    load4<T>(Cm + (bb * G + g) * N + n4 * 4, cv);
+    __syncthreads();
 
-    for (int64_t r0 = warp * kRows; r0 < rows; r0 += nwarps * kRows) {
-        float s[kRows][kMaxPieces][4];
+    float4* base = reinterpret_cast<float4*>(state + bh * P * N);
+    const int items = (int)(P * NV);
+    for (int k0 = 0; k0 < items; k0 += kBatch * kThreads) {
+        float4 sv[kBatch];
 #pragma unroll
-        for (int r = 0; r < kRows; ++r) {
-            const int64_t row = r0 + r;
-#pragma unroll
-            for (int k = 0; k < kMaxPieces; ++k) {
-                const int64_t n0 = (int64_t)(k * 32 + lane) * 4;
-                if (row < rows && n0 < N) {
-                    const float4 q = __ldcs(reinterpret_cast<const float4*>(state + row * N + n0));
-                    s[r][k][0] = q.x; s[r][k][1] = q.y; s[r][k][2] = q.z; s[r][k][3] = q.w;
-                }
-            }
+        for (int k = 0; k < kBatch; ++k) {
+            const int it = k0 + k * kThreads + tid;
+            if (it < items) sv[k] = __ldcs(base + it);
         }
 #pragma unroll
-        for (int r = 0; r < kRows; ++r) {
-            const int64_t row = r0 + r;
-            if (row >= rows) break;
-            const int64_t bh = row / P;
-            const int64_t bb = bh / H, h = bh - bb * H, g = h / hpg;
-            const float dtv = dt[bh];
-            const float a = expf(dtv * A[h]);
-            const float xv = to_f32(x[row]);
-            const float u = dtv * xv;
-            const T* Bt = Bm + (bb * G + g) * N;
-            const T* Ct = Cm + (bb * G + g) * N;
-            float acc = 0.f;
-#pragma unroll
-            for (int k = 0; k < kMaxPieces; ++k) {
-                const int64_t n0 = (int64_t)(k * 32 + lane) * 4;
-                if (n0 < N) {
-                    float bv[4], cv[4];
-                    load4<T>(Bt + n0, bv);
-                    load4<T>(Ct + n0, cv);
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        s[r][k][e] = fmaf(a, s[r][k][e], u * bv[e]);
-                        acc = fmaf(s[r][k][e], cv[e], acc);
-                    }
-                    __stcs(reinterpret_cast<float4*>(state + row * N + n0),
-                           make_float4(s[r][k][0], s[r][k][1], s[r][k][2], s[r][k][3]));
-                }
+        for (int k = 0; k < kBatch; ++k) {
+            const int it = k0 + k * kThreads + tid;
+            const bool valid = it < items;
+            const int p = it / NV;
+            float acc = 0.f, xv = 0.f;
+            if (valid) {
+                xv = s_x[p];
+                const float u = dtv * xv;
+                float4 q = sv[k];
+                q.x = fmaf(a, q.x, u * bv[0]);
+                q.y = fmaf(a, q.y, u * bv[1]);
+                q.z = fmaf(a, q.z, u * bv[2]);
+                q.w = fmaf(a, q.w, u * bv[3]);
+                __stcs(base + it, q);
+                acc = q.x * cv[0];
+                acc = fmaf(q.y, cv[1], acc);
+                acc = fmaf(q.z, cv[2], acc);
+                acc = fmaf(q.w, cv[3], acc);
             }
-            acc = warp_sum(acc);
-            if (lane == 0) y[row] = from_f32<T>(acc + Dv[h] * xv);
+#pragma unroll
+            for (int o = NV / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+            if (valid && n4 == 0) y[bh * P + p] = from_f32<T>(acc + Dh * xv);
         }
     }
 }
@@ -139,23 +134,27 @@ cudaError_t run(float* state, const void* x, const float* dt, const float* A, co
                 const void* C, const float* D, void* y, const Dims& d, cudaStream_t s) {
     const int64_t rows = d.b * d.H * d.P;
     if (rows == 0) return cudaSuccess;
-    int dev = 0, sms = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const int warps_per_block = kThreads / 32;
-    const bool v4 = (d.N % 4 == 0) && (d.N <= 128 * kMaxPieces);
-    const int64_t rows_per_block = warps_per_block * (v4 ? kRows : 1);
-    int64_t blocks = (rows + rows_per_block - 1) / rows_per_block;
-    const int64_t cap = (int64_t)sms * 8;  // 8 resident 256-thread blocks per SM
-    if (blocks > cap) blocks = cap;
-    if (v4) {
-        step_kernel_v4<T><<<(unsigned)blocks, kThreads, 0, s>>>(
-            state, static_cast<const T*>(x), dt, A, static_cast<const T*>(B),
-            static_cast<const T*>(C), D, static_cast<T*>(y), d.b, d.H, d.P, d.N, d.G);
+    const T* xp = static_cast<const T*>(x);
+    const T* Bp = static_cast<const T*>(B);
+    const T* Cp = static_cast<const T*>(C);
+    T* yp = static_cast<T*>(y);
+    const int64_t bh = d.b * d.H;
+    if (d.N == 128 && bh <= 0x7fffffffLL) {
+        step_kernel_bh<T, 32><<<(unsigned)bh, kThreads, 0, s>>>(state, xp, dt, A, Bp, Cp, D, yp,
+                                                              d.H, d.P, d.G);
+    } else if (d.N == 64 && bh <= 0x7fffffffLL) {
+        step_kernel_bh<T, 16><<<(unsigned)bh, kThreads, 0, s>>>(state, xp, dt, A, Bp, Cp, D, yp,
+                                                              d.H, d.P, d.G);
     } else {
-        step_kernel_scalar<T><<<(unsigned)blocks, kThreads, 0, s>>>(
-            state, static_cast<const T*>(x), dt, A, static_cast<const T*>(B),
-            static_cast<const T*>(C), D, static_cast<T*>(y), d.b, d.H, d.P, d.N, d.G);
+        int dev = 0, sms = 148;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        const int64_t warps_per_block = kThreads / 32;
+        int64_t blocks = (rows + warps_per_block - 1) / warps_per_block;
+        const int64_t cap = (int64_t)sms * 8;
+        if (blocks > cap) blocks = cap;
+        step_kernel_scalar<T><<<(unsigned)blocks, kThreads, 0, s>>>(state, xp, dt, A, Bp, Cp, D, yp,
+                                                                   d.b, d.H, d.P, d.N, d.G);
     }
     return cudaGetLastError();
 }

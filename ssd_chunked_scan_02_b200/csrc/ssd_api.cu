@@ -8,6 +8,7 @@
 
 #include "../../include/ssd.h"
 #include "ssd_internal.h"
+#include "tc_host.h"
 #include "tc_kernels.h"
 
 namespace {
@@ -246,6 +247,15 @@ ssd_status_t ssd_chunk_output_fwd(const void* x, const float* dt, const float* A
                         ? ssd::launch_chunk_out_tc(x, dt, A, B, C, D, prev_states, y, d, s)
                         : ssd::launch_chunk_out_simt(x, dt, A, B, C, D, prev_states, y, d, t, s);
     return e == cudaSuccess ? SSD_OK : cuda_fail(e, "chunk-output kernel");
+}
+
+ssd_status_t ssd_poll_device_status(void* stream) {
+    g_detail[0] = 0;
+    unsigned int v = 0;
+    cudaError_t e = ssd::read_and_clear_device_status(&v, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "device status read");
+    if (v != 0) return fail(SSD_ERR_TIMEOUT, "a bounded device-side wait gave up (code %u)", v);
+    return SSD_OK;
 }
 
 ssd_status_t ssd_step(float* state, const void* x, const float* dt, const float* A,

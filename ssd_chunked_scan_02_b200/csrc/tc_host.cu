@@ -1,0 +1,96 @@
+// tc_host.cu -- host-side support for the tcgen05 kernels: which shapes they
+// cover, TMA tensor-map encoding (through the driver entry point, so the
+// library does not link libcuda), and the device status word that bounded
+// waits write when they give up.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "../../include/ssd.h"
+#include "sm100.cuh"
+#include "tc_host.h"
+#include "tc_kernels.h"
+
+namespace ssd {
+namespace {
+// Device status word: 0 = fine, 4 = a bounded wait in a kernel gave up.
+__device__ unsigned int g_device_status = 0;
+constexpr int kMaxDevices = 64;
+std::mutex g_status_mu;
+unsigned int* g_status_ptr[kMaxDevices] = {};
+}  // namespace
+
+unsigned int* device_status_ptr() {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lock(g_status_mu);
+    if (!g_status_ptr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return nullptr;
+        g_status_ptr[dev] = static_cast<unsigned int*>(p);
+    }
+    return g_status_ptr[dev];
+}
+
+bool tc_supported(const Dims& d, Elt t) {
+    if (t != Elt::BF16) return false;
+    if (d.P != 64) return false;
+    if (d.N != 64 && d.N != 128) return false;
+    if (d.Q != 128 && d.Q != 256) return false;
+    if ((d.H / d.G) % 2 != 0) return false;
+    if (d.L <= 0 || d.b <= 0) return false;
+    if (d.L > 0x7fffffffLL || d.b > 0x7fffffffLL) return false;   // TMA coordinates are int32
+    return true;
+}
+
+namespace {
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+}  // namespace
+
+bool tma_encoder_available() {
+    std::call_once(g_encode_once, [] {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    });
+    return g_encode != nullptr;
+}
+
+cudaError_t make_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+                           const uint64_t* strides_bytes, const uint32_t* box) {
+    if (!tma_encoder_available()) return cudaErrorNotSupported;
+    cuuint32_t estride[5] = {1, 1, 1, 1, 1};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank,
+                          const_cast<void*>(base), reinterpret_cast<const cuuint64_t*>(dims),
+                          reinterpret_cast<const cuuint64_t*>(strides_bytes),
+                          reinterpret_cast<const cuuint32_t*>(box), estride,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+cudaError_t read_and_clear_device_status(unsigned int* out, cudaStream_t s) {
+    unsigned int v = 0, zero = 0;
+    cudaError_t e = cudaMemcpyFromSymbolAsync(&v, g_device_status, sizeof(v), 0,
+                                              cudaMemcpyDeviceToHost, s);
+    if (e != cudaSuccess) return e;
+    e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return e;
+    if (v != 0) {
+        e = cudaMemcpyToSymbolAsync(g_device_status, &zero, sizeof(zero), 0,
+                                    cudaMemcpyHostToDevice, s);
+        if (e != cudaSuccess) return e;
+        e = cudaStreamSynchronize(s);
+        if (e != cudaSuccess) return e;
+    }
+    *out = v;
+    return cudaSuccess;
+}
+
+}  // namespace ssd

@@ -1,0 +1,24 @@
+// tc_host.h -- host helpers shared by the tcgen05 kernel launchers.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace ssd {
+
+// Encodes a bf16 tiled tensor map with 128-byte swizzle and zero fill for
+// out-of-range elements.  dims[0] is the innermost (contiguous) dimension;
+// strides_bytes[i] is the byte stride of dims[i + 1].
+cudaError_t make_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+                           const uint64_t* strides_bytes, const uint32_t* box);
+
+bool tma_encoder_available();
+
+// Device address of the status word that bounded waits write (current
+// device; looked up once per device).  nullptr if unavailable.
+unsigned int* device_status_ptr();
+
+// Copies the device status word to the host (synchronising `s`) and clears it.
+cudaError_t read_and_clear_device_status(unsigned int* out, cudaStream_t s);
+
+}  // namespace ssd

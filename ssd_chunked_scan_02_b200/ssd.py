@@ -25,7 +25,7 @@ SSD_F32, SSD_BF16 = 0, 1
 EXPORTED = ("ssd_status_string", "ssd_last_error_detail", "ssd_chunk_scan_fwd_workspace_size",
             "ssd_chunk_scan_fwd", "ssd_step", "ssd_chunk_state_fwd", "ssd_state_passing_fwd",
             "ssd_chunk_output_fwd", "ssd_chunk_scan_fwd_uses_tensor_cores",
-            "ssd_chunk_scan_fwd_noalloc")
+            "ssd_chunk_scan_fwd_noalloc", "ssd_poll_device_status")
 
 
 class SSDError(RuntimeError):
@@ -69,6 +69,8 @@ def load(path: str = LIB_PATH):
     lib.ssd_chunk_scan_fwd_noalloc.restype = ctypes.c_int
     lib.ssd_chunk_scan_fwd_noalloc.argtypes = [_vp] * 6 + [ctypes.c_int, _vp, _vp, _vp, dims_p,
                                                            ctypes.c_int, _vp]
+    lib.ssd_poll_device_status.restype = ctypes.c_int
+    lib.ssd_poll_device_status.argtypes = [_vp]
     lib.ssd_step.restype = ctypes.c_int
     lib.ssd_step.argtypes = [_vp] * 8 + [dims_p, ctypes.c_int, _vp]
     lib.ssd_chunk_state_fwd.restype = ctypes.c_int
@@ -198,6 +200,12 @@ def ssd_step(state, x, dt, A, B, C, D, y=None, stream=None):
                          _ptr(y), ctypes.byref(dims), _dtype_code(x.dtype), _stream(stream))
     _check(st, "ssd_step")
     return y
+
+
+def ssd_poll_device_status(stream=None):
+    """Raise SSDError(SSD_ERR_TIMEOUT) if a bounded device-side wait gave up
+    since the last poll (synchronises the stream)."""
+    _check(load().ssd_poll_device_status(_stream(stream)), "ssd_poll_device_status")
 
 
 def n_chunks(seqlen: int, chunk_size: int) -> int:

@@ -4,6 +4,8 @@ run the fp64 oracle on the same inputs (whole tensors, or sampled
 from __future__ import annotations
 
 import concurrent.futures as cf
+import json
+import os
 
 import numpy as np
 import torch
@@ -12,6 +14,15 @@ import oracle
 from ssd_chunked_scan_02_b200 import ssd
 
 TOL = {"f32": 1e-4, "bf16": 5e-3}
+
+
+def record(name: str, **errs):
+    """Append measured errors to $SSD_PARITY_LOG (JSON lines), when set, so
+    the margins to the tolerances stay visible."""
+    path = os.environ.get("SSD_PARITY_LOG")
+    if path:
+        with open(path, "a") as f:
+            f.write(json.dumps({"case": name, **errs}) + "\n")
 
 
 def rel_err(a, ref) -> float:

@@ -11,7 +11,7 @@ import pytest
 import torch
 
 import oracle
-from parity import TOL, gpu_fwd, oracle_fwd, oracle_pairs, rel_err, sample_pairs, to_dev
+from parity import TOL, gpu_fwd, oracle_fwd, oracle_pairs, record, rel_err, sample_pairs, to_dev
 from ssd_chunked_scan_02_b200 import inputs, ssd
 
 pytestmark = pytest.mark.gpu
@@ -28,6 +28,7 @@ def _check_full(w, chunk=None):
     y_ref, f_ref = oracle_fwd(inp)
     tol = TOL[w.dtype]
     ey, ef = rel_err(y, y_ref), rel_err(f, f_ref)
+    record(f"{w.name}_Q{chunk or w.chunk}", y=ey, final=ef)
     assert np.all(np.isfinite(y)) and np.all(np.isfinite(f))
     assert ey <= tol, f"{w.name} Q={chunk or w.chunk}: y rel err {ey:.3g} > {tol}"
     assert ef <= tol, f"{w.name} Q={chunk or w.chunk}: final rel err {ef:.3g} > {tol}"
@@ -86,6 +87,7 @@ def _check_sampled(w, k, seed):
     f_ref = np.stack([r[1] for r in refs])
     tol = TOL[w.dtype]
     ey, ef = rel_err(ys, y_ref), rel_err(fs, f_ref)
+    record(w.name, y=ey, final=ef)
     assert torch.isfinite(y.float()).all().item()
     assert ey <= tol, f"{w.name}: sampled y rel err {ey:.3g} > {tol}"
     assert ef <= tol, f"{w.name}: sampled final rel err {ef:.3g} > {tol}"
@@ -129,6 +131,7 @@ def test_decode_1024_steps_sampled():
             den_y = max(den_y, float(np.max(np.abs(yo[0, 0]))))
     torch.cuda.synchronize()
     ey = num_y / den_y
+    record("decode_1024", y=ey)
     fs = np.stack([state[b, h].double().cpu().numpy() for (b, h) in pairs])
     fr = np.stack([ost[p] for p in pairs])
     es = rel_err(fs, fr)
