@@ -10,19 +10,29 @@
 // decay; review page, 核心概念 items 3 and 5; 关键洞察 item 1 (block
 // decomposition lets the tensor cores do the work).
 //
-// One CTA per (batch, chunk, 128-row tile of the chunk, group of HG heads
-// that share B and C).  Rows i of the tile need columns j < 128 (t + 1).
-//   1. G = C_tile B^T (M = 128, N = 128 (t+1), K = dstate) into TMEM once per
-//      CTA; it is shared by the CTA's heads (B, C are per group, not per head).
-//   2. Per head: the decay mask is built in registers from the prefix sums of
-//      dt*A: on the diagonal 128 x 128 block M_ij = G_ij exp(cs_i - cs_j) dt_j
-//      (j <= i); on the block left of it (t = 1) the decay factorises through
-//      the block boundary r, M_ij = G_ij * exp(cs_i - r) * (exp(r - cs_j) dt_j),
-//      both factors <= 1, so no exponentials per element are needed there.
-//      M is written to TMEM as packed bf16 and used as the A operand of
-//      Y = M X (kind::f16, A from TMEM, B = x tile from shared memory).
-//   3. Z = C_tile h_prev^T (A = C tile, B = the head's entering state, bf16).
-//   4. Epilogue: y = Y + exp(cs_i) Z + D_h x, rounded to bf16 once.
+// One CTA per (batch, chunk, 128-row tile t of the chunk, group of HG heads
+// sharing B and C).  Rows i of tile t need columns j < 128 (t + 1).
+//
+//   prologue: G = C_t B^T (M = 128, N = 128 (t+1), K = dstate) into TMEM,
+//             once for all the CTA's heads (B, C are per group).  For t = 1
+//             the block left of the diagonal (G_10) is copied to shared
+//             memory as bf16 and only the diagonal block stays in TMEM.
+//   per head (pipelined over heads by warp role):
+//     mask warps       build M (bf16) in TMEM, M_ij = G_ij exp(cs_i - cs_j) dt_j
+//                      for j <= i.  Wherever a whole 32-column block lies below
+//                      the diagonal the decay factorises through the block's
+//                      end r: exp(cs_i - r) * (exp(r - cs_j) dt_j), both factors
+//                      <= 1, so only the 32 x 32 blocks on the diagonal need an
+//                      exponential per element.
+//     MMA lane         Y = M X (A from TMEM, kind::f16) and Z = C_t h_prev^T
+//                      into a double-buffered accumulator slot.
+//     epilogue group   y = Y + exp(cs_i) Z + D_h x, rounded to bf16 once, staged
+//                      in shared memory and written by TMA store.
+//     producer lane    TMA of the next heads' x rows and entering states.
+//
+// Warps 0-7: mask (two per TMEM lane quarter, splitting the columns); 8-11:
+// epilogue; 12: TMA producer; 13: MMA issuer (and TMEM owner).  Every wait is bounded; a warpgroup leaves its loop only when all
+// its threads agree (bar.red.or), so no named barrier is left half-arrived.
 #include <cuda.h>
 #include <cuda_bf16.h>
 
@@ -36,37 +46,48 @@ namespace ssd {
 namespace {
 using namespace sm100;
 
-constexpr int kThreads = 128;
+constexpr int kThreads = 448;
+constexpr int kMaxHeads = 16;
 constexpr float kLog2e = 1.4426950408889634f;
 
 template <int Q, int N>
 struct OutSmem {
-    static constexpr int kNB = N / 64;                     // 64-wide blocks of dstate
-    static constexpr int kC = 0;                           // kNB x 128 rows x 128 B
+    static constexpr int kNB = N / 64;                      // 64-wide blocks of dstate
+    static constexpr int kHTile = kNB * 64 * 128;           // one head's h_prev (64 x N bf16)
+    static constexpr int kC = 0;                            // C tile: kNB x 128 rows x 128 B
     static constexpr int kCBytes = kNB * 128 * 128;
-    static constexpr int kB = kC + kCBytes;                // kNB x Q rows x 128 B
+    static constexpr int kBG = kC + kCBytes;                // B tile (prologue), then G_10 + h ring
+    static constexpr int kG10Off = 0;                       // bf16 128 x 128 (t = 1 only)
+    static constexpr int kHOff = (Q == 256) ? 32768 : 0;    // h ring: 2 slots
     static constexpr int kBBytes = kNB * Q * 128;
-    static constexpr int kXTile = Q * 128;                 // x rows [0, Q) of one head
-    static constexpr int kX = kB + kBBytes;                // 2 buffers
-    static constexpr int kHTile = kNB * 64 * 128;          // h_prev of one head (64 x N)
-    static constexpr int kH = kX + 2 * kXTile;             // 2 buffers
-    static constexpr int kMaxHeads = 8;                    // heads per CTA (at most)
-    static constexpr int kCs = kH + 2 * kHTile;            // float [kMaxHeads][Q] prefix sums (log2 units)
-    static constexpr int kDt = kCs + kMaxHeads * Q * 4;    // float [kMaxHeads][Q]
-    static constexpr int kBeta = kDt + kMaxHeads * Q * 4;  // float [128]
-    static constexpr int kBar = kBeta + 128 * 4;           // 5 mbarriers
-    static constexpr int kTmem = kBar + 8 * 8;
-    static constexpr int kAbort = kTmem + 4;
-    static constexpr int kTotal = kAbort + 4;
+    static constexpr int kBGBytes = (kBBytes > kHOff + 2 * kHTile) ? kBBytes : kHOff + 2 * kHTile;
+    static constexpr int kXTile = Q * 128;                  // x rows [0, Q) of one head
+    static constexpr int kX = kBG + kBGBytes;               // x ring: 2 slots
+    static constexpr int kDt = kX + 2 * kXTile;             // float [kMaxHeads][Q]
+    static constexpr int kCs = kDt + kMaxHeads * Q * 4;     // float [2][Q] prefix sums (log2 units)
+    static constexpr int kBeta = kCs + 2 * Q * 4;           // float [128]
+    static constexpr int kBeta2 = kBeta + 128 * 4;          // float [128]
+    static constexpr int kEz = kBeta2 + 128 * 4;            // float [2][128] exp(cs_i) per slot
+    static constexpr int kAD = kEz + 2 * 128 * 4;           // float [2][kMaxHeads]: A_h, D_h
+    static constexpr int kYs = ((kAD + 2 * kMaxHeads * 4 + 1023) / 1024) * 1024;  // y staging: 2 x 16 KB
+    static constexpr int kBar = kYs + 2 * 128 * 128;        // 16 mbarriers
+    static constexpr int kTmem = kBar + 16 * 8;
+    static constexpr int kFlags = kTmem + 16;               // abort flags
+    static constexpr int kTotal = kFlags + 16;
     static constexpr int kAlloc = kTotal + 1024;
+};
+
+// mbarrier indices
+enum {
+    BAR_BC = 0, BAR_G = 1, BAR_GCONV = 2, BAR_XFULL = 3, BAR_XEMPTY = 5, BAR_MFULL = 7,
+    BAR_MEMPTY = 8, BAR_ACCFULL = 9, BAR_ACCEMPTY = 11, BAR_EZFULL = 13, BAR_COUNT = 15
 };
 
 // TMEM columns
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColG = 0;       // fp32 G, up to 256 columns
-constexpr uint32_t kColM = 256;     // bf16 mask (A operand), up to 128 columns
-constexpr uint32_t kColY = 384;     // fp32 Y, 64 columns
-constexpr uint32_t kColZ = 448;     // fp32 Z, 64 columns
+constexpr uint32_t kColM = 0;       // bf16 mask (A operand), up to 128 columns; G_10 in the prologue
+constexpr uint32_t kColG = 128;     // fp32 diagonal block of G, 128 columns
+constexpr uint32_t kColAcc = 256;   // two slots of 128: Y (64) then Z (64)
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
     return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
@@ -76,8 +97,8 @@ template <int Q, int N>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmH,
-                    const float* __restrict__ dt, const float* __restrict__ A,
-                    const float* __restrict__ Dv, __nv_bfloat16* __restrict__ y, int64_t L, int H,
+                    const __grid_constant__ CUtensorMap tmY, const float* __restrict__ dt,
+                    const float* __restrict__ A, const float* __restrict__ Dv, int64_t L, int H,
                     int G, int64_t T, int HG, unsigned int* status) {
     using S = OutSmem<Q, N>;
     constexpr int kTiles = Q / 128;
@@ -97,26 +118,28 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
     uint8_t* sC = smem + S::kC;
-    uint8_t* sB = smem + S::kB;
+    uint8_t* sB = smem + S::kBG;
+    uint8_t* sG10 = smem + S::kBG + S::kG10Off;
+    uint8_t* sH = smem + S::kBG + S::kHOff;
     uint8_t* sX = smem + S::kX;
-    uint8_t* sH = smem + S::kH;
-    float* s_cs = reinterpret_cast<float*>(smem + S::kCs);
     float* s_dt = reinterpret_cast<float*>(smem + S::kDt);
+    float* s_cs = reinterpret_cast<float*>(smem + S::kCs);
     float* s_beta = reinterpret_cast<float*>(smem + S::kBeta);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::kBar);  // 0 BC, 1-2 xh, 3 G, 4 YZ
+    float* s_beta2 = reinterpret_cast<float*>(smem + S::kBeta2);
+    float* s_ez = reinterpret_cast<float*>(smem + S::kEz);
+    float* s_Ah = reinterpret_cast<float*>(smem + S::kAD);
+    float* s_Dh = s_Ah + kMaxHeads;
+    uint8_t* sY = smem + S::kYs;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::kBar);
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + S::kTmem);
-    volatile int* s_abort = reinterpret_cast<volatile int*>(smem + S::kAbort);
+    volatile int* s_flag = reinterpret_cast<volatile int*>(smem + S::kFlags);   // [0]: any abort
 
     if (tid == 0) {
-        for (int i = 0; i < 5; ++i) mbar_init(&bars[i], 1);
-        *s_abort = 0;
+        for (int i = 0; i < BAR_COUNT; ++i) mbar_init(&bars[i], 1);
+        s_flag[0] = 0;
         fence_mbar_init();
-        prefetch_tmap(&tmX);
-        prefetch_tmap(&tmB);
-        prefetch_tmap(&tmC);
-        prefetch_tmap(&tmH);
     }
-    if (warp == 0) {
+    if (warp == 13) {
         tmem_alloc(s_tmem, kTmemCols);
         tmem_relinquish();
     }
@@ -124,237 +147,315 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *s_tmem;
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
 
-    bool bc_pending = false;
-    int g_pending = -1, yz_pending = -1;
-    int xh_pending[2] = {-1, -1};
-    int xh_issues[2] = {0, 0};
-
-    auto issue_xh = [&](int hi) {
-        const int buf = hi & 1;
-        const int h = head0 + hi;
-        mbar_expect_tx(&bars[1 + buf], (uint32_t)(KJ * 128 + S::kHTile));
-        for (int rb = 0; rb <= t; ++rb)
-            tma_load_4d(sX + buf * S::kXTile + rb * 128 * 128, &tmX, &bars[1 + buf], 0, h,
-                        (int)(t0 + rb * 128), (int)b);
-        const int hrow = (int)(((b * T + c) * H + h) * 64);
-#pragma unroll
-        for (int nb = 0; nb < S::kNB; ++nb)
-            tma_load_2d(sH + buf * S::kHTile + nb * 64 * 128, &tmH, &bars[1 + buf], nb * 64, hrow);
-        xh_pending[buf] = xh_issues[buf] & 1;
-        xh_issues[buf]++;
-    };
-
-    if (tid == 0) {
-        mbar_expect_tx(&bars[0], (uint32_t)(S::kCBytes + S::kNB * KJ * 128));
-#pragma unroll
-        for (int nb = 0; nb < S::kNB; ++nb) {
-            tma_load_4d(sC + nb * 128 * 128, &tmC, &bars[0], nb * 64, g, (int)(t0 + row0), (int)b);
-            for (int rb = 0; rb <= t; ++rb)
-                tma_load_4d(sB + nb * Q * 128 + rb * 128 * 128, &tmB, &bars[0], nb * 64, g,
-                            (int)(t0 + rb * 128), (int)b);
-        }
-        bc_pending = true;
-        issue_xh(0);
-        if (HG > 1) issue_xh(1);
-    }
-
-    // ---- dt of all the CTA's heads over columns [0, KJ) in one coalesced pass
-    // (heads of a token are contiguous), then per head the inclusive prefix
-    // sum of dt*A in log2 units (warp shuffles).
-    for (int e = tid; e < HG * KJ; e += kThreads) {
-        const int j = e / HG, k = e - j * HG;
-        s_dt[k * Q + j] = (j < len) ? dt[(b * L + t0 + j) * H + head0 + k] : 0.f;
-    }
-    __syncthreads();
-    for (int k = warp; k < HG; k += kThreads / 32) {
-        const float Ah = A[head0 + k] * kLog2e;
-        float carry = 0.f;
-        for (int base = 0; base < KJ; base += 32) {
-            float v = s_dt[k * Q + base + lane] * Ah;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const float u = __shfl_up_sync(0xffffffffu, v, o);
-                if (lane >= o) v += u;
+    if (warp == 12) {
+        // ================================================== TMA producer
+        if (lane == 0) {
+            prefetch_tmap(&tmX);
+            prefetch_tmap(&tmB);
+            prefetch_tmap(&tmC);
+            prefetch_tmap(&tmH);
+            mbar_expect_tx(&bars[BAR_BC], (uint32_t)(S::kCBytes + S::kNB * KJ * 128));
+            for (int nb = 0; nb < S::kNB; ++nb) {
+                tma_load_4d(sC + nb * 128 * 128, &tmC, &bars[BAR_BC], nb * 64, g,
+                            (int)(t0 + row0), (int)b);
+                for (int rb = 0; rb <= t; ++rb)
+                    tma_load_4d(sB + nb * Q * 128 + rb * 128 * 128, &tmB, &bars[BAR_BC], nb * 64,
+                                g, (int)(t0 + rb * 128), (int)b);
             }
-            v += carry;
-            s_cs[k * Q + base + lane] = v;
-            carry = __shfl_sync(0xffffffffu, v, 31);
+            auto load_x = [&](int hi) {
+                const int s = hi & 1;
+                mbar_expect_tx(&bars[BAR_XFULL + s], (uint32_t)(KJ * 128 + S::kHTile));
+                for (int rb = 0; rb <= t; ++rb)
+                    tma_load_4d(sX + s * S::kXTile + rb * 128 * 128, &tmX, &bars[BAR_XFULL + s], 0,
+                                head0 + hi, (int)(t0 + rb * 128), (int)b);
+            };
+            auto load_h = [&](int hi) {
+                const int s = hi & 1;
+                const int hrow = (int)(((b * T + c) * H + head0 + hi) * 64);
+                for (int nb = 0; nb < S::kNB; ++nb)
+                    tma_load_2d(sH + s * S::kHTile + nb * 64 * 128, &tmH, &bars[BAR_XFULL + s],
+                                nb * 64, hrow);
+            };
+            const int first = HG < 2 ? HG : 2;
+            for (int hi = 0; hi < first; ++hi) load_x(hi);
+            // The h ring reuses the B tile's space: wait until G is computed
+            // (and G_10 copied out of TMEM into its place).
+            bool ok = mbar_wait(&bars[BAR_GCONV], 0, status);
+            if (ok) {
+                for (int hi = 0; hi < first; ++hi) load_h(hi);
+                for (int hi = 2; hi < HG && ok; ++hi) {
+                    const int s = hi & 1;
+                    ok = mbar_wait(&bars[BAR_XEMPTY + s], (uint32_t)(((hi >> 1) - 1) & 1), status);
+                    if (ok) { load_x(hi); load_h(hi); }
+                }
+            }
+            if (!ok) s_flag[0] = 1;
         }
-    }
-    __syncthreads();
-
-    // ---- 1. G = C_tile B^T over K = dstate, into TMEM columns [0, KJ).
-    if (!mbar_wait(&bars[0], 0, status)) *s_abort = 1;
-    __syncthreads();
-    bool aborted = *s_abort != 0;
-    if (!aborted) {
-        if (tid == 0) {
-            bc_pending = false;
+    } else if (warp == 13) {
+        // ================================================== MMA issuer
+        if (lane == 0) {
+            bool ok = mbar_wait(&bars[BAR_BC], 0, status);
+            if (ok) {
+                tc_fence_after();
+                const uint32_t idesc_g = idesc_bf16_f32(128, KJ, false, false);
+                const uint32_t c0 = smem_u32(sC), b0 = smem_u32(sB);
+                const uint32_t dcol = (t == 1) ? kColM : kColG;   // t=1: [G_10 | G_11] over 256 columns
+                for (int ks = 0; ks < N / 16; ++ks) {
+                    const int nb = ks >> 2, ko = (ks & 3) * 32;
+                    mma_ss(tmem + dcol, smem_desc_sw128(c0 + nb * 128 * 128 + ko, 16, 1024),
+                           smem_desc_sw128(b0 + nb * Q * 128 + ko, 16, 1024), idesc_g, ks > 0);
+                }
+                mma_commit(&bars[BAR_G]);
+            }
+            const uint32_t idesc_y = idesc_bf16_f32(128, 64, false, true);
+            const uint32_t idesc_z = idesc_bf16_f32(128, 64, false, false);
+            for (int hi = 0; hi < HG && ok; ++hi) {
+                const int s = hi & 1;
+                ok = mbar_wait(&bars[BAR_MFULL], (uint32_t)(hi & 1), status) &&
+                     mbar_wait(&bars[BAR_XFULL + s], (uint32_t)((hi >> 1) & 1), status) &&
+                     (hi < 2 || mbar_wait(&bars[BAR_ACCEMPTY + s], (uint32_t)(((hi >> 1) - 1) & 1),
+                                          status));
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t acc = tmem + kColAcc + 128 * s;
+                const uint32_t x0 = smem_u32(sX + s * S::kXTile);
+                for (int ks = 0; ks < KJ / 16; ++ks)
+                    mma_ts(acc, tmem + kColM + ks * 8, smem_desc_sw128(x0 + ks * 2048, 16, 1024),
+                           idesc_y, ks > 0);
+                const uint32_t c0 = smem_u32(sC), h0 = smem_u32(sH + s * S::kHTile);
+                for (int ks = 0; ks < N / 16; ++ks) {
+                    const int nb = ks >> 2, ko = (ks & 3) * 32;
+                    mma_ss(acc + 64, smem_desc_sw128(c0 + nb * 128 * 128 + ko, 16, 1024),
+                           smem_desc_sw128(h0 + nb * 64 * 128 + ko, 16, 1024), idesc_z, ks > 0);
+                }
+                mma_commit(&bars[BAR_MEMPTY]);
+                mma_commit(&bars[BAR_ACCFULL + s]);
+            }
+            if (!ok) s_flag[0] = 1;
+        }
+    } else if (warp < 8) {
+        // ================================================== mask warps (0-7)
+        // Warp w builds rows of TMEM lane quarter q = w % 4 (rows 32q..32q+31)
+        // over half hf = w / 4 of the tile's 32-column blocks.
+        const int q = warp & 3, hf = warp >> 2;
+        const int m = q * 32 + lane;               // row within the tile
+        const int i = row0 + m;                    // row within the chunk
+        const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+        for (int e = tid; e < HG * KJ; e += 256) {
+            const int j = e / HG, k = e - j * HG;
+            s_dt[k * Q + j] = (j < len) ? dt[(b * L + t0 + j) * H + head0 + k] : 0.f;
+        }
+        if (tid < HG) {
+            s_Ah[tid] = A[head0 + tid] * kLog2e;
+            s_Dh[tid] = Dv[head0 + tid];
+        }
+        bool fail = !mbar_wait(&bars[BAR_G], 0, status);
+        if (!named_bar_or(1, 256, fail)) {
             tc_fence_after();
-            const uint32_t idesc = idesc_bf16_f32(128, KJ, false, false);
-            const uint32_t c0 = smem_u32(sC), b0 = smem_u32(sB);
+            if (t == 1) {
+                // G_10 (TMEM columns [0, 128)) -> bf16 row m of sG10, 16-byte chunks
+                // placed at (chunk ^ (m & 15)) so that a warp's row reads spread over banks.
+                uint4* grow = reinterpret_cast<uint4*>(sG10 + m * 256);
+                for (int cb = 2 * hf; cb < 2 * hf + 2; ++cb) {
+                    uint32_t r[32];
+                    tmem_ld32(tmem + lane_base + kColM + cb * 32, r);
 #pragma unroll
-            for (int ks = 0; ks < N / 16; ++ks) {
-                const int nb = ks >> 2, ko = (ks & 3) * 32;
-                const uint64_t ad = smem_desc_sw128(c0 + nb * 128 * 128 + ko, 16, 1024);
-                const uint64_t bd = smem_desc_sw128(b0 + nb * Q * 128 + ko, 16, 1024);
-                mma_ss(tmem + kColG, ad, bd, idesc, ks > 0);
-            }
-            mma_commit(&bars[3]);
-            g_pending = 0;
-        }
-        if (!mbar_wait(&bars[3], 0, status)) *s_abort = 1;
-        tc_fence_after();
-        __syncthreads();
-        aborted = *s_abort != 0;
-        if (tid == 0 && !aborted) g_pending = -1;
-    }
-
-    const int m = tid;                 // this thread's row within the tile
-    const int i = row0 + m;            // ... within the chunk
-    const bool row_valid = i < len;
-
-    for (int hi = 0; hi < HG && !aborted; ++hi) {
-        const int buf = hi & 1;
-        const uint32_t use_parity = (uint32_t)((hi >> 1) & 1);
-        const int h = head0 + hi;
-
-        const float* hcs = s_cs + hi * Q;      // this head's prefix sums
-        const float* hdt = s_dt + hi * Q;
-        const float cs_i = hcs[i];
-        float alpha = 0.f;
-        if (t > 0) {
-            // factorised decay for the block left of the diagonal, through r = cs_{row0 - 1}
-            const float r = hcs[row0 - 1];
-            s_beta[m] = exp2f(r - hcs[m]) * hdt[m];
-            alpha = exp2f(cs_i - r);
-        }
-        if (!mbar_wait(&bars[1 + buf], use_parity, status)) *s_abort = 1;
-        __syncthreads();
-        if (*s_abort) { aborted = true; break; }
-        if (tid == 0) xh_pending[buf] = -1;
-
-        // ---- 2. decay mask -> TMEM (bf16 pairs), 32 columns at a time
-        for (int cb = 0; cb < KJ / 32; ++cb) {
-            const int j0 = cb * 32;
-            uint32_t packed[16];
-            if (j0 >= row0) {
-                // diagonal block: exact exponentials, causal mask
-                const int rel = (j0 - row0) >> 5;       // column block within the diagonal block
-                if (rel > warp) {
-#pragma unroll
-                    for (int q = 0; q < 16; ++q) packed[q] = 0u;
-                } else {
-                    uint32_t gr[32];
-                    tmem_ld32(tmem + lane_base + kColG + j0, gr);
-#pragma unroll
-                    for (int q = 0; q < 16; ++q) {
-                        const int ja = j0 + 2 * q, jb = ja + 1;
-                        const float va = (ja <= i) ? __uint_as_float(gr[2 * q]) *
-                                                         exp2f(cs_i - hcs[ja]) * hdt[ja]
-                                                   : 0.f;
-                        const float vb = (jb <= i) ? __uint_as_float(gr[2 * q + 1]) *
-                                                         exp2f(cs_i - hcs[jb]) * hdt[jb]
-                                                   : 0.f;
-                        packed[q] = pack_bf16x2(va, vb);
+                    for (int u = 0; u < 4; ++u) {
+                        const int lc = cb * 4 + u;
+                        grow[lc ^ (m & 15)] = make_uint4(
+                            pack_bf16x2(__uint_as_float(r[8 * u + 0]), __uint_as_float(r[8 * u + 1])),
+                            pack_bf16x2(__uint_as_float(r[8 * u + 2]), __uint_as_float(r[8 * u + 3])),
+                            pack_bf16x2(__uint_as_float(r[8 * u + 4]), __uint_as_float(r[8 * u + 5])),
+                            pack_bf16x2(__uint_as_float(r[8 * u + 6]), __uint_as_float(r[8 * u + 7])));
                     }
                 }
-            } else {
-                // block left of the diagonal: G_ij * alpha_i * beta_j
-                uint32_t gr[32];
-                tmem_ld32(tmem + lane_base + kColG + j0, gr);
+            }
+            tc_fence_before();
+            named_bar_sync(1, 256);
+            if (tid == 0) mbar_arrive(&bars[BAR_GCONV]);
+
+            const int nblk = KJ / 32;
+            for (int hi = 0; hi < HG; ++hi) {
+                const int s = hi & 1;
+                // slot s (exp(cs) row scales) is free once the epilogue of head
+                // hi - 2 is done
+                fail = hi >= 2 && !mbar_wait(&bars[BAR_ACCEMPTY + s], (uint32_t)(((hi >> 1) - 1) & 1),
+                                             status);
+                if (named_bar_or(1, 256, fail)) break;
+                float* cs = s_cs + s * Q;
+                const float* hdt = s_dt + hi * Q;
+                if (warp == 0) {
+                    const float Ah = s_Ah[hi];
+                    float carry = 0.f;
+                    for (int base = 0; base < KJ; base += 32) {
+                        float v = hdt[base + lane] * Ah;
 #pragma unroll
-                for (int q = 0; q < 16; ++q) {
-                    const int ja = j0 + 2 * q;
-                    const float va = __uint_as_float(gr[2 * q]) * alpha * s_beta[ja];
-                    const float vb = __uint_as_float(gr[2 * q + 1]) * alpha * s_beta[ja + 1];
-                    packed[q] = pack_bf16x2(va, vb);
+                        for (int o = 1; o < 32; o <<= 1) {
+                            const float u = __shfl_up_sync(0xffffffffu, v, o);
+                            if (lane >= o) v += u;
+                        }
+                        v += carry;
+                        cs[base + lane] = v;
+                        carry = __shfl_sync(0xffffffffu, v, 31);
+                    }
                 }
-            }
-            tmem_st16(tmem + lane_base + kColM + (uint32_t)(j0 >> 1), packed);
-        }
-        tc_fence_before();
-        __syncthreads();
+                named_bar_sync(1, 256);
+                const float cs_i = cs[i];
+                // Column factors.  The decay between row i and column j < i
+                // factorises through any boundary r with cs_j >= r >= cs_i:
+                // exp(cs_i - cs_j) = exp(cs_i - r) exp(r - cs_j), both <= 1.
+                //   s_beta[j]  block left of the diagonal (t = 1), r = cs_{127}
+                //   s_beta2[k] diagonal block, r = end of the 32-column block of j = row0 + k
+                if (hf == 0) {
+                    if (t == 1) s_beta[m] = exp2f(cs[127] - cs[m]) * hdt[m];
+                    s_ez[s * 128 + m] = exp2f(cs_i);
+                } else {
+                    const int j = row0 + m;
+                    s_beta2[m] = exp2f(cs[row0 + (m | 31)] - cs[j]) * hdt[j];
+                }
+                // M is free once the MMAs of the previous head completed
+                fail = hi >= 1 && !mbar_wait(&bars[BAR_MEMPTY], (uint32_t)((hi - 1) & 1), status);
+                if (named_bar_or(1, 256, fail)) break;      // also publishes the factors and s_ez
+                if (tid == 0) mbar_arrive(&bars[BAR_EZFULL + s]);
+                tc_fence_after();
 
-        // ---- 3. Y = M X (A from TMEM), Z = C_tile h_prev^T
-        if (tid == 0) {
-            tc_fence_after();
-            const uint32_t idesc_y = idesc_bf16_f32(128, 64, false, true);
-            const uint32_t x0 = smem_u32(sX + buf * S::kXTile);
-            for (int ks = 0; ks < KJ / 16; ++ks) {
-                const uint64_t bd = smem_desc_sw128(x0 + ks * 2048, 16, 1024);
-                mma_ts(tmem + kColY, tmem + kColM + ks * 8, bd, idesc_y, ks > 0);
-            }
-            const uint32_t idesc_z = idesc_bf16_f32(128, 64, false, false);
-            const uint32_t c0 = smem_u32(sC), h0 = smem_u32(sH + buf * S::kHTile);
+                const float alpha_off = (t == 1) ? exp2f(cs_i - cs[127]) : 0.f;
+                for (int cb = hf * (nblk / 2); cb < (hf + 1) * (nblk / 2); ++cb) {
+                    const int j0 = 32 * cb;
+                    uint32_t packed[16];
+                    if (j0 < row0) {
+                        // block left of the diagonal: G_10 (bf16, shared) * alpha * beta_j
+                        const uint4* grow = reinterpret_cast<const uint4*>(sG10 + m * 256);
 #pragma unroll
-            for (int ks = 0; ks < N / 16; ++ks) {
-                const int nb = ks >> 2, ko = (ks & 3) * 32;
-                const uint64_t ad = smem_desc_sw128(c0 + nb * 128 * 128 + ko, 16, 1024);
-                const uint64_t bd = smem_desc_sw128(h0 + nb * 64 * 128 + ko, 16, 1024);
-                mma_ss(tmem + kColZ, ad, bd, idesc_z, ks > 0);
+                        for (int u = 0; u < 4; ++u) {
+                            const int lc = cb * 4 + u;
+                            const uint4 gv = grow[lc ^ (m & 15)];
+                            const uint32_t* gu = reinterpret_cast<const uint32_t*>(&gv);
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const float2 gf =
+                                    __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&gu[e]));
+                                const int ja = 8 * lc + 2 * e;
+                                packed[4 * u + e] = pack_bf16x2(gf.x * alpha_off * s_beta[ja],
+                                                                gf.y * alpha_off * s_beta[ja + 1]);
+                            }
+                        }
+                    } else {
+                        const int rel = (j0 - row0) >> 5;   // 32-column block within the diagonal block
+                        if (rel > q) {
+#pragma unroll
+                            for (int u = 0; u < 16; ++u) packed[u] = 0u;
+                        } else {
+                            uint32_t gr[32];
+                            tmem_ld32(tmem + lane_base + kColG + 32 * rel, gr);
+                            if (rel < q) {
+                                // entirely below the diagonal: factorised decay
+                                const float alpha = exp2f(cs_i - cs[j0 + 31]);
+                                const float* bet = s_beta2 + 32 * rel;
+#pragma unroll
+                                for (int u = 0; u < 16; ++u)
+                                    packed[u] = pack_bf16x2(__uint_as_float(gr[2 * u]) * alpha * bet[2 * u],
+                                                            __uint_as_float(gr[2 * u + 1]) * alpha * bet[2 * u + 1]);
+                            } else {
+                                // 32 x 32 block on the diagonal: exact exponentials, causal mask
+#pragma unroll
+                                for (int u = 0; u < 16; ++u) {
+                                    const int ja = j0 + 2 * u, jb = ja + 1;
+                                    const float va = (ja <= i)
+                                        ? __uint_as_float(gr[2 * u]) * exp2f(cs_i - cs[ja]) * hdt[ja] : 0.f;
+                                    const float vb = (jb <= i)
+                                        ? __uint_as_float(gr[2 * u + 1]) * exp2f(cs_i - cs[jb]) * hdt[jb] : 0.f;
+                                    packed[u] = pack_bf16x2(va, vb);
+                                }
+                            }
+                        }
+                    }
+                    tmem_st16(tmem + lane_base + kColM + (uint32_t)(j0 >> 1), packed);
+                }
+                tc_fence_before();
+                named_bar_sync(1, 256);
+                if (tid == 0) mbar_arrive(&bars[BAR_MFULL]);
             }
-            mma_commit(&bars[4]);
-            yz_pending = (int)(hi & 1);
         }
-        if (!mbar_wait(&bars[4], (uint32_t)(hi & 1), status)) *s_abort = 1;
-        tc_fence_after();
-        __syncthreads();
-        if (*s_abort) { aborted = true; break; }
-        if (tid == 0) yz_pending = -1;
-
-        // ---- 4. epilogue: y = Y + exp(cs_i) Z + D_h x, one row per thread
-        {
-            const float ez = exp2f(cs_i);
-            const float Dh = Dv[h];
-            const uint8_t* xrow = sX + buf * S::kXTile + i * 128;
-            __nv_bfloat16* yrow = y + ((b * L + t0 + i) * H + h) * 64;
+        if (fail) s_flag[0] = 1;
+    } else {
+        // ================================================== epilogue warpgroup (warps 8-11)
+        // y rows go to a 128-byte-swizzled staging tile and leave by TMA store
+        // (coalesced; rows past the sequence end are clipped by the tensor map).
+        const int m = tid - 256;
+        const int i = row0 + m;
+        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+        bool fail = false;
+        for (int hi = 0; hi < HG; ++hi) {
+            const int s = hi & 1;
+            const int h = head0 + hi;
+            // x_full too: the epilogue reads the TMA-written x rows (D x term); the
+            // slot cannot be reloaded before this epilogue releases it.
+            fail = !(mbar_wait(&bars[BAR_ACCFULL + s], (uint32_t)((hi >> 1) & 1), status) &&
+                     mbar_wait(&bars[BAR_EZFULL + s], (uint32_t)((hi >> 1) & 1), status) &&
+                     mbar_wait(&bars[BAR_XFULL + s], (uint32_t)((hi >> 1) & 1), status));
+            // staging slot s is free once the store issued two heads ago has read it
+            if (m == 0) bulk_wait_group_read<1>();
+            if (named_bar_or(2, 128, fail)) break;
+            tc_fence_after();
+            const float ez = s_ez[s * 128 + m];
+            const float Dh = s_Dh[hi];
+            const uint8_t* xrow = sX + s * S::kXTile + i * 128;
+            uint4* ystage = reinterpret_cast<uint4*>(sY + s * 16384 + m * 128);
+            const uint32_t acc = tmem + lane_base + kColAcc + 128 * s;
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 uint32_t yr[32], zr[32];
-                tmem_ld32(tmem + lane_base + kColY + half * 32, yr);
-                tmem_ld32(tmem + lane_base + kColZ + half * 32, zr);
-                uint32_t out[16];
+                tmem_ld32x2(acc + half * 32, acc + 64 + half * 32, yr, zr);
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
-                    // logical 16-byte chunk (half*4 + q) of the swizzled x row
-                    const int lc = half * 4 + q;
+                    const int lc = half * 4 + q;   // logical 16-byte chunk of the row
                     const uint4 xv = *reinterpret_cast<const uint4*>(xrow + ((lc ^ (i & 7)) << 4));
                     const uint32_t* xu = reinterpret_cast<const uint32_t*>(&xv);
+                    uint32_t o[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const float2 xf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xu[e]));
+                        const float2 xf =
+                            __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xu[e]));
                         const int k = 8 * q + 2 * e;
                         const float v0 = __uint_as_float(yr[k]) + ez * __uint_as_float(zr[k]) + Dh * xf.x;
-                        const float v1 = __uint_as_float(yr[k + 1]) + ez * __uint_as_float(zr[k + 1]) + Dh * xf.y;
-                        out[4 * q + e] = pack_bf16x2(v0, v1);
+                        const float v1 =
+                            __uint_as_float(yr[k + 1]) + ez * __uint_as_float(zr[k + 1]) + Dh * xf.y;
+                        o[e] = pack_bf16x2(v0, v1);
                     }
-                }
-                if (row_valid) {
-                    uint4* dst = reinterpret_cast<uint4*>(yrow + half * 32);
-#pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        dst[q] = make_uint4(out[4 * q], out[4 * q + 1], out[4 * q + 2], out[4 * q + 3]);
+                    ystage[lc ^ (m & 7)] = make_uint4(o[0], o[1], o[2], o[3]);
                 }
             }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            named_bar_sync(2, 128);
+            if (m == 0) {
+                tma_store_4d(&tmY, sY + s * 16384, 0, h, (int)(t0 + row0), (int)b);
+                bulk_commit_group();
+                mbar_arrive(&bars[BAR_ACCEMPTY + s]);
+                mbar_arrive(&bars[BAR_XEMPTY + s]);
+            }
         }
-        tc_fence_before();
-        __syncthreads();
-        if (tid == 0 && hi + 2 < HG) issue_xh(hi + 2);
+        if (m == 0) bulk_wait_group<0>();      // stores done before the CTA leaves
+        if (fail) s_flag[0] = 1;
     }
 
-    if (aborted && tid == 0) {
-        if (bc_pending) mbar_wait(&bars[0], 0, status);
-        for (int k = 0; k < 2; ++k)
-            if (xh_pending[k] >= 0) mbar_wait(&bars[1 + k], (uint32_t)xh_pending[k], status);
-        if (g_pending >= 0) mbar_wait(&bars[3], (uint32_t)g_pending, status);
-        if (yz_pending >= 0) mbar_wait(&bars[4], (uint32_t)yz_pending, status);
-    }
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) {
+    if (s_flag[0] && tid == 12 * 32) {
+        // A wait gave up somewhere: before the CTA's shared memory and TMEM
+        // go away, give outstanding TMA loads and MMAs a last (bounded) chance
+        // to land.  Waiting on already-completed phases returns at once.
+        for (int k = 0; k < 2; ++k) {
+            mbar_wait(&bars[BAR_XFULL + k], 0, status);
+            mbar_wait(&bars[BAR_ACCFULL + k], 0, status);
+        }
+        mbar_wait(&bars[BAR_BC], 0, status);
+        mbar_wait(&bars[BAR_G], 0, status);
+    }
+    __syncthreads();
+    if (warp == 13) {
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
@@ -362,7 +463,7 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
 
 int pick_heads_per_cta(int64_t H, int64_t G) {
     const int64_t hpg = H / G;
-    for (int hg = 8; hg > 1; --hg)
+    for (int hg = kMaxHeads; hg > 1; --hg)
         if (hpg % hg == 0) return hg;
     return 1;
 }
@@ -385,6 +486,9 @@ cudaError_t launch_impl(const void* x, const float* dt, const float* A, const vo
     if (e != cudaSuccess) return e;
     e = make_tmap_bf16(&tmC, C, 4, bdims, bstr, box128);
     if (e != cudaSuccess) return e;
+    CUtensorMap tmY;
+    e = make_tmap_bf16(&tmY, y, 4, xdims, xstr, box128);
+    if (e != cudaSuccess) return e;
     const uint64_t hdims[2] = {(uint64_t)N, (uint64_t)(d.b * d.T * d.H * 64)};
     const uint64_t hstr[1] = {(uint64_t)N * 2};
     const uint32_t hbox[2] = {64, 64};
@@ -399,8 +503,7 @@ cudaError_t launch_impl(const void* x, const float* dt, const float* A, const vo
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)(d.b * d.T * (Q / 128)), (unsigned)(d.H / HG));
     chunk_out_tc_kernel<Q, N><<<grid, kThreads, S::kAlloc, s>>>(
-        tmX, tmB, tmC, tmH, dt, A, D, static_cast<__nv_bfloat16*>(y), d.L, (int)d.H, (int)d.G,
-        d.T, HG, status);
+        tmX, tmB, tmC, tmH, tmY, dt, A, D, d.L, (int)d.H, (int)d.G, d.T, HG, status);
     return cudaGetLastError();
 }
 
