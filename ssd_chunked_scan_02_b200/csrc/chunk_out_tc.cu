@@ -11,28 +11,34 @@
 // decomposition lets the tensor cores do the work).
 //
 // One CTA per (batch, chunk, 128-row tile t of the chunk, group of HG heads
-// sharing B and C).  Rows i of tile t need columns j < 128 (t + 1).
+// sharing B and C).  Tile t holds rows i in [128 t, 128 t + 128).
 //
-//   prologue: G = C_t B^T (M = 128, N = 128 (t+1), K = dstate) into TMEM,
-//             once for all the CTA's heads (B, C are per group).  For t = 1
-//             the block left of the diagonal (G_10) is copied to shared
-//             memory as bf16 and only the diagonal block stays in TMEM.
-//   per head (pipelined over heads by warp role):
-//     mask warps       build M (bf16) in TMEM, M_ij = G_ij exp(cs_i - cs_j) dt_j
-//                      for j <= i.  Wherever a whole 32-column block lies below
-//                      the diagonal the decay factorises through the block's
-//                      end r: exp(cs_i - r) * (exp(r - cs_j) dt_j), both factors
-//                      <= 1, so only the 32 x 32 blocks on the diagonal need an
-//                      exponential per element.
-//     MMA lane         Y = M X (A from TMEM, kind::f16) and Z = C_t h_prev^T
-//                      into a double-buffered accumulator slot.
-//     epilogue group   y = Y + exp(cs_i) Z + D_h x, rounded to bf16 once, staged
-//                      in shared memory and written by TMA store.
-//     producer lane    TMA of the next heads' x rows and entering states.
+// The decay between row i and column j < i factorises through any boundary r
+// with cs_j >= r >= cs_i: exp(cs_i - cs_j) = exp(cs_i - r) exp(r - cs_j), both
+// factors <= 1.  With r = cs_{127} for the block left of the diagonal (t = 1):
+//   sum_{j < 128} G_ij exp(cs_i - cs_j) dt_j x_j
+//      = alpha_i sum_j G_ij (beta_j x_j),   alpha_i = exp(cs_i - r), beta_j = exp(r - cs_j) dt_j
+// and the entering state term exp(cs_i) C_i h = alpha_i C_i (exp(r) h).  Both go
+// into one accumulator ZW = G_10 (beta x_{0..127}) + C_t (exp(r) h)^T, scaled
+// by alpha_i in the epilogue (for t = 0, r = 0: ZW = C_0 h^T, alpha_i = exp(cs_i)).
+// Only the diagonal 128 x 128 block needs a per-element mask:
+//   Y = M X_t,  M_ij = G_ij exp(cs_i - cs_j) dt_j (j <= i),
+// and within it each 32-column block below the diagonal factorises the same
+// way through the block's end, so only the 32 x 32 blocks on the diagonal
+// evaluate an exponential per element.  Output: y = Y + alpha_i ZW + D_h x.
 //
-// Warps 0-7: mask (two per TMEM lane quarter, splitting the columns); 8-11:
-// epilogue; 12: TMA producer; 13: MMA issuer (and TMEM owner).  Every wait is bounded; a warpgroup leaves its loop only when all
-// its threads agree (bar.red.or), so no named barrier is left half-arrived.
+// Roles (448 threads):
+//   warps 0-7   prologue: G = C_t B^T (M = 128, N = 128 (t+1), K = dstate) is
+//               copied from TMEM: the diagonal block stays in TMEM (fp32), the
+//               block to its left goes to shared memory as bf16 (the A operand
+//               of G_10 X~); per head: prefix sums, factors, scaling of
+//               x rows 0..127 by beta and of h by exp(r) in place, and the
+//               diagonal-block mask written to TMEM as bf16 (two slots);
+//   warps 8-11  epilogue: y staged in shared memory, TMA store;
+//   warp 12     TMA producer (x rows and entering states of the heads, ring of 2);
+//   warp 13     MMA issuer and TMEM owner.
+// Every wait is bounded; a warpgroup leaves its loop only when all its
+// threads agree (bar.red.or), so no named barrier is left half-arrived.
 #include <cuda.h>
 #include <cuda_bf16.h>
 
@@ -57,22 +63,22 @@ struct OutSmem {
     static constexpr int kC = 0;                            // C tile: kNB x 128 rows x 128 B
     static constexpr int kCBytes = kNB * 128 * 128;
     static constexpr int kBG = kC + kCBytes;                // B tile (prologue), then G_10 + h ring
-    static constexpr int kG10Off = 0;                       // bf16 128 x 128 (t = 1 only)
+    static constexpr int kG10Off = 0;                       // bf16 G_10, K-major SW128, 2 x 16 KB (t = 1)
     static constexpr int kHOff = (Q == 256) ? 32768 : 0;    // h ring: 2 slots
     static constexpr int kBBytes = kNB * Q * 128;
     static constexpr int kBGBytes = (kBBytes > kHOff + 2 * kHTile) ? kBBytes : kHOff + 2 * kHTile;
     static constexpr int kXTile = Q * 128;                  // x rows [0, Q) of one head
     static constexpr int kX = kBG + kBGBytes;               // x ring: 2 slots
-    static constexpr int kDt = kX + 2 * kXTile;             // float [kMaxHeads][Q]
+    static constexpr int kYs = kX + 2 * kXTile;             // y staging: 2 x 16 KB
+    static constexpr int kDt = kYs + 2 * 128 * 128;         // float [kMaxHeads][Q]
     static constexpr int kCs = kDt + kMaxHeads * Q * 4;     // float [2][Q] prefix sums (log2 units)
-    static constexpr int kBeta = kCs + 2 * Q * 4;           // float [128]
-    static constexpr int kBeta2 = kBeta + 128 * 4;          // float [128]
-    static constexpr int kEz = kBeta2 + 128 * 4;            // float [2][128] exp(cs_i) per slot
-    static constexpr int kAD = kEz + 2 * 128 * 4;           // float [2][kMaxHeads]: A_h, D_h
-    static constexpr int kYs = ((kAD + 2 * kMaxHeads * 4 + 1023) / 1024) * 1024;  // y staging: 2 x 16 KB
-    static constexpr int kBar = kYs + 2 * 128 * 128;        // 16 mbarriers
-    static constexpr int kTmem = kBar + 16 * 8;
-    static constexpr int kFlags = kTmem + 16;               // abort flags
+    static constexpr int kBeta = kCs + 2 * Q * 4;           // float [128]  (t = 1 block left of diagonal)
+    static constexpr int kBeta2 = kBeta + 128 * 4;          // float [128]  (diagonal block)
+    static constexpr int kAl = kBeta2 + 128 * 4;            // float [2][128] alpha_i per slot
+    static constexpr int kAD = kAl + 2 * 128 * 4;           // float [2][kMaxHeads]: A_h (log2), D_h
+    static constexpr int kBar = kAD + 2 * kMaxHeads * 4;    // mbarriers
+    static constexpr int kTmem = kBar + 24 * 8;
+    static constexpr int kFlags = kTmem + 16;
     static constexpr int kTotal = kFlags + 16;
     static constexpr int kAlloc = kTotal + 1024;
 };
@@ -80,17 +86,35 @@ struct OutSmem {
 // mbarrier indices
 enum {
     BAR_BC = 0, BAR_G = 1, BAR_GCONV = 2, BAR_XFULL = 3, BAR_XEMPTY = 5, BAR_MFULL = 7,
-    BAR_MEMPTY = 8, BAR_ACCFULL = 9, BAR_ACCEMPTY = 11, BAR_EZFULL = 13, BAR_COUNT = 15
+    BAR_MEMPTY = 9, BAR_ACCFULL = 11, BAR_ACCEMPTY = 13, BAR_ALFULL = 15, BAR_COUNT = 17
 };
 
 // TMEM columns
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColM = 0;       // bf16 mask (A operand), up to 128 columns; G_10 in the prologue
+constexpr uint32_t kColM = 0;       // bf16 diagonal-block mask, 2 slots of 64 columns (G_10 in the prologue)
 constexpr uint32_t kColG = 128;     // fp32 diagonal block of G, 128 columns
-constexpr uint32_t kColAcc = 256;   // two slots of 128: Y (64) then Z (64)
+constexpr uint32_t kColAcc = 256;   // two slots of 128: Y (64) then ZW (64)
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
     return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+// Scale `n16` 16-byte pieces (8 bf16 each) of a shared-memory tile in place by a
+// per-piece factor f(piece): done by `nthr` threads, thread index `t`.
+template <typename F>
+__device__ __forceinline__ void scale_pieces(uint8_t* base, int n16, int t, int nthr, F f) {
+    for (int k = t; k < n16; k += nthr) {
+        uint4* ptr = reinterpret_cast<uint4*>(base) + k;
+        uint4 v = *ptr;
+        const float s = f(k);
+        uint32_t* u = reinterpret_cast<uint32_t*>(&v);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float2 x = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&u[e]));
+            u[e] = pack_bf16x2(x.x * s, x.y * s);
+        }
+        *ptr = v;
+    }
 }
 
 template <int Q, int N>
@@ -122,14 +146,14 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
     uint8_t* sG10 = smem + S::kBG + S::kG10Off;
     uint8_t* sH = smem + S::kBG + S::kHOff;
     uint8_t* sX = smem + S::kX;
+    uint8_t* sY = smem + S::kYs;
     float* s_dt = reinterpret_cast<float*>(smem + S::kDt);
     float* s_cs = reinterpret_cast<float*>(smem + S::kCs);
     float* s_beta = reinterpret_cast<float*>(smem + S::kBeta);
     float* s_beta2 = reinterpret_cast<float*>(smem + S::kBeta2);
-    float* s_ez = reinterpret_cast<float*>(smem + S::kEz);
+    float* s_al = reinterpret_cast<float*>(smem + S::kAl);
     float* s_Ah = reinterpret_cast<float*>(smem + S::kAD);
     float* s_Dh = s_Ah + kMaxHeads;
-    uint8_t* sY = smem + S::kYs;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::kBar);
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + S::kTmem);
     volatile int* s_flag = reinterpret_cast<volatile int*>(smem + S::kFlags);   // [0]: any abort
@@ -155,6 +179,7 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
             prefetch_tmap(&tmB);
             prefetch_tmap(&tmC);
             prefetch_tmap(&tmH);
+            prefetch_tmap(&tmY);
             mbar_expect_tx(&bars[BAR_BC], (uint32_t)(S::kCBytes + S::kNB * KJ * 128));
             for (int nb = 0; nb < S::kNB; ++nb) {
                 tma_load_4d(sC + nb * 128 * 128, &tmC, &bars[BAR_BC], nb * 64, g,
@@ -179,8 +204,8 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
             };
             const int first = HG < 2 ? HG : 2;
             for (int hi = 0; hi < first; ++hi) load_x(hi);
-            // The h ring reuses the B tile's space: wait until G is computed
-            // (and G_10 copied out of TMEM into its place).
+            // The h ring (and G_10) reuse the B tile's space: wait until G is
+            // computed and copied out of TMEM.
             bool ok = mbar_wait(&bars[BAR_GCONV], 0, status);
             if (ok) {
                 for (int hi = 0; hi < first; ++hi) load_h(hi);
@@ -200,7 +225,7 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
                 tc_fence_after();
                 const uint32_t idesc_g = idesc_bf16_f32(128, KJ, false, false);
                 const uint32_t c0 = smem_u32(sC), b0 = smem_u32(sB);
-                const uint32_t dcol = (t == 1) ? kColM : kColG;   // t=1: [G_10 | G_11] over 256 columns
+                const uint32_t dcol = (t == 1) ? 0u : kColG;   // t=1: [G_10 | G_11] over 256 columns
                 for (int ks = 0; ks < N / 16; ++ks) {
                     const int nb = ks >> 2, ko = (ks & 3) * 32;
                     mma_ss(tmem + dcol, smem_desc_sw128(c0 + nb * 128 * 128 + ko, 16, 1024),
@@ -208,11 +233,12 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
                 }
                 mma_commit(&bars[BAR_G]);
             }
-            const uint32_t idesc_y = idesc_bf16_f32(128, 64, false, true);
-            const uint32_t idesc_z = idesc_bf16_f32(128, 64, false, false);
+            const uint32_t idesc_y = idesc_bf16_f32(128, 64, false, true);    // A in TMEM, x MN-major
+            const uint32_t idesc_w = idesc_bf16_f32(128, 64, false, true);    // G_10 K-major, x~ MN-major
+            const uint32_t idesc_z = idesc_bf16_f32(128, 64, false, false);   // C, h both K-major
             for (int hi = 0; hi < HG && ok; ++hi) {
                 const int s = hi & 1;
-                ok = mbar_wait(&bars[BAR_MFULL], (uint32_t)(hi & 1), status) &&
+                ok = mbar_wait(&bars[BAR_MFULL + s], (uint32_t)((hi >> 1) & 1), status) &&
                      mbar_wait(&bars[BAR_XFULL + s], (uint32_t)((hi >> 1) & 1), status) &&
                      (hi < 2 || mbar_wait(&bars[BAR_ACCEMPTY + s], (uint32_t)(((hi >> 1) - 1) & 1),
                                           status));
@@ -220,24 +246,35 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
                 tc_fence_after();
                 const uint32_t acc = tmem + kColAcc + 128 * s;
                 const uint32_t x0 = smem_u32(sX + s * S::kXTile);
-                for (int ks = 0; ks < KJ / 16; ++ks)
-                    mma_ts(acc, tmem + kColM + ks * 8, smem_desc_sw128(x0 + ks * 2048, 16, 1024),
-                           idesc_y, ks > 0);
+                // Y = M X_t over the diagonal block's 128 columns
+                for (int ks = 0; ks < 8; ++ks)
+                    mma_ts(acc, tmem + kColM + 64 * s + ks * 8,
+                           smem_desc_sw128(x0 + (row0 / 16 + ks) * 2048, 16, 1024), idesc_y, ks > 0);
+                // ZW = G_10 (beta x_{0..127}) [t = 1] + C_t (exp(r) h)^T
+                if (t == 1) {
+                    const uint32_t g0 = smem_u32(sG10);
+                    for (int ks = 0; ks < 8; ++ks) {
+                        const int kb = ks >> 2, ko = (ks & 3) * 32;
+                        mma_ss(acc + 64, smem_desc_sw128(g0 + kb * 16384 + ko, 16, 1024),
+                               smem_desc_sw128(x0 + ks * 2048, 16, 1024), idesc_w, ks > 0);
+                    }
+                }
                 const uint32_t c0 = smem_u32(sC), h0 = smem_u32(sH + s * S::kHTile);
                 for (int ks = 0; ks < N / 16; ++ks) {
                     const int nb = ks >> 2, ko = (ks & 3) * 32;
                     mma_ss(acc + 64, smem_desc_sw128(c0 + nb * 128 * 128 + ko, 16, 1024),
-                           smem_desc_sw128(h0 + nb * 64 * 128 + ko, 16, 1024), idesc_z, ks > 0);
+                           smem_desc_sw128(h0 + nb * 64 * 128 + ko, 16, 1024), idesc_z,
+                           t == 1 || ks > 0);
                 }
-                mma_commit(&bars[BAR_MEMPTY]);
+                mma_commit(&bars[BAR_MEMPTY + s]);
                 mma_commit(&bars[BAR_ACCFULL + s]);
             }
             if (!ok) s_flag[0] = 1;
         }
     } else if (warp < 8) {
-        // ================================================== mask warps (0-7)
-        // Warp w builds rows of TMEM lane quarter q = w % 4 (rows 32q..32q+31)
-        // over half hf = w / 4 of the tile's 32-column blocks.
+        // ================================================== mask / scale warps (0-7)
+        // Warp w owns TMEM lane quarter q = w % 4 (rows 32q..32q+31) and half
+        // hf = w / 4 of the diagonal block's four 32-column blocks.
         const int q = warp & 3, hf = warp >> 2;
         const int m = q * 32 + lane;               // row within the tile
         const int i = row0 + m;                    // row within the chunk
@@ -254,34 +291,36 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
         if (!named_bar_or(1, 256, fail)) {
             tc_fence_after();
             if (t == 1) {
-                // G_10 (TMEM columns [0, 128)) -> bf16 row m of sG10, 16-byte chunks
-                // placed at (chunk ^ (m & 15)) so that a warp's row reads spread over banks.
-                uint4* grow = reinterpret_cast<uint4*>(sG10 + m * 256);
+                // G_10 (TMEM columns [0, 128)) -> bf16 K-major SW128 tile: K-block
+                // kb = j / 64, row m at 128 B, 16-byte chunk c at (c ^ (m & 7)).
                 for (int cb = 2 * hf; cb < 2 * hf + 2; ++cb) {
                     uint32_t r[32];
-                    tmem_ld32(tmem + lane_base + kColM + cb * 32, r);
+                    tmem_ld32(tmem + lane_base + cb * 32, r);
+                    uint4* row = reinterpret_cast<uint4*>(sG10 + (cb >> 1) * 16384 + m * 128);
 #pragma unroll
                     for (int u = 0; u < 4; ++u) {
-                        const int lc = cb * 4 + u;
-                        grow[lc ^ (m & 15)] = make_uint4(
+                        const int lc = (cb & 1) * 4 + u;
+                        row[lc ^ (m & 7)] = make_uint4(
                             pack_bf16x2(__uint_as_float(r[8 * u + 0]), __uint_as_float(r[8 * u + 1])),
                             pack_bf16x2(__uint_as_float(r[8 * u + 2]), __uint_as_float(r[8 * u + 3])),
                             pack_bf16x2(__uint_as_float(r[8 * u + 4]), __uint_as_float(r[8 * u + 5])),
                             pack_bf16x2(__uint_as_float(r[8 * u + 6]), __uint_as_float(r[8 * u + 7])));
                     }
                 }
+                fence_proxy_async_smem();          // G_10 is read by the MMA (async proxy)
             }
             tc_fence_before();
             named_bar_sync(1, 256);
             if (tid == 0) mbar_arrive(&bars[BAR_GCONV]);
 
-            const int nblk = KJ / 32;
             for (int hi = 0; hi < HG; ++hi) {
                 const int s = hi & 1;
-                // slot s (exp(cs) row scales) is free once the epilogue of head
-                // hi - 2 is done
-                fail = hi >= 2 && !mbar_wait(&bars[BAR_ACCEMPTY + s], (uint32_t)(((hi >> 1) - 1) & 1),
-                                             status);
+                // slot s (alpha factors, M slot, x/h slot scaling) is free once
+                // the MMAs and the epilogue of head hi - 2 are done
+                fail = hi >= 2 && !(mbar_wait(&bars[BAR_ACCEMPTY + s], (uint32_t)(((hi >> 1) - 1) & 1),
+                                              status) &&
+                                    mbar_wait(&bars[BAR_MEMPTY + s], (uint32_t)(((hi >> 1) - 1) & 1),
+                                              status));
                 if (named_bar_or(1, 256, fail)) break;
                 float* cs = s_cs + s * Q;
                 const float* hdt = s_dt + hi * Q;
@@ -302,80 +341,70 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
                 }
                 named_bar_sync(1, 256);
                 const float cs_i = cs[i];
-                // Column factors.  The decay between row i and column j < i
-                // factorises through any boundary r with cs_j >= r >= cs_i:
-                // exp(cs_i - cs_j) = exp(cs_i - r) exp(r - cs_j), both <= 1.
-                //   s_beta[j]  block left of the diagonal (t = 1), r = cs_{127}
-                //   s_beta2[k] diagonal block, r = end of the 32-column block of j = row0 + k
+                const float r = (t == 1) ? cs[127] : 0.f;
                 if (hf == 0) {
-                    if (t == 1) s_beta[m] = exp2f(cs[127] - cs[m]) * hdt[m];
-                    s_ez[s * 128 + m] = exp2f(cs_i);
+                    if (t == 1) s_beta[m] = exp2f(r - cs[m]) * hdt[m];
+                    s_al[s * 128 + m] = exp2f(cs_i - r);
                 } else {
                     const int j = row0 + m;
                     s_beta2[m] = exp2f(cs[row0 + (m | 31)] - cs[j]) * hdt[j];
                 }
-                // M is free once the MMAs of the previous head completed
-                fail = hi >= 1 && !mbar_wait(&bars[BAR_MEMPTY], (uint32_t)((hi - 1) & 1), status);
-                if (named_bar_or(1, 256, fail)) break;      // also publishes the factors and s_ez
-                if (tid == 0) mbar_arrive(&bars[BAR_EZFULL + s]);
+                // the head's x rows and entering state must have landed
+                fail = !mbar_wait(&bars[BAR_XFULL + s], (uint32_t)((hi >> 1) & 1), status);
+                if (named_bar_or(1, 256, fail)) break;   // also publishes the factors
+                if (tid == 0) mbar_arrive(&bars[BAR_ALFULL + s]);
+                if (t == 1) {
+                    // x rows 0..127 *= beta_j (row j = piece / 8), h *= exp(r), in place
+                    const float er = exp2f(r);
+                    scale_pieces(sX + s * S::kXTile, 128 * 8, tid, 256,
+                                 [&](int k) { return s_beta[k >> 3]; });
+                    scale_pieces(sH + s * S::kHTile, S::kHTile / 16, tid, 256,
+                                 [&](int) { return er; });
+                    fence_proxy_async_smem();
+                }
                 tc_fence_after();
 
-                const float alpha_off = (t == 1) ? exp2f(cs_i - cs[127]) : 0.f;
-                for (int cb = hf * (nblk / 2); cb < (hf + 1) * (nblk / 2); ++cb) {
-                    const int j0 = 32 * cb;
+                // diagonal-block mask -> TMEM slot s (64 columns of bf16 pairs)
+                for (int cb = 2 * hf; cb < 2 * hf + 2; ++cb) {
+                    const int j0 = row0 + 32 * cb;
                     uint32_t packed[16];
-                    if (j0 < row0) {
-                        // block left of the diagonal: G_10 (bf16, shared) * alpha * beta_j
-                        const uint4* grow = reinterpret_cast<const uint4*>(sG10 + m * 256);
+                    if (cb > q) {
 #pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            const int lc = cb * 4 + u;
-                            const uint4 gv = grow[lc ^ (m & 15)];
-                            const uint32_t* gu = reinterpret_cast<const uint32_t*>(&gv);
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const float2 gf =
-                                    __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&gu[e]));
-                                const int ja = 8 * lc + 2 * e;
-                                packed[4 * u + e] = pack_bf16x2(gf.x * alpha_off * s_beta[ja],
-                                                                gf.y * alpha_off * s_beta[ja + 1]);
-                            }
-                        }
+                        for (int u = 0; u < 16; ++u) packed[u] = 0u;
                     } else {
-                        const int rel = (j0 - row0) >> 5;   // 32-column block within the diagonal block
-                        if (rel > q) {
+                        uint32_t gr[32];
+                        tmem_ld32(tmem + lane_base + kColG + 32 * cb, gr);
+                        if (cb < q) {
+                            // entirely below the diagonal: factorised through the block's end
+                            const float alpha = exp2f(cs_i - cs[j0 + 31]);
+                            const float4* bet = reinterpret_cast<const float4*>(s_beta2 + 32 * cb);
 #pragma unroll
-                            for (int u = 0; u < 16; ++u) packed[u] = 0u;
+                            for (int u = 0; u < 8; ++u) {
+                                const float4 bv = bet[u];
+                                packed[2 * u] = pack_bf16x2(__uint_as_float(gr[4 * u]) * alpha * bv.x,
+                                                            __uint_as_float(gr[4 * u + 1]) * alpha * bv.y);
+                                packed[2 * u + 1] =
+                                    pack_bf16x2(__uint_as_float(gr[4 * u + 2]) * alpha * bv.z,
+                                                __uint_as_float(gr[4 * u + 3]) * alpha * bv.w);
+                            }
                         } else {
-                            uint32_t gr[32];
-                            tmem_ld32(tmem + lane_base + kColG + 32 * rel, gr);
-                            if (rel < q) {
-                                // entirely below the diagonal: factorised decay
-                                const float alpha = exp2f(cs_i - cs[j0 + 31]);
-                                const float* bet = s_beta2 + 32 * rel;
+                            // 32 x 32 block on the diagonal: exact exponentials, causal mask
 #pragma unroll
-                                for (int u = 0; u < 16; ++u)
-                                    packed[u] = pack_bf16x2(__uint_as_float(gr[2 * u]) * alpha * bet[2 * u],
-                                                            __uint_as_float(gr[2 * u + 1]) * alpha * bet[2 * u + 1]);
-                            } else {
-                                // 32 x 32 block on the diagonal: exact exponentials, causal mask
-#pragma unroll
-                                for (int u = 0; u < 16; ++u) {
-                                    const int ja = j0 + 2 * u, jb = ja + 1;
-                                    const float va = (ja <= i)
-                                        ? __uint_as_float(gr[2 * u]) * exp2f(cs_i - cs[ja]) * hdt[ja] : 0.f;
-                                    const float vb = (jb <= i)
-                                        ? __uint_as_float(gr[2 * u + 1]) * exp2f(cs_i - cs[jb]) * hdt[jb] : 0.f;
-                                    packed[u] = pack_bf16x2(va, vb);
-                                }
+                            for (int u = 0; u < 16; ++u) {
+                                const int ja = j0 + 2 * u, jb = ja + 1;
+                                const float va = (ja <= i)
+                                    ? __uint_as_float(gr[2 * u]) * exp2f(cs_i - cs[ja]) * hdt[ja] : 0.f;
+                                const float vb = (jb <= i)
+                                    ? __uint_as_float(gr[2 * u + 1]) * exp2f(cs_i - cs[jb]) * hdt[jb] : 0.f;
+                                packed[u] = pack_bf16x2(va, vb);
                             }
                         }
                     }
-                    tmem_st16(tmem + lane_base + kColM + (uint32_t)(j0 >> 1), packed);
+                    tmem_st16(tmem + lane_base + kColM + 64 * s + 16 * cb, packed);
                 }
                 tc_fence_before();
                 named_bar_sync(1, 256);
-                if (tid == 0) mbar_arrive(&bars[BAR_MFULL]);
+                if (tid == 0) mbar_arrive(&bars[BAR_MFULL + s]);
             }
         }
         if (fail) s_flag[0] = 1;
@@ -389,17 +418,16 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
         bool fail = false;
         for (int hi = 0; hi < HG; ++hi) {
             const int s = hi & 1;
-            const int h = head0 + hi;
-            // x_full too: the epilogue reads the TMA-written x rows (D x term); the
+            // x_full: the epilogue reads the TMA-written x rows (D x term); the
             // slot cannot be reloaded before this epilogue releases it.
             fail = !(mbar_wait(&bars[BAR_ACCFULL + s], (uint32_t)((hi >> 1) & 1), status) &&
-                     mbar_wait(&bars[BAR_EZFULL + s], (uint32_t)((hi >> 1) & 1), status) &&
+                     mbar_wait(&bars[BAR_ALFULL + s], (uint32_t)((hi >> 1) & 1), status) &&
                      mbar_wait(&bars[BAR_XFULL + s], (uint32_t)((hi >> 1) & 1), status));
             // staging slot s is free once the store issued two heads ago has read it
             if (m == 0) bulk_wait_group_read<1>();
             if (named_bar_or(2, 128, fail)) break;
             tc_fence_after();
-            const float ez = s_ez[s * 128 + m];
+            const float al = s_al[s * 128 + m];
             const float Dh = s_Dh[hi];
             const uint8_t* xrow = sX + s * S::kXTile + i * 128;
             uint4* ystage = reinterpret_cast<uint4*>(sY + s * 16384 + m * 128);
@@ -409,8 +437,8 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
                 uint32_t yr[32], zr[32];
                 tmem_ld32x2(acc + half * 32, acc + 64 + half * 32, yr, zr);
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const int lc = half * 4 + q;   // logical 16-byte chunk of the row
+                for (int u = 0; u < 4; ++u) {
+                    const int lc = half * 4 + u;   // logical 16-byte chunk of the row
                     const uint4 xv = *reinterpret_cast<const uint4*>(xrow + ((lc ^ (i & 7)) << 4));
                     const uint32_t* xu = reinterpret_cast<const uint32_t*>(&xv);
                     uint32_t o[4];
@@ -418,10 +446,10 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
                     for (int e = 0; e < 4; ++e) {
                         const float2 xf =
                             __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xu[e]));
-                        const int k = 8 * q + 2 * e;
-                        const float v0 = __uint_as_float(yr[k]) + ez * __uint_as_float(zr[k]) + Dh * xf.x;
+                        const int k = 8 * u + 2 * e;
+                        const float v0 = fmaf(al, __uint_as_float(zr[k]), __uint_as_float(yr[k])) + Dh * xf.x;
                         const float v1 =
-                            __uint_as_float(yr[k + 1]) + ez * __uint_as_float(zr[k + 1]) + Dh * xf.y;
+                            fmaf(al, __uint_as_float(zr[k + 1]), __uint_as_float(yr[k + 1])) + Dh * xf.y;
                         o[e] = pack_bf16x2(v0, v1);
                     }
                     ystage[lc ^ (m & 7)] = make_uint4(o[0], o[1], o[2], o[3]);
@@ -431,7 +459,7 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
             tc_fence_before();
             named_bar_sync(2, 128);
             if (m == 0) {
-                tma_store_4d(&tmY, sY + s * 16384, 0, h, (int)(t0 + row0), (int)b);
+                tma_store_4d(&tmY, sY + s * 16384, 0, head0 + hi, (int)(t0 + row0), (int)b);
                 bulk_commit_group();
                 mbar_arrive(&bars[BAR_ACCEMPTY + s]);
                 mbar_arrive(&bars[BAR_XEMPTY + s]);
@@ -473,11 +501,13 @@ cudaError_t launch_impl(const void* x, const float* dt, const float* A, const vo
                         const void* C, const float* D, const void* prev, void* y, const Dims& d,
                         cudaStream_t s) {
     using S = OutSmem<Q, N>;
-    CUtensorMap tmX, tmB, tmC, tmH;
+    CUtensorMap tmX, tmB, tmC, tmH, tmY;
     const uint64_t xdims[4] = {64, (uint64_t)d.H, (uint64_t)d.L, (uint64_t)d.b};
     const uint64_t xstr[3] = {64 * 2, (uint64_t)(d.H * 64 * 2), (uint64_t)(d.L * d.H * 64 * 2)};
     const uint32_t box128[4] = {64, 1, 128, 1};
     cudaError_t e = make_tmap_bf16(&tmX, x, 4, xdims, xstr, box128);
+    if (e != cudaSuccess) return e;
+    e = make_tmap_bf16(&tmY, y, 4, xdims, xstr, box128);
     if (e != cudaSuccess) return e;
     const uint64_t bdims[4] = {(uint64_t)N, (uint64_t)d.G, (uint64_t)d.L, (uint64_t)d.b};
     const uint64_t bstr[3] = {(uint64_t)N * 2, (uint64_t)(d.G * N * 2),
@@ -485,9 +515,6 @@ cudaError_t launch_impl(const void* x, const float* dt, const float* A, const vo
     e = make_tmap_bf16(&tmB, B, 4, bdims, bstr, box128);
     if (e != cudaSuccess) return e;
     e = make_tmap_bf16(&tmC, C, 4, bdims, bstr, box128);
-    if (e != cudaSuccess) return e;
-    CUtensorMap tmY;
-    e = make_tmap_bf16(&tmY, y, 4, xdims, xstr, box128);
     if (e != cudaSuccess) return e;
     const uint64_t hdims[2] = {(uint64_t)N, (uint64_t)(d.b * d.T * d.H * 64)};
     const uint64_t hstr[1] = {(uint64_t)N * 2};
