@@ -192,6 +192,21 @@ SSD_API ssd_status_t ssd_chunk_scan_fwd_noalloc(const void* x, const float* dt, 
  */
 SSD_API ssd_status_t ssd_poll_device_status(void* stream);
 
+/*
+ * ssd_state_walk_fwd -- steps (2) and (3) fused, the way ssd_chunk_scan_fwd
+ * runs them when batch x nheads / 2 fills the GPU: one CTA per (batch, head
+ * pair) walks the chunks in order keeping the running fp32 state on chip
+ * (tensor memory), and writes only prev_states (b,T,H,P,N) bf16 -- the state
+ * entering each chunk, same contents as ssd_state_passing_fwd's -- and, if
+ * final_states is non-NULL, the fp32 state after the last chunk.  Covers the
+ * tensor-core sizes only (SSD_BF16, chunk_size 128 or 256, headdim 64, dstate
+ * 64 or 128, nheads / ngroups even); other sizes return SSD_ERR_UNSUPPORTED.
+ */
+SSD_API ssd_status_t ssd_state_walk_fwd(const void* x, const float* dt, const float* A,
+                                        const void* B, const float* init_states,
+                                        void* prev_states, float* final_states, int chunk_size,
+                                        const ssd_dims_t* dims, ssd_dtype_t dtype, void* stream);
+
 /* Which kernel family ssd_chunk_scan_fwd uses for these sizes:
  * 1 = tcgen05 tensor-core kernels, 0 = SIMT fp32 kernels, -1 = rejected. */
 SSD_API int ssd_chunk_scan_fwd_uses_tensor_cores(const ssd_dims_t* dims, int chunk_size,

@@ -249,6 +249,32 @@ ssd_status_t ssd_chunk_output_fwd(const void* x, const float* dt, const float* A
     return e == cudaSuccess ? SSD_OK : cuda_fail(e, "chunk-output kernel");
 }
 
+ssd_status_t ssd_state_walk_fwd(const void* x, const float* dt, const float* A, const void* B,
+                                const float* init_states, void* prev_states, float* final_states,
+                                int chunk_size, const ssd_dims_t* dims, ssd_dtype_t dtype,
+                                void* stream) {
+    g_detail[0] = 0;
+    ssd::Dims d; ssd::Elt t;
+    ssd_status_t st = check_dims(dims, chunk_size, true, dtype, &d, &t);
+    if (st != SSD_OK) return st;
+    OPTIONAL_PTR(init_states);
+    OPTIONAL_PTR(final_states);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (d.b == 0) return SSD_OK;
+    if (d.L == 0) {
+        if (!final_states) return SSD_OK;
+        cudaError_t e = ssd::launch_copy_or_zero(init_states, final_states, d.b * d.H * d.P * d.N, s);
+        return e == cudaSuccess ? SSD_OK : cuda_fail(e, "final-state copy");
+    }
+    if (!tc_eligible(d, t))
+        return fail(SSD_ERR_UNSUPPORTED,
+                    "the state walk covers bf16, chunk 128/256, headdim 64, dstate 64/128 and an "
+                    "even number of heads per group");
+    REQUIRE_PTR(x); REQUIRE_PTR(dt); REQUIRE_PTR(A); REQUIRE_PTR(B); REQUIRE_PTR(prev_states);
+    cudaError_t e = ssd::launch_state_walk_tc(x, dt, A, B, init_states, prev_states, final_states, d, s);
+    return e == cudaSuccess ? SSD_OK : cuda_fail(e, "state-walk kernel");
+}
+
 ssd_status_t ssd_poll_device_status(void* stream) {
     g_detail[0] = 0;
     unsigned int v = 0;

@@ -12,6 +12,15 @@ bool tc_supported(const Dims& d, Elt t);
 
 cudaError_t launch_chunk_state_tc(const void* x, const float* dt, const float* A, const void* B,
                                   float* states, float* logdecay, const Dims& d, cudaStream_t s);
+// Chunk states and the inter-chunk recurrence fused: one CTA per (batch,
+// head pair) walks the chunks; writes the entering states (bf16, layout
+// (b, T, H, P, N)) and the final state (fp32, nullable).
+cudaError_t launch_state_walk_tc(const void* x, const float* dt, const float* A, const void* B,
+                                 const float* init, void* prev, float* final_states,
+                                 const Dims& d, cudaStream_t s);
+// True when the fused walk has enough (batch, head pair) walkers to fill the GPU.
+bool walk_preferred(const Dims& d);
+
 cudaError_t launch_chunk_out_tc(const void* x, const float* dt, const float* A, const void* B,
                                 const void* C, const float* D, const void* prev, void* y,
                                 const Dims& d, cudaStream_t s);

@@ -25,7 +25,7 @@ SSD_F32, SSD_BF16 = 0, 1
 EXPORTED = ("ssd_status_string", "ssd_last_error_detail", "ssd_chunk_scan_fwd_workspace_size",
             "ssd_chunk_scan_fwd", "ssd_step", "ssd_chunk_state_fwd", "ssd_state_passing_fwd",
             "ssd_chunk_output_fwd", "ssd_chunk_scan_fwd_uses_tensor_cores",
-            "ssd_chunk_scan_fwd_noalloc", "ssd_poll_device_status")
+            "ssd_chunk_scan_fwd_noalloc", "ssd_poll_device_status", "ssd_state_walk_fwd")
 
 
 class SSDError(RuntimeError):
@@ -69,6 +69,8 @@ def load(path: str = LIB_PATH):
     lib.ssd_chunk_scan_fwd_noalloc.restype = ctypes.c_int
     lib.ssd_chunk_scan_fwd_noalloc.argtypes = [_vp] * 6 + [ctypes.c_int, _vp, _vp, _vp, dims_p,
                                                            ctypes.c_int, _vp]
+    lib.ssd_state_walk_fwd.restype = ctypes.c_int
+    lib.ssd_state_walk_fwd.argtypes = [_vp] * 7 + [ctypes.c_int, dims_p, ctypes.c_int, _vp]
     lib.ssd_poll_device_status.restype = ctypes.c_int
     lib.ssd_poll_device_status.argtypes = [_vp]
     lib.ssd_step.restype = ctypes.c_int
@@ -239,6 +241,23 @@ def ssd_state_passing_fwd(chunk_states, chunk_logdecay, chunk_size: int, seqlen:
                                       _ptr(prev), _ptr(final), int(chunk_size), ctypes.byref(dims),
                                       _dtype_code(dtype), _stream(stream))
     _check(st, "ssd_state_passing_fwd")
+    return prev, final
+
+
+def ssd_state_walk_fwd(x, dt, A, B, chunk_size: int, init_states=None, want_final: bool = True,
+                       stream=None):
+    """Steps (2) + (3) fused (the on-chip state walk): entering states
+    (b,T,H,P,N) bf16 and the final state (b,H,P,N) fp32."""
+    dims = _fwd_dims(x, B)
+    b, L, H, P = x.shape
+    N = B.shape[3]
+    T = n_chunks(L, chunk_size)
+    prev = torch.empty((b, T, H, P, N), device=x.device, dtype=torch.bfloat16)
+    final = torch.empty((b, H, P, N), device=x.device, dtype=torch.float32) if want_final else None
+    st = load().ssd_state_walk_fwd(_ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(init_states),
+                                   _ptr(prev), _ptr(final), int(chunk_size), ctypes.byref(dims),
+                                   _dtype_code(x.dtype), _stream(stream))
+    _check(st, "ssd_state_walk_fwd")
     return prev, final
 
 

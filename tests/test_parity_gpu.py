@@ -207,6 +207,36 @@ def test_stage_state_passing(case):
     assert rel_err(fin.double().cpu().numpy(), final_ref) <= TOL[dtype]
 
 
+WALK_CASES = [(2, 600, 4, 64, 128, 1, 256, True), (1, 512, 4, 64, 64, 2, 128, False),
+              (3, 100, 2, 64, 128, 1, 128, True), (1, 777, 6, 64, 64, 1, 256, True)]
+
+
+@pytest.mark.parametrize("case", WALK_CASES, ids=lambda c: "_".join(map(str, c)))
+def test_stage_state_walk(case):
+    """The fused walk (chunk states + recurrence on chip) against the oracle's
+    entering states and final state."""
+    b, L, H, P, N, G, Q, init = case
+    inp = inputs.make_inputs(_w("walk", b, L, H, P, N, G, Q, "bf16", init, seed=34))
+    _, _, prev_ref, final_ref = _oracle_chunk_views(inp, Q)
+    d = to_dev(inp)
+    prev, fin = ssd.ssd_state_walk_fwd(d["x"], d["dt"], d["A"], d["B"], Q, init_states=d["init"])
+    torch.cuda.synchronize()
+    ep = rel_err(prev.double().cpu().numpy(), prev_ref)
+    ef = rel_err(fin.double().cpu().numpy(), final_ref)
+    record(f"walk_{'_'.join(map(str, case))}", prev=ep, final=ef)
+    assert ep <= TOL["bf16"] and ef <= TOL["bf16"], (ep, ef)
+
+
+def test_walk_path_full_forward_ragged_groups():
+    """A shape above the walk threshold (batch x heads / 2 >= SM count) with a
+    ragged last chunk, two groups and initial states: the forward takes the
+    walk + output path; every element checked."""
+    w = _w("walk_fwd", 8, 700, 40, 64, 128, 2, 256, "bf16", True, seed=35)
+    dims = ssd.make_dims(8, 700, 40, 64, 128, 2)
+    assert ssd.ssd_chunk_scan_fwd_uses_tensor_cores(dims, 256, torch.bfloat16) == 1
+    _check_full(w)
+
+
 @pytest.mark.parametrize("case", STAGE_CASES, ids=lambda c: "_".join(map(str, c)))
 def test_stage_chunk_output(case):
     dtype, b, L, H, P, N, G, Q = case
