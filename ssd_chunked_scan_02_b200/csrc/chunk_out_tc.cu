@@ -69,10 +69,10 @@ struct OutSmem {
     static constexpr int kBGBytes = (kBBytes > kHOff + 2 * kHTile) ? kBBytes : kHOff + 2 * kHTile;
     static constexpr int kXTile = Q * 128;                  // x rows [0, Q) of one head
     static constexpr int kX = kBG + kBGBytes;               // x ring: 2 slots
-    static constexpr int kYs = kX + 2 * kXTile;             // y staging: 2 x 16 KB
-    static constexpr int kDt = kYs + 2 * 128 * 128;         // float [kMaxHeads][Q]
-    static constexpr int kCs = kDt + kMaxHeads * Q * 4;     // float [2][Q] prefix sums (log2 units)
-    static constexpr int kBeta = kCs + 2 * Q * 4;           // float [128]  (t = 1 block left of diagonal)
+    static constexpr int kYs = kX + 2 * kXTile;             // y staging: 16 KB
+    static constexpr int kDt = kYs + 128 * 128;             // float [kMaxHeads][Q]
+    static constexpr int kCs = kDt + kMaxHeads * Q * 4;     // float [kMaxHeads][Q] prefix sums (log2 units)
+    static constexpr int kBeta = kCs + kMaxHeads * Q * 4;   // float [128]  (t = 1 block left of diagonal)
     static constexpr int kBeta2 = kBeta + 128 * 4;          // float [128]  (diagonal block)
     static constexpr int kAl = kBeta2 + 128 * 4;            // float [2][128] alpha_i per slot
     static constexpr int kAD = kAl + 2 * 128 * 4;           // float [2][kMaxHeads]: A_h (log2), D_h
@@ -287,6 +287,26 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
             s_Ah[tid] = A[head0 + tid] * kLog2e;
             s_Dh[tid] = Dv[head0 + tid];
         }
+        named_bar_sync(1, 256);
+        // inclusive prefix sums of dt*A (log2 units) for every head, 8 warps in
+        // parallel, while the G MMA runs
+        for (int k = warp; k < HG; k += 8) {
+            const float Ah = s_Ah[k];
+            const float* dk = s_dt + k * Q;
+            float* ck = s_cs + k * Q;
+            float carry = 0.f;
+            for (int base = 0; base < KJ; base += 32) {
+                float v = dk[base + lane] * Ah;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const float u = __shfl_up_sync(0xffffffffu, v, o);
+                    if (lane >= o) v += u;
+                }
+                v += carry;
+                ck[base + lane] = v;
+                carry = __shfl_sync(0xffffffffu, v, 31);
+            }
+        }
         bool fail = !mbar_wait(&bars[BAR_G], 0, status);
         if (!named_bar_or(1, 256, fail)) {
             tc_fence_after();
@@ -309,6 +329,22 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
                 }
                 fence_proxy_async_smem();          // G_10 is read by the MMA (async proxy)
             }
+            // Blocks above the diagonal (column block cb > quarter q) are zero in
+            // every head's mask: write them once, in both M slots -- after every
+            // warp has finished reading G_10 out of the same TMEM columns.
+            tc_fence_before();
+            named_bar_sync(1, 256);
+            tc_fence_after();
+            {
+                uint32_t zeros[16];
+#pragma unroll
+                for (int u = 0; u < 16; ++u) zeros[u] = 0u;
+                for (int cb = 2 * hf; cb < 2 * hf + 2; ++cb)
+                    if (cb > q) {
+                        tmem_st16(tmem + lane_base + kColM + 16 * cb, zeros);
+                        tmem_st16(tmem + lane_base + kColM + 64 + 16 * cb, zeros);
+                    }
+            }
             tc_fence_before();
             named_bar_sync(1, 256);
             if (tid == 0) mbar_arrive(&bars[BAR_GCONV]);
@@ -322,32 +358,16 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
                                     mbar_wait(&bars[BAR_MEMPTY + s], (uint32_t)(((hi >> 1) - 1) & 1),
                                               status));
                 if (named_bar_or(1, 256, fail)) break;
-                float* cs = s_cs + s * Q;
+                const float* cs = s_cs + hi * Q;
                 const float* hdt = s_dt + hi * Q;
-                if (warp == 0) {
-                    const float Ah = s_Ah[hi];
-                    float carry = 0.f;
-                    for (int base = 0; base < KJ; base += 32) {
-                        float v = hdt[base + lane] * Ah;
-#pragma unroll
-                        for (int o = 1; o < 32; o <<= 1) {
-                            const float u = __shfl_up_sync(0xffffffffu, v, o);
-                            if (lane >= o) v += u;
-                        }
-                        v += carry;
-                        cs[base + lane] = v;
-                        carry = __shfl_sync(0xffffffffu, v, 31);
-                    }
-                }
-                named_bar_sync(1, 256);
                 const float cs_i = cs[i];
                 const float r = (t == 1) ? cs[127] : 0.f;
                 if (hf == 0) {
-                    if (t == 1) s_beta[m] = exp2f(r - cs[m]) * hdt[m];
-                    s_al[s * 128 + m] = exp2f(cs_i - r);
+                    if (t == 1) s_beta[m] = fast_exp2(r - cs[m]) * hdt[m];
+                    s_al[s * 128 + m] = fast_exp2(cs_i - r);
                 } else {
                     const int j = row0 + m;
-                    s_beta2[m] = exp2f(cs[row0 + (m | 31)] - cs[j]) * hdt[j];
+                    s_beta2[m] = fast_exp2(cs[row0 + (m | 31)] - cs[j]) * hdt[j];
                 }
                 // the head's x rows and entering state must have landed
                 fail = !mbar_wait(&bars[BAR_XFULL + s], (uint32_t)((hi >> 1) & 1), status);
@@ -355,7 +375,7 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
                 if (tid == 0) mbar_arrive(&bars[BAR_ALFULL + s]);
                 if (t == 1) {
                     // x rows 0..127 *= beta_j (row j = piece / 8), h *= exp(r), in place
-                    const float er = exp2f(r);
+                    const float er = fast_exp2(r);
                     scale_pieces(sX + s * S::kXTile, 128 * 8, tid, 256,
                                  [&](int k) { return s_beta[k >> 3]; });
                     scale_pieces(sH + s * S::kHTile, S::kHTile / 16, tid, 256,
@@ -368,15 +388,13 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
                 for (int cb = 2 * hf; cb < 2 * hf + 2; ++cb) {
                     const int j0 = row0 + 32 * cb;
                     uint32_t packed[16];
-                    if (cb > q) {
-#pragma unroll
-                        for (int u = 0; u < 16; ++u) packed[u] = 0u;
-                    } else {
+                    if (cb > q) continue;                 // zero block, written once
+                    {
                         uint32_t gr[32];
                         tmem_ld32(tmem + lane_base + kColG + 32 * cb, gr);
                         if (cb < q) {
                             // entirely below the diagonal: factorised through the block's end
-                            const float alpha = exp2f(cs_i - cs[j0 + 31]);
+                            const float alpha = fast_exp2(cs_i - cs[j0 + 31]);
                             const float4* bet = reinterpret_cast<const float4*>(s_beta2 + 32 * cb);
 #pragma unroll
                             for (int u = 0; u < 8; ++u) {
@@ -393,9 +411,9 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
                             for (int u = 0; u < 16; ++u) {
                                 const int ja = j0 + 2 * u, jb = ja + 1;
                                 const float va = (ja <= i)
-                                    ? __uint_as_float(gr[2 * u]) * exp2f(cs_i - cs[ja]) * hdt[ja] : 0.f;
+                                    ? __uint_as_float(gr[2 * u]) * fast_exp2(cs_i - cs[ja]) * hdt[ja] : 0.f;
                                 const float vb = (jb <= i)
-                                    ? __uint_as_float(gr[2 * u + 1]) * exp2f(cs_i - cs[jb]) * hdt[jb] : 0.f;
+                                    ? __uint_as_float(gr[2 * u + 1]) * fast_exp2(cs_i - cs[jb]) * hdt[jb] : 0.f;
                                 packed[u] = pack_bf16x2(va, vb);
                             }
                         }
@@ -423,14 +441,14 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
             fail = !(mbar_wait(&bars[BAR_ACCFULL + s], (uint32_t)((hi >> 1) & 1), status) &&
                      mbar_wait(&bars[BAR_ALFULL + s], (uint32_t)((hi >> 1) & 1), status) &&
                      mbar_wait(&bars[BAR_XFULL + s], (uint32_t)((hi >> 1) & 1), status));
-            // staging slot s is free once the store issued two heads ago has read it
-            if (m == 0) bulk_wait_group_read<1>();
+            // the staging tile is free once the previous head's store has read it
+            if (m == 0) bulk_wait_group_read<0>();
             if (named_bar_or(2, 128, fail)) break;
             tc_fence_after();
             const float al = s_al[s * 128 + m];
             const float Dh = s_Dh[hi];
             const uint8_t* xrow = sX + s * S::kXTile + i * 128;
-            uint4* ystage = reinterpret_cast<uint4*>(sY + s * 16384 + m * 128);
+            uint4* ystage = reinterpret_cast<uint4*>(sY + m * 128);
             const uint32_t acc = tmem + lane_base + kColAcc + 128 * s;
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
@@ -459,7 +477,7 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
             tc_fence_before();
             named_bar_sync(2, 128);
             if (m == 0) {
-                tma_store_4d(&tmY, sY + s * 16384, 0, head0 + hi, (int)(t0 + row0), (int)b);
+                tma_store_4d(&tmY, sY, 0, head0 + hi, (int)(t0 + row0), (int)b);
                 bulk_commit_group();
                 mbar_arrive(&bars[BAR_ACCEMPTY + s]);
                 mbar_arrive(&bars[BAR_XEMPTY + s]);
