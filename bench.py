@@ -79,9 +79,9 @@ def kernel_bytes(w):
 
 
 KERNEL_SOURCES = {
-    "chunk_state": ["chunk_state_tc.cu", "chunk_simt.cu"],
+    "chunk_state": ["chunk_state_tc.cu", "sm100.cuh"],
     "state_pass": ["state_pass.cu"],
-    "chunk_out": ["chunk_out_tc.cu", "chunk_simt.cu"],
+    "chunk_out": ["chunk_out_tc.cu", "sm100.cuh"],
     "decode": ["decode.cu"],
 }
 
@@ -160,27 +160,35 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------- distributed plumbing
-def dist_setup(n):
-    import torch
+def dist_setup(n, backend: str = "nccl"):
+    """One process per GPU (launched by torchrun): join the process group and
+    return (rank, world, local_rank).  backend "gloo" is for CPU tests of
+    this logic."""
     if n <= 1:
         return 0, 1, 0
+    import datetime
+
+    import torch
     import torch.distributed as dist
     rank = int(os.environ["RANK"])
     world = int(os.environ["WORLD_SIZE"])
     local = int(os.environ.get("LOCAL_RANK", rank))
-    torch.cuda.set_device(local)
-    import datetime
-    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                            device_id=torch.device("cuda", local))
+    kw = {}
+    if backend == "nccl":
+        torch.cuda.set_device(local)
+        kw["device_id"] = torch.device("cuda", local)
+    dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120), **kw)
     return rank, world, local
 
 
-def max_over_ranks(v: float, world: int) -> float:
+def max_over_ranks(v: float, world: int, device="cuda") -> float:
+    """The maximum of a per-rank number over all ranks (device time of the
+    slowest rank)."""
     if world <= 1:
         return v
     import torch
     import torch.distributed as dist
-    t = torch.tensor([v], device="cuda", dtype=torch.float64)
+    t = torch.tensor([v], device=device, dtype=torch.float64)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
@@ -189,6 +197,12 @@ def barrier(world):
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
+
+
+def weak_scaling_value(tokens_per_rank: int, world: int, ms_per_step: float) -> float:
+    """Whole-job throughput: every rank processes its own tokens_per_rank per
+    step; the step takes the slowest rank's time."""
+    return world * tokens_per_rank / (ms_per_step * 1e-3)
 
 
 # ---------------------------------------------------------------- CPU oracle baseline
@@ -429,7 +443,7 @@ def main():
     if rank == 0:
         f_alg, f_dense, bytes_min = fwd_model(w)
         t = ms_per_step * 1e-3
-        tok_s = world * w.tokens / t
+        tok_s = weak_scaling_value(w.tokens, world, ms_per_step)
         t_roof = max(bytes_min / (pk["hbm_gbs"] * 1e9), f_dense / (pk["bf16_tflops"] * 1e12))
         bound = "hbm"
         peak_gbs = pk["hbm_gbs"]

@@ -207,6 +207,16 @@ SSD_API ssd_status_t ssd_state_walk_fwd(const void* x, const float* dt, const fl
                                         void* prev_states, float* final_states, int chunk_size,
                                         const ssd_dims_t* dims, ssd_dtype_t dtype, void* stream);
 
+/*
+ * Test hook for the failure path of the bounded device-side waits: launches
+ * one CTA that waits on an mbarrier nothing ever arrives at, giving up after
+ * at most `polls` polls (1 .. 2^20), so it records SSD_ERR_TIMEOUT in the
+ * device status word exactly as a kernel whose wait ran out would.  The wait
+ * always ends; nothing faults or hangs.  Read the result with
+ * ssd_poll_device_status.
+ */
+SSD_API ssd_status_t ssd_debug_expire_wait(unsigned int polls, void* stream);
+
 /* Which kernel family ssd_chunk_scan_fwd uses for these sizes:
  * 1 = tcgen05 tensor-core kernels, 0 = SIMT fp32 kernels, -1 = rejected. */
 SSD_API int ssd_chunk_scan_fwd_uses_tensor_cores(const ssd_dims_t* dims, int chunk_size,

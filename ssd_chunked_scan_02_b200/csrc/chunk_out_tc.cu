@@ -123,7 +123,7 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
                     const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmH,
                     const __grid_constant__ CUtensorMap tmY, const float* __restrict__ dt,
                     const float* __restrict__ A, const float* __restrict__ Dv, int64_t L, int H,
-                    int G, int64_t T, int HG, unsigned int* status) {
+                    int G, int64_t T, int HG, WaitCtx status) {
     using S = OutSmem<Q, N>;
     constexpr int kTiles = Q / 128;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -539,8 +539,8 @@ cudaError_t launch_impl(const void* x, const float* dt, const float* A, const vo
     const uint32_t hbox[2] = {64, 64};
     e = make_tmap_bf16(&tmH, prev, 2, hdims, hstr, hbox);
     if (e != cudaSuccess) return e;
-    unsigned int* status = device_status_ptr();
-    if (!status) return cudaErrorUnknown;
+    const sm100::WaitCtx status = make_wait_ctx();
+    if (!status.word) return cudaErrorUnknown;
 
     const int HG = pick_heads_per_cta(d.H, d.G);
     e = cudaFuncSetAttribute(chunk_out_tc_kernel<Q, N>,

@@ -75,7 +75,7 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tmX,
                       const __grid_constant__ CUtensorMap tmB, const float* __restrict__ dt,
                       const float* __restrict__ A, float* __restrict__ states,
                       float* __restrict__ logdecay, int64_t L, int H, int G, int64_t T, int HP,
-                      unsigned int* status) {
+                      WaitCtx status) {
     using S = StateSmem<Q, N>;
     constexpr bool kTrans = (N == 128);
     extern __shared__ uint8_t smem_raw[];
@@ -310,8 +310,8 @@ cudaError_t launch_impl(const void* x, const float* dt, const float* A, const vo
     const uint32_t bbox[4] = {64, 1, Q, 1};
     e = make_tmap_bf16(&tmB, B, 4, bdims, bstr, bbox);
     if (e != cudaSuccess) return e;
-    unsigned int* status = device_status_ptr();
-    if (!status) return cudaErrorUnknown;
+    const sm100::WaitCtx status = make_wait_ctx();
+    if (!status.word) return cudaErrorUnknown;
 
     const int HP = pick_pairs_per_cta(d.H, d.G);
     e = cudaFuncSetAttribute(chunk_state_tc_kernel<Q, N>,

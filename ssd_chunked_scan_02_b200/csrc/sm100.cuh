@@ -3,8 +3,8 @@
 // and tcgen05 (TMEM allocation, MMA issue/commit, TMEM loads and stores).
 //
 // Every wait here is bounded: a wait that runs out of iterations returns
-// false, and the kernel that called it records SSD_ERR_TIMEOUT in the
-// device status word and leaves (after waiting, again bounded, for the
+// false and records the timeout in the device status word, and the kernel
+// that called it leaves (after waiting, again bounded, for the
 // copies and MMAs it has in flight, and after freeing its TMEM).
 #pragma once
 #include <cuda.h>
@@ -46,17 +46,25 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
+// Where a launch reports a wait that gave up: the device status word and
+// this launch's token (a non-zero number unique to the launch).
+struct WaitCtx {
+    unsigned int* word;
+    unsigned int token;
+};
+
 // Bounded wait for the phase with the given parity to complete.  On giving
-// up, records SSD_ERR_TIMEOUT (4) in the device status word `status`.  Once
-// any wait has given up (status != 0), later waits that do not succeed at
-// once give up within 1024 polls instead of their own full limit.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned int* status) {
+// up, writes the launch's token to the status word (SSD_ERR_TIMEOUT for the
+// host).  Once a wait of the same launch has given up, the launch's other
+// waits that do not succeed give up within 1024 polls instead of their own
+// full limit; waits of other launches are not affected.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const WaitCtx& st) {
     for (uint32_t i = 0; i < kSpinLimit; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 1023u) == 1023u && *reinterpret_cast<volatile unsigned int*>(status) != 0u)
+        if ((i & 1023u) == 1023u && *reinterpret_cast<volatile unsigned int*>(st.word) == st.token)
             return false;
     }
-    atomicExch(status, 4u);
+    atomicExch(st.word, st.token);
     return false;
 }
 
@@ -77,6 +85,15 @@ __device__ __forceinline__ bool named_bar_or(int id, int nthreads, bool pred) {
         : "r"((uint32_t)pred), "r"(id), "r"(nthreads)
         : "memory");
     return r != 0;
+}
+
+// Same as mbar_wait with a caller-chosen poll bound.
+__device__ __forceinline__ bool mbar_wait_polls(uint64_t* bar, uint32_t parity, uint32_t polls,
+                                                const WaitCtx& st) {
+    for (uint32_t i = 0; i < polls; ++i)
+        if (mbar_try_wait(bar, parity)) return true;
+    atomicExch(st.word, st.token);
+    return false;
 }
 
 __device__ __forceinline__ void fence_proxy_async_smem() {

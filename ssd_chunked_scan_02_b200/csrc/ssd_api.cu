@@ -275,6 +275,14 @@ ssd_status_t ssd_state_walk_fwd(const void* x, const float* dt, const float* A, 
     return e == cudaSuccess ? SSD_OK : cuda_fail(e, "state-walk kernel");
 }
 
+ssd_status_t ssd_debug_expire_wait(unsigned int polls, void* stream) {
+    g_detail[0] = 0;
+    if (polls < 1 || polls > (1u << 20))
+        return fail(SSD_ERR_INVALID_ARG, "polls must be in [1, 2^20], got %u", polls);
+    cudaError_t e = ssd::launch_expire_wait(polls, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? SSD_OK : cuda_fail(e, "expire-wait kernel");
+}
+
 ssd_status_t ssd_poll_device_status(void* stream) {
     g_detail[0] = 0;
     unsigned int v = 0;

@@ -75,7 +75,7 @@ state_walk_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
                      const float* __restrict__ dt, const float* __restrict__ A,
                      const float* __restrict__ init, __nv_bfloat16* __restrict__ prev,
                      float* __restrict__ fin, int64_t L, int H, int G, int64_t T,
-                     unsigned int* status) {
+                     WaitCtx status) {
     using S = WalkSmem<Q, N>;
     constexpr bool kTrans = (N == 128);
     constexpr int kNSub = Q / kSub;
@@ -384,8 +384,8 @@ cudaError_t launch_impl(const void* x, const float* dt, const float* A, const vo
     const uint64_t bstr[3] = {(uint64_t)N * 2, (uint64_t)(d.G * N * 2), (uint64_t)(d.L * d.G * N * 2)};
     e = make_tmap_bf16(&tmB, B, 4, bdims, bstr, box);
     if (e != cudaSuccess) return e;
-    unsigned int* status = device_status_ptr();
-    if (!status) return cudaErrorUnknown;
+    const sm100::WaitCtx status = make_wait_ctx();
+    if (!status.word) return cudaErrorUnknown;
     e = cudaFuncSetAttribute(state_walk_tc_kernel<Q, N>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, S::kAlloc);
     if (e != cudaSuccess) return e;

@@ -6,6 +6,7 @@
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "../../include/ssd.h"
@@ -32,6 +33,13 @@ unsigned int* device_status_ptr() {
         g_status_ptr[dev] = static_cast<unsigned int*>(p);
     }
     return g_status_ptr[dev];
+}
+
+sm100::WaitCtx make_wait_ctx() {
+    static std::atomic<unsigned int> next{1};
+    unsigned int tok = next.fetch_add(1);
+    if (tok == 0) tok = next.fetch_add(1);   // 0 means "no timeout"
+    return sm100::WaitCtx{device_status_ptr(), tok};
 }
 
 bool tc_supported(const Dims& d, Elt t) {
@@ -73,6 +81,25 @@ cudaError_t make_tmap_bf16(CUtensorMap* map, const void* base, int rank, const u
                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+namespace {
+// One thread waits, with at most `polls` polls, on an mbarrier that nothing
+// arrives at: the bounded wait gives up and records the timeout status.
+__global__ void expire_wait_kernel(uint32_t polls, sm100::WaitCtx status) {
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x != 0) return;
+    sm100::mbar_init(&bar, 1);
+    sm100::fence_mbar_init();
+    sm100::mbar_wait_polls(&bar, 0, polls, status);
+}
+}  // namespace
+
+cudaError_t launch_expire_wait(uint32_t polls, cudaStream_t s) {
+    const sm100::WaitCtx status = make_wait_ctx();
+    if (!status.word) return cudaErrorUnknown;
+    expire_wait_kernel<<<1, 32, 0, s>>>(polls, status);
+    return cudaGetLastError();
 }
 
 cudaError_t read_and_clear_device_status(unsigned int* out, cudaStream_t s) {

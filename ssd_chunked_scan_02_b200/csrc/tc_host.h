@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "sm100.cuh"
+
 namespace ssd {
 
 // Encodes a bf16 tiled tensor map with 128-byte swizzle and zero fill for
@@ -17,6 +19,13 @@ bool tma_encoder_available();
 // Device address of the status word that bounded waits write (current
 // device; looked up once per device).  nullptr if unavailable.
 unsigned int* device_status_ptr();
+
+// Launches one CTA whose bounded mbarrier wait (at most `polls` polls) is
+// bound to give up, recording SSD_ERR_TIMEOUT in the device status word.
+cudaError_t launch_expire_wait(uint32_t polls, cudaStream_t s);
+
+// Status word and a fresh token for one launch's bounded waits.
+sm100::WaitCtx make_wait_ctx();
 
 // Copies the device status word to the host (synchronising `s`) and clears it.
 cudaError_t read_and_clear_device_status(unsigned int* out, cudaStream_t s);

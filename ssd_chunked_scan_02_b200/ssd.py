@@ -25,7 +25,8 @@ SSD_F32, SSD_BF16 = 0, 1
 EXPORTED = ("ssd_status_string", "ssd_last_error_detail", "ssd_chunk_scan_fwd_workspace_size",
             "ssd_chunk_scan_fwd", "ssd_step", "ssd_chunk_state_fwd", "ssd_state_passing_fwd",
             "ssd_chunk_output_fwd", "ssd_chunk_scan_fwd_uses_tensor_cores",
-            "ssd_chunk_scan_fwd_noalloc", "ssd_poll_device_status", "ssd_state_walk_fwd")
+            "ssd_chunk_scan_fwd_noalloc", "ssd_poll_device_status", "ssd_state_walk_fwd",
+            "ssd_debug_expire_wait")
 
 
 class SSDError(RuntimeError):
@@ -71,6 +72,8 @@ def load(path: str = LIB_PATH):
                                                            ctypes.c_int, _vp]
     lib.ssd_state_walk_fwd.restype = ctypes.c_int
     lib.ssd_state_walk_fwd.argtypes = [_vp] * 7 + [ctypes.c_int, dims_p, ctypes.c_int, _vp]
+    lib.ssd_debug_expire_wait.restype = ctypes.c_int
+    lib.ssd_debug_expire_wait.argtypes = [ctypes.c_uint, _vp]
     lib.ssd_poll_device_status.restype = ctypes.c_int
     lib.ssd_poll_device_status.argtypes = [_vp]
     lib.ssd_step.restype = ctypes.c_int
@@ -208,6 +211,11 @@ def ssd_poll_device_status(stream=None):
     """Raise SSDError(SSD_ERR_TIMEOUT) if a bounded device-side wait gave up
     since the last poll (synchronises the stream)."""
     _check(load().ssd_poll_device_status(_stream(stream)), "ssd_poll_device_status")
+
+
+def ssd_debug_expire_wait(polls: int = 4096, stream=None):
+    """Launch the bounded-wait failure probe (see include/ssd.h)."""
+    _check(load().ssd_debug_expire_wait(int(polls), _stream(stream)), "ssd_debug_expire_wait")
 
 
 def n_chunks(seqlen: int, chunk_size: int) -> int:
