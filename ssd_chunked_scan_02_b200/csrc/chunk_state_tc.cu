@@ -9,22 +9,25 @@
 // hands on is one dense contraction over the chunk's tokens (B^T (w * X)),
 // which is what the tensor cores are for.
 //
-// One CTA per (batch, chunk, HP consecutive head pairs of one B/C group).
-// Per head pair one MMA group over K = chunk tokens.  With dstate N = 128 it
-// computes S^T (M = N state rows, N = two heads x P = 64 columns): A = the
-// chunk's B tile, B = the two heads' scaled x tiles, so a TMEM lane is a
-// state column n and the epilogue's stores of S[p][n] are contiguous across
-// a warp.  With N = 64 it computes S (M = two heads x P rows, N = dstate).
-// Both operands are MN-major 128-byte-swizzled tiles brought by TMA; the B
-// tile is loaded once per CTA.  The work is pipelined over head pairs by
-// warp role:
-//   warp 12 (one lane)  TMA producer: B once, then x tiles of the pairs into
-//                       a two-slot ring;
-//   warps 0-7           dt staging and prefix sums for all heads up front,
-//                       then per pair: scale the x rows in place by w_j (the
-//                       MMA sees bf16(w_j x_j));
+// Persistent kernel: one CTA per SM walks a contiguous range of work items,
+// an item being one head pair of one (batch, chunk); items are ordered
+// (batch, chunk, pair), so a CTA reloads the chunk's B tile only where its
+// range crosses into another chunk (or B/C group).  With dstate N = 128 an
+// item computes S^T (M = N state rows, N = two heads x P = 64 columns): A =
+// the chunk's B tile, B = the pair's scaled x tiles, so a TMEM lane is a state
+// column n.  With N = 64 it computes S (M = two heads x P rows, N = dstate).
+// Both operands are MN-major 128-byte-swizzled tiles brought by TMA; x comes
+// through a six-stage ring of 64-token pair tiles (16 KB), so loads of the
+// next items stream while the current one is scaled, multiplied and stored.
+// Roles:
+//   warp 12 (one lane)  TMA producer: B tile per chunk, x stages into the ring;
+//   warps 0-7           dt prefix sums and w_j per item (the next item's dt is
+//                       loaded while the current one is scaled), then x rows
+//                       scaled in place by w_j (the MMA sees bf16(w_j x_j));
 //   warp 13 (one lane)  MMA issuer (and TMEM owner), two accumulator slots;
-//   warps 8-11          epilogue: TMEM -> fp32 S in HBM, layout (b, T, H, P, N).
+//   warps 8-11          epilogue: TMEM -> fp32 S in HBM, layout (b, T, H, P, N);
+//                       with N = 128 through a shared-memory staging pair and
+//                       TMA bulk stores of 32 x 128 fp32 boxes.
 // Every wait is bounded; a warpgroup leaves its loop only when all its
 // threads agree (bar.red.or).
 #include <cuda.h>
@@ -41,65 +44,97 @@ namespace {
 using namespace sm100;
 
 constexpr int kThreads = 448;
-constexpr int kMaxPairs = 4;
+constexpr int kRing = 6;          // x ring stages
+constexpr int kStageTok = 64;     // tokens per ring stage
 
 template <int Q, int N>
 struct StateSmem {
-    static constexpr int kXTile = Q * 128;                 // one head's x tile (Q rows x 64 bf16)
+    static constexpr int kStages = Q / kStageTok;          // ring stages per item
+    static constexpr int kHeadStage = kStageTok * 128;     // one head: 64 tokens x 64 bf16 (8 KB)
+    static constexpr int kStage = 2 * kHeadStage;          // one ring stage: a head pair (16 KB)
     static constexpr int kB = 0;                           // N/64 blocks of Q rows x 128 B
     static constexpr int kBBytes = (N / 64) * Q * 128;
-    static constexpr int kX = kB + kBBytes;                // [2 slots][2 heads] x tiles
-    static constexpr int kDt = kX + 4 * kXTile;            // float [2 kMaxPairs][Q]: dt
-    static constexpr int kW = kDt + 2 * kMaxPairs * Q * 4; // float [2 kMaxPairs][Q]: w_j
-    static constexpr int kA = kW + 2 * kMaxPairs * Q * 4;  // float [2 kMaxPairs]: A_h
-    static constexpr int kBar = kA + 2 * kMaxPairs * 4;
-    static constexpr int kTmem = kBar + 16 * 8;
-    static constexpr int kFlags = kTmem + 16;
+    static constexpr int kX = kB + kBBytes;
+    static constexpr int kOut = kX + kRing * kStage;       // N = 128: 2 x [32][128] fp32 staging
+    static constexpr int kOutBytes = (N == 128) ? 2 * 32 * 128 * 4 : 0;
+    static constexpr int kDt = kOut + kOutBytes;           // float [2][Q]: dt of one item
+    static constexpr int kW = kDt + 2 * Q * 4;             // float [2 buffers][2 heads][Q]: w_j
+    static constexpr int kSeg = kW + 4 * Q * 4;            // float [8]: prefix segment sums
+    static constexpr int kBar = kSeg + 8 * 4;
+    static constexpr int kTmem = kBar + 32 * 8;
+    static constexpr int kCnt = kTmem + 16;                // producer's issue counts
+    static constexpr int kFlags = kCnt + 16;
     static constexpr int kTotal = kFlags + 16;
     static constexpr int kAlloc = kTotal + 1024;           // slack to align the base to 1 KB
     static constexpr uint32_t kTmemCols = (2 * N <= 128) ? 128 : 256;   // two fp32 D slots
 };
 
 enum {
-    BAR_B = 0, BAR_XFULL = 1, BAR_XSCALED = 3, BAR_XEMPTY = 5, BAR_ACCFULL = 7, BAR_ACCEMPTY = 9,
-    BAR_COUNT = 11
+    BAR_B = 0,
+    BAR_XFULL = 1,
+    BAR_XSCALED = BAR_XFULL + kRing,
+    BAR_XEMPTY = BAR_XSCALED + kRing,
+    BAR_ACCFULL = BAR_XEMPTY + kRing,
+    BAR_ACCEMPTY = BAR_ACCFULL + 2,
+    BAR_DRAIN = BAR_ACCEMPTY + 2,
+    BAR_COUNT = BAR_DRAIN + 1
 };
+static_assert(BAR_COUNT <= 32, "barrier area");
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
     return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
+// Work item i -> (batch, chunk, head pair) and the key of the B tile it uses.
+struct Item {
+    int64_t b, c, key;
+    int pair, g;
+};
+__device__ __forceinline__ Item decode_item(int64_t i, int pairs, int64_t T, int hpg, int G) {
+    Item w;
+    w.pair = (int)(i % pairs);
+    const int64_t bc = i / pairs;
+    w.c = bc % T;
+    w.b = bc / T;
+    w.g = (2 * w.pair) / hpg;
+    w.key = bc * G + w.g;
+    return w;
+}
+
 template <int Q, int N>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tmX,
-                      const __grid_constant__ CUtensorMap tmB, const float* __restrict__ dt,
+                      const __grid_constant__ CUtensorMap tmB,
+                      const __grid_constant__ CUtensorMap tmS, const float* __restrict__ dt,
                       const float* __restrict__ A, float* __restrict__ states,
-                      float* __restrict__ logdecay, int64_t L, int H, int G, int64_t T, int HP,
-                      WaitCtx status) {
+                      float* __restrict__ logdecay, int64_t L, int H, int G, int64_t T,
+                      int64_t items, WaitCtx status) {
     using S = StateSmem<Q, N>;
     constexpr bool kTrans = (N == 128);
+    constexpr int kSt = S::kStages;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
     uint8_t* sB = smem + S::kB;
     uint8_t* sX = smem + S::kX;
+    float* s_out = reinterpret_cast<float*>(smem + S::kOut);
     float* s_dt = reinterpret_cast<float*>(smem + S::kDt);
     float* s_w = reinterpret_cast<float*>(smem + S::kW);
-    float* s_A = reinterpret_cast<float*>(smem + S::kA);
+    float* s_seg = reinterpret_cast<float*>(smem + S::kSeg);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::kBar);
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + S::kTmem);
+    volatile uint32_t* s_cnt = reinterpret_cast<volatile uint32_t*>(smem + S::kCnt);
     volatile int* s_flag = reinterpret_cast<volatile int*>(smem + S::kFlags);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int64_t bt = blockIdx.x;
-    const int64_t c = bt % T, b = bt / T;
-    const int pair0 = blockIdx.y * HP;
-    const int g = (2 * pair0) / (H / G);
-    const int64_t t0 = c * Q;
-    const int len = (int)((L - t0) < Q ? (L - t0) : Q);
+    const int pairs = H / 2, hpg = H / G;
+    const int64_t i0 = (int64_t)blockIdx.x * items / gridDim.x;
+    const int64_t i1 = (int64_t)(blockIdx.x + 1) * items / gridDim.x;
 
     if (tid == 0) {
         for (int i = 0; i < BAR_COUNT; ++i) mbar_init(&bars[i], 1);
         s_flag[0] = 0;
+        s_cnt[0] = 0;
+        s_cnt[1] = 0;
         fence_mbar_init();
     }
     if (warp == 13) {
@@ -116,22 +151,43 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tmX,
         if (lane == 0) {
             prefetch_tmap(&tmX);
             prefetch_tmap(&tmB);
-            mbar_expect_tx(&bars[BAR_B], S::kBBytes);
-            for (int nb = 0; nb < N / 64; ++nb)
-                tma_load_4d(sB + nb * Q * 128, &tmB, &bars[BAR_B], nb * 64, g, (int)t0, (int)b);
             bool ok = true;
-            for (int pi = 0; pi < HP && ok; ++pi) {
-                const int s = pi & 1;
-                if (pi >= 2)
-                    ok = mbar_wait(&bars[BAR_XEMPTY + s], (uint32_t)(((pi >> 1) - 1) & 1), status);
-                if (!ok) break;
-                const int h0 = 2 * (pair0 + pi);
-                mbar_expect_tx(&bars[BAR_XFULL + s], 2 * S::kXTile);
-                tma_load_4d(sX + (2 * s + 0) * S::kXTile, &tmX, &bars[BAR_XFULL + s], 0, h0,
-                            (int)t0, (int)b);
-                tma_load_4d(sX + (2 * s + 1) * S::kXTile, &tmX, &bars[BAR_XFULL + s], 0, h0 + 1,
-                            (int)t0, (int)b);
+            uint32_t it = 0, nb = 0;
+            int64_t key_prev = -1;
+            for (int64_t i = i0; i < i1 && ok; ++i) {
+                const Item w = decode_item(i, pairs, T, hpg, G);
+                const int t0 = (int)(w.c * Q);
+                if (w.key != key_prev) {
+                    // The B buffer is single: before replacing it, every MMA that
+                    // reads it (up to the last stage issued) must have completed.
+                    if (it > 0)
+                        ok = mbar_wait(&bars[BAR_XEMPTY + (it - 1) % kRing],
+                                       ((it - 1) / kRing) & 1, status);
+                    if (!ok) break;
+                    mbar_expect_tx(&bars[BAR_B], S::kBBytes);
+                    for (int q = 0; q < N / 64; ++q)
+                        tma_load_4d(sB + q * Q * 128, &tmB, &bars[BAR_B], q * 64, w.g, t0,
+                                    (int)w.b);
+                    ++nb;
+                    key_prev = w.key;
+                }
+                const int h0 = 2 * w.pair;
+                for (int st = 0; st < kSt; ++st) {
+                    const uint32_t slot = it % kRing;
+                    if (it >= kRing)
+                        ok = mbar_wait(&bars[BAR_XEMPTY + slot], ((it / kRing) - 1) & 1, status);
+                    if (!ok) break;
+                    uint8_t* dst = sX + slot * S::kStage;
+                    mbar_expect_tx(&bars[BAR_XFULL + slot], S::kStage);
+                    tma_load_4d(dst, &tmX, &bars[BAR_XFULL + slot], 0, h0, t0 + st * kStageTok,
+                                (int)w.b);
+                    tma_load_4d(dst + S::kHeadStage, &tmX, &bars[BAR_XFULL + slot], 0, h0 + 1,
+                                t0 + st * kStageTok, (int)w.b);
+                    ++it;
+                }
             }
+            s_cnt[0] = it;
+            s_cnt[1] = nb;
             if (!ok) s_flag[0] = 1;
         }
     } else if (warp == 13) {
@@ -140,47 +196,75 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tmX,
             // N = 128: D = S^T = B^T (w x) (M = 128 state rows, N = 128 pair columns);
             // N = 64:  D = S   = (w x)^T B (M = 128 pair rows, N = 64 state columns).
             constexpr uint32_t kIdesc = idesc_bf16_f32(128, kTrans ? 128 : N, true, true);
-            bool ok = mbar_wait(&bars[BAR_B], 0, status);
-            for (int pi = 0; pi < HP && ok; ++pi) {
-                const int s = pi & 1;
-                ok = mbar_wait(&bars[BAR_XSCALED + s], (uint32_t)((pi >> 1) & 1), status) &&
-                     (pi < 2 || mbar_wait(&bars[BAR_ACCEMPTY + s], (uint32_t)(((pi >> 1) - 1) & 1),
-                                          status));
+            constexpr uint32_t kSlotCols = kTrans ? 128 : N;
+            const uint32_t b0 = smem_u32(sB), x0 = smem_u32(sX);
+            bool ok = true;
+            uint32_t it = 0, nb = 0, k = 0;
+            int64_t key_prev = -1;
+            for (int64_t i = i0; i < i1 && ok; ++i, ++k) {
+                const Item w = decode_item(i, pairs, T, hpg, G);
+                if (w.key != key_prev) {
+                    ok = mbar_wait(&bars[BAR_B], nb & 1, status);
+                    if (!ok) break;
+                    ++nb;
+                    key_prev = w.key;
+                }
+                const uint32_t as = k & 1;
+                if (k >= 2) ok = mbar_wait(&bars[BAR_ACCEMPTY + as], ((k >> 1) - 1) & 1, status);
                 if (!ok) break;
                 tc_fence_after();
-                const uint32_t x0 = smem_u32(sX + (2 * s) * S::kXTile);
-                const uint32_t b0 = smem_u32(sB);
-                for (int ks = 0; ks < Q / 16; ++ks) {
-                    // x pair: two 64-column atoms (heads) kXTile apart; B: 64-column
-                    // atoms of dstate Q * 128 apart; 8-row groups 1024 B apart.
-                    const uint64_t xd = smem_desc_sw128(x0 + ks * 2048, S::kXTile, 1024);
-                    const uint64_t bd = smem_desc_sw128(b0 + ks * 2048, Q * 128, 1024);
-                    if (kTrans) mma_ss(tmem + s * 128, bd, xd, kIdesc, ks > 0);
-                    else mma_ss(tmem + s * N, xd, bd, kIdesc, ks > 0);
+                const uint32_t d = tmem + as * kSlotCols;
+                for (int st = 0; st < kSt; ++st, ++it) {
+                    const uint32_t slot = it % kRing;
+                    ok = mbar_wait(&bars[BAR_XSCALED + slot], (it / kRing) & 1, status);
+                    if (!ok) break;
+                    tc_fence_after();
+                    for (int ks = 0; ks < kStageTok / 16; ++ks) {
+                        // x pair: two 64-column atoms (heads) kHeadStage apart; B: 64-column
+                        // atoms of dstate Q * 128 apart; 8-row groups 1024 B apart.
+                        const uint64_t xd =
+                            smem_desc_sw128(x0 + slot * S::kStage + ks * 2048, S::kHeadStage, 1024);
+                        const uint64_t bd = smem_desc_sw128(
+                            b0 + (uint32_t)(st * kStageTok + ks * 16) * 128, Q * 128, 1024);
+                        if (kTrans) mma_ss(d, bd, xd, kIdesc, (st | ks) != 0);
+                        else mma_ss(d, xd, bd, kIdesc, (st | ks) != 0);
+                    }
+                    mma_commit(&bars[BAR_XEMPTY + slot]);
                 }
-                mma_commit(&bars[BAR_XEMPTY + s]);
-                mma_commit(&bars[BAR_ACCFULL + s]);
+                if (!ok) break;
+                mma_commit(&bars[BAR_ACCFULL + as]);
             }
+            mma_commit(&bars[BAR_DRAIN]);
             if (!ok) s_flag[0] = 1;
         }
     } else if (warp < 8) {
         // ================================================== dt / scale warps (0-7)
-        // (a0) dt of every head of the CTA for the whole chunk in one coalesced
-        // pass (the heads of a token are contiguous), then per head the
-        // inclusive prefix sum of dt*A and w_j = exp(cs_last - cs_j) dt_j.
-        const int nh = 2 * HP;
-        for (int e = tid; e < nh * Q; e += 256) {
-            const int j = e / nh, k = e - j * nh;
-            s_dt[k * Q + j] = (j < len) ? dt[(b * L + t0 + j) * H + 2 * pair0 + k] : 0.f;
-        }
-        if (tid < nh) s_A[tid] = A[2 * pair0 + tid];
-        named_bar_sync(1, 256);
-        for (int k = warp; k < nh; k += 8) {
-            const float Ah = s_A[k];
-            const float* dk = s_dt + k * Q;
-            float* wk = s_w + k * Q;
+        // Per item: (a0) the pair's dt for the chunk (the next item's dt is
+        // loaded while the current item is scaled), the inclusive prefix sum
+        // of dt*A per head in four 64-token segments (one warp each), and
+        // w_j = exp(cs_last - cs_j) dt_j; then each x row j scaled by w_j.
+        constexpr int kPer = (2 * Q) / 256;   // dt values per thread per item
+        constexpr int kSeg = Q / 4;           // tokens per prefix segment
+        float dreg[kPer];
+        auto load_dt = [&](const Item& w) {
+            const int64_t t0 = w.c * Q;
+            const int64_t len = (L - t0) < Q ? (L - t0) : Q;
+#pragma unroll
+            for (int r = 0; r < kPer; ++r) {
+                const int e = tid + 256 * r, hk = e / Q, j = e - hk * Q;
+                dreg[r] = (j < len) ? dt[(w.b * L + t0 + j) * H + 2 * w.pair + hk] : 0.f;
+            }
+        };
+        auto prefix = [&](const Item& w, int buf) {
+#pragma unroll
+            for (int r = 0; r < kPer; ++r) s_dt[tid + 256 * r] = dreg[r];
+            named_bar_sync(1, 256);
+            const int hk = warp >> 2, sg = warp & 3;
+            const float Ah = A[2 * w.pair + hk];
+            const float* dk = s_dt + hk * Q;
+            float* wk = s_w + (buf * 2 + hk) * Q;
             float carry = 0.f;
-            for (int base = 0; base < Q; base += 32) {
+            for (int base = sg * kSeg; base < (sg + 1) * kSeg; base += 32) {
                 float v = dk[base + lane] * Ah;
 #pragma unroll
                 for (int o = 1; o < 32; o <<= 1) {
@@ -188,42 +272,67 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tmX,
                     if (lane >= o) v += u;
                 }
                 v += carry;
-                wk[base + lane] = v;                     // cs_j for now
+                wk[base + lane] = v;                     // local cs_j for now
                 carry = __shfl_sync(0xffffffffu, v, 31);
             }
-            const float last = carry;                    // tokens past the sequence end add 0
-            __syncwarp();
-            for (int j = lane; j < Q; j += 32) wk[j] = expf(last - wk[j]) * dk[j];
-            if (lane == 0) logdecay[(b * T + c) * H + 2 * pair0 + k] = last;
-        }
-        named_bar_sync(1, 256);
+            if (lane == 0) s_seg[warp] = carry;
+            named_bar_sync(1, 256);
+            float off = 0.f, last = 0.f;                 // tokens past the sequence end add 0
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const float sq = s_seg[hk * 4 + q];
+                if (q < sg) off += sq;
+                last += sq;
+            }
+            for (int j = sg * kSeg + lane; j < (sg + 1) * kSeg; j += 32)
+                wk[j] = expf(last - (wk[j] + off)) * dk[j];
+            if (sg == 0 && lane == 0) logdecay[(w.b * T + w.c) * H + 2 * w.pair + hk] = last;
+            named_bar_sync(1, 256);
+        };
+
         bool fail = false;
-        for (int pi = 0; pi < HP; ++pi) {
-            const int s = pi & 1;
-            fail = !mbar_wait(&bars[BAR_XFULL + s], (uint32_t)((pi >> 1) & 1), status);
-            if (named_bar_or(1, 256, fail)) break;
-            // (a2 operand) scale each x row j of both heads by w_j, in place
-            for (int r = tid; r < 2 * Q; r += 256) {
-                const int k = r / Q, j = r - k * Q;
-                const float wj = s_w[(2 * pi + k) * Q + j];
-                uint4* row = reinterpret_cast<uint4*>(sX + (2 * s + k) * S::kXTile + j * 128);
-                uint4 v[8];
+        uint32_t it = 0;
+        if (i0 < i1) {
+            const Item w = decode_item(i0, pairs, T, hpg, G);
+            load_dt(w);
+            prefix(w, 0);
+        }
+        for (int64_t i = i0, k = 0; i < i1 && !fail; ++i, ++k) {
+            const bool has_next = i + 1 < i1;
+            Item wn;
+            if (has_next) {
+                wn = decode_item(i + 1, pairs, T, hpg, G);
+                load_dt(wn);
+            }
+            const float* wbuf = s_w + (k & 1) * 2 * Q;
+            for (int st = 0; st < kSt; ++st, ++it) {
+                const uint32_t slot = it % kRing;
+                const bool miss = !mbar_wait(&bars[BAR_XFULL + slot], (it / kRing) & 1, status);
+                if (named_bar_or(1, 256, miss)) {
+                    fail = true;
+                    break;
+                }
+                // (a2 operand) 128 rows (two heads x 64 tokens) of 8 16-byte chunks;
+                // a warp covers four whole rows per access (no bank conflicts).
+                uint4* tile = reinterpret_cast<uint4*>(sX + slot * S::kStage);
 #pragma unroll
-                for (int q = 0; q < 8; ++q) v[q] = row[q];
-#pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    uint32_t* u = reinterpret_cast<uint32_t*>(&v[q]);
+                for (int q = 0; q < 4; ++q) {
+                    const int idx = tid + 256 * q, row = idx >> 3;
+                    const float wj = wbuf[(row >> 6) * Q + st * kStageTok + (row & 63)];
+                    uint4 v = tile[idx];
+                    uint32_t* u = reinterpret_cast<uint32_t*>(&v);
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&u[e]));
                         u[e] = pack_bf16x2(f.x * wj, f.y * wj);
                     }
-                    row[q] = v[q];
+                    tile[idx] = v;
                 }
+                fence_proxy_async_smem();       // generic writes -> visible to the MMA (async proxy)
+                named_bar_sync(1, 256);
+                if (tid == 0) mbar_arrive(&bars[BAR_XSCALED + slot]);
             }
-            fence_proxy_async_smem();           // generic writes -> visible to the MMA (async proxy)
-            named_bar_sync(1, 256);
-            if (tid == 0) mbar_arrive(&bars[BAR_XSCALED + s]);
+            if (!fail && has_next) prefix(wn, (int)((k + 1) & 1));
         }
         if (fail) s_flag[0] = 1;
     } else {
@@ -231,54 +340,74 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tmX,
         const int m = tid - 256;                 // TMEM lane
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
         bool fail = false;
-        for (int pi = 0; pi < HP; ++pi) {
-            const int s = pi & 1;
-            fail = !mbar_wait(&bars[BAR_ACCFULL + s], (uint32_t)((pi >> 1) & 1), status);
-            if (named_bar_or(2, 128, fail)) break;
+        uint32_t q = 0;                          // staging boxes written so far
+        int64_t k = 0;
+        for (int64_t i = i0; i < i1; ++i, ++k) {
+            const Item w = decode_item(i, pairs, T, hpg, G);
+            const uint32_t as = (uint32_t)(k & 1);
+            const bool miss = !mbar_wait(&bars[BAR_ACCFULL + as], (uint32_t)((k >> 1) & 1), status);
+            if (named_bar_or(2, 128, miss)) {
+                fail = true;
+                break;
+            }
             tc_fence_after();
             if (kTrans) {
-                // lane m = state column n; column c = (head c / 64, p = c % 64)
-                const int n = m;
-#pragma unroll
-                for (int cc = 0; cc < 4; ++cc) {
+                // lane m = state column n; column c = (head c / 64, p = c % 64).  The
+                // pair's 128 (head, p) rows of S are contiguous in HBM; each 32-column
+                // block goes out as one 32 x 128 fp32 box.
+#pragma unroll 1
+                for (int cc = 0; cc < 4; ++cc, ++q) {
                     uint32_t r[32];
-                    tmem_ld32(tmem + lane_base + s * 128 + cc * 32, r);
-                    const int h = 2 * (pair0 + pi) + (cc >> 1);
-                    float* out = states + (((b * T + c) * H + h) * 64 + (cc & 1) * 32) * (int64_t)N + n;
+                    tmem_ld32(tmem + lane_base + as * 128 + cc * 32, r);
+                    float* buf = s_out + (q & 1) * (32 * 128);
+                    if (m == 0) bulk_wait_group_read<1>();   // the store of two boxes ago is read
+                    named_bar_sync(2, 128);
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) out[(int64_t)e * N] = __uint_as_float(r[e]);
+                    for (int e = 0; e < 32; ++e) buf[e * 128 + m] = __uint_as_float(r[e]);
+                    fence_proxy_async_smem();
+                    if (cc == 3) tc_fence_before();
+                    named_bar_sync(2, 128);
+                    if (m == 0) {
+                        if (cc == 3) mbar_arrive(&bars[BAR_ACCEMPTY + as]);
+                        tma_store_3d(&tmS, buf, 0, 2 * w.pair * 64 + cc * 32, (int)(w.b * T + w.c));
+                        bulk_commit_group();
+                    }
                 }
             } else {
                 // lane m = (head m / 64, p = m % 64); columns = state n
-                const int h = 2 * (pair0 + pi) + (m >> 6);
-                float* out = states + (((b * T + c) * H + h) * 64 + (m & 63)) * (int64_t)N;
+                const int h = 2 * w.pair + (m >> 6);
+                float* out = states + (((w.b * T + w.c) * H + h) * 64 + (m & 63)) * (int64_t)N;
 #pragma unroll
                 for (int cc = 0; cc < N / 32; ++cc) {
                     uint32_t r[32];
-                    tmem_ld32(tmem + lane_base + s * N + cc * 32, r);
+                    tmem_ld32(tmem + lane_base + as * N + cc * 32, r);
                     float4* o4 = reinterpret_cast<float4*>(out + cc * 32);
 #pragma unroll
-                    for (int q = 0; q < 8; ++q)
-                        o4[q] = make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]),
-                                            __uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3]));
+                    for (int e = 0; e < 8; ++e)
+                        o4[e] = make_float4(__uint_as_float(r[4 * e]), __uint_as_float(r[4 * e + 1]),
+                                            __uint_as_float(r[4 * e + 2]), __uint_as_float(r[4 * e + 3]));
                 }
+                tc_fence_before();
+                named_bar_sync(2, 128);
+                if (m == 0) mbar_arrive(&bars[BAR_ACCEMPTY + as]);
             }
-            tc_fence_before();
-            named_bar_sync(2, 128);
-            if (m == 0) mbar_arrive(&bars[BAR_ACCEMPTY + s]);
         }
+        if (m == 0) bulk_wait_group<0>();        // stores done before the CTA leaves
         if (fail) s_flag[0] = 1;
     }
 
     tc_fence_before();
     __syncthreads();
-    if (s_flag[0] && tid == 12 * 32) {
-        // A wait gave up somewhere: give outstanding TMA loads and MMAs a last
-        // (bounded) chance to land before the shared memory and TMEM go away.
-        mbar_wait(&bars[BAR_B], 0, status);
-        for (int k = 0; k < 2; ++k) {
-            mbar_wait(&bars[BAR_XFULL + k], 0, status);
-            mbar_wait(&bars[BAR_ACCFULL + k], 0, status);
+    if (tid == 13 * 32) {
+        mbar_wait(&bars[BAR_DRAIN], 0, status);  // every MMA of this CTA has completed
+    } else if (s_flag[0] && tid == 12 * 32) {
+        // A wait gave up somewhere: give outstanding TMA loads a last (bounded)
+        // chance to land before the shared memory goes away.
+        const uint32_t issued = s_cnt[0], nb = s_cnt[1];
+        if (nb) mbar_wait(&bars[BAR_B], (nb - 1) & 1, status);
+        for (uint32_t s = 0; s < (uint32_t)kRing; ++s) {
+            const uint32_t uses = issued / kRing + (s < issued % kRing ? 1u : 0u);
+            if (uses) mbar_wait(&bars[BAR_XFULL + s], (uses - 1) & 1, status);
         }
     }
     __syncthreads();
@@ -288,21 +417,14 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tmX,
     }
 }
 
-int pick_pairs_per_cta(int64_t H, int64_t G) {
-    const int64_t pairs_in_group = (H / G) / 2;
-    for (int hp = kMaxPairs; hp > 1; --hp)
-        if (pairs_in_group % hp == 0) return hp;
-    return 1;
-}
-
 template <int Q, int N>
 cudaError_t launch_impl(const void* x, const float* dt, const float* A, const void* B,
                         float* states, float* logdecay, const Dims& d, cudaStream_t s) {
     using S = StateSmem<Q, N>;
-    CUtensorMap tmX, tmB;
+    CUtensorMap tmX, tmB, tmS;
     const uint64_t xdims[4] = {64, (uint64_t)d.H, (uint64_t)d.L, (uint64_t)d.b};
     const uint64_t xstr[3] = {64 * 2, (uint64_t)(d.H * 64 * 2), (uint64_t)(d.L * d.H * 64 * 2)};
-    const uint32_t xbox[4] = {64, 1, Q, 1};
+    const uint32_t xbox[4] = {64, 1, kStageTok, 1};
     cudaError_t e = make_tmap_bf16(&tmX, x, 4, xdims, xstr, xbox);
     if (e != cudaSuccess) return e;
     const uint64_t bdims[4] = {(uint64_t)N, (uint64_t)d.G, (uint64_t)d.L, (uint64_t)d.b};
@@ -310,16 +432,32 @@ cudaError_t launch_impl(const void* x, const float* dt, const float* A, const vo
     const uint32_t bbox[4] = {64, 1, Q, 1};
     e = make_tmap_bf16(&tmB, B, 4, bdims, bstr, bbox);
     if (e != cudaSuccess) return e;
+    if (N == 128) {
+        // states as rows (head, p) of N fp32 per (batch, chunk)
+        const uint64_t sdims[3] = {(uint64_t)N, (uint64_t)(d.H * 64), (uint64_t)(d.b * d.T)};
+        const uint64_t sstr[2] = {(uint64_t)N * 4, (uint64_t)(d.H * 64 * N * 4)};
+        const uint32_t sbox[3] = {128, 32, 1};
+        e = make_tmap_f32_plain(&tmS, states, 3, sdims, sstr, sbox);
+        if (e != cudaSuccess) return e;
+    } else {
+        tmS = CUtensorMap{};
+    }
     const sm100::WaitCtx status = make_wait_ctx();
     if (!status.word) return cudaErrorUnknown;
 
-    const int HP = pick_pairs_per_cta(d.H, d.G);
+    const int64_t items = d.b * d.T * (d.H / 2);
+    if (items == 0) return cudaSuccess;
+    int dev = 0, sms = 148;
+    e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    const int64_t grid = items < sms ? items : sms;
     e = cudaFuncSetAttribute(chunk_state_tc_kernel<Q, N>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, S::kAlloc);
     if (e != cudaSuccess) return e;
-    dim3 grid((unsigned)(d.b * d.T), (unsigned)(d.H / (2 * HP)));
-    chunk_state_tc_kernel<Q, N><<<grid, kThreads, S::kAlloc, s>>>(
-        tmX, tmB, dt, A, states, logdecay, d.L, (int)d.H, (int)d.G, d.T, HP, status);
+    chunk_state_tc_kernel<Q, N><<<(unsigned)grid, kThreads, S::kAlloc, s>>>(
+        tmX, tmB, tmS, dt, A, states, logdecay, d.L, (int)d.H, (int)d.G, d.T, items, status);
     return cudaGetLastError();
 }
 

@@ -14,6 +14,11 @@ namespace ssd {
 cudaError_t make_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
                            const uint64_t* strides_bytes, const uint32_t* box);
 
+// fp32 tiled tensor map without swizzle (dense row-major boxes in shared memory).
+cudaError_t make_tmap_f32_plain(CUtensorMap* map, const void* base, int rank,
+                                const uint64_t* dims, const uint64_t* strides_bytes,
+                                const uint32_t* box);
+
 bool tma_encoder_available();
 
 // Device address of the status word that bounded waits write (current
