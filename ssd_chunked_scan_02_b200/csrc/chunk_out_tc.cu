@@ -21,19 +21,29 @@
 // and the entering state term exp(cs_i) C_i h = alpha_i C_i (exp(r) h).  Both go
 // into one accumulator ZW = G_10 (beta x_{0..127}) + C_t (exp(r) h)^T, scaled
 // by alpha_i in the epilogue (for t = 0, r = 0: ZW = C_0 h^T, alpha_i = exp(cs_i)).
-// Only the diagonal 128 x 128 block needs a per-element mask:
-//   Y = M X_t,  M_ij = G_ij exp(cs_i - cs_j) dt_j (j <= i),
-// and within it each 32-column block below the diagonal factorises the same
-// way through the block's end, so only the 32 x 32 blocks on the diagonal
-// evaluate an exponential per element.  Output: y = Y + alpha_i ZW + D_h x.
+// The diagonal 128 x 128 block, Y_i = sum_{j <= i} G_ij exp(cs_i - cs_j) dt_j x_j,
+// factorises through one boundary r for the whole tile: with
+//   a_i = 2^(cs_i - r),  b_j = 2^(r - cs_j) dt_j   (cs in log2 units),
+//   Y = diag(a) (G o causal) (b * X_t),
+// so the bf16 operand G o causal is built once per CTA and shared by all its
+// heads; a head only scales its x rows by b_j (in place) and its output rows
+// by a_i.  With r the midpoint of the tile's prefix sums, the factors stay in
+// [2^-60, 2^60] whenever the tile's decay spans at most 120 (log2 units): the
+// fast path.  A head whose tile decays faster takes the exact path instead: a
+// per-element mask M_ij = G_ij exp(cs_i - cs_j) dt_j (j <= i) in TMEM, with each
+// 32-column block below the diagonal factorised through the block's end (both
+// factors <= 1) and exponentials per element only on the 32 x 32 diagonal
+// blocks.  Output: y = a_i Y + alpha_i ZW + D_h x (a_i = 1 on the exact path);
+// the epilogue reads x for the skip term from global memory, one head ahead.
 //
 // Roles (448 threads):
 //   warps 0-7   prologue: G = C_t B^T (M = 128, N = 128 (t+1), K = dstate) is
-//               copied from TMEM: the diagonal block stays in TMEM (fp32), the
-//               block to its left goes to shared memory as bf16 (the A operand
-//               of G_10 X~); per head: prefix sums, factors, scaling of
-//               x rows 0..127 by beta and of h by exp(r) in place, and the
-//               diagonal-block mask written to TMEM as bf16 (two slots);
+//               copied from TMEM: the diagonal block becomes G o causal in bf16
+//               (TMEM, the A operand of Y), the block to its left goes to
+//               shared memory as bf16 (the A operand of G_10 X~); per head:
+//               factors, then the x rows of the tile scaled by b_j (fast path)
+//               or the exact mask written to TMEM (two slots), and for t = 1
+//               x rows 0..127 scaled by beta and h by exp(r), in place;
 //   warps 8-11  epilogue: y staged in shared memory, TMA store;
 //   warp 12     TMA producer (x rows and entering states of the heads, ring of 2);
 //   warp 13     MMA issuer and TMEM owner.
@@ -75,7 +85,9 @@ struct OutSmem {
     static constexpr int kBeta = kCs + kMaxHeads * Q * 4;   // float [128]  (t = 1 block left of diagonal)
     static constexpr int kBeta2 = kBeta + 128 * 4;          // float [128]  (diagonal block)
     static constexpr int kAl = kBeta2 + 128 * 4;            // float [2][128] alpha_i per slot
-    static constexpr int kAD = kAl + 2 * 128 * 4;           // float [2][kMaxHeads]: A_h (log2), D_h
+    static constexpr int kRow = kAl + 2 * 128 * 4;          // float [2][128] a_i per slot (1: exact path)
+    static constexpr int kPath = kRow + 2 * 128 * 4;        // int [2]: 1 = fast path, per slot
+    static constexpr int kAD = kPath + 16;                  // float [2][kMaxHeads]: A_h (log2), D_h
     static constexpr int kBar = kAD + 2 * kMaxHeads * 4;    // mbarriers
     static constexpr int kTmem = kBar + 24 * 8;
     static constexpr int kFlags = kTmem + 16;
@@ -92,7 +104,9 @@ enum {
 // TMEM columns
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColM = 0;       // bf16 diagonal-block mask, 2 slots of 64 columns (G_10 in the prologue)
-constexpr uint32_t kColG = 128;     // fp32 diagonal block of G, 128 columns
+constexpr uint32_t kColG = 128;     // fp32 diagonal block of G, 128 columns (prologue)
+constexpr uint32_t kColGC = 128;    // then: bf16 G o causal, 64 columns
+constexpr float kFastSpan = 120.f;  // largest tile decay (log2 units) of the fast path
 constexpr uint32_t kColAcc = 256;   // two slots of 128: Y (64) then ZW (64)
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
@@ -121,7 +135,8 @@ template <int Q, int N>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmH,
-                    const __grid_constant__ CUtensorMap tmY, const float* __restrict__ dt,
+                    const __grid_constant__ CUtensorMap tmY,
+                    const __nv_bfloat16* __restrict__ xg, const float* __restrict__ dt,
                     const float* __restrict__ A, const float* __restrict__ Dv, int64_t L, int H,
                     int G, int64_t T, int HG, WaitCtx status) {
     using S = OutSmem<Q, N>;
@@ -152,6 +167,8 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
     float* s_beta = reinterpret_cast<float*>(smem + S::kBeta);
     float* s_beta2 = reinterpret_cast<float*>(smem + S::kBeta2);
     float* s_al = reinterpret_cast<float*>(smem + S::kAl);
+    float* s_row = reinterpret_cast<float*>(smem + S::kRow);
+    volatile int* s_path = reinterpret_cast<volatile int*>(smem + S::kPath);
     float* s_Ah = reinterpret_cast<float*>(smem + S::kAD);
     float* s_Dh = s_Ah + kMaxHeads;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::kBar);
@@ -246,9 +263,11 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
                 tc_fence_after();
                 const uint32_t acc = tmem + kColAcc + 128 * s;
                 const uint32_t x0 = smem_u32(sX + s * S::kXTile);
-                // Y = M X_t over the diagonal block's 128 columns
+                // Y = (G o causal) (b * X_t) [fast path] or M X_t [exact path] over the
+                // diagonal block's 128 columns
+                const uint32_t amat = s_path[s] ? tmem + kColGC : tmem + kColM + 64 * s;
                 for (int ks = 0; ks < 8; ++ks)
-                    mma_ts(acc, tmem + kColM + 64 * s + ks * 8,
+                    mma_ts(acc, amat + ks * 8,
                            smem_desc_sw128(x0 + (row0 / 16 + ks) * 2048, 16, 1024), idesc_y, ks > 0);
                 // ZW = G_10 (beta x_{0..127}) [t = 1] + C_t (exp(r) h)^T
                 if (t == 1) {
@@ -266,6 +285,7 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
                            smem_desc_sw128(h0 + nb * 64 * 128 + ko, 16, 1024), idesc_z,
                            t == 1 || ks > 0);
                 }
+                mma_commit(&bars[BAR_XEMPTY + s]);           // x and h slot s: no reader left
                 mma_commit(&bars[BAR_MEMPTY + s]);
                 mma_commit(&bars[BAR_ACCFULL + s]);
             }
@@ -345,6 +365,28 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
                         tmem_st16(tmem + lane_base + kColM + 64 + 16 * cb, zeros);
                     }
             }
+            {
+                // G o causal -> bf16 at kColGC, over the fp32 columns it is made
+                // from: every warp reads its two 32-column blocks, then all write.
+                uint32_t pk[2][16];
+#pragma unroll
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    const int cb = 2 * hf + h2;
+                    uint32_t gr[32];
+                    tmem_ld32(tmem + lane_base + kColG + 32 * cb, gr);
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const int jj = 32 * cb + 2 * e;  // column within the tile
+                        pk[h2][e] = pack_bf16x2(jj <= m ? __uint_as_float(gr[2 * e]) : 0.f,
+                                                jj + 1 <= m ? __uint_as_float(gr[2 * e + 1]) : 0.f);
+                    }
+                }
+                tc_fence_before();
+                named_bar_sync(1, 256);
+                tc_fence_after();
+                tmem_st16(tmem + lane_base + kColGC + 16 * (2 * hf), pk[0]);
+                tmem_st16(tmem + lane_base + kColGC + 16 * (2 * hf + 1), pk[1]);
+            }
             tc_fence_before();
             named_bar_sync(1, 256);
             if (tid == 0) mbar_arrive(&bars[BAR_GCONV]);
@@ -362,13 +404,20 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
                 const float* hdt = s_dt + hi * Q;
                 const float cs_i = cs[i];
                 const float r = (t == 1) ? cs[127] : 0.f;
+                // the tile's decay span decides the path (the same for every thread)
+                const float c_first = cs[row0], c_last = cs[row0 + 127];
+                const bool fast = fabsf(c_last - c_first) <= kFastSpan;
+                const float r1 = 0.5f * (c_first + c_last);
                 if (hf == 0) {
                     if (t == 1) s_beta[m] = fast_exp2(r - cs[m]) * hdt[m];
                     s_al[s * 128 + m] = fast_exp2(cs_i - r);
+                    s_row[s * 128 + m] = fast ? fast_exp2(cs_i - r1) : 1.f;
                 } else {
+                    // fast: b_j; exact: beta of j through the end of its 32-column block
                     const int j = row0 + m;
-                    s_beta2[m] = fast_exp2(cs[row0 + (m | 31)] - cs[j]) * hdt[j];
+                    s_beta2[m] = fast_exp2((fast ? r1 : cs[row0 + (m | 31)]) - cs[j]) * hdt[j];
                 }
+                if (tid == 0) s_path[s] = fast ? 1 : 0;
                 // the head's x rows and entering state must have landed
                 fail = !mbar_wait(&bars[BAR_XFULL + s], (uint32_t)((hi >> 1) & 1), status);
                 if (named_bar_or(1, 256, fail)) break;   // also publishes the factors
@@ -380,18 +429,32 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
                                  [&](int k) { return s_beta[k >> 3]; });
                     scale_pieces(sH + s * S::kHTile, S::kHTile / 16, tid, 256,
                                  [&](int) { return er; });
-                    fence_proxy_async_smem();
                 }
+                if (fast) {
+                    // the tile's x rows *= b_j, in place (the MMA's B operand)
+                    scale_pieces(sX + s * S::kXTile + row0 * 128, 128 * 8, tid, 256,
+                                 [&](int k) { return s_beta2[k >> 3]; });
+                }
+                fence_proxy_async_smem();
                 tc_fence_after();
 
-                // diagonal-block mask -> TMEM slot s (64 columns of bf16 pairs)
-                for (int cb = 2 * hf; cb < 2 * hf + 2; ++cb) {
+                // exact path: diagonal-block mask -> TMEM slot s (64 columns of bf16
+                // pairs), from the bf16 G o causal
+                for (int cb = 2 * hf; cb < 2 * hf + 2 && !fast; ++cb) {
                     const int j0 = row0 + 32 * cb;
                     uint32_t packed[16];
                     if (cb > q) continue;                 // zero block, written once
                     {
                         uint32_t gr[32];
-                        tmem_ld32(tmem + lane_base + kColG + 32 * cb, gr);
+                        {
+                            uint32_t gp[16];
+                            tmem_ld16(tmem + lane_base + kColGC + 16 * cb, gp);
+#pragma unroll
+                            for (int e = 0; e < 16; ++e) {
+                                gr[2 * e] = gp[e] << 16;
+                                gr[2 * e + 1] = gp[e] & 0xffff0000u;
+                            }
+                        }
                         if (cb < q) {
                             // entirely below the diagonal: factorised through the block's end
                             const float alpha = fast_exp2(cs_i - cs[j0 + 31]);
@@ -434,20 +497,27 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
         const int i = row0 + m;
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
         bool fail = false;
+        // x row i of the next head (the D x term), loaded one head ahead from
+        // global memory (the tile's x rows in shared memory are scaled)
+        const bool row_in = t0 + i < L;
+        const uint4* xsrc = reinterpret_cast<const uint4*>(xg + ((b * L + t0 + i) * H + head0) * 64);
+        uint4 xr[8];
+        auto load_x_row = [&](int hh) {
+#pragma unroll
+            for (int u = 0; u < 8; ++u) xr[u] = row_in ? __ldg(xsrc + hh * 8 + u) : make_uint4(0, 0, 0, 0);
+        };
+        load_x_row(0);
         for (int hi = 0; hi < HG; ++hi) {
             const int s = hi & 1;
-            // x_full: the epilogue reads the TMA-written x rows (D x term); the
-            // slot cannot be reloaded before this epilogue releases it.
             fail = !(mbar_wait(&bars[BAR_ACCFULL + s], (uint32_t)((hi >> 1) & 1), status) &&
-                     mbar_wait(&bars[BAR_ALFULL + s], (uint32_t)((hi >> 1) & 1), status) &&
-                     mbar_wait(&bars[BAR_XFULL + s], (uint32_t)((hi >> 1) & 1), status));
+                     mbar_wait(&bars[BAR_ALFULL + s], (uint32_t)((hi >> 1) & 1), status));
             // the staging tile is free once the previous head's store has read it
             if (m == 0) bulk_wait_group_read<0>();
             if (named_bar_or(2, 128, fail)) break;
             tc_fence_after();
             const float al = s_al[s * 128 + m];
+            const float ar = s_row[s * 128 + m];
             const float Dh = s_Dh[hi];
-            const uint8_t* xrow = sX + s * S::kXTile + i * 128;
             uint4* ystage = reinterpret_cast<uint4*>(sY + m * 128);
             const uint32_t acc = tmem + lane_base + kColAcc + 128 * s;
 #pragma unroll
@@ -457,7 +527,7 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
                     const int lc = half * 4 + u;   // logical 16-byte chunk of the row
-                    const uint4 xv = *reinterpret_cast<const uint4*>(xrow + ((lc ^ (i & 7)) << 4));
+                    const uint4 xv = xr[lc];
                     const uint32_t* xu = reinterpret_cast<const uint32_t*>(&xv);
                     uint32_t o[4];
 #pragma unroll
@@ -465,9 +535,10 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
                         const float2 xf =
                             __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xu[e]));
                         const int k = 8 * u + 2 * e;
-                        const float v0 = fmaf(al, __uint_as_float(zr[k]), __uint_as_float(yr[k])) + Dh * xf.x;
+                        const float v0 =
+                            fmaf(al, __uint_as_float(zr[k]), ar * __uint_as_float(yr[k])) + Dh * xf.x;
                         const float v1 =
-                            fmaf(al, __uint_as_float(zr[k + 1]), __uint_as_float(yr[k + 1])) + Dh * xf.y;
+                            fmaf(al, __uint_as_float(zr[k + 1]), ar * __uint_as_float(yr[k + 1])) + Dh * xf.y;
                         o[e] = pack_bf16x2(v0, v1);
                     }
                     ystage[lc ^ (m & 7)] = make_uint4(o[0], o[1], o[2], o[3]);
@@ -480,8 +551,8 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
                 tma_store_4d(&tmY, sY, 0, head0 + hi, (int)(t0 + row0), (int)b);
                 bulk_commit_group();
                 mbar_arrive(&bars[BAR_ACCEMPTY + s]);
-                mbar_arrive(&bars[BAR_XEMPTY + s]);
             }
+            if (hi + 1 < HG) load_x_row(hi + 1);
         }
         if (m == 0) bulk_wait_group<0>();      // stores done before the CTA leaves
         if (fail) s_flag[0] = 1;
@@ -548,7 +619,8 @@ cudaError_t launch_impl(const void* x, const float* dt, const float* A, const vo
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)(d.b * d.T * (Q / 128)), (unsigned)(d.H / HG));
     chunk_out_tc_kernel<Q, N><<<grid, kThreads, S::kAlloc, s>>>(
-        tmX, tmB, tmC, tmH, tmY, dt, A, D, d.L, (int)d.H, (int)d.G, d.T, HG, status);
+        tmX, tmB, tmC, tmH, tmY, static_cast<const __nv_bfloat16*>(x), dt, A, D, d.L, (int)d.H,
+        (int)d.G, d.T, HG, status);
     return cudaGetLastError();
 }
 

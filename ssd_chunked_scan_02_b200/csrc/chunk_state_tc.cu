@@ -85,21 +85,31 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
     return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
-// Work item i -> (batch, chunk, head pair) and the key of the B tile it uses.
-struct Item {
-    int64_t b, c, key;
-    int pair, g;
+// Walks work items in order: i -> (batch, chunk, head pair), advanced by
+// counters (one division per CTA, at the start); key names the B tile used.
+struct ItemIter {
+    int64_t b, c, T;
+    int pair, pairs, hpg, G;
+    __device__ __forceinline__ void init(int64_t i, int pairs_, int64_t T_, int hpg_, int G_) {
+        pairs = pairs_;
+        T = T_;
+        hpg = hpg_;
+        G = G_;
+        const int64_t bc = i / pairs;
+        pair = (int)(i - bc * pairs);
+        c = bc % T;
+        b = bc / T;
+    }
+    __device__ __forceinline__ void next() {
+        if (++pair < pairs) return;
+        pair = 0;
+        if (++c < T) return;
+        c = 0;
+        ++b;
+    }
+    __device__ __forceinline__ int g() const { return (2 * pair) / hpg; }
+    __device__ __forceinline__ int64_t key() const { return (b * T + c) * G + g(); }
 };
-__device__ __forceinline__ Item decode_item(int64_t i, int pairs, int64_t T, int hpg, int G) {
-    Item w;
-    w.pair = (int)(i % pairs);
-    const int64_t bc = i / pairs;
-    w.c = bc % T;
-    w.b = bc / T;
-    w.g = (2 * w.pair) / hpg;
-    w.key = bc * G + w.g;
-    return w;
-}
 
 template <int Q, int N>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -154,10 +164,12 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tmX,
             bool ok = true;
             uint32_t it = 0, nb = 0;
             int64_t key_prev = -1;
-            for (int64_t i = i0; i < i1 && ok; ++i) {
-                const Item w = decode_item(i, pairs, T, hpg, G);
+            ItemIter w;
+            w.init(i0, pairs, T, hpg, G);
+            for (int64_t i = i0; i < i1 && ok; ++i, w.next()) {
                 const int t0 = (int)(w.c * Q);
-                if (w.key != key_prev) {
+                const int64_t key = w.key();
+                if (key != key_prev) {
                     // The B buffer is single: before replacing it, every MMA that
                     // reads it (up to the last stage issued) must have completed.
                     if (it > 0)
@@ -166,10 +178,10 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tmX,
                     if (!ok) break;
                     mbar_expect_tx(&bars[BAR_B], S::kBBytes);
                     for (int q = 0; q < N / 64; ++q)
-                        tma_load_4d(sB + q * Q * 128, &tmB, &bars[BAR_B], q * 64, w.g, t0,
+                        tma_load_4d(sB + q * Q * 128, &tmB, &bars[BAR_B], q * 64, w.g(), t0,
                                     (int)w.b);
                     ++nb;
-                    key_prev = w.key;
+                    key_prev = key;
                 }
                 const int h0 = 2 * w.pair;
                 for (int st = 0; st < kSt; ++st) {
@@ -201,13 +213,15 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tmX,
             bool ok = true;
             uint32_t it = 0, nb = 0, k = 0;
             int64_t key_prev = -1;
-            for (int64_t i = i0; i < i1 && ok; ++i, ++k) {
-                const Item w = decode_item(i, pairs, T, hpg, G);
-                if (w.key != key_prev) {
+            ItemIter w;
+            w.init(i0, pairs, T, hpg, G);
+            for (int64_t i = i0; i < i1 && ok; ++i, ++k, w.next()) {
+                const int64_t key = w.key();
+                if (key != key_prev) {
                     ok = mbar_wait(&bars[BAR_B], nb & 1, status);
                     if (!ok) break;
                     ++nb;
-                    key_prev = w.key;
+                    key_prev = key;
                 }
                 const uint32_t as = k & 1;
                 if (k >= 2) ok = mbar_wait(&bars[BAR_ACCEMPTY + as], ((k >> 1) - 1) & 1, status);
@@ -246,7 +260,7 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tmX,
         constexpr int kPer = (2 * Q) / 256;   // dt values per thread per item
         constexpr int kSeg = Q / 4;           // tokens per prefix segment
         float dreg[kPer];
-        auto load_dt = [&](const Item& w) {
+        auto load_dt = [&](const ItemIter& w) {
             const int64_t t0 = w.c * Q;
             const int64_t len = (L - t0) < Q ? (L - t0) : Q;
 #pragma unroll
@@ -255,7 +269,7 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tmX,
                 dreg[r] = (j < len) ? dt[(w.b * L + t0 + j) * H + 2 * w.pair + hk] : 0.f;
             }
         };
-        auto prefix = [&](const Item& w, int buf) {
+        auto prefix = [&](const ItemIter& w, int buf) {
 #pragma unroll
             for (int r = 0; r < kPer; ++r) s_dt[tid + 256 * r] = dreg[r];
             named_bar_sync(1, 256);
@@ -292,18 +306,16 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tmX,
 
         bool fail = false;
         uint32_t it = 0;
+        ItemIter wn;
+        wn.init(i0, pairs, T, hpg, G);
         if (i0 < i1) {
-            const Item w = decode_item(i0, pairs, T, hpg, G);
-            load_dt(w);
-            prefix(w, 0);
+            load_dt(wn);
+            prefix(wn, 0);
         }
         for (int64_t i = i0, k = 0; i < i1 && !fail; ++i, ++k) {
             const bool has_next = i + 1 < i1;
-            Item wn;
-            if (has_next) {
-                wn = decode_item(i + 1, pairs, T, hpg, G);
-                load_dt(wn);
-            }
+            wn.next();                          // item i + 1
+            if (has_next) load_dt(wn);
             const float* wbuf = s_w + (k & 1) * 2 * Q;
             for (int st = 0; st < kSt; ++st, ++it) {
                 const uint32_t slot = it % kRing;
@@ -342,8 +354,9 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tmX,
         bool fail = false;
         uint32_t q = 0;                          // staging boxes written so far
         int64_t k = 0;
-        for (int64_t i = i0; i < i1; ++i, ++k) {
-            const Item w = decode_item(i, pairs, T, hpg, G);
+        ItemIter w;
+        w.init(i0, pairs, T, hpg, G);
+        for (int64_t i = i0; i < i1; ++i, ++k, w.next()) {
             const uint32_t as = (uint32_t)(k & 1);
             const bool miss = !mbar_wait(&bars[BAR_ACCFULL + as], (uint32_t)((k >> 1) & 1), status);
             if (named_bar_or(2, 128, miss)) {

@@ -2,7 +2,7 @@
 // tensor-core kernels use: mbarriers (with bounded waits), TMA tile loads,
 // and tcgen05 (TMEM allocation, MMA issue/commit, TMEM loads and stores).
 //
-// Every wait here is bounded: a wait that runs out of iterations returns
+// Every wait here is bounded: a wait that runs out of time (about a second) returns
 // false and records the timeout in the device status word, and the kernel
 // that called it leaves (after waiting, again bounded, for the
 // copies and MMAs it has in flight, and after freeing its TMEM).
@@ -14,7 +14,6 @@
 namespace ssd {
 namespace sm100 {
 
-constexpr uint32_t kSpinLimit = 1u << 24;   // polls before giving up (order of a second)
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -53,16 +52,43 @@ struct WaitCtx {
     unsigned int token;
 };
 
+// Same test, but a thread whose phase is not complete yet may be suspended
+// (for at most about `suspend_ns`) until it completes: waiting threads then
+// take no issue slots from the warps that are working.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity,
+                                                    uint32_t suspend_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(suspend_ns)
+        : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+constexpr uint32_t kSuspendNs = 100000;            // longest single suspension: 0.1 ms
+constexpr uint64_t kWaitLimitNs = 1000000000ull;   // a wait gives up after 1 s
+
 // Bounded wait for the phase with the given parity to complete.  On giving
-// up, writes the launch's token to the status word (SSD_ERR_TIMEOUT for the
-// host).  Once a wait of the same launch has given up, the launch's other
-// waits that do not succeed give up within 1024 polls instead of their own
-// full limit; waits of other launches are not affected.
+// up (after about a second), writes the launch's token to the status word
+// (SSD_ERR_TIMEOUT for the host).  Once a wait of the same launch has given
+// up, the launch's other waits that do not succeed give up at their next
+// wake-up instead of their own full limit; waits of other launches are not
+// affected.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const WaitCtx& st) {
-    for (uint32_t i = 0; i < kSpinLimit; ++i) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 1023u) == 1023u && *reinterpret_cast<volatile unsigned int*>(st.word) == st.token)
-            return false;
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    for (;;) {
+        if (mbar_try_wait_sleep(bar, parity, kSuspendNs)) return true;
+        if (*reinterpret_cast<volatile unsigned int*>(st.word) == st.token) return false;
+        if (global_ns() - t0 > kWaitLimitNs) break;
     }
     atomicExch(st.word, st.token);
     return false;
@@ -117,6 +143,21 @@ __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, u
         "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2),
         "r"(c3)
         : "memory");
+}
+// TMA prefetch of a tile into L2 (no shared memory, no completion to wait
+// for): a later load of the same tile then finds it in L2.
+__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* map, int32_t c0, int32_t c1) {
+    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(c0), "r"(c1)
+                 : "memory");
+}
+__device__ __forceinline__ void tma_prefetch_4d(const CUtensorMap* map, int32_t c0, int32_t c1,
+                                                int32_t c2, int32_t c3) {
+    asm volatile("cp.async.bulk.prefetch.tensor.4d.L2.global.tile [%0, {%1, %2, %3, %4}];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+                 : "memory");
 }
 // TMA tile store from shared memory (tracked by the issuing thread's bulk
 // groups).  Elements outside the tensor's bounds are not written.
@@ -217,6 +258,19 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
           "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
           "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
           "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+}
+// Warp-collective TMEM load of 32 lanes x 16 consecutive 32-bit columns,
+// followed by its wait.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
         : "r"(taddr)
         : "memory");
 }

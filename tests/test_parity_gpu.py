@@ -332,6 +332,24 @@ def test_a_zero_cumulative_sum(dtype):
     assert rel_err(f, f_ref) <= TOL[dtype]
 
 
+def test_mixed_decay_heads_one_cta():
+    """Heads whose 128-token tiles decay by more than 2^120 take the exact
+    (per-element mask) path of the tensor-core output kernel, the others the
+    factorised one; both kinds share a CTA here, with one head near the bound."""
+    w = _w("mixdecay", 2, 600, 8, 64, 128, 1, 256, "bf16", True, seed=47)
+    inp = inputs.make_inputs(w)
+    A = inp["A"].clone()
+    A[0], A[3], A[5], A[6] = -1.0e3, -30.0, -40.0, 0.0
+    inp["A"] = A
+    y, f = gpu_fwd(inp, 256)
+    y_ref, f_ref = oracle_fwd(inp)
+    ey, ef = rel_err(y, y_ref), rel_err(f, f_ref)
+    record("mixed_decay_heads", y=ey, final=ef)
+    assert ey <= TOL["bf16"] and ef <= TOL["bf16"], (ey, ef)
+    for h in (0, 3, 5, 6):
+        assert rel_err(y[:, :, h], y_ref[:, :, h]) <= TOL["bf16"], h
+
+
 def test_c_zero_gives_skip_only():
     w = _w("czero", 2, 300, 4, 64, 128, 1, 256, "bf16", True, seed=46)
     inp = inputs.make_inputs(w)
