@@ -84,12 +84,12 @@ struct OutSmem {
     static constexpr int kCs = kDt + kMaxHeads * Q * 4;     // float [kMaxHeads][Q] prefix sums (log2 units)
     static constexpr int kBeta = kCs + kMaxHeads * Q * 4;   // float [128]  (t = 1 block left of diagonal)
     static constexpr int kBeta2 = kBeta + 128 * 4;          // float [128]  (diagonal block)
-    static constexpr int kAl = kBeta2 + 128 * 4;            // float [2][128] alpha_i per slot
-    static constexpr int kRow = kAl + 2 * 128 * 4;          // float [2][128] a_i per slot (1: exact path)
-    static constexpr int kPath = kRow + 2 * 128 * 4;        // int [2]: 1 = fast path, per slot
+    static constexpr int kAl = kBeta2 + 128 * 4;            // float [4][128] alpha_i per factor slot
+    static constexpr int kRow = kAl + 4 * 128 * 4;          // float [4][128] a_i (1: exact path)
+    static constexpr int kPath = kRow + 4 * 128 * 4;        // int [4]: 1 = fast path
     static constexpr int kAD = kPath + 16;                  // float [2][kMaxHeads]: A_h (log2), D_h
     static constexpr int kBar = kAD + 2 * kMaxHeads * 4;    // mbarriers
-    static constexpr int kTmem = kBar + 24 * 8;
+    static constexpr int kTmem = kBar + 32 * 8;
     static constexpr int kFlags = kTmem + 16;
     static constexpr int kTotal = kFlags + 16;
     static constexpr int kAlloc = kTotal + 1024;
@@ -98,7 +98,10 @@ struct OutSmem {
 // mbarrier indices
 enum {
     BAR_BC = 0, BAR_G = 1, BAR_GCONV = 2, BAR_XFULL = 3, BAR_XEMPTY = 5, BAR_MFULL = 7,
-    BAR_MEMPTY = 9, BAR_ACCFULL = 11, BAR_ACCEMPTY = 13, BAR_ALFULL = 15, BAR_COUNT = 17
+    BAR_MEMPTY = 9, BAR_ACCFULL = 11, BAR_ACCEMPTY = 13,
+    BAR_ALFULL = 15,    // four factor slots (alpha_i, a_i, path) per head modulo 4
+    BAR_FEMPTY = 19,    // four: the epilogue has read the factor slot
+    BAR_COUNT = 23
 };
 
 // TMEM columns
@@ -253,6 +256,8 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
             const uint32_t idesc_y = idesc_bf16_f32(128, 64, false, true);    // A in TMEM, x MN-major
             const uint32_t idesc_w = idesc_bf16_f32(128, 64, false, true);    // G_10 K-major, x~ MN-major
             const uint32_t idesc_z = idesc_bf16_f32(128, 64, false, false);   // C, h both K-major
+            const uint64_t gd = smem_desc_sw128(smem_u32(sG10), 16, 1024);
+            const uint64_t cd = smem_desc_sw128(smem_u32(sC), 16, 1024);
             for (int hi = 0; hi < HG && ok; ++hi) {
                 const int s = hi & 1;
                 ok = mbar_wait(&bars[BAR_MFULL + s], (uint32_t)((hi >> 1) & 1), status) &&
@@ -262,29 +267,27 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
                 if (!ok) break;
                 tc_fence_after();
                 const uint32_t acc = tmem + kColAcc + 128 * s;
-                const uint32_t x0 = smem_u32(sX + s * S::kXTile);
+                // descriptors of each operand's first K step; a K step moves the start
+                // address (16-byte units, low bits of the descriptor) by a constant
+                const uint64_t xd = smem_desc_sw128(smem_u32(sX + s * S::kXTile), 16, 1024);
+                const uint64_t hd = smem_desc_sw128(smem_u32(sH + s * S::kHTile), 16, 1024);
                 // Y = (G o causal) (b * X_t) [fast path] or M X_t [exact path] over the
                 // diagonal block's 128 columns
-                const uint32_t amat = s_path[s] ? tmem + kColGC : tmem + kColM + 64 * s;
+                const uint32_t amat = s_path[hi & 3] ? tmem + kColGC : tmem + kColM + 64 * s;
+#pragma unroll
                 for (int ks = 0; ks < 8; ++ks)
-                    mma_ts(acc, amat + ks * 8,
-                           smem_desc_sw128(x0 + (row0 / 16 + ks) * 2048, 16, 1024), idesc_y, ks > 0);
+                    mma_ts(acc, amat + ks * 8, xd + (uint64_t)((row0 / 16 + ks) * 128), idesc_y, ks > 0);
                 // ZW = G_10 (beta x_{0..127}) [t = 1] + C_t (exp(r) h)^T
                 if (t == 1) {
-                    const uint32_t g0 = smem_u32(sG10);
-                    for (int ks = 0; ks < 8; ++ks) {
-                        const int kb = ks >> 2, ko = (ks & 3) * 32;
-                        mma_ss(acc + 64, smem_desc_sw128(g0 + kb * 16384 + ko, 16, 1024),
-                               smem_desc_sw128(x0 + ks * 2048, 16, 1024), idesc_w, ks > 0);
-                    }
+#pragma unroll
+                    for (int ks = 0; ks < 8; ++ks)
+                        mma_ss(acc + 64, gd + (uint64_t)((ks >> 2) * 1024 + (ks & 3) * 2),
+                               xd + (uint64_t)(ks * 128), idesc_w, ks > 0);
                 }
-                const uint32_t c0 = smem_u32(sC), h0 = smem_u32(sH + s * S::kHTile);
-                for (int ks = 0; ks < N / 16; ++ks) {
-                    const int nb = ks >> 2, ko = (ks & 3) * 32;
-                    mma_ss(acc + 64, smem_desc_sw128(c0 + nb * 128 * 128 + ko, 16, 1024),
-                           smem_desc_sw128(h0 + nb * 64 * 128 + ko, 16, 1024), idesc_z,
-                           t == 1 || ks > 0);
-                }
+#pragma unroll
+                for (int ks = 0; ks < N / 16; ++ks)
+                    mma_ss(acc + 64, cd + (uint64_t)((ks >> 2) * 1024 + (ks & 3) * 2),
+                           hd + (uint64_t)((ks >> 2) * 512 + (ks & 3) * 2), idesc_z, t == 1 || ks > 0);
                 mma_commit(&bars[BAR_XEMPTY + s]);           // x and h slot s: no reader left
                 mma_commit(&bars[BAR_MEMPTY + s]);
                 mma_commit(&bars[BAR_ACCFULL + s]);
@@ -299,9 +302,20 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
         const int m = q * 32 + lane;               // row within the tile
         const int i = row0 + m;                    // row within the chunk
         const uint32_t lane_base = (uint32_t)(q * 32) << 16;
-        for (int e = tid; e < HG * KJ; e += 256) {
-            const int j = e / HG, k = e - j * HG;
-            s_dt[k * Q + j] = (j < len) ? dt[(b * L + t0 + j) * H + head0 + k] : 0.f;
+        {
+            // all loads first (the heads of a token are contiguous), then the stores
+            constexpr int kPerT = kMaxHeads * Q / 256;
+            float v[kPerT];
+#pragma unroll
+            for (int r = 0; r < kPerT; ++r) {
+                const int e = tid + 256 * r, j = e / HG, k = e - j * HG;
+                v[r] = (e < HG * KJ && j < len) ? dt[(b * L + t0 + j) * H + head0 + k] : 0.f;
+            }
+#pragma unroll
+            for (int r = 0; r < kPerT; ++r) {
+                const int e = tid + 256 * r, j = e / HG, k = e - j * HG;
+                if (e < HG * KJ) s_dt[k * Q + j] = v[r];
+            }
         }
         if (tid < HG) {
             s_Ah[tid] = A[head0 + tid] * kLog2e;
@@ -392,13 +406,10 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
             if (tid == 0) mbar_arrive(&bars[BAR_GCONV]);
 
             for (int hi = 0; hi < HG; ++hi) {
-                const int s = hi & 1;
-                // slot s (alpha factors, M slot, x/h slot scaling) is free once
-                // the MMAs and the epilogue of head hi - 2 are done
-                fail = hi >= 2 && !(mbar_wait(&bars[BAR_ACCEMPTY + s], (uint32_t)(((hi >> 1) - 1) & 1),
-                                              status) &&
-                                    mbar_wait(&bars[BAR_MEMPTY + s], (uint32_t)(((hi >> 1) - 1) & 1),
-                                              status));
+                const int s = hi & 1;                 // x/h slot, mask slot, accumulator
+                const int f = hi & 3;                 // factor slot
+                // factor slot f is free once the epilogue of head hi - 4 has read it
+                fail = hi >= 4 && !mbar_wait(&bars[BAR_FEMPTY + f], (uint32_t)(((hi >> 2) - 1) & 1), status);
                 if (named_bar_or(1, 256, fail)) break;
                 const float* cs = s_cs + hi * Q;
                 const float* hdt = s_dt + hi * Q;
@@ -410,18 +421,21 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
                 const float r1 = 0.5f * (c_first + c_last);
                 if (hf == 0) {
                     if (t == 1) s_beta[m] = fast_exp2(r - cs[m]) * hdt[m];
-                    s_al[s * 128 + m] = fast_exp2(cs_i - r);
-                    s_row[s * 128 + m] = fast ? fast_exp2(cs_i - r1) : 1.f;
+                    s_al[f * 128 + m] = fast_exp2(cs_i - r);
+                    s_row[f * 128 + m] = fast ? fast_exp2(cs_i - r1) : 1.f;
                 } else {
                     // fast: b_j; exact: beta of j through the end of its 32-column block
                     const int j = row0 + m;
                     s_beta2[m] = fast_exp2((fast ? r1 : cs[row0 + (m | 31)]) - cs[j]) * hdt[j];
                 }
-                if (tid == 0) s_path[s] = fast ? 1 : 0;
-                // the head's x rows and entering state must have landed
-                fail = !mbar_wait(&bars[BAR_XFULL + s], (uint32_t)((hi >> 1) & 1), status);
+                if (tid == 0) s_path[f] = fast ? 1 : 0;
+                // the exact path writes mask slot s: free once the MMAs of head hi - 2
+                // have completed; both paths need the head's x rows and entering state
+                fail = (!fast && hi >= 2 &&
+                        !mbar_wait(&bars[BAR_MEMPTY + s], (uint32_t)(((hi >> 1) - 1) & 1), status)) ||
+                       !mbar_wait(&bars[BAR_XFULL + s], (uint32_t)((hi >> 1) & 1), status);
                 if (named_bar_or(1, 256, fail)) break;   // also publishes the factors
-                if (tid == 0) mbar_arrive(&bars[BAR_ALFULL + s]);
+                if (tid == 0) mbar_arrive(&bars[BAR_ALFULL + f]);
                 if (t == 1) {
                     // x rows 0..127 *= beta_j (row j = piece / 8), h *= exp(r), in place
                     const float er = fast_exp2(r);
@@ -510,13 +524,13 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
         for (int hi = 0; hi < HG; ++hi) {
             const int s = hi & 1;
             fail = !(mbar_wait(&bars[BAR_ACCFULL + s], (uint32_t)((hi >> 1) & 1), status) &&
-                     mbar_wait(&bars[BAR_ALFULL + s], (uint32_t)((hi >> 1) & 1), status));
+                     mbar_wait(&bars[BAR_ALFULL + (hi & 3)], (uint32_t)((hi >> 2) & 1), status));
             // the staging tile is free once the previous head's store has read it
             if (m == 0) bulk_wait_group_read<0>();
             if (named_bar_or(2, 128, fail)) break;
             tc_fence_after();
-            const float al = s_al[s * 128 + m];
-            const float ar = s_row[s * 128 + m];
+            const float al = s_al[(hi & 3) * 128 + m];
+            const float ar = s_row[(hi & 3) * 128 + m];
             const float Dh = s_Dh[hi];
             uint4* ystage = reinterpret_cast<uint4*>(sY + m * 128);
             const uint32_t acc = tmem + lane_base + kColAcc + 128 * s;
@@ -551,6 +565,7 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
                 tma_store_4d(&tmY, sY, 0, head0 + hi, (int)(t0 + row0), (int)b);
                 bulk_commit_group();
                 mbar_arrive(&bars[BAR_ACCEMPTY + s]);
+                mbar_arrive(&bars[BAR_FEMPTY + (hi & 3)]);
             }
             if (hi + 1 < HG) load_x_row(hi + 1);
         }
