@@ -273,6 +273,50 @@ def run_reference(args):
     return 0
 
 
+# ---------------------------------------------------------------- secondary configs
+def measure_config(w, dev, stream, flush, reps, world, rank):
+    """Forward time of one more workload (the 130M layer, the length sweep):
+    L2 flushed before every timed forward, device time, max over ranks."""
+    import torch
+    from ssd_chunked_scan_02_b200 import inputs, ssd
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(w.seed + 1000 * rank)
+    inp = inputs.make_inputs(w, device=dev, gen=gen)
+    y = torch.empty_like(inp["x"])
+    fin = (torch.empty((w.batch, w.nheads, w.headdim, w.dstate), device=dev, dtype=torch.float32)
+           if w.want_final else None)
+    dims = ssd.make_dims(w.batch, w.seqlen, w.nheads, w.headdim, w.dstate, w.ngroups)
+    ws = torch.empty(ssd.ssd_chunk_scan_fwd_workspace_size(dims, w.chunk, inp["x"].dtype),
+                     device=dev, dtype=torch.uint8)
+
+    def fwd():
+        ssd.ssd_chunk_scan_fwd(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], inp["D"],
+                               w.chunk, init_states=inp["init"], y=y, final_states=fin,
+                               workspace=ws, stream=stream)
+    for _ in range(3):
+        flush.zero_()
+        fwd()
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(reps)]
+    for st, en in evs:
+        flush.zero_()
+        st.record(stream)
+        fwd()
+        en.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = max_over_ranks(sum(st.elapsed_time(en) for st, en in evs), world) / reps
+    f_alg, f_dense, bytes_min = fwd_model(w)
+    t = ms * 1e-3
+    out = {"workload": w.name, "ms_per_step": ms, "tokens_per_s": world * w.tokens / t,
+           "tflops_alg": f_alg / t / 1e12, "tflops_dense": f_dense / t / 1e12,
+           "bytes_min": bytes_min, "hbm_gbs_at_bytes_min": bytes_min / t / 1e9}
+    del inp, y, fin, ws
+    torch.cuda.empty_cache()
+    return out
+
+
 # ---------------------------------------------------------------- GPU arm
 def main():
     ap = argparse.ArgumentParser()
@@ -282,6 +326,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--decode-steps", type=int, default=50)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra-configs", action="store_true",
+                    help="skip the 130M-layer and length-sweep lines")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
@@ -433,6 +479,16 @@ def main():
     torch.cuda.synchronize(dev)
     e2e_ms = max_over_ranks(s.elapsed_time(e), world) / e2e_steps
 
+    # ---- the other configurations of the metric: 130M layer and the N = 64 sweep
+    extra = None
+    if not args.no_extra_configs:
+        reps = max(3, args.steps // 4)
+        extra = [measure_config(cw, dev, stream, flush, reps, world, rank)
+                 for cw in (inputs.LAYER_130M,) + tuple(inputs.SWEEP)]
+        for e in extra:
+            e["hbm_frac_at_bytes_min"] = e["hbm_gbs_at_bytes_min"] / pk["hbm_gbs"]
+            e["pct_bf16_peak_dense"] = 100 * e["tflops_dense"] / pk["bf16_tflops"]
+
     # ---- CPU oracle baseline (rank 0, N = 1 only)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -474,6 +530,7 @@ def main():
                        "frac_hbm": dec_gbs / peak_gbs, "bytes_per_step": dec_bytes},
             "e2e": {"value": world * w.tokens / (e2e_ms * 1e-3), "unit": UNIT,
                     "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "other_configs": extra,
             "cpu_baseline": cpu,
             "gpu_launches": 3 * args.steps,
             "clocks": clocks,
