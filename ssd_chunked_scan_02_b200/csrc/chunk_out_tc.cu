@@ -116,21 +116,28 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
     return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
-// Scale `n16` 16-byte pieces (8 bf16 each) of a shared-memory tile in place by a
-// per-piece factor f(piece): done by `nthr` threads, thread index `t`.
-template <typename F>
-__device__ __forceinline__ void scale_pieces(uint8_t* base, int n16, int t, int nthr, F f) {
-    for (int k = t; k < n16; k += nthr) {
-        uint4* ptr = reinterpret_cast<uint4*>(base) + k;
-        uint4 v = *ptr;
-        const float s = f(k);
-        uint32_t* u = reinterpret_cast<uint32_t*>(&v);
+// Scale the 16-byte pieces (8 bf16 each) of a shared-memory tile in place by a
+// per-piece factor f(piece): 256 threads, NPER pieces each (piece t + 256 r for
+// thread t); all loads are issued before any arithmetic.
+template <int NPER, typename F>
+__device__ __forceinline__ void scale_pieces(uint8_t* base, int t, F f) {
+    uint4* p = reinterpret_cast<uint4*>(base);
+    uint4 v[NPER];
+    float sc[NPER];
+#pragma unroll
+    for (int r = 0; r < NPER; ++r) {
+        v[r] = p[t + 256 * r];
+        sc[r] = f(t + 256 * r);
+    }
+#pragma unroll
+    for (int r = 0; r < NPER; ++r) {
+        uint32_t* u = reinterpret_cast<uint32_t*>(&v[r]);
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
             const float2 x = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&u[e]));
-            u[e] = pack_bf16x2(x.x * s, x.y * s);
+            u[e] = pack_bf16x2(x.x * sc[r], x.y * sc[r]);
         }
-        *ptr = v;
+        p[t + 256 * r] = v[r];
     }
 }
 
@@ -439,15 +446,12 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
                 if (t == 1) {
                     // x rows 0..127 *= beta_j (row j = piece / 8), h *= exp(r), in place
                     const float er = fast_exp2(r);
-                    scale_pieces(sX + s * S::kXTile, 128 * 8, tid, 256,
-                                 [&](int k) { return s_beta[k >> 3]; });
-                    scale_pieces(sH + s * S::kHTile, S::kHTile / 16, tid, 256,
-                                 [&](int) { return er; });
+                    scale_pieces<4>(sX + s * S::kXTile, tid, [&](int k) { return s_beta[k >> 3]; });
+                    scale_pieces<S::kHTile / 4096>(sH + s * S::kHTile, tid, [&](int) { return er; });
                 }
                 if (fast) {
                     // the tile's x rows *= b_j, in place (the MMA's B operand)
-                    scale_pieces(sX + s * S::kXTile + row0 * 128, 128 * 8, tid, 256,
-                                 [&](int k) { return s_beta2[k >> 3]; });
+                    scale_pieces<4>(sX + s * S::kXTile + row0 * 128, tid, [&](int k) { return s_beta2[k >> 3]; });
                 }
                 fence_proxy_async_smem();
                 tc_fence_after();
