@@ -8,7 +8,8 @@
 // Every (batch, head, p, n) state element is an independent chain; a thread
 // owns VEC consecutive elements (16-byte fp32 loads), walks the chunks in
 // order and keeps the chain in registers.  Loads of later chunks do not
-// depend on the chain, so the unrolled loop keeps several in flight.
+// depend on the chain: a register ring keeps 16 chunks' loads in flight, so
+// the walk stays bandwidth-bound even with few chains (one long sequence).
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -16,6 +17,8 @@
 
 namespace ssd {
 namespace {
+
+constexpr int kAhead = 16;   // chunks whose loads are in flight per thread
 
 template <typename TP, int VEC>
 struct Store;
@@ -81,14 +84,40 @@ state_pass_kernel(const float* __restrict__ states, const float* __restrict__ lo
     const float* sp = states + (bb * T * H + h) * PN + off;
     const float* lp = logdecay + bb * T * H + h;
     TP* pp = prev + (bb * T * H + h) * PN + off;
-#pragma unroll 4
-    for (int64_t c = 0; c < T; ++c) {
-        float sv[VEC];
-        load_vec<VEC>(sp + c * cstride, sv);
-        const float a = expf(lp[c * H]);
-        Store<TP, VEC>::run(pp + c * cstride, hs);
+    // a ring of kAhead chunks' states and log-decays in registers: the loads
+    // of chunk c + kAhead are issued when chunk c is consumed
+    float sv[kAhead][VEC], lv[kAhead];
+    const float* sq = sp;                    // the next chunk to load
+    const float* lq = lp;
+    int64_t cl = 0;
 #pragma unroll
-        for (int k = 0; k < VEC; ++k) hs[k] = fmaf(a, hs[k], sv[k]);
+    for (int k = 0; k < kAhead; ++k) {
+        if (cl < T) {
+            load_vec<VEC>(sq, sv[k]);
+            lv[k] = *lq;
+        }
+        sq += cstride;
+        lq += H;
+        ++cl;
+    }
+    TP* pq = pp;
+    for (int64_t c0 = 0; c0 < T; c0 += kAhead) {
+#pragma unroll
+        for (int k = 0; k < kAhead; ++k) {
+            if (c0 + k >= T) break;
+            const float a = expf(lv[k]);
+            Store<TP, VEC>::run(pq, hs);
+            pq += cstride;
+#pragma unroll
+            for (int e = 0; e < VEC; ++e) hs[e] = fmaf(a, hs[e], sv[k][e]);
+            if (cl < T) {
+                load_vec<VEC>(sq, sv[k]);
+                lv[k] = *lq;
+            }
+            sq += cstride;
+            lq += H;
+            ++cl;
+        }
     }
     if (fin) {
         float* fp = fin + bh * PN + off;
