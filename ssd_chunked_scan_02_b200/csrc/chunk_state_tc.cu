@@ -25,9 +25,10 @@
 //                       loaded while the current one is scaled), then x rows
 //                       scaled in place by w_j (the MMA sees bf16(w_j x_j));
 //   warp 13 (one lane)  MMA issuer (and TMEM owner), two accumulator slots;
-//   warps 8-11          epilogue: TMEM -> fp32 S in HBM, layout (b, T, H, P, N);
-//                       with N = 128 through a shared-memory staging pair and
-//                       TMA bulk stores of 32 x 128 fp32 boxes.
+//   warps 8-11          epilogue: TMEM -> fp32 S in HBM, layout (b, T, H, P, N),
+//                       through a shared-memory staging pair and TMA bulk
+//                       stores (N = 128: 32 x 128 fp32 boxes; N = 64: 128 x 32,
+//                       128-byte swizzled).
 // Every wait is bounded; a warpgroup leaves its loop only when all its
 // threads agree (bar.red.or).
 #include <cuda.h>
@@ -56,7 +57,7 @@ struct StateSmem {
     static constexpr int kBBytes = (N / 64) * Q * 128;
     static constexpr int kX = kB + kBBytes;
     static constexpr int kOut = kX + kRing * kStage;       // N = 128: 2 x [32][128] fp32 staging
-    static constexpr int kOutBytes = (N == 128) ? 2 * 32 * 128 * 4 : 0;
+    static constexpr int kOutBytes = 2 * 32 * 128 * 4;     // two 16 KB staging boxes
     static constexpr int kDt = kOut + kOutBytes;           // float [2][Q]: dt of one item
     static constexpr int kW = kDt + 2 * Q * 4;             // float [2 buffers][2 heads][Q]: w_j
     static constexpr int kSeg = kW + 4 * Q * 4;            // float [8]: prefix segment sums
@@ -387,22 +388,30 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tmX,
                     }
                 }
             } else {
-                // lane m = (head m / 64, p = m % 64); columns = state n
-                const int h = 2 * w.pair + (m >> 6);
-                float* out = states + (((w.b * T + w.c) * H + h) * 64 + (m & 63)) * (int64_t)N;
-#pragma unroll
-                for (int cc = 0; cc < N / 32; ++cc) {
+                // lane m = (head m / 64, p = m % 64); columns = state n.  Each 32-column
+                // block of the pair's 128 rows goes out as one 128 x 32 fp32 box,
+                // staged with the 128-byte swizzle (chunk c of row m at c ^ (m & 7)).
+#pragma unroll 1
+                for (int cc = 0; cc < N / 32; ++cc, ++q) {
                     uint32_t r[32];
                     tmem_ld32(tmem + lane_base + as * N + cc * 32, r);
-                    float4* o4 = reinterpret_cast<float4*>(out + cc * 32);
+                    float* buf = s_out + (q & 1) * (32 * 128);
+                    if (m == 0) bulk_wait_group_read<1>();   // the store of two boxes ago is read
+                    named_bar_sync(2, 128);
+                    float4* b4 = reinterpret_cast<float4*>(buf) + m * 8;
 #pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        o4[e] = make_float4(__uint_as_float(r[4 * e]), __uint_as_float(r[4 * e + 1]),
-                                            __uint_as_float(r[4 * e + 2]), __uint_as_float(r[4 * e + 3]));
+                    for (int c4 = 0; c4 < 8; ++c4)
+                        b4[c4 ^ (m & 7)] = make_float4(__uint_as_float(r[4 * c4]), __uint_as_float(r[4 * c4 + 1]),
+                                                       __uint_as_float(r[4 * c4 + 2]), __uint_as_float(r[4 * c4 + 3]));
+                    fence_proxy_async_smem();
+                    if (cc == N / 32 - 1) tc_fence_before();
+                    named_bar_sync(2, 128);
+                    if (m == 0) {
+                        if (cc == N / 32 - 1) mbar_arrive(&bars[BAR_ACCEMPTY + as]);
+                        tma_store_3d(&tmS, buf, cc * 32, 2 * w.pair * 64, (int)(w.b * T + w.c));
+                        bulk_commit_group();
+                    }
                 }
-                tc_fence_before();
-                named_bar_sync(2, 128);
-                if (m == 0) mbar_arrive(&bars[BAR_ACCEMPTY + as]);
             }
         }
         if (m == 0) bulk_wait_group<0>();        // stores done before the CTA leaves
@@ -445,15 +454,14 @@ cudaError_t launch_impl(const void* x, const float* dt, const float* A, const vo
     const uint32_t bbox[4] = {64, 1, Q, 1};
     e = make_tmap_bf16(&tmB, B, 4, bdims, bstr, bbox);
     if (e != cudaSuccess) return e;
-    if (N == 128) {
-        // states as rows (head, p) of N fp32 per (batch, chunk)
+    {
+        // states as rows (head, p) of N fp32 per (batch, chunk); N = 128: boxes of
+        // 32 rows x 128 (plain), N = 64: boxes of 128 rows x 32 (128-byte swizzle)
         const uint64_t sdims[3] = {(uint64_t)N, (uint64_t)(d.H * 64), (uint64_t)(d.b * d.T)};
         const uint64_t sstr[2] = {(uint64_t)N * 4, (uint64_t)(d.H * 64 * N * 4)};
-        const uint32_t sbox[3] = {128, 32, 1};
-        e = make_tmap_f32_plain(&tmS, states, 3, sdims, sstr, sbox);
+        const uint32_t sbox128[3] = {128, 32, 1}, sbox64[3] = {32, 128, 1};
+        e = make_tmap_f32_plain(&tmS, states, 3, sdims, sstr, N == 128 ? sbox128 : sbox64, N != 128);
         if (e != cudaSuccess) return e;
-    } else {
-        tmS = CUtensorMap{};
     }
     const sm100::WaitCtx status = make_wait_ctx();
     if (!status.word) return cudaErrorUnknown;

@@ -85,14 +85,15 @@ cudaError_t make_tmap_bf16(CUtensorMap* map, const void* base, int rank, const u
 
 cudaError_t make_tmap_f32_plain(CUtensorMap* map, const void* base, int rank,
                                 const uint64_t* dims, const uint64_t* strides_bytes,
-                                const uint32_t* box) {
+                                const uint32_t* box, bool swizzle128) {
     if (!tma_encoder_available()) return cudaErrorNotSupported;
     cuuint32_t estride[5] = {1, 1, 1, 1, 1};
     CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, (cuuint32_t)rank,
                           const_cast<void*>(base), reinterpret_cast<const cuuint64_t*>(dims),
                           reinterpret_cast<const cuuint64_t*>(strides_bytes),
                           reinterpret_cast<const cuuint32_t*>(box), estride,
-                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                           CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }

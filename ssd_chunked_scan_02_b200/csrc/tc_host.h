@@ -14,10 +14,11 @@ namespace ssd {
 cudaError_t make_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
                            const uint64_t* strides_bytes, const uint32_t* box);
 
-// fp32 tiled tensor map without swizzle (dense row-major boxes in shared memory).
+// fp32 tiled tensor map: dense row-major boxes in shared memory, or with the
+// 128-byte swizzle (box rows of 32 floats, 16-byte chunk c of row r at c ^ (r % 8)).
 cudaError_t make_tmap_f32_plain(CUtensorMap* map, const void* base, int rank,
                                 const uint64_t* dims, const uint64_t* strides_bytes,
-                                const uint32_t* box);
+                                const uint32_t* box, bool swizzle128 = false);
 
 bool tma_encoder_available();
 
