@@ -459,23 +459,58 @@ def main():
               if v is not None and k not in ("A", "D")) + A.numel() * 4 + D.numel() * 4
     d2h = y.numel() * y.element_size() + fin.numel() * 4
 
-    def e2e_step():
-        for k in ("x", "dt", "B", "C", "init", "A", "D"):
-            if host[k] is not None:
-                inp[k].copy_(host[k], non_blocking=True)
-        fwd()
-        y_host.copy_(y, non_blocking=True)
-        f_host.copy_(fin, non_blocking=True)
-    for _ in range(3):
-        e2e_step()
+    # Two device buffer sets and three streams: step k uploads into set k % 2
+    # while step k - 1 computes and downloads, so host->device and
+    # device->host copies (full duplex) and compute overlap across steps.
+    # Every step still copies all of its inputs in and its y and final
+    # states out; the timed region covers all of it.
+    sets = [inp, {k: (torch.empty_like(v) if v is not None else None) for k, v in inp.items()}]
+    outs = [(y, fin), (torch.empty_like(y), torch.empty_like(fin))]
+    y_hosts = [y_host, torch.empty(y.shape, dtype=y.dtype, pin_memory=True)]
+    f_hosts = [f_host, torch.empty(fin.shape, dtype=fin.dtype, pin_memory=True)]
+    s_in = torch.cuda.Stream(dev)
+    s_out = torch.cuda.Stream(dev)
+    ev_in = [torch.cuda.Event() for _ in range(2)]      # inputs of set j uploaded
+    ev_used = [torch.cuda.Event() for _ in range(2)]    # forward on set j done
+    ev_out = [torch.cuda.Event() for _ in range(2)]     # results of set j downloaded
+    started = [False, False]
+
+    def e2e_step(k):
+        j = k & 1
+        d_in, (yy, ff) = sets[j], outs[j]
+        with torch.cuda.stream(s_in):
+            if started[j]:
+                s_in.wait_event(ev_used[j])
+            for key in ("x", "dt", "B", "C", "init", "A", "D"):
+                if host[key] is not None:
+                    d_in[key].copy_(host[key], non_blocking=True)
+            ev_in[j].record(s_in)
+        stream.wait_event(ev_in[j])
+        if started[j]:
+            stream.wait_event(ev_out[j])
+        ssd.ssd_chunk_scan_fwd(d_in["x"], d_in["dt"], d_in["A"], d_in["B"], d_in["C"], d_in["D"],
+                               w.chunk, init_states=d_in["init"], y=yy, final_states=ff,
+                               workspace=ws, stream=stream)
+        ev_used[j].record(stream)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_used[j])
+            y_hosts[j].copy_(yy, non_blocking=True)
+            f_hosts[j].copy_(ff, non_blocking=True)
+            ev_out[j].record(s_out)
+        started[j] = True
+
+    for k in range(4):
+        e2e_step(k)
     torch.cuda.synchronize(dev)
     barrier(world)
-    e2e_steps = max(3, args.steps // 4)
+    e2e_steps = max(8, args.steps // 2)
     s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
-    e.record(stream)
+    s.record(s_in)
+    for k in range(e2e_steps):
+        e2e_step(k)
+    s_in.wait_event(ev_out[(e2e_steps - 1) & 1])
+    s_in.wait_event(ev_out[e2e_steps & 1])
+    e.record(s_in)
     torch.cuda.synchronize(dev)
     e2e_ms = max_over_ranks(s.elapsed_time(e), world) / e2e_steps
 
