@@ -34,7 +34,9 @@
 // 32-column block below the diagonal factorised through the block's end (both
 // factors <= 1) and exponentials per element only on the 32 x 32 diagonal
 // blocks.  Output: y = a_i Y + alpha_i ZW + D_h x (a_i = 1 on the exact path);
-// the epilogue reads x for the skip term from global memory, one head ahead.
+// the x rows of the skip term reach the epilogue through TMEM: the warps that
+// scale a head's x rows in shared memory first copy them, unscaled, to one of
+// four TMEM slots.
 //
 // Roles (448 threads):
 //   warps 0-7   prologue: G = C_t B^T (M = 128, N = 128 (t+1), K = dstate) is
@@ -42,7 +44,7 @@
 //               (TMEM, the A operand of Y), the block to its left goes to
 //               shared memory as bf16 (the A operand of G_10 X~); per head:
 //               factors, then the x rows of the tile scaled by b_j (fast path)
-//               or the exact mask written to TMEM (two slots), and for t = 1
+//               or the exact mask written to TMEM (one slot), and for t = 1
 //               x rows 0..127 scaled by beta and h by exp(r), in place;
 //   warps 8-11  epilogue: y staged in shared memory, TMA store;
 //   warp 12     TMA producer (x rows and entering states of the heads, ring of 2);
@@ -80,8 +82,9 @@ struct OutSmem {
     static constexpr int kXTile = Q * 128;                  // x rows [0, Q) of one head
     static constexpr int kX = kBG + kBGBytes;               // x ring: 2 slots
     static constexpr int kYs = kX + 2 * kXTile;             // y staging: 16 KB
-    static constexpr int kDt = kYs + 128 * 128;             // float [kMaxHeads][Q]
-    static constexpr int kCs = kDt + kMaxHeads * Q * 4;     // float [kMaxHeads][Q] prefix sums (log2 units)
+    static constexpr int kDtStride = Q + 2;                 // dt row stride: conflict-free staging stores
+    static constexpr int kDt = kYs + 128 * 128;             // float [kMaxHeads][kDtStride]
+    static constexpr int kCs = kDt + kMaxHeads * kDtStride * 4;   // float [kMaxHeads][Q] prefix sums (log2 units)
     static constexpr int kBeta = kCs + kMaxHeads * Q * 4;   // float [128]  (t = 1 block left of diagonal)
     static constexpr int kBeta2 = kBeta + 128 * 4;          // float [128]  (diagonal block)
     static constexpr int kAl = kBeta2 + 128 * 4;            // float [4][128] alpha_i per factor slot
@@ -106,9 +109,12 @@ enum {
 
 // TMEM columns
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColM = 0;       // bf16 diagonal-block mask, 2 slots of 64 columns (G_10 in the prologue)
+constexpr uint32_t kColM = 0;       // bf16 exact-path mask, 64 columns (fp32 G_10 in the prologue)
 constexpr uint32_t kColG = 128;     // fp32 diagonal block of G, 128 columns (prologue)
 constexpr uint32_t kColGC = 128;    // then: bf16 G o causal, 64 columns
+// unscaled bf16 x rows of the tile for the skip term, 4 slots of 32 columns
+// (head modulo 4) in the columns the mask and G o causal leave free
+__device__ __forceinline__ uint32_t col_xs(int f) { return f < 2 ? 64u + 32u * f : 192u + 32u * (f - 2); }
 constexpr float kFastSpan = 120.f;  // largest tile decay (log2 units) of the fast path
 constexpr uint32_t kColAcc = 256;   // two slots of 128: Y (64) then ZW (64)
 
@@ -145,8 +151,7 @@ template <int Q, int N>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmH,
-                    const __grid_constant__ CUtensorMap tmY,
-                    const __nv_bfloat16* __restrict__ xg, const float* __restrict__ dt,
+                    const __grid_constant__ CUtensorMap tmY, const float* __restrict__ dt,
                     const float* __restrict__ A, const float* __restrict__ Dv, int64_t L, int H,
                     int G, int64_t T, int HG, WaitCtx status) {
     using S = OutSmem<Q, N>;
@@ -280,7 +285,7 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
                 const uint64_t hd = smem_desc_sw128(smem_u32(sH + s * S::kHTile), 16, 1024);
                 // Y = (G o causal) (b * X_t) [fast path] or M X_t [exact path] over the
                 // diagonal block's 128 columns
-                const uint32_t amat = s_path[hi & 3] ? tmem + kColGC : tmem + kColM + 64 * s;
+                const uint32_t amat = s_path[hi & 3] ? tmem + kColGC : tmem + kColM;
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks)
                     mma_ts(acc, amat + ks * 8, xd + (uint64_t)((row0 / 16 + ks) * 128), idesc_y, ks > 0);
@@ -296,7 +301,7 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
                     mma_ss(acc + 64, cd + (uint64_t)((ks >> 2) * 1024 + (ks & 3) * 2),
                            hd + (uint64_t)((ks >> 2) * 512 + (ks & 3) * 2), idesc_z, t == 1 || ks > 0);
                 mma_commit(&bars[BAR_XEMPTY + s]);           // x and h slot s: no reader left
-                mma_commit(&bars[BAR_MEMPTY + s]);
+                mma_commit(&bars[BAR_MEMPTY]);               // the mask slot: no reader left
                 mma_commit(&bars[BAR_ACCFULL + s]);
             }
             if (!ok) s_flag[0] = 1;
@@ -321,7 +326,7 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
 #pragma unroll
             for (int r = 0; r < kPerT; ++r) {
                 const int e = tid + 256 * r, j = e / HG, k = e - j * HG;
-                if (e < HG * KJ) s_dt[k * Q + j] = v[r];
+                if (e < HG * KJ) s_dt[k * S::kDtStride + j] = v[r];
             }
         }
         if (tid < HG) {
@@ -333,7 +338,7 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
         // parallel, while the G MMA runs
         for (int k = warp; k < HG; k += 8) {
             const float Ah = s_Ah[k];
-            const float* dk = s_dt + k * Q;
+            const float* dk = s_dt + k * S::kDtStride;
             float* ck = s_cs + k * Q;
             float carry = 0.f;
             for (int base = 0; base < KJ; base += 32) {
@@ -371,8 +376,8 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
                 fence_proxy_async_smem();          // G_10 is read by the MMA (async proxy)
             }
             // Blocks above the diagonal (column block cb > quarter q) are zero in
-            // every head's mask: write them once, in both M slots -- after every
-            // warp has finished reading G_10 out of the same TMEM columns.
+            // every head's mask: write them once -- after every warp has finished
+            // reading G_10 out of the same TMEM columns.
             tc_fence_before();
             named_bar_sync(1, 256);
             tc_fence_after();
@@ -381,10 +386,7 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
 #pragma unroll
                 for (int u = 0; u < 16; ++u) zeros[u] = 0u;
                 for (int cb = 2 * hf; cb < 2 * hf + 2; ++cb)
-                    if (cb > q) {
-                        tmem_st16(tmem + lane_base + kColM + 16 * cb, zeros);
-                        tmem_st16(tmem + lane_base + kColM + 64 + 16 * cb, zeros);
-                    }
+                    if (cb > q) tmem_st16(tmem + lane_base + kColM + 16 * cb, zeros);
             }
             {
                 // G o causal -> bf16 at kColGC, over the fp32 columns it is made
@@ -413,13 +415,13 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
             if (tid == 0) mbar_arrive(&bars[BAR_GCONV]);
 
             for (int hi = 0; hi < HG; ++hi) {
-                const int s = hi & 1;                 // x/h slot, mask slot, accumulator
-                const int f = hi & 3;                 // factor slot
+                const int s = hi & 1;                 // x/h slot and accumulator
+                const int f = hi & 3;                 // factor slot and skip-term x slot
                 // factor slot f is free once the epilogue of head hi - 4 has read it
                 fail = hi >= 4 && !mbar_wait(&bars[BAR_FEMPTY + f], (uint32_t)(((hi >> 2) - 1) & 1), status);
                 if (named_bar_or(1, 256, fail)) break;
                 const float* cs = s_cs + hi * Q;
-                const float* hdt = s_dt + hi * Q;
+                const float* hdt = s_dt + hi * S::kDtStride;
                 const float cs_i = cs[i];
                 const float r = (t == 1) ? cs[127] : 0.f;
                 // the tile's decay span decides the path (the same for every thread)
@@ -436,10 +438,10 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
                     s_beta2[m] = fast_exp2((fast ? r1 : cs[row0 + (m | 31)]) - cs[j]) * hdt[j];
                 }
                 if (tid == 0) s_path[f] = fast ? 1 : 0;
-                // the exact path writes mask slot s: free once the MMAs of head hi - 2
+                // the exact path writes the mask slot: free once the MMAs of head hi - 1
                 // have completed; both paths need the head's x rows and entering state
-                fail = (!fast && hi >= 2 &&
-                        !mbar_wait(&bars[BAR_MEMPTY + s], (uint32_t)(((hi >> 1) - 1) & 1), status)) ||
+                fail = (!fast && hi >= 1 &&
+                        !mbar_wait(&bars[BAR_MEMPTY], (uint32_t)((hi - 1) & 1), status)) ||
                        !mbar_wait(&bars[BAR_XFULL + s], (uint32_t)((hi >> 1) & 1), status);
                 if (named_bar_or(1, 256, fail)) break;   // also publishes the factors
                 if (tid == 0) mbar_arrive(&bars[BAR_ALFULL + f]);
@@ -449,15 +451,45 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
                     scale_pieces<4>(sX + s * S::kXTile, tid, [&](int k) { return s_beta[k >> 3]; });
                     scale_pieces<S::kHTile / 4096>(sH + s * S::kHTile, tid, [&](int) { return er; });
                 }
-                if (fast) {
-                    // the tile's x rows *= b_j, in place (the MMA's B operand)
-                    scale_pieces<4>(sX + s * S::kXTile + row0 * 128, tid, [&](int k) { return s_beta2[k >> 3]; });
+                {
+                    // The tile's x rows: warp (q, hf) takes row m, 16-byte chunks
+                    // 4 hf .. 4 hf + 3 (stored at chunk ^ (m & 7)).  Unscaled, they go to
+                    // TMEM slot f (columns = element / 2) for the epilogue's skip term;
+                    // on the fast path they are then scaled by b_m in place (the MMA's
+                    // B operand).
+                    uint4* xrow = reinterpret_cast<uint4*>(sX + s * S::kXTile + (row0 + m) * 128);
+                    uint4 v[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) v[u] = xrow[(4 * hf + u) ^ (m & 7)];
+                    {
+                        uint32_t w[16];
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            w[4 * u + 0] = v[u].x; w[4 * u + 1] = v[u].y;
+                            w[4 * u + 2] = v[u].z; w[4 * u + 3] = v[u].w;
+                        }
+                        tc_fence_after();          // slot f's previous reader (head hi - 4) is done
+                        tmem_st16(tmem + lane_base + col_xs(f) + 16 * hf, w);
+                    }
+                    if (fast) {
+                        const float bm = s_beta2[m];
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            uint32_t* e4 = reinterpret_cast<uint32_t*>(&v[u]);
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const float2 xf = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&e4[e]));
+                                e4[e] = pack_bf16x2(xf.x * bm, xf.y * bm);
+                            }
+                            xrow[(4 * hf + u) ^ (m & 7)] = v[u];
+                        }
+                    }
                 }
                 fence_proxy_async_smem();
                 tc_fence_after();
 
-                // exact path: diagonal-block mask -> TMEM slot s (64 columns of bf16
-                // pairs), from the bf16 G o causal
+                // exact path: diagonal-block mask -> the TMEM mask slot (64 columns of
+                // bf16 pairs), from the bf16 G o causal
                 for (int cb = 2 * hf; cb < 2 * hf + 2 && !fast; ++cb) {
                     const int j0 = row0 + 32 * cb;
                     uint32_t packed[16];
@@ -499,7 +531,7 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
                             }
                         }
                     }
-                    tmem_st16(tmem + lane_base + kColM + 64 * s + 16 * cb, packed);
+                    tmem_st16(tmem + lane_base + kColM + 16 * cb, packed);
                 }
                 tc_fence_before();
                 named_bar_sync(1, 256);
@@ -512,19 +544,8 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
         // y rows go to a 128-byte-swizzled staging tile and leave by TMA store
         // (coalesced; rows past the sequence end are clipped by the tensor map).
         const int m = tid - 256;
-        const int i = row0 + m;
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
         bool fail = false;
-        // x row i of the next head (the D x term), loaded one head ahead from
-        // global memory (the tile's x rows in shared memory are scaled)
-        const bool row_in = t0 + i < L;
-        const uint4* xsrc = reinterpret_cast<const uint4*>(xg + ((b * L + t0 + i) * H + head0) * 64);
-        uint4 xr[8];
-        auto load_x_row = [&](int hh) {
-#pragma unroll
-            for (int u = 0; u < 8; ++u) xr[u] = row_in ? __ldg(xsrc + hh * 8 + u) : make_uint4(0, 0, 0, 0);
-        };
-        load_x_row(0);
         for (int hi = 0; hi < HG; ++hi) {
             const int s = hi & 1;
             fail = !(mbar_wait(&bars[BAR_ACCFULL + s], (uint32_t)((hi >> 1) & 1), status) &&
@@ -538,20 +559,20 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
             const float Dh = s_Dh[hi];
             uint4* ystage = reinterpret_cast<uint4*>(sY + m * 128);
             const uint32_t acc = tmem + lane_base + kColAcc + 128 * s;
+            const uint32_t xs = tmem + lane_base + col_xs(hi & 3);   // unscaled x row
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                uint32_t yr[32], zr[32];
-                tmem_ld32x2(acc + half * 32, acc + 64 + half * 32, yr, zr);
+            for (int qq = 0; qq < 4; ++qq) {
+                // columns 16 qq .. 16 qq + 15 of Y and ZW, x elements 16 qq .. 16 qq + 15
+                uint32_t yr[16], zr[16], xw[8];
+                tmem_ld16x2_8(acc + 16 * qq, acc + 64 + 16 * qq, xs + 8 * qq, yr, zr, xw);
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int lc = half * 4 + u;   // logical 16-byte chunk of the row
-                    const uint4 xv = xr[lc];
-                    const uint32_t* xu = reinterpret_cast<const uint32_t*>(&xv);
+                for (int u = 0; u < 2; ++u) {
+                    const int lc = 2 * qq + u;     // logical 16-byte chunk of the row
                     uint32_t o[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const float2 xf =
-                            __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xu[e]));
+                            __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xw[4 * u + e]));
                         const int k = 8 * u + 2 * e;
                         const float v0 =
                             fmaf(al, __uint_as_float(zr[k]), ar * __uint_as_float(yr[k])) + Dh * xf.x;
@@ -571,7 +592,6 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
                 mbar_arrive(&bars[BAR_ACCEMPTY + s]);
                 mbar_arrive(&bars[BAR_FEMPTY + (hi & 3)]);
             }
-            if (hi + 1 < HG) load_x_row(hi + 1);
         }
         if (m == 0) bulk_wait_group<0>();      // stores done before the CTA leaves
         if (fail) s_flag[0] = 1;
@@ -638,7 +658,7 @@ cudaError_t launch_impl(const void* x, const float* dt, const float* A, const vo
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)(d.b * d.T * (Q / 128)), (unsigned)(d.H / HG));
     chunk_out_tc_kernel<Q, N><<<grid, kThreads, S::kAlloc, s>>>(
-        tmX, tmB, tmC, tmH, tmY, static_cast<const __nv_bfloat16*>(x), dt, A, D, d.L, (int)d.H,
+        tmX, tmB, tmC, tmH, tmY, dt, A, D, d.L, (int)d.H,
         (int)d.G, d.T, HG, status);
     return cudaGetLastError();
 }

@@ -300,6 +300,28 @@ __device__ __forceinline__ void tmem_ld32x2(uint32_t ta, uint32_t tb, uint32_t (
         : "r"(ta), "r"(tb)
         : "memory");
 }
+// Three warp-collective TMEM loads (16, 16 and 8 columns, from three
+// addresses) under a single wait.
+__device__ __forceinline__ void tmem_ld16x2_8(uint32_t ta, uint32_t tb, uint32_t tc,
+                                              uint32_t (&ra)[16], uint32_t (&rb)[16],
+                                              uint32_t (&rc)[8]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%40];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%41];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%32,%33,%34,%35,%36,%37,%38,%39}, [%42];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(ra[0]), "=r"(ra[1]), "=r"(ra[2]), "=r"(ra[3]), "=r"(ra[4]), "=r"(ra[5]),
+          "=r"(ra[6]), "=r"(ra[7]), "=r"(ra[8]), "=r"(ra[9]), "=r"(ra[10]), "=r"(ra[11]),
+          "=r"(ra[12]), "=r"(ra[13]), "=r"(ra[14]), "=r"(ra[15]), "=r"(rb[0]), "=r"(rb[1]),
+          "=r"(rb[2]), "=r"(rb[3]), "=r"(rb[4]), "=r"(rb[5]), "=r"(rb[6]), "=r"(rb[7]),
+          "=r"(rb[8]), "=r"(rb[9]), "=r"(rb[10]), "=r"(rb[11]), "=r"(rb[12]), "=r"(rb[13]),
+          "=r"(rb[14]), "=r"(rb[15]), "=r"(rc[0]), "=r"(rc[1]), "=r"(rc[2]), "=r"(rc[3]),
+          "=r"(rc[4]), "=r"(rc[5]), "=r"(rc[6]), "=r"(rc[7])
+        : "r"(ta), "r"(tb), "r"(tc)
+        : "memory");
+}
 // Warp-collective TMEM store of 32 lanes x 16 consecutive 32-bit columns,
 // followed by its wait (the registers are free and the data is in TMEM when
 // this returns).
