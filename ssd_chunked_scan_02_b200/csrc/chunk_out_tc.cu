@@ -76,11 +76,11 @@ struct OutSmem {
     static constexpr int kCBytes = kNB * 128 * 128;
     static constexpr int kBG = kC + kCBytes;                // B tile (prologue), then G_10 + h ring
     static constexpr int kG10Off = 0;                       // bf16 G_10, K-major SW128, 2 x 16 KB (t = 1)
-    static constexpr int kHOff = (Q == 256) ? 32768 : 0;    // h ring: 2 slots
+    static constexpr int kHOff = (Q == 256) ? 32768 : 0;    // h ring of a t = 1 tile: 2 slots after G_10
     static constexpr int kBBytes = kNB * Q * 128;
     static constexpr int kBGBytes = (kBBytes > kHOff + 2 * kHTile) ? kBBytes : kHOff + 2 * kHTile;
     static constexpr int kXTile = Q * 128;                  // x rows [0, Q) of one head
-    static constexpr int kX = kBG + kBGBytes;               // x ring: 2 slots
+    static constexpr int kX = kBG + kBGBytes;               // x ring: 2 slots of Q rows (or 4 of 128)
     static constexpr int kYs = kX + 2 * kXTile;             // y staging: 16 KB
     static constexpr int kDtStride = Q + 2;                 // dt row stride: conflict-free staging stores
     static constexpr int kDt = kYs + 128 * 128;             // float [kMaxHeads][kDtStride]
@@ -100,11 +100,15 @@ struct OutSmem {
 
 // mbarrier indices
 enum {
-    BAR_BC = 0, BAR_G = 1, BAR_GCONV = 2, BAR_XFULL = 3, BAR_XEMPTY = 5, BAR_MFULL = 7,
-    BAR_MEMPTY = 9, BAR_ACCFULL = 11, BAR_ACCEMPTY = 13,
-    BAR_ALFULL = 15,    // four factor slots (alpha_i, a_i, path) per head modulo 4
-    BAR_FEMPTY = 19,    // four: the epilogue has read the factor slot
-    BAR_COUNT = 23
+    BAR_BC = 0, BAR_G = 1, BAR_GCONV = 2,
+    BAR_XFULL = 3,      // up to four x/h ring slots
+    BAR_XEMPTY = 7,
+    BAR_MFULL = 11,     // four: the head's operands are ready (head modulo 4)
+    BAR_MEMPTY = 15,    // the exact-path mask slot
+    BAR_ACCFULL = 16, BAR_ACCEMPTY = 18,
+    BAR_ALFULL = 20,    // four factor slots (alpha_i, a_i, path) per head modulo 4
+    BAR_FEMPTY = 24,    // four: the epilogue has read the factor slot
+    BAR_COUNT = 28
 };
 
 // TMEM columns
@@ -168,13 +172,17 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
     const int g = head0 / (H / G);
     const int KJ = 128 * (t + 1);               // columns j this tile needs
     const int row0 = 128 * t;                   // first row of the tile within the chunk
+    // x/h ring: a tile-0 CTA of a 256-token chunk needs only 128 x rows and no
+    // G_10, so its ring has four slots in the same space; otherwise two
+    const int R = (Q == 256 && t == 0) ? 4 : 2;
+    const int kXSlot = KJ * 128;                // bytes of one slot's x rows
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
     uint8_t* sC = smem + S::kC;
     uint8_t* sB = smem + S::kBG;
     uint8_t* sG10 = smem + S::kBG + S::kG10Off;
-    uint8_t* sH = smem + S::kBG + S::kHOff;
+    uint8_t* sH = smem + S::kBG + (t == 1 ? S::kHOff : 0);
     uint8_t* sX = smem + S::kX;
     uint8_t* sY = smem + S::kYs;
     float* s_dt = reinterpret_cast<float*>(smem + S::kDt);
@@ -221,29 +229,29 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
                                 g, (int)(t0 + rb * 128), (int)b);
             }
             auto load_x = [&](int hi) {
-                const int s = hi & 1;
-                mbar_expect_tx(&bars[BAR_XFULL + s], (uint32_t)(KJ * 128 + S::kHTile));
+                const int s = hi & (R - 1);
+                mbar_expect_tx(&bars[BAR_XFULL + s], (uint32_t)(kXSlot + S::kHTile));
                 for (int rb = 0; rb <= t; ++rb)
-                    tma_load_4d(sX + s * S::kXTile + rb * 128 * 128, &tmX, &bars[BAR_XFULL + s], 0,
+                    tma_load_4d(sX + s * kXSlot + rb * 128 * 128, &tmX, &bars[BAR_XFULL + s], 0,
                                 head0 + hi, (int)(t0 + rb * 128), (int)b);
             };
             auto load_h = [&](int hi) {
-                const int s = hi & 1;
+                const int s = hi & (R - 1);
                 const int hrow = (int)(((b * T + c) * H + head0 + hi) * 64);
                 for (int nb = 0; nb < S::kNB; ++nb)
                     tma_load_2d(sH + s * S::kHTile + nb * 64 * 128, &tmH, &bars[BAR_XFULL + s],
                                 nb * 64, hrow);
             };
-            const int first = HG < 2 ? HG : 2;
+            const int first = HG < R ? HG : R;
             for (int hi = 0; hi < first; ++hi) load_x(hi);
             // The h ring (and G_10) reuse the B tile's space: wait until G is
             // computed and copied out of TMEM.
             bool ok = mbar_wait(&bars[BAR_GCONV], 0, status);
             if (ok) {
                 for (int hi = 0; hi < first; ++hi) load_h(hi);
-                for (int hi = 2; hi < HG && ok; ++hi) {
-                    const int s = hi & 1;
-                    ok = mbar_wait(&bars[BAR_XEMPTY + s], (uint32_t)(((hi >> 1) - 1) & 1), status);
+                for (int hi = R; hi < HG && ok; ++hi) {
+                    const int s = hi & (R - 1);
+                    ok = mbar_wait(&bars[BAR_XEMPTY + s], (uint32_t)((hi / R - 1) & 1), status);
                     if (ok) { load_x(hi); load_h(hi); }
                 }
             }
@@ -271,17 +279,18 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
             const uint64_t gd = smem_desc_sw128(smem_u32(sG10), 16, 1024);
             const uint64_t cd = smem_desc_sw128(smem_u32(sC), 16, 1024);
             for (int hi = 0; hi < HG && ok; ++hi) {
-                const int s = hi & 1;
-                ok = mbar_wait(&bars[BAR_MFULL + s], (uint32_t)((hi >> 1) & 1), status) &&
-                     mbar_wait(&bars[BAR_XFULL + s], (uint32_t)((hi >> 1) & 1), status) &&
-                     (hi < 2 || mbar_wait(&bars[BAR_ACCEMPTY + s], (uint32_t)(((hi >> 1) - 1) & 1),
+                const int s = hi & (R - 1);           // x/h ring slot
+                const int a = hi & 1;                 // accumulator slot
+                ok = mbar_wait(&bars[BAR_MFULL + (hi & 3)], (uint32_t)((hi >> 2) & 1), status) &&
+                     mbar_wait(&bars[BAR_XFULL + s], (uint32_t)((hi / R) & 1), status) &&
+                     (hi < 2 || mbar_wait(&bars[BAR_ACCEMPTY + a], (uint32_t)(((hi >> 1) - 1) & 1),
                                           status));
                 if (!ok) break;
                 tc_fence_after();
-                const uint32_t acc = tmem + kColAcc + 128 * s;
+                const uint32_t acc = tmem + kColAcc + 128 * a;
                 // descriptors of each operand's first K step; a K step moves the start
                 // address (16-byte units, low bits of the descriptor) by a constant
-                const uint64_t xd = smem_desc_sw128(smem_u32(sX + s * S::kXTile), 16, 1024);
+                const uint64_t xd = smem_desc_sw128(smem_u32(sX + s * kXSlot), 16, 1024);
                 const uint64_t hd = smem_desc_sw128(smem_u32(sH + s * S::kHTile), 16, 1024);
                 // Y = (G o causal) (b * X_t) [fast path] or M X_t [exact path] over the
                 // diagonal block's 128 columns
@@ -302,7 +311,7 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
                            hd + (uint64_t)((ks >> 2) * 512 + (ks & 3) * 2), idesc_z, t == 1 || ks > 0);
                 mma_commit(&bars[BAR_XEMPTY + s]);           // x and h slot s: no reader left
                 mma_commit(&bars[BAR_MEMPTY]);               // the mask slot: no reader left
-                mma_commit(&bars[BAR_ACCFULL + s]);
+                mma_commit(&bars[BAR_ACCFULL + a]);
             }
             if (!ok) s_flag[0] = 1;
         }
@@ -415,7 +424,7 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
             if (tid == 0) mbar_arrive(&bars[BAR_GCONV]);
 
             for (int hi = 0; hi < HG; ++hi) {
-                const int s = hi & 1;                 // x/h slot and accumulator
+                const int s = hi & (R - 1);           // x/h ring slot
                 const int f = hi & 3;                 // factor slot and skip-term x slot
                 // factor slot f is free once the epilogue of head hi - 4 has read it
                 fail = hi >= 4 && !mbar_wait(&bars[BAR_FEMPTY + f], (uint32_t)(((hi >> 2) - 1) & 1), status);
@@ -442,13 +451,13 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
                 // have completed; both paths need the head's x rows and entering state
                 fail = (!fast && hi >= 1 &&
                         !mbar_wait(&bars[BAR_MEMPTY], (uint32_t)((hi - 1) & 1), status)) ||
-                       !mbar_wait(&bars[BAR_XFULL + s], (uint32_t)((hi >> 1) & 1), status);
+                       !mbar_wait(&bars[BAR_XFULL + s], (uint32_t)((hi / R) & 1), status);
                 if (named_bar_or(1, 256, fail)) break;   // also publishes the factors
                 if (tid == 0) mbar_arrive(&bars[BAR_ALFULL + f]);
                 if (t == 1) {
                     // x rows 0..127 *= beta_j (row j = piece / 8), h *= exp(r), in place
                     const float er = fast_exp2(r);
-                    scale_pieces<4>(sX + s * S::kXTile, tid, [&](int k) { return s_beta[k >> 3]; });
+                    scale_pieces<4>(sX + s * kXSlot, tid, [&](int k) { return s_beta[k >> 3]; });
                     scale_pieces<S::kHTile / 4096>(sH + s * S::kHTile, tid, [&](int) { return er; });
                 }
                 {
@@ -457,7 +466,7 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
                     // TMEM slot f (columns = element / 2) for the epilogue's skip term;
                     // on the fast path they are then scaled by b_m in place (the MMA's
                     // B operand).
-                    uint4* xrow = reinterpret_cast<uint4*>(sX + s * S::kXTile + (row0 + m) * 128);
+                    uint4* xrow = reinterpret_cast<uint4*>(sX + s * kXSlot + (row0 + m) * 128);
                     uint4 v[4];
 #pragma unroll
                     for (int u = 0; u < 4; ++u) v[u] = xrow[(4 * hf + u) ^ (m & 7)];
@@ -535,7 +544,7 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
                 }
                 tc_fence_before();
                 named_bar_sync(1, 256);
-                if (tid == 0) mbar_arrive(&bars[BAR_MFULL + s]);
+                if (tid == 0) mbar_arrive(&bars[BAR_MFULL + f]);
             }
         }
         if (fail) s_flag[0] = 1;
@@ -603,10 +612,8 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
         // A wait gave up somewhere: before the CTA's shared memory and TMEM
         // go away, give outstanding TMA loads and MMAs a last (bounded) chance
         // to land.  Waiting on already-completed phases returns at once.
-        for (int k = 0; k < 2; ++k) {
-            mbar_wait(&bars[BAR_XFULL + k], 0, status);
-            mbar_wait(&bars[BAR_ACCFULL + k], 0, status);
-        }
+        for (int k = 0; k < R && k < HG; ++k) mbar_wait(&bars[BAR_XFULL + k], 0, status);
+        for (int k = 0; k < 2 && k < HG; ++k) mbar_wait(&bars[BAR_ACCFULL + k], 0, status);
         mbar_wait(&bars[BAR_BC], 0, status);
         mbar_wait(&bars[BAR_G], 0, status);
     }
