@@ -13,24 +13,27 @@
 // One CTA per (batch, chunk, 128-row tile t of the chunk, group of HG heads
 // sharing B and C).  Tile t holds rows i in [128 t, 128 t + 128).
 //
-// The decay between row i and column j < i factorises through any boundary r
-// with cs_j >= r >= cs_i: exp(cs_i - cs_j) = exp(cs_i - r) exp(r - cs_j), both
-// factors <= 1.  With r = cs_{127} for the block left of the diagonal (t = 1):
-//   sum_{j < 128} G_ij exp(cs_i - cs_j) dt_j x_j
-//      = alpha_i sum_j G_ij (beta_j x_j),   alpha_i = exp(cs_i - r), beta_j = exp(r - cs_j) dt_j
-// and the entering state term exp(cs_i) C_i h = alpha_i C_i (exp(r) h).  Both go
-// into one accumulator ZW = G_10 (beta x_{0..127}) + C_t (exp(r) h)^T, scaled
-// by alpha_i in the epilogue (for t = 0, r = 0: ZW = C_0 h^T, alpha_i = exp(cs_i)).
-// The diagonal 128 x 128 block, Y_i = sum_{j <= i} G_ij exp(cs_i - cs_j) dt_j x_j,
-// factorises through one boundary r for the whole tile: with
-//   a_i = 2^(cs_i - r),  b_j = 2^(r - cs_j) dt_j   (cs in log2 units),
+// The decay between row i and column j < i factorises through any boundary r:
+// exp(cs_i - cs_j) = exp(cs_i - r) exp(r - cs_j).  The diagonal 128 x 128
+// block, Y_i = sum_{j <= i} G_ij exp(cs_i - cs_j) dt_j x_j, factorises through
+// one boundary r1 for the whole tile: with
+//   a_i = 2^(cs_i - r1),  b_j = 2^(r1 - cs_j) dt_j   (cs in log2 units),
 //   Y = diag(a) (G o causal) (b * X_t),
 // so the bf16 operand G o causal is built once per CTA and shared by all its
 // heads; a head only scales its x rows by b_j (in place) and its output rows
-// by a_i.  With r the midpoint of the tile's prefix sums, the factors stay in
+// by a_i.  With r1 the midpoint of the tile's prefix sums, the factors stay in
 // [2^-60, 2^60] whenever the tile's decay spans at most 120 (log2 units): the
-// fast path.  A head whose tile decays faster takes the exact path instead: a
-// per-element mask M_ij = G_ij exp(cs_i - cs_j) dt_j (j <= i) in TMEM, with each
+// fast path.  There the block left of the diagonal (t = 1) uses the same
+// boundary, since cs_j >= r1 makes b_j <= dt_j for j < 128: G_10 (b * X_0)
+// accumulates into Y, and the entering state term exp(cs_i) C_i h goes into a
+// second accumulator ZW = C_t h^T scaled by alpha_i = exp(cs_i) <= 1.
+// A head whose tile decays faster takes the exact path instead.  Its left
+// block factorises through r = cs_{127} (both factors <= 1):
+//   sum_{j < 128} G_ij exp(cs_i - cs_j) dt_j x_j
+//      = alpha_i sum_j G_ij (beta_j x_j),   alpha_i = exp(cs_i - r), beta_j = exp(r - cs_j) dt_j,
+// and with the entering state term alpha_i C_i (exp(r) h) it forms ZW =
+// G_10 (beta x_{0..127}) + C_t (exp(r) h)^T (r = 0 for t = 0); its diagonal
+// block is a per-element mask M_ij = G_ij exp(cs_i - cs_j) dt_j (j <= i) in TMEM, with each
 // 32-column block below the diagonal factorised through the block's end (both
 // factors <= 1) and exponentials per element only on the 32 x 32 diagonal
 // blocks.  Output: y = a_i Y + alpha_i ZW + D_h x (a_i = 1 on the exact path);
@@ -45,7 +48,8 @@
 //               shared memory as bf16 (the A operand of G_10 X~); per head:
 //               factors, then the x rows of the tile scaled by b_j (fast path)
 //               or the exact mask written to TMEM (one slot), and for t = 1
-//               x rows 0..127 scaled by beta and h by exp(r), in place;
+//               x rows 0..127 scaled by b_j (fast) or beta_j and h by exp(r)
+//               (exact), in place;
 //   warps 8-11  epilogue: y staged in shared memory, TMA store;
 //   warp 12     TMA producer (x rows and entering states of the heads, ring of 2);
 //   warp 13     MMA issuer and TMEM owner.
@@ -294,21 +298,26 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
                 const uint64_t hd = smem_desc_sw128(smem_u32(sH + s * S::kHTile), 16, 1024);
                 // Y = (G o causal) (b * X_t) [fast path] or M X_t [exact path] over the
                 // diagonal block's 128 columns
-                const uint32_t amat = s_path[hi & 3] ? tmem + kColGC : tmem + kColM;
+                const bool fast = s_path[hi & 3] != 0;
+                const uint32_t amat = fast ? tmem + kColGC : tmem + kColM;
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks)
                     mma_ts(acc, amat + ks * 8, xd + (uint64_t)((row0 / 16 + ks) * 128), idesc_y, ks > 0);
-                // ZW = G_10 (beta x_{0..127}) [t = 1] + C_t (exp(r) h)^T
+                // t = 1: G_10 times x rows 0..127, scaled by b_j like the diagonal
+                // block's (fast path: into Y) or by beta_j (exact path: into ZW)
+                const uint32_t wacc = fast ? acc : acc + 64;
                 if (t == 1) {
 #pragma unroll
                     for (int ks = 0; ks < 8; ++ks)
-                        mma_ss(acc + 64, gd + (uint64_t)((ks >> 2) * 1024 + (ks & 3) * 2),
-                               xd + (uint64_t)(ks * 128), idesc_w, ks > 0);
+                        mma_ss(wacc, gd + (uint64_t)((ks >> 2) * 1024 + (ks & 3) * 2),
+                               xd + (uint64_t)(ks * 128), idesc_w, fast || ks > 0);
                 }
+                // ZW (+)= C_t h~^T: h unscaled on the fast path, h exp(r) on the exact one
+                const bool zacc = t == 1 && !fast;
 #pragma unroll
                 for (int ks = 0; ks < N / 16; ++ks)
                     mma_ss(acc + 64, cd + (uint64_t)((ks >> 2) * 1024 + (ks & 3) * 2),
-                           hd + (uint64_t)((ks >> 2) * 512 + (ks & 3) * 2), idesc_z, t == 1 || ks > 0);
+                           hd + (uint64_t)((ks >> 2) * 512 + (ks & 3) * 2), idesc_z, zacc || ks > 0);
                 mma_commit(&bars[BAR_XEMPTY + s]);           // x and h slot s: no reader left
                 mma_commit(&bars[BAR_MEMPTY]);               // the mask slot: no reader left
                 mma_commit(&bars[BAR_ACCFULL + a]);
@@ -438,8 +447,8 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
                 const bool fast = fabsf(c_last - c_first) <= kFastSpan;
                 const float r1 = 0.5f * (c_first + c_last);
                 if (hf == 0) {
-                    if (t == 1) s_beta[m] = fast_exp2(r - cs[m]) * hdt[m];
-                    s_al[f * 128 + m] = fast_exp2(cs_i - r);
+                    if (t == 1) s_beta[m] = fast_exp2((fast ? r1 : r) - cs[m]) * hdt[m];
+                    s_al[f * 128 + m] = fast_exp2(fast ? cs_i : cs_i - r);
                     s_row[f * 128 + m] = fast ? fast_exp2(cs_i - r1) : 1.f;
                 } else {
                     // fast: b_j; exact: beta of j through the end of its 32-column block
@@ -455,10 +464,13 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
                 if (named_bar_or(1, 256, fail)) break;   // also publishes the factors
                 if (tid == 0) mbar_arrive(&bars[BAR_ALFULL + f]);
                 if (t == 1) {
-                    // x rows 0..127 *= beta_j (row j = piece / 8), h *= exp(r), in place
-                    const float er = fast_exp2(r);
+                    // x rows 0..127 *= b_j (fast path) or beta_j (exact path), row j =
+                    // piece / 8; on the exact path also h *= exp(r); in place
                     scale_pieces<4>(sX + s * kXSlot, tid, [&](int k) { return s_beta[k >> 3]; });
-                    scale_pieces<S::kHTile / 4096>(sH + s * S::kHTile, tid, [&](int) { return er; });
+                    if (!fast) {
+                        const float er = fast_exp2(r);
+                        scale_pieces<S::kHTile / 4096>(sH + s * S::kHTile, tid, [&](int) { return er; });
+                    }
                 }
                 {
                     // The tile's x rows: warp (q, hf) takes row m, 16-byte chunks
