@@ -69,7 +69,7 @@ namespace {
 using namespace sm100;
 
 constexpr int kThreads = 448;
-constexpr int kMaxHeads = 16;
+constexpr int kMaxHeads = 32;
 constexpr float kLog2e = 1.4426950408889634f;
 
 template <int Q, int N>
@@ -88,8 +88,9 @@ struct OutSmem {
     static constexpr int kYs = kX + 2 * kXTile;             // y staging: 16 KB
     static constexpr int kDtStride = Q + 2;                 // dt row stride: conflict-free staging stores
     static constexpr int kDt = kYs + 128 * 128;             // float [kMaxHeads][kDtStride]
-    static constexpr int kCs = kDt + kMaxHeads * kDtStride * 4;   // float [kMaxHeads][Q] prefix sums (log2 units)
-    static constexpr int kBeta = kCs + kMaxHeads * Q * 4;   // float [128]  (t = 1 block left of diagonal)
+    static constexpr int kCs = kDt + kMaxHeads * kDtStride * 4;   // float [Q] one head's prefix sums (log2 units)
+    static constexpr int kWs = kCs + Q * 4;                 // float [16]: per-warp sums of the scan
+    static constexpr int kBeta = kWs + 16 * 4;              // float [128]  (t = 1 block left of diagonal)
     static constexpr int kBeta2 = kBeta + 128 * 4;          // float [128]  (diagonal block)
     static constexpr int kAl = kBeta2 + 128 * 4;            // float [4][128] alpha_i per factor slot
     static constexpr int kRow = kAl + 4 * 128 * 4;          // float [4][128] a_i (1: exact path)
@@ -191,6 +192,7 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
     uint8_t* sY = smem + S::kYs;
     float* s_dt = reinterpret_cast<float*>(smem + S::kDt);
     float* s_cs = reinterpret_cast<float*>(smem + S::kCs);
+    float* s_ws = reinterpret_cast<float*>(smem + S::kWs);
     float* s_beta = reinterpret_cast<float*>(smem + S::kBeta);
     float* s_beta2 = reinterpret_cast<float*>(smem + S::kBeta2);
     float* s_al = reinterpret_cast<float*>(smem + S::kAl);
@@ -352,25 +354,6 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
             s_Dh[tid] = Dv[head0 + tid];
         }
         named_bar_sync(1, 256);
-        // inclusive prefix sums of dt*A (log2 units) for every head, 8 warps in
-        // parallel, while the G MMA runs
-        for (int k = warp; k < HG; k += 8) {
-            const float Ah = s_Ah[k];
-            const float* dk = s_dt + k * S::kDtStride;
-            float* ck = s_cs + k * Q;
-            float carry = 0.f;
-            for (int base = 0; base < KJ; base += 32) {
-                float v = dk[base + lane] * Ah;
-#pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const float u = __shfl_up_sync(0xffffffffu, v, o);
-                    if (lane >= o) v += u;
-                }
-                v += carry;
-                ck[base + lane] = v;
-                carry = __shfl_sync(0xffffffffu, v, 31);
-            }
-        }
         bool fail = !mbar_wait(&bars[BAR_G], 0, status);
         if (!named_bar_or(1, 256, fail)) {
             tc_fence_after();
@@ -438,7 +421,23 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
                 // factor slot f is free once the epilogue of head hi - 4 has read it
                 fail = hi >= 4 && !mbar_wait(&bars[BAR_FEMPTY + f], (uint32_t)(((hi >> 2) - 1) & 1), status);
                 if (named_bar_or(1, 256, fail)) break;
-                const float* cs = s_cs + hi * Q;
+                {
+                    // inclusive prefix sums of dt*A (log2 units) of this head over the
+                    // tile's KJ columns: a shuffle scan per warp, then the warp offsets
+                    float v = (tid < KJ) ? s_dt[hi * S::kDtStride + tid] * s_Ah[hi] : 0.f;
+#pragma unroll
+                    for (int o = 1; o < 32; o <<= 1) {
+                        const float u = __shfl_up_sync(0xffffffffu, v, o);
+                        if (lane >= o) v += u;
+                    }
+                    if (lane == 31) s_ws[warp] = v;
+                    named_bar_sync(1, 256);
+                    float off = 0.f;
+                    for (int w2 = 0; w2 < warp; ++w2) off += s_ws[w2];
+                    if (tid < KJ) s_cs[tid] = v + off;
+                    named_bar_sync(1, 256);
+                }
+                const float* cs = s_cs;
                 const float* hdt = s_dt + hi * S::kDtStride;
                 const float cs_i = cs[i];
                 const float r = (t == 1) ? cs[127] : 0.f;
