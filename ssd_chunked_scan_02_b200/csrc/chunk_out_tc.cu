@@ -287,7 +287,8 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
             for (int hi = 0; hi < HG && ok; ++hi) {
                 const int s = hi & (R - 1);           // x/h ring slot
                 const int a = hi & 1;                 // accumulator slot
-                ok = mbar_wait(&bars[BAR_MFULL + (hi & 3)], (uint32_t)((hi >> 2) & 1), status) &&
+                const int f = hi & 3;                 // factor slot (path of the head)
+                ok = mbar_wait(&bars[BAR_ALFULL + f], (uint32_t)((hi >> 2) & 1), status) &&
                      mbar_wait(&bars[BAR_XFULL + s], (uint32_t)((hi / R) & 1), status) &&
                      (hi < 2 || mbar_wait(&bars[BAR_ACCEMPTY + a], (uint32_t)(((hi >> 1) - 1) & 1),
                                           status));
@@ -298,9 +299,22 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
                 // address (16-byte units, low bits of the descriptor) by a constant
                 const uint64_t xd = smem_desc_sw128(smem_u32(sX + s * kXSlot), 16, 1024);
                 const uint64_t hd = smem_desc_sw128(smem_u32(sH + s * S::kHTile), 16, 1024);
+                const bool fast = s_path[f] != 0;
+                // ZW (+)= C_t h~^T.  On the fast path h is used as loaded, so these
+                // MMAs go first, while the head's x rows are still being scaled; on
+                // the exact path h exp(r) is ready only with the rest.
+                auto issue_z = [&](bool acc_first) {
+#pragma unroll
+                    for (int ks = 0; ks < N / 16; ++ks)
+                        mma_ss(acc + 64, cd + (uint64_t)((ks >> 2) * 1024 + (ks & 3) * 2),
+                               hd + (uint64_t)((ks >> 2) * 512 + (ks & 3) * 2), idesc_z, acc_first || ks > 0);
+                };
+                if (fast) issue_z(false);
+                ok = mbar_wait(&bars[BAR_MFULL + f], (uint32_t)((hi >> 2) & 1), status);
+                if (!ok) break;
+                tc_fence_after();
                 // Y = (G o causal) (b * X_t) [fast path] or M X_t [exact path] over the
                 // diagonal block's 128 columns
-                const bool fast = s_path[hi & 3] != 0;
                 const uint32_t amat = fast ? tmem + kColGC : tmem + kColM;
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks)
@@ -314,12 +328,7 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
                         mma_ss(wacc, gd + (uint64_t)((ks >> 2) * 1024 + (ks & 3) * 2),
                                xd + (uint64_t)(ks * 128), idesc_w, fast || ks > 0);
                 }
-                // ZW (+)= C_t h~^T: h unscaled on the fast path, h exp(r) on the exact one
-                const bool zacc = t == 1 && !fast;
-#pragma unroll
-                for (int ks = 0; ks < N / 16; ++ks)
-                    mma_ss(acc + 64, cd + (uint64_t)((ks >> 2) * 1024 + (ks & 3) * 2),
-                           hd + (uint64_t)((ks >> 2) * 512 + (ks & 3) * 2), idesc_z, zacc || ks > 0);
+                if (!fast) issue_z(t == 1);
                 mma_commit(&bars[BAR_XEMPTY + s]);           // x and h slot s: no reader left
                 mma_commit(&bars[BAR_MEMPTY]);               // the mask slot: no reader left
                 mma_commit(&bars[BAR_ACCFULL + a]);
