@@ -428,8 +428,6 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
                 const int s = hi & (R - 1);           // x/h ring slot
                 const int f = hi & 3;                 // factor slot and skip-term x slot
                 // factor slot f is free once the epilogue of head hi - 4 has read it
-                fail = hi >= 4 && !mbar_wait(&bars[BAR_FEMPTY + f], (uint32_t)(((hi >> 2) - 1) & 1), status);
-                if (named_bar_or(1, 256, fail)) break;
                 {
                     // inclusive prefix sums of dt*A (log2 units) of this head over the
                     // tile's KJ columns: a shuffle scan per warp, then the warp offsets
@@ -440,7 +438,10 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
                         if (lane >= o) v += u;
                     }
                     if (lane == 31) s_ws[warp] = v;
-                    named_bar_sync(1, 256);
+                    // (the barrier that publishes the warp sums also shares the verdict
+                    // of the factor slot's wait)
+                    fail = hi >= 4 && !mbar_wait(&bars[BAR_FEMPTY + f], (uint32_t)(((hi >> 2) - 1) & 1), status);
+                    if (named_bar_or(1, 256, fail)) break;
                     float off = 0.f;
                     for (int w2 = 0; w2 < warp; ++w2) off += s_ws[w2];
                     if (tid < KJ) s_cs[tid] = v + off;
