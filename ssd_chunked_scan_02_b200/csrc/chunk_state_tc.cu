@@ -142,7 +142,9 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tmX,
     const int64_t i1 = (int64_t)(blockIdx.x + 1) * items / gridDim.x;
 
     if (tid == 0) {
-        for (int i = 0; i < BAR_COUNT; ++i) mbar_init(&bars[i], 1);
+        // a stage counts as scaled once each of the 8 scale warps has arrived
+        for (int i = 0; i < BAR_COUNT; ++i)
+            mbar_init(&bars[i], (i >= BAR_XSCALED && i < BAR_XSCALED + kRing) ? 8 : 1);
         s_flag[0] = 0;
         s_cnt[0] = 0;
         s_cnt[1] = 0;
@@ -318,10 +320,13 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tmX,
             wn.next();                          // item i + 1
             if (has_next) load_dt(wn);
             const float* wbuf = s_w + (k & 1) * 2 * Q;
-            for (int st = 0; st < kSt; ++st, ++it) {
+            // Each warp scales its own rows of a stage and reports it scaled by
+            // itself (a stage's barrier counts 8 arrivals): no block barrier per
+            // stage.  A failed wait makes the warp stop arriving; the verdict is
+            // shared once per item, before the next item's prefix sums.
+            for (int st = 0; st < kSt && !fail; ++st, ++it) {
                 const uint32_t slot = it % kRing;
-                const bool miss = !mbar_wait(&bars[BAR_XFULL + slot], (it / kRing) & 1, status);
-                if (named_bar_or(1, 256, miss)) {
+                if (!mbar_wait(&bars[BAR_XFULL + slot], (it / kRing) & 1, status)) {
                     fail = true;
                     break;
                 }
@@ -342,10 +347,14 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tmX,
                     tile[idx] = v;
                 }
                 fence_proxy_async_smem();       // generic writes -> visible to the MMA (async proxy)
-                named_bar_sync(1, 256);
-                if (tid == 0) mbar_arrive(&bars[BAR_XSCALED + slot]);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars[BAR_XSCALED + slot]);
             }
-            if (!fail && has_next) prefix(wn, (int)((k + 1) & 1));
+            if (named_bar_or(1, 256, fail)) {
+                fail = true;
+                break;
+            }
+            if (has_next) prefix(wn, (int)((k + 1) & 1));
         }
         if (fail) s_flag[0] = 1;
     } else {
