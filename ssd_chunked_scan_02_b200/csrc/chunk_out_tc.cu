@@ -205,7 +205,9 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
     volatile int* s_flag = reinterpret_cast<volatile int*>(smem + S::kFlags);   // [0]: any abort
 
     if (tid == 0) {
-        for (int i = 0; i < BAR_COUNT; ++i) mbar_init(&bars[i], 1);
+        // a head's operands are ready once each of the 8 scale warps has arrived
+        for (int i = 0; i < BAR_COUNT; ++i)
+            mbar_init(&bars[i], (i >= BAR_MFULL && i < BAR_MFULL + 4) ? 8 : 1);
         s_flag[0] = 0;
         fence_mbar_init();
     }
@@ -563,9 +565,13 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
                     }
                     tmem_st16(tmem + lane_base + kColM + 16 * cb, packed);
                 }
+                // Each warp reports its share (scaled rows, mask blocks) by itself.  No
+                // block barrier is needed here: the next head's first barrier keeps
+                // its writes of the single-buffered factors and sums after every
+                // warp is done with this head's.
                 tc_fence_before();
-                named_bar_sync(1, 256);
-                if (tid == 0) mbar_arrive(&bars[BAR_MFULL + f]);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars[BAR_MFULL + f]);
             }
         }
         if (fail) s_flag[0] = 1;
