@@ -58,8 +58,7 @@ struct StateSmem {
     static constexpr int kX = kB + kBBytes;
     static constexpr int kOut = kX + kRing * kStage;       // N = 128: 2 x [32][128] fp32 staging
     static constexpr int kOutBytes = 2 * 32 * 128 * 4;     // two 16 KB staging boxes
-    static constexpr int kDt = kOut + kOutBytes;           // float [2][Q]: dt of one item
-    static constexpr int kW = kDt + 2 * Q * 4;             // float [2 buffers][2 heads][Q]: w_j
+    static constexpr int kW = kOut + kOutBytes;            // float [2 buffers][2 heads][Q]: w_j
     static constexpr int kSeg = kW + 4 * Q * 4;            // float [8]: prefix segment sums
     static constexpr int kBar = kSeg + 8 * 4;
     static constexpr int kTmem = kBar + 32 * 8;
@@ -128,7 +127,6 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tmX,
     uint8_t* sB = smem + S::kB;
     uint8_t* sX = smem + S::kX;
     float* s_out = reinterpret_cast<float*>(smem + S::kOut);
-    float* s_dt = reinterpret_cast<float*>(smem + S::kDt);
     float* s_w = reinterpret_cast<float*>(smem + S::kW);
     float* s_seg = reinterpret_cast<float*>(smem + S::kSeg);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::kBar);
@@ -256,55 +254,55 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tmX,
         }
     } else if (warp < 8) {
         // ================================================== dt / scale warps (0-7)
-        // Per item: (a0) the pair's dt for the chunk (the next item's dt is
-        // loaded while the current item is scaled), the inclusive prefix sum
-        // of dt*A per head in four 64-token segments (one warp each), and
-        // w_j = exp(cs_last - cs_j) dt_j; then each x row j scaled by w_j.
-        constexpr int kPer = (2 * Q) / 256;   // dt values per thread per item
-        constexpr int kSeg = Q / 4;           // tokens per prefix segment
+        // Per item: (a0) the pair's dt for the chunk, loaded by warp (head hk =
+        // w / 4, segment sg = w % 4) straight for its Q / 4 tokens (the next
+        // item's dt is loaded while the current one is scaled); the inclusive
+        // prefix sum of dt*A per segment (Q / 128 consecutive tokens a lane, a
+        // shuffle scan of the lane totals), segment offsets through shared
+        // memory, and w_j = exp(cs_last - cs_j) dt_j; then each x row j scaled
+        // by w_j.
+        constexpr int kPer = Q / 128;         // tokens per lane of a segment
+        constexpr int kSegTok = Q / 4;        // tokens per segment
+        const int hk = warp >> 2, sg = warp & 3;
         float dreg[kPer];
         auto load_dt = [&](const ItemIter& w) {
             const int64_t t0 = w.c * Q;
             const int64_t len = (L - t0) < Q ? (L - t0) : Q;
 #pragma unroll
-            for (int r = 0; r < kPer; ++r) {
-                const int e = tid + 256 * r, hk = e / Q, j = e - hk * Q;
-                dreg[r] = (j < len) ? dt[(w.b * L + t0 + j) * H + 2 * w.pair + hk] : 0.f;
+            for (int k = 0; k < kPer; ++k) {
+                const int j = sg * kSegTok + lane * kPer + k;
+                dreg[k] = (j < len) ? dt[(w.b * L + t0 + j) * H + 2 * w.pair + hk] : 0.f;
             }
         };
+        // w_j of the item into buffer buf (published by the caller's barrier)
         auto prefix = [&](const ItemIter& w, int buf) {
-#pragma unroll
-            for (int r = 0; r < kPer; ++r) s_dt[tid + 256 * r] = dreg[r];
-            named_bar_sync(1, 256);
-            const int hk = warp >> 2, sg = warp & 3;
             const float Ah = A[2 * w.pair + hk];
-            const float* dk = s_dt + hk * Q;
-            float* wk = s_w + (buf * 2 + hk) * Q;
-            float carry = 0.f;
-            for (int base = sg * kSeg; base < (sg + 1) * kSeg; base += 32) {
-                float v = dk[base + lane] * Ah;
+            float v[kPer];
+            float run = 0.f;                       // tokens past the sequence end add 0
 #pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const float u = __shfl_up_sync(0xffffffffu, v, o);
-                    if (lane >= o) v += u;
-                }
-                v += carry;
-                wk[base + lane] = v;                     // local cs_j for now
-                carry = __shfl_sync(0xffffffffu, v, 31);
+            for (int k = 0; k < kPer; ++k) {
+                run += dreg[k] * Ah;
+                v[k] = run;
             }
-            if (lane == 0) s_seg[warp] = carry;
+            float incl = run;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float u = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += u;
+            }
+            if (lane == 31) s_seg[warp] = incl;
             named_bar_sync(1, 256);
-            float off = 0.f, last = 0.f;                 // tokens past the sequence end add 0
+            float off = incl - run, last = 0.f;
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 const float sq = s_seg[hk * 4 + q];
                 if (q < sg) off += sq;
                 last += sq;
             }
-            for (int j = sg * kSeg + lane; j < (sg + 1) * kSeg; j += 32)
-                wk[j] = expf(last - (wk[j] + off)) * dk[j];
+            float* wk = s_w + (buf * 2 + hk) * Q + sg * kSegTok + lane * kPer;
+#pragma unroll
+            for (int k = 0; k < kPer; ++k) wk[k] = expf(last - (v[k] + off)) * dreg[k];
             if (sg == 0 && lane == 0) logdecay[(w.b * T + w.c) * H + 2 * w.pair + hk] = last;
-            named_bar_sync(1, 256);
         };
 
         bool fail = false;
@@ -315,6 +313,7 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tmX,
             load_dt(wn);
             prefix(wn, 0);
         }
+        named_bar_sync(1, 256);
         for (int64_t i = i0, k = 0; i < i1 && !fail; ++i, ++k) {
             const bool has_next = i + 1 < i1;
             wn.next();                          // item i + 1
@@ -323,7 +322,7 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tmX,
             // Each warp scales its own rows of a stage and reports it scaled by
             // itself (a stage's barrier counts 8 arrivals): no block barrier per
             // stage.  A failed wait makes the warp stop arriving; the verdict is
-            // shared once per item, before the next item's prefix sums.
+            // shared once per item, after the next item's prefix sums.
             for (int st = 0; st < kSt && !fail; ++st, ++it) {
                 const uint32_t slot = it % kRing;
                 if (!mbar_wait(&bars[BAR_XFULL + slot], (it / kRing) & 1, status)) {
@@ -350,11 +349,12 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tmX,
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars[BAR_XSCALED + slot]);
             }
+            if (has_next) prefix(wn, (int)((k + 1) & 1));
+            // publishes the next item's w_j and shares the verdict of the waits
             if (named_bar_or(1, 256, fail)) {
                 fail = true;
                 break;
             }
-            if (has_next) prefix(wn, (int)((k + 1) & 1));
         }
         if (fail) s_flag[0] = 1;
     } else {
