@@ -86,9 +86,8 @@ struct OutSmem {
     static constexpr int kXTile = Q * 128;                  // x rows [0, Q) of one head
     static constexpr int kX = kBG + kBGBytes;               // x ring: 2 slots of Q rows (or 4 of 128)
     static constexpr int kYs = kX + 2 * kXTile;             // y staging: 16 KB
-    static constexpr int kDtStride = Q + 2;                 // dt row stride: conflict-free staging stores
-    static constexpr int kDt = kYs + 128 * 128;             // float [kMaxHeads][kDtStride]
-    static constexpr int kCs = kDt + kMaxHeads * kDtStride * 4;   // float [Q] one head's prefix sums (log2 units)
+    static constexpr int kDt = kYs + 128 * 128;             // float [Q] dt of one head
+    static constexpr int kCs = kDt + Q * 4;                 // float [Q] its prefix sums (log2 units)
     static constexpr int kWs = kCs + Q * 4;                 // float [16]: per-warp sums of the scan
     static constexpr int kBeta = kWs + 16 * 4;              // float [128]  (t = 1 block left of diagonal)
     static constexpr int kBeta2 = kBeta + 128 * 4;          // float [128]  (diagonal block)
@@ -345,21 +344,11 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
         const int m = q * 32 + lane;               // row within the tile
         const int i = row0 + m;                    // row within the chunk
         const uint32_t lane_base = (uint32_t)(q * 32) << 16;
-        {
-            // all loads first (the heads of a token are contiguous), then the stores
-            constexpr int kPerT = kMaxHeads * Q / 256;
-            float v[kPerT];
-#pragma unroll
-            for (int r = 0; r < kPerT; ++r) {
-                const int e = tid + 256 * r, j = e / HG, k = e - j * HG;
-                v[r] = (e < HG * KJ && j < len) ? dt[(b * L + t0 + j) * H + head0 + k] : 0.f;
-            }
-#pragma unroll
-            for (int r = 0; r < kPerT; ++r) {
-                const int e = tid + 256 * r, j = e / HG, k = e - j * HG;
-                if (e < HG * KJ) s_dt[k * S::kDtStride + j] = v[r];
-            }
-        }
+        // Thread tid < KJ holds dt of token tid for the head in turn, loaded one
+        // head ahead (the first one while the prologue runs).
+        const bool tok_in = tid < KJ && tid < len;
+        const float* dt_tok = dt + (b * L + t0 + tid) * H + head0;
+        float dt_next = tok_in ? dt_tok[0] : 0.f;
         if (tid < HG) {
             s_Ah[tid] = A[head0 + tid] * kLog2e;
             s_Dh[tid] = Dv[head0 + tid];
@@ -433,7 +422,9 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
                 {
                     // inclusive prefix sums of dt*A (log2 units) of this head over the
                     // tile's KJ columns: a shuffle scan per warp, then the warp offsets
-                    float v = (tid < KJ) ? s_dt[hi * S::kDtStride + tid] * s_Ah[hi] : 0.f;
+                    const float dt_cur = dt_next;
+                    if (hi + 1 < HG) dt_next = tok_in ? dt_tok[hi + 1] : 0.f;
+                    float v = dt_cur * s_Ah[hi];
 #pragma unroll
                     for (int o = 1; o < 32; o <<= 1) {
                         const float u = __shfl_up_sync(0xffffffffu, v, o);
@@ -446,11 +437,14 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
                     if (named_bar_or(1, 256, fail)) break;
                     float off = 0.f;
                     for (int w2 = 0; w2 < warp; ++w2) off += s_ws[w2];
-                    if (tid < KJ) s_cs[tid] = v + off;
+                    if (tid < KJ) {
+                        s_cs[tid] = v + off;
+                        s_dt[tid] = dt_cur;
+                    }
                     named_bar_sync(1, 256);
                 }
                 const float* cs = s_cs;
-                const float* hdt = s_dt + hi * S::kDtStride;
+                const float* hdt = s_dt;
                 const float cs_i = cs[i];
                 const float r = (t == 1) ? cs[127] : 0.f;
                 // the tile's decay span decides the path (the same for every thread)
