@@ -46,12 +46,15 @@
 //               copied from TMEM: the diagonal block becomes G o causal in bf16
 //               (TMEM, the A operand of Y), the block to its left goes to
 //               shared memory as bf16 (the A operand of G_10 X~); per head:
-//               factors, then the x rows of the tile scaled by b_j (fast path)
-//               or the exact mask written to TMEM (one slot), and for t = 1
-//               x rows 0..127 scaled by b_j (fast) or beta_j and h by exp(r)
-//               (exact), in place;
+//               dt (held one token a thread, loaded a head ahead) and its prefix
+//               sums, factors, then the x rows of the tile scaled by b_j (fast
+//               path) or the exact mask written to TMEM (one slot), and for
+//               t = 1 x rows 0..127 scaled by b_j (fast) or beta_j and h by
+//               exp(r) (exact), in place; each warp reports its share of a
+//               head's operands by its own mbarrier arrival;
 //   warps 8-11  epilogue: y staged in shared memory, TMA store;
-//   warp 12     TMA producer (x rows and entering states of the heads, ring of 2);
+//   warp 12     TMA producer (x rows and entering states of the heads, a ring
+//               of four slots for tile 0 of a 256-token chunk, two otherwise);
 //   warp 13     MMA issuer and TMEM owner.
 // Every wait is bounded; a warpgroup leaves its loop only when all its
 // threads agree (bar.red.or), so no named barrier is left half-arrived.
