@@ -126,7 +126,7 @@ ssd_status_t ssd_chunk_scan_fwd_workspace_size(const ssd_dims_t* dims, int chunk
                                                ssd_dtype_t dtype, size_t* bytes) {
     g_detail[0] = 0;
     if (!bytes) return fail(SSD_ERR_INVALID_ARG, "bytes is NULL");
-    ssd::Dims d; ssd::Elt t;
+    ssd::Dims d{}; ssd::Elt t = ssd::Elt::BF16;
     ssd_status_t st = check_dims(dims, chunk_size, true, dtype, &d, &t);
     if (st != SSD_OK) return st;
     *bytes = ws_layout(d, t).total;
@@ -135,7 +135,7 @@ ssd_status_t ssd_chunk_scan_fwd_workspace_size(const ssd_dims_t* dims, int chunk
 
 int ssd_chunk_scan_fwd_uses_tensor_cores(const ssd_dims_t* dims, int chunk_size,
                                          ssd_dtype_t dtype) {
-    ssd::Dims d; ssd::Elt t;
+    ssd::Dims d{}; ssd::Elt t = ssd::Elt::BF16;
     if (check_dims(dims, chunk_size, true, dtype, &d, &t) != SSD_OK) return -1;
     return tc_eligible(d, t) ? 1 : 0;
 }
@@ -146,7 +146,7 @@ ssd_status_t ssd_chunk_scan_fwd(const void* x, const float* dt, const float* A, 
                                 const ssd_dims_t* dims, ssd_dtype_t dtype, void* workspace,
                                 size_t workspace_bytes, void* stream) {
     g_detail[0] = 0;
-    ssd::Dims d; ssd::Elt t;
+    ssd::Dims d{}; ssd::Elt t = ssd::Elt::BF16;
     ssd_status_t st = check_dims(dims, chunk_size, true, dtype, &d, &t);
     if (st != SSD_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -194,7 +194,7 @@ ssd_status_t ssd_chunk_state_fwd(const void* x, const float* dt, const float* A,
                                  int chunk_size, float* chunk_states, float* chunk_logdecay,
                                  const ssd_dims_t* dims, ssd_dtype_t dtype, void* stream) {
     g_detail[0] = 0;
-    ssd::Dims d; ssd::Elt t;
+    ssd::Dims d{}; ssd::Elt t = ssd::Elt::BF16;
     ssd_status_t st = check_dims(dims, chunk_size, true, dtype, &d, &t);
     if (st != SSD_OK) return st;
     if (d.b == 0 || d.L == 0) return SSD_OK;
@@ -213,7 +213,7 @@ ssd_status_t ssd_state_passing_fwd(const float* chunk_states, const float* chunk
                                    float* final_states, int chunk_size, const ssd_dims_t* dims,
                                    ssd_dtype_t dtype, void* stream) {
     g_detail[0] = 0;
-    ssd::Dims d; ssd::Elt t;
+    ssd::Dims d{}; ssd::Elt t = ssd::Elt::BF16;
     ssd_status_t st = check_dims(dims, chunk_size, true, dtype, &d, &t);
     if (st != SSD_OK) return st;
     OPTIONAL_PTR(init_states);
@@ -236,7 +236,7 @@ ssd_status_t ssd_chunk_output_fwd(const void* x, const float* dt, const float* A
                                   int chunk_size, void* y, const ssd_dims_t* dims,
                                   ssd_dtype_t dtype, void* stream) {
     g_detail[0] = 0;
-    ssd::Dims d; ssd::Elt t;
+    ssd::Dims d{}; ssd::Elt t = ssd::Elt::BF16;
     ssd_status_t st = check_dims(dims, chunk_size, true, dtype, &d, &t);
     if (st != SSD_OK) return st;
     if (d.b == 0 || d.L == 0) return SSD_OK;
@@ -254,7 +254,7 @@ ssd_status_t ssd_state_walk_fwd(const void* x, const float* dt, const float* A, 
                                 int chunk_size, const ssd_dims_t* dims, ssd_dtype_t dtype,
                                 void* stream) {
     g_detail[0] = 0;
-    ssd::Dims d; ssd::Elt t;
+    ssd::Dims d{}; ssd::Elt t = ssd::Elt::BF16;
     ssd_status_t st = check_dims(dims, chunk_size, true, dtype, &d, &t);
     if (st != SSD_OK) return st;
     OPTIONAL_PTR(init_states);
@@ -296,7 +296,7 @@ ssd_status_t ssd_step(float* state, const void* x, const float* dt, const float*
                       const void* B, const void* C, const float* D, void* y,
                       const ssd_dims_t* dims, ssd_dtype_t dtype, void* stream) {
     g_detail[0] = 0;
-    ssd::Dims d; ssd::Elt t;
+    ssd::Dims d{}; ssd::Elt t = ssd::Elt::BF16;
     ssd_status_t st = check_dims(dims, 0, false, dtype, &d, &t);
     if (st != SSD_OK) return st;
     if (d.b == 0) return SSD_OK;
