@@ -16,7 +16,10 @@ Spaces", section 状态空间模型 (discretise, then evaluate as a linear
 recurrence) and "Transformers are SSMs" (CiteArk), AI research summary
 (1-semiseparable selective SSM).  Every function is pinned by the ``not gpu``
 tests in ``tests/test_oracle_pins.py`` against closed forms, the materialised
-semiseparable matrix and brute-force expansions.
+semiseparable matrix and brute-force expansions.  ``backward`` (the gradients
+of the same recurrence, for the training use the pages name) is pinned in
+``tests/test_oracle_backward.py`` against central finite differences of the
+forward recurrence and closed forms.
 """
 from __future__ import annotations
 
@@ -50,6 +53,8 @@ def _open(path):
     lib.ssd_oracle_recurrence.argtypes = [_i64] * 6 + [_dbl_p] * 9 + [ctypes.c_int]
     lib.ssd_oracle_step.restype = ctypes.c_int
     lib.ssd_oracle_step.argtypes = [_i64] * 5 + [_dbl_p] * 8
+    lib.ssd_oracle_backward.restype = ctypes.c_int
+    lib.ssd_oracle_backward.argtypes = [_i64] * 6 + [_dbl_p] * 16
     return lib
 
 
@@ -120,3 +125,36 @@ def step(state, x, dt, A, B, C, D):
     if rc != 0:
         raise ValueError("ssd_oracle_step rejected its arguments")
     return y, st
+
+
+def backward(x, dt, A, B, C, D, init, dy, dfinal=None, _lib_override=None):
+    """Gradients of the fp64 recurrence for a loss with dL/dy = dy (b,L,H,P)
+    and dL/dfinal = dfinal (b,H,P,N) or None (zero).  init None means a zero
+    initial state.  Returns a dict of float64 arrays: dx (b,L,H,P), ddt
+    (b,L,H), dA (H), dB (b,L,G,N), dC (b,L,G,N), dD (H), dinit (b,H,P,N)."""
+    x, dt, A, B, C, D, init, dy, dfinal = (_f64(v) for v in (x, dt, A, B, C, D, init, dy, dfinal))
+    b, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    assert dy.shape == x.shape
+    if dfinal is not None:
+        assert dfinal.shape == (b, H, P, N)
+    out = {"dx": np.empty((b, L, H, P)), "ddt": np.empty((b, L, H)), "dA": np.empty((H,)),
+           "dB": np.empty((b, L, G, N)), "dC": np.empty((b, L, G, N)), "dD": np.empty((H,)),
+           "dinit": np.empty((b, H, P, N))}
+    lib = _lib_override if _lib_override is not None else _load()
+    rc = lib.ssd_oracle_backward(b, L, H, P, N, G, _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C),
+                                 _ptr(D), _ptr(init), _ptr(dy), _ptr(dfinal), _ptr(out["dx"]),
+                                 _ptr(out["ddt"]), _ptr(out["dA"]), _ptr(out["dB"]),
+                                 _ptr(out["dC"]), _ptr(out["dD"]), _ptr(out["dinit"]))
+    if rc != 0:
+        raise ValueError("ssd_oracle_backward rejected its arguments")
+    return out
+
+
+def backward_from(path):
+    """A ``backward`` bound to another build of ssd_oracle.c (mutation tests)."""
+    lib = _open(path)
+
+    def bwd(x, dt, A, B, C, D, init, dy, dfinal=None):
+        return backward(x, dt, A, B, C, D, init, dy, dfinal, _lib_override=lib)
+    return bwd

@@ -152,3 +152,126 @@ int ssd_oracle_step(int64_t batch, int64_t nheads, int64_t headdim, int64_t dsta
     }
     return 0;
 }
+
+/* ------------------------------------------------------------------ backward
+ * Gradients of the recurrence above for a loss whose derivatives with respect
+ * to the outputs are dy (like y) and dfinal (like the final state; NULL = 0).
+ * "Transformers are SSMs" (CiteArk), AI research summary: training is the
+ * use the layer is built for; the gradients below are the chain rule applied
+ * to the same token-by-token recurrence, in reverse token order:
+ *
+ *     G      = dL/dS_t          (starts at dfinal, then G += dy_t C_t^T)
+ *     dC_t  += S_t^T dy_t        dx_t = D_h dy_t + dt_t G B_t
+ *     dB_t  += dt_t G^T x_t      ddt_t = x_t^T G B_t + A_h a_t <G, S_{t-1}>
+ *     dA_h  += dt_t a_t <G, S_{t-1}>     dD_h += dy_t . x_t
+ *     G      = a_t G            (dL/dS_{t-1}); dinit = G after token 0
+ *
+ * The states S_t are kept from a forward sweep (test sizes only).  dB and dC
+ * sum over the heads of a group, dA and dD over batch and tokens.  Outputs
+ * are overwritten (not accumulated into).  Return 0, or -1 on an invalid
+ * argument or allocation failure. */
+static void bwd_one(int64_t b, int64_t h, int64_t L, int64_t H, int64_t P, int64_t N,
+                    int64_t G, const double* x, const double* dt, const double* A,
+                    const double* B, const double* C, const double* D, const double* init,
+                    const double* dy, const double* dfinal, double* dx, double* ddt,
+                    double* dA_part, double* dB, double* dC, double* dD_part, double* dinit,
+                    double* Sall, double* Gm) {
+    const int64_t g = h * G / H;
+    const int64_t PN = P * N;
+    /* forward sweep: Sall[0] = initial state, Sall[t + 1] = S_t */
+    if (init != NULL)
+        memcpy(Sall, init + (b * H + h) * PN, sizeof(double) * (size_t)PN);
+    else
+        memset(Sall, 0, sizeof(double) * (size_t)PN);
+    for (int64_t t = 0; t < L; ++t) {
+        const double dtv = dt[(b * L + t) * H + h];
+        const double at = exp(A[h] * dtv);
+        const double* xt = x + ((b * L + t) * H + h) * P;
+        const double* Bt = B + ((b * L + t) * G + g) * N;
+        const double* Sp = Sall + t * PN;
+        double* Sn = Sall + (t + 1) * PN;
+        for (int64_t p = 0; p < P; ++p)
+            for (int64_t n = 0; n < N; ++n)
+                Sn[p * N + n] = at * Sp[p * N + n] + dtv * xt[p] * Bt[n];
+    }
+    /* reverse sweep */
+    if (dfinal != NULL)
+        memcpy(Gm, dfinal + (b * H + h) * PN, sizeof(double) * (size_t)PN);
+    else
+        memset(Gm, 0, sizeof(double) * (size_t)PN);
+    for (int64_t t = L - 1; t >= 0; --t) {
+        const double dtv = dt[(b * L + t) * H + h];
+        const double at = exp(A[h] * dtv);
+        const double* xt = x + ((b * L + t) * H + h) * P;
+        const double* Bt = B + ((b * L + t) * G + g) * N;
+        const double* Ct = C + ((b * L + t) * G + g) * N;
+        const double* dyt = dy + ((b * L + t) * H + h) * P;
+        const double* St = Sall + (t + 1) * PN;   /* S_t */
+        const double* Sp = Sall + t * PN;         /* S_{t-1} */
+        double* dxt = dx + ((b * L + t) * H + h) * P;
+        double* dBt = dB + ((b * L + t) * G + g) * N;
+        double* dCt = dC + ((b * L + t) * G + g) * N;
+        /* y_t = S_t C_t + D x_t */
+        for (int64_t p = 0; p < P; ++p)
+            for (int64_t n = 0; n < N; ++n) {
+                Gm[p * N + n] += dyt[p] * Ct[n];
+                dCt[n] += St[p * N + n] * dyt[p];
+            }
+        double xgb = 0.0, gs = 0.0, dydx = 0.0;
+        for (int64_t p = 0; p < P; ++p) {
+            double gb = 0.0;
+            for (int64_t n = 0; n < N; ++n) {
+                gb += Gm[p * N + n] * Bt[n];
+                dBt[n] += dtv * Gm[p * N + n] * xt[p];
+                gs += Gm[p * N + n] * Sp[p * N + n];
+            }
+            dxt[p] = D[h] * dyt[p] + dtv * gb;
+            xgb += xt[p] * gb;
+            dydx += dyt[p] * xt[p];
+        }
+        /* S_t = a_t S_{t-1} + dt_t x_t B_t^T,  a_t = exp(dt_t A_h) */
+        ddt[(b * L + t) * H + h] = xgb + A[h] * at * gs;
+        dA_part[h] += dtv * at * gs;
+        dD_part[h] += dydx;
+        for (int64_t k = 0; k < PN; ++k) Gm[k] *= at;
+    }
+    if (dinit) memcpy(dinit + (b * H + h) * PN, Gm, sizeof(double) * (size_t)PN);
+}
+
+int ssd_oracle_backward(int64_t batch, int64_t seqlen, int64_t nheads, int64_t headdim,
+                        int64_t dstate, int64_t ngroups, const double* x, const double* dt,
+                        const double* A, const double* B, const double* C, const double* D,
+                        const double* init, const double* dy, const double* dfinal,
+                        double* dx, double* ddt, double* dA, double* dB, double* dC,
+                        double* dD, double* dinit) {
+    if (!dims_ok(batch, seqlen, nheads, headdim, dstate, ngroups)) return -1;
+    if (!A || !D || !dA || !dD) return -1;
+    const int have_tokens = seqlen > 0 && batch > 0;
+    if (have_tokens && (!x || !dt || !B || !C || !dy || !dx || !ddt || !dB || !dC)) return -1;
+    const int64_t H = nheads, P = headdim, N = dstate, G = ngroups, L = seqlen;
+    const int64_t PN = P * N;
+    if (have_tokens) {
+        memset(dx, 0, sizeof(double) * (size_t)(batch * L * H * P));
+        memset(ddt, 0, sizeof(double) * (size_t)(batch * L * H));
+        memset(dB, 0, sizeof(double) * (size_t)(batch * L * G * N));
+        memset(dC, 0, sizeof(double) * (size_t)(batch * L * G * N));
+    }
+    memset(dA, 0, sizeof(double) * (size_t)H);
+    memset(dD, 0, sizeof(double) * (size_t)H);
+    double* Sall = (double*)malloc(sizeof(double) * (size_t)((L + 1) * PN));
+    double* Gm = (double*)malloc(sizeof(double) * (size_t)PN);
+    if (!Sall || !Gm) {
+        free(Sall);
+        free(Gm);
+        return -1;
+    }
+    /* sequential over (batch, head): dB, dC are shared by a group's heads and
+     * dA, dD by the batch, so one order of summation, no races */
+    for (int64_t b = 0; b < batch; ++b)
+        for (int64_t h = 0; h < H; ++h)
+            bwd_one(b, h, L, H, P, N, G, x, dt, A, B, C, D, init, dy, dfinal, dx, ddt, dA, dB,
+                    dC, dD, dinit, Sall, Gm);
+    free(Sall);
+    free(Gm);
+    return 0;
+}
