@@ -21,9 +21,11 @@
 // next items stream while the current one is scaled, multiplied and stored.
 // Roles:
 //   warp 12 (one lane)  TMA producer: B tile per chunk, x stages into the ring;
-//   warps 0-7           dt prefix sums and w_j per item (the next item's dt is
-//                       loaded while the current one is scaled), then x rows
-//                       scaled in place by w_j (the MMA sees bf16(w_j x_j));
+//   warps 0-7           dt prefix sums and w_j per item (each warp loads its
+//                       own 64-token segment of one head's dt, the next item's
+//                       while the current one is scaled), then x rows scaled
+//                       in place by w_j (the MMA sees bf16(w_j x_j)); each warp
+//                       reports a stage scaled by its own mbarrier arrival;
 //   warp 13 (one lane)  MMA issuer (and TMEM owner), two accumulator slots;
 //   warps 8-11          epilogue: TMEM -> fp32 S in HBM, layout (b, T, H, P, N),
 //                       through a shared-memory staging pair and TMA bulk
