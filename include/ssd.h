@@ -184,6 +184,37 @@ SSD_API ssd_status_t ssd_chunk_scan_fwd_noalloc(const void* x, const float* dt, 
                                                 void* stream);
 
 /*
+ * Gradients of ssd_chunk_scan_fwd (a first version: exact fp32 arithmetic on
+ * the CUDA cores, one CTA per (batch, head) walking the sequence; slow next
+ * to the forward).  "Transformers are SSMs" (CiteArk), AI research summary:
+ * training is what the layer is for; the gradients are the chain rule on
+ * the recurrence h_t = exp(dt_t A_h) h_{t-1} + dt_t x_t B_t^T, y_t = h_t C_t
+ * + D_h x_t, taken in reverse token order.
+ * Inputs: the forward's inputs (x, B, C in dtype; dt, A, D, init_states
+ * fp32; init_states NULL = zero), dy (b,L,H,P) in dtype = dL/dy, and
+ * dfinal_states (b,H,P,N) fp32 = dL/dfinal_states or NULL (zero).
+ * Outputs, all fp32 and fully written: dx (b,L,H,P), ddt (b,L,H), dA (H),
+ * dB (b,L,G,N), dC (b,L,G,N) (summed over the heads of each group), dD (H),
+ * dinit_states (b,H,P,N) = dL/dinit_states (NULL = not wanted).  dA, dD, dB
+ * and dC are zeroed, then accumulated with atomics, so their rounding (not
+ * their value) may differ between runs.  Requires headdim * dstate <= 8192
+ * (else SSD_ERR_UNSUPPORTED).  workspace: >= the size reported by
+ * ssd_chunk_scan_bwd_workspace_size (fp32 state checkpoints every 64 tokens
+ * and one 64-token segment of states, per (batch, head)); NULL only when that
+ * size is 0.  Inputs and outputs must not alias.
+ */
+SSD_API ssd_status_t ssd_chunk_scan_bwd_workspace_size(const ssd_dims_t* dims, ssd_dtype_t dtype,
+                                                       size_t* bytes);
+SSD_API ssd_status_t ssd_chunk_scan_bwd(const void* x, const float* dt, const float* A,
+                                        const void* B, const void* C, const float* D,
+                                        const float* init_states, const void* dy,
+                                        const float* dfinal_states, float* dx, float* ddt,
+                                        float* dA, float* dB, float* dC, float* dD,
+                                        float* dinit_states, const ssd_dims_t* dims,
+                                        ssd_dtype_t dtype, void* workspace,
+                                        size_t workspace_bytes, void* stream);
+
+/*
  * Reports, and clears, a device-side wait that gave up in an earlier call on
  * the current device: the tensor-core kernels bound every wait, and one that
  * runs out records SSD_ERR_TIMEOUT in a device status word and ends the

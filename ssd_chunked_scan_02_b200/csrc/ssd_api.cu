@@ -307,4 +307,47 @@ ssd_status_t ssd_step(float* state, const void* x, const float* dt, const float*
     return e == cudaSuccess ? SSD_OK : cuda_fail(e, "decode-step kernel");
 }
 
+ssd_status_t ssd_chunk_scan_bwd_workspace_size(const ssd_dims_t* dims, ssd_dtype_t dtype,
+                                               size_t* bytes) {
+    g_detail[0] = 0;
+    ssd::Dims d{}; ssd::Elt t = ssd::Elt::BF16;
+    ssd_status_t st = check_dims(dims, 0, false, dtype, &d, &t);
+    if (st != SSD_OK) return st;
+    if (!bytes) return fail(SSD_ERR_INVALID_ARG, "bytes is NULL");
+    if (!ssd::backward_supported(d))
+        return fail(SSD_ERR_UNSUPPORTED, "the backward needs headdim * dstate <= 8192");
+    *bytes = (d.b == 0 || d.L == 0) ? 0 : ssd::backward_workspace_bytes(d);
+    return SSD_OK;
+}
+
+ssd_status_t ssd_chunk_scan_bwd(const void* x, const float* dt, const float* A, const void* B,
+                                const void* C, const float* D, const float* init_states,
+                                const void* dy, const float* dfinal_states, float* dx,
+                                float* ddt, float* dA, float* dB, float* dC, float* dD,
+                                float* dinit_states, const ssd_dims_t* dims, ssd_dtype_t dtype,
+                                void* workspace, size_t workspace_bytes, void* stream) {
+    g_detail[0] = 0;
+    ssd::Dims d{}; ssd::Elt t = ssd::Elt::BF16;
+    ssd_status_t st = check_dims(dims, 0, false, dtype, &d, &t);
+    if (st != SSD_OK) return st;
+    if (!ssd::backward_supported(d))
+        return fail(SSD_ERR_UNSUPPORTED, "the backward needs headdim * dstate <= 8192");
+    REQUIRE_PTR(A); REQUIRE_PTR(D); REQUIRE_PTR(dA); REQUIRE_PTR(dD);
+    OPTIONAL_PTR(init_states); OPTIONAL_PTR(dfinal_states); OPTIONAL_PTR(dinit_states);
+    if (d.b > 0 && d.L > 0) {
+        REQUIRE_PTR(x); REQUIRE_PTR(dt); REQUIRE_PTR(B); REQUIRE_PTR(C); REQUIRE_PTR(dy);
+        REQUIRE_PTR(dx); REQUIRE_PTR(ddt); REQUIRE_PTR(dB); REQUIRE_PTR(dC);
+        const size_t need = ssd::backward_workspace_bytes(d);
+        if (workspace_bytes < need)
+            return fail(SSD_ERR_INVALID_ARG, "workspace_bytes %zu < required %zu", workspace_bytes,
+                        need);
+        REQUIRE_PTR(workspace);
+    }
+    cudaError_t e = ssd::launch_backward(x, dt, A, B, C, D, init_states, dy, dfinal_states, dx,
+                                         ddt, dA, dB, dC, dD, dinit_states,
+                                         static_cast<float*>(workspace), d, t,
+                                         static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? SSD_OK : cuda_fail(e, "backward kernel");
+}
+
 }  // extern "C"

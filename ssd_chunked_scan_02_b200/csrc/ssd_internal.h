@@ -36,4 +36,13 @@ cudaError_t launch_step(float* state, const void* x, const float* dt, const floa
 cudaError_t launch_copy_or_zero(const float* init, float* final_states, int64_t n,
                                 cudaStream_t s);
 
+// Backward (gradients of the forward), exact fp32 on the CUDA cores.
+size_t backward_workspace_bytes(const Dims& d);
+bool backward_supported(const Dims& d);
+cudaError_t launch_backward(const void* x, const float* dt, const float* A, const void* B,
+                            const void* C, const float* D, const float* init, const void* dy,
+                            const float* dfinal, float* dx, float* ddt, float* dA, float* dB,
+                            float* dC, float* dD, float* dinit, float* ws, const Dims& d, Elt t,
+                            cudaStream_t s);
+
 }  // namespace ssd

@@ -26,7 +26,7 @@ EXPORTED = ("ssd_status_string", "ssd_last_error_detail", "ssd_chunk_scan_fwd_wo
             "ssd_chunk_scan_fwd", "ssd_step", "ssd_chunk_state_fwd", "ssd_state_passing_fwd",
             "ssd_chunk_output_fwd", "ssd_chunk_scan_fwd_uses_tensor_cores",
             "ssd_chunk_scan_fwd_noalloc", "ssd_poll_device_status", "ssd_state_walk_fwd",
-            "ssd_debug_expire_wait")
+            "ssd_debug_expire_wait", "ssd_chunk_scan_bwd_workspace_size", "ssd_chunk_scan_bwd")
 
 
 class SSDError(RuntimeError):
@@ -85,6 +85,12 @@ def load(path: str = LIB_PATH):
     lib.ssd_state_passing_fwd.argtypes = [_vp] * 5 + [ctypes.c_int, dims_p, ctypes.c_int, _vp]
     lib.ssd_chunk_output_fwd.restype = ctypes.c_int
     lib.ssd_chunk_output_fwd.argtypes = [_vp] * 7 + [ctypes.c_int, _vp, dims_p, ctypes.c_int, _vp]
+    lib.ssd_chunk_scan_bwd_workspace_size.restype = ctypes.c_int
+    lib.ssd_chunk_scan_bwd_workspace_size.argtypes = [dims_p, ctypes.c_int,
+                                                      ctypes.POINTER(ctypes.c_size_t)]
+    lib.ssd_chunk_scan_bwd.restype = ctypes.c_int
+    lib.ssd_chunk_scan_bwd.argtypes = [_vp] * 16 + [dims_p, ctypes.c_int, _vp, ctypes.c_size_t,
+                                                    _vp]
     _lib = lib
     return lib
 
@@ -279,3 +285,37 @@ def ssd_chunk_output_fwd(x, dt, A, B, C, D, prev_states, chunk_size: int, y=None
                                      ctypes.byref(dims), _dtype_code(x.dtype), _stream(stream))
     _check(st, "ssd_chunk_output_fwd")
     return y
+
+
+def ssd_chunk_scan_bwd_workspace_size(dims: ssd_dims_t, dtype: torch.dtype) -> int:
+    n = ctypes.c_size_t(0)
+    _check(load().ssd_chunk_scan_bwd_workspace_size(ctypes.byref(dims), _dtype_code(dtype),
+                                                    ctypes.byref(n)),
+           "ssd_chunk_scan_bwd_workspace_size")
+    return int(n.value)
+
+
+def ssd_chunk_scan_bwd(x, dt, A, B, C, D, dy, init_states=None, dfinal_states=None,
+                       want_dinit: bool = True, workspace=None, stream=None):
+    """Gradients of ssd_chunk_scan_fwd for dL/dy = dy (b,L,H,P, x's dtype) and
+    dL/dfinal_states = dfinal_states ((b,H,P,N) fp32 or None).  Returns a dict
+    of fp32 tensors: dx, ddt, dA, dB, dC, dD and (if want_dinit) dinit."""
+    dims = _fwd_dims(x, B)
+    b, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    f32 = dict(device=x.device, dtype=torch.float32)
+    out = {"dx": torch.empty((b, L, H, P), **f32), "ddt": torch.empty((b, L, H), **f32),
+           "dA": torch.empty((H,), **f32), "dB": torch.empty((b, L, G, N), **f32),
+           "dC": torch.empty((b, L, G, N), **f32), "dD": torch.empty((H,), **f32),
+           "dinit": torch.empty((b, H, P, N), **f32) if want_dinit else None}
+    need = ssd_chunk_scan_bwd_workspace_size(dims, x.dtype)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), device=x.device, dtype=torch.uint8)
+    st = load().ssd_chunk_scan_bwd(_ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+                                   _ptr(init_states), _ptr(dy), _ptr(dfinal_states),
+                                   _ptr(out["dx"]), _ptr(out["ddt"]), _ptr(out["dA"]),
+                                   _ptr(out["dB"]), _ptr(out["dC"]), _ptr(out["dD"]),
+                                   _ptr(out["dinit"]), ctypes.byref(dims), _dtype_code(x.dtype),
+                                   _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(st, "ssd_chunk_scan_bwd")
+    return out

@@ -1,0 +1,95 @@
+"""GPU parity of the backward (ssd_chunk_scan_bwd, through the C ABI) with the
+oracle's fp64 backward on the same inputs (bf16 inputs rounded once, then
+widened for the oracle).  Every gradient element is compared; the metric is
+max|g - g_ref| / max|g_ref| per gradient tensor.  The GPU computes in fp32
+(inputs as given), so the bound is the fp32 one, 1e-4."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from parity import record
+from ssd_chunked_scan_02_b200 import ssd
+
+TOL = 1e-4
+NAMES = ("dx", "ddt", "dA", "dB", "dC", "dD", "dinit")
+
+
+def _inputs(seed, b, L, H, P, N, G, dtype, with_init, with_dfinal):
+    g = torch.Generator().manual_seed(seed)
+    t = lambda *s: torch.randn(*s, generator=g)
+    inp = dict(
+        x=t(b, L, H, P).to(dtype), dt=torch.nn.functional.softplus(t(b, L, H) - 1.0),
+        A=-torch.exp(torch.rand(H, generator=g) * np.log(8.0)),
+        B=(t(b, L, G, N) / np.sqrt(N)).to(dtype), C=(t(b, L, G, N) / np.sqrt(N)).to(dtype),
+        D=t(H), init=(0.3 * t(b, H, P, N)) if with_init else None,
+        dy=t(b, L, H, P).to(dtype), dfinal=t(b, H, P, N) if with_dfinal else None)
+    return inp
+
+
+def _run(name, seed, b, L, H, P, N, G, dtype, with_init=True, with_dfinal=True):
+    inp = _inputs(seed, b, L, H, P, N, G, dtype, with_init, with_dfinal)
+    dev = {k: (v.cuda().contiguous() if v is not None else None) for k, v in inp.items()}
+    out = ssd.ssd_chunk_scan_bwd(dev["x"], dev["dt"], dev["A"], dev["B"], dev["C"], dev["D"],
+                                 dev["dy"], init_states=dev["init"], dfinal_states=dev["dfinal"])
+    torch.cuda.synchronize()
+    f = lambda v: None if v is None else v.double().numpy()
+    ref = oracle.backward(f(inp["x"]), f(inp["dt"]), f(inp["A"]), f(inp["B"]), f(inp["C"]),
+                          f(inp["D"]), f(inp["init"]), f(inp["dy"]), f(inp["dfinal"]))
+    errs = {}
+    for k in NAMES:
+        got = out[k].double().cpu().numpy()
+        r = ref[k]
+        scale = float(np.abs(r).max()) if r.size else 0.0
+        errs[k] = float(np.abs(got - r).max() / scale) if scale > 0 else float(np.abs(got).max() if got.size else 0.0)
+    record("bwd_" + name, **errs)
+    assert max(errs.values()) <= TOL, errs
+    return out, ref
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32], ids=["bf16", "fp32"])
+@pytest.mark.parametrize("G,with_init,with_dfinal", [(2, True, True), (1, False, True), (2, True, False)])
+def test_backward_small(dtype, G, with_init, with_dfinal):
+    # 150 tokens: two whole 64-token checkpoint segments and a ragged third
+    _run(f"small_G{G}_{int(with_init)}{int(with_dfinal)}_{str(dtype)[6:]}", 71 + G, 2, 150, 4,
+         16, 32, G, dtype, with_init, with_dfinal)
+
+
+@pytest.mark.gpu
+def test_backward_largest_state():
+    # P x N = 8192: 32 state elements per thread, one segment and a ragged one
+    _run("P64_N128", 81, 1, 130, 2, 64, 128, 1, torch.bfloat16)
+
+
+@pytest.mark.gpu
+def test_backward_odd_sizes_single_token():
+    _run("odd_L1", 82, 3, 1, 3, 5, 7, 1, torch.float32)
+    _run("odd_L65", 83, 1, 65, 6, 12, 20, 3, torch.bfloat16)
+
+
+@pytest.mark.gpu
+def test_backward_no_tokens():
+    # L = 0: the initial state's gradient is the final state's; the rest is zero
+    b, H, P, N, G = 2, 4, 8, 16, 2
+    x = torch.zeros(b, 0, H, P, device="cuda", dtype=torch.bfloat16)
+    dt = torch.zeros(b, 0, H, device="cuda")
+    Bm = torch.zeros(b, 0, G, N, device="cuda", dtype=torch.bfloat16)
+    A = -torch.ones(H, device="cuda")
+    D = torch.ones(H, device="cuda")
+    dfinal = torch.randn(b, H, P, N, device="cuda")
+    out = ssd.ssd_chunk_scan_bwd(x, dt, A, Bm, Bm, D, x, dfinal_states=dfinal)
+    torch.cuda.synchronize()
+    assert torch.equal(out["dinit"], dfinal)
+    assert float(out["dA"].abs().max()) == 0.0 and float(out["dD"].abs().max()) == 0.0
+
+
+@pytest.mark.gpu
+def test_backward_rejects_oversized_state():
+    x = torch.zeros(1, 4, 1, 128, device="cuda", dtype=torch.bfloat16)
+    Bm = torch.zeros(1, 4, 1, 128, device="cuda", dtype=torch.bfloat16)
+    dt = torch.zeros(1, 4, 1, device="cuda")
+    one = torch.ones(1, device="cuda")
+    with pytest.raises(ssd.SSDError) as e:
+        ssd.ssd_chunk_scan_bwd(x, dt, one, Bm, Bm, one, x)
+    assert e.value.status == ssd.SSD_ERR_UNSUPPORTED
