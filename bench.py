@@ -317,6 +317,59 @@ def measure_config(w, dev, stream, flush, reps, world, rank):
     return out
 
 
+def bwd_bytes(w) -> int:
+    """Algorithmic bytes of the backward: its inputs read once (x, dy, B, C in
+    the input dtype; dt fp32; the initial state when given) and its outputs
+    written once (dx, ddt, dB, dC, d(initial state) in fp32)."""
+    s = 2 if w.dtype == "bf16" else 4
+    bl = w.batch * w.seqlen
+    reads = bl * (2 * w.nheads * w.headdim * s + 2 * w.ngroups * w.dstate * s + 4 * w.nheads)
+    writes = bl * (w.nheads * w.headdim * 4 + 4 * w.nheads + 2 * w.ngroups * w.dstate * 4)
+    states = 4 * w.batch * w.nheads * w.headdim * w.dstate * ((1 if w.with_init else 0) + 1)
+    return reads + writes + states
+
+
+def measure_backward(w, dev, stream, flush, reps, world, rank, peak_gbs):
+    """Device time of ssd_chunk_scan_bwd on one workload (L2 flushed before
+    every timed call, max over ranks), with its HBM roofline fraction."""
+    import torch
+    from ssd_chunked_scan_02_b200 import inputs, ssd
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(w.seed + 2000 + 1000 * rank)
+    inp = inputs.make_inputs(w, device=dev, gen=gen)
+    dy = torch.randn(inp["x"].shape, device=dev, generator=gen).to(inp["x"].dtype)
+    dims = ssd.make_dims(w.batch, w.seqlen, w.nheads, w.headdim, w.dstate, w.ngroups)
+    ws = torch.empty(max(16, ssd.ssd_chunk_scan_bwd_workspace_size(dims, inp["x"].dtype)),
+                     device=dev, dtype=torch.uint8)
+
+    def bwd():
+        ssd.ssd_chunk_scan_bwd(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], inp["D"], dy,
+                               init_states=inp["init"], workspace=ws, stream=stream)
+    for _ in range(3):
+        flush.zero_()
+        bwd()
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(reps)]
+    for st, en in evs:
+        flush.zero_()
+        st.record(stream)
+        bwd()
+        en.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = max_over_ranks(sum(st.elapsed_time(en) for st, en in evs), world) / reps
+    nbytes = bwd_bytes(w)
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    out = {"workload": w.name, "kernel": "exact fp32 SIMT, one CTA per (batch, head)",
+           "ms_per_step": ms, "tokens_per_s": world * w.tokens / (ms * 1e-3),
+           "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak_gbs, "unit": "GB/s",
+                        "frac": gbs / peak_gbs, "alg_bytes_per_launch": nbytes}}
+    del inp, dy, ws
+    torch.cuda.empty_cache()
+    return out
+
+
 # ---------------------------------------------------------------- GPU arm
 def main():
     ap = argparse.ArgumentParser()
@@ -327,7 +380,7 @@ def main():
     ap.add_argument("--decode-steps", type=int, default=50)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra-configs", action="store_true",
-                    help="skip the 130M-layer and length-sweep lines")
+                    help="skip the 130M-layer and length-sweep lines and the backward")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
@@ -523,6 +576,11 @@ def main():
         for e in extra:
             e["hbm_frac_at_bytes_min"] = e["hbm_gbs_at_bytes_min"] / pk["hbm_gbs"]
             e["pct_bf16_peak_dense"] = 100 * e["tflops_dense"] / pk["bf16_tflops"]
+    # ---- the backward (gradients), at the 130M-layer shape
+    bwd = None
+    if not args.no_extra_configs:
+        bwd = measure_backward(inputs.LAYER_130M, dev, stream, flush, max(3, args.steps // 4),
+                               world, rank, pk["hbm_gbs"])
 
     # ---- CPU oracle baseline (rank 0, N = 1 only)
     cpu = None
@@ -566,6 +624,7 @@ def main():
             "e2e": {"value": world * w.tokens / (e2e_ms * 1e-3), "unit": UNIT,
                     "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "other_configs": extra,
+            "backward": bwd,
             "cpu_baseline": cpu,
             "gpu_launches": 3 * args.steps,
             "clocks": clocks,

@@ -64,6 +64,7 @@ ssd_bwd_kernel(const T* __restrict__ x, const float* __restrict__ dt, const floa
     float* sw = rc + N;          // 2 x 8 warp partials
 
     const float Ah = A[h], Dh = Dv[h];
+    const bool warp_rows = (N % 32) == 0;        // then P N % 32 == 0 too: warp-uniform guards
     float S[kMaxPer], Gm[kMaxPer];
 #pragma unroll
     for (int k = 0; k < kMaxPer; ++k) {
@@ -113,6 +114,7 @@ ssd_bwd_kernel(const T* __restrict__ x, const float* __restrict__ dt, const floa
         }
         for (int64_t t = t0; t < t1; ++t) {
             advance(t);
+            if (t + 1 == t1) break;              // S_{t1-1} stays in registers
             float* o = sg + (t - t0) * PN;
 #pragma unroll
             for (int k = 0; k < kMaxPer; ++k) {
@@ -136,8 +138,10 @@ ssd_bwd_kernel(const T* __restrict__ x, const float* __restrict__ dt, const floa
             __syncthreads();
             const float dtv = dt[(b * L + t) * H + h];
             const float a = expf(dtv * Ah);
-            const float* St = sg + (t - t0) * PN;                        // S_t (this thread's own writes)
-            const float* Sp = (t == t0) ? c : sg + (t - t0 - 1) * PN;   // S_{t-1}
+            // S holds S_t (the recompute ended there; each step below moves it
+            // back one token); S_{t-1} comes from the segment scratch (this
+            // thread's own writes) or the checkpoint
+            const float* Sp = (t == t0) ? c : sg + (t - t0 - 1) * PN;
             float xgb = 0.f, gs = 0.f;
 #pragma unroll
             for (int k = 0; k < kMaxPer; ++k) {
@@ -147,11 +151,19 @@ ssd_bwd_kernel(const T* __restrict__ x, const float* __restrict__ dt, const floa
                     const float gv = Gm[k] + sdy[p] * sC[n];             // dL/dS_t
                     Gm[k] = gv;
                     const float gb = gv * sB[n];
-                    atomicAdd(&rx[p], gb);
+                    if (warp_rows) {
+                        // N % 32 == 0: a warp's 32 elements share one row p
+                        const float r = warp_sum(gb);
+                        if (lane == 0) atomicAdd(&rx[p], r);
+                    } else {
+                        atomicAdd(&rx[p], gb);
+                    }
                     atomicAdd(&rb[n], gv * sx[p]);
-                    atomicAdd(&rc[n], St[e] * sdy[p]);
+                    atomicAdd(&rc[n], S[k] * sdy[p]);
                     xgb += sx[p] * gb;
-                    gs += gv * Sp[e];
+                    const float sp = Sp[e];
+                    gs += gv * sp;
+                    S[k] = sp;                                            // S_{t-1}
                 }
             }
             xgb = warp_sum(xgb);
