@@ -361,7 +361,7 @@ def measure_backward(w, dev, stream, flush, reps, world, rank, peak_gbs):
     ms = max_over_ranks(sum(st.elapsed_time(en) for st, en in evs), world) / reps
     nbytes = bwd_bytes(w)
     gbs = nbytes / (ms * 1e-3) / 1e9
-    out = {"workload": w.name, "kernel": "exact fp32 SIMT, one CTA per (batch, head)",
+    out = {"workload": w.name, "kernel": "exact fp32 SIMT, one CTA per block of state rows of a (batch, head)",
            "ms_per_step": ms, "tokens_per_s": world * w.tokens / (ms * 1e-3),
            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak_gbs, "unit": "GB/s",
                         "frac": gbs / peak_gbs, "alg_bytes_per_launch": nbytes}}

@@ -185,8 +185,8 @@ SSD_API ssd_status_t ssd_chunk_scan_fwd_noalloc(const void* x, const float* dt, 
 
 /*
  * Gradients of ssd_chunk_scan_fwd (a first version: exact fp32 arithmetic on
- * the CUDA cores, one CTA per (batch, head) walking the sequence; slow next
- * to the forward).  "Transformers are SSMs" (CiteArk), AI research summary:
+ * the CUDA cores, one CTA per block of state rows of a (batch, head) walking
+ * the sequence; slow next to the forward).  "Transformers are SSMs" (CiteArk), AI research summary:
  * training is what the layer is for; the gradients are the chain rule on
  * the recurrence h_t = exp(dt_t A_h) h_{t-1} + dt_t x_t B_t^T, y_t = h_t C_t
  * + D_h x_t, taken in reverse token order.
@@ -197,10 +197,10 @@ SSD_API ssd_status_t ssd_chunk_scan_fwd_noalloc(const void* x, const float* dt, 
  * dB (b,L,G,N), dC (b,L,G,N) (summed over the heads of each group), dD (H),
  * dinit_states (b,H,P,N) = dL/dinit_states (NULL = not wanted).  dA, dD, dB
  * and dC are zeroed, then accumulated with atomics, so their rounding (not
- * their value) may differ between runs.  Requires headdim * dstate <= 8192
- * (else SSD_ERR_UNSUPPORTED).  workspace: >= the size reported by
+ * their value) may differ between runs.  workspace: >= the size reported by
  * ssd_chunk_scan_bwd_workspace_size (fp32 state checkpoints every 64 tokens
- * and one 64-token segment of states, per (batch, head)); NULL only when that
+ * and one 64-token segment of states, per (batch, head) and block of state
+ * rows); NULL only when that
  * size is 0.  Inputs and outputs must not alias.
  */
 SSD_API ssd_status_t ssd_chunk_scan_bwd_workspace_size(const ssd_dims_t* dims, ssd_dtype_t dtype,

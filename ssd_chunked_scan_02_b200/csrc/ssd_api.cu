@@ -315,7 +315,7 @@ ssd_status_t ssd_chunk_scan_bwd_workspace_size(const ssd_dims_t* dims, ssd_dtype
     if (st != SSD_OK) return st;
     if (!bytes) return fail(SSD_ERR_INVALID_ARG, "bytes is NULL");
     if (!ssd::backward_supported(d))
-        return fail(SSD_ERR_UNSUPPORTED, "the backward needs headdim * dstate <= 8192");
+        return fail(SSD_ERR_UNSUPPORTED, "dstate too large for the backward");
     *bytes = (d.b == 0 || d.L == 0) ? 0 : ssd::backward_workspace_bytes(d);
     return SSD_OK;
 }
@@ -331,7 +331,7 @@ ssd_status_t ssd_chunk_scan_bwd(const void* x, const float* dt, const float* A, 
     ssd_status_t st = check_dims(dims, 0, false, dtype, &d, &t);
     if (st != SSD_OK) return st;
     if (!ssd::backward_supported(d))
-        return fail(SSD_ERR_UNSUPPORTED, "the backward needs headdim * dstate <= 8192");
+        return fail(SSD_ERR_UNSUPPORTED, "dstate too large for the backward");
     REQUIRE_PTR(A); REQUIRE_PTR(D); REQUIRE_PTR(dA); REQUIRE_PTR(dD);
     OPTIONAL_PTR(init_states); OPTIONAL_PTR(dfinal_states); OPTIONAL_PTR(dinit_states);
     if (d.b > 0 && d.L > 0) {

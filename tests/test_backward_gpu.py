@@ -57,9 +57,10 @@ def test_backward_small(dtype, G, with_init, with_dfinal):
 
 
 @pytest.mark.gpu
-def test_backward_largest_state():
-    # P x N = 8192: 32 state elements per thread, one segment and a ragged one
+def test_backward_layer_states():
+    # the layers' P 64 x N 128 (8 row blocks of 8 rows), and P 128 x N 128
     _run("P64_N128", 81, 1, 130, 2, 64, 128, 1, torch.bfloat16)
+    _run("P128_N128", 84, 1, 70, 2, 128, 128, 2, torch.bfloat16)
 
 
 @pytest.mark.gpu
@@ -86,8 +87,8 @@ def test_backward_no_tokens():
 
 @pytest.mark.gpu
 def test_backward_rejects_oversized_state():
-    x = torch.zeros(1, 4, 1, 128, device="cuda", dtype=torch.bfloat16)
-    Bm = torch.zeros(1, 4, 1, 128, device="cuda", dtype=torch.bfloat16)
+    x = torch.zeros(1, 4, 1, 64, device="cuda", dtype=torch.bfloat16)
+    Bm = torch.zeros(1, 4, 1, 512, device="cuda", dtype=torch.bfloat16)
     dt = torch.zeros(1, 4, 1, device="cuda")
     one = torch.ones(1, device="cuda")
     with pytest.raises(ssd.SSDError) as e:
