@@ -190,3 +190,51 @@ def test_binding_refuses_cpu_tensors(lib):
     with pytest.raises(ValueError, match="CUDA"):
         ssd.ssd_chunk_scan_fwd(x, torch.zeros(1, 64, 2), torch.zeros(2), torch.zeros(1, 64, 1, 8),
                                torch.zeros(1, 64, 1, 8), torch.zeros(2), 64)
+
+
+# ------------------------------------------------------------------ backward
+def _bwd_ws(dims, dt):
+    n = ctypes.c_size_t(0)
+    st = ssd.load().ssd_chunk_scan_bwd_workspace_size(ctypes.byref(dims), dt, ctypes.byref(n))
+    return st, n.value
+
+
+@pytest.mark.parametrize("b,L,H,P,N,G,dt", [
+    (8, 2048, 24, 64, 128, 1, ssd.SSD_BF16),    # 8 rows of 128 a CTA, 32 segments
+    (2, 150, 4, 16, 32, 2, ssd.SSD_F32),        # 16 rows (all of P) a CTA, 3 segments
+    (1, 65, 6, 12, 20, 3, ssd.SSD_BF16),        # 12 rows (P < 1024 / N), 2 segments
+    (1, 70, 2, 128, 128, 2, ssd.SSD_BF16),      # 8 rows a CTA, 16 row blocks
+])
+def test_backward_workspace_size_formula(lib, b, L, H, P, N, G, dt):
+    # per (batch, head, block of R = min(P, 1024 / N) state rows): fp32
+    # checkpoints every 64 tokens plus one 64-token segment of states
+    st, n = _bwd_ws(ssd.make_dims(b, L, H, P, N, G), dt)
+    assert st == ssd.SSD_OK
+    R = min(P, 1024 // N)
+    blocks = b * H * ((P + R - 1) // R)
+    assert n == blocks * ((L + 63) // 64 + 64) * R * N * 4
+
+
+def test_backward_workspace_zero_for_empty(lib):
+    assert _bwd_ws(ssd.make_dims(0, 100, 4, 8, 8, 1), ssd.SSD_F32) == (ssd.SSD_OK, 0)
+    assert _bwd_ws(ssd.make_dims(2, 0, 4, 8, 8, 1), ssd.SSD_BF16) == (ssd.SSD_OK, 0)
+
+
+def test_backward_rejects_bad_arguments_before_launching(lib):
+    L = ssd.load()
+    dims = ssd.make_dims(1, 64, 4, 8, 8, 1)
+    bad = ssd.make_dims(1, 64, 4, 8, 8, 3)          # H % G != 0
+    big = ssd.make_dims(1, 64, 4, 8, 512, 1)        # dstate > 256
+    null16 = [None] * 16
+
+    def call(d, ws=None, wsb=0, args=null16):
+        return L.ssd_chunk_scan_bwd(*args, ctypes.byref(d), ssd.SSD_BF16, ws, wsb, None)
+    assert call(bad) == ssd.SSD_ERR_INVALID_ARG
+    assert call(big) == ssd.SSD_ERR_UNSUPPORTED
+    assert call(dims) == ssd.SSD_ERR_INVALID_ARG     # NULL A, D, dA, dD
+    # valid-looking (never dereferenced) aligned addresses, but a short workspace
+    fake = [ctypes.c_void_p(0x10000 * (i + 1)) for i in range(16)]
+    fake[6] = fake[8] = fake[15] = None              # init, dfinal, dinit are optional
+    st = call(dims, ctypes.c_void_p(0x1000000), 16, fake)
+    assert st == ssd.SSD_ERR_INVALID_ARG
+    assert b"workspace_bytes" in L.ssd_last_error_detail()
