@@ -1,10 +1,8 @@
 """Failure detection without a GPU fault: a bounded device-side wait that
 runs out reports SSD_ERR_TIMEOUT through the status word, the context stays
 usable, and the host-side checks reject bad calls before any launch."""
-import ctypes
 
 import pytest
-import torch
 
 from parity import TOL, gpu_fwd, oracle_fwd, rel_err
 from ssd_chunked_scan_02_b200 import build as ssd_build

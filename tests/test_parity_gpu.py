@@ -4,7 +4,6 @@ Error metric (per tensor): max|gpu - oracle| / max|oracle|; bound 5e-3 for
 bf16 storage, 1e-4 for fp32.  Small cases compare every element; the full
 workload sizes compare sampled (batch, head) pairs, each recomputed by the
 oracle over the whole sequence."""
-import math
 
 import numpy as np
 import pytest
