@@ -60,8 +60,14 @@ def fwd_model(w):
 
 
 def kernel_bytes(w):
-    """Bytes each kernel of the three-kernel forward must move (its inputs
-    and outputs, each once)."""
+    """Per kernel of either data flow: (alg, io).
+
+    alg: the kernel's share of the forward's minimum bytes (bytes_min: x, y,
+    B, C, dt, initial and final states, each once) -- the inputs and outputs
+    of the layer that the kernel itself must read or write.  Intermediates
+    (chunk states, entering states) count zero: a better data flow removes
+    them.  io: everything the kernel reads and writes, intermediates
+    included, each once."""
     b, L, H, P, N, G, Q = w.batch, w.seqlen, w.nheads, w.headdim, w.dstate, w.ngroups, w.chunk
     sx = 2 if w.dtype == "bf16" else 4
     T = (L + Q - 1) // Q
@@ -71,14 +77,17 @@ def kernel_bytes(w):
     dt = b * L * H * 4
     init = 4 * b * H * P * N * int(w.with_init)
     fin = 4 * b * H * P * N * int(w.want_final)
+    ld = 4 * b * T * H
     return {
-        "chunk_state": x + bc + dt + 4 * ns + 4 * b * T * H,
-        "state_pass": 4 * ns + 4 * b * T * H + sx * ns + init + fin,
-        "chunk_out": 2 * x + 2 * bc + dt + sx * ns,
+        "chunk_state": (x + bc + dt, x + bc + dt + 4 * ns + ld),
+        "state_pass": (init + fin, 4 * ns + ld + sx * ns + init + fin),
+        "state_walk": (x + bc + dt + init + fin, x + bc + dt + sx * ns + init + fin),
+        "chunk_out": (2 * x + 2 * bc + dt, 2 * x + 2 * bc + dt + sx * ns),
     }
 
 
 KERNEL_SOURCES = {
+    "state_walk": ["state_walk_tc.cu", "sm100.cuh"],
     "chunk_state": ["chunk_state_tc.cu", "sm100.cuh"],
     "state_pass": ["state_pass.cu"],
     "chunk_out": ["chunk_out_tc.cu", "sm100.cuh"],
@@ -239,6 +248,85 @@ def cpu_oracle_sample(w, inp_cpu, seconds_budget: float = 12.0):
     return tok_s, desc, cores
 
 
+def cpu_model() -> str:
+    """The host CPU's model name (lscpu), or the platform's processor string."""
+    try:
+        out = subprocess.run(["lscpu"], capture_output=True, text=True, timeout=10).stdout
+        for line in out.splitlines():
+            if line.lower().startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except (OSError, subprocess.SubprocessError):
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
+def cpu_baselines(w, inp_cpu, budget_s: float = 12.0):
+    """The oracle timed on the host as it stands (a reported baseline, not a
+    target), on bounded samples of each workload:
+      - the 2.7B layer on all cores (batch 0, all heads, the whole sequence)
+        and on one thread (batch 0, heads 0..7);
+      - the 130M layer on all cores (batch 0, all heads);
+      - decode (b256 H80 P64 N128): 16 sequences x 1024 steps of the same
+        recurrence on all cores, reported per step of the full batch.
+    Returns the cpu_baseline object of the bench line."""
+    import oracle
+    from ssd_chunked_scan_02_b200 import inputs
+    cores = os.cpu_count() or 1
+    tok_s, desc, cores = cpu_oracle_sample(w, inp_cpu, seconds_budget=budget_s)
+
+    def timed(fn, budget):
+        t0 = time.perf_counter()
+        reps = 0
+        while True:
+            fn()
+            reps += 1
+            el = time.perf_counter() - t0
+            if el > budget or reps >= 1000:
+                return el / reps, reps
+
+    # one thread, 8 heads of batch 0 of the same layer
+    hs = 8
+    one = [oracle._f64(inp_cpu[k][0:1, :, :hs]) for k in ("x", "dt")]
+    args1 = [one[0], one[1], oracle._f64(inp_cpu["A"][:hs]), oracle._f64(inp_cpu["B"][0:1]),
+             oracle._f64(inp_cpu["C"][0:1]), oracle._f64(inp_cpu["D"][:hs])]
+    init1 = oracle._f64(inp_cpu["init"][0:1, :hs]) if inp_cpu.get("init") is not None else None
+    per1, reps1 = timed(lambda: oracle.recurrence(*args1, init1, threads=1), 4.0)
+    tok1 = w.seqlen * hs / w.nheads / per1
+    # the 130M layer, batch 0, all heads, all cores
+    w1 = inputs.LAYER_130M
+    i1 = inputs.make_inputs(w1.with_(batch=1))
+    a130 = [oracle._f64(i1[k]) for k in ("x", "dt", "A", "B", "C", "D")]
+    per130, reps130 = timed(lambda: oracle.recurrence(*a130, None, threads=cores), 3.0)
+    # decode: 16 sequences x 1024 steps
+    dw = inputs.DECODE_2P7B
+    nb, steps = 16, dw.steps
+    dd = inputs.make_inputs(inputs.Workload("decode_cpu_sample", nb, steps, dw.nheads, dw.headdim,
+                                            dw.dstate, dw.ngroups, 256, dw.dtype, with_init=True,
+                                            want_final=True, seed=dw.seed))
+    adec = [oracle._f64(dd[k]) for k in ("x", "dt", "A", "B", "C", "D")]
+    idec = oracle._f64(dd["init"])
+    perd, _ = timed(lambda: oracle.recurrence(*adec, idec, threads=cores), 1.0)
+    step_s_full = perd / steps * (dw.batch / nb)          # one step of the full b=256 batch
+    dec_bytes = 2 * 4 * dw.batch * dw.nheads * dw.headdim * dw.dstate
+    return {
+        "value": tok_s, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc,
+        "cpu_model": cpu_model(),
+        "single_thread": {"value": tok1, "unit": UNIT, "cores": 1,
+                          "sample": f"batch 0, heads 0..{hs - 1} of {w.nheads}, L={w.seqlen} "
+                                    f"({reps1} reps, {per1:.3f} s each); tokens/s scaled by heads"},
+        "other_configs": [
+            {"workload": w1.name, "value": w1.seqlen / per130, "unit": UNIT, "cores": cores,
+             "sample": f"batch 0 of {w1.batch}, all {w1.nheads} heads, L={w1.seqlen} "
+                       f"({reps130} reps, {per130:.3f} s each)"},
+            {"workload": dw.name, "ms_per_step": 1e3 * step_s_full, "cores": cores,
+             "state_gbs": dec_bytes / step_s_full / 1e9,
+             "sample": f"{nb} of {dw.batch} sequences x {steps} steps as one recurrence "
+                       f"({perd:.2f} s); per step of the full batch by scaling"},
+        ],
+    }
+
+
 # ---------------------------------------------------------------- reference arm
 def run_reference(args):
     """The reference arm here is the fp64 CPU oracle, timed as it stands."""
@@ -309,7 +397,10 @@ def measure_config(w, dev, stream, flush, reps, world, rank):
     ms = max_over_ranks(sum(st.elapsed_time(en) for st, en in evs), world) / reps
     f_alg, f_dense, bytes_min = fwd_model(w)
     t = ms * 1e-3
-    out = {"workload": w.name, "ms_per_step": ms, "tokens_per_s": world * w.tokens / t,
+    flow = ssd.ssd_chunk_scan_fwd_data_flow(dims, w.chunk, inp["x"].dtype)
+    out = {"workload": w.name, "data_flow": {ssd.SSD_FLOW_WALK_OUTPUT: "walk+output",
+                                              ssd.SSD_FLOW_TC_THREE_KERNEL: "three-kernel"}
+           .get(flow, "simt"), "ms_per_step": ms, "tokens_per_s": world * w.tokens / t,
            "tflops_alg": f_alg / t / 1e12, "tflops_dense": f_dense / t / 1e12,
            "bytes_min": bytes_min, "hbm_gbs_at_bytes_min": bytes_min / t / 1e9}
     del inp, y, fin, ws
@@ -368,6 +459,62 @@ def measure_backward(w, dev, stream, flush, reps, world, rank, peak_gbs):
     del inp, dy, ws
     torch.cuda.empty_cache()
     return out
+
+
+# ---------------------------------------------------------------- per-kernel timing
+FLOW_KERNELS = {1: ("chunk_state", "state_pass", "chunk_out"), 2: ("state_walk", "chunk_out")}
+
+
+def kernel_times(w, flow, inp, y, fin, dims, dev, stream, flush, reps):
+    """Mean device time (ms) of each kernel of a tensor-core data flow, each
+    launched through its own entry point, with CUDA events on the launching
+    stream between the launches."""
+    import ctypes
+
+    import torch
+    from ssd_chunked_scan_02_b200 import ssd
+    x, dt, A, Bm, Cm, D, init = (inp[k] for k in ("x", "dt", "A", "B", "C", "D", "init"))
+    T = (w.seqlen + w.chunk - 1) // w.chunk
+    shape = (w.batch, T, w.nheads, w.headdim, w.dstate)
+    prev_buf = torch.empty(shape, device=dev, dtype=x.dtype)
+    S_buf = (torch.empty(shape, device=dev, dtype=torch.float32)
+             if flow == ssd.SSD_FLOW_TC_THREE_KERNEL else None)
+    ld_buf = torch.empty((w.batch, T, w.nheads), device=dev, dtype=torch.float32)
+    lib = ssd.load()
+    sp = ctypes.c_void_p(stream.cuda_stream)
+    P = lambda t: ctypes.c_void_p(t.data_ptr()) if t is not None else None
+    names = FLOW_KERNELS[flow]
+    kt = {k: [] for k in names}
+
+    def launch(k):
+        if k == "chunk_state":
+            st = lib.ssd_chunk_state_fwd(P(x), P(dt), P(A), P(Bm), w.chunk, P(S_buf), P(ld_buf),
+                                         ctypes.byref(dims), ssd.SSD_BF16, sp)
+        elif k == "state_pass":
+            st = lib.ssd_state_passing_fwd(P(S_buf), P(ld_buf), P(init), P(prev_buf), P(fin),
+                                           w.chunk, ctypes.byref(dims), ssd.SSD_BF16, sp)
+        elif k == "state_walk":
+            st = lib.ssd_state_walk_fwd(P(x), P(dt), P(A), P(Bm), P(init), P(prev_buf), P(fin),
+                                        w.chunk, ctypes.byref(dims), ssd.SSD_BF16, sp)
+        else:
+            st = lib.ssd_chunk_output_fwd(P(x), P(dt), P(A), P(Bm), P(Cm), P(D), P(prev_buf),
+                                          w.chunk, P(y), ctypes.byref(dims), ssd.SSD_BF16, sp)
+        if st != ssd.SSD_OK:
+            raise RuntimeError(f"{k}: {ssd.status_name(st)}: {lib.ssd_last_error_detail()}")
+
+    for r in range(reps + 2):
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)]
+        flush.zero_()
+        ev[0].record(stream)
+        for i, k in enumerate(names):
+            launch(k)
+            ev[i + 1].record(stream)
+        torch.cuda.synchronize(dev)
+        if r >= 2:
+            for i, k in enumerate(names):
+                kt[k].append(ev[i].elapsed_time(ev[i + 1]))
+    del prev_buf, S_buf, ld_buf
+    return {k: statistics.mean(v) for k, v in kt.items()}
 
 
 # ---------------------------------------------------------------- GPU arm
@@ -437,41 +584,20 @@ def main():
     clocks = sampler.stop() if sampler else None
     ms_per_step = total_ms / args.steps
 
-    # ---- per-kernel times (same stream, CUDA events between the three launches)
-    T = (w.seqlen + w.chunk - 1) // w.chunk
-    S_buf = torch.empty((w.batch, T, w.nheads, w.headdim, w.dstate), device=dev,
-                        dtype=torch.float32)
-    ld_buf = torch.empty((w.batch, T, w.nheads), device=dev, dtype=torch.float32)
-    prev_buf = torch.empty((w.batch, T, w.nheads, w.headdim, w.dstate), device=dev,
-                           dtype=x.dtype)
-    lib = ssd.load()
-    import ctypes
-    sp = ctypes.c_void_p(stream.cuda_stream)
-    P = lambda t: ctypes.c_void_p(t.data_ptr()) if t is not None else None
-    kt = {"chunk_state": [], "state_pass": [], "chunk_out": []}
-    reps = max(5, args.steps // 2)
-    for r in range(reps + 2):
-        ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
-        flush.zero_()
-        ev[0].record(stream)
-        lib.ssd_chunk_state_fwd(P(x), P(dt), P(A), P(Bm), w.chunk, P(S_buf), P(ld_buf),
-                                ctypes.byref(dims), ssd.SSD_BF16, sp)
-        ev[1].record(stream)
-        lib.ssd_state_passing_fwd(P(S_buf), P(ld_buf), P(init), P(prev_buf), P(fin), w.chunk,
-                                  ctypes.byref(dims), ssd.SSD_BF16, sp)
-        ev[2].record(stream)
-        lib.ssd_chunk_output_fwd(P(x), P(dt), P(A), P(Bm), P(Cm), P(D), P(prev_buf), w.chunk,
-                                 P(y), ctypes.byref(dims), ssd.SSD_BF16, sp)
-        ev[3].record(stream)
-        torch.cuda.synchronize(dev)
-        if r >= 2:
-            kt["chunk_state"].append(ev[0].elapsed_time(ev[1]))
-            kt["state_pass"].append(ev[1].elapsed_time(ev[2]))
-            kt["chunk_out"].append(ev[2].elapsed_time(ev[3]))
-    kmean = {k: statistics.mean(v) for k, v in kt.items()}
+    # ---- per-kernel times: the kernels of the forward's data flow, launched
+    # one by one through their entry points on the same stream, CUDA events
+    # between them (L2 flushed before each sequence)
+    flow = ssd.ssd_chunk_scan_fwd_data_flow(dims, w.chunk, x.dtype)
+    kmean = kernel_times(w, flow, inp, y, fin, dims, dev, stream, flush, max(5, args.steps // 2))
+    # the other tensor-core flow, for comparison (not part of the forward)
+    alt_flow = (ssd.SSD_FLOW_TC_THREE_KERNEL if flow == ssd.SSD_FLOW_WALK_OUTPUT
+                else ssd.SSD_FLOW_WALK_OUTPUT)
+    kalt = kernel_times(w, alt_flow, inp, y, fin, dims, dev, stream, flush,
+                        max(5, args.steps // 4))
     dom = max(kmean, key=kmean.get)
     kb = kernel_bytes(w)
-    dom_gbs = kb[dom] / (kmean[dom] * 1e-3) / 1e9
+    dom_gbs = kb[dom][0] / (kmean[dom] * 1e-3) / 1e9
+    dom_io_gbs = kb[dom][1] / (kmean[dom] * 1e-3) / 1e9
 
     # ---- decode step (b=256, H=80, P=64, N=128), state resident
     dw = inputs.DECODE_2P7B
@@ -566,6 +692,27 @@ def main():
     e.record(s_in)
     torch.cuda.synchronize(dev)
     e2e_ms = max_over_ranks(s.elapsed_time(e), world) / e2e_steps
+    # the link alone: one host->device copy of a step's input bytes and one
+    # device->host copy of its output bytes (pinned buffers), each timed by
+    # itself, to show what bounds the end-to-end number
+    link = {}
+    for name, nbytes, src_host in (("h2d", h2d, True), ("d2h", d2h, False)):
+        hb = torch.empty(nbytes, dtype=torch.uint8, pin_memory=True)
+        db = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+        ts = []
+        for r in range(4):
+            a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            if src_host:
+                db.copy_(hb, non_blocking=True)
+            else:
+                hb.copy_(db, non_blocking=True)
+            z.record(stream)
+            torch.cuda.synchronize(dev)
+            if r:
+                ts.append(a.elapsed_time(z))
+        link[name] = {"ms": statistics.mean(ts), "gbs": nbytes / (statistics.mean(ts) * 1e-3) / 1e9}
+        del hb, db
 
     # ---- the other configurations of the metric: 130M layer and the N = 64 sweep
     extra = None
@@ -586,8 +733,7 @@ def main():
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         inp_cpu = {k: (v.cpu() if v is not None else None) for k, v in inp.items()}
-        tok_s, desc, cores = cpu_oracle_sample(w, inp_cpu)
-        cpu = {"value": tok_s, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc}
+        cpu = cpu_baselines(w, inp_cpu)
 
     if rank == 0:
         f_alg, f_dense, bytes_min = fwd_model(w)
@@ -610,23 +756,36 @@ def main():
                        "pct_bf16_peak_dense": 100 * f_dense / t / 1e12 / pk["bf16_tflops"],
                        "pct_bf16_peak_alg": 100 * f_alg / t / 1e12 / pk["bf16_tflops"],
                        "peak_tflops": pk["bf16_tflops"], "peak_source": pk["source"]},
+            "roofline_step": {"bound": "hbm", "bytes_min": bytes_min,
+                              "achieved_gbs": bytes_min / t / 1e9,
+                              "t_min_ms": 1e3 * t_roof, "frac": t_roof / t,
+                              "note": "the whole forward against its minimum bytes: the "
+                                      "headline roofline figure"},
             "roofline": {"bound": bound, "kernel": dom, "achieved": dom_gbs, "peak": peak_gbs,
                          "unit": "GB/s", "frac": dom_gbs / peak_gbs,
                          "traffic": traffic_for(dom, w.name),
-                         "alg_bytes_per_launch": kb[dom], "ms_per_launch": kmean[dom],
-                         "peak_source": pk["source"]},
-            "roofline_step": {"bound": "hbm", "bytes_min": bytes_min,
-                              "achieved_gbs": bytes_min / t / 1e9,
-                              "t_min_ms": 1e3 * t_roof, "frac": t_roof / t},
+                         "alg_bytes_per_launch": kb[dom][0],
+                         "alg_bytes": "the kernel's share of bytes_min (layer inputs and "
+                                      "outputs it touches, each once; intermediates count 0)",
+                         "io_bytes_per_launch": kb[dom][1],
+                         "io_gbs": dom_io_gbs, "io_frac": dom_io_gbs / peak_gbs,
+                         "ms_per_launch": kmean[dom], "peak_source": pk["source"]},
+            "data_flow": {ssd.SSD_FLOW_WALK_OUTPUT: "walk+output",
+                          ssd.SSD_FLOW_TC_THREE_KERNEL: "three-kernel"}.get(flow, "simt"),
             "kernels_ms": kmean,
+            "kernels_ms_other_flow": kalt,
             "decode": {"workload": dw.name, "ms_per_step": dec_ms, "gbs": dec_gbs,
                        "frac_hbm": dec_gbs / peak_gbs, "bytes_per_step": dec_bytes},
             "e2e": {"value": world * w.tokens / (e2e_ms * 1e-3), "unit": UNIT,
-                    "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                    "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "device_ms_per_step": ms_per_step, "link": link,
+                    "bound": "host<->device copies: the layer's input and output are as "
+                             "large as its own HBM traffic, so the copies (h2d and d2h "
+                             "overlapping, full duplex) take far longer than the forward"},
             "other_configs": extra,
             "backward": bwd,
             "cpu_baseline": cpu,
-            "gpu_launches": 3 * args.steps,
+            "gpu_launches": len(FLOW_KERNELS.get(flow, (0, 0, 0))) * args.steps,
             "clocks": clocks,
         }
         print(json.dumps(line))

@@ -24,13 +24,26 @@
  *    G = ngroups, T = ceil(L / chunk_size)):
  *        x, y            (b, L, H, P)   element type = dtype
  *        dt              (b, L, H)      fp32, already positive (no softplus is applied)
- *        A, D            (H)            fp32
+ *        A, D            (H)            fp32 (A <= 0: a decaying state, see below)
  *        B, C            (b, L, G, N)   element type = dtype
  *        states          (b, H, P, N)   fp32 (init_states, final_states, ssd_step's state)
  *    Head h reads B/C group g = h / (H / G).
  *  - dtype: SSD_F32 (all fp32; exact fp32 arithmetic) or SSD_BF16 (x, B, C, y
  *    in bf16; products on the tensor cores with fp32 accumulation; decays,
  *    prefix sums, the inter-chunk recurrence and all states in fp32).
+ *  - A: the model's regime is A <= 0 (exp(dt*A) <= 1); the tensor-core
+ *    kernels factorise the decay through per-row and per-column factors that
+ *    are exact for any A <= 0.  A > 0 (a growing state) is computed
+ *    correctly as long as the growth over one chunk, exp(sum dt*A), stays
+ *    below 2^60; beyond that the result overflows fp32 in any case.
+ *  - Sizes are passed as a pointer to ssd_dims_t (a by-value struct of six
+ *    int64 is awkward for some FFI layers; the pointee is only read, during
+ *    the call), and the stream as void* (a cudaStream_t, so that this header
+ *    does not need the CUDA headers).
+ *  - Device: every pointer must belong to the CUDA device that is current
+ *    on the calling thread; the library looks up per-device state (tensor
+ *    maps, status word, built-in scratch) for that device and assumes its
+ *    primary context (do not call cudaDeviceReset between calls).
  *  - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
  *    stream) and runs asynchronously: no call synchronises the device.
  *  - Errors: arguments are validated on the host before anything is
@@ -62,7 +75,7 @@ typedef enum {
     SSD_ERR_INVALID_ARG = 1,  /* null pointer, bad size, misalignment, too-small workspace */
     SSD_ERR_UNSUPPORTED = 2,  /* well-formed but outside what the kernels implement */
     SSD_ERR_CUDA = 3,         /* a CUDA runtime/driver call or a launch failed */
-    SSD_ERR_TIMEOUT = 4       /* reserved: a bounded device-side wait gave up */
+    SSD_ERR_TIMEOUT = 4       /* a bounded device-side wait gave up (ssd_poll_device_status) */
 } ssd_status_t;
 
 typedef enum { SSD_F32 = 0, SSD_BF16 = 1 } ssd_dtype_t;
@@ -224,14 +237,16 @@ SSD_API ssd_status_t ssd_chunk_scan_bwd(const void* x, const float* dt, const fl
 SSD_API ssd_status_t ssd_poll_device_status(void* stream);
 
 /*
- * ssd_state_walk_fwd -- steps (2) and (3) fused, the way ssd_chunk_scan_fwd
- * runs them when batch x nheads / 2 fills the GPU: one CTA per (batch, head
- * pair) walks the chunks in order keeping the running fp32 state on chip
- * (tensor memory), and writes only prev_states (b,T,H,P,N) bf16 -- the state
- * entering each chunk, same contents as ssd_state_passing_fwd's -- and, if
- * final_states is non-NULL, the fp32 state after the last chunk.  Covers the
- * tensor-core sizes only (SSD_BF16, chunk_size 128 or 256, headdim 64, dstate
- * 64 or 128, nheads / ngroups even); other sizes return SSD_ERR_UNSUPPORTED.
+ * ssd_state_walk_fwd -- steps (2) and (3) fused: one CTA per (batch, head
+ * pair) walks the chunks in order keeping the running fp32 state and each
+ * chunk's contribution on chip (tensor memory), and writes only prev_states
+ * (b,T,H,P,N) bf16 -- the state entering each chunk, same contents as
+ * ssd_state_passing_fwd's -- and, if final_states is non-NULL, the fp32
+ * state after the last chunk.  ssd_chunk_scan_fwd runs it (followed by
+ * ssd_chunk_output_fwd's kernel) whenever ssd_chunk_scan_fwd_data_flow
+ * reports SSD_FLOW_WALK_OUTPUT.  Covers the tensor-core sizes only
+ * (SSD_BF16, chunk_size 128 or 256, headdim 64, dstate 64 or 128, nheads /
+ * ngroups even); other sizes return SSD_ERR_UNSUPPORTED.
  */
 SSD_API ssd_status_t ssd_state_walk_fwd(const void* x, const float* dt, const float* A,
                                         const void* B, const float* init_states,
@@ -251,6 +266,25 @@ SSD_API ssd_status_t ssd_debug_expire_wait(unsigned int polls, void* stream);
 /* Which kernel family ssd_chunk_scan_fwd uses for these sizes:
  * 1 = tcgen05 tensor-core kernels, 0 = SIMT fp32 kernels, -1 = rejected. */
 SSD_API int ssd_chunk_scan_fwd_uses_tensor_cores(const ssd_dims_t* dims, int chunk_size,
+                                         ssd_dtype_t dtype);
+
+/* Which data flow ssd_chunk_scan_fwd takes for these sizes (decided from the
+ * sizes alone; the workspace size follows from it):
+ *   SSD_FLOW_WALK_OUTPUT     state walk (steps 2+3 on chip, entering states
+ *                            written in bf16) then the tensor-core output
+ *                            kernel (steps 1+4): two launches;
+ *   SSD_FLOW_TC_THREE_KERNEL tensor-core chunk states (fp32, in the
+ *                            workspace), the state pass, the tensor-core
+ *                            output kernel: three launches;
+ *   SSD_FLOW_SIMT            the same three steps as exact-fp32 SIMT kernels;
+ *   -1                       the sizes are rejected.
+ * The walk is taken when there are enough (batch, head pair) walkers to
+ * cover the GPU and enough chunks per walker (few long sequences keep the
+ * three-kernel flow, whose state pass parallelises over state elements). */
+#define SSD_FLOW_SIMT 0
+#define SSD_FLOW_TC_THREE_KERNEL 1
+#define SSD_FLOW_WALK_OUTPUT 2
+SSD_API int ssd_chunk_scan_fwd_data_flow(const ssd_dims_t* dims, int chunk_size,
                                          ssd_dtype_t dtype);
 
 #ifdef __cplusplus

@@ -452,8 +452,12 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
                 const float r = (t == 1) ? cs[127] : 0.f;
                 // the tile's decay span decides the path (the same for every thread)
                 const float c_first = cs[row0], c_last = cs[row0 + 127];
-                const bool fast = fabsf(c_last - c_first) <= kFastSpan;
                 const float r1 = 0.5f * (c_first + c_last);
+                // fast path: the tile's own factors stay within 2^+-60; for t = 1 the
+                // left block's b_j = 2^(r1 - cs_j) dt_j must too, which holds for any
+                // A <= 0 (cs_j >= r1) and bounds a growing state (A > 0)
+                const bool fast = fabsf(c_last - c_first) <= kFastSpan &&
+                                  (t == 0 || r1 - cs[0] <= 0.5f * kFastSpan);
                 if (hf == 0) {
                     if (t == 1) s_beta[m] = fast_exp2((fast ? r1 : r) - cs[m]) * hdt[m];
                     s_al[f * 128 + m] = fast_exp2(fast ? cs_i : cs_i - r);

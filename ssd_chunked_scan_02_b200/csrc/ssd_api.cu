@@ -67,6 +67,20 @@ ssd_status_t check_dims(const ssd_dims_t* dims, int chunk, bool need_chunk, ssd_
     return SSD_OK;
 }
 
+bool tc_eligible(const ssd::Dims& d, ssd::Elt t) { return ssd::tc_supported(d, t); }
+
+// The forward's data flow for these sizes (decided from the sizes alone, so
+// the workspace size needs no device).
+enum class Flow { Simt = 0, ThreeKernel = 1, Walk = 2 };
+
+Flow pick_flow(const ssd::Dims& d, ssd::Elt t) {
+    if (!tc_eligible(d, t)) return Flow::Simt;
+    return ssd::walk_preferred(d) ? Flow::Walk : Flow::ThreeKernel;
+}
+
+// Workspace regions (each 256-byte aligned).  The three-kernel flows keep the
+// chunk states (fp32) and log-decays; the walk keeps its chunk states on chip
+// and needs only the entering states.
 struct WsLayout {
     size_t states, logdecay, prev, total;
 };
@@ -75,12 +89,46 @@ WsLayout ws_layout(const ssd::Dims& d, ssd::Elt t) {
     const size_t nstate = (size_t)(d.b * d.T * d.H) * (size_t)(d.P * d.N);
     WsLayout w;
     w.states = 0;
-    w.logdecay = round_up(nstate * 4, 256);
-    w.prev = w.logdecay + round_up((size_t)(d.b * d.T * d.H) * 4, 256);
+    if (pick_flow(d, t) == Flow::Walk) {
+        w.logdecay = 0;
+        w.prev = 0;
+    } else {
+        w.logdecay = round_up(nstate * 4, 256);
+        w.prev = w.logdecay + round_up((size_t)(d.b * d.T * d.H) * 4, 256);
+    }
     w.total = w.prev + round_up(nstate * elt_size(t), 256);
     if (nstate == 0) w.total = 0;
     return w;
 }
+
+// A tensor handed to the kernels must be device memory of the current device:
+// tensor maps, the status word and scratch are looked up per current device,
+// and a kernel on one GPU given another GPU's (or unregistered host) memory
+// faults or reads the wrong memory.  Checked once per call, after every other
+// validation, on the call's main input.
+ssd_status_t check_current_device(const void* p, const char* name) {
+    cudaPointerAttributes a{};
+    cudaError_t e = cudaPointerGetAttributes(&a, p);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return cuda_fail(e, "cudaPointerGetAttributes");
+    }
+    if (a.type != cudaMemoryTypeDevice && a.type != cudaMemoryTypeManaged)
+        return fail(SSD_ERR_INVALID_ARG, "%s is not device memory", name);
+    int dev = -1;
+    e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (a.type == cudaMemoryTypeDevice && a.device != dev)
+        return fail(SSD_ERR_INVALID_ARG, "%s is on device %d but device %d is current", name,
+                    a.device, dev);
+    return SSD_OK;
+}
+
+#define REQUIRE_DEVICE(p)                                                                \
+    do {                                                                                 \
+        ssd_status_t st_dev_ = check_current_device((p), #p);                            \
+        if (st_dev_ != SSD_OK) return st_dev_;                                           \
+    } while (0)
 
 #define REQUIRE_PTR(p)                                                                   \
     do {                                                                                 \
@@ -92,8 +140,6 @@ WsLayout ws_layout(const ssd::Dims& d, ssd::Elt t) {
         if ((p) && !aligned16(p))                                                        \
             return fail(SSD_ERR_INVALID_ARG, "%s is not 16-byte aligned", #p);           \
     } while (0)
-
-bool tc_eligible(const ssd::Dims& d, ssd::Elt t) { return ssd::tc_supported(d, t); }
 
 }  // namespace
 
@@ -140,6 +186,16 @@ int ssd_chunk_scan_fwd_uses_tensor_cores(const ssd_dims_t* dims, int chunk_size,
     return tc_eligible(d, t) ? 1 : 0;
 }
 
+int ssd_chunk_scan_fwd_data_flow(const ssd_dims_t* dims, int chunk_size, ssd_dtype_t dtype) {
+    ssd::Dims d{}; ssd::Elt t = ssd::Elt::BF16;
+    if (check_dims(dims, chunk_size, true, dtype, &d, &t) != SSD_OK) return -1;
+    switch (pick_flow(d, t)) {
+        case Flow::Walk: return SSD_FLOW_WALK_OUTPUT;
+        case Flow::ThreeKernel: return SSD_FLOW_TC_THREE_KERNEL;
+        default: return SSD_FLOW_SIMT;
+    }
+}
+
 ssd_status_t ssd_chunk_scan_fwd(const void* x, const float* dt, const float* A, const void* B,
                                 const void* C, const float* D, int chunk_size,
                                 const float* init_states, void* y, float* final_states,
@@ -166,13 +222,22 @@ ssd_status_t ssd_chunk_scan_fwd(const void* x, const float* dt, const float* A, 
                     workspace_bytes, w.total);
     REQUIRE_PTR(workspace);
     if (!aligned16(workspace)) return fail(SSD_ERR_INVALID_ARG, "workspace not 16-byte aligned");
+    REQUIRE_DEVICE(x);
     char* ws = static_cast<char*>(workspace);
     float* states = reinterpret_cast<float*>(ws + w.states);
     float* logdecay = reinterpret_cast<float*>(ws + w.logdecay);
     void* prev = ws + w.prev;
 
     cudaError_t e;
-    if (tc_eligible(d, t)) {
+    const Flow flow = pick_flow(d, t);
+    if (flow == Flow::Walk) {
+        e = ssd::launch_state_walk_tc(x, dt, A, B, init_states, prev, final_states, d, s);
+        if (e != cudaSuccess) return cuda_fail(e, "state-walk kernel (tcgen05)");
+        e = ssd::launch_chunk_out_tc(x, dt, A, B, C, D, prev, y, d, s);
+        if (e != cudaSuccess) return cuda_fail(e, "chunk-output kernel (tcgen05)");
+        return SSD_OK;
+    }
+    if (flow == Flow::ThreeKernel) {
         e = ssd::launch_chunk_state_tc(x, dt, A, B, states, logdecay, d, s);
         if (e != cudaSuccess) return cuda_fail(e, "chunk-state kernel (tcgen05)");
         e = ssd::launch_state_pass(states, logdecay, init_states, prev, final_states, d, t, s);
@@ -200,6 +265,7 @@ ssd_status_t ssd_chunk_state_fwd(const void* x, const float* dt, const float* A,
     if (d.b == 0 || d.L == 0) return SSD_OK;
     REQUIRE_PTR(x); REQUIRE_PTR(dt); REQUIRE_PTR(A); REQUIRE_PTR(B);
     REQUIRE_PTR(chunk_states); REQUIRE_PTR(chunk_logdecay);
+    REQUIRE_DEVICE(x);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaError_t e = tc_eligible(d, t)
                         ? ssd::launch_chunk_state_tc(x, dt, A, B, chunk_states, chunk_logdecay, d, s)
@@ -226,6 +292,7 @@ ssd_status_t ssd_state_passing_fwd(const float* chunk_states, const float* chunk
         return e == cudaSuccess ? SSD_OK : cuda_fail(e, "final-state copy");
     }
     REQUIRE_PTR(chunk_states); REQUIRE_PTR(chunk_logdecay); REQUIRE_PTR(prev_states);
+    REQUIRE_DEVICE(chunk_states);
     cudaError_t e = ssd::launch_state_pass(chunk_states, chunk_logdecay, init_states, prev_states,
                                            final_states, d, t, s);
     return e == cudaSuccess ? SSD_OK : cuda_fail(e, "state-passing kernel");
@@ -242,6 +309,7 @@ ssd_status_t ssd_chunk_output_fwd(const void* x, const float* dt, const float* A
     if (d.b == 0 || d.L == 0) return SSD_OK;
     REQUIRE_PTR(x); REQUIRE_PTR(dt); REQUIRE_PTR(A); REQUIRE_PTR(B); REQUIRE_PTR(C);
     REQUIRE_PTR(D); REQUIRE_PTR(prev_states); REQUIRE_PTR(y);
+    REQUIRE_DEVICE(x);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaError_t e = tc_eligible(d, t)
                         ? ssd::launch_chunk_out_tc(x, dt, A, B, C, D, prev_states, y, d, s)
@@ -271,6 +339,7 @@ ssd_status_t ssd_state_walk_fwd(const void* x, const float* dt, const float* A, 
                     "the state walk covers bf16, chunk 128/256, headdim 64, dstate 64/128 and an "
                     "even number of heads per group");
     REQUIRE_PTR(x); REQUIRE_PTR(dt); REQUIRE_PTR(A); REQUIRE_PTR(B); REQUIRE_PTR(prev_states);
+    REQUIRE_DEVICE(x);
     cudaError_t e = ssd::launch_state_walk_tc(x, dt, A, B, init_states, prev_states, final_states, d, s);
     return e == cudaSuccess ? SSD_OK : cuda_fail(e, "state-walk kernel");
 }
@@ -302,6 +371,7 @@ ssd_status_t ssd_step(float* state, const void* x, const float* dt, const float*
     if (d.b == 0) return SSD_OK;
     REQUIRE_PTR(state); REQUIRE_PTR(x); REQUIRE_PTR(dt); REQUIRE_PTR(A); REQUIRE_PTR(B);
     REQUIRE_PTR(C); REQUIRE_PTR(D); REQUIRE_PTR(y);
+    REQUIRE_DEVICE(state);
     cudaError_t e = ssd::launch_step(state, x, dt, A, B, C, D, y, d, t,
                                      static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? SSD_OK : cuda_fail(e, "decode-step kernel");
@@ -342,6 +412,7 @@ ssd_status_t ssd_chunk_scan_bwd(const void* x, const float* dt, const float* A, 
             return fail(SSD_ERR_INVALID_ARG, "workspace_bytes %zu < required %zu", workspace_bytes,
                         need);
         REQUIRE_PTR(workspace);
+        REQUIRE_DEVICE(x);
     }
     cudaError_t e = ssd::launch_backward(x, dt, A, B, C, D, init_states, dy, dfinal_states, dx,
                                          ddt, dA, dB, dC, dD, dinit_states,

@@ -18,7 +18,7 @@ cudaError_t launch_chunk_state_tc(const void* x, const float* dt, const float* A
 cudaError_t launch_state_walk_tc(const void* x, const float* dt, const float* A, const void* B,
                                  const float* init, void* prev, float* final_states,
                                  const Dims& d, cudaStream_t s);
-// True when the fused walk has enough (batch, head pair) walkers to fill the GPU.
+// True when the forward runs the walk: enough (batch, head pair) walkers.
 bool walk_preferred(const Dims& d);
 
 cudaError_t launch_chunk_out_tc(const void* x, const float* dt, const float* A, const void* B,

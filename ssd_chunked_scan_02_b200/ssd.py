@@ -26,7 +26,11 @@ EXPORTED = ("ssd_status_string", "ssd_last_error_detail", "ssd_chunk_scan_fwd_wo
             "ssd_chunk_scan_fwd", "ssd_step", "ssd_chunk_state_fwd", "ssd_state_passing_fwd",
             "ssd_chunk_output_fwd", "ssd_chunk_scan_fwd_uses_tensor_cores",
             "ssd_chunk_scan_fwd_noalloc", "ssd_poll_device_status", "ssd_state_walk_fwd",
-            "ssd_debug_expire_wait", "ssd_chunk_scan_bwd_workspace_size", "ssd_chunk_scan_bwd")
+            "ssd_debug_expire_wait", "ssd_chunk_scan_bwd_workspace_size", "ssd_chunk_scan_bwd",
+            "ssd_chunk_scan_fwd_data_flow")
+
+# ssd_chunk_scan_fwd_data_flow results
+SSD_FLOW_SIMT, SSD_FLOW_TC_THREE_KERNEL, SSD_FLOW_WALK_OUTPUT = 0, 1, 2
 
 
 class SSDError(RuntimeError):
@@ -64,6 +68,8 @@ def load(path: str = LIB_PATH):
                                                       ctypes.POINTER(ctypes.c_size_t)]
     lib.ssd_chunk_scan_fwd_uses_tensor_cores.restype = ctypes.c_int
     lib.ssd_chunk_scan_fwd_uses_tensor_cores.argtypes = [dims_p, ctypes.c_int, ctypes.c_int]
+    lib.ssd_chunk_scan_fwd_data_flow.restype = ctypes.c_int
+    lib.ssd_chunk_scan_fwd_data_flow.argtypes = [dims_p, ctypes.c_int, ctypes.c_int]
     lib.ssd_chunk_scan_fwd.restype = ctypes.c_int
     lib.ssd_chunk_scan_fwd.argtypes = [_vp] * 6 + [ctypes.c_int, _vp, _vp, _vp, dims_p,
                                                    ctypes.c_int, _vp, ctypes.c_size_t, _vp]
@@ -122,12 +128,54 @@ def _ptr(t):
     return ctypes.c_void_p(t.data_ptr())
 
 
-def _stream(stream):
+def _stream(stream, device=None):
     if stream is None:
-        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+        return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
     if isinstance(stream, torch.cuda.Stream):
         return ctypes.c_void_p(stream.cuda_stream)
     return ctypes.c_void_p(int(stream))
+
+
+def _device_of(t):
+    """The CUDA device the call runs on: the main input's.  Calls are made
+    with that device current (the library looks up its per-device state for
+    the current device and rejects tensors of another one)."""
+    if not t.is_cuda:
+        raise ValueError("tensors must be on a CUDA device (there is no CPU path)")
+    return t.device
+
+
+def _expect(name, t, shape, dtype, device):
+    """Shape, dtype and device of one argument, checked before the C call (a
+    wrong shape would otherwise become an out-of-bounds access)."""
+    if t is None:
+        return
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if t.dtype != dtype:
+        raise ValueError(f"{name}: dtype {t.dtype}, expected {dtype}")
+    if t.device != device:
+        raise ValueError(f"{name}: on {t.device}, expected {device} (the device of x)")
+
+
+def _check_fwd_args(x, dt, A, B, C, D, init, y, final):
+    """Shapes, dtypes and devices of the forward's arguments (against x and
+    B), then that they are on a CUDA device.  Returns that device."""
+    if x.dim() != 4 or B.dim() != 4:
+        raise ValueError("x must be (b, L, H, P) and B (b, L, G, N)")
+    dev = x.device
+    b, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    f32 = torch.float32
+    _expect("dt", dt, (b, L, H), f32, dev)
+    _expect("A", A, (H,), f32, dev)
+    _expect("D", D, (H,), f32, dev)
+    _expect("B", B, (b, L, G, N), x.dtype, dev)
+    _expect("C", C, (b, L, G, N), x.dtype, dev)
+    _expect("init_states", init, (b, H, P, N), f32, dev)
+    _expect("y", y, (b, L, H, P), x.dtype, dev)
+    _expect("final_states", final, (b, H, P, N), f32, dev)
+    return _device_of(x)
 
 
 def make_dims(batch, seqlen, nheads, headdim, dstate, ngroups) -> ssd_dims_t:
@@ -155,10 +203,17 @@ def ssd_chunk_scan_fwd_uses_tensor_cores(dims: ssd_dims_t, chunk_size: int,
                                                            _dtype_code(dtype)))
 
 
+def ssd_chunk_scan_fwd_data_flow(dims: ssd_dims_t, chunk_size: int, dtype: torch.dtype) -> int:
+    """SSD_FLOW_WALK_OUTPUT, SSD_FLOW_TC_THREE_KERNEL, SSD_FLOW_SIMT or -1 (rejected)."""
+    return int(load().ssd_chunk_scan_fwd_data_flow(ctypes.byref(dims), int(chunk_size),
+                                                   _dtype_code(dtype)))
+
+
 def ssd_chunk_scan_fwd(x, dt, A, B, C, D, chunk_size: int, init_states=None,
                        return_final_states: bool = False, y=None, final_states=None,
                        workspace=None, stream=None):
     """y (b,L,H,P) [, final_states (b,H,P,N) fp32] for the whole sequences."""
+    dev = _check_fwd_args(x, dt, A, B, C, D, init_states, y, final_states)
     dims = _fwd_dims(x, B)
     if y is None:
         y = torch.empty_like(x)
@@ -168,10 +223,12 @@ def ssd_chunk_scan_fwd(x, dt, A, B, C, D, chunk_size: int, init_states=None,
     need = ssd_chunk_scan_fwd_workspace_size(dims, chunk_size, x.dtype)
     if workspace is None:
         workspace = torch.empty(max(need, 16), device=x.device, dtype=torch.uint8)
-    st = load().ssd_chunk_scan_fwd(_ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
-                                   int(chunk_size), _ptr(init_states), _ptr(y),
-                                   _ptr(final_states), ctypes.byref(dims), _dtype_code(x.dtype),
-                                   _ptr(workspace), workspace.numel(), _stream(stream))
+    with torch.cuda.device(dev):
+        st = load().ssd_chunk_scan_fwd(_ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+                                       int(chunk_size), _ptr(init_states), _ptr(y),
+                                       _ptr(final_states), ctypes.byref(dims),
+                                       _dtype_code(x.dtype), _ptr(workspace), workspace.numel(),
+                                       _stream(stream, dev))
     _check(st, "ssd_chunk_scan_fwd")
     return (y, final_states) if (return_final_states or final_states is not None) else y
 
@@ -183,16 +240,18 @@ def ssd_chunk_scan_fwd_noalloc(x, dt, A, B, C, D, chunk_size: int, init_states=N
     scratch array (SSD_NOALLOC_SCRATCH_BYTES) is used instead.  For callers
     that cannot allocate device memory; calls that overlap on the GPU race on
     that array."""
+    dev = _check_fwd_args(x, dt, A, B, C, D, init_states, y, final_states)
     dims = _fwd_dims(x, B)
     if y is None:
         y = torch.empty_like(x)
     if return_final_states and final_states is None:
         final_states = torch.empty((x.shape[0], x.shape[2], x.shape[3], B.shape[3]),
                                    device=x.device, dtype=torch.float32)
-    st = load().ssd_chunk_scan_fwd_noalloc(_ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
-                                           int(chunk_size), _ptr(init_states), _ptr(y),
-                                           _ptr(final_states), ctypes.byref(dims),
-                                           _dtype_code(x.dtype), _stream(stream))
+    with torch.cuda.device(dev):
+        st = load().ssd_chunk_scan_fwd_noalloc(_ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C),
+                                               _ptr(D), int(chunk_size), _ptr(init_states),
+                                               _ptr(y), _ptr(final_states), ctypes.byref(dims),
+                                               _dtype_code(x.dtype), _stream(stream, dev))
     _check(st, "ssd_chunk_scan_fwd_noalloc")
     return (y, final_states) if (return_final_states or final_states is not None) else y
 
@@ -204,11 +263,23 @@ def ssd_step(state, x, dt, A, B, C, D, y=None, stream=None):
     """One decode step; ``state`` (b,H,P,N) fp32 is updated in place.  Returns y (b,H,P)."""
     b, H, P = x.shape
     G, N = B.shape[1], B.shape[2]
+    dev = x.device
+    f32 = torch.float32
+    _expect("state", state, (b, H, P, N), f32, dev)
+    _expect("dt", dt, (b, H), f32, dev)
+    _expect("A", A, (H,), f32, dev)
+    _expect("D", D, (H,), f32, dev)
+    _expect("B", B, (b, G, N), x.dtype, dev)
+    _expect("C", C, (b, G, N), x.dtype, dev)
+    _expect("y", y, (b, H, P), x.dtype, dev)
+    dev = _device_of(x)
     dims = make_dims(b, 1, H, P, N, G)
     if y is None:
         y = torch.empty_like(x)
-    st = load().ssd_step(_ptr(state), _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
-                         _ptr(y), ctypes.byref(dims), _dtype_code(x.dtype), _stream(stream))
+    with torch.cuda.device(dev):
+        st = load().ssd_step(_ptr(state), _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+                             _ptr(y), ctypes.byref(dims), _dtype_code(x.dtype),
+                             _stream(stream, dev))
     _check(st, "ssd_step")
     return y
 
@@ -233,11 +304,13 @@ def ssd_chunk_state_fwd(x, dt, A, B, chunk_size: int, stream=None):
     dims = _fwd_dims(x, B)
     b, L, H, P = x.shape
     T = n_chunks(L, chunk_size)
+    dev = _check_fwd_args(x, dt, A, B, None, None, None, None, None)
     states = torch.empty((b, T, H, P, B.shape[3]), device=x.device, dtype=torch.float32)
     logdecay = torch.empty((b, T, H), device=x.device, dtype=torch.float32)
-    st = load().ssd_chunk_state_fwd(_ptr(x), _ptr(dt), _ptr(A), _ptr(B), int(chunk_size),
-                                    _ptr(states), _ptr(logdecay), ctypes.byref(dims),
-                                    _dtype_code(x.dtype), _stream(stream))
+    with torch.cuda.device(dev):
+        st = load().ssd_chunk_state_fwd(_ptr(x), _ptr(dt), _ptr(A), _ptr(B), int(chunk_size),
+                                        _ptr(states), _ptr(logdecay), ctypes.byref(dims),
+                                        _dtype_code(x.dtype), _stream(stream, dev))
     _check(st, "ssd_chunk_state_fwd")
     return states, logdecay
 
@@ -248,12 +321,21 @@ def ssd_state_passing_fwd(chunk_states, chunk_logdecay, chunk_size: int, seqlen:
     """Step (3): states entering each chunk (b,T,H,P,N) in ``dtype`` and the final state."""
     b, T, H, P, N = chunk_states.shape
     dims = make_dims(b, seqlen, H, P, N, 1)
+    dev = _device_of(chunk_states)
+    _expect("chunk_states", chunk_states, (b, T, H, P, N), torch.float32, dev)
+    _expect("chunk_logdecay", chunk_logdecay, (b, T, H), torch.float32, dev)
+    _expect("init_states", init_states, (b, H, P, N), torch.float32, dev)
+    if n_chunks(seqlen, chunk_size) != T:
+        raise ValueError(f"chunk_states has {T} chunks; seqlen {seqlen} / chunk {chunk_size} "
+                         f"gives {n_chunks(seqlen, chunk_size)}")
     prev = torch.empty((b, T, H, P, N), device=chunk_states.device, dtype=dtype)
     final = (torch.empty((b, H, P, N), device=chunk_states.device, dtype=torch.float32)
              if want_final else None)
-    st = load().ssd_state_passing_fwd(_ptr(chunk_states), _ptr(chunk_logdecay), _ptr(init_states),
-                                      _ptr(prev), _ptr(final), int(chunk_size), ctypes.byref(dims),
-                                      _dtype_code(dtype), _stream(stream))
+    with torch.cuda.device(dev):
+        st = load().ssd_state_passing_fwd(_ptr(chunk_states), _ptr(chunk_logdecay),
+                                          _ptr(init_states), _ptr(prev), _ptr(final),
+                                          int(chunk_size), ctypes.byref(dims),
+                                          _dtype_code(dtype), _stream(stream, dev))
     _check(st, "ssd_state_passing_fwd")
     return prev, final
 
@@ -266,23 +348,32 @@ def ssd_state_walk_fwd(x, dt, A, B, chunk_size: int, init_states=None, want_fina
     b, L, H, P = x.shape
     N = B.shape[3]
     T = n_chunks(L, chunk_size)
+    dev = _check_fwd_args(x, dt, A, B, None, None, init_states, None, None)
     prev = torch.empty((b, T, H, P, N), device=x.device, dtype=torch.bfloat16)
     final = torch.empty((b, H, P, N), device=x.device, dtype=torch.float32) if want_final else None
-    st = load().ssd_state_walk_fwd(_ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(init_states),
-                                   _ptr(prev), _ptr(final), int(chunk_size), ctypes.byref(dims),
-                                   _dtype_code(x.dtype), _stream(stream))
+    with torch.cuda.device(dev):
+        st = load().ssd_state_walk_fwd(_ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(init_states),
+                                       _ptr(prev), _ptr(final), int(chunk_size),
+                                       ctypes.byref(dims), _dtype_code(x.dtype),
+                                       _stream(stream, dev))
     _check(st, "ssd_state_walk_fwd")
     return prev, final
 
 
 def ssd_chunk_output_fwd(x, dt, A, B, C, D, prev_states, chunk_size: int, y=None, stream=None):
     """Steps (1) and (4): y from the inputs and the states entering each chunk."""
+    dev = _check_fwd_args(x, dt, A, B, C, D, None, y, None)
+    b, L, H, P = x.shape
+    _expect("prev_states", prev_states, (b, n_chunks(L, chunk_size), H, P, B.shape[3]), x.dtype,
+            dev)
     dims = _fwd_dims(x, B)
     if y is None:
         y = torch.empty_like(x)
-    st = load().ssd_chunk_output_fwd(_ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
-                                     _ptr(prev_states), int(chunk_size), _ptr(y),
-                                     ctypes.byref(dims), _dtype_code(x.dtype), _stream(stream))
+    with torch.cuda.device(dev):
+        st = load().ssd_chunk_output_fwd(_ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+                                         _ptr(prev_states), int(chunk_size), _ptr(y),
+                                         ctypes.byref(dims), _dtype_code(x.dtype),
+                                         _stream(stream, dev))
     _check(st, "ssd_chunk_output_fwd")
     return y
 
@@ -300,6 +391,8 @@ def ssd_chunk_scan_bwd(x, dt, A, B, C, D, dy, init_states=None, dfinal_states=No
     """Gradients of ssd_chunk_scan_fwd for dL/dy = dy (b,L,H,P, x's dtype) and
     dL/dfinal_states = dfinal_states ((b,H,P,N) fp32 or None).  Returns a dict
     of fp32 tensors: dx, ddt, dA, dB, dC, dD and (if want_dinit) dinit."""
+    dev = _check_fwd_args(x, dt, A, B, C, D, init_states, None, dfinal_states)
+    _expect("dy", dy, tuple(x.shape), x.dtype, dev)
     dims = _fwd_dims(x, B)
     b, L, H, P = x.shape
     G, N = B.shape[2], B.shape[3]
@@ -311,11 +404,13 @@ def ssd_chunk_scan_bwd(x, dt, A, B, C, D, dy, init_states=None, dfinal_states=No
     need = ssd_chunk_scan_bwd_workspace_size(dims, x.dtype)
     if workspace is None:
         workspace = torch.empty(max(need, 16), device=x.device, dtype=torch.uint8)
-    st = load().ssd_chunk_scan_bwd(_ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
-                                   _ptr(init_states), _ptr(dy), _ptr(dfinal_states),
-                                   _ptr(out["dx"]), _ptr(out["ddt"]), _ptr(out["dA"]),
-                                   _ptr(out["dB"]), _ptr(out["dC"]), _ptr(out["dD"]),
-                                   _ptr(out["dinit"]), ctypes.byref(dims), _dtype_code(x.dtype),
-                                   _ptr(workspace), workspace.numel(), _stream(stream))
+    with torch.cuda.device(dev):
+        st = load().ssd_chunk_scan_bwd(_ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+                                       _ptr(init_states), _ptr(dy), _ptr(dfinal_states),
+                                       _ptr(out["dx"]), _ptr(out["ddt"]), _ptr(out["dA"]),
+                                       _ptr(out["dB"]), _ptr(out["dC"]), _ptr(out["dD"]),
+                                       _ptr(out["dinit"]), ctypes.byref(dims),
+                                       _dtype_code(x.dtype), _ptr(workspace), workspace.numel(),
+                                       _stream(stream, dev))
     _check(st, "ssd_chunk_scan_bwd")
     return out

@@ -63,12 +63,41 @@ def _round(v):
     (3, 1, 2, 3, 5, 1, 16, ssd.SSD_F32),
 ])
 def test_workspace_size_formula(lib, b, L, H, P, N, G, Q, dt):
-    st, n = _ws(ssd.make_dims(b, L, H, P, N, G), Q, dt)
+    dims = ssd.make_dims(b, L, H, P, N, G)
+    st, n = _ws(dims, Q, dt)
     assert st == ssd.SSD_OK
     T = (L + Q - 1) // Q
     elt = 4 if dt == ssd.SSD_F32 else 2
     ns = b * T * H * P * N
-    assert n == _round(ns * 4) + _round(b * T * H * 4) + _round(ns * elt)
+    if lib.ssd_chunk_scan_fwd_data_flow(ctypes.byref(dims), Q, dt) == ssd.SSD_FLOW_WALK_OUTPUT:
+        # the walk keeps chunk states on chip: only the entering states
+        assert n == _round(ns * elt)
+    else:
+        # chunk states (fp32), per-chunk log-decays, entering states
+        assert n == _round(ns * 4) + _round(b * T * H * 4) + _round(ns * elt)
+
+
+@pytest.mark.parametrize("b,L,H,P,N,G,Q,dt,flow", [
+    (4, 8192, 80, 64, 128, 1, 256, ssd.SSD_BF16, ssd.SSD_FLOW_WALK_OUTPUT),   # 2.7B layer
+    (8, 2048, 24, 64, 128, 1, 256, ssd.SSD_BF16, ssd.SSD_FLOW_WALK_OUTPUT),   # 130M layer
+    (1024, 512, 32, 64, 64, 1, 256, ssd.SSD_BF16, ssd.SSD_FLOW_WALK_OUTPUT),  # 2 chunks
+    (1, 524288, 32, 64, 64, 1, 256, ssd.SSD_BF16, ssd.SSD_FLOW_TC_THREE_KERNEL),  # 16 walkers
+    (4, 131072, 32, 64, 64, 1, 256, ssd.SSD_BF16, ssd.SSD_FLOW_TC_THREE_KERNEL),  # 64 walkers
+    (6, 32768, 32, 64, 64, 1, 256, ssd.SSD_BF16, ssd.SSD_FLOW_WALK_OUTPUT),  # 96 walkers
+    (2, 600, 4, 64, 128, 1, 256, ssd.SSD_BF16, ssd.SSD_FLOW_TC_THREE_KERNEL),
+    (4, 8192, 80, 64, 128, 1, 256, ssd.SSD_F32, ssd.SSD_FLOW_SIMT),
+    (4, 8192, 80, 32, 128, 1, 256, ssd.SSD_BF16, ssd.SSD_FLOW_SIMT),
+])
+def test_data_flow_query(lib, b, L, H, P, N, G, Q, dt, flow):
+    dims = ssd.make_dims(b, L, H, P, N, G)
+    assert lib.ssd_chunk_scan_fwd_data_flow(ctypes.byref(dims), Q, dt) == flow
+    tc = lib.ssd_chunk_scan_fwd_uses_tensor_cores(ctypes.byref(dims), Q, dt)
+    assert tc == (0 if flow == ssd.SSD_FLOW_SIMT else 1)
+
+
+def test_data_flow_query_rejects(lib):
+    bad = ssd.make_dims(1, 64, 4, 8, 8, 3)
+    assert lib.ssd_chunk_scan_fwd_data_flow(ctypes.byref(bad), 64, ssd.SSD_F32) == -1
 
 
 def test_workspace_zero_for_empty(lib):
@@ -182,6 +211,29 @@ def test_tensor_core_selection_query(lib):
     f = lib.ssd_chunk_scan_fwd_uses_tensor_cores
     assert f(ctypes.byref(ssd.make_dims(1, 64, 4, 8, 8, 3)), 64, 0) == -1
     assert f(ctypes.byref(ssd.make_dims(1, 256, 4, 16, 16, 1)), 64, ssd.SSD_F32) == 0
+
+
+def test_binding_checks_shapes_and_dtypes_before_calling(lib):
+    import torch
+    b, L, H, P, N = 1, 64, 2, 8, 4
+    args = dict(x=torch.zeros(b, L, H, P), dt=torch.zeros(b, L, H), A=torch.zeros(H),
+                B=torch.zeros(b, L, 1, N), C=torch.zeros(b, L, 1, N), D=torch.zeros(H))
+    for key, bad, what in [("dt", torch.zeros(b, L, H + 1), "shape"),
+                           ("A", torch.zeros(H, dtype=torch.float64), "dtype"),
+                           ("C", torch.zeros(b, L, 1, N + 1), "shape"),
+                           ("D", torch.zeros(H + 1), "shape")]:
+        a = dict(args)
+        a[key] = bad
+        with pytest.raises(ValueError, match=f"{key}: {what}"):
+            ssd.ssd_chunk_scan_fwd(a["x"], a["dt"], a["A"], a["B"], a["C"], a["D"], 64)
+    with pytest.raises(ValueError, match="init_states: shape"):
+        ssd.ssd_chunk_scan_fwd(*args.values(), 64, init_states=torch.zeros(b, H, P, N + 1))
+    with pytest.raises(ValueError, match="y: dtype"):
+        ssd.ssd_chunk_scan_fwd(*args.values(), 64, y=torch.zeros(b, L, H, P,
+                                                                   dtype=torch.bfloat16))
+    with pytest.raises(ValueError, match="state: shape"):
+        ssd.ssd_step(torch.zeros(b, H, P, N + 1), torch.zeros(b, H, P), torch.zeros(b, H),
+                     torch.zeros(H), torch.zeros(b, 1, N), torch.zeros(b, 1, N), torch.zeros(H))
 
 
 def test_binding_refuses_cpu_tensors(lib):

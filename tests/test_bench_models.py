@@ -26,10 +26,22 @@ def test_forward_models_at_the_workload_shapes():
         assert round(nbytes / 1e9, 2) == 4.50
 
 
-def test_kernel_bytes_of_the_three_kernel_forward():
+def test_kernel_bytes_of_both_data_flows():
+    """io: each kernel's own reads and writes (intermediates included); alg:
+    its share of bytes_min (x, y, B, C, dt, init, final; no intermediates)."""
     kb = bench.kernel_bytes(inputs.LAYER_2P7B)
-    assert {k: round(v / 1e6, 1) for k, v in kb.items() if k != "decode"} == {
-        "chunk_state": 690.0, "state_pass": 524.3, "chunk_out": 866.1}
+    io = {k: round(v[1] / 1e6, 1) for k, v in kb.items()}
+    assert io == {"chunk_state": 690.0, "state_pass": 524.3, "chunk_out": 866.1,
+                  "state_walk": 543.2}
+    alg = {k: round(v[0] / 1e6, 1) for k, v in kb.items()}
+    # chunk_out: x read + y written + B + C + dt = 698.4 MB
+    assert alg["chunk_out"] == 698.4
+    # the walk: x + B + dt + initial and final states (fp32, 10.5 MB each)
+    b, L, H, P, N = 4, 8192, 80, 64, 128
+    assert kb["state_walk"][0] == b * L * (H * P * 2 + N * 2 + 4 * H) + 2 * 4 * b * H * P * N
+    # the walk + output flow touches every byte of bytes_min; no share exceeds it
+    _, _, nbytes = bench.fwd_model(inputs.LAYER_2P7B)
+    assert max(v[0] for v in kb.values()) <= nbytes
 
 
 def test_backward_bytes():

@@ -226,14 +226,43 @@ def test_stage_state_walk(case):
     assert ep <= TOL["bf16"] and ef <= TOL["bf16"], (ep, ef)
 
 
-def test_walk_path_full_forward_ragged_groups():
-    """A shape above the walk threshold (batch x heads / 2 >= SM count) with a
-    ragged last chunk, two groups and initial states: the forward takes the
-    walk + output path; every element checked."""
-    w = _w("walk_fwd", 8, 700, 40, 64, 128, 2, 256, "bf16", True, seed=35)
-    dims = ssd.make_dims(8, 700, 40, 64, 128, 2)
-    assert ssd.ssd_chunk_scan_fwd_uses_tensor_cores(dims, 256, torch.bfloat16) == 1
-    _check_full(w)
+WALK_FWD_CASES = [
+    # name,                b,  L,    H,  P,  N,  G,  Q,  init
+    ("walk_fwd_n128_g2", 8, 900, 40, 64, 128, 2, 256, True),    # 4 chunks, last one partial
+    ("walk_fwd_n64_q128", 16, 1100, 12, 64, 64, 2, 128, True),  # 9 chunks, last one partial
+]
+
+
+@pytest.mark.parametrize("case", WALK_FWD_CASES, ids=[c[0] for c in WALK_FWD_CASES])
+def test_walk_path_full_forward_ragged_groups(case):
+    """Shapes the forward runs as walk + output (enough (batch, head pair)
+    walkers and chunks), with a ragged last chunk, two groups and initial
+    states; every element checked."""
+    name, b, L, H, P, N, G, Q, init = case
+    dims = ssd.make_dims(b, L, H, P, N, G)
+    assert ssd.ssd_chunk_scan_fwd_data_flow(dims, Q, torch.bfloat16) == ssd.SSD_FLOW_WALK_OUTPUT
+    _check_full(_w(name, b, L, H, P, N, G, Q, "bf16", init, seed=35))
+
+
+def test_walk_and_three_kernel_flows_agree():
+    """The same inputs through both tensor-core data flows, driven step by
+    step: walk + output against chunk states + state pass + output."""
+    w = _w("flows", 4, 1500, 8, 64, 128, 1, 256, "bf16", True, seed=36)
+    d = to_dev(inputs.make_inputs(w))
+    prev_w, fin_w = ssd.ssd_state_walk_fwd(d["x"], d["dt"], d["A"], d["B"], 256,
+                                           init_states=d["init"])
+    S, ld = ssd.ssd_chunk_state_fwd(d["x"], d["dt"], d["A"], d["B"], 256)
+    prev_t, fin_t = ssd.ssd_state_passing_fwd(S, ld, 256, w.seqlen, torch.bfloat16,
+                                              init_states=d["init"])
+    y_w = ssd.ssd_chunk_output_fwd(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], prev_w, 256)
+    y_t = ssd.ssd_chunk_output_fwd(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], prev_t, 256)
+    torch.cuda.synchronize()
+    y_ref, f_ref = oracle_fwd(inputs.make_inputs(w))
+    for y in (y_w, y_t):
+        assert rel_err(y.double().cpu().numpy(), y_ref) <= TOL["bf16"]
+    for f in (fin_w, fin_t):
+        assert rel_err(f.double().cpu().numpy(), f_ref) <= TOL["bf16"]
+    assert rel_err(prev_w.double().cpu().numpy(), prev_t.double().cpu().numpy()) <= TOL["bf16"]
 
 
 @pytest.mark.parametrize("case", STAGE_CASES, ids=lambda c: "_".join(map(str, c)))
@@ -403,6 +432,68 @@ def test_guard_bands_and_full_coverage():
 
 
 def test_tensor_core_path_selected_for_layer_shapes():
+    """Every bf16 workload of the benchmark runs on the tcgen05 kernels (so the
+    sampled full-size parity tests above exercise them), the fp32 one on the
+    exact SIMT kernels."""
+    for w in (inputs.LAYER_130M, inputs.LAYER_2P7B) + tuple(inputs.SWEEP):
+        dims = ssd.make_dims(w.batch, w.seqlen, w.nheads, w.headdim, w.dstate, w.ngroups)
+        assert ssd.ssd_chunk_scan_fwd_uses_tensor_cores(dims, w.chunk, torch.bfloat16) == 1, w.name
+        assert ssd.ssd_chunk_scan_fwd_data_flow(dims, w.chunk, torch.bfloat16) in (
+            ssd.SSD_FLOW_WALK_OUTPUT, ssd.SSD_FLOW_TC_THREE_KERNEL), w.name
+    for w in (inputs.LAYER_130M, inputs.LAYER_2P7B):
+        dims = ssd.make_dims(w.batch, w.seqlen, w.nheads, w.headdim, w.dstate, w.ngroups)
+        assert ssd.ssd_chunk_scan_fwd_data_flow(dims, w.chunk, torch.bfloat16) == \
+            ssd.SSD_FLOW_WALK_OUTPUT, w.name
+    t = inputs.TINY_F32
+    dims = ssd.make_dims(t.batch, t.seqlen, t.nheads, t.headdim, t.dstate, t.ngroups)
+    assert ssd.ssd_chunk_scan_fwd_uses_tensor_cores(dims, t.chunk, torch.float32) == 0
     dims = ssd.make_dims(4, 8192, 80, 64, 128, 1)
-    assert ssd.ssd_chunk_scan_fwd_uses_tensor_cores(dims, 256, torch.bfloat16) in (0, 1)
     assert ssd.ssd_chunk_scan_fwd_uses_tensor_cores(dims, 256, torch.float32) == 0
+
+
+POSITIVE_A_CASES = [
+    # a growing state: A > 0 with a modest growth per chunk, through each data flow
+    ("posA_three_kernel", 2, 600, 4, 64, 128, 1, 256, "bf16"),
+    ("posA_walk", 8, 1100, 24, 64, 128, 1, 256, "bf16"),
+    ("posA_simt_f32", 1, 500, 3, 16, 32, 1, 64, "f32"),
+]
+
+
+@pytest.mark.parametrize("case", POSITIVE_A_CASES, ids=[c[0] for c in POSITIVE_A_CASES])
+def test_positive_a_growing_state(case):
+    name, b, L, H, P, N, G, Q, dtype = case
+    w = _w(name, b, L, H, P, N, G, Q, dtype, True, seed=48)
+    inp = inputs.make_inputs(w)
+    g = torch.Generator().manual_seed(48)
+    inp["A"] = 0.1 + 0.9 * torch.rand(H, generator=g)     # A in [0.1, 1.0]: exp(dt A) > 1
+    y, f = gpu_fwd(inp, Q)
+    y_ref, f_ref = oracle_fwd(inp)
+    ey, ef = rel_err(y, y_ref), rel_err(f, f_ref)
+    record(name, y=ey, final=ef)
+    assert np.max(np.abs(f_ref)) > np.max(np.abs(inp["init"].numpy())), "state did not grow"
+    assert ey <= TOL[dtype] and ef <= TOL[dtype], (ey, ef)
+
+
+def test_rejects_memory_not_on_the_current_device():
+    """x in (unregistered) host memory: rejected before any launch, with the
+    reason; the library stays usable."""
+    import ctypes
+    import numpy as npx
+    w = _w("devchk", 1, 256, 2, 64, 128, 1, 256, "bf16", False, seed=49)
+    d = to_dev(inputs.make_inputs(w))
+    host = npx.zeros(d["x"].numel() * 2 + 64, dtype=npx.uint8)
+    addr = (host.ctypes.data + 15) // 16 * 16
+    lib = ssd.load()
+    dims = ssd.make_dims(1, 256, 2, 64, 128, 1)
+    y = torch.empty_like(d["x"])
+    ws = torch.empty(ssd.ssd_chunk_scan_fwd_workspace_size(dims, 256, torch.bfloat16) + 16,
+                     device="cuda", dtype=torch.uint8)
+    P = lambda t: ctypes.c_void_p(t.data_ptr())
+    st = lib.ssd_chunk_scan_fwd(ctypes.c_void_p(addr), P(d["dt"]), P(d["A"]), P(d["B"]),
+                                P(d["C"]), P(d["D"]), 256, None, P(y), None, ctypes.byref(dims),
+                                ssd.SSD_BF16, P(ws), ws.numel(), None)
+    assert st == ssd.SSD_ERR_INVALID_ARG
+    assert "not device memory" in lib.ssd_last_error_detail().decode()
+    with pytest.raises(ValueError, match="expected cuda"):
+        ssd.ssd_chunk_scan_fwd(d["x"], d["dt"].cpu(), d["A"], d["B"], d["C"], d["D"], 256)
+    _check_full(w)
