@@ -461,6 +461,86 @@ def measure_backward(w, dev, stream, flush, reps, world, rank, peak_gbs):
     return out
 
 
+# ---------------------------------------------------------------- sequence-parallel split
+def correction_bytes(w, Ls):
+    """Algorithmic bytes of one shard's correction (every token corrected):
+    C and dt read, y read and written, h_in read, final state read and
+    written."""
+    sx = 2 if w.dtype == "bf16" else 4
+    ns = w.batch * w.nheads * w.headdim * w.dstate
+    return (w.batch * Ls * (w.ngroups * w.dstate * sx + 4 * w.nheads + 2 * w.nheads * w.headdim * sx)
+            + 4 * ns + 2 * 4 * ns)
+
+
+def measure_seqpar(w, dev, stream, flush, reps, shards=2):
+    """Per-rank device time of the sequence-parallel forward with the
+    sequence split into ``shards`` equal pieces, each rank's steps run on
+    this GPU one rank after another: the shard's zero-start forward, its
+    log-decay, the combine of the gathered values and the correction.  The
+    all-gather between them needs several GPUs and is not timed here."""
+    import torch
+    from ssd_chunked_scan_02_b200 import inputs, seqpar, ssd
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(w.seed + 4000)
+    inp = inputs.make_inputs(w, device=dev, gen=gen)
+    Ls = w.seqlen // shards
+    parts = [{k: inp[k][:, r * Ls:(r + 1) * Ls].contiguous() for k in ("x", "dt", "B", "C")}
+             for r in range(shards)]
+    A, D, init = inp["A"], inp["D"], inp["init"]
+    y = torch.empty_like(parts[0]["x"])
+    fin = torch.empty((w.batch, w.nheads, w.headdim, w.dstate), device=dev)
+    dims = ssd.make_dims(w.batch, Ls, w.nheads, w.headdim, w.dstate, w.ngroups)
+    ws = torch.empty(ssd.ssd_chunk_scan_fwd_workspace_size(dims, w.chunk, y.dtype), device=dev,
+                     dtype=torch.uint8)
+    cws = torch.empty(max(16, ssd.ssd_state_correction_workspace_size(dims, y.dtype)),
+                      device=dev, dtype=torch.uint8)
+    # the gathered values every rank would receive
+    outs = []
+    for p in parts:
+        yy, ff = ssd.ssd_chunk_scan_fwd(p["x"], p["dt"], A, p["B"], p["C"], D, w.chunk,
+                                        return_final_states=True)
+        outs.append(seqpar.pack(ff, ssd.ssd_seq_logdecay(p["dt"], A)))
+    finals, lds = seqpar.unpack(torch.stack(outs), tuple(fin.shape), (w.batch, w.nheads))
+    h_in = torch.empty_like(fin)
+    names = ("forward", "logdecay", "combine", "correction")
+    per = {r: {k: [] for k in names} for r in range(shards)}
+    for it in range(reps + 2):
+        for r, p in enumerate(parts):
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+            flush.zero_()
+            ev[0].record(stream)
+            ssd.ssd_chunk_scan_fwd(p["x"], p["dt"], A, p["B"], p["C"], D, w.chunk, y=y,
+                                   final_states=fin, workspace=ws, stream=stream)
+            ev[1].record(stream)
+            ssd.ssd_seq_logdecay(p["dt"], A, stream=stream)
+            ev[2].record(stream)
+            ssd.ssd_state_exchange_combine(finals, lds, r, init_states=init, out=h_in,
+                                           stream=stream)
+            ev[3].record(stream)
+            ssd.ssd_state_correction_fwd(h_in, p["dt"], A, p["C"], y, final_states=fin,
+                                         workspace=cws, stream=stream)
+            ev[4].record(stream)
+            torch.cuda.synchronize(dev)
+            if it >= 2:
+                for i, k in enumerate(names):
+                    per[r][k].append(ev[i].elapsed_time(ev[i + 1]))
+    means = {r: {k: statistics.mean(v) for k, v in per[r].items()} for r in range(shards)}
+    rank_ms = {r: sum(m.values()) for r, m in means.items()}
+    slow = max(rank_ms, key=rank_ms.get)
+    cb = correction_bytes(w, Ls)
+    corr_ms = max(m["correction"] for m in means.values())
+    del inp, parts, y, fin, ws, cws, finals, lds, h_in
+    torch.cuda.empty_cache()
+    return {"workload": w.name, "shards": shards, "tokens_per_shard": Ls,
+            "ms_per_rank": rank_ms, "steps_ms_slowest_rank": means[slow],
+            "tokens_per_s_if_parallel": w.tokens / (rank_ms[slow] * 1e-3),
+            "correction": {"ms": corr_ms, "alg_bytes_if_all_tokens": cb,
+                           "gbs_if_all_tokens": cb / (corr_ms * 1e-3) / 1e9,
+                           "note": "tokens whose decay from the shard start underflowed to "
+                                   "zero are skipped, so fewer bytes move than counted here"},
+            "all_gather": "not timed: it needs one GPU per rank (b*H*(P*N+1) fp32 per rank)"}
+
+
 # ---------------------------------------------------------------- per-kernel timing
 FLOW_KERNELS = {1: ("chunk_state", "state_pass", "chunk_out"), 2: ("state_walk", "chunk_out")}
 
@@ -729,6 +809,10 @@ def main():
         bwd = measure_backward(inputs.LAYER_130M, dev, stream, flush, max(3, args.steps // 4),
                                world, rank, pk["hbm_gbs"])
 
+    # ---- the sequence-parallel split (per-rank work, on this GPU)
+    spl = None
+    if not args.no_extra_configs and world == 1:
+        spl = measure_seqpar(inputs.LAYER_2P7B, dev, stream, flush, max(3, args.steps // 4))
     # ---- CPU oracle baseline (rank 0, N = 1 only)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -784,6 +868,7 @@ def main():
                              "overlapping, full duplex) take far longer than the forward"},
             "other_configs": extra,
             "backward": bwd,
+            "seqpar": spl,
             "cpu_baseline": cpu,
             "gpu_launches": len(FLOW_KERNELS.get(flow, (0, 0, 0))) * args.steps,
             "clocks": clocks,

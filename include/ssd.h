@@ -112,7 +112,10 @@ SSD_API ssd_status_t ssd_chunk_scan_fwd_workspace_size(const ssd_dims_t* dims, i
  * "Review: Transformers are SSMs (Mamba-2)", 核心概念 item 5 (SSD algorithm:
  * block decomposition that uses the tensor cores and stays linear in L).
  * The sequence is cut into chunks of `chunk_size` tokens (a power of two,
- * 16..256; the last chunk may be partial).  Four steps:
+ * 16..256; the last chunk may be partial).  The result does not depend on
+ * the chunk size beyond rounding; for bf16 the tensor-core kernels run
+ * 128- or 256-token chunks, and a smaller chunk_size runs as 128-token
+ * chunks on them (the workspace size accounts for it).  Four steps:
  *   (1) per chunk, the intra-chunk quadratic term (C B^T masked by the
  *       exp(segsum(dt*A)) decay) applied to dt*x;
  *   (2) per chunk, the state it contributes, B^T (decay * dt * x);
@@ -183,7 +186,10 @@ SSD_API ssd_status_t ssd_chunk_output_fwd(const void* x, const float* dt, const 
  * the process exits.  Sizes whose workspace (ssd_chunk_scan_fwd_workspace_size)
  * exceeds that return SSD_ERR_UNSUPPORTED with a message.  The first call
  * on each device looks up the array's device address (cudaGetSymbolAddress)
- * with that device current; make it before any stream capture.  Nothing is
+ * with that device current; make it before any stream capture.  The address
+ * is kept for the life of the process, per device ordinal: it assumes the
+ * device's primary context throughout (no cudaDeviceReset, no other driver
+ * context made current between calls).  Nothing is
  * allocated or freed.  All calls share the array and it keeps the last
  * call's contents (every byte read is rewritten first within a call, so no
  * clearing is needed), so calls that overlap on the GPU race: serialise them.
@@ -228,6 +234,56 @@ SSD_API ssd_status_t ssd_chunk_scan_bwd(const void* x, const float* dt, const fl
                                         size_t workspace_bytes, void* stream);
 
 /*
+ * Sequence parallelism: splitting L across ranks with one exchange.
+ * "Transformers are SSMs" (CiteArk), what this means: the layer lends
+ * itself to large-scale training with model parallelism.  The state is the
+ * only thing a later part of the sequence needs from an earlier one, and it
+ * enters linearly: with h_in the state entering a shard,
+ *     y_t = y_t|zero start + exp(cs_t) h_in C_t,    cs_t = sum_{k <= t} dt_k A_h,
+ *     h_end = h_end|zero start + exp(cs_last) h_in
+ * (cs from the shard's first token).  So rank r runs ssd_chunk_scan_fwd on
+ * its shard from a zero state, takes ssd_seq_logdecay of its shard, and the
+ * ranks all-gather (local final state, log-decay) -- b*H*(P*N+1) fp32 per
+ * rank; ssd_state_exchange_combine then gives each rank its h_in (the
+ * exclusive scan over the ranks before it), and ssd_state_correction_fwd
+ * adds h_in's contribution to the shard's y and final state.
+ *
+ * ssd_seq_logdecay: logdecay (b,H) fp32 = sum over the L tokens of dt[b,t,h]
+ *   * A[h] (natural-log units, summed in fp64).  dims->seqlen = the shard's L.
+ * ssd_state_exchange_combine: local_final (R,b,H,P,N) fp32 and logdecay
+ *   (R,b,H) fp32 are the gathered values of ranks 0..R-1 (rank order);
+ *   init (b,H,P,N) fp32 or NULL (zero) is the state entering rank 0's shard.
+ *   Writes h_in (b,H,P,N) fp32 = the state entering rank `rank`'s shard:
+ *   h_0 = init, h_{q+1} = exp(logdecay_q) h_q + local_final_q, for
+ *   0 <= rank <= R (rank = R gives the state after the whole sequence).
+ *   dims->seqlen is ignored.
+ * ssd_state_correction_fwd: y (b,L,H,P) in dtype is updated in place,
+ *   y_t += exp(cs_t) h_in C_t (computed in fp32, rounded once to dtype);
+ *   final_states (b,H,P,N) fp32, if non-NULL, is updated in place,
+ *   final += exp(cs_last) h_in.  h_in (b,H,P,N) fp32; dt, A, C as in the
+ *   forward.  For bf16 with headdim 64..256 (a multiple of 64) and dstate
+ *   64 or 128 the contraction
+ *   runs on the tcgen05 tensor cores (h_in rounded to bf16 as an operand,
+ *   as the forward does with its entering states); otherwise in exact fp32
+ *   on the CUDA cores.  Tokens whose decay from the shard start underflows
+ *   to zero (A <= 0) are left untouched.  workspace: >= the size
+ *   ssd_state_correction_workspace_size reports (NULL only when that is 0).
+ */
+SSD_API ssd_status_t ssd_seq_logdecay(const float* dt, const float* A, float* logdecay,
+                                      const ssd_dims_t* dims, void* stream);
+SSD_API ssd_status_t ssd_state_exchange_combine(const float* local_final, const float* logdecay,
+                                                const float* init, int rank, int nranks,
+                                                float* h_in, const ssd_dims_t* dims,
+                                                void* stream);
+SSD_API ssd_status_t ssd_state_correction_workspace_size(const ssd_dims_t* dims,
+                                                         ssd_dtype_t dtype, size_t* bytes);
+SSD_API ssd_status_t ssd_state_correction_fwd(const float* h_in, const float* dt, const float* A,
+                                              const void* C, void* y, float* final_states,
+                                              const ssd_dims_t* dims, ssd_dtype_t dtype,
+                                              void* workspace, size_t workspace_bytes,
+                                              void* stream);
+
+/*
  * Reports, and clears, a device-side wait that gave up in an earlier call on
  * the current device: the tensor-core kernels bound every wait, and one that
  * runs out records SSD_ERR_TIMEOUT in a device status word and ends the
@@ -245,8 +301,9 @@ SSD_API ssd_status_t ssd_poll_device_status(void* stream);
  * state after the last chunk.  ssd_chunk_scan_fwd runs it (followed by
  * ssd_chunk_output_fwd's kernel) whenever ssd_chunk_scan_fwd_data_flow
  * reports SSD_FLOW_WALK_OUTPUT.  Covers the tensor-core sizes only
- * (SSD_BF16, chunk_size 128 or 256, headdim 64, dstate 64 or 128, nheads /
- * ngroups even); other sizes return SSD_ERR_UNSUPPORTED.
+ * (SSD_BF16, chunk_size 128 or 256, headdim 64, 128, 192 or 256, dstate 64
+ * or 128, any number of heads per group); other sizes return
+ * SSD_ERR_UNSUPPORTED.
  */
 SSD_API ssd_status_t ssd_state_walk_fwd(const void* x, const float* dt, const float* A,
                                         const void* B, const float* init_states,
@@ -264,7 +321,11 @@ SSD_API ssd_status_t ssd_state_walk_fwd(const void* x, const float* dt, const fl
 SSD_API ssd_status_t ssd_debug_expire_wait(unsigned int polls, void* stream);
 
 /* Which kernel family ssd_chunk_scan_fwd uses for these sizes:
- * 1 = tcgen05 tensor-core kernels, 0 = SIMT fp32 kernels, -1 = rejected. */
+ * 1 = tcgen05 tensor-core kernels, 0 = SIMT fp32 kernels, -1 = rejected.
+ * The tensor cores take SSD_BF16 with headdim 64, 128, 192 or 256 (a head of
+ * headdim 64 k runs as k heads of 64 sharing dt, A, D), dstate 64 or 128,
+ * any number of heads per group and any chunk_size; everything else (and all
+ * of SSD_F32, whose 1e-4 bound rules out bf16 operands) runs exact fp32. */
 SSD_API int ssd_chunk_scan_fwd_uses_tensor_cores(const ssd_dims_t* dims, int chunk_size,
                                          ssd_dtype_t dtype);
 

@@ -11,7 +11,8 @@
 // decomposition lets the tensor cores do the work).
 //
 // One CTA per (batch, chunk, 128-row tile t of the chunk, group of HG heads
-// sharing B and C).  Tile t holds rows i in [128 t, 128 t + 128).
+// sharing B and C).  Heads are virtual heads of headdim 64: a head of
+// headdim 64 k is k of them, sharing dt, A and D.  Tile t holds rows i in [128 t, 128 t + 128).
 //
 // The decay between row i and column j < i factorises through any boundary r:
 // exp(cs_i - cs_j) = exp(cs_i - r) exp(r - cs_j).  The diagonal 128 x 128
@@ -111,7 +112,7 @@ enum {
     BAR_XFULL = 3,      // up to four x/h ring slots
     BAR_XEMPTY = 7,
     BAR_MFULL = 11,     // four: the head's operands are ready (head modulo 4)
-    BAR_MEMPTY = 15,    // the exact-path mask slot
+                        // 15: unused
     BAR_ACCFULL = 16, BAR_ACCEMPTY = 18,
     BAR_ALFULL = 20,    // four factor slots (alpha_i, a_i, path) per head modulo 4
     BAR_FEMPTY = 24,    // four: the epilogue has read the factor slot
@@ -164,7 +165,9 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
                     const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmH,
                     const __grid_constant__ CUtensorMap tmY, const float* __restrict__ dt,
                     const float* __restrict__ A, const float* __restrict__ Dv, int64_t L, int H,
-                    int G, int64_t T, int HG, WaitCtx status) {
+                    int G, int64_t T, int HG, int ksplit, WaitCtx status) {
+    // H counts virtual heads (headdim 64); real head = virtual head / ksplit
+    const int Hr = H / ksplit;
     using S = OutSmem<Q, N>;
     constexpr int kTiles = Q / 128;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -334,7 +337,6 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
                 }
                 if (!fast) issue_z(t == 1);
                 mma_commit(&bars[BAR_XEMPTY + s]);           // x and h slot s: no reader left
-                mma_commit(&bars[BAR_MEMPTY]);               // the mask slot: no reader left
                 mma_commit(&bars[BAR_ACCFULL + a]);
             }
             if (!ok) s_flag[0] = 1;
@@ -350,11 +352,11 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
         // Thread tid < KJ holds dt of token tid for the head in turn, loaded one
         // head ahead (the first one while the prologue runs).
         const bool tok_in = tid < KJ && tid < len;
-        const float* dt_tok = dt + (b * L + t0 + tid) * H + head0;
-        float dt_next = tok_in ? dt_tok[0] : 0.f;
+        const float* dt_tok = dt + (b * L + t0 + tid) * Hr;
+        float dt_next = tok_in ? dt_tok[head0 / ksplit] : 0.f;
         if (tid < HG) {
-            s_Ah[tid] = A[head0 + tid] * kLog2e;
-            s_Dh[tid] = Dv[head0 + tid];
+            s_Ah[tid] = A[(head0 + tid) / ksplit] * kLog2e;
+            s_Dh[tid] = Dv[(head0 + tid) / ksplit];
         }
         named_bar_sync(1, 256);
         bool fail = !mbar_wait(&bars[BAR_G], 0, status);
@@ -426,7 +428,7 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
                     // inclusive prefix sums of dt*A (log2 units) of this head over the
                     // tile's KJ columns: a shuffle scan per warp, then the warp offsets
                     const float dt_cur = dt_next;
-                    if (hi + 1 < HG) dt_next = tok_in ? dt_tok[hi + 1] : 0.f;
+                    if (hi + 1 < HG) dt_next = tok_in ? dt_tok[(head0 + hi + 1) / ksplit] : 0.f;
                     float v = dt_cur * s_Ah[hi];
 #pragma unroll
                     for (int o = 1; o < 32; o <<= 1) {
@@ -469,9 +471,14 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
                 }
                 if (tid == 0) s_path[f] = fast ? 1 : 0;
                 // the exact path writes the mask slot: free once the MMAs of head hi - 1
-                // have completed; both paths need the head's x rows and entering state
+                // have completed, which the end of that head's epilogue implies (a wait
+                // on the MMAs' own commit could alias: the scale warps may be more than
+                // one head ahead of the MMAs, while the epilogue of head hi - 5 is
+                // known to be done, so this barrier lags by at most one phase); both
+                // paths need the head's x rows and entering state
                 fail = (!fast && hi >= 1 &&
-                        !mbar_wait(&bars[BAR_MEMPTY], (uint32_t)((hi - 1) & 1), status)) ||
+                        !mbar_wait(&bars[BAR_FEMPTY + ((hi - 1) & 3)],
+                                   (uint32_t)(((hi - 1) >> 2) & 1), status)) ||
                        !mbar_wait(&bars[BAR_XFULL + s], (uint32_t)((hi / R) & 1), status);
                 if (named_bar_or(1, 256, fail)) break;   // also publishes the factors
                 if (tid == 0) mbar_arrive(&bars[BAR_ALFULL + f]);
@@ -661,7 +668,7 @@ int pick_heads_per_cta(int64_t H, int64_t G) {
 
 template <int Q, int N>
 cudaError_t launch_impl(const void* x, const float* dt, const float* A, const void* B,
-                        const void* C, const float* D, const void* prev, void* y, const Dims& d,
+                        const void* C, const float* D, const void* prev, void* y, const Dims& d, int ksplit,
                         cudaStream_t s) {
     using S = OutSmem<Q, N>;
     CUtensorMap tmX, tmB, tmC, tmH, tmY;
@@ -694,7 +701,7 @@ cudaError_t launch_impl(const void* x, const float* dt, const float* A, const vo
     dim3 grid((unsigned)(d.b * d.T * (Q / 128)), (unsigned)(d.H / HG));
     chunk_out_tc_kernel<Q, N><<<grid, kThreads, S::kAlloc, s>>>(
         tmX, tmB, tmC, tmH, tmY, dt, A, D, d.L, (int)d.H,
-        (int)d.G, d.T, HG, status);
+        (int)d.G, d.T, HG, ksplit, status);
     return cudaGetLastError();
 }
 
@@ -703,10 +710,12 @@ cudaError_t launch_impl(const void* x, const float* dt, const float* A, const vo
 cudaError_t launch_chunk_out_tc(const void* x, const float* dt, const float* A, const void* B,
                                 const void* C, const float* D, const void* prev, void* y,
                                 const Dims& d, cudaStream_t s) {
-    if (d.Q == 256 && d.N == 128) return launch_impl<256, 128>(x, dt, A, B, C, D, prev, y, d, s);
-    if (d.Q == 256 && d.N == 64) return launch_impl<256, 64>(x, dt, A, B, C, D, prev, y, d, s);
-    if (d.Q == 128 && d.N == 128) return launch_impl<128, 128>(x, dt, A, B, C, D, prev, y, d, s);
-    if (d.Q == 128 && d.N == 64) return launch_impl<128, 64>(x, dt, A, B, C, D, prev, y, d, s);
+    int k = 1;
+    const Dims v = virtual_heads(d, &k);
+    if (v.Q == 256 && v.N == 128) return launch_impl<256, 128>(x, dt, A, B, C, D, prev, y, v, k, s);
+    if (v.Q == 256 && v.N == 64) return launch_impl<256, 64>(x, dt, A, B, C, D, prev, y, v, k, s);
+    if (v.Q == 128 && v.N == 128) return launch_impl<128, 128>(x, dt, A, B, C, D, prev, y, v, k, s);
+    if (v.Q == 128 && v.N == 64) return launch_impl<128, 64>(x, dt, A, B, C, D, prev, y, v, k, s);
     return cudaErrorNotSupported;
 }
 

@@ -89,13 +89,14 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
 
 // Walks work items in order: i -> (batch, chunk, head pair), advanced by
 // counters (one division per CTA, at the start); key names the B tile used.
+// Pairs are pairs of (virtual) heads of one group (HeadPairs).
 struct ItemIter {
     int64_t b, c, T;
-    int pair, pairs, hpg, G;
-    __device__ __forceinline__ void init(int64_t i, int pairs_, int64_t T_, int hpg_, int G_) {
+    int pair, pairs, ppg, G;
+    __device__ __forceinline__ void init(int64_t i, int pairs_, int64_t T_, int ppg_, int G_) {
         pairs = pairs_;
         T = T_;
-        hpg = hpg_;
+        ppg = ppg_;
         G = G_;
         const int64_t bc = i / pairs;
         pair = (int)(i - bc * pairs);
@@ -109,7 +110,7 @@ struct ItemIter {
         c = 0;
         ++b;
     }
-    __device__ __forceinline__ int g() const { return (2 * pair) / hpg; }
+    __device__ __forceinline__ int g() const { return pair / ppg; }
     __device__ __forceinline__ int64_t key() const { return (b * T + c) * G + g(); }
 };
 
@@ -120,7 +121,7 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tmX,
                       const __grid_constant__ CUtensorMap tmS, const float* __restrict__ dt,
                       const float* __restrict__ A, float* __restrict__ states,
                       float* __restrict__ logdecay, int64_t L, int H, int G, int64_t T,
-                      int64_t items, WaitCtx status) {
+                      int64_t items, int ksplit, WaitCtx status) {
     using S = StateSmem<Q, N>;
     constexpr bool kTrans = (N == 128);
     constexpr int kSt = S::kStages;
@@ -137,7 +138,10 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tmX,
     volatile int* s_flag = reinterpret_cast<volatile int*>(smem + S::kFlags);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int pairs = H / 2, hpg = H / G;
+    // H counts virtual heads (headdim 64); real head = virtual head / ksplit
+    const HeadPairs hp(H, G);
+    const int pairs = G * hp.per_group(), ppg = hp.per_group();
+    const int Hr = H / ksplit;
     const int64_t i0 = (int64_t)blockIdx.x * items / gridDim.x;
     const int64_t i1 = (int64_t)(blockIdx.x + 1) * items / gridDim.x;
 
@@ -168,7 +172,7 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tmX,
             uint32_t it = 0, nb = 0;
             int64_t key_prev = -1;
             ItemIter w;
-            w.init(i0, pairs, T, hpg, G);
+            w.init(i0, pairs, T, ppg, G);
             for (int64_t i = i0; i < i1 && ok; ++i, w.next()) {
                 const int t0 = (int)(w.c * Q);
                 const int64_t key = w.key();
@@ -186,7 +190,10 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tmX,
                     ++nb;
                     key_prev = key;
                 }
-                const int h0 = 2 * w.pair;
+                int gg, h0;
+                bool has1;
+                hp.map(w.pair, &gg, &h0, &has1);
+                const int h1x = has1 ? h0 + 1 : H;    // the phantom's x: out of range, zeros
                 for (int st = 0; st < kSt; ++st) {
                     const uint32_t slot = it % kRing;
                     if (it >= kRing)
@@ -196,7 +203,7 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tmX,
                     mbar_expect_tx(&bars[BAR_XFULL + slot], S::kStage);
                     tma_load_4d(dst, &tmX, &bars[BAR_XFULL + slot], 0, h0, t0 + st * kStageTok,
                                 (int)w.b);
-                    tma_load_4d(dst + S::kHeadStage, &tmX, &bars[BAR_XFULL + slot], 0, h0 + 1,
+                    tma_load_4d(dst + S::kHeadStage, &tmX, &bars[BAR_XFULL + slot], 0, h1x,
                                 t0 + st * kStageTok, (int)w.b);
                     ++it;
                 }
@@ -217,7 +224,7 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tmX,
             uint32_t it = 0, nb = 0, k = 0;
             int64_t key_prev = -1;
             ItemIter w;
-            w.init(i0, pairs, T, hpg, G);
+            w.init(i0, pairs, T, ppg, G);
             for (int64_t i = i0; i < i1 && ok; ++i, ++k, w.next()) {
                 const int64_t key = w.key();
                 if (key != key_prev) {
@@ -267,18 +274,29 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tmX,
         constexpr int kSegTok = Q / 4;        // tokens per segment
         const int hk = warp >> 2, sg = warp & 3;
         float dreg[kPer];
+        auto head_of = [&](const ItemIter& w, bool* real) {
+            int gg, h0;
+            bool has1;
+            hp.map(w.pair, &gg, &h0, &has1);
+            *real = hk == 0 || has1;
+            return h0 + hk;
+        };
         auto load_dt = [&](const ItemIter& w) {
             const int64_t t0 = w.c * Q;
             const int64_t len = (L - t0) < Q ? (L - t0) : Q;
+            bool real;
+            const int hv = head_of(w, &real);
 #pragma unroll
             for (int k = 0; k < kPer; ++k) {
                 const int j = sg * kSegTok + lane * kPer + k;
-                dreg[k] = (j < len) ? dt[(w.b * L + t0 + j) * H + 2 * w.pair + hk] : 0.f;
+                dreg[k] = (real && j < len) ? dt[(w.b * L + t0 + j) * Hr + hv / ksplit] : 0.f;
             }
         };
         // w_j of the item into buffer buf (published by the caller's barrier)
         auto prefix = [&](const ItemIter& w, int buf) {
-            const float Ah = A[2 * w.pair + hk];
+            bool real;
+            const int hv = head_of(w, &real);
+            const float Ah = real ? A[hv / ksplit] : 0.f;
             float v[kPer];
             float run = 0.f;                       // tokens past the sequence end add 0
 #pragma unroll
@@ -304,13 +322,15 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tmX,
             float* wk = s_w + (buf * 2 + hk) * Q + sg * kSegTok + lane * kPer;
 #pragma unroll
             for (int k = 0; k < kPer; ++k) wk[k] = expf(last - (v[k] + off)) * dreg[k];
-            if (sg == 0 && lane == 0) logdecay[(w.b * T + w.c) * H + 2 * w.pair + hk] = last;
+            // one log-decay per real head: the first of its virtual heads writes it
+            if (sg == 0 && lane == 0 && real && hv % ksplit == 0)
+                logdecay[(w.b * T + w.c) * Hr + hv / ksplit] = last;
         };
 
         bool fail = false;
         uint32_t it = 0;
         ItemIter wn;
-        wn.init(i0, pairs, T, hpg, G);
+        wn.init(i0, pairs, T, ppg, G);
         if (i0 < i1) {
             load_dt(wn);
             prefix(wn, 0);
@@ -367,7 +387,7 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tmX,
         uint32_t q = 0;                          // staging boxes written so far
         int64_t k = 0;
         ItemIter w;
-        w.init(i0, pairs, T, hpg, G);
+        w.init(i0, pairs, T, ppg, G);
         for (int64_t i = i0; i < i1; ++i, ++k, w.next()) {
             const uint32_t as = (uint32_t)(k & 1);
             const bool miss = !mbar_wait(&bars[BAR_ACCFULL + as], (uint32_t)((k >> 1) & 1), status);
@@ -380,6 +400,9 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tmX,
                 // lane m = state column n; column c = (head c / 64, p = c % 64).  The
                 // pair's 128 (head, p) rows of S are contiguous in HBM; each 32-column
                 // block goes out as one 32 x 128 fp32 box.
+                int gg, h0;
+                bool has1;
+                hp.map(w.pair, &gg, &h0, &has1);
 #pragma unroll 1
                 for (int cc = 0; cc < 4; ++cc, ++q) {
                     uint32_t r[32];
@@ -394,14 +417,19 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tmX,
                     named_bar_sync(2, 128);
                     if (m == 0) {
                         if (cc == 3) mbar_arrive(&bars[BAR_ACCEMPTY + as]);
-                        tma_store_3d(&tmS, buf, 0, 2 * w.pair * 64 + cc * 32, (int)(w.b * T + w.c));
+                        // (the phantom's rows, cc >= 2 without a second head, are not stored)
+                        if (cc < 2 || has1)
+                            tma_store_3d(&tmS, buf, 0, h0 * 64 + cc * 32, (int)(w.b * T + w.c));
                         bulk_commit_group();
                     }
                 }
             } else {
                 // lane m = (head m / 64, p = m % 64); columns = state n.  Each 32-column
-                // block of the pair's 128 rows goes out as one 128 x 32 fp32 box,
-                // staged with the 128-byte swizzle (chunk c of row m at c ^ (m & 7)).
+                // block of a head's 64 rows goes out as one 64 x 32 fp32 box, staged
+                // with the 128-byte swizzle (chunk c of row m at c ^ (m & 7)).
+                int gg, h0;
+                bool has1;
+                hp.map(w.pair, &gg, &h0, &has1);
 #pragma unroll 1
                 for (int cc = 0; cc < N / 32; ++cc, ++q) {
                     uint32_t r[32];
@@ -419,7 +447,10 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tmX,
                     named_bar_sync(2, 128);
                     if (m == 0) {
                         if (cc == N / 32 - 1) mbar_arrive(&bars[BAR_ACCEMPTY + as]);
-                        tma_store_3d(&tmS, buf, cc * 32, 2 * w.pair * 64, (int)(w.b * T + w.c));
+                        tma_store_3d(&tmS, buf, cc * 32, h0 * 64, (int)(w.b * T + w.c));
+                        if (has1)
+                            tma_store_3d(&tmS, buf + 64 * 32, cc * 32, (h0 + 1) * 64,
+                                         (int)(w.b * T + w.c));
                         bulk_commit_group();
                     }
                 }
@@ -452,7 +483,8 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tmX,
 
 template <int Q, int N>
 cudaError_t launch_impl(const void* x, const float* dt, const float* A, const void* B,
-                        float* states, float* logdecay, const Dims& d, cudaStream_t s) {
+                        float* states, float* logdecay, const Dims& d, int ksplit,
+                        cudaStream_t s) {
     using S = StateSmem<Q, N>;
     CUtensorMap tmX, tmB, tmS;
     const uint64_t xdims[4] = {64, (uint64_t)d.H, (uint64_t)d.L, (uint64_t)d.b};
@@ -467,17 +499,17 @@ cudaError_t launch_impl(const void* x, const float* dt, const float* A, const vo
     if (e != cudaSuccess) return e;
     {
         // states as rows (head, p) of N fp32 per (batch, chunk); N = 128: boxes of
-        // 32 rows x 128 (plain), N = 64: boxes of 128 rows x 32 (128-byte swizzle)
+        // 32 rows x 128 (plain), N = 64: boxes of 64 rows x 32 (128-byte swizzle)
         const uint64_t sdims[3] = {(uint64_t)N, (uint64_t)(d.H * 64), (uint64_t)(d.b * d.T)};
         const uint64_t sstr[2] = {(uint64_t)N * 4, (uint64_t)(d.H * 64 * N * 4)};
-        const uint32_t sbox128[3] = {128, 32, 1}, sbox64[3] = {32, 128, 1};
+        const uint32_t sbox128[3] = {128, 32, 1}, sbox64[3] = {32, 64, 1};
         e = make_tmap_f32_plain(&tmS, states, 3, sdims, sstr, N == 128 ? sbox128 : sbox64, N != 128);
         if (e != cudaSuccess) return e;
     }
     const sm100::WaitCtx status = make_wait_ctx();
     if (!status.word) return cudaErrorUnknown;
 
-    const int64_t items = d.b * d.T * (d.H / 2);
+    const int64_t items = d.b * d.T * d.G * HeadPairs((int)d.H, (int)d.G).per_group();
     if (items == 0) return cudaSuccess;
     int dev = 0, sms = 148;
     e = cudaGetDevice(&dev);
@@ -489,7 +521,7 @@ cudaError_t launch_impl(const void* x, const float* dt, const float* A, const vo
                              cudaFuncAttributeMaxDynamicSharedMemorySize, S::kAlloc);
     if (e != cudaSuccess) return e;
     chunk_state_tc_kernel<Q, N><<<(unsigned)grid, kThreads, S::kAlloc, s>>>(
-        tmX, tmB, tmS, dt, A, states, logdecay, d.L, (int)d.H, (int)d.G, d.T, items, status);
+        tmX, tmB, tmS, dt, A, states, logdecay, d.L, (int)d.H, (int)d.G, d.T, items, ksplit, status);
     return cudaGetLastError();
 }
 
@@ -497,10 +529,12 @@ cudaError_t launch_impl(const void* x, const float* dt, const float* A, const vo
 
 cudaError_t launch_chunk_state_tc(const void* x, const float* dt, const float* A, const void* B,
                                   float* states, float* logdecay, const Dims& d, cudaStream_t s) {
-    if (d.Q == 256 && d.N == 128) return launch_impl<256, 128>(x, dt, A, B, states, logdecay, d, s);
-    if (d.Q == 256 && d.N == 64) return launch_impl<256, 64>(x, dt, A, B, states, logdecay, d, s);
-    if (d.Q == 128 && d.N == 128) return launch_impl<128, 128>(x, dt, A, B, states, logdecay, d, s);
-    if (d.Q == 128 && d.N == 64) return launch_impl<128, 64>(x, dt, A, B, states, logdecay, d, s);
+    int k = 1;
+    const Dims v = virtual_heads(d, &k);
+    if (v.Q == 256 && v.N == 128) return launch_impl<256, 128>(x, dt, A, B, states, logdecay, v, k, s);
+    if (v.Q == 256 && v.N == 64) return launch_impl<256, 64>(x, dt, A, B, states, logdecay, v, k, s);
+    if (v.Q == 128 && v.N == 128) return launch_impl<128, 128>(x, dt, A, B, states, logdecay, v, k, s);
+    if (v.Q == 128 && v.N == 64) return launch_impl<128, 64>(x, dt, A, B, states, logdecay, v, k, s);
     return cudaErrorNotSupported;
 }
 

@@ -7,6 +7,7 @@
 #include <stdio.h>
 
 #include "../../include/ssd.h"
+#include "seqpar.h"
 #include "ssd_internal.h"
 #include "tc_host.h"
 #include "tc_kernels.h"
@@ -68,6 +69,19 @@ ssd_status_t check_dims(const ssd_dims_t* dims, int chunk, bool need_chunk, ssd_
 }
 
 bool tc_eligible(const ssd::Dims& d, ssd::Elt t) { return ssd::tc_supported(d, t); }
+
+// The block size the forward runs with.  The decomposition's result does not
+// depend on the block size (beyond rounding); the tensor-core kernels take
+// 128- and 256-token blocks, so a bf16 forward asked for smaller blocks runs
+// with 128-token blocks on them.  The step entry points keep the caller's
+// chunk size exactly (their outputs are per chunk).
+ssd::Dims forward_dims(const ssd::Dims& d, ssd::Elt t) {
+    if (t != ssd::Elt::BF16 || d.Q >= 128) return d;
+    ssd::Dims q = d;
+    q.Q = 128;
+    q.T = (d.L + 127) / 128;
+    return tc_eligible(q, t) ? q : d;
+}
 
 // The forward's data flow for these sizes (decided from the sizes alone, so
 // the workspace size needs no device).
@@ -175,7 +189,7 @@ ssd_status_t ssd_chunk_scan_fwd_workspace_size(const ssd_dims_t* dims, int chunk
     ssd::Dims d{}; ssd::Elt t = ssd::Elt::BF16;
     ssd_status_t st = check_dims(dims, chunk_size, true, dtype, &d, &t);
     if (st != SSD_OK) return st;
-    *bytes = ws_layout(d, t).total;
+    *bytes = ws_layout(forward_dims(d, t), t).total;
     return SSD_OK;
 }
 
@@ -183,13 +197,13 @@ int ssd_chunk_scan_fwd_uses_tensor_cores(const ssd_dims_t* dims, int chunk_size,
                                          ssd_dtype_t dtype) {
     ssd::Dims d{}; ssd::Elt t = ssd::Elt::BF16;
     if (check_dims(dims, chunk_size, true, dtype, &d, &t) != SSD_OK) return -1;
-    return tc_eligible(d, t) ? 1 : 0;
+    return tc_eligible(forward_dims(d, t), t) ? 1 : 0;
 }
 
 int ssd_chunk_scan_fwd_data_flow(const ssd_dims_t* dims, int chunk_size, ssd_dtype_t dtype) {
     ssd::Dims d{}; ssd::Elt t = ssd::Elt::BF16;
     if (check_dims(dims, chunk_size, true, dtype, &d, &t) != SSD_OK) return -1;
-    switch (pick_flow(d, t)) {
+    switch (pick_flow(forward_dims(d, t), t)) {
         case Flow::Walk: return SSD_FLOW_WALK_OUTPUT;
         case Flow::ThreeKernel: return SSD_FLOW_TC_THREE_KERNEL;
         default: return SSD_FLOW_SIMT;
@@ -205,6 +219,7 @@ ssd_status_t ssd_chunk_scan_fwd(const void* x, const float* dt, const float* A, 
     ssd::Dims d{}; ssd::Elt t = ssd::Elt::BF16;
     ssd_status_t st = check_dims(dims, chunk_size, true, dtype, &d, &t);
     if (st != SSD_OK) return st;
+    d = forward_dims(d, t);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     OPTIONAL_PTR(init_states);
     OPTIONAL_PTR(final_states);
@@ -336,12 +351,106 @@ ssd_status_t ssd_state_walk_fwd(const void* x, const float* dt, const float* A, 
     }
     if (!tc_eligible(d, t))
         return fail(SSD_ERR_UNSUPPORTED,
-                    "the state walk covers bf16, chunk 128/256, headdim 64, dstate 64/128 and an "
-                    "even number of heads per group");
+                    "the state walk covers bf16, chunk 128/256, headdim 64/128/192/256 and "
+                    "dstate 64/128");
     REQUIRE_PTR(x); REQUIRE_PTR(dt); REQUIRE_PTR(A); REQUIRE_PTR(B); REQUIRE_PTR(prev_states);
     REQUIRE_DEVICE(x);
     cudaError_t e = ssd::launch_state_walk_tc(x, dt, A, B, init_states, prev_states, final_states, d, s);
     return e == cudaSuccess ? SSD_OK : cuda_fail(e, "state-walk kernel");
+}
+
+// ---------------------------------------------------------------- sequence parallelism
+ssd_status_t ssd_seq_logdecay(const float* dt, const float* A, float* logdecay,
+                              const ssd_dims_t* dims, void* stream) {
+    g_detail[0] = 0;
+    ssd::Dims d{}; ssd::Elt t = ssd::Elt::BF16;
+    ssd_status_t st = check_dims(dims, 0, false, SSD_F32, &d, &t);
+    if (st != SSD_OK) return st;
+    if (d.b == 0) return SSD_OK;
+    REQUIRE_PTR(A); REQUIRE_PTR(logdecay);
+    if (d.L > 0) REQUIRE_PTR(dt);
+    REQUIRE_DEVICE(logdecay);
+    cudaError_t e = ssd::launch_seq_logdecay(dt, A, logdecay, d, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? SSD_OK : cuda_fail(e, "log-decay kernel");
+}
+
+ssd_status_t ssd_state_exchange_combine(const float* local_final, const float* logdecay,
+                                        const float* init, int rank, int nranks, float* h_in,
+                                        const ssd_dims_t* dims, void* stream) {
+    g_detail[0] = 0;
+    ssd::Dims d{}; ssd::Elt t = ssd::Elt::BF16;
+    ssd_status_t st = check_dims(dims, 0, false, SSD_F32, &d, &t);
+    if (st != SSD_OK) return st;
+    if (nranks < 1 || rank < 0 || rank > nranks)
+        return fail(SSD_ERR_INVALID_ARG, "need 0 <= rank (%d) <= nranks (%d), nranks >= 1", rank,
+                    nranks);
+    OPTIONAL_PTR(init);
+    if (d.b == 0) return SSD_OK;
+    REQUIRE_PTR(h_in);
+    if (rank > 0) {
+        REQUIRE_PTR(local_final);
+        REQUIRE_PTR(logdecay);
+    }
+    REQUIRE_DEVICE(h_in);
+    cudaError_t e = ssd::launch_state_combine(local_final, logdecay, init, h_in, rank, d,
+                                              static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? SSD_OK : cuda_fail(e, "state-combine kernel");
+}
+
+namespace {
+struct CorrLayout {
+    size_t prefix, hbf, total;
+};
+CorrLayout corr_layout(const ssd::Dims& d, ssd::Elt t) {
+    CorrLayout c;
+    c.prefix = 0;
+    c.hbf = round_up((size_t)(d.b * ssd::correction_tiles(d) * d.H) * 4, 256);
+    c.total = c.hbf;
+    if (ssd::correction_tc_supported(d, t)) c.total += round_up((size_t)(d.b * d.H * d.P * d.N) * 2, 256);
+    if (d.b == 0 || d.L == 0) c.total = 0;
+    return c;
+}
+}  // namespace
+
+ssd_status_t ssd_state_correction_workspace_size(const ssd_dims_t* dims, ssd_dtype_t dtype,
+                                                 size_t* bytes) {
+    g_detail[0] = 0;
+    if (!bytes) return fail(SSD_ERR_INVALID_ARG, "bytes is NULL");
+    ssd::Dims d{}; ssd::Elt t = ssd::Elt::BF16;
+    ssd_status_t st = check_dims(dims, 0, false, dtype, &d, &t);
+    if (st != SSD_OK) return st;
+    *bytes = corr_layout(d, t).total;
+    return SSD_OK;
+}
+
+ssd_status_t ssd_state_correction_fwd(const float* h_in, const float* dt, const float* A,
+                                      const void* C, void* y, float* final_states,
+                                      const ssd_dims_t* dims, ssd_dtype_t dtype,
+                                      void* workspace, size_t workspace_bytes, void* stream) {
+    g_detail[0] = 0;
+    ssd::Dims d{}; ssd::Elt t = ssd::Elt::BF16;
+    ssd_status_t st = check_dims(dims, 0, false, dtype, &d, &t);
+    if (st != SSD_OK) return st;
+    OPTIONAL_PTR(final_states);
+    if (d.b == 0 || d.L == 0) return SSD_OK;     // an empty shard: h_in passes through unchanged
+    REQUIRE_PTR(h_in); REQUIRE_PTR(dt); REQUIRE_PTR(A); REQUIRE_PTR(C); REQUIRE_PTR(y);
+    const CorrLayout w = corr_layout(d, t);
+    if (workspace_bytes < w.total)
+        return fail(SSD_ERR_INVALID_ARG, "workspace too small: %zu bytes given, %zu needed",
+                    workspace_bytes, w.total);
+    REQUIRE_PTR(workspace);
+    REQUIRE_DEVICE(y);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    char* ws = static_cast<char*>(workspace);
+    float* prefix = reinterpret_cast<float*>(ws + w.prefix);
+    const bool tc = ssd::correction_tc_supported(d, t);
+    __nv_bfloat16* hbf = tc ? reinterpret_cast<__nv_bfloat16*>(ws + w.hbf) : nullptr;
+    cudaError_t e = ssd::launch_correction_prep(h_in, dt, A, prefix, final_states, hbf, d, s);
+    if (e != cudaSuccess) return cuda_fail(e, "correction prep kernel");
+    e = tc ? ssd::launch_correction_tc(hbf, dt, A, C, prefix, y, d, s)
+           : ssd::launch_correction_simt(h_in, dt, A, C, prefix, y, d, t, s);
+    return e == cudaSuccess ? SSD_OK : cuda_fail(e, tc ? "correction kernel (tcgen05)"
+                                                       : "correction kernel");
 }
 
 ssd_status_t ssd_debug_expire_wait(unsigned int polls, void* stream) {

@@ -15,6 +15,9 @@
 // names a host-side stand-in), so the device address is looked up with
 // cudaGetSymbolAddress once per device, on the first call made while that
 // device is current; make that first call before any stream capture begins.
+// The address is cached per device ordinal for the life of the process, which
+// assumes the device's primary context throughout: no cudaDeviceReset, and no
+// other driver-API context made current between calls.
 //
 // Every call shares the one array and leaves its last contents behind.  The
 // forward writes every scratch byte it reads earlier in the same call, so

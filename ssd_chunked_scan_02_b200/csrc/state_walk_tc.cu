@@ -9,8 +9,10 @@
 // chunk per step; "Transformers are SSMs" (CiteArk), AI research summary: the
 // chunk's contribution is one dense contraction.
 //
-// One CTA per (batch, head pair) walks the chunks in order; S_c never leaves
-// the chip.  Tensor memory holds two fp32 tiles: the running state h and the
+// One CTA per (batch, head pair of one group) walks the chunks in order; S_c
+// never leaves the chip.  Heads are the kernels' virtual heads of headdim 64
+// (a head of headdim 64 k is k of them); a group with an odd number of heads
+// pairs its last head with a zero phantom.  Tensor memory holds two fp32 tiles: the running state h and the
 // chunk's accumulator S.  The MMAs of chunk c write S from zero; the
 // epilogue warps then read h and S, form h' = exp(cs_last) h + S, store h'
 // back over h and write it out as the state entering chunk c + 1 (bf16), or
@@ -99,16 +101,21 @@ state_walk_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
                      const float* __restrict__ dt, const float* __restrict__ A,
                      const float* __restrict__ init, __nv_bfloat16* __restrict__ prev,
                      float* __restrict__ fin, int64_t L, int H, int G, int64_t T,
-                     WaitCtx status) {
+                     int ksplit, WaitCtx status) {
     using S = WalkSmem<Q, N>;
     constexpr bool kTrans = (N == 128);
     constexpr int kNSub = Q / kSub;
     constexpr int kStages = S::kStages;
     constexpr int kSSlots = S::kSSlots;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int64_t b = blockIdx.x / (H / 2);
-    const int h0 = 2 * (int)(blockIdx.x % (H / 2));
-    const int g = h0 / (H / G);
+    // H counts virtual heads (headdim 64); real head = virtual head / ksplit
+    const HeadPairs hp(H, G);
+    const int64_t b = blockIdx.x / (G * hp.per_group());
+    int g, h0;
+    bool has1;
+    hp.map((int)(blockIdx.x % (G * hp.per_group())), &g, &h0, &has1);
+    const int Hr = H / ksplit;
+    const int h1x = has1 ? h0 + 1 : H;       // the phantom's x is read out of range: zeros
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
@@ -154,13 +161,13 @@ state_walk_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
                     const int64_t sp = si + kPrefetch;
                     const int prow = (int)((sp / kNSub) * Q + (sp % kNSub) * kSub);
                     tma_prefetch_4d(&tmX, 0, h0, prow, (int)b);
-                    tma_prefetch_4d(&tmX, 0, h0 + 1, prow, (int)b);
+                    if (has1) tma_prefetch_4d(&tmX, 0, h0 + 1, prow, (int)b);
                     for (int nb = 0; nb < N / 64; ++nb) tma_prefetch_4d(&tmB, nb * 64, g, prow, (int)b);
                 }
                 uint8_t* ent = ring + e * S::kEntry;
                 mbar_expect_tx(&bars[BAR_FULL + e], S::kEntry);
                 tma_load_4d(ent, &tmX, &bars[BAR_FULL + e], 0, h0, row, (int)b);
-                tma_load_4d(ent + kSub * 128, &tmX, &bars[BAR_FULL + e], 0, h0 + 1, row, (int)b);
+                tma_load_4d(ent + kSub * 128, &tmX, &bars[BAR_FULL + e], 0, h1x, row, (int)b);
                 for (int nb = 0; nb < N / 64; ++nb)
                     tma_load_4d(ent + S::kXPart + nb * kSub * 128, &tmB, &bars[BAR_FULL + e],
                                 nb * 64, g, row, (int)b);
@@ -213,13 +220,14 @@ state_walk_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
         constexpr int kPer = Q / 64;
         constexpr int kHalf = Q / 2;
         const int hk = warp >> 1, sg = warp & 1;
-        const float Ak = A[h0 + hk];
+        const bool real = hk == 0 || has1;
+        const float Ak = real ? A[(h0 + hk) / ksplit] : 0.f;
         float dreg[kPer];
         auto load_dt = [&](int64_t c) {
 #pragma unroll
             for (int k = 0; k < kPer; ++k) {
                 const int64_t tok = c * Q + sg * kHalf + lane * kPer + k;
-                dreg[k] = (tok < L) ? dt[(b * L + tok) * H + h0 + hk] : 0.f;
+                dreg[k] = (real && tok < L) ? dt[(b * L + tok) * Hr + (h0 + hk) / ksplit] : 0.f;
             }
         };
         // w_j and the chunk decay of this head into buffer buf
@@ -310,13 +318,16 @@ state_walk_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
             for (int cc = 0; cc < 4; ++cc) {
                 const int k = cc >> 1, p0 = (cc & 1) * 32;
                 const int64_t srow = ((b * H + h0 + k) * 64 + p0) * (int64_t)N + n;
+                const bool real = k == 0 || has1;
                 uint32_t r[32];
 #pragma unroll
                 for (int e = 0; e < 32; ++e)
-                    r[e] = __float_as_uint(init ? init[srow + (int64_t)e * N] : 0.f);
-                __nv_bfloat16* pr = prev + (((b * T) * H + h0 + k) * 64 + p0) * (int64_t)N + n;
+                    r[e] = __float_as_uint((init && real) ? init[srow + (int64_t)e * N] : 0.f);
+                if (real) {
+                    __nv_bfloat16* pr = prev + (((b * T) * H + h0 + k) * 64 + p0) * (int64_t)N + n;
 #pragma unroll
-                for (int e = 0; e < 32; ++e) pr[(int64_t)e * N] = __float2bfloat16_rn(__uint_as_float(r[e]));
+                    for (int e = 0; e < 32; ++e) pr[(int64_t)e * N] = __float2bfloat16_rn(__uint_as_float(r[e]));
+                }
                 uint32_t lo[16], hi[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
@@ -329,11 +340,12 @@ state_walk_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
         } else {
             // lane m = (head m / 64, p = m % 64); TMEM columns = state n (N = 64)
             const int k = m >> 6, p = m & 63;
+            const bool real = k == 0 || has1;
             const int64_t srow = ((b * H + h0 + k) * 64 + p) * (int64_t)N;
 #pragma unroll 1
             for (int cc = 0; cc < N / 32; ++cc) {
                 uint32_t r[32];
-                if (init) {
+                if (init && real) {
                     const float4* s4 = reinterpret_cast<const float4*>(init + srow + cc * 32);
 #pragma unroll
                     for (int q = 0; q < 8; ++q) {
@@ -349,7 +361,7 @@ state_walk_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
                 }
                 __nv_bfloat16* pr = prev + (((b * T) * H + h0 + k) * 64 + p) * (int64_t)N + cc * 32;
 #pragma unroll
-                for (int e = 0; e < 32; e += 8) {
+                for (int e = 0; e < 32 && real; e += 8) {
                     uint4 v;
                     v.x = pack_bf16x2(__uint_as_float(r[e]), __uint_as_float(r[e + 1]));
                     v.y = pack_bf16x2(__uint_as_float(r[e + 2]), __uint_as_float(r[e + 3]));
@@ -413,6 +425,7 @@ state_walk_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
 #pragma unroll 1
                 for (int cc = 0; cc < 4; ++cc) {
                     const int k = cc >> 1, p0 = (cc & 1) * 32;
+                    if (k == 1 && !has1) break;       // the phantom's state is not written
                     uint32_t hr[32];
                     tmem_ld32(tH + cc * 32, hr);
                     if (!last) {
@@ -429,10 +442,12 @@ state_walk_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
                 }
             } else {
                 const int k = m >> 6, p = m & 63;
+                const bool real = k == 0 || has1;
 #pragma unroll 1
                 for (int cc = 0; cc < N / 32; ++cc) {
                     uint32_t hr[32];
                     tmem_ld32(tH + cc * 32, hr);
+                    if (!real) continue;                  // the phantom's state is not written
                     if (!last) {
                         __nv_bfloat16* pr =
                             prev + (((b * T + c + 1) * H + h0 + k) * 64 + p) * (int64_t)N + cc * 32;
@@ -476,7 +491,8 @@ state_walk_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
 
 template <int Q, int N>
 cudaError_t launch_impl(const void* x, const float* dt, const float* A, const void* B,
-                        const float* init, void* prev, float* fin, const Dims& d, cudaStream_t s) {
+                        const float* init, void* prev, float* fin, const Dims& d, int ksplit,
+                        cudaStream_t s) {
     using S = WalkSmem<Q, N>;
     CUtensorMap tmX, tmB;
     const uint64_t xdims[4] = {64, (uint64_t)d.H, (uint64_t)d.L, (uint64_t)d.b};
@@ -493,10 +509,10 @@ cudaError_t launch_impl(const void* x, const float* dt, const float* A, const vo
     e = cudaFuncSetAttribute(state_walk_tc_kernel<Q, N>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, S::kAlloc);
     if (e != cudaSuccess) return e;
-    const int64_t grid = d.b * (d.H / 2);
+    const int64_t grid = d.b * d.G * HeadPairs((int)d.H, (int)d.G).per_group();
     state_walk_tc_kernel<Q, N><<<(unsigned)grid, kThreads, S::kAlloc, s>>>(
         tmX, tmB, dt, A, init, static_cast<__nv_bfloat16*>(prev), fin, d.L, (int)d.H, (int)d.G,
-        d.T, status);
+        d.T, ksplit, status);
     return cudaGetLastError();
 }
 
@@ -507,18 +523,23 @@ bool walk_preferred(const Dims& d) {
     // the walk pays off once there are enough walkers to keep most SMs busy
     // (measured: 96 walkers and more beat chunk states + state pass at every
     // workload shape, 64 and fewer lose to them).
-    const int64_t walkers = d.b * (d.H / 2);
+    int ksplit = 1;
+    const Dims v = virtual_heads(d, &ksplit);
+    const int64_t walkers = v.b * v.G * HeadPairs((int)v.H, (int)v.G).per_group();
     return walkers >= 96 && walkers <= 0x7fffffffLL;
 }
 
 cudaError_t launch_state_walk_tc(const void* x, const float* dt, const float* A, const void* B,
                                  const float* init, void* prev, float* fin, const Dims& d,
                                  cudaStream_t s) {
-    if (d.b * (d.H / 2) > 0x7fffffffLL) return cudaErrorInvalidValue;
-    if (d.Q == 256 && d.N == 128) return launch_impl<256, 128>(x, dt, A, B, init, prev, fin, d, s);
-    if (d.Q == 256 && d.N == 64) return launch_impl<256, 64>(x, dt, A, B, init, prev, fin, d, s);
-    if (d.Q == 128 && d.N == 128) return launch_impl<128, 128>(x, dt, A, B, init, prev, fin, d, s);
-    if (d.Q == 128 && d.N == 64) return launch_impl<128, 64>(x, dt, A, B, init, prev, fin, d, s);
+    int k = 1;
+    const Dims v = virtual_heads(d, &k);
+    if (v.b * v.G * HeadPairs((int)v.H, (int)v.G).per_group() > 0x7fffffffLL)
+        return cudaErrorInvalidValue;
+    if (v.Q == 256 && v.N == 128) return launch_impl<256, 128>(x, dt, A, B, init, prev, fin, v, k, s);
+    if (v.Q == 256 && v.N == 64) return launch_impl<256, 64>(x, dt, A, B, init, prev, fin, v, k, s);
+    if (v.Q == 128 && v.N == 128) return launch_impl<128, 128>(x, dt, A, B, init, prev, fin, v, k, s);
+    if (v.Q == 128 && v.N == 64) return launch_impl<128, 64>(x, dt, A, B, init, prev, fin, v, k, s);
     return cudaErrorNotSupported;
 }
 

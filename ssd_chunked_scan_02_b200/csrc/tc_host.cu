@@ -44,12 +44,12 @@ sm100::WaitCtx make_wait_ctx() {
 
 bool tc_supported(const Dims& d, Elt t) {
     if (t != Elt::BF16) return false;
-    if (d.P != 64) return false;
+    if (d.P % 64 != 0 || d.P > 256) return false;     // k virtual heads of headdim 64
     if (d.N != 64 && d.N != 128) return false;
     if (d.Q != 128 && d.Q != 256) return false;
-    if ((d.H / d.G) % 2 != 0) return false;
     if (d.L <= 0 || d.b <= 0) return false;
     if (d.L > 0x7fffffffLL || d.b > 0x7fffffffLL) return false;   // TMA coordinates are int32
+    if (d.H * (d.P / 64) > 0x7fffffffLL / 64) return false;       // head rows of the state maps
     return true;
 }
 

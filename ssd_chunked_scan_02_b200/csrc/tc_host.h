@@ -23,7 +23,8 @@ cudaError_t make_tmap_f32_plain(CUtensorMap* map, const void* base, int rank,
 bool tma_encoder_available();
 
 // Device address of the status word that bounded waits write (current
-// device; looked up once per device).  nullptr if unavailable.
+// device; looked up once per device ordinal and kept for the process, which
+// assumes the device's primary context throughout).  nullptr if unavailable.
 unsigned int* device_status_ptr();
 
 // Launches one CTA whose bounded mbarrier wait (at most `polls` polls) is

@@ -7,6 +7,36 @@
 
 namespace ssd {
 
+// The tcgen05 kernels work on heads of headdim 64.  A head of headdim 64 k is
+// handled as k such (virtual) heads that share dt, A and D -- the rows of a
+// state evolve independently, and x, y and the states (b, ., H, P, .) are
+// the same memory as (b, ., H k, 64, .).  Returns the virtual sizes (H k,
+// P 64) and k.
+inline Dims virtual_heads(const Dims& d, int* ksplit) {
+    Dims v = d;
+    *ksplit = (int)(d.P / 64);
+    v.H = d.H * *ksplit;
+    v.P = 64;
+    return v;
+}
+
+// The state kernels work on pairs of (virtual) heads of one group.  A group
+// with an odd number of heads pairs its last head with a phantom: its x is
+// read as zeros (an out-of-range head coordinate) and its outputs are not
+// written.
+struct HeadPairs {
+    int hpg, ppg;      // heads and pairs per group
+    __host__ __device__ explicit HeadPairs(int H, int G) : hpg(H / G), ppg((H / G + 1) / 2) {}
+    __host__ __device__ int per_group() const { return ppg; }
+    // pair -> its group, first head, and whether the second head exists
+    __host__ __device__ void map(int pair, int* g, int* h0, bool* has1) const {
+        *g = pair / ppg;
+        const int l = pair - *g * ppg;
+        *h0 = *g * hpg + 2 * l;
+        *has1 = 2 * l + 1 < hpg;
+    }
+};
+
 // True when the tensor-core kernels cover these sizes and dtype.
 bool tc_supported(const Dims& d, Elt t);
 

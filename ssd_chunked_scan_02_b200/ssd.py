@@ -27,7 +27,8 @@ EXPORTED = ("ssd_status_string", "ssd_last_error_detail", "ssd_chunk_scan_fwd_wo
             "ssd_chunk_output_fwd", "ssd_chunk_scan_fwd_uses_tensor_cores",
             "ssd_chunk_scan_fwd_noalloc", "ssd_poll_device_status", "ssd_state_walk_fwd",
             "ssd_debug_expire_wait", "ssd_chunk_scan_bwd_workspace_size", "ssd_chunk_scan_bwd",
-            "ssd_chunk_scan_fwd_data_flow")
+            "ssd_chunk_scan_fwd_data_flow", "ssd_seq_logdecay", "ssd_state_exchange_combine",
+            "ssd_state_correction_workspace_size", "ssd_state_correction_fwd")
 
 # ssd_chunk_scan_fwd_data_flow results
 SSD_FLOW_SIMT, SSD_FLOW_TC_THREE_KERNEL, SSD_FLOW_WALK_OUTPUT = 0, 1, 2
@@ -97,6 +98,17 @@ def load(path: str = LIB_PATH):
     lib.ssd_chunk_scan_bwd.restype = ctypes.c_int
     lib.ssd_chunk_scan_bwd.argtypes = [_vp] * 16 + [dims_p, ctypes.c_int, _vp, ctypes.c_size_t,
                                                     _vp]
+    lib.ssd_seq_logdecay.restype = ctypes.c_int
+    lib.ssd_seq_logdecay.argtypes = [_vp] * 3 + [dims_p, _vp]
+    lib.ssd_state_exchange_combine.restype = ctypes.c_int
+    lib.ssd_state_exchange_combine.argtypes = [_vp] * 3 + [ctypes.c_int, ctypes.c_int, _vp, dims_p,
+                                                           _vp]
+    lib.ssd_state_correction_workspace_size.restype = ctypes.c_int
+    lib.ssd_state_correction_workspace_size.argtypes = [dims_p, ctypes.c_int,
+                                                        ctypes.POINTER(ctypes.c_size_t)]
+    lib.ssd_state_correction_fwd.restype = ctypes.c_int
+    lib.ssd_state_correction_fwd.argtypes = [_vp] * 6 + [dims_p, ctypes.c_int, _vp,
+                                                         ctypes.c_size_t, _vp]
     _lib = lib
     return lib
 
@@ -414,3 +426,76 @@ def ssd_chunk_scan_bwd(x, dt, A, B, C, D, dy, init_states=None, dfinal_states=No
                                        _stream(stream, dev))
     _check(st, "ssd_chunk_scan_bwd")
     return out
+
+
+# ---------------------------------------------------------------- sequence parallelism
+def ssd_seq_logdecay(dt, A, stream=None):
+    """sum_t dt[b,t,h] * A[h] over the (shard's) sequence: (b, H) fp32."""
+    b, L, H = dt.shape
+    _expect("dt", dt, (b, L, H), torch.float32, dt.device)
+    _expect("A", A, (H,), torch.float32, dt.device)
+    dev = _device_of(dt)
+    out = torch.empty((b, H), device=dt.device, dtype=torch.float32)
+    dims = make_dims(b, L, H, 1, 1, 1)
+    with torch.cuda.device(dev):
+        st = load().ssd_seq_logdecay(_ptr(dt), _ptr(A), _ptr(out), ctypes.byref(dims),
+                                     _stream(stream, dev))
+    _check(st, "ssd_seq_logdecay")
+    return out
+
+
+def ssd_state_exchange_combine(local_final, logdecay, rank: int, init_states=None, out=None,
+                               stream=None):
+    """The state entering rank ``rank``'s shard from the gathered local final
+    states (R,b,H,P,N) and log-decays (R,b,H) of all ranks (rank order) and
+    the state entering the whole sequence (None = zero).  rank = R gives the
+    state after the whole sequence."""
+    R, b, H, P, N = local_final.shape
+    dev = local_final.device
+    _expect("logdecay", logdecay, (R, b, H), torch.float32, dev)
+    _expect("local_final", local_final, (R, b, H, P, N), torch.float32, dev)
+    _expect("init_states", init_states, (b, H, P, N), torch.float32, dev)
+    _expect("out", out, (b, H, P, N), torch.float32, dev)
+    dev = _device_of(local_final)
+    if out is None:
+        out = torch.empty((b, H, P, N), device=local_final.device, dtype=torch.float32)
+    dims = make_dims(b, 0, H, P, N, 1)
+    with torch.cuda.device(dev):
+        st = load().ssd_state_exchange_combine(_ptr(local_final), _ptr(logdecay), _ptr(init_states),
+                                               int(rank), int(R), _ptr(out), ctypes.byref(dims),
+                                               _stream(stream, dev))
+    _check(st, "ssd_state_exchange_combine")
+    return out
+
+
+def ssd_state_correction_workspace_size(dims: ssd_dims_t, dtype: torch.dtype) -> int:
+    n = ctypes.c_size_t(0)
+    _check(load().ssd_state_correction_workspace_size(ctypes.byref(dims), _dtype_code(dtype),
+                                                      ctypes.byref(n)),
+           "ssd_state_correction_workspace_size")
+    return int(n.value)
+
+
+def ssd_state_correction_fwd(h_in, dt, A, C, y, final_states=None, workspace=None, stream=None):
+    """In place: y_t += exp(cs_t) h_in C_t over the shard and, if given,
+    final_states += exp(cs_last) h_in.  h_in (b,H,P,N) fp32."""
+    b, L, H, P = y.shape
+    G, N = C.shape[2], C.shape[3]
+    dev = y.device
+    _expect("h_in", h_in, (b, H, P, N), torch.float32, dev)
+    _expect("dt", dt, (b, L, H), torch.float32, dev)
+    _expect("A", A, (H,), torch.float32, dev)
+    _expect("C", C, (b, L, G, N), y.dtype, dev)
+    _expect("final_states", final_states, (b, H, P, N), torch.float32, dev)
+    dev = _device_of(y)
+    dims = make_dims(b, L, H, P, N, G)
+    need = ssd_state_correction_workspace_size(dims, y.dtype)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), device=y.device, dtype=torch.uint8)
+    with torch.cuda.device(dev):
+        st = load().ssd_state_correction_fwd(_ptr(h_in), _ptr(dt), _ptr(A), _ptr(C), _ptr(y),
+                                             _ptr(final_states), ctypes.byref(dims),
+                                             _dtype_code(y.dtype), _ptr(workspace),
+                                             workspace.numel(), _stream(stream, dev))
+    _check(st, "ssd_state_correction_fwd")
+    return y

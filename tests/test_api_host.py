@@ -61,12 +61,16 @@ def _round(v):
     (1, 256, 4, 16, 16, 1, 64, ssd.SSD_F32),
     (2, 600, 4, 64, 128, 2, 128, ssd.SSD_BF16),   # ragged: 5 chunks, last one partial
     (3, 1, 2, 3, 5, 1, 16, ssd.SSD_F32),
+    (2, 300, 4, 64, 128, 1, 64, ssd.SSD_BF16),    # bf16 below 128: runs 128-token chunks
+    (2, 300, 4, 32, 128, 1, 64, ssd.SSD_BF16),    # headdim 32: SIMT, chunks as asked
 ])
 def test_workspace_size_formula(lib, b, L, H, P, N, G, Q, dt):
     dims = ssd.make_dims(b, L, H, P, N, G)
     st, n = _ws(dims, Q, dt)
     assert st == ssd.SSD_OK
-    T = (L + Q - 1) // Q
+    tc = lib.ssd_chunk_scan_fwd_uses_tensor_cores(ctypes.byref(dims), Q, dt) == 1
+    Qe = max(Q, 128) if tc else Q
+    T = (L + Qe - 1) // Qe
     elt = 4 if dt == ssd.SSD_F32 else 2
     ns = b * T * H * P * N
     if lib.ssd_chunk_scan_fwd_data_flow(ctypes.byref(dims), Q, dt) == ssd.SSD_FLOW_WALK_OUTPUT:
@@ -87,6 +91,11 @@ def test_workspace_size_formula(lib, b, L, H, P, N, G, Q, dt):
     (2, 600, 4, 64, 128, 1, 256, ssd.SSD_BF16, ssd.SSD_FLOW_TC_THREE_KERNEL),
     (4, 8192, 80, 64, 128, 1, 256, ssd.SSD_F32, ssd.SSD_FLOW_SIMT),
     (4, 8192, 80, 32, 128, 1, 256, ssd.SSD_BF16, ssd.SSD_FLOW_SIMT),
+    (4, 8192, 40, 128, 128, 1, 256, ssd.SSD_BF16, ssd.SSD_FLOW_WALK_OUTPUT),  # 80 virtual heads
+    (2, 600, 6, 64, 128, 2, 256, ssd.SSD_BF16, ssd.SSD_FLOW_TC_THREE_KERNEL),  # 3 heads a group
+    (16, 600, 10, 64, 128, 2, 256, ssd.SSD_BF16, ssd.SSD_FLOW_WALK_OUTPUT),   # 96 walkers
+    (2, 300, 4, 64, 128, 1, 64, ssd.SSD_BF16, ssd.SSD_FLOW_TC_THREE_KERNEL),  # chunk 64
+    (2, 300, 4, 64, 48, 1, 256, ssd.SSD_BF16, ssd.SSD_FLOW_SIMT),             # dstate 48
 ])
 def test_data_flow_query(lib, b, L, H, P, N, G, Q, dt, flow):
     dims = ssd.make_dims(b, L, H, P, N, G)
@@ -290,3 +299,41 @@ def test_backward_rejects_bad_arguments_before_launching(lib):
     st = call(dims, ctypes.c_void_p(0x1000000), 16, fake)
     assert st == ssd.SSD_ERR_INVALID_ARG
     assert b"workspace_bytes" in L.ssd_last_error_detail()
+
+
+# ------------------------------------------------------------------ sequence parallelism
+def test_seqpar_entries_reject_bad_arguments_before_launching(lib):
+    dims = ssd.make_dims(2, 64, 4, 8, 8, 1)
+    d = ctypes.byref(dims)
+    assert lib.ssd_seq_logdecay(A16, None, A16, d, None) == ssd.SSD_ERR_INVALID_ARG
+    assert lib.ssd_seq_logdecay(A16 + 4, A16, A16, d, None) == ssd.SSD_ERR_INVALID_ARG
+    # rank outside [0, nranks], nranks < 1, missing gathered values for rank > 0
+    assert lib.ssd_state_exchange_combine(A16, A16, None, 3, 2, A16, d, None) == \
+        ssd.SSD_ERR_INVALID_ARG
+    assert lib.ssd_state_exchange_combine(A16, A16, None, -1, 2, A16, d, None) == \
+        ssd.SSD_ERR_INVALID_ARG
+    assert lib.ssd_state_exchange_combine(A16, A16, None, 0, 0, A16, d, None) == \
+        ssd.SSD_ERR_INVALID_ARG
+    assert lib.ssd_state_exchange_combine(None, A16, None, 1, 2, A16, d, None) == \
+        ssd.SSD_ERR_INVALID_ARG
+    assert lib.ssd_state_exchange_combine(A16, A16, None, 1, 2, None, d, None) == \
+        ssd.SSD_ERR_INVALID_ARG
+    n = ctypes.c_size_t(0)
+    assert lib.ssd_state_correction_workspace_size(d, ssd.SSD_F32, ctypes.byref(n)) == ssd.SSD_OK
+    # tile prefixes of 128-token tiles, (b, tiles, H) fp32
+    assert n.value == _round(2 * 1 * 4 * 4)
+    st = lib.ssd_state_correction_fwd(A16, A16, A16, A16, A16, None, d, ssd.SSD_F32, A16,
+                                      n.value - 1, None)
+    assert st == ssd.SSD_ERR_INVALID_ARG and "workspace" in lib.ssd_last_error_detail().decode()
+    st = lib.ssd_state_correction_fwd(None, A16, A16, A16, A16, None, d, ssd.SSD_F32, A16,
+                                      n.value, None)
+    assert st == ssd.SSD_ERR_INVALID_ARG
+
+
+def test_correction_workspace_size_tensor_core_shape(lib):
+    """bf16, P 64, N 128: tile prefixes plus h_in rounded to bf16."""
+    dims = ssd.make_dims(4, 4096, 80, 64, 128, 1)
+    n = ctypes.c_size_t(0)
+    assert lib.ssd_state_correction_workspace_size(ctypes.byref(dims), ssd.SSD_BF16,
+                                                   ctypes.byref(n)) == ssd.SSD_OK
+    assert n.value == _round(4 * 32 * 80 * 4) + _round(4 * 80 * 64 * 128 * 2)

@@ -51,6 +51,32 @@ SMALL_BF16 = [
 ]
 
 
+# shapes the tensor cores cover through virtual heads (headdim 64 k), phantom
+# heads (an odd number of heads per group) and 128-token chunks for smaller
+# chunk sizes, through both tensor-core data flows
+TC_SHAPES = [
+    # name,                     b,  L,   H,  P,   N,  G,  Q,  init
+    ("tc_p128_three_kernel", 2, 600, 4, 128, 128, 1, 256, True),
+    ("tc_p128_walk_n64", 8, 700, 24, 128, 64, 2, 128, True),
+    ("tc_p192_odd_virtual", 2, 400, 3, 192, 64, 1, 128, True),
+    ("tc_p256", 1, 500, 2, 256, 128, 1, 256, True),
+    ("tc_odd_hpg_three_kernel", 2, 600, 6, 64, 128, 2, 256, True),
+    ("tc_odd_hpg_n64_three_kernel", 1, 700, 10, 64, 64, 2, 128, True),
+    ("tc_odd_hpg_walk", 16, 600, 10, 64, 128, 2, 256, True),
+    ("tc_odd_hpg_walk_n64", 48, 300, 3, 64, 64, 1, 128, False),
+    ("tc_q32_runs_q128", 2, 333, 4, 64, 128, 1, 32, True),
+    ("tc_q16_ragged", 1, 77, 2, 64, 64, 1, 16, True),
+]
+
+
+@pytest.mark.parametrize("case", TC_SHAPES, ids=[c[0] for c in TC_SHAPES])
+def test_tensor_core_shapes(case):
+    name, b, L, H, P, N, G, Q, init = case
+    dims = ssd.make_dims(b, L, H, P, N, G)
+    assert ssd.ssd_chunk_scan_fwd_uses_tensor_cores(dims, Q, torch.bfloat16) == 1
+    _check_full(_w(name, b, L, H, P, N, G, Q, "bf16", init, seed=120 + len(name)))
+
+
 @pytest.mark.parametrize("case", SMALL_BF16, ids=[c[0] for c in SMALL_BF16])
 def test_small_bf16(case):
     name, b, L, H, P, N, G, Q, init = case
@@ -157,7 +183,9 @@ def test_decode_f32_small_full():
 # --- each step of the forward on its own -------------------------------------------------
 
 STAGE_CASES = [("bf16", 2, 600, 4, 64, 128, 1, 256), ("bf16", 1, 512, 4, 64, 64, 2, 128),
-               ("f32", 2, 333, 3, 16, 16, 1, 64)]
+               ("f32", 2, 333, 3, 16, 16, 1, 64),
+               ("bf16", 2, 300, 6, 64, 64, 2, 128),       # 3 heads a group: phantom heads
+               ("bf16", 1, 400, 3, 128, 128, 1, 256)]     # headdim 128: virtual heads
 
 
 def _oracle_chunk_views(inp, Q):
@@ -207,7 +235,8 @@ def test_stage_state_passing(case):
 
 
 WALK_CASES = [(2, 600, 4, 64, 128, 1, 256, True), (1, 512, 4, 64, 64, 2, 128, False),
-              (3, 100, 2, 64, 128, 1, 128, True), (1, 777, 6, 64, 64, 1, 256, True)]
+              (3, 100, 2, 64, 128, 1, 128, True), (1, 777, 6, 64, 64, 1, 256, True),
+              (2, 300, 6, 64, 128, 2, 256, True), (1, 400, 3, 128, 64, 1, 128, True)]
 
 
 @pytest.mark.parametrize("case", WALK_CASES, ids=lambda c: "_".join(map(str, c)))
