@@ -118,7 +118,8 @@ template <int Q, int N>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tmX,
                       const __grid_constant__ CUtensorMap tmB,
-                      const __grid_constant__ CUtensorMap tmS, const float* __restrict__ dt,
+                      const __grid_constant__ CUtensorMap tmS,
+                      const __grid_constant__ CUtensorMap tmS1, const float* __restrict__ dt,
                       const float* __restrict__ A, float* __restrict__ states,
                       float* __restrict__ logdecay, int64_t L, int H, int G, int64_t T,
                       int64_t items, int ksplit, WaitCtx status) {
@@ -425,8 +426,9 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tmX,
                 }
             } else {
                 // lane m = (head m / 64, p = m % 64); columns = state n.  Each 32-column
-                // block of a head's 64 rows goes out as one 64 x 32 fp32 box, staged
-                // with the 128-byte swizzle (chunk c of row m at c ^ (m & 7)).
+                // block of the pair's 128 rows goes out as one 128 x 32 fp32 box (64 x
+                // 32 for a head paired with a phantom), staged with the 128-byte
+                // swizzle (chunk c of row m at c ^ (m & 7)).
                 int gg, h0;
                 bool has1;
                 hp.map(w.pair, &gg, &h0, &has1);
@@ -447,10 +449,9 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tmX,
                     named_bar_sync(2, 128);
                     if (m == 0) {
                         if (cc == N / 32 - 1) mbar_arrive(&bars[BAR_ACCEMPTY + as]);
-                        tma_store_3d(&tmS, buf, cc * 32, h0 * 64, (int)(w.b * T + w.c));
-                        if (has1)
-                            tma_store_3d(&tmS, buf + 64 * 32, cc * 32, (h0 + 1) * 64,
-                                         (int)(w.b * T + w.c));
+                        // the pair's 128 rows as one box; a phantom's half is not stored
+                        if (has1) tma_store_3d(&tmS, buf, cc * 32, h0 * 64, (int)(w.b * T + w.c));
+                        else tma_store_3d(&tmS1, buf, cc * 32, h0 * 64, (int)(w.b * T + w.c));
                         bulk_commit_group();
                     }
                 }
@@ -486,7 +487,7 @@ cudaError_t launch_impl(const void* x, const float* dt, const float* A, const vo
                         float* states, float* logdecay, const Dims& d, int ksplit,
                         cudaStream_t s) {
     using S = StateSmem<Q, N>;
-    CUtensorMap tmX, tmB, tmS;
+    CUtensorMap tmX, tmB, tmS, tmS1;
     const uint64_t xdims[4] = {64, (uint64_t)d.H, (uint64_t)d.L, (uint64_t)d.b};
     const uint64_t xstr[3] = {64 * 2, (uint64_t)(d.H * 64 * 2), (uint64_t)(d.L * d.H * 64 * 2)};
     const uint32_t xbox[4] = {64, 1, kStageTok, 1};
@@ -499,11 +500,14 @@ cudaError_t launch_impl(const void* x, const float* dt, const float* A, const vo
     if (e != cudaSuccess) return e;
     {
         // states as rows (head, p) of N fp32 per (batch, chunk); N = 128: boxes of
-        // 32 rows x 128 (plain), N = 64: boxes of 64 rows x 32 (128-byte swizzle)
+        // 32 rows x 128 (plain), N = 64: boxes of 128 (or 64) rows x 32 (128-byte swizzle)
         const uint64_t sdims[3] = {(uint64_t)N, (uint64_t)(d.H * 64), (uint64_t)(d.b * d.T)};
         const uint64_t sstr[2] = {(uint64_t)N * 4, (uint64_t)(d.H * 64 * N * 4)};
-        const uint32_t sbox128[3] = {128, 32, 1}, sbox64[3] = {32, 64, 1};
+        const uint32_t sbox128[3] = {128, 32, 1}, sbox64[3] = {32, 128, 1}, sbox64h[3] = {32, 64, 1};
         e = make_tmap_f32_plain(&tmS, states, 3, sdims, sstr, N == 128 ? sbox128 : sbox64, N != 128);
+        if (e != cudaSuccess) return e;
+        // N = 64, a head paired with a phantom: its 64 rows alone
+        e = make_tmap_f32_plain(&tmS1, states, 3, sdims, sstr, N == 128 ? sbox128 : sbox64h, N != 128);
         if (e != cudaSuccess) return e;
     }
     const sm100::WaitCtx status = make_wait_ctx();
@@ -521,7 +525,8 @@ cudaError_t launch_impl(const void* x, const float* dt, const float* A, const vo
                              cudaFuncAttributeMaxDynamicSharedMemorySize, S::kAlloc);
     if (e != cudaSuccess) return e;
     chunk_state_tc_kernel<Q, N><<<(unsigned)grid, kThreads, S::kAlloc, s>>>(
-        tmX, tmB, tmS, dt, A, states, logdecay, d.L, (int)d.H, (int)d.G, d.T, items, ksplit, status);
+        tmX, tmB, tmS, tmS1, dt, A, states, logdecay, d.L, (int)d.H, (int)d.G, d.T, items, ksplit,
+        status);
     return cudaGetLastError();
 }
 

@@ -63,16 +63,33 @@ seq_logdecay_kernel(const float* __restrict__ dt, const float* __restrict__ A,
 }
 
 // ------------------------------------------------------------------ exchange combine
+// Thread per VEC consecutive state elements of one (batch, head): the fold
+// over the ranks before `rank`, one decay factor per rank.
+template <int VEC>
 __global__ void __launch_bounds__(256)
 combine_kernel(const float* __restrict__ F, const float* __restrict__ ld,
                const float* __restrict__ init, float* __restrict__ out, int rank, int64_t BH,
                int64_t PN) {
-    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t i = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * VEC;
     if (i >= BH * PN) return;
     const int64_t bh = i / PN;
-    float h = init ? init[i] : 0.f;
-    for (int q = 0; q < rank; ++q) h = fmaf(expf(ld[(int64_t)q * BH + bh]), h, F[(int64_t)q * BH * PN + i]);
-    out[i] = h;
+    float h[VEC];
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) h[e] = init ? init[i + e] : 0.f;
+    for (int q = 0; q < rank; ++q) {
+        const float a = expf(ld[(int64_t)q * BH + bh]);
+        const float* f = F + (int64_t)q * BH * PN + i;
+        if constexpr (VEC == 4) {
+            const float4 v = *reinterpret_cast<const float4*>(f);
+            h[0] = fmaf(a, h[0], v.x); h[1] = fmaf(a, h[1], v.y);
+            h[2] = fmaf(a, h[2], v.z); h[3] = fmaf(a, h[3], v.w);
+        } else {
+#pragma unroll
+            for (int e = 0; e < VEC; ++e) h[e] = fmaf(a, h[e], f[e]);
+        }
+    }
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) out[i + e] = h[e];
 }
 
 // ------------------------------------------------------------------ correction prep
@@ -236,8 +253,13 @@ cudaError_t launch_state_combine(const float* F, const float* ld, const float* i
                                  int rank, const Dims& d, cudaStream_t s) {
     const int64_t BH = d.b * d.H, PN = d.P * d.N;
     if (BH * PN == 0) return cudaSuccess;
-    combine_kernel<<<(unsigned)((BH * PN + 255) / 256), 256, 0, s>>>(F, ld, init, out, rank, BH,
-                                                                     PN);
+    if (PN % 4 == 0) {
+        const int64_t n = BH * PN / 4;
+        combine_kernel<4><<<(unsigned)((n + 255) / 256), 256, 0, s>>>(F, ld, init, out, rank, BH, PN);
+    } else {
+        combine_kernel<1><<<(unsigned)((BH * PN + 255) / 256), 256, 0, s>>>(F, ld, init, out, rank,
+                                                                            BH, PN);
+    }
     return cudaGetLastError();
 }
 

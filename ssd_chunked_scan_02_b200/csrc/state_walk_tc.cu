@@ -24,12 +24,10 @@
 // P = 64), so a TMEM lane is a state column and a warp's prev/final stores are
 // contiguous along n; with N = 64 it forms S (M = two heads x P rows, N = 64),
 // a lane is a (head, p) row.  x and B come by TMA in 64-token sub-steps
-// through a ring of three (N = 128) or four (N = 64) entries, each fetched
-// into L2 six entries ahead of its load; x rows are scaled in place by the
-// decay weights w_j = exp(cs_last - cs_j) dt_j before the MMA reads them.
-// With N = 64 there are two accumulators, so a chunk's MMAs never wait for
-// the previous chunk's epilogue.  Sized for two CTAs per SM (about 105 KB of
-// shared memory and 256 TMEM columns each).
+// through a three-entry ring; x rows are scaled in place by the decay
+// weights w_j = exp(cs_last - cs_j) dt_j before the MMA reads them.  Sized
+// for two CTAs per SM (about 105 KB of shared memory and 256 or 128 TMEM
+// columns each).
 //
 // Roles (320 threads): warps 0-3 dt prefix sums (warp = (head, half of the
 // chunk)) and x scaling (warp w scales rows 32 w .. 32 w + 31 of each ring
@@ -52,15 +50,14 @@ using namespace sm100;
 
 constexpr int kThreads = 320;
 constexpr int kSub = 64;                 // tokens per ring entry
-constexpr int kPrefetch = 6;             // ring entries fetched into L2 ahead of their load
 
 template <int Q, int N>
 struct WalkSmem {
-    // ring entries: three of 32 KB (N = 128) or four of 24 KB (N = 64)
-    static constexpr int kStages = (N == 128) ? 3 : 4;
-    // chunk accumulators: one (N = 128: 2 x 128 columns with the state) or
-    // two (N = 64), so the next chunk's MMAs need not wait for the epilogue
-    static constexpr int kSSlots = (N == 128) ? 1 : 2;
+    // ring entries of 64 tokens (32 KB for N = 128, 24 KB for N = 64)
+    static constexpr int kStages = 3;
+    // one chunk accumulator: the next chunk's MMAs wait only until the
+    // epilogue has read it (two measured no faster for N = 64)
+    static constexpr int kSSlots = 1;
     static constexpr int kXPart = 2 * kSub * 128;          // two heads x 64 rows x 128 B
     static constexpr int kBPart = (N / 64) * kSub * 128;   // N/64 blocks x 64 rows x 128 B
     static constexpr int kEntry = kXPart + kBPart;
@@ -77,7 +74,7 @@ struct WalkSmem {
     static constexpr uint32_t kCols = (N == 128) ? 128 : 64;   // columns of one tile
     static constexpr uint32_t kColH = 0;
     static constexpr uint32_t kColS = kCols;
-    static constexpr uint32_t kTmemCols = 256;                 // 2 x 128, or 64 + 2 x 64
+    static constexpr uint32_t kTmemCols = 2 * kCols;
 };
 
 enum {
@@ -155,15 +152,6 @@ state_walk_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
                 if (u >= 1) ok = mbar_wait(&bars[BAR_EMPTY + e], (uint32_t)((u - 1) & 1), status);
                 if (!ok) break;
                 const int row = (int)((si / kNSub) * Q + (si % kNSub) * kSub);
-                // fetch a later entry's tiles into L2, so that its load, issued
-                // once a ring slot frees, does not wait on DRAM
-                if (si + kPrefetch < nsteps) {
-                    const int64_t sp = si + kPrefetch;
-                    const int prow = (int)((sp / kNSub) * Q + (sp % kNSub) * kSub);
-                    tma_prefetch_4d(&tmX, 0, h0, prow, (int)b);
-                    if (has1) tma_prefetch_4d(&tmX, 0, h0 + 1, prow, (int)b);
-                    for (int nb = 0; nb < N / 64; ++nb) tma_prefetch_4d(&tmB, nb * 64, g, prow, (int)b);
-                }
                 uint8_t* ent = ring + e * S::kEntry;
                 mbar_expect_tx(&bars[BAR_FULL + e], S::kEntry);
                 tma_load_4d(ent, &tmX, &bars[BAR_FULL + e], 0, h0, row, (int)b);
