@@ -452,7 +452,11 @@ def measure_backward(w, dev, stream, flush, reps, world, rank, peak_gbs):
     ms = max_over_ranks(sum(st.elapsed_time(en) for st, en in evs), world) / reps
     nbytes = bwd_bytes(w)
     gbs = nbytes / (ms * 1e-3) / 1e9
-    out = {"workload": w.name, "kernel": "exact fp32 SIMT, one CTA per block of state rows of a (batch, head)",
+    tc = ssd.ssd_chunk_scan_bwd_uses_tensor_cores(dims, inp["x"].dtype) == 1
+    kind = ("tcgen05 block decomposition in 128-token chunks (entering states, reverse pass "
+            "over the chunks for dL/dh, then dx/ddt and dB/dC kernels)" if tc else
+            "exact fp32 SIMT, one CTA per block of state rows of a (batch, head)")
+    out = {"workload": w.name, "kernel": kind, "tensor_cores": tc,
            "ms_per_step": ms, "tokens_per_s": world * w.tokens / (ms * 1e-3),
            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak_gbs, "unit": "GB/s",
                         "frac": gbs / peak_gbs, "alg_bytes_per_launch": nbytes}}

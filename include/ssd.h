@@ -203,27 +203,41 @@ SSD_API ssd_status_t ssd_chunk_scan_fwd_noalloc(const void* x, const float* dt, 
                                                 void* stream);
 
 /*
- * Gradients of ssd_chunk_scan_fwd (a first version: exact fp32 arithmetic on
- * the CUDA cores, one CTA per block of state rows of a (batch, head) walking
- * the sequence; slow next to the forward).  "Transformers are SSMs" (CiteArk), AI research summary:
- * training is what the layer is for; the gradients are the chain rule on
- * the recurrence h_t = exp(dt_t A_h) h_{t-1} + dt_t x_t B_t^T, y_t = h_t C_t
- * + D_h x_t, taken in reverse token order.
+ * Gradients of ssd_chunk_scan_fwd.  "Transformers are SSMs" (CiteArk), AI
+ * research summary: training is what the layer is for; the gradients are the
+ * chain rule on the recurrence h_t = exp(dt_t A_h) h_{t-1} + dt_t x_t B_t^T,
+ * y_t = h_t C_t + D_h x_t.  Two implementations, chosen from the sizes and
+ * dtype (ssd_chunk_scan_bwd_uses_tensor_cores tells which):
+ *   - SSD_BF16 with headdim 64..256 (a multiple of 64) and dstate 64 or 128:
+ *     the block decomposition in 128-token chunks on the tcgen05 tensor cores
+ *     (the forward's entering states recomputed, a reverse pass over the
+ *     chunks for dL/dh, then per chunk the masked products C B^T o E and
+ *     dy x^T o E and the state terms), bf16 operands with fp32 accumulation;
+ *     the decay gradients come from fp32 products.  Accuracy: the bf16
+ *     bound, 5e-3 of each gradient's largest element.
+ *   - everything else (all of SSD_F32): exact fp32 on the CUDA cores, one CTA
+ *     per block of state rows of a (batch, head) walking the sequence in
+ *     reverse token order (slow next to the forward).
  * Inputs: the forward's inputs (x, B, C in dtype; dt, A, D, init_states
  * fp32; init_states NULL = zero), dy (b,L,H,P) in dtype = dL/dy, and
  * dfinal_states (b,H,P,N) fp32 = dL/dfinal_states or NULL (zero).
  * Outputs, all fp32 and fully written: dx (b,L,H,P), ddt (b,L,H), dA (H),
  * dB (b,L,G,N), dC (b,L,G,N) (summed over the heads of each group), dD (H),
- * dinit_states (b,H,P,N) = dL/dinit_states (NULL = not wanted).  dA, dD, dB
- * and dC are zeroed, then accumulated with atomics, so their rounding (not
- * their value) may differ between runs.  workspace: >= the size reported by
- * ssd_chunk_scan_bwd_workspace_size (fp32 state checkpoints every 64 tokens
- * and one 64-token segment of states, per (batch, head) and block of state
- * rows); NULL only when that
+ * dinit_states (b,H,P,N) = dL/dinit_states (NULL = not wanted).  dA and dD
+ * (and on the CUDA-core path dB and dC) are zeroed, then accumulated with
+ * atomics, so their rounding (not their value) may differ between runs.
+ * workspace: >= the size reported by ssd_chunk_scan_bwd_workspace_size
+ * (tensor cores: the entering states and dL/dh per 128-token chunk in bf16
+ * plus one fp32 copy, b*ceil(L/128)*H*P*N*8 bytes and change; CUDA cores:
+ * fp32 state checkpoints every 64 tokens and one 64-token segment of
+ * states, per (batch, head) and block of state rows); NULL only when that
  * size is 0.  Inputs and outputs must not alias.
  */
 SSD_API ssd_status_t ssd_chunk_scan_bwd_workspace_size(const ssd_dims_t* dims, ssd_dtype_t dtype,
                                                        size_t* bytes);
+/* Which implementation ssd_chunk_scan_bwd uses for these sizes: 1 = tcgen05
+ * tensor cores, 0 = exact fp32 on the CUDA cores, -1 = rejected. */
+SSD_API int ssd_chunk_scan_bwd_uses_tensor_cores(const ssd_dims_t* dims, ssd_dtype_t dtype);
 SSD_API ssd_status_t ssd_chunk_scan_bwd(const void* x, const float* dt, const float* A,
                                         const void* B, const void* C, const float* D,
                                         const float* init_states, const void* dy,

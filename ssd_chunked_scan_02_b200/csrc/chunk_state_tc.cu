@@ -5,6 +5,11 @@
 //   w_j   = exp(cs_last - cs_j) dt_j        (decay to the chunk's end, times dt)
 //   S[p, n] = sum_j (w_j x_j[p]) B_j[n]    (P x N chunk state, zero start)
 //
+// The backward's reverse pass uses the same contraction with w_j = exp(cs_j)
+// (the decay from the chunk's start), dy in x's place and C in B's:
+// sum_j exp(cs_j) dy_j C_j^T is what a chunk adds to dL/dh of the state
+// entering it.
+//
 // "Transformers are SSMs" (CiteArk), AI research summary: the state a chunk
 // hands on is one dense contraction over the chunk's tokens (B^T (w * X)),
 // which is what the tensor cores are for.
@@ -122,7 +127,7 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tmX,
                       const __grid_constant__ CUtensorMap tmS1, const float* __restrict__ dt,
                       const float* __restrict__ A, float* __restrict__ states,
                       float* __restrict__ logdecay, int64_t L, int H, int G, int64_t T,
-                      int64_t items, int ksplit, WaitCtx status) {
+                      int64_t items, int ksplit, int rev, WaitCtx status) {
     using S = StateSmem<Q, N>;
     constexpr bool kTrans = (N == 128);
     constexpr int kSt = S::kStages;
@@ -322,7 +327,8 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tmX,
             }
             float* wk = s_w + (buf * 2 + hk) * Q + sg * kSegTok + lane * kPer;
 #pragma unroll
-            for (int k = 0; k < kPer; ++k) wk[k] = expf(last - (v[k] + off)) * dreg[k];
+            for (int k = 0; k < kPer; ++k)
+                wk[k] = rev ? expf(v[k] + off) : expf(last - (v[k] + off)) * dreg[k];
             // one log-decay per real head: the first of its virtual heads writes it
             if (sg == 0 && lane == 0 && real && hv % ksplit == 0)
                 logdecay[(w.b * T + w.c) * Hr + hv / ksplit] = last;
@@ -484,7 +490,7 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tmX,
 
 template <int Q, int N>
 cudaError_t launch_impl(const void* x, const float* dt, const float* A, const void* B,
-                        float* states, float* logdecay, const Dims& d, int ksplit,
+                        float* states, float* logdecay, const Dims& d, int ksplit, bool rev,
                         cudaStream_t s) {
     using S = StateSmem<Q, N>;
     CUtensorMap tmX, tmB, tmS, tmS1;
@@ -526,20 +532,21 @@ cudaError_t launch_impl(const void* x, const float* dt, const float* A, const vo
     if (e != cudaSuccess) return e;
     chunk_state_tc_kernel<Q, N><<<(unsigned)grid, kThreads, S::kAlloc, s>>>(
         tmX, tmB, tmS, tmS1, dt, A, states, logdecay, d.L, (int)d.H, (int)d.G, d.T, items, ksplit,
-        status);
+        rev ? 1 : 0, status);
     return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_chunk_state_tc(const void* x, const float* dt, const float* A, const void* B,
-                                  float* states, float* logdecay, const Dims& d, cudaStream_t s) {
+                                  float* states, float* logdecay, const Dims& d, cudaStream_t s,
+                                  bool rev) {
     int k = 1;
     const Dims v = virtual_heads(d, &k);
-    if (v.Q == 256 && v.N == 128) return launch_impl<256, 128>(x, dt, A, B, states, logdecay, v, k, s);
-    if (v.Q == 256 && v.N == 64) return launch_impl<256, 64>(x, dt, A, B, states, logdecay, v, k, s);
-    if (v.Q == 128 && v.N == 128) return launch_impl<128, 128>(x, dt, A, B, states, logdecay, v, k, s);
-    if (v.Q == 128 && v.N == 64) return launch_impl<128, 64>(x, dt, A, B, states, logdecay, v, k, s);
+    if (v.Q == 256 && v.N == 128) return launch_impl<256, 128>(x, dt, A, B, states, logdecay, v, k, rev, s);
+    if (v.Q == 256 && v.N == 64) return launch_impl<256, 64>(x, dt, A, B, states, logdecay, v, k, rev, s);
+    if (v.Q == 128 && v.N == 128) return launch_impl<128, 128>(x, dt, A, B, states, logdecay, v, k, rev, s);
+    if (v.Q == 128 && v.N == 64) return launch_impl<128, 64>(x, dt, A, B, states, logdecay, v, k, rev, s);
     return cudaErrorNotSupported;
 }
 

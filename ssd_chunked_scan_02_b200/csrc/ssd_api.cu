@@ -493,10 +493,25 @@ ssd_status_t ssd_chunk_scan_bwd_workspace_size(const ssd_dims_t* dims, ssd_dtype
     ssd_status_t st = check_dims(dims, 0, false, dtype, &d, &t);
     if (st != SSD_OK) return st;
     if (!bytes) return fail(SSD_ERR_INVALID_ARG, "bytes is NULL");
+    if (d.b == 0 || d.L == 0) {
+        *bytes = 0;
+        return SSD_OK;
+    }
+    if (ssd::backward_tc_supported(d, t)) {
+        *bytes = ssd::backward_tc_workspace_bytes(d);
+        return SSD_OK;
+    }
     if (!ssd::backward_supported(d))
         return fail(SSD_ERR_UNSUPPORTED, "dstate too large for the backward");
-    *bytes = (d.b == 0 || d.L == 0) ? 0 : ssd::backward_workspace_bytes(d);
+    *bytes = ssd::backward_workspace_bytes(d);
     return SSD_OK;
+}
+
+int ssd_chunk_scan_bwd_uses_tensor_cores(const ssd_dims_t* dims, ssd_dtype_t dtype) {
+    ssd::Dims d{}; ssd::Elt t = ssd::Elt::BF16;
+    if (check_dims(dims, 0, false, dtype, &d, &t) != SSD_OK) return -1;
+    if (ssd::backward_tc_supported(d, t)) return 1;
+    return ssd::backward_supported(d) ? 0 : -1;
 }
 
 ssd_status_t ssd_chunk_scan_bwd(const void* x, const float* dt, const float* A, const void* B,
@@ -509,19 +524,26 @@ ssd_status_t ssd_chunk_scan_bwd(const void* x, const float* dt, const float* A, 
     ssd::Dims d{}; ssd::Elt t = ssd::Elt::BF16;
     ssd_status_t st = check_dims(dims, 0, false, dtype, &d, &t);
     if (st != SSD_OK) return st;
-    if (!ssd::backward_supported(d))
+    const bool tc = d.b > 0 && d.L > 0 && ssd::backward_tc_supported(d, t);
+    if (!tc && !ssd::backward_supported(d))
         return fail(SSD_ERR_UNSUPPORTED, "dstate too large for the backward");
     REQUIRE_PTR(A); REQUIRE_PTR(D); REQUIRE_PTR(dA); REQUIRE_PTR(dD);
     OPTIONAL_PTR(init_states); OPTIONAL_PTR(dfinal_states); OPTIONAL_PTR(dinit_states);
     if (d.b > 0 && d.L > 0) {
         REQUIRE_PTR(x); REQUIRE_PTR(dt); REQUIRE_PTR(B); REQUIRE_PTR(C); REQUIRE_PTR(dy);
         REQUIRE_PTR(dx); REQUIRE_PTR(ddt); REQUIRE_PTR(dB); REQUIRE_PTR(dC);
-        const size_t need = ssd::backward_workspace_bytes(d);
+        const size_t need = tc ? ssd::backward_tc_workspace_bytes(d) : ssd::backward_workspace_bytes(d);
         if (workspace_bytes < need)
             return fail(SSD_ERR_INVALID_ARG, "workspace_bytes %zu < required %zu", workspace_bytes,
                         need);
         REQUIRE_PTR(workspace);
         REQUIRE_DEVICE(x);
+    }
+    if (tc) {
+        cudaError_t e = ssd::launch_backward_tc(x, dt, A, B, C, D, init_states, dy, dfinal_states,
+                                                dx, ddt, dA, dB, dC, dD, dinit_states, workspace,
+                                                d, static_cast<cudaStream_t>(stream));
+        return e == cudaSuccess ? SSD_OK : cuda_fail(e, "backward kernels (tcgen05)");
     }
     cudaError_t e = ssd::launch_backward(x, dt, A, B, C, D, init_states, dy, dfinal_states, dx,
                                          ddt, dA, dB, dC, dD, dinit_states,

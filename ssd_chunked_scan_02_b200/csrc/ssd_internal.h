@@ -22,10 +22,11 @@ cudaError_t launch_chunk_out_simt(const void* x, const float* dt, const float* A
                                   const void* C, const float* D, const void* prev, void* y,
                                   const Dims& d, Elt t, cudaStream_t s);
 
-// Inter-chunk recurrence (fp32), writes prev states in `t` and the final state.
+// Inter-chunk recurrence (fp32), writes prev states in `t` and the final state;
+// reverse: the chunks last to first (the backward's pass over dL/dh).
 cudaError_t launch_state_pass(const float* states, const float* logdecay, const float* init,
                               void* prev, float* final_states, const Dims& d, Elt t,
-                              cudaStream_t s);
+                              cudaStream_t s, bool reverse = false);
 
 // Decode step.
 cudaError_t launch_step(float* state, const void* x, const float* dt, const float* A,
@@ -44,5 +45,15 @@ cudaError_t launch_backward(const void* x, const float* dt, const float* A, cons
                             const float* dfinal, float* dx, float* ddt, float* dA, float* dB,
                             float* dC, float* dD, float* dinit, float* ws, const Dims& d, Elt t,
                             cudaStream_t s);
+
+// Backward on the tcgen05 tensor cores (bf16, the block decomposition in
+// 128-token chunks): the shapes it covers, its workspace, and the launch.
+bool backward_tc_supported(const Dims& d, Elt t);
+size_t backward_tc_workspace_bytes(const Dims& d);
+cudaError_t launch_backward_tc(const void* x, const float* dt, const float* A, const void* B,
+                               const void* C, const float* D, const float* init, const void* dy,
+                               const float* dfinal, float* dx, float* ddt, float* dA, float* dB,
+                               float* dC, float* dD, float* dinit, void* ws, const Dims& d,
+                               cudaStream_t s);
 
 }  // namespace ssd

@@ -2,7 +2,10 @@
 // block-decomposed SSD forward), in fp32:
 //     h_{-1} = init (or 0),   prev_c = h_{c-1},   h_c = exp(logdecay_c) h_{c-1} + S_c
 // where S_c is the chunk's own state (chunk started from zero) and logdecay_c
-// = sum_{t in chunk c} dt_t A_h.  "论文解读：Mamba: ...", 状态空间模型: the
+// = sum_{t in chunk c} dt_t A_h.  The backward runs the same recurrence with
+// the chunks in reverse order: g_{T-1} = dL/dfinal, out_c = g_c (dL/dh of the
+// state chunk c hands on), g_{c-1} = exp(logdecay_c) g_c + dS_c, dL/dinit =
+// g_{-1}.  "论文解读：Mamba: ...", 状态空间模型: the
 // linear-recurrence form, here taken one chunk per step instead of one token.
 //
 // Every (batch, head, p, n) state element is an independent chain; a thread
@@ -65,7 +68,8 @@ template <typename TP, int VEC>
 __global__ void __launch_bounds__(256)
 state_pass_kernel(const float* __restrict__ states, const float* __restrict__ logdecay,
                   const float* __restrict__ init, TP* __restrict__ prev,
-                  float* __restrict__ fin, int64_t b, int64_t T, int64_t H, int64_t PN) {
+                  float* __restrict__ fin, int64_t b, int64_t T, int64_t H, int64_t PN,
+                  int reverse) {
     const int64_t nvec = PN / VEC;
     const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (idx >= b * H * nvec) return;
@@ -80,10 +84,13 @@ state_pass_kernel(const float* __restrict__ states, const float* __restrict__ lo
 #pragma unroll
         for (int k = 0; k < VEC; ++k) hs[k] = 0.f;
     }
-    const int64_t cstride = H * PN;
-    const float* sp = states + (bb * T * H + h) * PN + off;
-    const float* lp = logdecay + bb * T * H + h;
-    TP* pp = prev + (bb * T * H + h) * PN + off;
+    // chunk order: 0 .. T-1, or T-1 .. 0 (reverse)
+    const int64_t c_first = reverse ? T - 1 : 0;
+    const int64_t cstride = reverse ? -H * PN : H * PN;
+    const int64_t lstride = reverse ? -H : H;
+    const float* sp = states + ((bb * T + c_first) * H + h) * PN + off;
+    const float* lp = logdecay + (bb * T + c_first) * H + h;
+    TP* pp = prev + ((bb * T + c_first) * H + h) * PN + off;
     // a ring of kAhead chunks' states and log-decays in registers: the loads
     // of chunk c + kAhead are issued when chunk c is consumed
     float sv[kAhead][VEC], lv[kAhead];
@@ -97,7 +104,7 @@ state_pass_kernel(const float* __restrict__ states, const float* __restrict__ lo
             lv[k] = *lq;
         }
         sq += cstride;
-        lq += H;
+        lq += lstride;
         ++cl;
     }
     TP* pq = pp;
@@ -115,7 +122,7 @@ state_pass_kernel(const float* __restrict__ states, const float* __restrict__ lo
                 lv[k] = *lq;
             }
             sq += cstride;
-            lq += H;
+            lq += lstride;
             ++cl;
         }
     }
@@ -134,27 +141,28 @@ __global__ void copy_or_zero_kernel(const float* __restrict__ src, float* __rest
 
 template <typename TP, int VEC>
 cudaError_t run(const float* states, const float* logdecay, const float* init, void* prev,
-                float* fin, const Dims& d, cudaStream_t s) {
+                float* fin, const Dims& d, bool reverse, cudaStream_t s) {
     const int64_t PN = d.P * d.N;
     const int64_t threads = d.b * d.H * (PN / VEC);
     if (threads == 0) return cudaSuccess;
     const int bs = 256;
     const int64_t blocks = (threads + bs - 1) / bs;
     state_pass_kernel<TP, VEC><<<(unsigned)blocks, bs, 0, s>>>(
-        states, logdecay, init, static_cast<TP*>(prev), fin, d.b, d.T, d.H, PN);
+        states, logdecay, init, static_cast<TP*>(prev), fin, d.b, d.T, d.H, PN, reverse ? 1 : 0);
     return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_state_pass(const float* states, const float* logdecay, const float* init,
-                              void* prev, float* fin, const Dims& d, Elt t, cudaStream_t s) {
+                              void* prev, float* fin, const Dims& d, Elt t, cudaStream_t s,
+                              bool reverse) {
     const bool v4 = ((d.P * d.N) % 4) == 0;
     if (t == Elt::F32)
-        return v4 ? run<float, 4>(states, logdecay, init, prev, fin, d, s)
-                  : run<float, 1>(states, logdecay, init, prev, fin, d, s);
-    return v4 ? run<__nv_bfloat16, 4>(states, logdecay, init, prev, fin, d, s)
-              : run<__nv_bfloat16, 1>(states, logdecay, init, prev, fin, d, s);
+        return v4 ? run<float, 4>(states, logdecay, init, prev, fin, d, reverse, s)
+                  : run<float, 1>(states, logdecay, init, prev, fin, d, reverse, s);
+    return v4 ? run<__nv_bfloat16, 4>(states, logdecay, init, prev, fin, d, reverse, s)
+              : run<__nv_bfloat16, 1>(states, logdecay, init, prev, fin, d, reverse, s);
 }
 
 cudaError_t launch_copy_or_zero(const float* init, float* fin, int64_t n, cudaStream_t s) {

@@ -40,8 +40,11 @@ struct HeadPairs {
 // True when the tensor-core kernels cover these sizes and dtype.
 bool tc_supported(const Dims& d, Elt t);
 
+// rev: the backward's per-chunk dL/dh contributions instead (weights
+// exp(cs_j); pass dy as x and C as B).
 cudaError_t launch_chunk_state_tc(const void* x, const float* dt, const float* A, const void* B,
-                                  float* states, float* logdecay, const Dims& d, cudaStream_t s);
+                                  float* states, float* logdecay, const Dims& d, cudaStream_t s,
+                                  bool rev = false);
 // Chunk states and the inter-chunk recurrence fused: one CTA per (batch,
 // head pair) walks the chunks; writes the entering states (bf16, layout
 // (b, T, H, P, N)) and the final state (fp32, nullable).

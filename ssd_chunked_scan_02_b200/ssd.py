@@ -25,6 +25,7 @@ SSD_F32, SSD_BF16 = 0, 1
 EXPORTED = ("ssd_status_string", "ssd_last_error_detail", "ssd_chunk_scan_fwd_workspace_size",
             "ssd_chunk_scan_fwd", "ssd_step", "ssd_chunk_state_fwd", "ssd_state_passing_fwd",
             "ssd_chunk_output_fwd", "ssd_chunk_scan_fwd_uses_tensor_cores",
+            "ssd_chunk_scan_bwd_uses_tensor_cores",
             "ssd_chunk_scan_fwd_noalloc", "ssd_poll_device_status", "ssd_state_walk_fwd",
             "ssd_debug_expire_wait", "ssd_chunk_scan_bwd_workspace_size", "ssd_chunk_scan_bwd",
             "ssd_chunk_scan_fwd_data_flow", "ssd_seq_logdecay", "ssd_state_exchange_combine",
@@ -69,6 +70,8 @@ def load(path: str = LIB_PATH):
                                                       ctypes.POINTER(ctypes.c_size_t)]
     lib.ssd_chunk_scan_fwd_uses_tensor_cores.restype = ctypes.c_int
     lib.ssd_chunk_scan_fwd_uses_tensor_cores.argtypes = [dims_p, ctypes.c_int, ctypes.c_int]
+    lib.ssd_chunk_scan_bwd_uses_tensor_cores.restype = ctypes.c_int
+    lib.ssd_chunk_scan_bwd_uses_tensor_cores.argtypes = [dims_p, ctypes.c_int]
     lib.ssd_chunk_scan_fwd_data_flow.restype = ctypes.c_int
     lib.ssd_chunk_scan_fwd_data_flow.argtypes = [dims_p, ctypes.c_int, ctypes.c_int]
     lib.ssd_chunk_scan_fwd.restype = ctypes.c_int
@@ -388,6 +391,12 @@ def ssd_chunk_output_fwd(x, dt, A, B, C, D, prev_states, chunk_size: int, y=None
                                          _stream(stream, dev))
     _check(st, "ssd_chunk_output_fwd")
     return y
+
+
+def ssd_chunk_scan_bwd_uses_tensor_cores(dims: ssd_dims_t, dtype: torch.dtype) -> int:
+    """1: the backward runs on the tcgen05 tensor cores; 0: exact fp32 on the
+    CUDA cores; -1: these sizes are rejected."""
+    return int(load().ssd_chunk_scan_bwd_uses_tensor_cores(ctypes.byref(dims), _dtype_code(dtype)))
 
 
 def ssd_chunk_scan_bwd_workspace_size(dims: ssd_dims_t, dtype: torch.dtype) -> int:

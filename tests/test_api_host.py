@@ -261,19 +261,49 @@ def _bwd_ws(dims, dt):
 
 
 @pytest.mark.parametrize("b,L,H,P,N,G,dt", [
-    (8, 2048, 24, 64, 128, 1, ssd.SSD_BF16),    # 8 rows of 128 a CTA, 32 segments
+    (8, 2048, 24, 64, 128, 1, ssd.SSD_F32),     # 8 rows of 128 a CTA, 32 segments
     (2, 150, 4, 16, 32, 2, ssd.SSD_F32),        # 16 rows (all of P) a CTA, 3 segments
     (1, 65, 6, 12, 20, 3, ssd.SSD_BF16),        # 12 rows (P < 1024 / N), 2 segments
-    (1, 70, 2, 128, 128, 2, ssd.SSD_BF16),      # 8 rows a CTA, 16 row blocks
+    (1, 70, 2, 128, 128, 2, ssd.SSD_F32),       # 8 rows a CTA, 16 row blocks
 ])
 def test_backward_workspace_size_formula(lib, b, L, H, P, N, G, dt):
-    # per (batch, head, block of R = min(P, 1024 / N) state rows): fp32
-    # checkpoints every 64 tokens plus one 64-token segment of states
-    st, n = _bwd_ws(ssd.make_dims(b, L, H, P, N, G), dt)
+    # CUDA-core path, per (batch, head, block of R = min(P, 1024 / N) state
+    # rows): fp32 checkpoints every 64 tokens plus one 64-token segment of states
+    dims = ssd.make_dims(b, L, H, P, N, G)
+    assert ssd.load().ssd_chunk_scan_bwd_uses_tensor_cores(ctypes.byref(dims), dt) == 0
+    st, n = _bwd_ws(dims, dt)
     assert st == ssd.SSD_OK
     R = min(P, 1024 // N)
     blocks = b * H * ((P + R - 1) // R)
     assert n == blocks * ((L + 63) // 64 + 64) * R * N * 4
+
+
+@pytest.mark.parametrize("b,L,H,P,N,G", [
+    (8, 2048, 24, 64, 128, 1), (1, 70, 2, 128, 128, 2), (2, 300, 4, 64, 64, 2), (1, 1, 3, 192, 128, 1),
+])
+def test_backward_tensor_core_workspace_size_formula(lib, b, L, H, P, N, G):
+    # tensor-core path (bf16): per 128-token chunk the entering states and
+    # dL/dh in bf16, one fp32 buffer of the same size and the chunks' log
+    # decays, each rounded up to 256 bytes
+    dims = ssd.make_dims(b, L, H, P, N, G)
+    assert ssd.load().ssd_chunk_scan_bwd_uses_tensor_cores(ctypes.byref(dims), ssd.SSD_BF16) == 1
+    st, n = _bwd_ws(dims, ssd.SSD_BF16)
+    assert st == ssd.SSD_OK
+    up = lambda v: (v + 255) // 256 * 256
+    T = (L + 127) // 128
+    e = b * T * H * P * N
+    assert n == up(e * 2) + up(e * 2) + up(e * 4) + up(b * T * H * 4)
+
+
+@pytest.mark.parametrize("P,N,dt,want", [
+    (64, 128, ssd.SSD_BF16, 1), (256, 64, ssd.SSD_BF16, 1), (64, 128, ssd.SSD_F32, 0),
+    (32, 128, ssd.SSD_BF16, 0), (64, 96, ssd.SSD_BF16, 0), (96, 64, ssd.SSD_BF16, 0),
+    (320, 64, ssd.SSD_BF16, -1),
+    (64, 512, ssd.SSD_BF16, -1),
+])
+def test_backward_path_query(lib, P, N, dt, want):
+    dims = ssd.make_dims(2, 100, 4, P, N, 2)
+    assert ssd.load().ssd_chunk_scan_bwd_uses_tensor_cores(ctypes.byref(dims), dt) == want
 
 
 def test_backward_workspace_zero_for_empty(lib):
