@@ -27,7 +27,10 @@
 //
 // Two kernels, one CTA per (batch, chunk, group) looping over the group's
 // heads, 192 threads: warps 0-3 = the epilogue (thread u = token row u = TMEM
-// lane u), warp 4 = TMA producer, warp 5 = MMA issuer (and TMEM owner).
+// lane u), warp 4 = TMA producer, warp 5 = MMA issuer (and TMEM owner).  A
+// head's inputs come into one of two slots while the previous head computes
+// (bwd_dx: x and dy in two slots, Gam and h in one, released once <Gam, h>
+// and the MMAs that read them are done; bwd_dbc: all four in two slots).
 //   bwd_dx:  G once; per head R, X1 = B Gam^T, Ys = C h^T, then M1 =
 //            bf16(G o E) built by the epilogue (with W's row and column
 //            sums), then dxi = M1^T dy; the epilogue writes dx, ddt and adds
@@ -55,29 +58,33 @@ constexpr int kQ = 128;          // tokens per chunk
 constexpr int kThreads = 192;
 constexpr float kLog2e = 1.4426950408889634f;
 
-template <int N>
+template <int N, int XY, int GH, bool kCols>
 struct BwdSmem {
     static constexpr int kNB = N / 64;                // 64-column blocks of dstate
     static constexpr int kTok = kQ * 128;             // 128 token rows x 128 B
     static constexpr int kSt = 64 * 128;              // 64 state rows (p) x 128 B
+    static constexpr int kGH = kNB * kSt;             // one state tile (Gam or h)
     static constexpr int kC = 0;                      // C tile (kNB blocks)
     static constexpr int kB = kC + kNB * kTok;        // B tile
-    static constexpr int kX = kB + kNB * kTok;        // x of the head
-    static constexpr int kDy = kX + kTok;             // dy of the head
-    static constexpr int kGam = kDy + kTok;           // dL/dh of the head (kNB blocks)
-    static constexpr int kHp = kGam + kNB * kSt;      // entering state of the head
-    static constexpr int kM = kHp + kNB * kSt;        // bf16 128 x 128 (two 64-column blocks)
+    static constexpr int kX = kB + kNB * kTok;        // x slots
+    static constexpr int kDy = kX + XY * kTok;        // dy slots
+    static constexpr int kGam = kDy + XY * kTok;      // dL/dh slots (kNB blocks each)
+    static constexpr int kHp = kGam + GH * kGH;       // entering-state slots
+    static constexpr int kM = kHp + GH * kGH;         // bf16 128 x 128 (two 64-column blocks)
     static constexpr int kCs = kM + 2 * kTok;         // float[128]: cs (log2 units)
     static constexpr int kDt = kCs + kQ * 4;          // float[128]: dt
     static constexpr int kCol = kDt + kQ * 4;         // float[4][128]: per-warp column sums of W
-    static constexpr int kRed = kCol + 4 * kQ * 4;    // float[32]: reductions
+    static constexpr int kRed = kCol + (kCols ? 4 * kQ * 4 : 0);   // float[32]: reductions
     static constexpr int kBar = kRed + 32 * 4;
     static constexpr int kTmem = kBar + 16 * 8;
-    static constexpr int kCnt = kTmem + 16;           // [0] loads issued, [1] MMA groups committed
+    static constexpr int kCnt = kTmem + 16;           // [0] heads loaded, [1] MMAs issued
     static constexpr int kFlags = kCnt + 16;
     static constexpr int kTotal = kFlags + 16;
     static constexpr int kAlloc = kTotal + 1024;      // slack to align the base to 1 KB
+    static_assert(kAlloc <= 232448, "shared memory per CTA");
 };
+template <int N> using DxSmem = BwdSmem<N, 2, 1, true>;
+template <int N> using DbcSmem = BwdSmem<N, 2, 2, false>;
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
     return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
@@ -129,26 +136,30 @@ __device__ __forceinline__ float chunk_prefix(float a2, int warp, int lane, floa
 
 enum {
     BAR_BC = 0,        // C and B tiles loaded
-    BAR_INFULL = 1,    // the head's x, dy, Gam, h loaded
-    BAR_INEMPTY = 2,   // the head's inputs consumed
-    BAR_G = 3,         // dx: G computed
-    BAR_ACC1 = 4,      // dx: R, X1, Ys computed / dbc: R computed
-    BAR_MREADY = 5,    // the epilogue's bf16 operand (and scaled rows) written
-    BAR_ACC2 = 6,      // dx: dxi computed
-    BAR_ACCEMPTY = 7,  // dx: the epilogue has read the head's accumulators
-    BAR_DONE = 8,      // dbc: all heads' MMAs completed
-    BAR_COUNT = 9
+    BAR_XYFULL = 1,    // 2: a slot's x and dy loaded
+    BAR_XYEMPTY = 3,   // 2: a slot's x and dy consumed
+    BAR_GHFULL = 5,    // 2: a slot's Gam and h loaded
+    BAR_GHEMPTY = 7,   // 2: a slot's Gam and h consumed
+    BAR_G = 9,         // dx: G computed
+    BAR_ACC1 = 10,     // dx: R, X1, Ys computed / dbc: R computed
+    BAR_MREADY = 11,   // the epilogue's bf16 operand (and scaled rows) written
+    BAR_ACC2 = 12,     // dx: dxi computed
+    BAR_ACCEMPTY = 13, // dx: the epilogue has read the head's accumulators
+    BAR_DONE = 14,     // dbc: all heads' MMAs completed
+    BAR_DRAIN = 15,    // every MMA issued has completed (error path)
+    BAR_COUNT = 16
 };
 
-// Producer: the C and B tiles of the chunk, then per head x, dy, Gam, h.
-template <int N>
+// Producer: the C and B tiles of the chunk, then per head x, dy (slot i % 2)
+// and Gam, h (slot i % GH), each as soon as its slot is free.
+template <class S>
 __device__ __forceinline__ void produce(uint8_t* smem, uint64_t* bars, const CUtensorMap* tmX,
                                         const CUtensorMap* tmDy, const CUtensorMap* tmB,
                                         const CUtensorMap* tmC, const CUtensorMap* tmGam,
                                         const CUtensorMap* tmHp, int64_t b, int64_t c, int64_t T,
-                                        int g, int H, int head0, int nh, volatile int* s_cnt,
-                                        volatile int* s_flag, const WaitCtx& status) {
-    using S = BwdSmem<N>;
+                                        int g, int H, int head0, int nh, int GH,
+                                        volatile int* s_cnt, volatile int* s_flag,
+                                        const WaitCtx& status) {
     const int t0 = (int)(c * kQ);
     mbar_expect_tx(&bars[BAR_BC], 2 * S::kNB * S::kTok);
     for (int nb = 0; nb < S::kNB; ++nb) {
@@ -157,23 +168,42 @@ __device__ __forceinline__ void produce(uint8_t* smem, uint64_t* bars, const CUt
     }
     bool ok = true;
     for (int i = 0; i < nh && ok; ++i) {
-        if (i >= 1) ok = mbar_wait(&bars[BAR_INEMPTY], (uint32_t)((i - 1) & 1), status);
-        if (!ok) break;
         const int hv = head0 + i;
-        mbar_expect_tx(&bars[BAR_INFULL], 2 * S::kTok + 2 * S::kNB * S::kSt);
-        tma_load_4d(smem + S::kX, tmX, &bars[BAR_INFULL], 0, hv, t0, (int)b);
-        tma_load_4d(smem + S::kDy, tmDy, &bars[BAR_INFULL], 0, hv, t0, (int)b);
+        const int sx = i & 1, sg = i % GH;
+        if (i >= 2) ok = mbar_wait(&bars[BAR_XYEMPTY + sx], (uint32_t)(((i >> 1) - 1) & 1), status);
+        if (!ok) break;
+        mbar_expect_tx(&bars[BAR_XYFULL + sx], 2 * S::kTok);
+        tma_load_4d(smem + S::kX + sx * S::kTok, tmX, &bars[BAR_XYFULL + sx], 0, hv, t0, (int)b);
+        tma_load_4d(smem + S::kDy + sx * S::kTok, tmDy, &bars[BAR_XYFULL + sx], 0, hv, t0, (int)b);
+        if (i >= GH) ok = mbar_wait(&bars[BAR_GHEMPTY + sg], (uint32_t)((i / GH - 1) & 1), status);
+        if (!ok) break;
         const int row = (int)(((b * T + c) * H + hv) * 64);
+        mbar_expect_tx(&bars[BAR_GHFULL + sg], 2 * S::kGH);
         for (int nb = 0; nb < S::kNB; ++nb) {
-            tma_load_2d(smem + S::kGam + nb * S::kSt, tmGam, &bars[BAR_INFULL], nb * 64, row);
-            tma_load_2d(smem + S::kHp + nb * S::kSt, tmHp, &bars[BAR_INFULL], nb * 64, row);
+            tma_load_2d(smem + S::kGam + sg * S::kGH + nb * S::kSt, tmGam, &bars[BAR_GHFULL + sg],
+                        nb * 64, row);
+            tma_load_2d(smem + S::kHp + sg * S::kGH + nb * S::kSt, tmHp, &bars[BAR_GHFULL + sg],
+                        nb * 64, row);
         }
         s_cnt[0] = i + 1;
     }
     if (!ok) s_flag[0] = 1;
 }
 
-template <int N>
+// Error path: before shared memory and TMEM go away, wait (bounded) for the
+// loads of the last heads issued and for every MMA issued (the MMA thread
+// commits BAR_DRAIN on its way out).
+template <int GH>
+__device__ __forceinline__ void drain(uint64_t* bars, volatile int* s_cnt, const WaitCtx& status) {
+    mbar_wait(&bars[BAR_BC], 0, status);
+    const int nl = s_cnt[0];
+    for (int i = (nl > 2 ? nl - 2 : 0); i < nl; ++i) {
+        mbar_wait(&bars[BAR_XYFULL + (i & 1)], (uint32_t)((i >> 1) & 1), status);
+        mbar_wait(&bars[BAR_GHFULL + i % GH], (uint32_t)((i / GH) & 1), status);
+    }
+    if (s_cnt[1] > 0) mbar_wait(&bars[BAR_DRAIN], 0, status);
+}
+
 __device__ __forceinline__ uint64_t desc(const uint8_t* p, uint32_t lbo) {
     return smem_desc_sw128(smem_u32(p), lbo, 1024);
 }
@@ -189,7 +219,7 @@ bwd_dx_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                  float* __restrict__ dA, float* __restrict__ dD, int64_t L, int H, int G,
                  int64_t T, int ksplit, WaitCtx status) {
     // H counts virtual heads (headdim 64); real head = virtual head / ksplit
-    using S = BwdSmem<N>;
+    using S = DxSmem<N>;
     constexpr uint32_t kColG = 0, kColR = 128, kColDx = 256, kColX1 = 320, kColYs = 384;
     constexpr uint32_t kTmemCols = 512;
     const int Hr = H / ksplit;
@@ -204,8 +234,6 @@ bwd_dx_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
     uint8_t* smem = align1024(smem_raw);
     uint8_t* sC = smem + S::kC;
     uint8_t* sB = smem + S::kB;
-    uint8_t* sX = smem + S::kX;
-    uint8_t* sDy = smem + S::kDy;
     uint8_t* sGam = smem + S::kGam;
     uint8_t* sHp = smem + S::kHp;
     uint8_t* sM = smem + S::kM;
@@ -237,8 +265,8 @@ bwd_dx_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
     if (warp == 4) {
         // ================================================== TMA producer
         if (lane == 0)
-            produce<N>(smem, bars, &tmX, &tmDy, &tmB, &tmC, &tmGam, &tmHp, b, c, T, g, H, head0,
-                       nh, s_cnt, s_flag, status);
+            produce<S>(smem, bars, &tmX, &tmDy, &tmB, &tmC, &tmGam, &tmHp, b, c, T, g, H, head0,
+                       nh, 1, s_cnt, s_flag, status);
     } else if (warp == 5) {
         // ================================================== MMA issuer
         if (lane == 0) {
@@ -250,33 +278,36 @@ bwd_dx_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
 #pragma unroll
                 for (int ks = 0; ks < N / 16; ++ks) {
                     const int ko = (ks >> 2) * S::kTok + (ks & 3) * 32;
-                    mma_ss(tmem + kColG, desc<N>(sC + ko, 16), desc<N>(sB + ko, 16), idG, ks > 0);
+                    mma_ss(tmem + kColG, desc(sC + ko, 16), desc(sB + ko, 16), idG, ks > 0);
                 }
                 mma_commit(&bars[BAR_G]);
+                s_cnt[1] = 1;
             }
             const uint32_t idR = idesc_bf16_f32(128, 128, false, false);   // dy, x K-major
             const uint32_t idS = idesc_bf16_f32(128, 64, false, false);    // B|C, Gam|h K-major
             const uint32_t idD = idesc_bf16_f32(128, 64, true, true);      // M1, dy MN-major
             for (int i = 0; i < nh && ok; ++i) {
-                ok = mbar_wait(&bars[BAR_INFULL], (uint32_t)(i & 1), status) &&
+                const int sx = i & 1;
+                ok = mbar_wait(&bars[BAR_XYFULL + sx], (uint32_t)((i >> 1) & 1), status) &&
+                     mbar_wait(&bars[BAR_GHFULL], (uint32_t)(i & 1), status) &&
                      (i == 0 || mbar_wait(&bars[BAR_ACCEMPTY], (uint32_t)((i - 1) & 1), status));
                 if (!ok) break;
                 tc_fence_after();
+                const uint8_t* sX = smem + S::kX + sx * S::kTok;
+                const uint8_t* sDy = smem + S::kDy + sx * S::kTok;
                 // R = dy x^T (M = t, N = s, K = p)
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
-                    mma_ss(tmem + kColR, desc<N>(sDy + ks * 32, 16), desc<N>(sX + ks * 32, 16), idR,
-                           ks > 0);
+                    mma_ss(tmem + kColR, desc(sDy + ks * 32, 16), desc(sX + ks * 32, 16), idR, ks > 0);
                 // X1 = B Gam^T (M = s, N = p, K = n); Ys = C h^T (M = t, N = p, K = n)
 #pragma unroll
                 for (int ks = 0; ks < N / 16; ++ks) {
                     const int ko = (ks >> 2) * S::kTok + (ks & 3) * 32;
                     const int so = (ks >> 2) * S::kSt + (ks & 3) * 32;
-                    mma_ss(tmem + kColX1, desc<N>(sB + ko, 16), desc<N>(sGam + so, 16), idS, ks > 0);
-                    mma_ss(tmem + kColYs, desc<N>(sC + ko, 16), desc<N>(sHp + so, 16), idS, ks > 0);
+                    mma_ss(tmem + kColX1, desc(sB + ko, 16), desc(sGam + so, 16), idS, ks > 0);
+                    mma_ss(tmem + kColYs, desc(sC + ko, 16), desc(sHp + so, 16), idS, ks > 0);
                 }
                 mma_commit(&bars[BAR_ACC1]);
-                s_cnt[1] = 2 * i + 1;
                 ok = mbar_wait(&bars[BAR_MREADY], (uint32_t)(i & 1), status);
                 if (!ok) break;
                 tc_fence_after();
@@ -284,11 +315,11 @@ bwd_dx_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                 // contiguous) is MN-major, its two 64-column blocks 16 KB apart
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks)
-                    mma_ss(tmem + kColDx, desc<N>(sM + ks * 2048, S::kTok),
-                           desc<N>(sDy + ks * 2048, 16), idD, ks > 0);
+                    mma_ss(tmem + kColDx, desc(sM + ks * 2048, S::kTok), desc(sDy + ks * 2048, 16),
+                           idD, ks > 0);
                 mma_commit(&bars[BAR_ACC2]);
-                s_cnt[1] = 2 * i + 2;
             }
+            if (s_cnt[1]) mma_commit(&bars[BAR_DRAIN]);
             if (!ok) s_flag[0] = 1;
         }
     } else {
@@ -296,12 +327,15 @@ bwd_dx_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
         const int u = tid;
         const uint32_t lb = (uint32_t)(warp * 32) << 16;
         const bool row_in = t0 + u < L;
+        const float* dt_row = dt + (b * L + t0 + u) * Hr;
         bool fail = false;
         float ddt_acc = 0.f, dA_acc = 0.f, dD_acc = 0.f;
+        float dt_next = (row_in && nh > 0) ? dt_row[head0 / ksplit] : 0.f;
         for (int i = 0; i < nh; ++i) {
             const int hv = head0 + i, hr = hv / ksplit;
             const float Ah = A[hr];
-            const float dtu = row_in ? dt[(b * L + t0 + u) * Hr + hr] : 0.f;
+            const float dtu = dt_next;
+            if (i + 1 < nh) dt_next = row_in ? dt_row[(hv + 1) / ksplit] : 0.f;
             float csL;
             const float csu = chunk_prefix(dtu * Ah * kLog2e, warp, lane, s_red, &csL);
             s_cs[u] = csu;
@@ -313,6 +347,23 @@ bwd_dx_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                 break;
             }
             tc_fence_after();
+            // ---- <Gam, h> over this thread's share (both tiles share one layout)
+            float zp = 0.f;
+            {
+                const uint4* g4 = reinterpret_cast<const uint4*>(sGam);
+                const uint4* h4 = reinterpret_cast<const uint4*>(sHp);
+#pragma unroll
+                for (int k = 0; k < S::kGH / 16 / 128; ++k) {
+                    const uint4 gv = g4[u + 128 * k], hv4 = h4[u + 128 * k];
+                    const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
+                    const uint32_t hw[4] = {hv4.x, hv4.y, hv4.z, hv4.w};
+#pragma unroll
+                    for (int e2 = 0; e2 < 4; ++e2) {
+                        const float2 a = bf2(gw[e2]), bb = bf2(hw[e2]);
+                        zp = fmaf(a.x, bb.x, fmaf(a.y, bb.y, zp));
+                    }
+                }
+            }
             // ---- M1 = bf16(G o E) (row u), W = G o E o dt_s o R: row sum, column sums
             float rowsum = 0.f;
 #pragma unroll 1
@@ -350,7 +401,10 @@ bwd_dx_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
             fence_proxy_async_smem();
             tc_fence_before();
             named_bar_sync(1, 128);
-            if (u == 0) mbar_arrive(&bars[BAR_MREADY]);
+            if (u == 0) {
+                mbar_arrive(&bars[BAR_MREADY]);
+                mbar_arrive(&bars[BAR_GHEMPTY]);   // Gam, h: read by their MMAs and above
+            }
             float dcs = rowsum - (s_col[u] + s_col[128 + u] + s_col[256 + u] + s_col[384 + u]);
 
             // ---- dx, and the row's dot products
@@ -363,8 +417,8 @@ bwd_dx_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
             const float el = fast_exp2(csL - csu), ei = fast_exp2(csu);
             const float Dh = Dv[hr];
             float dexpl = 0.f, sU = 0.f, dyys = 0.f, dxd = 0.f;
-            const uint4* xrow = reinterpret_cast<const uint4*>(sX + u * 128);
-            const uint4* dyrow = reinterpret_cast<const uint4*>(sDy + u * 128);
+            const uint4* xrow = reinterpret_cast<const uint4*>(smem + S::kX + (i & 1) * S::kTok + u * 128);
+            const uint4* dyrow = reinterpret_cast<const uint4*>(smem + S::kDy + (i & 1) * S::kTok + u * 128);
             float* dxo = dx + ((b * L + t0 + u) * H + hv) * 64;
 #pragma unroll 1
             for (int k = 0; k < 2; ++k) {
@@ -402,23 +456,6 @@ bwd_dx_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                 }
             }
             tc_fence_before();
-            // <Gam, h> over this thread's share (both tiles share one layout)
-            float zp = 0.f;
-            {
-                const uint4* g4 = reinterpret_cast<const uint4*>(sGam);
-                const uint4* h4 = reinterpret_cast<const uint4*>(sHp);
-#pragma unroll
-                for (int k = 0; k < S::kNB * S::kSt / 16 / 128; ++k) {
-                    const uint4 gv = g4[u + 128 * k], hv4 = h4[u + 128 * k];
-                    const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
-                    const uint32_t hw[4] = {hv4.x, hv4.y, hv4.z, hv4.w};
-#pragma unroll
-                    for (int e2 = 0; e2 < 4; ++e2) {
-                        const float2 a = bf2(gw[e2]), bb = bf2(hw[e2]);
-                        zp = fmaf(a.x, bb.x, fmaf(a.y, bb.y, zp));
-                    }
-                }
-            }
             const float Uu = dtu * el * sU;
             dcs += ei * dyys - Uu;
             {
@@ -428,10 +465,10 @@ bwd_dx_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                     s_red[8 + warp] = wz;
                 }
             }
-            named_bar_sync(1, 128);   // every read of the head's TMEM and inputs is done
+            named_bar_sync(1, 128);   // every read of the head's TMEM, x and dy is done
             if (u == 0) {
                 mbar_arrive(&bars[BAR_ACCEMPTY]);
-                mbar_arrive(&bars[BAR_INEMPTY]);
+                mbar_arrive(&bars[BAR_XYEMPTY + (i & 1)]);
             }
             if (u == kQ - 1) {
                 const float sumU = s_red[4] + s_red[5] + s_red[6] + s_red[7];
@@ -473,18 +510,7 @@ bwd_dx_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
 
     tc_fence_before();
     __syncthreads();
-    if (s_flag[0] && tid == 4 * 32) {
-        // A wait gave up somewhere: give the last loads and MMAs issued a
-        // last (bounded) chance to land before shared memory and TMEM go away.
-        mbar_wait(&bars[BAR_BC], 0, status);
-        const int nl = s_cnt[0], nm = s_cnt[1];
-        if (nl > 0) mbar_wait(&bars[BAR_INFULL], (uint32_t)((nl - 1) & 1), status);
-        if (nm > 0) {
-            const int hi = (nm - 1) >> 1;
-            mbar_wait(&bars[(nm & 1) ? BAR_ACC1 : BAR_ACC2], (uint32_t)(hi & 1), status);
-        }
-        mbar_wait(&bars[BAR_G], 0, status);
-    }
+    if (s_flag[0] && tid == 4 * 32) drain<1>(bars, s_cnt, status);
     __syncthreads();
     if (warp == 5) {
         tc_fence_after();
@@ -501,7 +527,7 @@ bwd_dbc_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                   const float* __restrict__ dt, const float* __restrict__ A,
                   float* __restrict__ dB, float* __restrict__ dC, int64_t L, int H, int G,
                   int64_t T, int ksplit, WaitCtx status) {
-    using S = BwdSmem<N>;
+    using S = DbcSmem<N>;
     constexpr uint32_t kColR = 0, kColDC = 128, kColDB = 128 + N;
     constexpr uint32_t kTmemCols = (N == 128) ? 512 : 256;
     const int Hr = H / ksplit;
@@ -516,10 +542,6 @@ bwd_dbc_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
     uint8_t* smem = align1024(smem_raw);
     uint8_t* sC = smem + S::kC;
     uint8_t* sB = smem + S::kB;
-    uint8_t* sX = smem + S::kX;
-    uint8_t* sDy = smem + S::kDy;
-    uint8_t* sGam = smem + S::kGam;
-    uint8_t* sHp = smem + S::kHp;
     uint8_t* sM = smem + S::kM;
     float* s_cs = reinterpret_cast<float*>(smem + S::kCs);
     float* s_dt = reinterpret_cast<float*>(smem + S::kDt);
@@ -547,8 +569,8 @@ bwd_dbc_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
 
     if (warp == 4) {
         if (lane == 0)
-            produce<N>(smem, bars, &tmX, &tmDy, &tmB, &tmC, &tmGam, &tmHp, b, c, T, g, H, head0,
-                       nh, s_cnt, s_flag, status);
+            produce<S>(smem, bars, &tmX, &tmDy, &tmB, &tmC, &tmGam, &tmHp, b, c, T, g, H, head0,
+                       nh, 2, s_cnt, s_flag, status);
     } else if (warp == 5) {
         if (lane == 0) {
             bool ok = mbar_wait(&bars[BAR_BC], 0, status);
@@ -557,51 +579,61 @@ bwd_dbc_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             const uint32_t idB = idesc_bf16_f32(128, N, true, true);       // M2^T MN-major; C MN-major
             const uint32_t idB2 = idesc_bf16_f32(128, N, false, true);     // x' K-major; Gam MN-major
             for (int i = 0; i < nh && ok; ++i) {
-                ok = mbar_wait(&bars[BAR_INFULL], (uint32_t)(i & 1), status);
+                const int sl = i & 1;
+                const uint32_t par = (uint32_t)((i >> 1) & 1);
+                ok = mbar_wait(&bars[BAR_XYFULL + sl], par, status) &&
+                     mbar_wait(&bars[BAR_GHFULL + sl], par, status);
                 if (!ok) break;
                 tc_fence_after();
-                // R = dy x^T
+                const uint8_t* sX = smem + S::kX + sl * S::kTok;
+                const uint8_t* sDy = smem + S::kDy + sl * S::kTok;
+                const uint8_t* sGam = smem + S::kGam + sl * S::kGH;
+                const uint8_t* sHp = smem + S::kHp + sl * S::kGH;
+                // R = dy x^T (the previous head's R was read before its MREADY)
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
-                    mma_ss(tmem + kColR, desc<N>(sDy + ks * 32, 16), desc<N>(sX + ks * 32, 16), idR,
-                           ks > 0);
+                    mma_ss(tmem + kColR, desc(sDy + ks * 32, 16), desc(sX + ks * 32, 16), idR, ks > 0);
                 mma_commit(&bars[BAR_ACC1]);
-                s_cnt[1] = 2 * i + 1;
+                s_cnt[1] = 1;
                 ok = mbar_wait(&bars[BAR_MREADY], (uint32_t)(i & 1), status);
                 if (!ok) break;
                 tc_fence_after();
                 // dC += M2 B (M = t, N = n, K = s); dC += dy' h (K = p)
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks)
-                    mma_ss(tmem + kColDC, desc<N>(sM + (ks >> 2) * S::kTok + (ks & 3) * 32, 16),
-                           desc<N>(sB + ks * 2048, S::kTok), idC, i > 0 || ks > 0);
+                    mma_ss(tmem + kColDC, desc(sM + (ks >> 2) * S::kTok + (ks & 3) * 32, 16),
+                           desc(sB + ks * 2048, S::kTok), idC, i > 0 || ks > 0);
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
-                    mma_ss(tmem + kColDC, desc<N>(sDy + ks * 32, 16), desc<N>(sHp + ks * 2048, S::kSt),
-                           idC, true);
+                    mma_ss(tmem + kColDC, desc(sDy + ks * 32, 16), desc(sHp + ks * 2048, S::kSt), idC,
+                           true);
                 // dB += M2^T C (M = s, N = n, K = t); dB += x' Gam (K = p)
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks)
-                    mma_ss(tmem + kColDB, desc<N>(sM + ks * 2048, S::kTok), desc<N>(sC + ks * 2048, S::kTok),
+                    mma_ss(tmem + kColDB, desc(sM + ks * 2048, S::kTok), desc(sC + ks * 2048, S::kTok),
                            idB, i > 0 || ks > 0);
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
-                    mma_ss(tmem + kColDB, desc<N>(sX + ks * 32, 16), desc<N>(sGam + ks * 2048, S::kSt),
-                           idB2, true);
-                mma_commit(&bars[BAR_INEMPTY]);
-                s_cnt[1] = 2 * i + 2;
+                    mma_ss(tmem + kColDB, desc(sX + ks * 32, 16), desc(sGam + ks * 2048, S::kSt), idB2,
+                           true);
+                mma_commit(&bars[BAR_XYEMPTY + sl]);
+                mma_commit(&bars[BAR_GHEMPTY + sl]);
             }
             if (ok) mma_commit(&bars[BAR_DONE]);
+            if (s_cnt[1]) mma_commit(&bars[BAR_DRAIN]);
             if (!ok) s_flag[0] = 1;
         }
     } else {
         const int u = tid;
         const uint32_t lb = (uint32_t)(warp * 32) << 16;
         const bool row_in = t0 + u < L;
+        const float* dt_row = dt + (b * L + t0 + u) * Hr;
         bool fail = false;
+        float dt_next = (row_in && nh > 0) ? dt_row[head0 / ksplit] : 0.f;
         for (int i = 0; i < nh; ++i) {
             const int hv = head0 + i, hr = hv / ksplit;
-            const float dtu = row_in ? dt[(b * L + t0 + u) * Hr + hr] : 0.f;
+            const float dtu = dt_next;
+            if (i + 1 < nh) dt_next = row_in ? dt_row[(hv + 1) / ksplit] : 0.f;
             float csL;
             const float csu = chunk_prefix(dtu * A[hr] * kLog2e, warp, lane, s_red, &csL);
             s_cs[u] = csu;
@@ -612,7 +644,8 @@ bwd_dbc_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                 break;
             }
             tc_fence_after();
-            // ---- M2 = bf16(R o E o dt_s) (row u)
+            // ---- M2 = bf16(R o E o dt_s) (row u); R(i) completing implies the
+            // previous head's MMAs, the last readers of M2, have completed
 #pragma unroll 1
             for (int j = 0; j < 4; ++j) {
                 uint4* mrow = reinterpret_cast<uint4*>(sM + (j >> 1) * S::kTok + u * 128);
@@ -641,8 +674,8 @@ bwd_dbc_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             // ---- x row *= dt_u el_u, dy row *= ei_u, in place (R has consumed them)
             {
                 const float sx = dtu * fast_exp2(csL - csu), sy = fast_exp2(csu);
-                uint4* xrow = reinterpret_cast<uint4*>(sX + u * 128);
-                uint4* yrow = reinterpret_cast<uint4*>(sDy + u * 128);
+                uint4* xrow = reinterpret_cast<uint4*>(smem + S::kX + (i & 1) * S::kTok + u * 128);
+                uint4* yrow = reinterpret_cast<uint4*>(smem + S::kDy + (i & 1) * S::kTok + u * 128);
 #pragma unroll
                 for (int q = 0; q < 8; ++q) {
                     uint4 xv = xrow[q], yv = yrow[q];
@@ -695,15 +728,7 @@ bwd_dbc_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
 
     tc_fence_before();
     __syncthreads();
-    if (s_flag[0] && tid == 4 * 32) {
-        mbar_wait(&bars[BAR_BC], 0, status);
-        const int nl = s_cnt[0], nm = s_cnt[1];
-        if (nl > 0) mbar_wait(&bars[BAR_INFULL], (uint32_t)((nl - 1) & 1), status);
-        if (nm > 0) {
-            const int hi = (nm - 1) >> 1;
-            mbar_wait(&bars[(nm & 1) ? BAR_ACC1 : BAR_INEMPTY], (uint32_t)(hi & 1), status);
-        }
-    }
+    if (s_flag[0] && tid == 4 * 32) drain<2>(bars, s_cnt, status);
     __syncthreads();
     if (warp == 5) {
         tc_fence_after();
@@ -716,7 +741,6 @@ cudaError_t launch_impl(const void* x, const void* dy, const float* dt, const fl
                         const void* B, const void* C, const float* D, const void* hp,
                         const void* gam, float* dx, float* ddt, float* dA, float* dB, float* dC,
                         float* dD, const Dims& d, int ksplit, cudaStream_t s) {
-    using S = BwdSmem<N>;
     CUtensorMap tmX, tmDy, tmB, tmC, tmGam, tmHp;
     const uint64_t xdims[4] = {64, (uint64_t)d.H, (uint64_t)d.L, (uint64_t)d.b};
     const uint64_t xstr[3] = {64 * 2, (uint64_t)(d.H * 64 * 2), (uint64_t)(d.L * d.H * 64 * 2)};
@@ -744,17 +768,17 @@ cudaError_t launch_impl(const void* x, const void* dy, const float* dt, const fl
     const int64_t grid = d.b * d.T * d.G;
     if (grid == 0) return cudaSuccess;
     e = cudaFuncSetAttribute(bwd_dx_tc_kernel<N>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             S::kAlloc);
+                             DxSmem<N>::kAlloc);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(bwd_dbc_tc_kernel<N>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             S::kAlloc);
+                             DbcSmem<N>::kAlloc);
     if (e != cudaSuccess) return e;
-    bwd_dx_tc_kernel<N><<<(unsigned)grid, kThreads, S::kAlloc, s>>>(
+    bwd_dx_tc_kernel<N><<<(unsigned)grid, kThreads, DxSmem<N>::kAlloc, s>>>(
         tmX, tmDy, tmB, tmC, tmGam, tmHp, dt, A, D, dx, ddt, dA, dD, d.L, (int)d.H, (int)d.G, d.T,
         ksplit, status);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    bwd_dbc_tc_kernel<N><<<(unsigned)grid, kThreads, S::kAlloc, s>>>(
+    bwd_dbc_tc_kernel<N><<<(unsigned)grid, kThreads, DbcSmem<N>::kAlloc, s>>>(
         tmX, tmDy, tmB, tmC, tmGam, tmHp, dt, A, dB, dC, d.L, (int)d.H, (int)d.G, d.T, ksplit,
         status);
     return cudaGetLastError();
