@@ -208,13 +208,15 @@ SSD_API ssd_status_t ssd_chunk_scan_fwd_noalloc(const void* x, const float* dt, 
  * chain rule on the recurrence h_t = exp(dt_t A_h) h_{t-1} + dt_t x_t B_t^T,
  * y_t = h_t C_t + D_h x_t.  Two implementations, chosen from the sizes and
  * dtype (ssd_chunk_scan_bwd_uses_tensor_cores tells which):
- *   - SSD_BF16 with headdim 64..256 (a multiple of 64) and dstate 64 or 128:
+ *   - SSD_BF16 with headdim 32 or 64..256 (a multiple of 64) and dstate 64
+ *     or 128:
  *     the block decomposition in 128-token chunks on the tcgen05 tensor cores
  *     (the forward's entering states recomputed, a reverse pass over the
  *     chunks for dL/dh, then per chunk the masked products C B^T o E and
  *     dy x^T o E and the state terms), bf16 operands with fp32 accumulation;
- *     the decay gradients come from fp32 products.  Accuracy: the bf16
- *     bound, 5e-3 of each gradient's largest element.
+ *     the decay gradients come from fp32 products, and the states enter
+ *     them as bf16 value + residue pairs (their sums cancel there).
+ *     Accuracy: the bf16 bound, 5e-3 of each gradient's largest element.
  *   - everything else (all of SSD_F32): exact fp32 on the CUDA cores, one CTA
  *     per block of state rows of a (batch, head) walking the sequence in
  *     reverse token order (slow next to the forward).
@@ -227,8 +229,9 @@ SSD_API ssd_status_t ssd_chunk_scan_fwd_noalloc(const void* x, const float* dt, 
  * (and on the CUDA-core path dB and dC) are zeroed, then accumulated with
  * atomics, so their rounding (not their value) may differ between runs.
  * workspace: >= the size reported by ssd_chunk_scan_bwd_workspace_size
- * (tensor cores: the entering states and dL/dh per 128-token chunk in bf16
- * plus one fp32 copy, b*ceil(L/128)*H*P*N*8 bytes and change; CUDA cores:
+ * (tensor cores: the entering states and dL/dh per 128-token chunk, each
+ * as a bf16 value and its bf16 rounding residue, plus one fp32 buffer,
+ * b*ceil(L/128)*H*max(P,64)*N*12 bytes and change; CUDA cores:
  * fp32 state checkpoints every 64 tokens and one 64-token segment of
  * states, per (batch, head) and block of state rows); NULL only when that
  * size is 0.  Inputs and outputs must not alias.
@@ -336,10 +339,15 @@ SSD_API ssd_status_t ssd_debug_expire_wait(unsigned int polls, void* stream);
 
 /* Which kernel family ssd_chunk_scan_fwd uses for these sizes:
  * 1 = tcgen05 tensor-core kernels, 0 = SIMT fp32 kernels, -1 = rejected.
- * The tensor cores take SSD_BF16 with headdim 64, 128, 192 or 256 (a head of
- * headdim 64 k runs as k heads of 64 sharing dt, A, D), dstate 64 or 128,
- * any number of heads per group and any chunk_size; everything else (and all
- * of SSD_F32, whose 1e-4 bound rules out bf16 operands) runs exact fp32. */
+ * The tensor cores take SSD_BF16 with headdim 32, 64, 128, 192 or 256 (a
+ * head of headdim 64 k runs as k heads of 64 sharing dt, A, D; one of 32 as
+ * a head of 64 whose other 32 columns are zero, its internal states padded
+ * to 64 rows), dstate 64 or 128, any number of heads per group and any
+ * chunk_size; everything else (and all of SSD_F32, whose 1e-4 bound rules
+ * out bf16 operands) runs exact fp32.  The step entry points
+ * (ssd_chunk_state_fwd, ssd_chunk_output_fwd, ssd_state_walk_fwd), whose
+ * state buffers are the caller's, take the tensor cores for headdim 64 k
+ * only. */
 SSD_API int ssd_chunk_scan_fwd_uses_tensor_cores(const ssd_dims_t* dims, int chunk_size,
                                          ssd_dtype_t dtype);
 

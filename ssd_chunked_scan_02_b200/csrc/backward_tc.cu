@@ -58,8 +58,12 @@ constexpr int kQ = 128;          // tokens per chunk
 constexpr int kThreads = 192;
 constexpr float kLog2e = 1.4426950408889634f;
 
-template <int N, int XY, int GH, bool kCols>
+// XY: slots for x and dy; GH: slots for Gam and h; kCols: the column-sum
+// scratch of W; kLo: Gam and h come with their rounding residues (hi + lo).
+template <int N, int XY, int GH, bool kCols, bool kLo>
 struct BwdSmem {
+    static constexpr int kXY = XY, kGHn = GH;
+    static constexpr bool kHasLo = kLo;
     static constexpr int kNB = N / 64;                // 64-column blocks of dstate
     static constexpr int kTok = kQ * 128;             // 128 token rows x 128 B
     static constexpr int kSt = 64 * 128;              // 64 state rows (p) x 128 B
@@ -68,9 +72,12 @@ struct BwdSmem {
     static constexpr int kB = kC + kNB * kTok;        // B tile
     static constexpr int kX = kB + kNB * kTok;        // x slots
     static constexpr int kDy = kX + XY * kTok;        // dy slots
-    static constexpr int kGam = kDy + XY * kTok;      // dL/dh slots (kNB blocks each)
-    static constexpr int kHp = kGam + GH * kGH;       // entering-state slots
-    static constexpr int kM = kHp + GH * kGH;         // bf16 128 x 128 (two 64-column blocks)
+    // a Gam/h slot: Gam, [Gam lo], h, [h lo]
+    static constexpr int kGHSlot = (kLo ? 4 : 2) * kGH;
+    static constexpr int kGHBase = kDy + XY * kTok;
+    static constexpr int kGamOff = 0, kGamLoOff = kGH;
+    static constexpr int kHpOff = (kLo ? 2 : 1) * kGH, kHpLoOff = 3 * kGH;
+    static constexpr int kM = kGHBase + GH * kGHSlot; // bf16 128 x 128 (two 64-column blocks)
     static constexpr int kCs = kM + 2 * kTok;         // float[128]: cs (log2 units)
     static constexpr int kDt = kCs + kQ * 4;          // float[128]: dt
     static constexpr int kCol = kDt + kQ * 4;         // float[4][128]: per-warp column sums of W
@@ -83,8 +90,8 @@ struct BwdSmem {
     static constexpr int kAlloc = kTotal + 1024;      // slack to align the base to 1 KB
     static_assert(kAlloc <= 232448, "shared memory per CTA");
 };
-template <int N> using DxSmem = BwdSmem<N, 2, 1, true>;
-template <int N> using DbcSmem = BwdSmem<N, 2, 2, false>;
+template <int N> using DxSmem = BwdSmem<N, 1, 1, true, true>;
+template <int N> using DbcSmem = BwdSmem<N, 2, 2, false, false>;
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
     return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
@@ -150,16 +157,17 @@ enum {
     BAR_COUNT = 16
 };
 
-// Producer: the C and B tiles of the chunk, then per head x, dy (slot i % 2)
-// and Gam, h (slot i % GH), each as soon as its slot is free.
+// Producer: the C and B tiles of the chunk, then per head x, dy (slot i % XY)
+// and Gam, h (and their residues; slot i % GH), each as soon as its slot is free.
 template <class S>
 __device__ __forceinline__ void produce(uint8_t* smem, uint64_t* bars, const CUtensorMap* tmX,
                                         const CUtensorMap* tmDy, const CUtensorMap* tmB,
                                         const CUtensorMap* tmC, const CUtensorMap* tmGam,
-                                        const CUtensorMap* tmHp, int64_t b, int64_t c, int64_t T,
-                                        int g, int H, int head0, int nh, int GH,
-                                        volatile int* s_cnt, volatile int* s_flag,
-                                        const WaitCtx& status) {
+                                        const CUtensorMap* tmHp, const CUtensorMap* tmGamLo,
+                                        const CUtensorMap* tmHpLo, int64_t b, int64_t c, int64_t T,
+                                        int g, int H, int head0, int nh, volatile int* s_cnt,
+                                        volatile int* s_flag, const WaitCtx& status) {
+    constexpr int XY = S::kXY, GH = S::kGHn;
     const int t0 = (int)(c * kQ);
     mbar_expect_tx(&bars[BAR_BC], 2 * S::kNB * S::kTok);
     for (int nb = 0; nb < S::kNB; ++nb) {
@@ -169,8 +177,8 @@ __device__ __forceinline__ void produce(uint8_t* smem, uint64_t* bars, const CUt
     bool ok = true;
     for (int i = 0; i < nh && ok; ++i) {
         const int hv = head0 + i;
-        const int sx = i & 1, sg = i % GH;
-        if (i >= 2) ok = mbar_wait(&bars[BAR_XYEMPTY + sx], (uint32_t)(((i >> 1) - 1) & 1), status);
+        const int sx = i % XY, sg = i % GH;
+        if (i >= XY) ok = mbar_wait(&bars[BAR_XYEMPTY + sx], (uint32_t)((i / XY - 1) & 1), status);
         if (!ok) break;
         mbar_expect_tx(&bars[BAR_XYFULL + sx], 2 * S::kTok);
         tma_load_4d(smem + S::kX + sx * S::kTok, tmX, &bars[BAR_XYFULL + sx], 0, hv, t0, (int)b);
@@ -178,12 +186,17 @@ __device__ __forceinline__ void produce(uint8_t* smem, uint64_t* bars, const CUt
         if (i >= GH) ok = mbar_wait(&bars[BAR_GHEMPTY + sg], (uint32_t)((i / GH - 1) & 1), status);
         if (!ok) break;
         const int row = (int)(((b * T + c) * H + hv) * 64);
-        mbar_expect_tx(&bars[BAR_GHFULL + sg], 2 * S::kGH);
+        uint8_t* slot = smem + S::kGHBase + sg * S::kGHSlot;
+        mbar_expect_tx(&bars[BAR_GHFULL + sg], S::kGHSlot);
         for (int nb = 0; nb < S::kNB; ++nb) {
-            tma_load_2d(smem + S::kGam + sg * S::kGH + nb * S::kSt, tmGam, &bars[BAR_GHFULL + sg],
-                        nb * 64, row);
-            tma_load_2d(smem + S::kHp + sg * S::kGH + nb * S::kSt, tmHp, &bars[BAR_GHFULL + sg],
-                        nb * 64, row);
+            tma_load_2d(slot + S::kGamOff + nb * S::kSt, tmGam, &bars[BAR_GHFULL + sg], nb * 64, row);
+            tma_load_2d(slot + S::kHpOff + nb * S::kSt, tmHp, &bars[BAR_GHFULL + sg], nb * 64, row);
+            if constexpr (S::kHasLo) {
+                tma_load_2d(slot + S::kGamLoOff + nb * S::kSt, tmGamLo, &bars[BAR_GHFULL + sg],
+                            nb * 64, row);
+                tma_load_2d(slot + S::kHpLoOff + nb * S::kSt, tmHpLo, &bars[BAR_GHFULL + sg],
+                            nb * 64, row);
+            }
         }
         s_cnt[0] = i + 1;
     }
@@ -193,12 +206,13 @@ __device__ __forceinline__ void produce(uint8_t* smem, uint64_t* bars, const CUt
 // Error path: before shared memory and TMEM go away, wait (bounded) for the
 // loads of the last heads issued and for every MMA issued (the MMA thread
 // commits BAR_DRAIN on its way out).
-template <int GH>
+template <class S>
 __device__ __forceinline__ void drain(uint64_t* bars, volatile int* s_cnt, const WaitCtx& status) {
+    constexpr int XY = S::kXY, GH = S::kGHn;
     mbar_wait(&bars[BAR_BC], 0, status);
     const int nl = s_cnt[0];
     for (int i = (nl > 2 ? nl - 2 : 0); i < nl; ++i) {
-        mbar_wait(&bars[BAR_XYFULL + (i & 1)], (uint32_t)((i >> 1) & 1), status);
+        mbar_wait(&bars[BAR_XYFULL + i % XY], (uint32_t)((i / XY) & 1), status);
         mbar_wait(&bars[BAR_GHFULL + i % GH], (uint32_t)((i / GH) & 1), status);
     }
     if (s_cnt[1] > 0) mbar_wait(&bars[BAR_DRAIN], 0, status);
@@ -214,10 +228,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 bwd_dx_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmDy,
                  const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmC,
                  const __grid_constant__ CUtensorMap tmGam, const __grid_constant__ CUtensorMap tmHp,
+                 const __grid_constant__ CUtensorMap tmGamLo, const __grid_constant__ CUtensorMap tmHpLo,
                  const float* __restrict__ dt, const float* __restrict__ A,
                  const float* __restrict__ Dv, float* __restrict__ dx, float* __restrict__ ddt,
                  float* __restrict__ dA, float* __restrict__ dD, int64_t L, int H, int G,
-                 int64_t T, int ksplit, WaitCtx status) {
+                 int64_t T, int ksplit, int pcols, WaitCtx status) {
     // H counts virtual heads (headdim 64); real head = virtual head / ksplit
     using S = DxSmem<N>;
     constexpr uint32_t kColG = 0, kColR = 128, kColDx = 256, kColX1 = 320, kColYs = 384;
@@ -234,8 +249,10 @@ bwd_dx_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
     uint8_t* smem = align1024(smem_raw);
     uint8_t* sC = smem + S::kC;
     uint8_t* sB = smem + S::kB;
-    uint8_t* sGam = smem + S::kGam;
-    uint8_t* sHp = smem + S::kHp;
+    uint8_t* sGam = smem + S::kGHBase + S::kGamOff;     // one Gam/h slot
+    uint8_t* sGamLo = smem + S::kGHBase + S::kGamLoOff;
+    uint8_t* sHp = smem + S::kGHBase + S::kHpOff;
+    uint8_t* sHpLo = smem + S::kGHBase + S::kHpLoOff;
     uint8_t* sM = smem + S::kM;
     float* s_cs = reinterpret_cast<float*>(smem + S::kCs);
     float* s_dt = reinterpret_cast<float*>(smem + S::kDt);
@@ -265,8 +282,8 @@ bwd_dx_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
     if (warp == 4) {
         // ================================================== TMA producer
         if (lane == 0)
-            produce<S>(smem, bars, &tmX, &tmDy, &tmB, &tmC, &tmGam, &tmHp, b, c, T, g, H, head0,
-                       nh, 1, s_cnt, s_flag, status);
+            produce<S>(smem, bars, &tmX, &tmDy, &tmB, &tmC, &tmGam, &tmHp, &tmGamLo, &tmHpLo, b, c,
+                       T, g, H, head0, nh, s_cnt, s_flag, status);
     } else if (warp == 5) {
         // ================================================== MMA issuer
         if (lane == 0) {
@@ -287,8 +304,8 @@ bwd_dx_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
             const uint32_t idS = idesc_bf16_f32(128, 64, false, false);    // B|C, Gam|h K-major
             const uint32_t idD = idesc_bf16_f32(128, 64, true, true);      // M1, dy MN-major
             for (int i = 0; i < nh && ok; ++i) {
-                const int sx = i & 1;
-                ok = mbar_wait(&bars[BAR_XYFULL + sx], (uint32_t)((i >> 1) & 1), status) &&
+                const int sx = i % S::kXY;
+                ok = mbar_wait(&bars[BAR_XYFULL + sx], (uint32_t)((i / S::kXY) & 1), status) &&
                      mbar_wait(&bars[BAR_GHFULL], (uint32_t)(i & 1), status) &&
                      (i == 0 || mbar_wait(&bars[BAR_ACCEMPTY], (uint32_t)((i - 1) & 1), status));
                 if (!ok) break;
@@ -299,13 +316,23 @@ bwd_dx_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
                     mma_ss(tmem + kColR, desc(sDy + ks * 32, 16), desc(sX + ks * 32, 16), idR, ks > 0);
-                // X1 = B Gam^T (M = s, N = p, K = n); Ys = C h^T (M = t, N = p, K = n)
+                // X1 = B Gam^T (M = s, N = p, K = n); Ys = C h^T (M = t, N = p, K = n);
+                // Gam and h as hi + lo (their bf16 rounding residue), so these
+                // two products, whose sums cancel in the decay gradient, carry
+                // Gam and h to near fp32
 #pragma unroll
                 for (int ks = 0; ks < N / 16; ++ks) {
                     const int ko = (ks >> 2) * S::kTok + (ks & 3) * 32;
                     const int so = (ks >> 2) * S::kSt + (ks & 3) * 32;
                     mma_ss(tmem + kColX1, desc(sB + ko, 16), desc(sGam + so, 16), idS, ks > 0);
                     mma_ss(tmem + kColYs, desc(sC + ko, 16), desc(sHp + so, 16), idS, ks > 0);
+                }
+#pragma unroll
+                for (int ks = 0; ks < N / 16; ++ks) {
+                    const int ko = (ks >> 2) * S::kTok + (ks & 3) * 32;
+                    const int so = (ks >> 2) * S::kSt + (ks & 3) * 32;
+                    mma_ss(tmem + kColX1, desc(sB + ko, 16), desc(sGamLo + so, 16), idS, true);
+                    mma_ss(tmem + kColYs, desc(sC + ko, 16), desc(sHpLo + so, 16), idS, true);
                 }
                 mma_commit(&bars[BAR_ACC1]);
                 ok = mbar_wait(&bars[BAR_MREADY], (uint32_t)(i & 1), status);
@@ -347,20 +374,27 @@ bwd_dx_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                 break;
             }
             tc_fence_after();
-            // ---- <Gam, h> over this thread's share (both tiles share one layout)
+            // ---- <Gam, h> over this thread's share (the tiles share one layout),
+            // each as hi + lo
             float zp = 0.f;
             {
                 const uint4* g4 = reinterpret_cast<const uint4*>(sGam);
+                const uint4* gl4 = reinterpret_cast<const uint4*>(sGamLo);
                 const uint4* h4 = reinterpret_cast<const uint4*>(sHp);
-#pragma unroll
+                const uint4* hl4 = reinterpret_cast<const uint4*>(sHpLo);
+#pragma unroll 2
                 for (int k = 0; k < S::kGH / 16 / 128; ++k) {
                     const uint4 gv = g4[u + 128 * k], hv4 = h4[u + 128 * k];
+                    const uint4 glv = gl4[u + 128 * k], hlv = hl4[u + 128 * k];
                     const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
                     const uint32_t hw[4] = {hv4.x, hv4.y, hv4.z, hv4.w};
+                    const uint32_t glw[4] = {glv.x, glv.y, glv.z, glv.w};
+                    const uint32_t hlw[4] = {hlv.x, hlv.y, hlv.z, hlv.w};
 #pragma unroll
                     for (int e2 = 0; e2 < 4; ++e2) {
-                        const float2 a = bf2(gw[e2]), bb = bf2(hw[e2]);
-                        zp = fmaf(a.x, bb.x, fmaf(a.y, bb.y, zp));
+                        const float2 a = bf2(gw[e2]), al = bf2(glw[e2]);
+                        const float2 bb = bf2(hw[e2]), bl = bf2(hlw[e2]);
+                        zp = fmaf(a.x + al.x, bb.x + bl.x, fmaf(a.y + al.y, bb.y + bl.y, zp));
                     }
                 }
             }
@@ -417,9 +451,11 @@ bwd_dx_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
             const float el = fast_exp2(csL - csu), ei = fast_exp2(csu);
             const float Dh = Dv[hr];
             float dexpl = 0.f, sU = 0.f, dyys = 0.f, dxd = 0.f;
-            const uint4* xrow = reinterpret_cast<const uint4*>(smem + S::kX + (i & 1) * S::kTok + u * 128);
-            const uint4* dyrow = reinterpret_cast<const uint4*>(smem + S::kDy + (i & 1) * S::kTok + u * 128);
-            float* dxo = dx + ((b * L + t0 + u) * H + hv) * 64;
+            const int sx = i % S::kXY;
+            const uint4* xrow = reinterpret_cast<const uint4*>(smem + S::kX + sx * S::kTok + u * 128);
+            const uint4* dyrow = reinterpret_cast<const uint4*>(smem + S::kDy + sx * S::kTok + u * 128);
+            // dx: (b, L, H, pcols) with pcols = 64, or 32 (a head of headdim 32)
+            float* dxo = dx + ((b * L + t0 + u) * H + hv) * pcols;
 #pragma unroll 1
             for (int k = 0; k < 2; ++k) {
                 uint32_t dr[32], xr1[32], yr[32];
@@ -448,7 +484,7 @@ bwd_dx_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                             dxd += ye[h2] * xe[h2];
                         }
                     }
-                    if (row_in) {
+                    if (row_in && 32 * k < pcols) {
                         float4* d4 = reinterpret_cast<float4*>(dxo + 32 * k + 8 * q);
                         d4[0] = make_float4(o[0], o[1], o[2], o[3]);
                         d4[1] = make_float4(o[4], o[5], o[6], o[7]);
@@ -468,7 +504,7 @@ bwd_dx_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
             named_bar_sync(1, 128);   // every read of the head's TMEM, x and dy is done
             if (u == 0) {
                 mbar_arrive(&bars[BAR_ACCEMPTY]);
-                mbar_arrive(&bars[BAR_XYEMPTY + (i & 1)]);
+                mbar_arrive(&bars[BAR_XYEMPTY + sx]);
             }
             if (u == kQ - 1) {
                 const float sumU = s_red[4] + s_red[5] + s_red[6] + s_red[7];
@@ -510,7 +546,7 @@ bwd_dx_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
 
     tc_fence_before();
     __syncthreads();
-    if (s_flag[0] && tid == 4 * 32) drain<1>(bars, s_cnt, status);
+    if (s_flag[0] && tid == 4 * 32) drain<S>(bars, s_cnt, status);
     __syncthreads();
     if (warp == 5) {
         tc_fence_after();
@@ -569,8 +605,8 @@ bwd_dbc_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
 
     if (warp == 4) {
         if (lane == 0)
-            produce<S>(smem, bars, &tmX, &tmDy, &tmB, &tmC, &tmGam, &tmHp, b, c, T, g, H, head0,
-                       nh, 2, s_cnt, s_flag, status);
+            produce<S>(smem, bars, &tmX, &tmDy, &tmB, &tmC, &tmGam, &tmHp, nullptr, nullptr, b, c,
+                       T, g, H, head0, nh, s_cnt, s_flag, status);
     } else if (warp == 5) {
         if (lane == 0) {
             bool ok = mbar_wait(&bars[BAR_BC], 0, status);
@@ -587,8 +623,8 @@ bwd_dbc_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                 tc_fence_after();
                 const uint8_t* sX = smem + S::kX + sl * S::kTok;
                 const uint8_t* sDy = smem + S::kDy + sl * S::kTok;
-                const uint8_t* sGam = smem + S::kGam + sl * S::kGH;
-                const uint8_t* sHp = smem + S::kHp + sl * S::kGH;
+                const uint8_t* sGam = smem + S::kGHBase + sl * S::kGHSlot + S::kGamOff;
+                const uint8_t* sHp = smem + S::kGHBase + sl * S::kGHSlot + S::kHpOff;
                 // R = dy x^T (the previous head's R was read before its MREADY)
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
@@ -728,7 +764,7 @@ bwd_dbc_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
 
     tc_fence_before();
     __syncthreads();
-    if (s_flag[0] && tid == 4 * 32) drain<2>(bars, s_cnt, status);
+    if (s_flag[0] && tid == 4 * 32) drain<S>(bars, s_cnt, status);
     __syncthreads();
     if (warp == 5) {
         tc_fence_after();
@@ -739,11 +775,13 @@ bwd_dbc_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
 template <int N>
 cudaError_t launch_impl(const void* x, const void* dy, const float* dt, const float* A,
                         const void* B, const void* C, const float* D, const void* hp,
-                        const void* gam, float* dx, float* ddt, float* dA, float* dB, float* dC,
-                        float* dD, const Dims& d, int ksplit, cudaStream_t s) {
-    CUtensorMap tmX, tmDy, tmB, tmC, tmGam, tmHp;
-    const uint64_t xdims[4] = {64, (uint64_t)d.H, (uint64_t)d.L, (uint64_t)d.b};
-    const uint64_t xstr[3] = {64 * 2, (uint64_t)(d.H * 64 * 2), (uint64_t)(d.L * d.H * 64 * 2)};
+                        const void* hp_lo, const void* gam, const void* gam_lo, float* dx,
+                        float* ddt, float* dA, float* dB, float* dC, float* dD, const Dims& d,
+                        int ksplit, int pc, cudaStream_t s) {
+    CUtensorMap tmX, tmDy, tmB, tmC, tmGam, tmHp, tmGamLo, tmHpLo;
+    // x and dy: pc columns a (virtual) head; a 64-column box reads zeros past them
+    const uint64_t xdims[4] = {(uint64_t)pc, (uint64_t)d.H, (uint64_t)d.L, (uint64_t)d.b};
+    const uint64_t xstr[3] = {(uint64_t)pc * 2, (uint64_t)(d.H * pc * 2), (uint64_t)(d.L * d.H * pc * 2)};
     const uint32_t box128[4] = {64, 1, kQ, 1};
     cudaError_t e = make_tmap_bf16(&tmX, x, 4, xdims, xstr, box128);
     if (e != cudaSuccess) return e;
@@ -755,13 +793,16 @@ cudaError_t launch_impl(const void* x, const void* dy, const float* dt, const fl
     if (e != cudaSuccess) return e;
     e = make_tmap_bf16(&tmC, C, 4, bdims, bstr, box128);
     if (e != cudaSuccess) return e;
+    // per-chunk states: rows (b, T, H, 64) of N bf16
     const uint64_t hdims[2] = {(uint64_t)N, (uint64_t)(d.b * d.T * d.H * 64)};
     const uint64_t hstr[1] = {(uint64_t)N * 2};
     const uint32_t hbox[2] = {64, 64};
-    e = make_tmap_bf16(&tmGam, gam, 2, hdims, hstr, hbox);
-    if (e != cudaSuccess) return e;
-    e = make_tmap_bf16(&tmHp, hp, 2, hdims, hstr, hbox);
-    if (e != cudaSuccess) return e;
+    const void* planes[4] = {gam, hp, gam_lo, hp_lo};
+    CUtensorMap* maps[4] = {&tmGam, &tmHp, &tmGamLo, &tmHpLo};
+    for (int k = 0; k < 4; ++k) {
+        e = make_tmap_bf16(maps[k], planes[k], 2, hdims, hstr, hbox);
+        if (e != cudaSuccess) return e;
+    }
     const sm100::WaitCtx status = make_wait_ctx();
     if (!status.word) return cudaErrorUnknown;
 
@@ -774,8 +815,8 @@ cudaError_t launch_impl(const void* x, const void* dy, const float* dt, const fl
                              DbcSmem<N>::kAlloc);
     if (e != cudaSuccess) return e;
     bwd_dx_tc_kernel<N><<<(unsigned)grid, kThreads, DxSmem<N>::kAlloc, s>>>(
-        tmX, tmDy, tmB, tmC, tmGam, tmHp, dt, A, D, dx, ddt, dA, dD, d.L, (int)d.H, (int)d.G, d.T,
-        ksplit, status);
+        tmX, tmDy, tmB, tmC, tmGam, tmHp, tmGamLo, tmHpLo, dt, A, D, dx, ddt, dA, dD, d.L,
+        (int)d.H, (int)d.G, d.T, ksplit, pc, status);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     bwd_dbc_tc_kernel<N><<<(unsigned)grid, kThreads, DbcSmem<N>::kAlloc, s>>>(
@@ -784,17 +825,21 @@ cudaError_t launch_impl(const void* x, const void* dy, const float* dt, const fl
     return cudaGetLastError();
 }
 
-// Workspace carve-up of the tensor-core backward (Q = 128 chunks).
+// Workspace carve-up of the tensor-core backward (Q = 128 chunks): the
+// entering states and dL/dh per chunk, each as bf16 hi and lo planes; one
+// fp32 buffer of chunk states (forward, then reverse); the log-decays.
 struct BwdLayout {
-    size_t prev = 0, gam = 0, states = 0, logdecay = 0, total = 0;
+    size_t prev = 0, prev_lo = 0, gam = 0, gam_lo = 0, states = 0, logdecay = 0, total = 0;
 };
 BwdLayout bwd_layout(const Dims& q) {
     auto up = [](size_t v) { return (v + 255) & ~size_t(255); };
-    const size_t elems = (size_t)(q.b * q.T * q.H * q.P * q.N);
+    const size_t elems = (size_t)(q.b * q.T * q.H * state_rows(q.P) * q.N);
     BwdLayout w;
     w.prev = 0;
-    w.gam = up(w.prev + elems * 2);
-    w.states = up(w.gam + elems * 2);
+    w.prev_lo = up(w.prev + elems * 2);
+    w.gam = up(w.prev_lo + elems * 2);
+    w.gam_lo = up(w.gam + elems * 2);
+    w.states = up(w.gam_lo + elems * 2);
     w.logdecay = up(w.states + elems * 4);
     w.total = up(w.logdecay + (size_t)(q.b * q.T * q.H) * 4);
     return w;
@@ -819,27 +864,27 @@ cudaError_t launch_backward_tc(const void* x, const float* dt, const float* A, c
                                float* dC, float* dD, float* dinit, void* ws, const Dims& d,
                                cudaStream_t s) {
     const Dims q = chunks128(d);
+    Dims qs = q;                          // the state buffers' rows a head
+    qs.P = state_rows(d.P);
     const BwdLayout w = bwd_layout(q);
     char* base = static_cast<char*>(ws);
     void* prev = base + w.prev;
+    void* prev_lo = base + w.prev_lo;
     void* gam = base + w.gam;
+    void* gam_lo = base + w.gam_lo;
     float* states = reinterpret_cast<float*>(base + w.states);
     float* logdecay = reinterpret_cast<float*>(base + w.logdecay);
-    // the states entering each chunk (the forward's, recomputed)
-    cudaError_t e;
-    if (walk_preferred(q)) {
-        e = launch_state_walk_tc(x, dt, A, B, init, prev, nullptr, q, s);
-        if (e != cudaSuccess) return e;
-    } else {
-        e = launch_chunk_state_tc(x, dt, A, B, states, logdecay, q, s);
-        if (e != cudaSuccess) return e;
-        e = launch_state_pass(states, logdecay, init, prev, nullptr, q, Elt::BF16, s);
-        if (e != cudaSuccess) return e;
-    }
-    // dL/dh of the state each chunk hands on, and dL/dinit
+    // the states entering each chunk (the forward's, recomputed), hi + lo
+    cudaError_t e = launch_chunk_state_tc(x, dt, A, B, states, logdecay, q, s);
+    if (e != cudaSuccess) return e;
+    e = launch_state_pass(states, logdecay, init, prev, nullptr, qs, Elt::BF16, s, false, d.P,
+                          prev_lo);
+    if (e != cudaSuccess) return e;
+    // dL/dh of the state each chunk hands on (hi + lo), and dL/dinit
     e = launch_chunk_state_tc(dy, dt, A, C, states, logdecay, q, s, true);
     if (e != cudaSuccess) return e;
-    e = launch_state_pass(states, logdecay, dfinal, gam, dinit, q, Elt::BF16, s, true);
+    e = launch_state_pass(states, logdecay, dfinal, gam, dinit, qs, Elt::BF16, s, true, d.P,
+                          gam_lo);
     if (e != cudaSuccess) return e;
     e = cudaMemsetAsync(dA, 0, sizeof(float) * (size_t)d.H, s);
     if (e != cudaSuccess) return e;
@@ -848,9 +893,11 @@ cudaError_t launch_backward_tc(const void* x, const float* dt, const float* A, c
     int k = 1;
     const Dims v = virtual_heads(q, &k);
     if (v.N == 128)
-        return launch_impl<128>(x, dy, dt, A, B, C, D, prev, gam, dx, ddt, dA, dB, dC, dD, v, k, s);
+        return launch_impl<128>(x, dy, dt, A, B, C, D, prev, prev_lo, gam, gam_lo, dx, ddt, dA, dB,
+                                dC, dD, v, k, head_cols(d), s);
     if (v.N == 64)
-        return launch_impl<64>(x, dy, dt, A, B, C, D, prev, gam, dx, ddt, dA, dB, dC, dD, v, k, s);
+        return launch_impl<64>(x, dy, dt, A, B, C, D, prev, prev_lo, gam, gam_lo, dx, ddt, dA, dB,
+                               dC, dD, v, k, head_cols(d), s);
     return cudaErrorNotSupported;
 }
 

@@ -669,11 +669,13 @@ int pick_heads_per_cta(int64_t H, int64_t G) {
 template <int Q, int N>
 cudaError_t launch_impl(const void* x, const float* dt, const float* A, const void* B,
                         const void* C, const float* D, const void* prev, void* y, const Dims& d, int ksplit,
-                        cudaStream_t s) {
+                        int pc, cudaStream_t s) {
     using S = OutSmem<Q, N>;
     CUtensorMap tmX, tmB, tmC, tmH, tmY;
-    const uint64_t xdims[4] = {64, (uint64_t)d.H, (uint64_t)d.L, (uint64_t)d.b};
-    const uint64_t xstr[3] = {64 * 2, (uint64_t)(d.H * 64 * 2), (uint64_t)(d.L * d.H * 64 * 2)};
+    // x and y: pc columns a (virtual) head; a 64-column box reads zeros past
+    // them and stores only up to them
+    const uint64_t xdims[4] = {(uint64_t)pc, (uint64_t)d.H, (uint64_t)d.L, (uint64_t)d.b};
+    const uint64_t xstr[3] = {(uint64_t)pc * 2, (uint64_t)(d.H * pc * 2), (uint64_t)(d.L * d.H * pc * 2)};
     const uint32_t box128[4] = {64, 1, 128, 1};
     cudaError_t e = make_tmap_bf16(&tmX, x, 4, xdims, xstr, box128);
     if (e != cudaSuccess) return e;
@@ -712,10 +714,10 @@ cudaError_t launch_chunk_out_tc(const void* x, const float* dt, const float* A, 
                                 const Dims& d, cudaStream_t s) {
     int k = 1;
     const Dims v = virtual_heads(d, &k);
-    if (v.Q == 256 && v.N == 128) return launch_impl<256, 128>(x, dt, A, B, C, D, prev, y, v, k, s);
-    if (v.Q == 256 && v.N == 64) return launch_impl<256, 64>(x, dt, A, B, C, D, prev, y, v, k, s);
-    if (v.Q == 128 && v.N == 128) return launch_impl<128, 128>(x, dt, A, B, C, D, prev, y, v, k, s);
-    if (v.Q == 128 && v.N == 64) return launch_impl<128, 64>(x, dt, A, B, C, D, prev, y, v, k, s);
+    if (v.Q == 256 && v.N == 128) return launch_impl<256, 128>(x, dt, A, B, C, D, prev, y, v, k, head_cols(d), s);
+    if (v.Q == 256 && v.N == 64) return launch_impl<256, 64>(x, dt, A, B, C, D, prev, y, v, k, head_cols(d), s);
+    if (v.Q == 128 && v.N == 128) return launch_impl<128, 128>(x, dt, A, B, C, D, prev, y, v, k, head_cols(d), s);
+    if (v.Q == 128 && v.N == 64) return launch_impl<128, 64>(x, dt, A, B, C, D, prev, y, v, k, head_cols(d), s);
     return cudaErrorNotSupported;
 }
 

@@ -491,11 +491,12 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tmX,
 template <int Q, int N>
 cudaError_t launch_impl(const void* x, const float* dt, const float* A, const void* B,
                         float* states, float* logdecay, const Dims& d, int ksplit, bool rev,
-                        cudaStream_t s) {
+                        int pc, cudaStream_t s) {
     using S = StateSmem<Q, N>;
     CUtensorMap tmX, tmB, tmS, tmS1;
-    const uint64_t xdims[4] = {64, (uint64_t)d.H, (uint64_t)d.L, (uint64_t)d.b};
-    const uint64_t xstr[3] = {64 * 2, (uint64_t)(d.H * 64 * 2), (uint64_t)(d.L * d.H * 64 * 2)};
+    // x: pc columns a (virtual) head; a 64-column box reads zeros past them
+    const uint64_t xdims[4] = {(uint64_t)pc, (uint64_t)d.H, (uint64_t)d.L, (uint64_t)d.b};
+    const uint64_t xstr[3] = {(uint64_t)pc * 2, (uint64_t)(d.H * pc * 2), (uint64_t)(d.L * d.H * pc * 2)};
     const uint32_t xbox[4] = {64, 1, kStageTok, 1};
     cudaError_t e = make_tmap_bf16(&tmX, x, 4, xdims, xstr, xbox);
     if (e != cudaSuccess) return e;
@@ -543,10 +544,10 @@ cudaError_t launch_chunk_state_tc(const void* x, const float* dt, const float* A
                                   bool rev) {
     int k = 1;
     const Dims v = virtual_heads(d, &k);
-    if (v.Q == 256 && v.N == 128) return launch_impl<256, 128>(x, dt, A, B, states, logdecay, v, k, rev, s);
-    if (v.Q == 256 && v.N == 64) return launch_impl<256, 64>(x, dt, A, B, states, logdecay, v, k, rev, s);
-    if (v.Q == 128 && v.N == 128) return launch_impl<128, 128>(x, dt, A, B, states, logdecay, v, k, rev, s);
-    if (v.Q == 128 && v.N == 64) return launch_impl<128, 64>(x, dt, A, B, states, logdecay, v, k, rev, s);
+    if (v.Q == 256 && v.N == 128) return launch_impl<256, 128>(x, dt, A, B, states, logdecay, v, k, rev, head_cols(d), s);
+    if (v.Q == 256 && v.N == 64) return launch_impl<256, 64>(x, dt, A, B, states, logdecay, v, k, rev, head_cols(d), s);
+    if (v.Q == 128 && v.N == 128) return launch_impl<128, 128>(x, dt, A, B, states, logdecay, v, k, rev, head_cols(d), s);
+    if (v.Q == 128 && v.N == 64) return launch_impl<128, 64>(x, dt, A, B, states, logdecay, v, k, rev, head_cols(d), s);
     return cudaErrorNotSupported;
 }
 

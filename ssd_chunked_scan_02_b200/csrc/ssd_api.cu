@@ -68,7 +68,10 @@ ssd_status_t check_dims(const ssd_dims_t* dims, int chunk, bool need_chunk, ssd_
     return SSD_OK;
 }
 
-bool tc_eligible(const ssd::Dims& d, ssd::Elt t) { return ssd::tc_supported(d, t); }
+// The fused forward's tensor-core kernels (headdim 32 included), and the
+// step entry points' (whose state buffers are the caller's: multiples of 64).
+bool fwd_tc(const ssd::Dims& d, ssd::Elt t) { return ssd::tc_supported(d, t); }
+bool tc_eligible(const ssd::Dims& d, ssd::Elt t) { return ssd::tc_supported(d, t) && d.P % 64 == 0; }
 
 // The block size the forward runs with.  The decomposition's result does not
 // depend on the block size (beyond rounding); the tensor-core kernels take
@@ -80,7 +83,7 @@ ssd::Dims forward_dims(const ssd::Dims& d, ssd::Elt t) {
     ssd::Dims q = d;
     q.Q = 128;
     q.T = (d.L + 127) / 128;
-    return tc_eligible(q, t) ? q : d;
+    return fwd_tc(q, t) ? q : d;
 }
 
 // The forward's data flow for these sizes (decided from the sizes alone, so
@@ -88,7 +91,7 @@ ssd::Dims forward_dims(const ssd::Dims& d, ssd::Elt t) {
 enum class Flow { Simt = 0, ThreeKernel = 1, Walk = 2 };
 
 Flow pick_flow(const ssd::Dims& d, ssd::Elt t) {
-    if (!tc_eligible(d, t)) return Flow::Simt;
+    if (!fwd_tc(d, t)) return Flow::Simt;
     return ssd::walk_preferred(d) ? Flow::Walk : Flow::ThreeKernel;
 }
 
@@ -100,10 +103,13 @@ struct WsLayout {
 };
 
 WsLayout ws_layout(const ssd::Dims& d, ssd::Elt t) {
-    const size_t nstate = (size_t)(d.b * d.T * d.H) * (size_t)(d.P * d.N);
+    // the tensor-core flows keep 64 state rows for a head of headdim 32
+    const Flow flow = pick_flow(d, t);
+    const int64_t rows = flow == Flow::Simt ? d.P : ssd::state_rows(d.P);
+    const size_t nstate = (size_t)(d.b * d.T * d.H) * (size_t)(rows * d.N);
     WsLayout w;
     w.states = 0;
-    if (pick_flow(d, t) == Flow::Walk) {
+    if (flow == Flow::Walk) {
         w.logdecay = 0;
         w.prev = 0;
     } else {
@@ -197,7 +203,7 @@ int ssd_chunk_scan_fwd_uses_tensor_cores(const ssd_dims_t* dims, int chunk_size,
                                          ssd_dtype_t dtype) {
     ssd::Dims d{}; ssd::Elt t = ssd::Elt::BF16;
     if (check_dims(dims, chunk_size, true, dtype, &d, &t) != SSD_OK) return -1;
-    return tc_eligible(forward_dims(d, t), t) ? 1 : 0;
+    return fwd_tc(forward_dims(d, t), t) ? 1 : 0;
 }
 
 int ssd_chunk_scan_fwd_data_flow(const ssd_dims_t* dims, int chunk_size, ssd_dtype_t dtype) {
@@ -255,7 +261,11 @@ ssd_status_t ssd_chunk_scan_fwd(const void* x, const float* dt, const float* A, 
     if (flow == Flow::ThreeKernel) {
         e = ssd::launch_chunk_state_tc(x, dt, A, B, states, logdecay, d, s);
         if (e != cudaSuccess) return cuda_fail(e, "chunk-state kernel (tcgen05)");
-        e = ssd::launch_state_pass(states, logdecay, init_states, prev, final_states, d, t, s);
+        // the state buffers have state_rows(P) rows a head; init and final P
+        ssd::Dims ds = d;
+        ds.P = ssd::state_rows(d.P);
+        e = ssd::launch_state_pass(states, logdecay, init_states, prev, final_states, ds, t, s,
+                                   false, d.P);
         if (e != cudaSuccess) return cuda_fail(e, "state-passing kernel");
         e = ssd::launch_chunk_out_tc(x, dt, A, B, C, D, prev, y, d, s);
         if (e != cudaSuccess) return cuda_fail(e, "chunk-output kernel (tcgen05)");

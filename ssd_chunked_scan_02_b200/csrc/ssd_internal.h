@@ -24,9 +24,14 @@ cudaError_t launch_chunk_out_simt(const void* x, const float* dt, const float* A
 
 // Inter-chunk recurrence (fp32), writes prev states in `t` and the final state;
 // reverse: the chunks last to first (the backward's pass over dL/dh).
+// p_ext (when non-zero and below d.P): init and final_states have p_ext rows
+// per head ((b, H, p_ext, N)), the state buffers d.P (rows p_ext.. zero).
+// prev_lo (bf16 only, nullable): also the rounding residue of each prev
+// element, bf16(h - bf16(h)).
 cudaError_t launch_state_pass(const float* states, const float* logdecay, const float* init,
                               void* prev, float* final_states, const Dims& d, Elt t,
-                              cudaStream_t s, bool reverse = false);
+                              cudaStream_t s, bool reverse = false, int64_t p_ext = 0,
+                              void* prev_lo = nullptr);
 
 // Decode step.
 cudaError_t launch_step(float* state, const void* x, const float* dt, const float* A,

@@ -25,6 +25,10 @@ constexpr int kAhead = 16;   // chunks whose loads are in flight per thread
 
 template <typename TP, int VEC>
 struct Store;
+template <typename TP, int VEC>
+struct StoreLo {
+    static __device__ __forceinline__ void run(TP*, const float*) {}
+};
 template <int VEC>
 struct Store<float, VEC> {
     static __device__ __forceinline__ void run(float* dst, const float* v) {
@@ -64,12 +68,24 @@ __device__ __forceinline__ void load_vec(const float* __restrict__ src, float* v
     }
 }
 
+// The rounding residue of a bf16 store: lo = bf16(v - bf16(v)), so that
+// hi + lo carries v to about 16 bits more than hi alone.
+template <int VEC>
+struct StoreLo<__nv_bfloat16, VEC> {
+    static __device__ __forceinline__ void run(__nv_bfloat16* dst, const float* v) {
+        float r[VEC];
+#pragma unroll
+        for (int k = 0; k < VEC; ++k) r[k] = v[k] - __bfloat162float(__float2bfloat16_rn(v[k]));
+        Store<__nv_bfloat16, VEC>::run(dst, r);
+    }
+};
+
 template <typename TP, int VEC>
 __global__ void __launch_bounds__(256)
 state_pass_kernel(const float* __restrict__ states, const float* __restrict__ logdecay,
                   const float* __restrict__ init, TP* __restrict__ prev,
                   float* __restrict__ fin, int64_t b, int64_t T, int64_t H, int64_t PN,
-                  int reverse) {
+                  int reverse, int64_t N, int64_t p_ext, TP* __restrict__ prev_lo) {
     const int64_t nvec = PN / VEC;
     const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (idx >= b * H * nvec) return;
@@ -77,9 +93,13 @@ state_pass_kernel(const float* __restrict__ states, const float* __restrict__ lo
     const int64_t off = (idx - bh * nvec) * VEC;
     const int64_t bb = bh / H, h = bh - bb * H;
 
+    // init and fin: (b, H, p_ext, N) when p_ext rows of the PN / N are the caller's
+    const int64_t p = off / N;
+    const bool ext_row = p < p_ext;
+    const int64_t ext = (bh * p_ext + p) * N + (off - p * N);
     float hs[VEC];
-    if (init) {
-        load_vec<VEC>(init + bh * PN + off, hs);
+    if (init && ext_row) {
+        load_vec<VEC>(init + ext, hs);
     } else {
 #pragma unroll
         for (int k = 0; k < VEC; ++k) hs[k] = 0.f;
@@ -91,6 +111,7 @@ state_pass_kernel(const float* __restrict__ states, const float* __restrict__ lo
     const float* sp = states + ((bb * T + c_first) * H + h) * PN + off;
     const float* lp = logdecay + (bb * T + c_first) * H + h;
     TP* pp = prev + ((bb * T + c_first) * H + h) * PN + off;
+    TP* pl = prev_lo ? prev_lo + ((bb * T + c_first) * H + h) * PN + off : nullptr;
     // a ring of kAhead chunks' states and log-decays in registers: the loads
     // of chunk c + kAhead are issued when chunk c is consumed
     float sv[kAhead][VEC], lv[kAhead];
@@ -115,6 +136,10 @@ state_pass_kernel(const float* __restrict__ states, const float* __restrict__ lo
             const float a = expf(lv[k]);
             Store<TP, VEC>::run(pq, hs);
             pq += cstride;
+            if (pl) {
+                StoreLo<TP, VEC>::run(pl, hs);
+                pl += cstride;
+            }
 #pragma unroll
             for (int e = 0; e < VEC; ++e) hs[e] = fmaf(a, hs[e], sv[k][e]);
             if (cl < T) {
@@ -126,8 +151,8 @@ state_pass_kernel(const float* __restrict__ states, const float* __restrict__ lo
             ++cl;
         }
     }
-    if (fin) {
-        float* fp = fin + bh * PN + off;
+    if (fin && ext_row) {
+        float* fp = fin + ext;
 #pragma unroll
         for (int k = 0; k < VEC; ++k) fp[k] = hs[k];
     }
@@ -141,14 +166,15 @@ __global__ void copy_or_zero_kernel(const float* __restrict__ src, float* __rest
 
 template <typename TP, int VEC>
 cudaError_t run(const float* states, const float* logdecay, const float* init, void* prev,
-                float* fin, const Dims& d, bool reverse, cudaStream_t s) {
+                float* fin, const Dims& d, bool reverse, int64_t p_ext, void* prev_lo, cudaStream_t s) {
     const int64_t PN = d.P * d.N;
     const int64_t threads = d.b * d.H * (PN / VEC);
     if (threads == 0) return cudaSuccess;
     const int bs = 256;
     const int64_t blocks = (threads + bs - 1) / bs;
     state_pass_kernel<TP, VEC><<<(unsigned)blocks, bs, 0, s>>>(
-        states, logdecay, init, static_cast<TP*>(prev), fin, d.b, d.T, d.H, PN, reverse ? 1 : 0);
+        states, logdecay, init, static_cast<TP*>(prev), fin, d.b, d.T, d.H, PN, reverse ? 1 : 0,
+        d.N, p_ext, static_cast<TP*>(prev_lo));
     return cudaGetLastError();
 }
 
@@ -156,13 +182,15 @@ cudaError_t run(const float* states, const float* logdecay, const float* init, v
 
 cudaError_t launch_state_pass(const float* states, const float* logdecay, const float* init,
                               void* prev, float* fin, const Dims& d, Elt t, cudaStream_t s,
-                              bool reverse) {
-    const bool v4 = ((d.P * d.N) % 4) == 0;
+                              bool reverse, int64_t p_ext, void* prev_lo) {
+    // with p_ext rows a vector of 4 must stay within one state row
+    const int64_t pe = (p_ext > 0 && p_ext < d.P) ? p_ext : d.P;
+    const bool v4 = pe == d.P ? ((d.P * d.N) % 4) == 0 : (d.N % 4) == 0;
     if (t == Elt::F32)
-        return v4 ? run<float, 4>(states, logdecay, init, prev, fin, d, reverse, s)
-                  : run<float, 1>(states, logdecay, init, prev, fin, d, reverse, s);
-    return v4 ? run<__nv_bfloat16, 4>(states, logdecay, init, prev, fin, d, reverse, s)
-              : run<__nv_bfloat16, 1>(states, logdecay, init, prev, fin, d, reverse, s);
+        return v4 ? run<float, 4>(states, logdecay, init, prev, fin, d, reverse, pe, nullptr, s)
+                  : run<float, 1>(states, logdecay, init, prev, fin, d, reverse, pe, nullptr, s);
+    return v4 ? run<__nv_bfloat16, 4>(states, logdecay, init, prev, fin, d, reverse, pe, prev_lo, s)
+              : run<__nv_bfloat16, 1>(states, logdecay, init, prev, fin, d, reverse, pe, prev_lo, s);
 }
 
 cudaError_t launch_copy_or_zero(const float* init, float* fin, int64_t n, cudaStream_t s) {

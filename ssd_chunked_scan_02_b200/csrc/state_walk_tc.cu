@@ -98,7 +98,7 @@ state_walk_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
                      const float* __restrict__ dt, const float* __restrict__ A,
                      const float* __restrict__ init, __nv_bfloat16* __restrict__ prev,
                      float* __restrict__ fin, int64_t L, int H, int G, int64_t T,
-                     int ksplit, WaitCtx status) {
+                     int ksplit, int pcols, WaitCtx status) {
     using S = WalkSmem<Q, N>;
     constexpr bool kTrans = (N == 128);
     constexpr int kNSub = Q / kSub;
@@ -305,12 +305,14 @@ state_walk_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
 #pragma unroll 1
             for (int cc = 0; cc < 4; ++cc) {
                 const int k = cc >> 1, p0 = (cc & 1) * 32;
-                const int64_t srow = ((b * H + h0 + k) * 64 + p0) * (int64_t)N + n;
+                // init: (b, H, pcols, N), pcols = 64 or 32 (rows pcols .. 63 zero)
+                const int64_t srow = ((b * H + h0 + k) * pcols + p0) * (int64_t)N + n;
                 const bool real = k == 0 || has1;
+                const bool rows = init && real && p0 < pcols;
                 uint32_t r[32];
 #pragma unroll
                 for (int e = 0; e < 32; ++e)
-                    r[e] = __float_as_uint((init && real) ? init[srow + (int64_t)e * N] : 0.f);
+                    r[e] = __float_as_uint(rows ? init[srow + (int64_t)e * N] : 0.f);
                 if (real) {
                     __nv_bfloat16* pr = prev + (((b * T) * H + h0 + k) * 64 + p0) * (int64_t)N + n;
 #pragma unroll
@@ -329,11 +331,11 @@ state_walk_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
             // lane m = (head m / 64, p = m % 64); TMEM columns = state n (N = 64)
             const int k = m >> 6, p = m & 63;
             const bool real = k == 0 || has1;
-            const int64_t srow = ((b * H + h0 + k) * 64 + p) * (int64_t)N;
+            const int64_t srow = ((b * H + h0 + k) * pcols + p) * (int64_t)N;
 #pragma unroll 1
             for (int cc = 0; cc < N / 32; ++cc) {
                 uint32_t r[32];
-                if (init && real) {
+                if (init && real && p < pcols) {
                     const float4* s4 = reinterpret_cast<const float4*>(init + srow + cc * 32);
 #pragma unroll
                     for (int q = 0; q < 8; ++q) {
@@ -422,8 +424,8 @@ state_walk_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
 #pragma unroll
                         for (int e = 0; e < 32; ++e)
                             pr[(int64_t)e * N] = __float2bfloat16_rn(__uint_as_float(hr[e]));
-                    } else {
-                        float* fp = fin + ((b * H + h0 + k) * 64 + p0) * (int64_t)N + n;
+                    } else if (p0 < pcols) {
+                        float* fp = fin + ((b * H + h0 + k) * pcols + p0) * (int64_t)N + n;
 #pragma unroll
                         for (int e = 0; e < 32; ++e) fp[(int64_t)e * N] = __uint_as_float(hr[e]);
                     }
@@ -448,9 +450,9 @@ state_walk_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
                             v.w = pack_bf16x2(__uint_as_float(hr[e + 6]), __uint_as_float(hr[e + 7]));
                             *reinterpret_cast<uint4*>(pr + e) = v;
                         }
-                    } else {
+                    } else if (p < pcols) {
                         float4* f4 = reinterpret_cast<float4*>(
-                            fin + ((b * H + h0 + k) * 64 + p) * (int64_t)N + cc * 32);
+                            fin + ((b * H + h0 + k) * pcols + p) * (int64_t)N + cc * 32);
 #pragma unroll
                         for (int q = 0; q < 8; ++q)
                             f4[q] = make_float4(__uint_as_float(hr[4 * q]), __uint_as_float(hr[4 * q + 1]),
@@ -480,11 +482,12 @@ state_walk_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
 template <int Q, int N>
 cudaError_t launch_impl(const void* x, const float* dt, const float* A, const void* B,
                         const float* init, void* prev, float* fin, const Dims& d, int ksplit,
-                        cudaStream_t s) {
+                        int pc, cudaStream_t s) {
     using S = WalkSmem<Q, N>;
     CUtensorMap tmX, tmB;
-    const uint64_t xdims[4] = {64, (uint64_t)d.H, (uint64_t)d.L, (uint64_t)d.b};
-    const uint64_t xstr[3] = {64 * 2, (uint64_t)(d.H * 64 * 2), (uint64_t)(d.L * d.H * 64 * 2)};
+    // x: pc columns a (virtual) head; a 64-column box reads zeros past them
+    const uint64_t xdims[4] = {(uint64_t)pc, (uint64_t)d.H, (uint64_t)d.L, (uint64_t)d.b};
+    const uint64_t xstr[3] = {(uint64_t)pc * 2, (uint64_t)(d.H * pc * 2), (uint64_t)(d.L * d.H * pc * 2)};
     const uint32_t box[4] = {64, 1, kSub, 1};
     cudaError_t e = make_tmap_bf16(&tmX, x, 4, xdims, xstr, box);
     if (e != cudaSuccess) return e;
@@ -500,7 +503,7 @@ cudaError_t launch_impl(const void* x, const float* dt, const float* A, const vo
     const int64_t grid = d.b * d.G * HeadPairs((int)d.H, (int)d.G).per_group();
     state_walk_tc_kernel<Q, N><<<(unsigned)grid, kThreads, S::kAlloc, s>>>(
         tmX, tmB, dt, A, init, static_cast<__nv_bfloat16*>(prev), fin, d.L, (int)d.H, (int)d.G,
-        d.T, ksplit, status);
+        d.T, ksplit, pc, status);
     return cudaGetLastError();
 }
 
@@ -524,10 +527,10 @@ cudaError_t launch_state_walk_tc(const void* x, const float* dt, const float* A,
     const Dims v = virtual_heads(d, &k);
     if (v.b * v.G * HeadPairs((int)v.H, (int)v.G).per_group() > 0x7fffffffLL)
         return cudaErrorInvalidValue;
-    if (v.Q == 256 && v.N == 128) return launch_impl<256, 128>(x, dt, A, B, init, prev, fin, v, k, s);
-    if (v.Q == 256 && v.N == 64) return launch_impl<256, 64>(x, dt, A, B, init, prev, fin, v, k, s);
-    if (v.Q == 128 && v.N == 128) return launch_impl<128, 128>(x, dt, A, B, init, prev, fin, v, k, s);
-    if (v.Q == 128 && v.N == 64) return launch_impl<128, 64>(x, dt, A, B, init, prev, fin, v, k, s);
+    if (v.Q == 256 && v.N == 128) return launch_impl<256, 128>(x, dt, A, B, init, prev, fin, v, k, head_cols(d), s);
+    if (v.Q == 256 && v.N == 64) return launch_impl<256, 64>(x, dt, A, B, init, prev, fin, v, k, head_cols(d), s);
+    if (v.Q == 128 && v.N == 128) return launch_impl<128, 128>(x, dt, A, B, init, prev, fin, v, k, head_cols(d), s);
+    if (v.Q == 128 && v.N == 64) return launch_impl<128, 64>(x, dt, A, B, init, prev, fin, v, k, head_cols(d), s);
     return cudaErrorNotSupported;
 }
 

@@ -44,7 +44,8 @@ sm100::WaitCtx make_wait_ctx() {
 
 bool tc_supported(const Dims& d, Elt t) {
     if (t != Elt::BF16) return false;
-    if (d.P % 64 != 0 || d.P > 256) return false;     // k virtual heads of headdim 64
+    // k virtual heads of headdim 64, or one padded from 32
+    if (d.P != 32 && (d.P % 64 != 0 || d.P > 256)) return false;
     if (d.N != 64 && d.N != 128) return false;
     if (d.Q != 128 && d.Q != 256) return false;
     if (d.L <= 0 || d.b <= 0) return false;

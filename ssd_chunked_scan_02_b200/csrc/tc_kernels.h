@@ -10,15 +10,23 @@ namespace ssd {
 // The tcgen05 kernels work on heads of headdim 64.  A head of headdim 64 k is
 // handled as k such (virtual) heads that share dt, A and D -- the rows of a
 // state evolve independently, and x, y and the states (b, ., H, P, .) are
-// the same memory as (b, ., H k, 64, .).  Returns the virtual sizes (H k,
-// P 64) and k.
+// the same memory as (b, ., H k, 64, .).  A head of headdim 32 runs as a head
+// of 64 whose last 32 rows are zero: its x tiles are loaded with zeros past
+// column 32 (the tensor map's edge), y tiles are stored up to column 32, the
+// kernels' own state buffers keep 64 rows, and states in the caller's
+// (b, H, 32, N) layout are read and written row by row.  Returns the virtual
+// sizes (H k, P 64) and k.
 inline Dims virtual_heads(const Dims& d, int* ksplit) {
     Dims v = d;
-    *ksplit = (int)(d.P / 64);
+    *ksplit = d.P >= 64 ? (int)(d.P / 64) : 1;
     v.H = d.H * *ksplit;
     v.P = 64;
     return v;
 }
+// Columns of x (and y) per virtual head, and the rows per head of the
+// internal state buffers, for a head of the caller's headdim.
+inline int head_cols(const Dims& d) { return d.P < 64 ? (int)d.P : 64; }
+inline int64_t state_rows(int64_t P) { return P < 64 ? 64 : P; }
 
 // The state kernels work on pairs of (virtual) heads of one group.  A group
 // with an odd number of heads pairs its last head with a phantom: its x is
@@ -37,7 +45,9 @@ struct HeadPairs {
     }
 };
 
-// True when the tensor-core kernels cover these sizes and dtype.
+// True when the tensor-core kernels cover these sizes and dtype (headdim 32
+// or 64 k up to 256; the step entry points, whose state buffers are the
+// caller's, take the multiples of 64 only).
 bool tc_supported(const Dims& d, Elt t);
 
 // rev: the backward's per-chunk dL/dh contributions instead (weights

@@ -62,7 +62,8 @@ def _round(v):
     (2, 600, 4, 64, 128, 2, 128, ssd.SSD_BF16),   # ragged: 5 chunks, last one partial
     (3, 1, 2, 3, 5, 1, 16, ssd.SSD_F32),
     (2, 300, 4, 64, 128, 1, 64, ssd.SSD_BF16),    # bf16 below 128: runs 128-token chunks
-    (2, 300, 4, 32, 128, 1, 64, ssd.SSD_BF16),    # headdim 32: SIMT, chunks as asked
+    (2, 300, 4, 32, 128, 1, 64, ssd.SSD_BF16),    # headdim 32: tensor cores, 64 state rows
+    (2, 300, 4, 32, 128, 1, 64, ssd.SSD_F32),     # headdim 32 in fp32: SIMT, chunks as asked
 ])
 def test_workspace_size_formula(lib, b, L, H, P, N, G, Q, dt):
     dims = ssd.make_dims(b, L, H, P, N, G)
@@ -72,7 +73,8 @@ def test_workspace_size_formula(lib, b, L, H, P, N, G, Q, dt):
     Qe = max(Q, 128) if tc else Q
     T = (L + Qe - 1) // Qe
     elt = 4 if dt == ssd.SSD_F32 else 2
-    ns = b * T * H * P * N
+    # the tensor-core flows keep 64 state rows for a head of headdim 32
+    ns = b * T * H * (max(P, 64) if tc else P) * N
     if lib.ssd_chunk_scan_fwd_data_flow(ctypes.byref(dims), Q, dt) == ssd.SSD_FLOW_WALK_OUTPUT:
         # the walk keeps chunk states on chip: only the entering states
         assert n == _round(ns * elt)
@@ -90,7 +92,9 @@ def test_workspace_size_formula(lib, b, L, H, P, N, G, Q, dt):
     (6, 32768, 32, 64, 64, 1, 256, ssd.SSD_BF16, ssd.SSD_FLOW_WALK_OUTPUT),  # 96 walkers
     (2, 600, 4, 64, 128, 1, 256, ssd.SSD_BF16, ssd.SSD_FLOW_TC_THREE_KERNEL),
     (4, 8192, 80, 64, 128, 1, 256, ssd.SSD_F32, ssd.SSD_FLOW_SIMT),
-    (4, 8192, 80, 32, 128, 1, 256, ssd.SSD_BF16, ssd.SSD_FLOW_SIMT),
+    (4, 8192, 80, 32, 128, 1, 256, ssd.SSD_BF16, ssd.SSD_FLOW_WALK_OUTPUT),   # headdim 32
+    (2, 600, 4, 32, 128, 1, 256, ssd.SSD_BF16, ssd.SSD_FLOW_TC_THREE_KERNEL),
+    (2, 600, 4, 96, 128, 1, 256, ssd.SSD_BF16, ssd.SSD_FLOW_SIMT),            # headdim 96
     (4, 8192, 40, 128, 128, 1, 256, ssd.SSD_BF16, ssd.SSD_FLOW_WALK_OUTPUT),  # 80 virtual heads
     (2, 600, 6, 64, 128, 2, 256, ssd.SSD_BF16, ssd.SSD_FLOW_TC_THREE_KERNEL),  # 3 heads a group
     (16, 600, 10, 64, 128, 2, 256, ssd.SSD_BF16, ssd.SSD_FLOW_WALK_OUTPUT),   # 96 walkers
@@ -280,24 +284,26 @@ def test_backward_workspace_size_formula(lib, b, L, H, P, N, G, dt):
 
 @pytest.mark.parametrize("b,L,H,P,N,G", [
     (8, 2048, 24, 64, 128, 1), (1, 70, 2, 128, 128, 2), (2, 300, 4, 64, 64, 2), (1, 1, 3, 192, 128, 1),
+    (2, 300, 4, 32, 64, 2),
 ])
 def test_backward_tensor_core_workspace_size_formula(lib, b, L, H, P, N, G):
     # tensor-core path (bf16): per 128-token chunk the entering states and
-    # dL/dh in bf16, one fp32 buffer of the same size and the chunks' log
-    # decays, each rounded up to 256 bytes
+    # dL/dh, each as two bf16 planes (value and rounding residue), one fp32
+    # buffer of the same size and the chunks' log decays, each rounded up to
+    # 256 bytes; a head of headdim 32 keeps 64 state rows
     dims = ssd.make_dims(b, L, H, P, N, G)
     assert ssd.load().ssd_chunk_scan_bwd_uses_tensor_cores(ctypes.byref(dims), ssd.SSD_BF16) == 1
     st, n = _bwd_ws(dims, ssd.SSD_BF16)
     assert st == ssd.SSD_OK
     up = lambda v: (v + 255) // 256 * 256
     T = (L + 127) // 128
-    e = b * T * H * P * N
-    assert n == up(e * 2) + up(e * 2) + up(e * 4) + up(b * T * H * 4)
+    e = b * T * H * max(P, 64) * N
+    assert n == 4 * up(e * 2) + up(e * 4) + up(b * T * H * 4)
 
 
 @pytest.mark.parametrize("P,N,dt,want", [
     (64, 128, ssd.SSD_BF16, 1), (256, 64, ssd.SSD_BF16, 1), (64, 128, ssd.SSD_F32, 0),
-    (32, 128, ssd.SSD_BF16, 0), (64, 96, ssd.SSD_BF16, 0), (96, 64, ssd.SSD_BF16, 0),
+    (32, 128, ssd.SSD_BF16, 1), (64, 96, ssd.SSD_BF16, 0), (96, 64, ssd.SSD_BF16, 0),
     (320, 64, ssd.SSD_BF16, -1),
     (64, 512, ssd.SSD_BF16, -1),
 ])

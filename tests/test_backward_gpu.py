@@ -89,6 +89,8 @@ TC_CASES = [
     ("L129_P192_G3",   95, 1, 129, 6, 192, 64,  3, False, False),
     ("L1",             96, 2, 1,   2, 64,  128, 1, True,  True),
     ("L640_H8_G2",     97, 1, 640, 8, 64,  128, 2, True,  True),
+    ("L300_P32",       98, 2, 300, 4, 32,  128, 1, True,  True),
+    ("L200_P32_N64_G2", 99, 1, 200, 4, 32, 64,  2, False, True),
 ]
 
 

@@ -66,6 +66,11 @@ TC_SHAPES = [
     ("tc_odd_hpg_walk_n64", 48, 300, 3, 64, 64, 1, 128, False),
     ("tc_q32_runs_q128", 2, 333, 4, 64, 128, 1, 32, True),
     ("tc_q16_ragged", 1, 77, 2, 64, 64, 1, 16, True),
+    # headdim 32: a head of 64 with 32 zero columns, internal states padded
+    ("tc_p32_three_kernel", 2, 600, 4, 32, 128, 1, 256, True),
+    ("tc_p32_walk", 16, 500, 12, 32, 128, 2, 128, True),
+    ("tc_p32_walk_n64_odd_hpg", 48, 300, 3, 32, 64, 1, 256, True),
+    ("tc_p32_n64_groups2_q64", 2, 333, 6, 32, 64, 2, 64, False),
 ]
 
 
