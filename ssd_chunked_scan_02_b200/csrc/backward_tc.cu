@@ -75,8 +75,10 @@ struct BwdSmem {
     // a Gam/h slot: Gam, [Gam lo], h, [h lo]
     static constexpr int kGHSlot = (kLo ? 4 : 2) * kGH;
     static constexpr int kGHBase = kDy + XY * kTok;
-    static constexpr int kGamOff = 0, kGamLoOff = kGH;
-    static constexpr int kHpOff = (kLo ? 2 : 1) * kGH, kHpLoOff = 3 * kGH;
+    static constexpr int kGamOff = 0;
+    static constexpr int kHpOff = (kLo ? 2 : 1) * kGH;
+    static constexpr int gam_lo_off() { return kGH; }
+    static constexpr int hp_lo_off() { return 3 * kGH; }
     static constexpr int kM = kGHBase + GH * kGHSlot; // bf16 128 x 128 (two 64-column blocks)
     static constexpr int kCs = kM + 2 * kTok;         // float[128]: cs (log2 units)
     static constexpr int kDt = kCs + kQ * 4;          // float[128]: dt
@@ -192,9 +194,9 @@ __device__ __forceinline__ void produce(uint8_t* smem, uint64_t* bars, const CUt
             tma_load_2d(slot + S::kGamOff + nb * S::kSt, tmGam, &bars[BAR_GHFULL + sg], nb * 64, row);
             tma_load_2d(slot + S::kHpOff + nb * S::kSt, tmHp, &bars[BAR_GHFULL + sg], nb * 64, row);
             if constexpr (S::kHasLo) {
-                tma_load_2d(slot + S::kGamLoOff + nb * S::kSt, tmGamLo, &bars[BAR_GHFULL + sg],
+                tma_load_2d(slot + S::gam_lo_off() + nb * S::kSt, tmGamLo, &bars[BAR_GHFULL + sg],
                             nb * 64, row);
-                tma_load_2d(slot + S::kHpLoOff + nb * S::kSt, tmHpLo, &bars[BAR_GHFULL + sg],
+                tma_load_2d(slot + S::hp_lo_off() + nb * S::kSt, tmHpLo, &bars[BAR_GHFULL + sg],
                             nb * 64, row);
             }
         }
@@ -250,9 +252,9 @@ bwd_dx_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
     uint8_t* sC = smem + S::kC;
     uint8_t* sB = smem + S::kB;
     uint8_t* sGam = smem + S::kGHBase + S::kGamOff;     // one Gam/h slot
-    uint8_t* sGamLo = smem + S::kGHBase + S::kGamLoOff;
+    uint8_t* sGamLo = smem + S::kGHBase + S::gam_lo_off();
     uint8_t* sHp = smem + S::kGHBase + S::kHpOff;
-    uint8_t* sHpLo = smem + S::kGHBase + S::kHpLoOff;
+    uint8_t* sHpLo = smem + S::kGHBase + S::hp_lo_off();
     uint8_t* sM = smem + S::kM;
     float* s_cs = reinterpret_cast<float*>(smem + S::kCs);
     float* s_dt = reinterpret_cast<float*>(smem + S::kDt);
