@@ -416,12 +416,15 @@ bwd_dx_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                 tmem_ld32x2(tmem + lb + kColG + 32 * j, tmem + lb + kColR + 32 * j, gr, rr);
                 float v[32];
                 uint32_t pk[16];
+                // every element computed, the mask applied by selects: no branch
+                // per element, so the loads and exponentials overlap (past the
+                // diagonal the exponential may overflow; it is never selected)
 #pragma unroll
                 for (int e = 0; e < 32; e += 2) {
                     const int s0 = 32 * j + e;
-                    float m0 = 0.f, m1 = 0.f;
-                    if (s0 <= u) m0 = __uint_as_float(gr[e]) * fast_exp2(csu - s_cs[s0]);
-                    if (s0 + 1 <= u) m1 = __uint_as_float(gr[e + 1]) * fast_exp2(csu - s_cs[s0 + 1]);
+                    const float e0 = __uint_as_float(gr[e]) * fast_exp2(csu - s_cs[s0]);
+                    const float e1 = __uint_as_float(gr[e + 1]) * fast_exp2(csu - s_cs[s0 + 1]);
+                    const float m0 = s0 <= u ? e0 : 0.f, m1 = s0 + 1 <= u ? e1 : 0.f;
                     pk[e >> 1] = pack_bf16x2(m0, m1);
                     v[e] = m0 * s_dt[s0] * __uint_as_float(rr[e]);
                     v[e + 1] = m1 * s_dt[s0 + 1] * __uint_as_float(rr[e + 1]);
@@ -695,14 +698,13 @@ bwd_dbc_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                 uint32_t rr[32];
                 tmem_ld32(tmem + lb + kColR + 32 * j, rr);
                 uint32_t pk[16];
+                // as in the dx kernel: every element, the mask by selects
 #pragma unroll
                 for (int e = 0; e < 32; e += 2) {
                     const int s0 = 32 * j + e;
-                    float m0 = 0.f, m1 = 0.f;
-                    if (s0 <= u) m0 = __uint_as_float(rr[e]) * fast_exp2(csu - s_cs[s0]) * s_dt[s0];
-                    if (s0 + 1 <= u)
-                        m1 = __uint_as_float(rr[e + 1]) * fast_exp2(csu - s_cs[s0 + 1]) * s_dt[s0 + 1];
-                    pk[e >> 1] = pack_bf16x2(m0, m1);
+                    const float e0 = __uint_as_float(rr[e]) * fast_exp2(csu - s_cs[s0]) * s_dt[s0];
+                    const float e1 = __uint_as_float(rr[e + 1]) * fast_exp2(csu - s_cs[s0 + 1]) * s_dt[s0 + 1];
+                    pk[e >> 1] = pack_bf16x2(s0 <= u ? e0 : 0.f, s0 + 1 <= u ? e1 : 0.f);
                 }
 #pragma unroll
                 for (int q = 0; q < 4; ++q)
@@ -715,7 +717,10 @@ bwd_dbc_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                 uint4* xrow = reinterpret_cast<uint4*>(smem + S::kX + (i & 1) * S::kTok + u * 128);
                 uint4* yrow = reinterpret_cast<uint4*>(smem + S::kDy + (i & 1) * S::kTok + u * 128);
 #pragma unroll
-                for (int q = 0; q < 8; ++q) {
+                for (int q0 = 0; q0 < 8; ++q0) {
+                    // the row's 16-byte chunks in a rotated order: the lanes of a
+                    // phase (rows 128 bytes apart) then hit different banks
+                    const int q = q0 ^ (u & 7);
                     uint4 xv = xrow[q], yv = yrow[q];
                     uint32_t* xw = reinterpret_cast<uint32_t*>(&xv);
                     uint32_t* yw = reinterpret_cast<uint32_t*>(&yv);
