@@ -29,12 +29,13 @@
 // heads, 192 threads: warps 0-3 = the epilogue (thread u = token row u = TMEM
 // lane u), warp 4 = TMA producer, warp 5 = MMA issuer (and TMEM owner).  A
 // head's inputs come into one of two slots while the previous head computes
-// (bwd_dx: x and dy in two slots, Gam and h in one, released once <Gam, h>
-// and the MMAs that read them are done; bwd_dbc: all four in two slots).
+// (bwd_dx: x and dy in two slots, Gam and h with their residues in one,
+// released once <Gam, h> and the MMAs that read them are done; bwd_dbc: all
+// four in two slots).
 //   bwd_dx:  G once; per head R, X1 = B Gam^T, Ys = C h^T, then M1 =
 //            bf16(G o E) built by the epilogue (with W's row and column
-//            sums), then dxi = M1^T dy; the epilogue writes dx, ddt and adds
-//            the head's dA and dD.
+//            sums), then dxi = M1^T dy; the epilogue stages dx in the M1 tile
+//            for a TMA store, writes ddt and adds the head's dA and dD.
 //   bwd_dbc: per head R, then M2 = bf16(R o E o dt_s) and x, dy scaled in
 //            place (dt_s el_s x_s, ei_t dy_t), then dC += M2 B + dy' h and
 //            dB += M2^T C + x' Gam accumulated in TMEM over the heads; the
@@ -82,8 +83,8 @@ struct BwdSmem {
     static constexpr int kM = kGHBase + GH * kGHSlot; // bf16 128 x 128 (two 64-column blocks)
     static constexpr int kCs = kM + 2 * kTok;         // float[128]: cs (log2 units)
     static constexpr int kDt = kCs + kQ * 4;          // float[128]: dt
-    static constexpr int kCol = kDt + kQ * 4;         // float[4][128]: per-warp column sums of W
-    static constexpr int kRed = kCol + (kCols ? 4 * kQ * 4 : 0);   // float[32]: reductions
+    static constexpr int kCol = kDt + kQ * 4;         // float[128]: column sums of W
+    static constexpr int kRed = kCol + (kCols ? kQ * 4 : 0);       // float[32]: reductions
     static constexpr int kBar = kRed + 32 * 4;
     static constexpr int kTmem = kBar + 16 * 8;
     static constexpr int kCnt = kTmem + 16;           // [0] heads loaded, [1] MMAs issued
@@ -92,7 +93,7 @@ struct BwdSmem {
     static constexpr int kAlloc = kTotal + 1024;      // slack to align the base to 1 KB
     static_assert(kAlloc <= 232448, "shared memory per CTA");
 };
-template <int N> using DxSmem = BwdSmem<N, 1, 1, true, true>;
+template <int N> using DxSmem = BwdSmem<N, 2, 1, true, true>;
 template <int N> using DbcSmem = BwdSmem<N, 2, 2, false, false>;
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
@@ -231,6 +232,7 @@ bwd_dx_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                  const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmC,
                  const __grid_constant__ CUtensorMap tmGam, const __grid_constant__ CUtensorMap tmHp,
                  const __grid_constant__ CUtensorMap tmGamLo, const __grid_constant__ CUtensorMap tmHpLo,
+                 const __grid_constant__ CUtensorMap tmDx,
                  const float* __restrict__ dt, const float* __restrict__ A,
                  const float* __restrict__ Dv, float* __restrict__ dx, float* __restrict__ ddt,
                  float* __restrict__ dA, float* __restrict__ dD, int64_t L, int H, int G,
@@ -360,6 +362,7 @@ bwd_dx_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
         bool fail = false;
         float ddt_acc = 0.f, dA_acc = 0.f, dD_acc = 0.f;
         float dt_next = (row_in && nh > 0) ? dt_row[head0 / ksplit] : 0.f;
+        s_col[u] = 0.f;   // column sums of W: added to by the warps, read and cleared by thread u
         for (int i = 0; i < nh; ++i) {
             const int hv = head0 + i, hr = hv / ksplit;
             const float Ah = A[hr];
@@ -371,6 +374,9 @@ bwd_dx_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
             s_dt[u] = dtu;
             if (i == 0) fail = fail || !mbar_wait(&bars[BAR_G], 0, status);
             fail = fail || !mbar_wait(&bars[BAR_ACC1], (uint32_t)(i & 1), status);
+            // the M1 tile is rewritten below: the previous head's dx store must
+            // have read it
+            if (u == 0) bulk_wait_group_read<0>();
             if (named_bar_or(2, 128, fail)) {   // also publishes s_cs, s_dt
                 fail = true;
                 break;
@@ -409,7 +415,6 @@ bwd_dx_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                     // columns s = 32 j .. 32 j + 31 all lie past every row of this warp
 #pragma unroll
                     for (int q = 0; q < 4; ++q) mrow[((j & 1) * 4 + q) ^ (u & 7)] = make_uint4(0, 0, 0, 0);
-                    s_col[warp * 128 + 32 * j + lane] = 0.f;
                     continue;
                 }
                 uint32_t gr[32], rr[32];
@@ -435,7 +440,7 @@ bwd_dx_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                     mrow[((j & 1) * 4 + q) ^ (u & 7)] =
                         make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
                 warp_column_sums(v, lane);
-                s_col[warp * 128 + 32 * j + lane] = v[0];
+                atomicAdd(&s_col[32 * j + lane], v[0]);
             }
             fence_proxy_async_smem();
             tc_fence_before();
@@ -444,7 +449,8 @@ bwd_dx_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                 mbar_arrive(&bars[BAR_MREADY]);
                 mbar_arrive(&bars[BAR_GHEMPTY]);   // Gam, h: read by their MMAs and above
             }
-            float dcs = rowsum - (s_col[u] + s_col[128 + u] + s_col[256 + u] + s_col[384 + u]);
+            float dcs = rowsum - s_col[u];
+            s_col[u] = 0.f;   // the next head's additions come after more barriers
 
             // ---- dx, and the row's dot products
             fail = !mbar_wait(&bars[BAR_ACC2], (uint32_t)(i & 1), status);
@@ -459,8 +465,9 @@ bwd_dx_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
             const int sx = i % S::kXY;
             const uint4* xrow = reinterpret_cast<const uint4*>(smem + S::kX + sx * S::kTok + u * 128);
             const uint4* dyrow = reinterpret_cast<const uint4*>(smem + S::kDy + sx * S::kTok + u * 128);
-            // dx: (b, L, H, pcols) with pcols = 64, or 32 (a head of headdim 32)
-            float* dxo = dx + ((b * L + t0 + u) * H + hv) * pcols;
+            // dx rows are staged in the M1 tile (free once the M1^T dy MMAs
+            // are done) as 32-column fp32 boxes, 128-byte swizzled, then stored
+            // by TMA (rows past the sequence end clipped by the tensor map)
 #pragma unroll 1
             for (int k = 0; k < 2; ++k) {
                 uint32_t dr[32], xr1[32], yr[32];
@@ -489,13 +496,12 @@ bwd_dx_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                             dxd += ye[h2] * xe[h2];
                         }
                     }
-                    if (row_in && 32 * k < pcols) {
-                        float4* d4 = reinterpret_cast<float4*>(dxo + 32 * k + 8 * q);
-                        d4[0] = make_float4(o[0], o[1], o[2], o[3]);
-                        d4[1] = make_float4(o[4], o[5], o[6], o[7]);
-                    }
+                    float4* box = reinterpret_cast<float4*>(sM + k * S::kTok + u * 128);
+                    box[(2 * q) ^ (u & 7)] = make_float4(o[0], o[1], o[2], o[3]);
+                    box[(2 * q + 1) ^ (u & 7)] = make_float4(o[4], o[5], o[6], o[7]);
                 }
             }
+            fence_proxy_async_smem();
             tc_fence_before();
             const float Uu = dtu * el * sU;
             dcs += ei * dyys - Uu;
@@ -510,6 +516,9 @@ bwd_dx_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
             if (u == 0) {
                 mbar_arrive(&bars[BAR_ACCEMPTY]);
                 mbar_arrive(&bars[BAR_XYEMPTY + sx]);
+                for (int k = 0; k < pcols / 32; ++k)
+                    tma_store_4d(&tmDx, sM + k * S::kTok, 32 * k, hv, (int)t0, (int)b);
+                bulk_commit_group();
             }
             if (u == kQ - 1) {
                 const float sumU = s_red[4] + s_red[5] + s_red[6] + s_red[7];
@@ -546,6 +555,7 @@ bwd_dx_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                 ddt_acc = dA_acc = dD_acc = 0.f;
             }
         }
+        if (u == 0) bulk_wait_group<0>();      // dx stores done before the CTA leaves
         if (fail) s_flag[0] = 1;
     }
 
@@ -810,6 +820,15 @@ cudaError_t launch_impl(const void* x, const void* dy, const float* dt, const fl
         e = make_tmap_bf16(maps[k], planes[k], 2, hdims, hstr, hbox);
         if (e != cudaSuccess) return e;
     }
+    // dx (b, L, H, pc) fp32 as 32-column boxes of 128 rows, 128-byte swizzled
+    CUtensorMap tmDx;
+    {
+        const uint64_t ddims[4] = {(uint64_t)pc, (uint64_t)d.H, (uint64_t)d.L, (uint64_t)d.b};
+        const uint64_t dstr[3] = {(uint64_t)pc * 4, (uint64_t)(d.H * pc * 4), (uint64_t)(d.L * d.H * pc * 4)};
+        const uint32_t dbox[4] = {32, 1, kQ, 1};
+        e = make_tmap_f32_plain(&tmDx, dx, 4, ddims, dstr, dbox, true);
+        if (e != cudaSuccess) return e;
+    }
     const sm100::WaitCtx status = make_wait_ctx();
     if (!status.word) return cudaErrorUnknown;
 
@@ -822,7 +841,7 @@ cudaError_t launch_impl(const void* x, const void* dy, const float* dt, const fl
                              DbcSmem<N>::kAlloc);
     if (e != cudaSuccess) return e;
     bwd_dx_tc_kernel<N><<<(unsigned)grid, kThreads, DxSmem<N>::kAlloc, s>>>(
-        tmX, tmDy, tmB, tmC, tmGam, tmHp, tmGamLo, tmHpLo, dt, A, D, dx, ddt, dA, dD, d.L,
+        tmX, tmDy, tmB, tmC, tmGam, tmHp, tmGamLo, tmHpLo, tmDx, dt, A, D, dx, ddt, dA, dD, d.L,
         (int)d.H, (int)d.G, d.T, ksplit, pc, status);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
