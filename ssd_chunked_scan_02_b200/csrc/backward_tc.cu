@@ -421,19 +421,41 @@ bwd_dx_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                 tmem_ld32x2(tmem + lb + kColG + 32 * j, tmem + lb + kColR + 32 * j, gr, rr);
                 float v[32];
                 uint32_t pk[16];
-                // every element computed, the mask applied by selects: no branch
-                // per element, so the loads and exponentials overlap (past the
-                // diagonal the exponential may overflow; it is never selected)
+                if (j < warp) {
+                    // a block wholly below the diagonal: the decay factorises
+                    // through the block's last column r, 2^(cs_u - cs_s) =
+                    // 2^(cs_u - r) 2^(r - cs_s) (both <= 1), one exponential a
+                    // row; lane l computes column 32 j + l's factor and the
+                    // others take it by shuffle
+                    const float r = s_cs[32 * j + 31];
+                    const float a = fast_exp2(csu - r);
+                    const float bl = fast_exp2(r - s_cs[32 * j + lane]);
 #pragma unroll
-                for (int e = 0; e < 32; e += 2) {
-                    const int s0 = 32 * j + e;
-                    const float e0 = __uint_as_float(gr[e]) * fast_exp2(csu - s_cs[s0]);
-                    const float e1 = __uint_as_float(gr[e + 1]) * fast_exp2(csu - s_cs[s0 + 1]);
-                    const float m0 = s0 <= u ? e0 : 0.f, m1 = s0 + 1 <= u ? e1 : 0.f;
-                    pk[e >> 1] = pack_bf16x2(m0, m1);
-                    v[e] = m0 * s_dt[s0] * __uint_as_float(rr[e]);
-                    v[e + 1] = m1 * s_dt[s0 + 1] * __uint_as_float(rr[e + 1]);
-                    rowsum += v[e] + v[e + 1];
+                    for (int e = 0; e < 32; e += 2) {
+                        const int s0 = 32 * j + e;
+                        const float m0 = __uint_as_float(gr[e]) * a * __shfl_sync(0xffffffffu, bl, e);
+                        const float m1 = __uint_as_float(gr[e + 1]) * a * __shfl_sync(0xffffffffu, bl, e + 1);
+                        pk[e >> 1] = pack_bf16x2(m0, m1);
+                        v[e] = m0 * s_dt[s0] * __uint_as_float(rr[e]);
+                        v[e + 1] = m1 * s_dt[s0 + 1] * __uint_as_float(rr[e + 1]);
+                        rowsum += v[e] + v[e + 1];
+                    }
+                } else {
+                    // the diagonal block: an exponential per element, the mask by
+                    // selects (no branch per element, so the loads and
+                    // exponentials overlap; past the diagonal the exponential
+                    // may overflow, and is never selected)
+#pragma unroll
+                    for (int e = 0; e < 32; e += 2) {
+                        const int s0 = 32 * j + e;
+                        const float e0 = __uint_as_float(gr[e]) * fast_exp2(csu - s_cs[s0]);
+                        const float e1 = __uint_as_float(gr[e + 1]) * fast_exp2(csu - s_cs[s0 + 1]);
+                        const float m0 = s0 <= u ? e0 : 0.f, m1 = s0 + 1 <= u ? e1 : 0.f;
+                        pk[e >> 1] = pack_bf16x2(m0, m1);
+                        v[e] = m0 * s_dt[s0] * __uint_as_float(rr[e]);
+                        v[e + 1] = m1 * s_dt[s0 + 1] * __uint_as_float(rr[e + 1]);
+                        rowsum += v[e] + v[e + 1];
+                    }
                 }
 #pragma unroll
                 for (int q = 0; q < 4; ++q)
@@ -708,13 +730,28 @@ bwd_dbc_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                 uint32_t rr[32];
                 tmem_ld32(tmem + lb + kColR + 32 * j, rr);
                 uint32_t pk[16];
-                // as in the dx kernel: every element, the mask by selects
+                if (j < warp) {
+                    // as in the dx kernel: below the diagonal, the decay through
+                    // the block's last column (one exponential a row, column
+                    // factors times dt by shuffle)
+                    const float r = s_cs[32 * j + 31];
+                    const float a = fast_exp2(csu - r);
+                    const float bl = fast_exp2(r - s_cs[32 * j + lane]) * s_dt[32 * j + lane];
 #pragma unroll
-                for (int e = 0; e < 32; e += 2) {
-                    const int s0 = 32 * j + e;
-                    const float e0 = __uint_as_float(rr[e]) * fast_exp2(csu - s_cs[s0]) * s_dt[s0];
-                    const float e1 = __uint_as_float(rr[e + 1]) * fast_exp2(csu - s_cs[s0 + 1]) * s_dt[s0 + 1];
-                    pk[e >> 1] = pack_bf16x2(s0 <= u ? e0 : 0.f, s0 + 1 <= u ? e1 : 0.f);
+                    for (int e = 0; e < 32; e += 2)
+                        pk[e >> 1] = pack_bf16x2(
+                            __uint_as_float(rr[e]) * a * __shfl_sync(0xffffffffu, bl, e),
+                            __uint_as_float(rr[e + 1]) * a * __shfl_sync(0xffffffffu, bl, e + 1));
+                } else {
+                    // the diagonal block, as in the dx kernel: an exponential per
+                    // element, the mask by selects
+#pragma unroll
+                    for (int e = 0; e < 32; e += 2) {
+                        const int s0 = 32 * j + e;
+                        const float e0 = __uint_as_float(rr[e]) * fast_exp2(csu - s_cs[s0]) * s_dt[s0];
+                        const float e1 = __uint_as_float(rr[e + 1]) * fast_exp2(csu - s_cs[s0 + 1]) * s_dt[s0 + 1];
+                        pk[e >> 1] = pack_bf16x2(s0 <= u ? e0 : 0.f, s0 + 1 <= u ? e1 : 0.f);
+                    }
                 }
 #pragma unroll
                 for (int q = 0; q < 4; ++q)

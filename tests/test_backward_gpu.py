@@ -91,6 +91,8 @@ TC_CASES = [
     ("L640_H8_G2",     97, 1, 640, 8, 64,  128, 2, True,  True),
     ("L300_P32",       98, 2, 300, 4, 32,  128, 1, True,  True),
     ("L200_P32_N64_G2", 99, 1, 200, 4, 32, 64,  2, False, True),
+    ("L260_P256",     100, 1, 260, 2, 256, 128, 1, True,  True),
+    ("L300_P128_N64_G2", 102, 2, 300, 4, 128, 64, 2, True, False),
 ]
 
 
