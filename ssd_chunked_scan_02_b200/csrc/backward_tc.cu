@@ -24,6 +24,11 @@
 // The decay terms are taken from W in fp32 (its row and column sums), not
 // from the bf16 operands of the other products: their row and column sums
 // cancel to within rounding of each other, and bf16 rounding there would not.
+// For the same reason Gam and h enter X1, Ys and <Gam, h> (whose sums nearly
+// cancel at a chunk's last token) as bf16 value + residue pairs, near fp32.
+// Below the diagonal E factorises through each 32-column block's last column
+// r (E_ts = 2^(cs_t - r) 2^(r - cs_s), both <= 1): one exponential a row and
+// one a column; the diagonal blocks take one per element.
 //
 // Two kernels, one CTA per (batch, chunk, group) looping over the group's
 // heads, 192 threads: warps 0-3 = the epilogue (thread u = token row u = TMEM
@@ -234,7 +239,7 @@ bwd_dx_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                  const __grid_constant__ CUtensorMap tmGamLo, const __grid_constant__ CUtensorMap tmHpLo,
                  const __grid_constant__ CUtensorMap tmDx,
                  const float* __restrict__ dt, const float* __restrict__ A,
-                 const float* __restrict__ Dv, float* __restrict__ dx, float* __restrict__ ddt,
+                 const float* __restrict__ Dv, float* __restrict__ ddt,
                  float* __restrict__ dA, float* __restrict__ dD, int64_t L, int H, int G,
                  int64_t T, int ksplit, int pcols, WaitCtx status) {
     // H counts virtual heads (headdim 64); real head = virtual head / ksplit
@@ -878,7 +883,7 @@ cudaError_t launch_impl(const void* x, const void* dy, const float* dt, const fl
                              DbcSmem<N>::kAlloc);
     if (e != cudaSuccess) return e;
     bwd_dx_tc_kernel<N><<<(unsigned)grid, kThreads, DxSmem<N>::kAlloc, s>>>(
-        tmX, tmDy, tmB, tmC, tmGam, tmHp, tmGamLo, tmHpLo, tmDx, dt, A, D, dx, ddt, dA, dD, d.L,
+        tmX, tmDy, tmB, tmC, tmGam, tmHp, tmGamLo, tmHpLo, tmDx, dt, A, D, ddt, dA, dD, d.L,
         (int)d.H, (int)d.G, d.T, ksplit, pc, status);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
