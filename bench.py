@@ -83,14 +83,20 @@ def kernel_bytes(w):
         "state_pass": (init + fin, 4 * ns + ld + sx * ns + init + fin),
         "state_walk": (x + bc + dt + init + fin, x + bc + dt + sx * ns + init + fin),
         "chunk_out": (2 * x + 2 * bc + dt, 2 * x + 2 * bc + dt + sx * ns),
+        # walkers and output tiles in one launch: the whole forward's bytes_min;
+        # its own I/O reads x and B twice (walkers and tiles) and writes and
+        # reads the entering states
+        "walk_out": (2 * x + 2 * bc + dt + init + fin,
+                     3 * x + 3 * bc + 2 * dt + init + fin + 2 * sx * ns),
     }
 
 
 KERNEL_SOURCES = {
-    "state_walk": ["state_walk_tc.cu", "sm100.cuh"],
+    "state_walk": ["state_walk_tc.cu", "state_walk_body.cuh", "sm100.cuh"],
     "chunk_state": ["chunk_state_tc.cu", "sm100.cuh"],
     "state_pass": ["state_pass.cu"],
-    "chunk_out": ["chunk_out_tc.cu", "sm100.cuh"],
+    "chunk_out": ["chunk_out_tc.cu", "chunk_out_body.cuh", "sm100.cuh"],
+    "walk_out": ["walk_out_tc.cu", "state_walk_body.cuh", "chunk_out_body.cuh", "sm100.cuh"],
     "decode": ["decode.cu"],
 }
 
@@ -398,9 +404,7 @@ def measure_config(w, dev, stream, flush, reps, world, rank):
     f_alg, f_dense, bytes_min = fwd_model(w)
     t = ms * 1e-3
     flow = ssd.ssd_chunk_scan_fwd_data_flow(dims, w.chunk, inp["x"].dtype)
-    out = {"workload": w.name, "data_flow": {ssd.SSD_FLOW_WALK_OUTPUT: "walk+output",
-                                              ssd.SSD_FLOW_TC_THREE_KERNEL: "three-kernel"}
-           .get(flow, "simt"), "ms_per_step": ms, "tokens_per_s": world * w.tokens / t,
+    out = {"workload": w.name, "data_flow": FLOW_NAMES.get(flow, "simt"), "ms_per_step": ms, "tokens_per_s": world * w.tokens / t,
            "tflops_alg": f_alg / t / 1e12, "tflops_dense": f_dense / t / 1e12,
            "bytes_min": bytes_min, "hbm_gbs_at_bytes_min": bytes_min / t / 1e9}
     del inp, y, fin, ws
@@ -546,7 +550,9 @@ def measure_seqpar(w, dev, stream, flush, reps, shards=2):
 
 
 # ---------------------------------------------------------------- per-kernel timing
-FLOW_KERNELS = {1: ("chunk_state", "state_pass", "chunk_out"), 2: ("state_walk", "chunk_out")}
+FLOW_KERNELS = {1: ("chunk_state", "state_pass", "chunk_out"), 2: ("state_walk", "chunk_out"),
+                3: ("walk_out",)}
+FLOW_NAMES = {1: "three-kernel", 2: "walk+output", 3: "walk+output, one launch"}
 
 
 def kernel_times(w, flow, inp, y, fin, dims, dev, stream, flush, reps):
@@ -569,9 +575,20 @@ def kernel_times(w, flow, inp, y, fin, dims, dev, stream, flush, reps):
     P = lambda t: ctypes.c_void_p(t.data_ptr()) if t is not None else None
     names = FLOW_KERNELS[flow]
     kt = {k: [] for k in names}
+    ws = None
+    if flow == ssd.SSD_FLOW_WALK_OUTPUT_FUSED:
+        # one launch (after the memset of its scheduling counters): the forward
+        # itself, in that data flow
+        ws = torch.empty(max(ssd.ssd_chunk_scan_fwd_workspace_size(dims, w.chunk, x.dtype,
+                                                                   flow=flow), 16),
+                         device=dev, dtype=torch.uint8)
 
     def launch(k):
-        if k == "chunk_state":
+        if k == "walk_out":
+            st = lib.ssd_chunk_scan_fwd_with_flow(P(x), P(dt), P(A), P(Bm), P(Cm), P(D), w.chunk,
+                                                  P(init), P(y), P(fin), ctypes.byref(dims),
+                                                  ssd.SSD_BF16, P(ws), ws.numel(), sp, flow)
+        elif k == "chunk_state":
             st = lib.ssd_chunk_state_fwd(P(x), P(dt), P(A), P(Bm), w.chunk, P(S_buf), P(ld_buf),
                                          ctypes.byref(dims), ssd.SSD_BF16, sp)
         elif k == "state_pass":
@@ -597,7 +614,7 @@ def kernel_times(w, flow, inp, y, fin, dims, dev, stream, flush, reps):
         if r >= 2:
             for i, k in enumerate(names):
                 kt[k].append(ev[i].elapsed_time(ev[i + 1]))
-    del prev_buf, S_buf, ld_buf
+    del prev_buf, S_buf, ld_buf, ws
     return {k: statistics.mean(v) for k, v in kt.items()}
 
 
@@ -674,8 +691,9 @@ def main():
     flow = ssd.ssd_chunk_scan_fwd_data_flow(dims, w.chunk, x.dtype)
     kmean = kernel_times(w, flow, inp, y, fin, dims, dev, stream, flush, max(5, args.steps // 2))
     # the other tensor-core flow, for comparison (not part of the forward)
-    alt_flow = (ssd.SSD_FLOW_TC_THREE_KERNEL if flow == ssd.SSD_FLOW_WALK_OUTPUT
-                else ssd.SSD_FLOW_WALK_OUTPUT)
+    alt_flow = {ssd.SSD_FLOW_WALK_OUTPUT_FUSED: ssd.SSD_FLOW_WALK_OUTPUT,
+                ssd.SSD_FLOW_WALK_OUTPUT: ssd.SSD_FLOW_TC_THREE_KERNEL}.get(
+                    flow, ssd.SSD_FLOW_WALK_OUTPUT)
     kalt = kernel_times(w, alt_flow, inp, y, fin, dims, dev, stream, flush,
                         max(5, args.steps // 4))
     dom = max(kmean, key=kmean.get)
@@ -858,8 +876,7 @@ def main():
                          "io_bytes_per_launch": kb[dom][1],
                          "io_gbs": dom_io_gbs, "io_frac": dom_io_gbs / peak_gbs,
                          "ms_per_launch": kmean[dom], "peak_source": pk["source"]},
-            "data_flow": {ssd.SSD_FLOW_WALK_OUTPUT: "walk+output",
-                          ssd.SSD_FLOW_TC_THREE_KERNEL: "three-kernel"}.get(flow, "simt"),
+            "data_flow": FLOW_NAMES.get(flow, "simt"),
             "kernels_ms": kmean,
             "kernels_ms_other_flow": kalt,
             "decode": {"workload": dw.name, "ms_per_step": dec_ms, "gbs": dec_gbs,

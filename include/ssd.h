@@ -98,7 +98,9 @@ SSD_API const char* ssd_last_error_detail(void);
 
 /*
  * Bytes of device workspace ssd_chunk_scan_fwd needs for these sizes
- * (chunk states, per-chunk log-decays and the states entering each chunk).
+ * (chunk states, per-chunk log-decays and the states entering each chunk,
+ * as the data flow needs them, and for the one-launch flow a few scheduling
+ * counters).
  * Writes the size to *bytes.  Returns SSD_ERR_INVALID_ARG / UNSUPPORTED on
  * sizes that ssd_chunk_scan_fwd would reject.
  */
@@ -353,6 +355,14 @@ SSD_API int ssd_chunk_scan_fwd_uses_tensor_cores(const ssd_dims_t* dims, int chu
 
 /* Which data flow ssd_chunk_scan_fwd takes for these sizes (decided from the
  * sizes alone; the workspace size follows from it):
+ *   SSD_FLOW_WALK_OUTPUT_FUSED  the same two parts in one launch: walkers
+ *                            of four heads and output tiles side by side, an
+ *                            output tile starting once the walkers have
+ *                            written the states entering its chunk (dstate
+ *                            128, heads per group a multiple of 4 after the
+ *                            headdim split, 16 chunks or more; a memset of
+ *                            the workspace's scheduling counters comes
+ *                            first);
  *   SSD_FLOW_WALK_OUTPUT     state walk (steps 2+3 on chip, entering states
  *                            written in bf16) then the tensor-core output
  *                            kernel (steps 1+4): two launches;
@@ -367,8 +377,32 @@ SSD_API int ssd_chunk_scan_fwd_uses_tensor_cores(const ssd_dims_t* dims, int chu
 #define SSD_FLOW_SIMT 0
 #define SSD_FLOW_TC_THREE_KERNEL 1
 #define SSD_FLOW_WALK_OUTPUT 2
+#define SSD_FLOW_WALK_OUTPUT_FUSED 3
 SSD_API int ssd_chunk_scan_fwd_data_flow(const ssd_dims_t* dims, int chunk_size,
                                          ssd_dtype_t dtype);
+
+/*
+ * ssd_chunk_scan_fwd with the data flow chosen by the caller: `flow` is one
+ * of the SSD_FLOW_* values above, or -1 for the library's own choice (what
+ * ssd_chunk_scan_fwd does).  Every flow computes the same result up to
+ * rounding; SSD_FLOW_SIMT covers every size, the tensor-core flows the
+ * sizes ssd_chunk_scan_fwd_uses_tensor_cores accepts, and
+ * SSD_FLOW_WALK_OUTPUT_FUSED further needs dstate 128 and a multiple of 4
+ * (virtual) heads per group.  A flow that does not cover the sizes returns
+ * SSD_ERR_UNSUPPORTED, an unknown one SSD_ERR_INVALID_ARG.  The workspace
+ * must hold ssd_chunk_scan_fwd_flow_workspace_size(.., flow, ..) bytes.
+ * For benchmarks and tests that compare the flows.
+ */
+SSD_API ssd_status_t ssd_chunk_scan_fwd_flow_workspace_size(const ssd_dims_t* dims,
+                                                            int chunk_size, ssd_dtype_t dtype,
+                                                            int flow, size_t* bytes);
+SSD_API ssd_status_t ssd_chunk_scan_fwd_with_flow(const void* x, const float* dt, const float* A,
+                                                  const void* B, const void* C, const float* D,
+                                                  int chunk_size, const float* init_states,
+                                                  void* y, float* final_states,
+                                                  const ssd_dims_t* dims, ssd_dtype_t dtype,
+                                                  void* workspace, size_t workspace_bytes,
+                                                  void* stream, int flow);
 
 #ifdef __cplusplus
 }

@@ -125,6 +125,50 @@ __device__ __forceinline__ bool mbar_wait_polls(uint64_t* bar, uint32_t parity, 
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
+// Orders this thread's generic-proxy view of global memory with its later
+// async-proxy (TMA) accesses: data seen through an acquire is then what a
+// TMA load issued afterwards reads.
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// ---------------------------------------------------------------- flags between CTAs
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release_gpu(int* p, int v) {
+    asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ int ld_acquire_cta_smem(const volatile int* p) {
+    int v;
+    asm volatile("ld.acquire.cta.shared::cta.b32 %0, [%1];"
+                 : "=r"(v)
+                 : "r"(smem_u32(const_cast<const int*>(p)))
+                 : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release_cta_smem(volatile int* p, int v) {
+    asm volatile("st.release.cta.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(const_cast<int*>(p))),
+                 "r"(v)
+                 : "memory");
+}
+// Bounded wait until the flag at p (written by another CTA of the same
+// launch with st_release_gpu) is at least v.  Gives up like mbar_wait: after
+// about a second, or at once when another wait of the launch already has.
+__device__ __forceinline__ bool flag_wait_geq(const int* p, int v, const WaitCtx& st) {
+    if (ld_acquire_gpu(p) >= v) return true;
+    const uint64_t t0 = global_ns();
+    for (;;) {
+        __nanosleep(256);
+        if (ld_acquire_gpu(p) >= v) return true;
+        if (*reinterpret_cast<volatile unsigned int*>(st.word) == st.token) return false;
+        if (global_ns() - t0 > kWaitLimitNs) break;
+    }
+    atomicExch(st.word, st.token);
+    return false;
+}
 
 // ---------------------------------------------------------------- TMA (no multicast)
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar,

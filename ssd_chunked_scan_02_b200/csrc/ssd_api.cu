@@ -88,35 +88,65 @@ ssd::Dims forward_dims(const ssd::Dims& d, ssd::Elt t) {
 
 // The forward's data flow for these sizes (decided from the sizes alone, so
 // the workspace size needs no device).
-enum class Flow { Simt = 0, ThreeKernel = 1, Walk = 2 };
+enum class Flow { Simt = 0, ThreeKernel = 1, Walk = 2, Fused = 3 };
 
 Flow pick_flow(const ssd::Dims& d, ssd::Elt t) {
     if (!fwd_tc(d, t)) return Flow::Simt;
-    return ssd::walk_preferred(d) ? Flow::Walk : Flow::ThreeKernel;
+    if (!ssd::walk_preferred(d)) return Flow::ThreeKernel;
+    return ssd::walk_out_preferred(d) ? Flow::Fused : Flow::Walk;
+}
+
+// Whether a data flow covers these sizes (the SIMT kernels cover all).
+bool flow_covers(Flow f, const ssd::Dims& d, ssd::Elt t) {
+    switch (f) {
+        case Flow::Simt: return true;
+        case Flow::ThreeKernel:
+        case Flow::Walk: return fwd_tc(d, t);
+        case Flow::Fused: return fwd_tc(d, t) && ssd::walk_out_supported(d);
+    }
+    return false;
+}
+
+// The forward's sizes and data flow: the library's choice (requested < 0) or
+// the requested SSD_FLOW_* (SSD_ERR_UNSUPPORTED if it does not cover them).
+// The tensor-core flows run bf16 blocks of 128 tokens or more.
+ssd_status_t resolve_flow(ssd::Dims* d, ssd::Elt t, int requested, Flow* f) {
+    if (requested < 0) {
+        *d = forward_dims(*d, t);
+        *f = pick_flow(*d, t);
+        return SSD_OK;
+    }
+    if (requested > (int)Flow::Fused) return fail(SSD_ERR_INVALID_ARG, "unknown data flow %d", requested);
+    *f = static_cast<Flow>(requested);
+    if (*f != Flow::Simt) *d = forward_dims(*d, t);
+    if (!flow_covers(*f, *d, t))
+        return fail(SSD_ERR_UNSUPPORTED, "data flow %d does not cover these sizes", requested);
+    return SSD_OK;
 }
 
 // Workspace regions (each 256-byte aligned).  The three-kernel flows keep the
 // chunk states (fp32) and log-decays; the walk keeps its chunk states on chip
 // and needs only the entering states.
 struct WsLayout {
-    size_t states, logdecay, prev, total;
+    size_t states, logdecay, prev, sched, total;
 };
 
-WsLayout ws_layout(const ssd::Dims& d, ssd::Elt t) {
+WsLayout ws_layout(const ssd::Dims& d, ssd::Elt t, Flow flow) {
     // the tensor-core flows keep 64 state rows for a head of headdim 32
-    const Flow flow = pick_flow(d, t);
     const int64_t rows = flow == Flow::Simt ? d.P : ssd::state_rows(d.P);
     const size_t nstate = (size_t)(d.b * d.T * d.H) * (size_t)(rows * d.N);
     WsLayout w;
     w.states = 0;
-    if (flow == Flow::Walk) {
+    if (flow == Flow::Walk || flow == Flow::Fused) {
         w.logdecay = 0;
         w.prev = 0;
     } else {
         w.logdecay = round_up(nstate * 4, 256);
         w.prev = w.logdecay + round_up((size_t)(d.b * d.T * d.H) * 4, 256);
     }
-    w.total = w.prev + round_up(nstate * elt_size(t), 256);
+    w.sched = w.prev + round_up(nstate * elt_size(t), 256);
+    // the fused flow's ticket counter and walker progress flags
+    w.total = w.sched + (flow == Flow::Fused ? round_up(ssd::walk_out_sched_bytes(d), 256) : 0);
     if (nstate == 0) w.total = 0;
     return w;
 }
@@ -188,15 +218,23 @@ const char* ssd_status_string(ssd_status_t s) {
 
 const char* ssd_last_error_detail(void) { return g_detail; }
 
-ssd_status_t ssd_chunk_scan_fwd_workspace_size(const ssd_dims_t* dims, int chunk_size,
-                                               ssd_dtype_t dtype, size_t* bytes) {
+ssd_status_t ssd_chunk_scan_fwd_flow_workspace_size(const ssd_dims_t* dims, int chunk_size,
+                                                    ssd_dtype_t dtype, int flow, size_t* bytes) {
     g_detail[0] = 0;
     if (!bytes) return fail(SSD_ERR_INVALID_ARG, "bytes is NULL");
     ssd::Dims d{}; ssd::Elt t = ssd::Elt::BF16;
     ssd_status_t st = check_dims(dims, chunk_size, true, dtype, &d, &t);
     if (st != SSD_OK) return st;
-    *bytes = ws_layout(forward_dims(d, t), t).total;
+    Flow f = Flow::Simt;
+    st = resolve_flow(&d, t, flow, &f);
+    if (st != SSD_OK) return st;
+    *bytes = ws_layout(d, t, f).total;
     return SSD_OK;
+}
+
+ssd_status_t ssd_chunk_scan_fwd_workspace_size(const ssd_dims_t* dims, int chunk_size,
+                                               ssd_dtype_t dtype, size_t* bytes) {
+    return ssd_chunk_scan_fwd_flow_workspace_size(dims, chunk_size, dtype, -1, bytes);
 }
 
 int ssd_chunk_scan_fwd_uses_tensor_cores(const ssd_dims_t* dims, int chunk_size,
@@ -210,6 +248,7 @@ int ssd_chunk_scan_fwd_data_flow(const ssd_dims_t* dims, int chunk_size, ssd_dty
     ssd::Dims d{}; ssd::Elt t = ssd::Elt::BF16;
     if (check_dims(dims, chunk_size, true, dtype, &d, &t) != SSD_OK) return -1;
     switch (pick_flow(forward_dims(d, t), t)) {
+        case Flow::Fused: return SSD_FLOW_WALK_OUTPUT_FUSED;
         case Flow::Walk: return SSD_FLOW_WALK_OUTPUT;
         case Flow::ThreeKernel: return SSD_FLOW_TC_THREE_KERNEL;
         default: return SSD_FLOW_SIMT;
@@ -221,11 +260,24 @@ ssd_status_t ssd_chunk_scan_fwd(const void* x, const float* dt, const float* A, 
                                 const float* init_states, void* y, float* final_states,
                                 const ssd_dims_t* dims, ssd_dtype_t dtype, void* workspace,
                                 size_t workspace_bytes, void* stream) {
+    return ssd_chunk_scan_fwd_with_flow(x, dt, A, B, C, D, chunk_size, init_states, y,
+                                        final_states, dims, dtype, workspace, workspace_bytes,
+                                        stream, -1);
+}
+
+ssd_status_t ssd_chunk_scan_fwd_with_flow(const void* x, const float* dt, const float* A,
+                                          const void* B, const void* C, const float* D,
+                                          int chunk_size, const float* init_states, void* y,
+                                          float* final_states, const ssd_dims_t* dims,
+                                          ssd_dtype_t dtype, void* workspace,
+                                          size_t workspace_bytes, void* stream, int flow_req) {
     g_detail[0] = 0;
     ssd::Dims d{}; ssd::Elt t = ssd::Elt::BF16;
     ssd_status_t st = check_dims(dims, chunk_size, true, dtype, &d, &t);
     if (st != SSD_OK) return st;
-    d = forward_dims(d, t);
+    Flow flow = Flow::Simt;
+    st = resolve_flow(&d, t, flow_req, &flow);
+    if (st != SSD_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     OPTIONAL_PTR(init_states);
     OPTIONAL_PTR(final_states);
@@ -237,7 +289,7 @@ ssd_status_t ssd_chunk_scan_fwd(const void* x, const float* dt, const float* A, 
     }
     REQUIRE_PTR(x); REQUIRE_PTR(dt); REQUIRE_PTR(A); REQUIRE_PTR(B); REQUIRE_PTR(C);
     REQUIRE_PTR(D); REQUIRE_PTR(y);
-    const WsLayout w = ws_layout(d, t);
+    const WsLayout w = ws_layout(d, t, flow);
     if (workspace_bytes < w.total)
         return fail(SSD_ERR_INVALID_ARG, "workspace too small: %zu bytes given, %zu needed",
                     workspace_bytes, w.total);
@@ -250,7 +302,12 @@ ssd_status_t ssd_chunk_scan_fwd(const void* x, const float* dt, const float* A, 
     void* prev = ws + w.prev;
 
     cudaError_t e;
-    const Flow flow = pick_flow(d, t);
+    if (flow == Flow::Fused) {
+        e = ssd::launch_walk_out_tc(x, dt, A, B, C, D, init_states, prev, y, final_states,
+                                    reinterpret_cast<int*>(ws + w.sched), d, s);
+        if (e != cudaSuccess) return cuda_fail(e, "walk + output kernel (tcgen05)");
+        return SSD_OK;
+    }
     if (flow == Flow::Walk) {
         e = ssd::launch_state_walk_tc(x, dt, A, B, init_states, prev, final_states, d, s);
         if (e != cudaSuccess) return cuda_fail(e, "state-walk kernel (tcgen05)");

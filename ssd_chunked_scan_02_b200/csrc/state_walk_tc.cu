@@ -1,46 +1,22 @@
-// state_walk_tc.cu -- chunk states and the inter-chunk recurrence in one pass
-// (steps a0 + a2 + a3 of the block-decomposed SSD forward, bf16 inputs):
-//
-//   h_{-1} = init (or 0);  for each chunk c:  prev_c = h_{c-1}   (written, bf16)
-//                                            h_c = exp(cs_last) h_{c-1} + S_c
-//   S_c = sum_j (exp(cs_last - cs_j) dt_j x_j) B_j^T   (tensor cores, fp32 accumulation)
+// state_walk_tc.cu -- the standalone walk kernel: chunk states and the
+// inter-chunk recurrence in one pass (steps a0 + a2 + a3 of the
+// block-decomposed SSD forward, bf16 inputs), one CTA per (batch, head pair
+// of one group) walking the chunks in order (the walker is in
+// state_walk_body.cuh).  Heads are the kernels' virtual heads of headdim 64
+// (a head of headdim 64 k is k of them); a group with an odd number of heads
+// pairs its last head with a zero phantom.  Sized for two CTAs per SM (about
+// 105 KB of shared memory and 256 or 128 TMEM columns each).
 //
 // "论文解读：Mamba: ...", 状态空间模型: the linear-recurrence form, taken one
 // chunk per step; "Transformers are SSMs" (CiteArk), AI research summary: the
 // chunk's contribution is one dense contraction.
-//
-// One CTA per (batch, head pair of one group) walks the chunks in order; S_c
-// never leaves the chip.  Heads are the kernels' virtual heads of headdim 64
-// (a head of headdim 64 k is k of them); a group with an odd number of heads
-// pairs its last head with a zero phantom.  Tensor memory holds two fp32 tiles: the running state h and the
-// chunk's accumulator S.  The MMAs of chunk c write S from zero; the
-// epilogue warps then read h and S, form h' = exp(cs_last) h + S, store h'
-// back over h and write it out as the state entering chunk c + 1 (bf16), or
-// as the final state (fp32) after the last chunk.  The MMAs of chunk c + 1
-// wait only until the epilogue has read S, not for its stores, so the loads,
-// scaling and MMAs of the next chunk stream while the epilogue works.
-//
-// With dstate N = 128 the MMA forms S^T (M = 128 state rows n, N = two heads x
-// P = 64), so a TMEM lane is a state column and a warp's prev/final stores are
-// contiguous along n; with N = 64 it forms S (M = two heads x P rows, N = 64),
-// a lane is a (head, p) row.  x and B come by TMA in 64-token sub-steps
-// through a three-entry ring; x rows are scaled in place by the decay
-// weights w_j = exp(cs_last - cs_j) dt_j before the MMA reads them.  Sized
-// for two CTAs per SM (about 105 KB of shared memory and 256 or 128 TMEM
-// columns each).
-//
-// Roles (320 threads): warps 0-3 dt prefix sums (warp = (head, half of the
-// chunk)) and x scaling (warp w scales rows 32 w .. 32 w + 31 of each ring
-// entry and reports them by its own arrival); warps 4-7 state epilogue;
-// warp 8 TMA producer; warp 9 MMA issuer and TMEM owner.  Every wait is
-// bounded; a warpgroup leaves its loop only when all its threads agree
-// (bar.red.or).
 #include <cuda.h>
 #include <cuda_bf16.h>
 
 #include "common.cuh"
 #include "sm100.cuh"
 #include "ssd_internal.h"
+#include "state_walk_body.cuh"
 #include "tc_host.h"
 #include "tc_kernels.h"
 
@@ -48,45 +24,7 @@ namespace ssd {
 namespace {
 using namespace sm100;
 
-constexpr int kThreads = 320;
-constexpr int kSub = 64;                 // tokens per ring entry
-
-template <int Q, int N>
-struct WalkSmem {
-    // ring entries of 64 tokens (32 KB for N = 128, 24 KB for N = 64)
-    static constexpr int kStages = 3;
-    // one chunk accumulator: the next chunk's MMAs wait only until the
-    // epilogue has read it (two measured no faster for N = 64)
-    static constexpr int kSSlots = 1;
-    static constexpr int kXPart = 2 * kSub * 128;          // two heads x 64 rows x 128 B
-    static constexpr int kBPart = (N / 64) * kSub * 128;   // N/64 blocks x 64 rows x 128 B
-    static constexpr int kEntry = kXPart + kBPart;
-    static constexpr int kRing = 0;
-    static constexpr int kW = kRing + kStages * kEntry;    // float [2 buf][2 heads][Q]: w_j
-    static constexpr int kA = kW + 2 * 2 * Q * 4;          // float [2 buf][2]: chunk decays
-    static constexpr int kSeg = kA + 16;                   // float [2 buf][4]: segment sums
-    static constexpr int kBar = kSeg + 32;
-    static constexpr int kTmem = kBar + 24 * 8;
-    static constexpr int kFlags = kTmem + 16;
-    static constexpr int kTotal = kFlags + 16;
-    static constexpr int kAlloc = kTotal + 1024;
-    // TMEM: the running state h, then the chunk accumulator(s) S
-    static constexpr uint32_t kCols = (N == 128) ? 128 : 64;   // columns of one tile
-    static constexpr uint32_t kColH = 0;
-    static constexpr uint32_t kColS = kCols;
-    static constexpr uint32_t kTmemCols = 2 * kCols;
-};
-
-enum {
-    BAR_FULL = 0,        // 4: ring entry loaded (TMA transaction count)
-    BAR_EMPTY = 4,       // 4: ring entry read by the MMAs
-    BAR_SCALED = 8,      // 4: ring entry's x rows scaled (4 warp arrivals)
-    BAR_AREADY = 12,     // 2: chunk decays of buffer cb published
-    BAR_AFREE = 14,      // 2: the epilogue has read buffer cb's decays
-    BAR_SFULL = 16,      // 2: the chunk's MMAs into accumulator slot s have completed
-    BAR_SEMPTY = 18,     // 2: the epilogue has read accumulator slot s
-    BAR_COUNT = 20
-};
+constexpr int kThreads = walk::Roles<2>::kThreads;
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
     return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
@@ -99,396 +37,26 @@ state_walk_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
                      const float* __restrict__ init, __nv_bfloat16* __restrict__ prev,
                      float* __restrict__ fin, int64_t L, int H, int G, int64_t T,
                      int ksplit, int pcols, WaitCtx status) {
-    using S = WalkSmem<Q, N>;
-    constexpr bool kTrans = (N == 128);
-    constexpr int kNSub = Q / kSub;
-    constexpr int kStages = S::kStages;
-    constexpr int kSSlots = S::kSSlots;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    // H counts virtual heads (headdim 64); real head = virtual head / ksplit
     const HeadPairs hp(H, G);
     const int64_t b = blockIdx.x / (G * hp.per_group());
     int g, h0;
     bool has1;
     hp.map((int)(blockIdx.x % (G * hp.per_group())), &g, &h0, &has1);
-    const int Hr = H / ksplit;
-    const int h1x = has1 ? h0 + 1 : H;       // the phantom's x is read out of range: zeros
-
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = align1024(smem_raw);
-    uint8_t* ring = smem + S::kRing;
-    float* s_w = reinterpret_cast<float*>(smem + S::kW);
-    float* s_a = reinterpret_cast<float*>(smem + S::kA);
-    float* s_seg = reinterpret_cast<float*>(smem + S::kSeg);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::kBar);
-    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + S::kTmem);
-    volatile int* s_flag = reinterpret_cast<volatile int*>(smem + S::kFlags);
-
-    if (tid == 0) {
-        for (int i = 0; i < BAR_COUNT; ++i)
-            mbar_init(&bars[i], (i >= BAR_SCALED && i < BAR_SCALED + kStages) ? 4 : 1);
-        s_flag[0] = 0;
-        fence_mbar_init();
-    }
-    if (warp == 9) {
-        tmem_alloc(s_tmem, S::kTmemCols);
-        tmem_relinquish();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = *s_tmem;
-    const int64_t nsteps = T * kNSub;
-
-    if (warp == 8) {
-        // ================================================== TMA producer
-        if (lane == 0) {
-            prefetch_tmap(&tmX);
-            prefetch_tmap(&tmB);
-            bool ok = true;
-            for (int64_t si = 0; si < nsteps && ok; ++si) {
-                const int e = (int)(si % kStages);
-                const int64_t u = si / kStages;
-                if (u >= 1) ok = mbar_wait(&bars[BAR_EMPTY + e], (uint32_t)((u - 1) & 1), status);
-                if (!ok) break;
-                const int row = (int)((si / kNSub) * Q + (si % kNSub) * kSub);
-                uint8_t* ent = ring + e * S::kEntry;
-                mbar_expect_tx(&bars[BAR_FULL + e], S::kEntry);
-                tma_load_4d(ent, &tmX, &bars[BAR_FULL + e], 0, h0, row, (int)b);
-                tma_load_4d(ent + kSub * 128, &tmX, &bars[BAR_FULL + e], 0, h1x, row, (int)b);
-                for (int nb = 0; nb < N / 64; ++nb)
-                    tma_load_4d(ent + S::kXPart + nb * kSub * 128, &tmB, &bars[BAR_FULL + e],
-                                nb * 64, g, row, (int)b);
-            }
-            if (!ok) s_flag[0] = 1;
-        }
-    } else if (warp == 9) {
-        // ================================================== MMA issuer
-        if (lane == 0) {
-            // N = 128: S^T (M = 128 state rows, N = 128 pair columns) = B^T (w x)
-            // N = 64:  S   (M = 128 pair rows,  N = 64 state columns) = (w x)^T B
-            constexpr uint32_t kIdesc = idesc_bf16_f32(128, kTrans ? 128 : N, true, true);
-            bool ok = true;
-            int64_t si = 0;
-            for (int64_t c = 0; c < T && ok; ++c) {
-                // accumulator slot sl is free once the epilogue has read the S of
-                // chunk c - kSSlots
-                const int sl = (int)(c % kSSlots);
-                const uint32_t dS = tmem + S::kColS + sl * S::kCols;
-                if (c >= kSSlots)
-                    ok = mbar_wait(&bars[BAR_SEMPTY + sl], (uint32_t)(((c / kSSlots) - 1) & 1), status);
-                for (int sub = 0; sub < kNSub && ok; ++sub, ++si) {
-                    const int e = (int)(si % kStages);
-                    const int64_t u = si / kStages;
-                    ok = mbar_wait(&bars[BAR_SCALED + e], (uint32_t)(u & 1), status);
-                    if (!ok) break;
-                    tc_fence_after();
-                    const uint32_t x0 = smem_u32(ring + e * S::kEntry);
-                    const uint32_t b0 = x0 + S::kXPart;
-#pragma unroll
-                    for (int ks = 0; ks < kSub / 16; ++ks) {
-                        // x pair: two 64-column atoms (heads) 8 KB apart; B: 64-column
-                        // atoms of dstate 8 KB apart; 8-row groups 1024 B apart.
-                        const uint64_t xd = smem_desc_sw128(x0 + ks * 2048, kSub * 128, 1024);
-                        const uint64_t bd = smem_desc_sw128(b0 + ks * 2048, kSub * 128, 1024);
-                        const bool acc = (sub | ks) != 0;
-                        if (kTrans) mma_ss(dS, bd, xd, kIdesc, acc);
-                        else mma_ss(dS, xd, bd, kIdesc, acc);
-                    }
-                    mma_commit(&bars[BAR_EMPTY + e]);
-                }
-                if (ok) mma_commit(&bars[BAR_SFULL + sl]);
-            }
-            if (!ok) s_flag[0] = 1;
-        }
-    } else if (warp < 4) {
-        // ================================================== dt prefix sums and x scaling
-        // Warp w: head hk = w / 2 of the pair, half sg = w % 2 of the chunk; lane
-        // holds kPer consecutive tokens' dt, loaded one chunk ahead.
-        constexpr int kPer = Q / 64;
-        constexpr int kHalf = Q / 2;
-        const int hk = warp >> 1, sg = warp & 1;
-        const bool real = hk == 0 || has1;
-        const float Ak = real ? A[(h0 + hk) / ksplit] : 0.f;
-        float dreg[kPer];
-        auto load_dt = [&](int64_t c) {
-#pragma unroll
-            for (int k = 0; k < kPer; ++k) {
-                const int64_t tok = c * Q + sg * kHalf + lane * kPer + k;
-                dreg[k] = (real && tok < L) ? dt[(b * L + tok) * Hr + (h0 + hk) / ksplit] : 0.f;
-            }
-        };
-        // w_j and the chunk decay of this head into buffer buf
-        auto prefix = [&](int buf) {
-            float v[kPer];
-            float run = 0.f;                       // tokens past the sequence end add 0
-#pragma unroll
-            for (int k = 0; k < kPer; ++k) {
-                run += dreg[k] * Ak;
-                v[k] = run;
-            }
-            float incl = run;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const float uu = __shfl_up_sync(0xffffffffu, incl, o);
-                if (lane >= o) incl += uu;
-            }
-            if (lane == 31) s_seg[buf * 4 + warp] = incl;
-            named_bar_sync(1, 128);
-            const float s0 = s_seg[buf * 4 + hk * 2], s1 = s_seg[buf * 4 + hk * 2 + 1];
-            const float off = (incl - run) + (sg ? s0 : 0.f);
-            const float last = s0 + s1;
-            float* wk = s_w + (buf * 2 + hk) * Q + sg * kHalf + lane * kPer;
-#pragma unroll
-            for (int k = 0; k < kPer; ++k) wk[k] = expf(last - (v[k] + off)) * dreg[k];
-            if (sg == 0 && lane == 0) s_a[buf * 2 + hk] = expf(last);
-        };
-        bool fail = false;
-        int64_t si = 0;
-        load_dt(0);
-        for (int64_t c = 0; c < T; ++c) {
-            const int cb = (int)(c & 1);
-            // buffer cb is free once the epilogue has read chunk c-2's decays
-            if (!fail && c >= 2)
-                fail = !mbar_wait(&bars[BAR_AFREE + cb], (uint32_t)(((c >> 1) - 1) & 1), status);
-            prefix(cb);
-            if (c + 1 < T) load_dt(c + 1);
-            // publishes w_j and the decays, and shares every thread's verdict
-            if (named_bar_or(1, 128, fail)) {
-                fail = true;
-                break;
-            }
-            if (tid == 0) mbar_arrive(&bars[BAR_AREADY + cb]);
-            const float* wb = s_w + cb * 2 * Q;
-            for (int sub = 0; sub < kNSub; ++sub, ++si) {
-                const int e = (int)(si % kStages);
-                const int64_t u = si / kStages;
-                const bool ok = mbar_wait(&bars[BAR_FULL + e], (uint32_t)(u & 1), status);
-                if (__any_sync(0xffffffffu, !ok)) {
-                    fail = true;                      // shared at the next chunk's barrier
-                    break;
-                }
-                // row tid of the entry: head tid / 64, token sub * 64 + tid % 64; its
-                // 16-byte chunks are visited in a per-row rotated order (bank-conflict free)
-                const int k = tid >> 6, jl = tid & 63;
-                const float wj = wb[k * Q + sub * kSub + jl];
-                uint4* row = reinterpret_cast<uint4*>(ring + e * S::kEntry + k * kSub * 128 + jl * 128);
-                uint4 v[8];
-#pragma unroll
-                for (int q = 0; q < 8; ++q) v[q] = row[q ^ (jl & 7)];
-#pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    uint32_t* uw = reinterpret_cast<uint32_t*>(&v[q]);
-#pragma unroll
-                    for (int ee = 0; ee < 4; ++ee) {
-                        const float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&uw[ee]));
-                        uw[ee] = pack_bf16x2(f.x * wj, f.y * wj);
-                    }
-                    row[q ^ (jl & 7)] = v[q];
-                }
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&bars[BAR_SCALED + e]);
-            }
-        }
-        if (fail) s_flag[0] = 1;
-    } else {
-        // ================================================== state epilogue (warps 4-7)
-        const int m = tid - 128;                       // TMEM lane
-        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-        const uint32_t tH = tmem + lane_base + S::kColH;
-        bool fail = false;
-        // h_{-1} = init (or zero): into the state tile, and out as chunk 0's entering state
-        if (kTrans) {
-            // lane m = state column n; TMEM column cc*32+e = (head cc/2, p = (cc&1)*32 + e)
-            const int n = m;
-#pragma unroll 1
-            for (int cc = 0; cc < 4; ++cc) {
-                const int k = cc >> 1, p0 = (cc & 1) * 32;
-                // init: (b, H, pcols, N), pcols = 64 or 32 (rows pcols .. 63 zero)
-                const int64_t srow = ((b * H + h0 + k) * pcols + p0) * (int64_t)N + n;
-                const bool real = k == 0 || has1;
-                const bool rows = init && real && p0 < pcols;
-                uint32_t r[32];
-#pragma unroll
-                for (int e = 0; e < 32; ++e)
-                    r[e] = __float_as_uint(rows ? init[srow + (int64_t)e * N] : 0.f);
-                if (real) {
-                    __nv_bfloat16* pr = prev + (((b * T) * H + h0 + k) * 64 + p0) * (int64_t)N + n;
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) pr[(int64_t)e * N] = __float2bfloat16_rn(__uint_as_float(r[e]));
-                }
-                uint32_t lo[16], hi[16];
-#pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    lo[e] = r[e];
-                    hi[e] = r[16 + e];
-                }
-                tmem_st16(tH + cc * 32, lo);
-                tmem_st16(tH + cc * 32 + 16, hi);
-            }
-        } else {
-            // lane m = (head m / 64, p = m % 64); TMEM columns = state n (N = 64)
-            const int k = m >> 6, p = m & 63;
-            const bool real = k == 0 || has1;
-            const int64_t srow = ((b * H + h0 + k) * pcols + p) * (int64_t)N;
-#pragma unroll 1
-            for (int cc = 0; cc < N / 32; ++cc) {
-                uint32_t r[32];
-                if (init && real && p < pcols) {
-                    const float4* s4 = reinterpret_cast<const float4*>(init + srow + cc * 32);
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        const float4 f = s4[q];
-                        r[4 * q] = __float_as_uint(f.x);
-                        r[4 * q + 1] = __float_as_uint(f.y);
-                        r[4 * q + 2] = __float_as_uint(f.z);
-                        r[4 * q + 3] = __float_as_uint(f.w);
-                    }
-                } else {
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) r[e] = 0u;
-                }
-                __nv_bfloat16* pr = prev + (((b * T) * H + h0 + k) * 64 + p) * (int64_t)N + cc * 32;
-#pragma unroll
-                for (int e = 0; e < 32 && real; e += 8) {
-                    uint4 v;
-                    v.x = pack_bf16x2(__uint_as_float(r[e]), __uint_as_float(r[e + 1]));
-                    v.y = pack_bf16x2(__uint_as_float(r[e + 2]), __uint_as_float(r[e + 3]));
-                    v.z = pack_bf16x2(__uint_as_float(r[e + 4]), __uint_as_float(r[e + 5]));
-                    v.w = pack_bf16x2(__uint_as_float(r[e + 6]), __uint_as_float(r[e + 7]));
-                    *reinterpret_cast<uint4*>(pr + e) = v;
-                }
-                uint32_t lo[16], hi[16];
-#pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    lo[e] = r[e];
-                    hi[e] = r[16 + e];
-                }
-                tmem_st16(tH + cc * 32, lo);
-                tmem_st16(tH + cc * 32 + 16, hi);
-            }
-        }
-
-        for (int64_t c = 0; c < T; ++c) {
-            const int cb = (int)(c & 1);
-            const int sl = (int)(c % kSSlots);
-            const uint32_t tS = tmem + lane_base + S::kColS + sl * S::kCols;
-            fail = !mbar_wait(&bars[BAR_AREADY + cb], (uint32_t)((c >> 1) & 1), status) ||
-                   !mbar_wait(&bars[BAR_SFULL + sl], (uint32_t)((c / kSSlots) & 1), status);
-            if (named_bar_or(2, 128, fail)) {
-                fail = true;
-                break;
-            }
-            tc_fence_after();
-            const float a0 = s_a[cb * 2 + 0], a1 = s_a[cb * 2 + 1];
-            named_bar_sync(2, 128);
-            if (m == 0) mbar_arrive(&bars[BAR_AFREE + cb]);
-            // pass 1: h' = a h + S in TMEM (h' over h); then S is free for the next chunk
-            {
-                const int nk = kTrans ? 4 : N / 32;
-#pragma unroll 1
-                for (int cc = 0; cc < nk; ++cc) {
-                    const int k = kTrans ? (cc >> 1) : (m >> 6);
-                    const float a = k ? a1 : a0;
-                    uint32_t hr[32], sr[32];
-                    tmem_ld32x2(tH + cc * 32, tS + cc * 32, hr, sr);
-                    uint32_t lo[16], hi[16];
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        lo[e] = __float_as_uint(fmaf(a, __uint_as_float(hr[e]), __uint_as_float(sr[e])));
-                        hi[e] = __float_as_uint(
-                            fmaf(a, __uint_as_float(hr[16 + e]), __uint_as_float(sr[16 + e])));
-                    }
-                    tmem_st16(tH + cc * 32, lo);
-                    tmem_st16(tH + cc * 32 + 16, hi);
-                }
-            }
-            tc_fence_before();
-            named_bar_sync(2, 128);
-            if (m == 0) mbar_arrive(&bars[BAR_SEMPTY + sl]);
-            // pass 2: h' out, as the state entering chunk c + 1 (bf16) or the final state
-            const bool last = (c + 1 == T);
-            if (last && !fin) continue;
-            if (kTrans) {
-                const int n = m;
-#pragma unroll 1
-                for (int cc = 0; cc < 4; ++cc) {
-                    const int k = cc >> 1, p0 = (cc & 1) * 32;
-                    if (k == 1 && !has1) break;       // the phantom's state is not written
-                    uint32_t hr[32];
-                    tmem_ld32(tH + cc * 32, hr);
-                    if (!last) {
-                        __nv_bfloat16* pr =
-                            prev + (((b * T + c + 1) * H + h0 + k) * 64 + p0) * (int64_t)N + n;
-#pragma unroll
-                        for (int e = 0; e < 32; ++e)
-                            pr[(int64_t)e * N] = __float2bfloat16_rn(__uint_as_float(hr[e]));
-                    } else if (p0 < pcols) {
-                        float* fp = fin + ((b * H + h0 + k) * pcols + p0) * (int64_t)N + n;
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) fp[(int64_t)e * N] = __uint_as_float(hr[e]);
-                    }
-                }
-            } else {
-                const int k = m >> 6, p = m & 63;
-                const bool real = k == 0 || has1;
-#pragma unroll 1
-                for (int cc = 0; cc < N / 32; ++cc) {
-                    uint32_t hr[32];
-                    tmem_ld32(tH + cc * 32, hr);
-                    if (!real) continue;                  // the phantom's state is not written
-                    if (!last) {
-                        __nv_bfloat16* pr =
-                            prev + (((b * T + c + 1) * H + h0 + k) * 64 + p) * (int64_t)N + cc * 32;
-#pragma unroll
-                        for (int e = 0; e < 32; e += 8) {
-                            uint4 v;
-                            v.x = pack_bf16x2(__uint_as_float(hr[e]), __uint_as_float(hr[e + 1]));
-                            v.y = pack_bf16x2(__uint_as_float(hr[e + 2]), __uint_as_float(hr[e + 3]));
-                            v.z = pack_bf16x2(__uint_as_float(hr[e + 4]), __uint_as_float(hr[e + 5]));
-                            v.w = pack_bf16x2(__uint_as_float(hr[e + 6]), __uint_as_float(hr[e + 7]));
-                            *reinterpret_cast<uint4*>(pr + e) = v;
-                        }
-                    } else if (p < pcols) {
-                        float4* f4 = reinterpret_cast<float4*>(
-                            fin + ((b * H + h0 + k) * pcols + p) * (int64_t)N + cc * 32);
-#pragma unroll
-                        for (int q = 0; q < 8; ++q)
-                            f4[q] = make_float4(__uint_as_float(hr[4 * q]), __uint_as_float(hr[4 * q + 1]),
-                                                __uint_as_float(hr[4 * q + 2]), __uint_as_float(hr[4 * q + 3]));
-                    }
-                }
-            }
-        }
-        if (fail) s_flag[0] = 1;
-    }
-
-    tc_fence_before();
-    __syncthreads();
-    if (s_flag[0] && tid == 8 * 32) {
-        // A wait gave up somewhere: give outstanding TMA loads and MMAs a last
-        // (bounded) chance to land before the shared memory and TMEM go away.
-        for (int k = 0; k < kStages; ++k) mbar_wait(&bars[BAR_FULL + k], 0, status);
-        for (int k = 0; k < kSSlots; ++k) mbar_wait(&bars[BAR_SFULL + k], 0, status);
-    }
-    __syncthreads();
-    if (warp == 9) {
-        tc_fence_after();
-        tmem_dealloc(tmem, S::kTmemCols);
-    }
+    walk::body<Q, N, 2>(&tmX, &tmB, dt, A, init, prev, fin, L, H, G, T, ksplit, pcols, b, g, h0,
+                        has1 ? 2 : 1, align1024(smem_raw), nullptr, status);
 }
 
 template <int Q, int N>
 cudaError_t launch_impl(const void* x, const float* dt, const float* A, const void* B,
                         const float* init, void* prev, float* fin, const Dims& d, int ksplit,
                         int pc, cudaStream_t s) {
-    using S = WalkSmem<Q, N>;
+    using S = walk::Smem<Q, N, 2>;
     CUtensorMap tmX, tmB;
     // x: pc columns a (virtual) head; a 64-column box reads zeros past them
     const uint64_t xdims[4] = {(uint64_t)pc, (uint64_t)d.H, (uint64_t)d.L, (uint64_t)d.b};
     const uint64_t xstr[3] = {(uint64_t)pc * 2, (uint64_t)(d.H * pc * 2), (uint64_t)(d.L * d.H * pc * 2)};
-    const uint32_t box[4] = {64, 1, kSub, 1};
+    const uint32_t box[4] = {64, 1, walk::kSub, 1};
     cudaError_t e = make_tmap_bf16(&tmX, x, 4, xdims, xstr, box);
     if (e != cudaSuccess) return e;
     const uint64_t bdims[4] = {(uint64_t)N, (uint64_t)d.G, (uint64_t)d.L, (uint64_t)d.b};

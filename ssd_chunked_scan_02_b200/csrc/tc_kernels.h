@@ -64,6 +64,20 @@ cudaError_t launch_state_walk_tc(const void* x, const float* dt, const float* A,
 // True when the forward runs the walk: enough (batch, head pair) walkers.
 bool walk_preferred(const Dims& d);
 
+// The whole forward in one launch (walkers of four heads and output tiles
+// side by side; walk_out_tc.cu): dstate 128, chunk 128 or 256, heads per
+// group a multiple of 4 (virtual heads).  `sched` is device scratch of
+// walk_out_sched_bytes(d) bytes (zeroed by the launcher on `s`); prev as for
+// the walk.
+bool walk_out_supported(const Dims& d);
+// ... and the forward takes it (enough chunks for the overlap to pay).
+bool walk_out_preferred(const Dims& d);
+size_t walk_out_sched_bytes(const Dims& d);
+cudaError_t launch_walk_out_tc(const void* x, const float* dt, const float* A, const void* B,
+                               const void* C, const float* D, const float* init, void* prev,
+                               void* y, float* final_states, int* sched, const Dims& d,
+                               cudaStream_t s);
+
 cudaError_t launch_chunk_out_tc(const void* x, const float* dt, const float* A, const void* B,
                                 const void* C, const float* D, const void* prev, void* y,
                                 const Dims& d, cudaStream_t s);

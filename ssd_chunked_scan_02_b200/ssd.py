@@ -29,10 +29,11 @@ EXPORTED = ("ssd_status_string", "ssd_last_error_detail", "ssd_chunk_scan_fwd_wo
             "ssd_chunk_scan_fwd_noalloc", "ssd_poll_device_status", "ssd_state_walk_fwd",
             "ssd_debug_expire_wait", "ssd_chunk_scan_bwd_workspace_size", "ssd_chunk_scan_bwd",
             "ssd_chunk_scan_fwd_data_flow", "ssd_seq_logdecay", "ssd_state_exchange_combine",
-            "ssd_state_correction_workspace_size", "ssd_state_correction_fwd")
+            "ssd_state_correction_workspace_size", "ssd_state_correction_fwd",
+            "ssd_chunk_scan_fwd_flow_workspace_size", "ssd_chunk_scan_fwd_with_flow")
 
 # ssd_chunk_scan_fwd_data_flow results
-SSD_FLOW_SIMT, SSD_FLOW_TC_THREE_KERNEL, SSD_FLOW_WALK_OUTPUT = 0, 1, 2
+SSD_FLOW_SIMT, SSD_FLOW_TC_THREE_KERNEL, SSD_FLOW_WALK_OUTPUT, SSD_FLOW_WALK_OUTPUT_FUSED = 0, 1, 2, 3
 
 
 class SSDError(RuntimeError):
@@ -77,6 +78,12 @@ def load(path: str = LIB_PATH):
     lib.ssd_chunk_scan_fwd.restype = ctypes.c_int
     lib.ssd_chunk_scan_fwd.argtypes = [_vp] * 6 + [ctypes.c_int, _vp, _vp, _vp, dims_p,
                                                    ctypes.c_int, _vp, ctypes.c_size_t, _vp]
+    lib.ssd_chunk_scan_fwd_flow_workspace_size.restype = ctypes.c_int
+    lib.ssd_chunk_scan_fwd_flow_workspace_size.argtypes = [dims_p, ctypes.c_int, ctypes.c_int,
+                                                           ctypes.c_int,
+                                                           ctypes.POINTER(ctypes.c_size_t)]
+    lib.ssd_chunk_scan_fwd_with_flow.restype = ctypes.c_int
+    lib.ssd_chunk_scan_fwd_with_flow.argtypes = lib.ssd_chunk_scan_fwd.argtypes + [ctypes.c_int]
     lib.ssd_chunk_scan_fwd_noalloc.restype = ctypes.c_int
     lib.ssd_chunk_scan_fwd_noalloc.argtypes = [_vp] * 6 + [ctypes.c_int, _vp, _vp, _vp, dims_p,
                                                            ctypes.c_int, _vp]
@@ -204,10 +211,12 @@ def _fwd_dims(x, B) -> ssd_dims_t:
     return make_dims(b, L, H, P, N, G)
 
 
-def ssd_chunk_scan_fwd_workspace_size(dims: ssd_dims_t, chunk_size: int, dtype: torch.dtype) -> int:
+def ssd_chunk_scan_fwd_workspace_size(dims: ssd_dims_t, chunk_size: int, dtype: torch.dtype,
+                                      flow=None) -> int:
     n = ctypes.c_size_t(0)
-    _check(load().ssd_chunk_scan_fwd_workspace_size(ctypes.byref(dims), int(chunk_size),
-                                                    _dtype_code(dtype), ctypes.byref(n)),
+    fl = -1 if flow is None else int(flow)
+    _check(load().ssd_chunk_scan_fwd_flow_workspace_size(ctypes.byref(dims), int(chunk_size),
+                                                         _dtype_code(dtype), fl, ctypes.byref(n)),
            "ssd_chunk_scan_fwd_workspace_size")
     return int(n.value)
 
@@ -219,15 +228,18 @@ def ssd_chunk_scan_fwd_uses_tensor_cores(dims: ssd_dims_t, chunk_size: int,
 
 
 def ssd_chunk_scan_fwd_data_flow(dims: ssd_dims_t, chunk_size: int, dtype: torch.dtype) -> int:
-    """SSD_FLOW_WALK_OUTPUT, SSD_FLOW_TC_THREE_KERNEL, SSD_FLOW_SIMT or -1 (rejected)."""
+    """SSD_FLOW_WALK_OUTPUT_FUSED, SSD_FLOW_WALK_OUTPUT, SSD_FLOW_TC_THREE_KERNEL,
+    SSD_FLOW_SIMT or -1 (rejected)."""
     return int(load().ssd_chunk_scan_fwd_data_flow(ctypes.byref(dims), int(chunk_size),
                                                    _dtype_code(dtype)))
 
 
 def ssd_chunk_scan_fwd(x, dt, A, B, C, D, chunk_size: int, init_states=None,
                        return_final_states: bool = False, y=None, final_states=None,
-                       workspace=None, stream=None):
-    """y (b,L,H,P) [, final_states (b,H,P,N) fp32] for the whole sequences."""
+                       workspace=None, stream=None, flow=None):
+    """y (b,L,H,P) [, final_states (b,H,P,N) fp32] for the whole sequences.
+    ``flow``: an SSD_FLOW_* value to force that data flow (None: the
+    library's choice)."""
     dev = _check_fwd_args(x, dt, A, B, C, D, init_states, y, final_states)
     dims = _fwd_dims(x, B)
     if y is None:
@@ -235,15 +247,15 @@ def ssd_chunk_scan_fwd(x, dt, A, B, C, D, chunk_size: int, init_states=None,
     if return_final_states and final_states is None:
         final_states = torch.empty((x.shape[0], x.shape[2], x.shape[3], B.shape[3]),
                                    device=x.device, dtype=torch.float32)
-    need = ssd_chunk_scan_fwd_workspace_size(dims, chunk_size, x.dtype)
+    fl = -1 if flow is None else int(flow)
+    need = ssd_chunk_scan_fwd_workspace_size(dims, chunk_size, x.dtype, flow=flow)
     if workspace is None:
         workspace = torch.empty(max(need, 16), device=x.device, dtype=torch.uint8)
     with torch.cuda.device(dev):
-        st = load().ssd_chunk_scan_fwd(_ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
-                                       int(chunk_size), _ptr(init_states), _ptr(y),
-                                       _ptr(final_states), ctypes.byref(dims),
-                                       _dtype_code(x.dtype), _ptr(workspace), workspace.numel(),
-                                       _stream(stream, dev))
+        st = load().ssd_chunk_scan_fwd_with_flow(
+            _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D), int(chunk_size),
+            _ptr(init_states), _ptr(y), _ptr(final_states), ctypes.byref(dims),
+            _dtype_code(x.dtype), _ptr(workspace), workspace.numel(), _stream(stream, dev), fl)
     _check(st, "ssd_chunk_scan_fwd")
     return (y, final_states) if (return_final_states or final_states is not None) else y
 

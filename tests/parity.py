@@ -39,11 +39,13 @@ def to_dev(inp: dict, device="cuda") -> dict:
     return {k: (v.to(device) if v is not None else None) for k, v in inp.items()}
 
 
-def gpu_fwd(inp: dict, chunk: int, want_final=True):
-    """CUDA path; returns (y float64 numpy on host, final or None)."""
+def gpu_fwd(inp: dict, chunk: int, want_final=True, flow=None):
+    """CUDA path (the library's data flow, or the SSD_FLOW_* given); returns
+    (y float64 numpy on host, final or None)."""
     d = to_dev(inp)
     out = ssd.ssd_chunk_scan_fwd(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], chunk,
-                                 init_states=d["init"], return_final_states=want_final)
+                                 init_states=d["init"], return_final_states=want_final,
+                                 flow=flow)
     torch.cuda.synchronize()
     if want_final:
         y, f = out

@@ -58,6 +58,9 @@ def _round(v):
 
 @pytest.mark.parametrize("b,L,H,P,N,G,Q,dt", [
     (4, 8192, 80, 64, 128, 1, 256, ssd.SSD_BF16),
+    (8, 2048, 24, 64, 128, 1, 128, ssd.SSD_BF16),   # one launch, 128-token chunks
+    (4, 8192, 40, 128, 128, 1, 256, ssd.SSD_BF16),  # one launch, headdim 128
+    (1024, 512, 32, 64, 64, 1, 256, ssd.SSD_BF16),  # walk + output (dstate 64)
     (1, 256, 4, 16, 16, 1, 64, ssd.SSD_F32),
     (2, 600, 4, 64, 128, 2, 128, ssd.SSD_BF16),   # ragged: 5 chunks, last one partial
     (3, 1, 2, 3, 5, 1, 16, ssd.SSD_F32),
@@ -75,29 +78,36 @@ def test_workspace_size_formula(lib, b, L, H, P, N, G, Q, dt):
     elt = 4 if dt == ssd.SSD_F32 else 2
     # the tensor-core flows keep 64 state rows for a head of headdim 32
     ns = b * T * H * (max(P, 64) if tc else P) * N
-    if lib.ssd_chunk_scan_fwd_data_flow(ctypes.byref(dims), Q, dt) == ssd.SSD_FLOW_WALK_OUTPUT:
+    flow = lib.ssd_chunk_scan_fwd_data_flow(ctypes.byref(dims), Q, dt)
+    if flow == ssd.SSD_FLOW_WALK_OUTPUT:
         # the walk keeps chunk states on chip: only the entering states
         assert n == _round(ns * elt)
+    elif flow == ssd.SSD_FLOW_WALK_OUTPUT_FUSED:
+        # entering states, then a ticket counter (32 ints with padding) and one
+        # progress counter per walker of four virtual heads
+        Hv = H * max(P, 64) // 64
+        assert n == _round(ns * elt) + _round((32 + b * Hv // 4) * 4)
     else:
         # chunk states (fp32), per-chunk log-decays, entering states
         assert n == _round(ns * 4) + _round(b * T * H * 4) + _round(ns * elt)
 
 
 @pytest.mark.parametrize("b,L,H,P,N,G,Q,dt,flow", [
-    (4, 8192, 80, 64, 128, 1, 256, ssd.SSD_BF16, ssd.SSD_FLOW_WALK_OUTPUT),   # 2.7B layer
-    (8, 2048, 24, 64, 128, 1, 256, ssd.SSD_BF16, ssd.SSD_FLOW_WALK_OUTPUT),   # 130M layer
+    (4, 8192, 80, 64, 128, 1, 256, ssd.SSD_BF16, ssd.SSD_FLOW_WALK_OUTPUT_FUSED),   # 2.7B layer
+    (8, 2048, 24, 64, 128, 1, 256, ssd.SSD_BF16, ssd.SSD_FLOW_WALK_OUTPUT),   # 130M layer (8 chunks)
+    (8, 2048, 24, 64, 128, 1, 128, ssd.SSD_BF16, ssd.SSD_FLOW_WALK_OUTPUT_FUSED),   # 16 chunks
     (1024, 512, 32, 64, 64, 1, 256, ssd.SSD_BF16, ssd.SSD_FLOW_WALK_OUTPUT),  # 2 chunks
     (1, 524288, 32, 64, 64, 1, 256, ssd.SSD_BF16, ssd.SSD_FLOW_TC_THREE_KERNEL),  # 16 walkers
     (4, 131072, 32, 64, 64, 1, 256, ssd.SSD_BF16, ssd.SSD_FLOW_TC_THREE_KERNEL),  # 64 walkers
     (6, 32768, 32, 64, 64, 1, 256, ssd.SSD_BF16, ssd.SSD_FLOW_WALK_OUTPUT),  # 96 walkers
     (2, 600, 4, 64, 128, 1, 256, ssd.SSD_BF16, ssd.SSD_FLOW_TC_THREE_KERNEL),
     (4, 8192, 80, 64, 128, 1, 256, ssd.SSD_F32, ssd.SSD_FLOW_SIMT),
-    (4, 8192, 80, 32, 128, 1, 256, ssd.SSD_BF16, ssd.SSD_FLOW_WALK_OUTPUT),   # headdim 32
+    (4, 8192, 80, 32, 128, 1, 256, ssd.SSD_BF16, ssd.SSD_FLOW_WALK_OUTPUT_FUSED),   # headdim 32
     (2, 600, 4, 32, 128, 1, 256, ssd.SSD_BF16, ssd.SSD_FLOW_TC_THREE_KERNEL),
     (2, 600, 4, 96, 128, 1, 256, ssd.SSD_BF16, ssd.SSD_FLOW_SIMT),            # headdim 96
-    (4, 8192, 40, 128, 128, 1, 256, ssd.SSD_BF16, ssd.SSD_FLOW_WALK_OUTPUT),  # 80 virtual heads
+    (4, 8192, 40, 128, 128, 1, 256, ssd.SSD_BF16, ssd.SSD_FLOW_WALK_OUTPUT_FUSED),  # 80 virtual heads
     (2, 600, 6, 64, 128, 2, 256, ssd.SSD_BF16, ssd.SSD_FLOW_TC_THREE_KERNEL),  # 3 heads a group
-    (16, 600, 10, 64, 128, 2, 256, ssd.SSD_BF16, ssd.SSD_FLOW_WALK_OUTPUT),   # 96 walkers
+    (16, 600, 10, 64, 128, 2, 256, ssd.SSD_BF16, ssd.SSD_FLOW_WALK_OUTPUT),   # 96 walkers, 5 heads a group
     (2, 300, 4, 64, 128, 1, 64, ssd.SSD_BF16, ssd.SSD_FLOW_TC_THREE_KERNEL),  # chunk 64
     (2, 300, 4, 64, 48, 1, 256, ssd.SSD_BF16, ssd.SSD_FLOW_SIMT),             # dstate 48
 ])
@@ -106,6 +116,40 @@ def test_data_flow_query(lib, b, L, H, P, N, G, Q, dt, flow):
     assert lib.ssd_chunk_scan_fwd_data_flow(ctypes.byref(dims), Q, dt) == flow
     tc = lib.ssd_chunk_scan_fwd_uses_tensor_cores(ctypes.byref(dims), Q, dt)
     assert tc == (0 if flow == ssd.SSD_FLOW_SIMT else 1)
+
+
+def test_forced_flow_workspace_and_rejections(lib):
+    """The flow-choosing entry points: each flow's workspace (the default's is
+    the chosen flow's), SSD_ERR_UNSUPPORTED for a flow that does not cover the
+    sizes, SSD_ERR_INVALID_ARG for an unknown one -- all before any device
+    work."""
+    n = ctypes.c_size_t(0)
+
+    def ws(dims, Q, flow):
+        st = lib.ssd_chunk_scan_fwd_flow_workspace_size(ctypes.byref(dims), Q, ssd.SSD_BF16,
+                                                        flow, ctypes.byref(n))
+        return st, int(n.value)
+
+    d = ssd.make_dims(8, 2048, 24, 64, 128, 1)
+    T, ns = 8, 8 * 8 * 24 * 64 * 128
+    assert ws(d, 256, -1) == ws(d, 256, ssd.SSD_FLOW_WALK_OUTPUT)
+    assert ws(d, 256, ssd.SSD_FLOW_WALK_OUTPUT)[1] == _round(2 * ns)
+    assert ws(d, 256, ssd.SSD_FLOW_WALK_OUTPUT_FUSED)[1] == _round(2 * ns) + _round((32 + 8 * 6) * 4)
+    three = _round(4 * ns) + _round(8 * T * 24 * 4) + _round(2 * ns)
+    assert ws(d, 256, ssd.SSD_FLOW_TC_THREE_KERNEL)[1] == three
+    assert ws(d, 256, ssd.SSD_FLOW_SIMT)[1] == three
+    odd = ssd.make_dims(16, 600, 10, 64, 128, 2)            # 5 heads a group
+    assert ws(odd, 256, ssd.SSD_FLOW_WALK_OUTPUT_FUSED)[0] == ssd.SSD_ERR_UNSUPPORTED
+    n64 = ssd.make_dims(8, 2048, 24, 64, 64, 1)             # dstate 64
+    assert ws(n64, 256, ssd.SSD_FLOW_WALK_OUTPUT_FUSED)[0] == ssd.SSD_ERR_UNSUPPORTED
+    p96 = ssd.make_dims(2, 600, 4, 96, 128, 1)              # no tensor cores
+    assert ws(p96, 256, ssd.SSD_FLOW_WALK_OUTPUT)[0] == ssd.SSD_ERR_UNSUPPORTED
+    assert ws(p96, 256, ssd.SSD_FLOW_SIMT)[0] == ssd.SSD_OK
+    assert ws(d, 256, 7)[0] == ssd.SSD_ERR_INVALID_ARG
+    st = lib.ssd_chunk_scan_fwd_with_flow(None, None, None, None, None, None, 256, None, None,
+                                          None, ctypes.byref(odd), ssd.SSD_BF16, None, 0, None,
+                                          ssd.SSD_FLOW_WALK_OUTPUT_FUSED)
+    assert st == ssd.SSD_ERR_UNSUPPORTED
 
 
 def test_data_flow_query_rejects(lib):

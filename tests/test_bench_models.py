@@ -32,16 +32,23 @@ def test_kernel_bytes_of_both_data_flows():
     kb = bench.kernel_bytes(inputs.LAYER_2P7B)
     io = {k: round(v[1] / 1e6, 1) for k, v in kb.items()}
     assert io == {"chunk_state": 690.0, "state_pass": 524.3, "chunk_out": 866.1,
-                  "state_walk": 543.2}
+                  "state_walk": 543.2, "walk_out": 1409.3}
     alg = {k: round(v[0] / 1e6, 1) for k, v in kb.items()}
     # chunk_out: x read + y written + B + C + dt = 698.4 MB
     assert alg["chunk_out"] == 698.4
     # the walk: x + B + dt + initial and final states (fp32, 10.5 MB each)
     b, L, H, P, N = 4, 8192, 80, 64, 128
     assert kb["state_walk"][0] == b * L * (H * P * 2 + N * 2 + 4 * H) + 2 * 4 * b * H * P * N
-    # the walk + output flow touches every byte of bytes_min; no share exceeds it
+    # the walk + output flow touches every byte of bytes_min; no share exceeds it,
+    # and the one-launch flow's kernel has all of it
     _, _, nbytes = bench.fwd_model(inputs.LAYER_2P7B)
     assert max(v[0] for v in kb.values()) <= nbytes
+    assert kb["walk_out"][0] == nbytes
+    # its own I/O: x and B read by walkers and tiles, C once, dt twice, the
+    # entering states written and read (bf16)
+    ns = b * (L // 256) * H * P * N
+    assert kb["walk_out"][1] == (3 * b * L * H * P * 2 + 3 * b * L * N * 2 + 2 * 4 * b * L * H
+                                 + 2 * 4 * b * H * P * N + 2 * 2 * ns)
 
 
 def test_backward_bytes():

@@ -21,9 +21,9 @@ def _w(name, b, L, H, P, N, G, Q, dtype, init, seed):
                            seed=seed)
 
 
-def _check_full(w, chunk=None):
+def _check_full(w, chunk=None, flow=None):
     inp = inputs.make_inputs(w)
-    y, f = gpu_fwd(inp, chunk or w.chunk)
+    y, f = gpu_fwd(inp, chunk or w.chunk, flow=flow)
     y_ref, f_ref = oracle_fwd(inp)
     tol = TOL[w.dtype]
     ey, ef = rel_err(y, y_ref), rel_err(f, f_ref)
@@ -261,21 +261,73 @@ def test_stage_state_walk(case):
 
 
 WALK_FWD_CASES = [
-    # name,                b,  L,    H,  P,  N,  G,  Q,  init
-    ("walk_fwd_n128_g2", 8, 900, 40, 64, 128, 2, 256, True),    # 4 chunks, last one partial
-    ("walk_fwd_n64_q128", 16, 1100, 12, 64, 64, 2, 128, True),  # 9 chunks, last one partial
+    # name,                   b,  L,    H,  P,  N,  G,  Q,  init
+    ("walk_fwd_n128_g2_odd", 16, 700, 10, 64, 128, 2, 256, True),  # 5 heads a group, 3 chunks
+    ("walk_fwd_n64_q128", 16, 1100, 12, 64, 64, 2, 128, True),     # 9 chunks, last one partial
 ]
 
 
 @pytest.mark.parametrize("case", WALK_FWD_CASES, ids=[c[0] for c in WALK_FWD_CASES])
 def test_walk_path_full_forward_ragged_groups(case):
-    """Shapes the forward runs as walk + output (enough (batch, head pair)
-    walkers and chunks), with a ragged last chunk, two groups and initial
+    """Shapes the forward runs as walk + output in two launches (enough
+    (batch, head pair) walkers; dstate 64 or a head count per group that is
+    not a multiple of 4), with a ragged last chunk, two groups and initial
     states; every element checked."""
     name, b, L, H, P, N, G, Q, init = case
     dims = ssd.make_dims(b, L, H, P, N, G)
     assert ssd.ssd_chunk_scan_fwd_data_flow(dims, Q, torch.bfloat16) == ssd.SSD_FLOW_WALK_OUTPUT
     _check_full(_w(name, b, L, H, P, N, G, Q, "bf16", init, seed=35))
+
+
+FUSED_FWD_CASES = [
+    # name,                 b,  L,    H,  P,   N,  G,  Q,  init
+    ("fused_n128_g2", 8, 900, 40, 64, 128, 2, 256, True),       # 4 chunks, last one partial
+    ("fused_q128_p128", 8, 1000, 24, 128, 128, 1, 128, True),   # 48 virtual heads, 8 chunks
+    ("fused_p32", 8, 600, 48, 32, 128, 1, 256, False),          # headdim 32 (zero-padded)
+    ("fused_tile_heads_18", 6, 700, 36, 64, 128, 1, 256, True),  # tiles of 18 heads: a walker's
+                                                                 # four heads split between tiles
+    ("fused_192_walkers", 48, 520, 16, 64, 128, 1, 256, True),  # more walkers than SMs
+    ("fused_one_chunk", 4, 200, 8, 64, 128, 1, 256, True),      # a single (partial) chunk
+    ("fused_few_walkers", 1, 1300, 4, 64, 128, 1, 256, True),   # one walker
+]
+
+
+@pytest.mark.parametrize("case", FUSED_FWD_CASES, ids=[c[0] for c in FUSED_FWD_CASES])
+def test_fused_walk_output_full_forward(case):
+    """The one-launch data flow (walkers of four heads and output tiles side
+    by side, the tiles waiting on the walkers' progress counters), forced on
+    small shapes: ragged chunks, two groups, 128-token chunks, headdim 32 and
+    128, tiles whose heads straddle walkers, more walkers than the GPU has SMs
+    (so that walkers start in waves), a single chunk and a single walker;
+    every element checked."""
+    name, b, L, H, P, N, G, Q, init = case
+    _check_full(_w(name, b, L, H, P, N, G, Q, "bf16", init, seed=37),
+                flow=ssd.SSD_FLOW_WALK_OUTPUT_FUSED)
+    ssd.ssd_poll_device_status()       # raises if a bounded wait gave up
+
+
+def test_fused_flow_taken_for_long_sequences():
+    """With 16 chunks or more the forward takes the one-launch flow by itself
+    (ragged last chunk; every element checked)."""
+    w = _w("fused_default", 4, 3900, 48, 64, 128, 2, 256, "bf16", True, seed=38)
+    dims = ssd.make_dims(w.batch, w.seqlen, w.nheads, w.headdim, w.dstate, w.ngroups)
+    assert ssd.ssd_chunk_scan_fwd_data_flow(dims, 256, torch.bfloat16) == \
+        ssd.SSD_FLOW_WALK_OUTPUT_FUSED
+    _check_full(w)
+
+
+def test_every_flow_agrees_with_the_oracle():
+    """One input set through every data flow the sizes allow, each against the
+    oracle (the SIMT flow at the fp32 kernels' accuracy on bf16 inputs)."""
+    w = _w("all_flows", 8, 1300, 24, 64, 128, 1, 256, "bf16", True, seed=39)
+    inp = inputs.make_inputs(w)
+    y_ref, f_ref = oracle_fwd(inp)
+    for flow in (ssd.SSD_FLOW_SIMT, ssd.SSD_FLOW_TC_THREE_KERNEL, ssd.SSD_FLOW_WALK_OUTPUT,
+                 ssd.SSD_FLOW_WALK_OUTPUT_FUSED):
+        y, f = gpu_fwd(inp, 256, flow=flow)
+        ey, ef = rel_err(y, y_ref), rel_err(f, f_ref)
+        record(f"all_flows_{flow}", y=ey, final=ef)
+        assert ey <= TOL["bf16"] and ef <= TOL["bf16"], (flow, ey, ef)
 
 
 def test_walk_and_three_kernel_flows_agree():
@@ -473,11 +525,12 @@ def test_tensor_core_path_selected_for_layer_shapes():
         dims = ssd.make_dims(w.batch, w.seqlen, w.nheads, w.headdim, w.dstate, w.ngroups)
         assert ssd.ssd_chunk_scan_fwd_uses_tensor_cores(dims, w.chunk, torch.bfloat16) == 1, w.name
         assert ssd.ssd_chunk_scan_fwd_data_flow(dims, w.chunk, torch.bfloat16) in (
-            ssd.SSD_FLOW_WALK_OUTPUT, ssd.SSD_FLOW_TC_THREE_KERNEL), w.name
-    for w in (inputs.LAYER_130M, inputs.LAYER_2P7B):
+            ssd.SSD_FLOW_WALK_OUTPUT_FUSED, ssd.SSD_FLOW_WALK_OUTPUT,
+            ssd.SSD_FLOW_TC_THREE_KERNEL), w.name
+    for w, flow in ((inputs.LAYER_130M, ssd.SSD_FLOW_WALK_OUTPUT),
+                    (inputs.LAYER_2P7B, ssd.SSD_FLOW_WALK_OUTPUT_FUSED)):
         dims = ssd.make_dims(w.batch, w.seqlen, w.nheads, w.headdim, w.dstate, w.ngroups)
-        assert ssd.ssd_chunk_scan_fwd_data_flow(dims, w.chunk, torch.bfloat16) == \
-            ssd.SSD_FLOW_WALK_OUTPUT, w.name
+        assert ssd.ssd_chunk_scan_fwd_data_flow(dims, w.chunk, torch.bfloat16) == flow, w.name
     t = inputs.TINY_F32
     dims = ssd.make_dims(t.batch, t.seqlen, t.nheads, t.headdim, t.dstate, t.ngroups)
     assert ssd.ssd_chunk_scan_fwd_uses_tensor_cores(dims, t.chunk, torch.float32) == 0
@@ -489,6 +542,7 @@ POSITIVE_A_CASES = [
     # a growing state: A > 0 with a modest growth per chunk, through each data flow
     ("posA_three_kernel", 2, 600, 4, 64, 128, 1, 256, "bf16"),
     ("posA_walk", 8, 1100, 24, 64, 128, 1, 256, "bf16"),
+    ("posA_fused", 8, 1100, 24, 64, 128, 1, 256, "bf16"),
     ("posA_simt_f32", 1, 500, 3, 16, 32, 1, 64, "f32"),
 ]
 
@@ -500,7 +554,7 @@ def test_positive_a_growing_state(case):
     inp = inputs.make_inputs(w)
     g = torch.Generator().manual_seed(48)
     inp["A"] = 0.1 + 0.9 * torch.rand(H, generator=g)     # A in [0.1, 1.0]: exp(dt A) > 1
-    y, f = gpu_fwd(inp, Q)
+    y, f = gpu_fwd(inp, Q, flow=ssd.SSD_FLOW_WALK_OUTPUT_FUSED if name == "posA_fused" else None)
     y_ref, f_ref = oracle_fwd(inp)
     ey, ef = rel_err(y, y_ref), rel_err(f, f_ref)
     record(name, y=ey, final=ef)
