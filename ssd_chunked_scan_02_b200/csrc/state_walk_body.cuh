@@ -55,6 +55,7 @@ namespace walk {
 using namespace sm100;
 
 constexpr int kSub = 64;                 // tokens per ring entry
+constexpr int kPrefetch = 6;             // L2 prefetch distance, in ring entries
 
 template <int HP>
 struct Roles {
@@ -174,6 +175,15 @@ __device__ __forceinline__ void body(const CUtensorMap* tmX, const CUtensorMap* 
                 for (int nb = 0; nb < N / 64; ++nb)
                     tma_load_4d(ent + S::kXPart + nb * kSub * 128, tmB, &bars[BAR_FULL + e],
                                 nb * 64, g, row, (int)b);
+                // the boxes six entries on into L2, so that their loads (issued when
+                // a ring entry frees) find them there
+                if (si + kPrefetch < nsteps) {
+                    const int rp = (int)(((si + kPrefetch) / kNSub) * Q + ((si + kPrefetch) % kNSub) * kSub);
+#pragma unroll
+                    for (int k = 0; k < HP; ++k)
+                        if (k < nreal) tma_prefetch_4d(tmX, 0, h0 + k, rp, (int)b);
+                    for (int nb = 0; nb < N / 64; ++nb) tma_prefetch_4d(tmB, nb * 64, g, rp, (int)b);
+                }
             }
             if (!ok) s_flag[0] = 1;
         } else if (lane == 1 && progress) {
