@@ -356,12 +356,11 @@ SSD_API int ssd_chunk_scan_fwd_uses_tensor_cores(const ssd_dims_t* dims, int chu
 /* Which data flow ssd_chunk_scan_fwd takes for these sizes (decided from the
  * sizes alone; the workspace size follows from it):
  *   SSD_FLOW_WALK_OUTPUT_FUSED  the same two parts in one launch: walkers
- *                            of four heads and output tiles side by side, an
- *                            output tile starting once the walkers have
- *                            written the states entering its chunk (dstate
- *                            128, heads per group a multiple of 4 after the
- *                            headdim split, 16 chunks or more; a memset of
- *                            the workspace's scheduling counters comes
+ *                            of two or four heads and output tiles side by
+ *                            side, an output tile starting once the walkers
+ *                            have written the states entering its chunk (16
+ *                            chunks or more and at most 160 walkers; a memset
+ *                            of the workspace's scheduling counters comes
  *                            first);
  *   SSD_FLOW_WALK_OUTPUT     state walk (steps 2+3 on chip, entering states
  *                            written in bf16) then the tensor-core output
@@ -386,9 +385,8 @@ SSD_API int ssd_chunk_scan_fwd_data_flow(const ssd_dims_t* dims, int chunk_size,
  * of the SSD_FLOW_* values above, or -1 for the library's own choice (what
  * ssd_chunk_scan_fwd does).  Every flow computes the same result up to
  * rounding; SSD_FLOW_SIMT covers every size, the tensor-core flows the
- * sizes ssd_chunk_scan_fwd_uses_tensor_cores accepts, and
- * SSD_FLOW_WALK_OUTPUT_FUSED further needs dstate 128 and a multiple of 4
- * (virtual) heads per group.  A flow that does not cover the sizes returns
+ * sizes ssd_chunk_scan_fwd_uses_tensor_cores accepts.  A flow that does not
+ * cover the sizes returns
  * SSD_ERR_UNSUPPORTED, an unknown one SSD_ERR_INVALID_ARG.  The workspace
  * must hold ssd_chunk_scan_fwd_flow_workspace_size(.., flow, ..) bytes.
  * For benchmarks and tests that compare the flows.

@@ -158,10 +158,11 @@ __device__ __forceinline__ void scale_pieces(uint8_t* base, int t, F f) {
 // One tile: rows [128 t, 128 t + 128) of chunk c of sequence b, heads
 // head0 .. head0 + HG - 1 (virtual heads of headdim 64; H counts them, real
 // head = virtual head / ksplit).  `smem` is 1024-aligned.  When `progress`
-// is given, the entering states are produced by walkers of the same launch:
-// before loading the entering state of head h the producer waits until
-// progress[b * (H / 4) + h / 4] (the walker of h's four heads) has reached
-// c + 1.
+// is given, the entering states are produced by walkers of the same launch,
+// each of `whp` consecutive heads of one group (ceil(heads per group / whp)
+// walkers a group, numbered by batch, group, first head): before loading the
+// entering state of head h the producer waits until the count of h's walker
+// has reached c + 1.
 template <int Q, int N>
 __device__ __forceinline__ void body(const CUtensorMap* tmX, const CUtensorMap* tmB,
                                      const CUtensorMap* tmC, const CUtensorMap* tmH,
@@ -169,7 +170,7 @@ __device__ __forceinline__ void body(const CUtensorMap* tmX, const CUtensorMap* 
                                      const float* __restrict__ A, const float* __restrict__ Dv,
                                      int64_t L, int H, int G, int64_t T, int HG, int ksplit,
                                      int64_t b, int64_t c, int t, int head0, uint8_t* smem,
-                                     const int* progress, const WaitCtx& status) {
+                                     const int* progress, int whp, const WaitCtx& status) {
     // H counts virtual heads (headdim 64); real head = virtual head / ksplit
     const int Hr = H / ksplit;
     using S = OutSmem<Q, N>;
@@ -252,14 +253,16 @@ __device__ __forceinline__ void body(const CUtensorMap* tmX, const CUtensorMap* 
                                 nb * 64, hrow);
             };
             // entering states written by walkers of this launch: wait for the
-            // walker of head hi's four heads to have written chunk c's
-            int ready_q = -1;
+            // walker of head hi to have written chunk c's
+            int64_t ready_w = -1;
             auto wait_h = [&](int hi) -> bool {
                 if (!progress) return true;
-                const int q = (head0 + hi) >> 2;
-                if (q <= ready_q) return true;
-                ready_q = q;
-                const bool r = flag_wait_geq(progress + b * (H >> 2) + q, (int)c + 1, status);
+                const int h = head0 + hi, hpg = H / G, gg = h / hpg;
+                const int wpg = (hpg + whp - 1) / whp;
+                const int64_t w = (b * G + gg) * wpg + (h - gg * hpg) / whp;
+                if (w <= ready_w) return true;
+                ready_w = w;
+                const bool r = flag_wait_geq(progress + w, (int)c + 1, status);
                 fence_proxy_async_global();
                 return r;
             };

@@ -25,15 +25,17 @@
 // P = 64), so a TMEM lane is a state column and a warp's prev/final stores are
 // contiguous along n; with N = 64 (HP = 2) it forms S (M = two heads x P rows,
 // N = 64), a lane is a (head, p) row.  x and B come by TMA in 64-token
-// sub-steps through a ring of three or four entries; x rows are scaled in place by the
+// sub-steps through a three-entry ring; x rows are scaled in place by the
 // decay weights w_j = exp(cs_last - cs_j) dt_j before the MMA reads them.
 //
 // Roles (32 (2 HP + 6) threads): warps 0 .. 2HP-1 dt prefix sums (warp =
 // (head, half of the chunk)) and x scaling (thread t scales row t of each
 // ring entry: head t / 64, token t % 64, and each warp reports its rows by
 // its own arrival); the next four warps the state epilogue; then the TMA
-// producer and the MMA issuer (TMEM owner).  Every wait is bounded; a
-// warpgroup leaves its loop only when all its threads agree (bar.red.or).
+// producer and the MMA issuer (TMEM owner).  Warps past these (a walker run
+// by a larger block) only take part in the block's barriers.  Every wait is
+// bounded; a warpgroup leaves its loop only when all its threads agree
+// (bar.red.or).
 //
 // When `progress` is given (the walker of four heads), the walker publishes
 // how many entering states are in global memory (c + 1 once prev_c is
@@ -341,7 +343,7 @@ __device__ __forceinline__ void body(const CUtensorMap* tmX, const CUtensorMap* 
             }
         }
         if (fail) s_flag[0] = 1;
-    } else {
+    } else if (warp < R::kEpi + 4) {
         // ================================================== state epilogue (four warps)
         const int m = tid - 32 * R::kEpi;              // TMEM lane
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;

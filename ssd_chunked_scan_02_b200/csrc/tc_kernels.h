@@ -64,11 +64,10 @@ cudaError_t launch_state_walk_tc(const void* x, const float* dt, const float* A,
 // True when the forward runs the walk: enough (batch, head pair) walkers.
 bool walk_preferred(const Dims& d);
 
-// The whole forward in one launch (walkers of four heads and output tiles
-// side by side; walk_out_tc.cu): dstate 128, chunk 128 or 256, heads per
-// group a multiple of 4 (virtual heads).  `sched` is device scratch of
-// walk_out_sched_bytes(d) bytes (zeroed by the launcher on `s`); prev as for
-// the walk.
+// The whole forward in one launch (walkers of two or four heads and output
+// tiles side by side; walk_out_tc.cu): dstate 64 or 128, chunk 128 or 256.
+// `sched` is device scratch of walk_out_sched_bytes(d) bytes (zeroed by the
+// launcher on `s`); prev as for the walk.
 bool walk_out_supported(const Dims& d);
 // ... and the forward takes it (enough chunks for the overlap to pay).
 bool walk_out_preferred(const Dims& d);

@@ -1,5 +1,5 @@
-// walk_out_tc.cu -- the whole tensor-core forward in one launch (bf16, dstate
-// 128): walkers (steps a0 + a2 + a3: chunk states and the inter-chunk
+// walk_out_tc.cu -- the whole tensor-core forward in one launch (bf16):
+// walkers (steps a0 + a2 + a3: chunk states and the inter-chunk
 // recurrence, state_walk_body.cuh) and output tiles (steps a1 + a4, the
 // masked C B^T term, the entering-state term and the skip,
 // chunk_out_body.cuh) run side by side, so the output tiles of chunk c start
@@ -13,7 +13,8 @@
 //
 // Scheduling.  Every CTA first takes a ticket (one atomic add on a counter
 // the host zeroes before the launch).  Tickets 0 .. W-1 are the walkers, one
-// per (batch, four heads of one group), each holding an SM to itself;
+// per (batch, HP heads of one group: four for dstate 128 when walkers of two
+// would not leave SMs for the tiles, else two), each holding an SM to itself;
 // tickets W and up are output tiles in chunk-major order.  A walker waits on
 // nothing outside its CTA.  An output tile waits (bounded, like every wait
 // here) only on walkers, and only for walkers whose tickets were taken before
@@ -38,14 +39,14 @@ namespace ssd {
 namespace {
 using namespace sm100;
 
-constexpr int kHP = 4;                              // heads per walker
 constexpr int kThreads = outk::kThreads;
-static_assert(walk::Roles<kHP>::kThreads == outk::kThreads, "one block size for both roles");
+static_assert(walk::Roles<4>::kThreads == outk::kThreads, "one block size for both roles");
+static_assert(walk::Roles<2>::kThreads <= outk::kThreads, "one block size for both roles");
 
-template <int Q>
+template <int Q, int N, int HP>
 struct FusedSmem {
-    static constexpr int kWalk = walk::Smem<Q, 128, kHP>::kAlloc;
-    static constexpr int kOut = outk::OutSmem<Q, 128>::kAlloc;
+    static constexpr int kWalk = walk::Smem<Q, N, HP>::kAlloc;
+    static constexpr int kOut = outk::OutSmem<Q, N>::kAlloc;
     static constexpr int kAlloc = kWalk > kOut ? kWalk : kOut;
     static_assert(kAlloc <= 227 * 1024, "shared memory");
 };
@@ -54,8 +55,29 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
     return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
+// The launch's shape: HP heads a walker, HG heads an output tile.
+struct Cfg {
+    int hp, hg;
+};
+
+Cfg config(const Dims& v) {
+    Cfg c;
+    const int64_t hpg = v.H / v.G;
+    const int64_t pairs = v.b * v.G * ((hpg + 1) / 2);
+    // walkers of two heads walk faster (4.5 against 6 us a chunk) but must
+    // leave SMs for the output tiles; four heads (dstate 128 only) halve them
+    c.hp = (v.N == 128 && pairs > 100) ? 4 : 2;
+    c.hg = outk::pick_heads_per_cta(v.H, v.G);
+    return c;
+}
+
+int64_t walkers(const Dims& v, int hp) {
+    const int64_t hpg = v.H / v.G;
+    return v.b * v.G * ((hpg + hp - 1) / hp);
+}
+
 // sched[0]: ticket counter; sched[32 + w]: entering states written by walker w.
-template <int Q>
+template <int Q, int N, int HP>
 __global__ void __launch_bounds__(kThreads, 1)
 walk_out_tc_kernel(const __grid_constant__ CUtensorMap tmXw, const __grid_constant__ CUtensorMap tmBw,
                    const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
@@ -73,32 +95,36 @@ walk_out_tc_kernel(const __grid_constant__ CUtensorMap tmXw, const __grid_consta
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
     int* progress = sched + 32;
-    const int quads = H >> 2;                       // walkers per batch (H / G a multiple of 4)
+    const int hpg = H / G;
+    const int wpg = (hpg + HP - 1) / HP;             // walkers a group
     if (tk < nwalk) {
-        const int64_t b = tk / quads;
-        const int h0 = (tk % quads) * kHP;
-        walk::body<Q, 128, kHP>(&tmXw, &tmBw, dt, A, init, prev, fin, L, H, G, T, ksplit, pcols,
-                                b, h0 / (H / G), h0, kHP, smem, progress + tk, status);
+        const int64_t b = tk / (G * wpg);
+        const int r = tk % (G * wpg);
+        const int g = r / wpg, l = r % wpg;
+        const int h0 = g * hpg + HP * l;
+        const int nreal = hpg - HP * l < HP ? hpg - HP * l : HP;
+        walk::body<Q, N, HP>(&tmXw, &tmBw, dt, A, init, prev, fin, L, H, G, T, ksplit, pcols,
+                             b, g, h0, nreal, smem, progress + tk, status);
     } else {
         const int nhg = H / HG;
-        const int64_t per_chunk = (int64_t)(nwalk / quads) * kTiles * nhg;   // batch x tiles x groups
+        const int64_t per_chunk = (int64_t)(nwalk / (G * wpg)) * kTiles * nhg;   // batch x tiles x groups
         const int64_t o = tk - nwalk;
         const int64_t c = o / per_chunk;
         const int64_t r = o - c * per_chunk;
         const int64_t b = r / (kTiles * nhg);
         const int r2 = (int)(r - b * (kTiles * nhg));
         const int t = r2 / nhg, hg = r2 - t * nhg;
-        outk::body<Q, 128>(&tmX, &tmB, &tmC, &tmH, &tmY, dt, A, Dv, L, H, G, T, HG, ksplit, b, c,
-                           t, hg * HG, smem, progress, status);
+        outk::body<Q, N>(&tmX, &tmB, &tmC, &tmH, &tmY, dt, A, Dv, L, H, G, T, HG, ksplit, b, c,
+                         t, hg * HG, smem, progress, HP, status);
     }
 }
 
-template <int Q>
+template <int Q, int N, int HP>
 cudaError_t launch_impl(const void* x, const float* dt, const float* A, const void* B,
                         const void* C, const float* D, const float* init, void* prev, void* y,
-                        float* fin, int* sched, const Dims& d, int ksplit, int pc, cudaStream_t s) {
-    constexpr int N = 128;
-    using FS = FusedSmem<Q>;
+                        float* fin, int* sched, const Dims& d, int ksplit, int pc, int HG,
+                        cudaStream_t s) {
+    using FS = FusedSmem<Q, N, HP>;
     CUtensorMap tmXw, tmBw, tmX, tmB, tmC, tmH, tmY;
     // x and y: pc columns a (virtual) head; a 64-column box reads zeros past
     // them and stores only up to them
@@ -123,16 +149,15 @@ cudaError_t launch_impl(const void* x, const float* dt, const float* A, const vo
     const sm100::WaitCtx status = make_wait_ctx();
     if (!status.word) return cudaErrorUnknown;
 
-    const int HG = outk::pick_heads_per_cta(d.H, d.G);
-    const int64_t nwalk = d.b * (d.H / kHP);
+    const int64_t nwalk = walkers(d, HP);
     const int64_t grid = nwalk + d.b * d.T * (Q / 128) * (d.H / HG);
     if (grid > 0x7fffffffLL) return cudaErrorInvalidValue;
-    e = cudaMemsetAsync(sched, 0, walk_out_sched_bytes(d), s);
+    e = cudaMemsetAsync(sched, 0, (size_t)(32 + nwalk) * sizeof(int), s);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(walk_out_tc_kernel<Q>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             FS::kAlloc);
+    e = cudaFuncSetAttribute(walk_out_tc_kernel<Q, N, HP>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, FS::kAlloc);
     if (e != cudaSuccess) return e;
-    walk_out_tc_kernel<Q><<<(unsigned)grid, kThreads, FS::kAlloc, s>>>(
+    walk_out_tc_kernel<Q, N, HP><<<(unsigned)grid, kThreads, FS::kAlloc, s>>>(
         tmXw, tmBw, tmX, tmB, tmC, tmH, tmY, dt, A, D, init, static_cast<__nv_bfloat16*>(prev), fin,
         d.L, (int)d.H, (int)d.G, d.T, HG, ksplit, pc, sched, (int)nwalk, status);
     return cudaGetLastError();
@@ -143,22 +168,24 @@ cudaError_t launch_impl(const void* x, const float* dt, const float* A, const vo
 bool walk_out_supported(const Dims& d) {
     int k = 1;
     const Dims v = virtual_heads(d, &k);
-    return v.N == 128 && (v.Q == 128 || v.Q == 256) && (v.H / v.G) % kHP == 0 &&
-           v.b * (v.H / kHP) <= 0x7fffffffLL;
+    return (v.N == 128 || v.N == 64) && (v.Q == 128 || v.Q == 256) &&
+           walkers(v, 2) <= 0x7fffffffLL;
 }
 
 bool walk_out_preferred(const Dims& d) {
     // The overlap pays once the walk is long: with few chunks the output tiles
     // of the last chunk start only when the walk ends, and the two launches
-    // (whose walkers, two heads a CTA, walk faster) win (measured: 8 chunks
-    // lose, 16 and 32 win).
-    return walk_out_supported(d) && d.T >= 16;
+    // win (measured: 8 chunks lose, 16 and 32 win); with more walkers than SMs
+    // the walk runs in waves and tiles start only after the last wave.
+    int k = 1;
+    const Dims v = virtual_heads(d, &k);
+    return walk_out_supported(d) && d.T >= 16 && walkers(v, config(v).hp) <= 160;
 }
 
 size_t walk_out_sched_bytes(const Dims& d) {
     int k = 1;
     const Dims v = virtual_heads(d, &k);
-    return (size_t)(32 + v.b * (v.H / kHP)) * sizeof(int);
+    return (size_t)(32 + walkers(v, config(v).hp)) * sizeof(int);
 }
 
 cudaError_t launch_walk_out_tc(const void* x, const float* dt, const float* A, const void* B,
@@ -168,11 +195,20 @@ cudaError_t launch_walk_out_tc(const void* x, const float* dt, const float* A, c
     if (!walk_out_supported(d)) return cudaErrorNotSupported;
     int k = 1;
     const Dims v = virtual_heads(d, &k);
-    if (v.Q == 256)
-        return launch_impl<256>(x, dt, A, B, C, D, init, prev, y, final_states, sched, v, k,
-                                head_cols(d), s);
-    return launch_impl<128>(x, dt, A, B, C, D, init, prev, y, final_states, sched, v, k,
-                            head_cols(d), s);
+    const Cfg cf = config(v);
+    const int pc = head_cols(d);
+#define SSD_WALK_OUT(Q_, N_, HP_)                                                             \
+    if (v.Q == Q_ && v.N == N_ && cf.hp == HP_)                                               \
+        return launch_impl<Q_, N_, HP_>(x, dt, A, B, C, D, init, prev, y, final_states, sched, v, \
+                                        k, pc, cf.hg, s);
+    SSD_WALK_OUT(256, 128, 4)
+    SSD_WALK_OUT(128, 128, 4)
+    SSD_WALK_OUT(256, 128, 2)
+    SSD_WALK_OUT(128, 128, 2)
+    SSD_WALK_OUT(256, 64, 2)
+    SSD_WALK_OUT(128, 64, 2)
+#undef SSD_WALK_OUT
+    return cudaErrorNotSupported;
 }
 
 }  // namespace ssd

@@ -97,9 +97,10 @@ def test_workspace_size_formula(lib, b, L, H, P, N, G, Q, dt):
     (8, 2048, 24, 64, 128, 1, 256, ssd.SSD_BF16, ssd.SSD_FLOW_WALK_OUTPUT),   # 130M layer (8 chunks)
     (8, 2048, 24, 64, 128, 1, 128, ssd.SSD_BF16, ssd.SSD_FLOW_WALK_OUTPUT_FUSED),   # 16 chunks
     (1024, 512, 32, 64, 64, 1, 256, ssd.SSD_BF16, ssd.SSD_FLOW_WALK_OUTPUT),  # 2 chunks
+    (16, 32768, 32, 64, 64, 1, 256, ssd.SSD_BF16, ssd.SSD_FLOW_WALK_OUTPUT),  # 256 walkers: in waves
     (1, 524288, 32, 64, 64, 1, 256, ssd.SSD_BF16, ssd.SSD_FLOW_TC_THREE_KERNEL),  # 16 walkers
     (4, 131072, 32, 64, 64, 1, 256, ssd.SSD_BF16, ssd.SSD_FLOW_TC_THREE_KERNEL),  # 64 walkers
-    (6, 32768, 32, 64, 64, 1, 256, ssd.SSD_BF16, ssd.SSD_FLOW_WALK_OUTPUT),  # 96 walkers
+    (6, 32768, 32, 64, 64, 1, 256, ssd.SSD_BF16, ssd.SSD_FLOW_WALK_OUTPUT_FUSED),  # 96 walkers of two heads
     (2, 600, 4, 64, 128, 1, 256, ssd.SSD_BF16, ssd.SSD_FLOW_TC_THREE_KERNEL),
     (4, 8192, 80, 64, 128, 1, 256, ssd.SSD_F32, ssd.SSD_FLOW_SIMT),
     (4, 8192, 80, 32, 128, 1, 256, ssd.SSD_BF16, ssd.SSD_FLOW_WALK_OUTPUT_FUSED),   # headdim 32
@@ -134,20 +135,22 @@ def test_forced_flow_workspace_and_rejections(lib):
     T, ns = 8, 8 * 8 * 24 * 64 * 128
     assert ws(d, 256, -1) == ws(d, 256, ssd.SSD_FLOW_WALK_OUTPUT)
     assert ws(d, 256, ssd.SSD_FLOW_WALK_OUTPUT)[1] == _round(2 * ns)
-    assert ws(d, 256, ssd.SSD_FLOW_WALK_OUTPUT_FUSED)[1] == _round(2 * ns) + _round((32 + 8 * 6) * 4)
     three = _round(4 * ns) + _round(8 * T * 24 * 4) + _round(2 * ns)
     assert ws(d, 256, ssd.SSD_FLOW_TC_THREE_KERNEL)[1] == three
     assert ws(d, 256, ssd.SSD_FLOW_SIMT)[1] == three
-    odd = ssd.make_dims(16, 600, 10, 64, 128, 2)            # 5 heads a group
-    assert ws(odd, 256, ssd.SSD_FLOW_WALK_OUTPUT_FUSED)[0] == ssd.SSD_ERR_UNSUPPORTED
-    n64 = ssd.make_dims(8, 2048, 24, 64, 64, 1)             # dstate 64
+    # walkers of two heads below 100 pairs: 96 walkers, then 32 + 96 counters
+    assert ws(d, 256, ssd.SSD_FLOW_WALK_OUTPUT_FUSED)[1] == _round(2 * ns) + _round((32 + 96) * 4)
+    odd = ssd.make_dims(16, 600, 10, 64, 128, 2)            # 5 heads a group: 3 walkers a group
+    assert ws(odd, 256, ssd.SSD_FLOW_WALK_OUTPUT_FUSED)[1] == \
+        _round(16 * 3 * 10 * 64 * 128 * 2) + _round((32 + 16 * 2 * 3) * 4)
+    n64 = ssd.make_dims(8, 2048, 24, 64, 48, 1)             # dstate 48: SIMT only
     assert ws(n64, 256, ssd.SSD_FLOW_WALK_OUTPUT_FUSED)[0] == ssd.SSD_ERR_UNSUPPORTED
     p96 = ssd.make_dims(2, 600, 4, 96, 128, 1)              # no tensor cores
     assert ws(p96, 256, ssd.SSD_FLOW_WALK_OUTPUT)[0] == ssd.SSD_ERR_UNSUPPORTED
     assert ws(p96, 256, ssd.SSD_FLOW_SIMT)[0] == ssd.SSD_OK
     assert ws(d, 256, 7)[0] == ssd.SSD_ERR_INVALID_ARG
     st = lib.ssd_chunk_scan_fwd_with_flow(None, None, None, None, None, None, 256, None, None,
-                                          None, ctypes.byref(odd), ssd.SSD_BF16, None, 0, None,
+                                          None, ctypes.byref(p96), ssd.SSD_BF16, None, 0, None,
                                           ssd.SSD_FLOW_WALK_OUTPUT_FUSED)
     assert st == ssd.SSD_ERR_UNSUPPORTED
 

@@ -288,18 +288,22 @@ FUSED_FWD_CASES = [
                                                                  # four heads split between tiles
     ("fused_192_walkers", 48, 520, 16, 64, 128, 1, 256, True),  # more walkers than SMs
     ("fused_one_chunk", 4, 200, 8, 64, 128, 1, 256, True),      # a single (partial) chunk
-    ("fused_few_walkers", 1, 1300, 4, 64, 128, 1, 256, True),   # one walker
+    ("fused_few_walkers", 1, 1300, 4, 64, 128, 1, 256, True),   # walkers of two heads
+    ("fused_quad_phantoms", 40, 300, 6, 64, 128, 1, 256, True),  # walkers of four heads, 6 a
+                                                                 # group: two phantom heads
+    ("fused_pair_phantom", 16, 600, 10, 64, 128, 2, 256, True),  # walkers of two, 5 heads a group
+    ("fused_n64", 16, 1100, 12, 64, 64, 2, 128, True),          # dstate 64 (walkers of two)
 ]
 
 
 @pytest.mark.parametrize("case", FUSED_FWD_CASES, ids=[c[0] for c in FUSED_FWD_CASES])
 def test_fused_walk_output_full_forward(case):
-    """The one-launch data flow (walkers of four heads and output tiles side
-    by side, the tiles waiting on the walkers' progress counters), forced on
-    small shapes: ragged chunks, two groups, 128-token chunks, headdim 32 and
-    128, tiles whose heads straddle walkers, more walkers than the GPU has SMs
-    (so that walkers start in waves), a single chunk and a single walker;
-    every element checked."""
+    """The one-launch data flow (walkers of two or four heads and output tiles
+    side by side, the tiles waiting on the walkers' progress counters), forced
+    on small shapes: ragged chunks, two groups, 128-token chunks, headdim 32
+    and 128, dstate 64, tiles whose heads straddle walkers, walkers with
+    phantom heads, more walkers than the GPU has SMs (so that walkers start
+    in waves), a single chunk and a single walker; every element checked."""
     name, b, L, H, P, N, G, Q, init = case
     _check_full(_w(name, b, L, H, P, N, G, Q, "bf16", init, seed=37),
                 flow=ssd.SSD_FLOW_WALK_OUTPUT_FUSED)
