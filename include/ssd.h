@@ -358,7 +358,7 @@ SSD_API int ssd_chunk_scan_fwd_uses_tensor_cores(const ssd_dims_t* dims, int chu
  *   SSD_FLOW_WALK_OUTPUT_FUSED  the same two parts in one launch: walkers
  *                            of two or four heads and output tiles side by
  *                            side, an output tile starting once the walkers
- *                            have written the states entering its chunk (16
+ *                            have written the states entering its chunk (8
  *                            chunks or more and at most 160 walkers; a memset
  *                            of the workspace's scheduling counters comes
  *                            first);

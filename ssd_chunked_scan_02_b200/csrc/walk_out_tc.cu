@@ -55,9 +55,10 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
     return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
-// The launch's shape: HP heads a walker, HG heads an output tile.
+// The launch's shape: HP heads a walker, HG heads an output tile (HG2 in the
+// last KS chunks: smaller tiles there shorten the launch's ragged end).
 struct Cfg {
-    int hp, hg;
+    int hp, hg, hg2, ks;
 };
 
 Cfg config(const Dims& v) {
@@ -68,7 +69,17 @@ Cfg config(const Dims& v) {
     // leave SMs for the output tiles; four heads (dstate 128 only) halve them
     c.hp = (v.N == 128 && pairs > 100) ? 4 : 2;
     c.hg = outk::pick_heads_per_cta(v.H, v.G);
+    c.ks = (c.hg % 2 == 0 && c.hg >= 8 && v.T > 2) ? 2 : 0;
+    c.hg2 = c.ks ? c.hg / 2 : c.hg;
     return c;
+}
+
+// Output tiles of chunks [0, T - ks) (hg heads each) then of the last ks
+// chunks (hg2 heads each), each chunk's in (batch, row block, head block)
+// order.
+int64_t out_tiles(const Dims& v, const Cfg& c) {
+    const int64_t per = v.b * (v.Q / 128);
+    return per * ((v.T - c.ks) * (v.H / c.hg) + c.ks * (v.H / c.hg2));
 }
 
 int64_t walkers(const Dims& v, int hp) {
@@ -86,7 +97,8 @@ walk_out_tc_kernel(const __grid_constant__ CUtensorMap tmXw, const __grid_consta
                    const float* __restrict__ A, const float* __restrict__ Dv,
                    const float* __restrict__ init, __nv_bfloat16* __restrict__ prev,
                    float* __restrict__ fin, int64_t L, int H, int G, int64_t T, int HG,
-                   int ksplit, int pcols, int* __restrict__ sched, int nwalk, WaitCtx status) {
+                   int HG2, int KS, int ksplit, int pcols, int* __restrict__ sched, int nwalk,
+                   WaitCtx status) {
     constexpr int kTiles = Q / 128;
     __shared__ int s_ticket;
     if (threadIdx.x == 0) s_ticket = atomicAdd(sched, 1);
@@ -106,24 +118,33 @@ walk_out_tc_kernel(const __grid_constant__ CUtensorMap tmXw, const __grid_consta
         walk::body<Q, N, HP>(&tmXw, &tmBw, dt, A, init, prev, fin, L, H, G, T, ksplit, pcols,
                              b, g, h0, nreal, smem, progress + tk, status);
     } else {
-        const int nhg = H / HG;
-        const int64_t per_chunk = (int64_t)(nwalk / (G * wpg)) * kTiles * nhg;   // batch x tiles x groups
-        const int64_t o = tk - nwalk;
-        const int64_t c = o / per_chunk;
-        const int64_t r = o - c * per_chunk;
+        const int64_t nb = nwalk / (G * wpg);           // batch
+        const int64_t first = (T - KS) * nb * kTiles * (H / HG);
+        int64_t o = tk - nwalk;
+        int hgs = HG;
+        int64_t c0 = 0;
+        if (o >= first) {                               // the last KS chunks: smaller tiles
+            o -= first;
+            hgs = HG2;
+            c0 = T - KS;
+        }
+        const int nhg = H / hgs;
+        const int64_t per_chunk = nb * kTiles * nhg;    // batch x row blocks x head blocks
+        const int64_t c = c0 + o / per_chunk;
+        const int64_t r = o % per_chunk;
         const int64_t b = r / (kTiles * nhg);
         const int r2 = (int)(r - b * (kTiles * nhg));
         const int t = r2 / nhg, hg = r2 - t * nhg;
-        outk::body<Q, N>(&tmX, &tmB, &tmC, &tmH, &tmY, dt, A, Dv, L, H, G, T, HG, ksplit, b, c,
-                         t, hg * HG, smem, progress, HP, status);
+        outk::body<Q, N>(&tmX, &tmB, &tmC, &tmH, &tmY, dt, A, Dv, L, H, G, T, hgs, ksplit, b, c,
+                         t, hg * hgs, smem, progress, HP, status);
     }
 }
 
 template <int Q, int N, int HP>
 cudaError_t launch_impl(const void* x, const float* dt, const float* A, const void* B,
                         const void* C, const float* D, const float* init, void* prev, void* y,
-                        float* fin, int* sched, const Dims& d, int ksplit, int pc, int HG,
-                        cudaStream_t s) {
+                        float* fin, int* sched, const Dims& d, int ksplit, int pc,
+                        const Cfg& cf, cudaStream_t s) {
     using FS = FusedSmem<Q, N, HP>;
     CUtensorMap tmXw, tmBw, tmX, tmB, tmC, tmH, tmY;
     // x and y: pc columns a (virtual) head; a 64-column box reads zeros past
@@ -150,7 +171,7 @@ cudaError_t launch_impl(const void* x, const float* dt, const float* A, const vo
     if (!status.word) return cudaErrorUnknown;
 
     const int64_t nwalk = walkers(d, HP);
-    const int64_t grid = nwalk + d.b * d.T * (Q / 128) * (d.H / HG);
+    const int64_t grid = nwalk + out_tiles(d, cf);
     if (grid > 0x7fffffffLL) return cudaErrorInvalidValue;
     e = cudaMemsetAsync(sched, 0, (size_t)(32 + nwalk) * sizeof(int), s);
     if (e != cudaSuccess) return e;
@@ -159,7 +180,7 @@ cudaError_t launch_impl(const void* x, const float* dt, const float* A, const vo
     if (e != cudaSuccess) return e;
     walk_out_tc_kernel<Q, N, HP><<<(unsigned)grid, kThreads, FS::kAlloc, s>>>(
         tmXw, tmBw, tmX, tmB, tmC, tmH, tmY, dt, A, D, init, static_cast<__nv_bfloat16*>(prev), fin,
-        d.L, (int)d.H, (int)d.G, d.T, HG, ksplit, pc, sched, (int)nwalk, status);
+        d.L, (int)d.H, (int)d.G, d.T, cf.hg, cf.hg2, cf.ks, ksplit, pc, sched, (int)nwalk, status);
     return cudaGetLastError();
 }
 
@@ -173,13 +194,14 @@ bool walk_out_supported(const Dims& d) {
 }
 
 bool walk_out_preferred(const Dims& d) {
-    // The overlap pays once the walk is long: with few chunks the output tiles
-    // of the last chunk start only when the walk ends, and the two launches
-    // win (measured: 8 chunks lose, 16 and 32 win); with more walkers than SMs
-    // the walk runs in waves and tiles start only after the last wave.
+    // The overlap pays once the walk is long enough: the output tiles of the
+    // last chunk start only when the walk ends (measured: 8 chunks even to 2 %
+    // ahead, 16 and 32 chunks 10-14 % ahead, 4 chunks behind); with more
+    // walkers than SMs the walk runs in waves and tiles start only after the
+    // last wave.
     int k = 1;
     const Dims v = virtual_heads(d, &k);
-    return walk_out_supported(d) && d.T >= 16 && walkers(v, config(v).hp) <= 160;
+    return walk_out_supported(d) && d.T >= 8 && walkers(v, config(v).hp) <= 160;
 }
 
 size_t walk_out_sched_bytes(const Dims& d) {
@@ -200,7 +222,7 @@ cudaError_t launch_walk_out_tc(const void* x, const float* dt, const float* A, c
 #define SSD_WALK_OUT(Q_, N_, HP_)                                                             \
     if (v.Q == Q_ && v.N == N_ && cf.hp == HP_)                                               \
         return launch_impl<Q_, N_, HP_>(x, dt, A, B, C, D, init, prev, y, final_states, sched, v, \
-                                        k, pc, cf.hg, s);
+                                        k, pc, cf, s);
     SSD_WALK_OUT(256, 128, 4)
     SSD_WALK_OUT(128, 128, 4)
     SSD_WALK_OUT(256, 128, 2)

@@ -94,7 +94,8 @@ def test_workspace_size_formula(lib, b, L, H, P, N, G, Q, dt):
 
 @pytest.mark.parametrize("b,L,H,P,N,G,Q,dt,flow", [
     (4, 8192, 80, 64, 128, 1, 256, ssd.SSD_BF16, ssd.SSD_FLOW_WALK_OUTPUT_FUSED),   # 2.7B layer
-    (8, 2048, 24, 64, 128, 1, 256, ssd.SSD_BF16, ssd.SSD_FLOW_WALK_OUTPUT),   # 130M layer (8 chunks)
+    (8, 2048, 24, 64, 128, 1, 256, ssd.SSD_BF16, ssd.SSD_FLOW_WALK_OUTPUT_FUSED),   # 130M layer (8 chunks)
+    (8, 1024, 24, 64, 128, 1, 256, ssd.SSD_BF16, ssd.SSD_FLOW_WALK_OUTPUT),   # 4 chunks
     (8, 2048, 24, 64, 128, 1, 128, ssd.SSD_BF16, ssd.SSD_FLOW_WALK_OUTPUT_FUSED),   # 16 chunks
     (1024, 512, 32, 64, 64, 1, 256, ssd.SSD_BF16, ssd.SSD_FLOW_WALK_OUTPUT),  # 2 chunks
     (16, 32768, 32, 64, 64, 1, 256, ssd.SSD_BF16, ssd.SSD_FLOW_WALK_OUTPUT),  # 256 walkers: in waves
@@ -133,7 +134,7 @@ def test_forced_flow_workspace_and_rejections(lib):
 
     d = ssd.make_dims(8, 2048, 24, 64, 128, 1)
     T, ns = 8, 8 * 8 * 24 * 64 * 128
-    assert ws(d, 256, -1) == ws(d, 256, ssd.SSD_FLOW_WALK_OUTPUT)
+    assert ws(d, 256, -1) == ws(d, 256, ssd.SSD_FLOW_WALK_OUTPUT_FUSED)
     assert ws(d, 256, ssd.SSD_FLOW_WALK_OUTPUT)[1] == _round(2 * ns)
     three = _round(4 * ns) + _round(8 * T * 24 * 4) + _round(2 * ns)
     assert ws(d, 256, ssd.SSD_FLOW_TC_THREE_KERNEL)[1] == three

@@ -263,7 +263,7 @@ def test_stage_state_walk(case):
 WALK_FWD_CASES = [
     # name,                   b,  L,    H,  P,  N,  G,  Q,  init
     ("walk_fwd_n128_g2_odd", 16, 700, 10, 64, 128, 2, 256, True),  # 5 heads a group, 3 chunks
-    ("walk_fwd_n64_q128", 16, 1100, 12, 64, 64, 2, 128, True),     # 9 chunks, last one partial
+    ("walk_fwd_n64_q128", 16, 800, 12, 64, 64, 2, 128, True),      # 7 chunks, last one partial
 ]
 
 
@@ -311,8 +311,8 @@ def test_fused_walk_output_full_forward(case):
 
 
 def test_fused_flow_taken_for_long_sequences():
-    """With 16 chunks or more the forward takes the one-launch flow by itself
-    (ragged last chunk; every element checked)."""
+    """With 8 chunks or more the forward takes the one-launch flow by itself
+    (16 chunks, ragged last chunk; every element checked)."""
     w = _w("fused_default", 4, 3900, 48, 64, 128, 2, 256, "bf16", True, seed=38)
     dims = ssd.make_dims(w.batch, w.seqlen, w.nheads, w.headdim, w.dstate, w.ngroups)
     assert ssd.ssd_chunk_scan_fwd_data_flow(dims, 256, torch.bfloat16) == \
@@ -531,7 +531,7 @@ def test_tensor_core_path_selected_for_layer_shapes():
         assert ssd.ssd_chunk_scan_fwd_data_flow(dims, w.chunk, torch.bfloat16) in (
             ssd.SSD_FLOW_WALK_OUTPUT_FUSED, ssd.SSD_FLOW_WALK_OUTPUT,
             ssd.SSD_FLOW_TC_THREE_KERNEL), w.name
-    for w, flow in ((inputs.LAYER_130M, ssd.SSD_FLOW_WALK_OUTPUT),
+    for w, flow in ((inputs.LAYER_130M, ssd.SSD_FLOW_WALK_OUTPUT_FUSED),
                     (inputs.LAYER_2P7B, ssd.SSD_FLOW_WALK_OUTPUT_FUSED)):
         dims = ssd.make_dims(w.batch, w.seqlen, w.nheads, w.headdim, w.dstate, w.ngroups)
         assert ssd.ssd_chunk_scan_fwd_data_flow(dims, w.chunk, torch.bfloat16) == flow, w.name
