@@ -58,7 +58,17 @@
 //   warps 8-11  epilogue: y staged in shared memory, TMA store;
 //   warp 12     TMA producer (x rows and entering states of the heads, a ring
 //               of four slots for tile 0 of a 256-token chunk, two otherwise);
-//   warp 13     MMA issuer and TMEM owner.
+//   warp 13     MMA issuer and TMEM owner (G, Y, the left block, and on the
+//               exact path ZW);
+//   warp 14     with z2: second MMA issuer, ZW = C_t h^T on the fast path,
+//               concurrently with warp 13's MMAs (a single thread issues an
+//               MMA of these shapes no faster than one every few tens of ns,
+//               whatever N, so two issuers halve a head's MMA time); a slot's
+//               x/h and an accumulator are then released by both issuers'
+//               commits.  Without z2 warp 13 issues ZW too and warp 14 idles
+//               (where the scale warps bound the tile, the second stream of
+//               MMA operand reads slows their shared-memory work more than it
+//               saves).
 // Every wait is bounded; a warpgroup leaves its loop only when all its
 // threads agree (bar.red.or), so no named barrier is left half-arrived.
 #pragma once
@@ -72,7 +82,7 @@ namespace ssd {
 namespace outk {
 using namespace sm100;
 
-constexpr int kThreads = 448;
+constexpr int kThreads = 480;
 constexpr int kMaxHeads = 32;
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -90,12 +100,13 @@ struct OutSmem {
     static constexpr int kXTile = Q * 128;                  // x rows [0, Q) of one head
     static constexpr int kX = kBG + kBGBytes;               // x ring: 2 slots of Q rows (or 4 of 128)
     static constexpr int kYs = kX + 2 * kXTile;             // y staging: 16 KB
-    static constexpr int kDt = kYs + 128 * 128;             // float [Q] dt of one head
-    static constexpr int kCs = kDt + Q * 4;                 // float [Q] its prefix sums (log2 units)
-    static constexpr int kWs = kCs + Q * 4;                 // float [16]: per-warp sums of the scan
-    static constexpr int kBeta = kWs + 16 * 4;              // float [128]  (t = 1 block left of diagonal)
-    static constexpr int kBeta2 = kBeta + 128 * 4;          // float [128]  (diagonal block)
-    static constexpr int kAl = kBeta2 + 128 * 4;            // float [4][128] alpha_i per factor slot
+    // per head modulo 4 (the scans of four heads are taken together)
+    static constexpr int kDt = kYs + 128 * 128;             // float [4][Q] dt of a head
+    static constexpr int kCs = kDt + 4 * Q * 4;             // float [4][Q] its prefix sums (log2 units)
+    static constexpr int kWs = kCs + 4 * Q * 4;             // float [16]: per-warp sums of the scan
+    static constexpr int kBeta = kWs + 16 * 4;              // float [4][128]  (t = 1 block left of diagonal)
+    static constexpr int kBeta2 = kBeta + 4 * 128 * 4;      // float [4][128]  (diagonal block)
+    static constexpr int kAl = kBeta2 + 4 * 128 * 4;        // float [4][128] alpha_i per factor slot
     static constexpr int kRow = kAl + 4 * 128 * 4;          // float [4][128] a_i (1: exact path)
     static constexpr int kPath = kRow + 4 * 128 * 4;        // int [4]: 1 = fast path
     static constexpr int kAD = kPath + 16;                  // float [2][kMaxHeads]: A_h (log2), D_h
@@ -170,7 +181,8 @@ __device__ __forceinline__ void body(const CUtensorMap* tmX, const CUtensorMap* 
                                      const float* __restrict__ A, const float* __restrict__ Dv,
                                      int64_t L, int H, int G, int64_t T, int HG, int ksplit,
                                      int64_t b, int64_t c, int t, int head0, uint8_t* smem,
-                                     const int* progress, int whp, const WaitCtx& status) {
+                                     const int* progress, int whp, bool z2,
+                                     const WaitCtx& status) {
     // H counts virtual heads (headdim 64); real head = virtual head / ksplit
     const int Hr = H / ksplit;
     using S = OutSmem<Q, N>;
@@ -207,9 +219,12 @@ __device__ __forceinline__ void body(const CUtensorMap* tmX, const CUtensorMap* 
     volatile int* s_flag = reinterpret_cast<volatile int*>(smem + S::kFlags);   // [0]: any abort
 
     if (tid == 0) {
-        // a head's operands are ready once each of the 8 scale warps has arrived
+        // a head's operands are ready once each of the 8 scale warps has arrived;
+        // a slot's x/h and an accumulator are released by both MMA issuers
         for (int i = 0; i < BAR_COUNT; ++i)
-            mbar_init(&bars[i], (i >= BAR_MFULL && i < BAR_MFULL + 4) ? 8 : 1);
+            mbar_init(&bars[i], (i >= BAR_MFULL && i < BAR_MFULL + 4) ? 8
+                                : (z2 && ((i >= BAR_XEMPTY && i < BAR_XEMPTY + 4) ||
+                                          (i >= BAR_ACCFULL && i < BAR_ACCFULL + 2))) ? 2 : 1);
         s_flag[0] = 0;
         fence_mbar_init();
     }
@@ -322,15 +337,16 @@ __device__ __forceinline__ void body(const CUtensorMap* tmX, const CUtensorMap* 
                 const uint64_t hd = smem_desc_sw128(smem_u32(sH + s * S::kHTile), 16, 1024);
                 const bool fast = s_path[f] != 0;
                 // ZW (+)= C_t h~^T.  On the fast path h is used as loaded, so these
-                // MMAs go first, while the head's x rows are still being scaled; on
-                // the exact path h exp(r) is ready only with the rest.
+                // MMAs go first (or to the second issuer), while the head's x rows are
+                // still being scaled; on the exact path h exp(r) is ready only with
+                // the rest.
                 auto issue_z = [&](bool acc_first) {
 #pragma unroll
                     for (int ks = 0; ks < N / 16; ++ks)
                         mma_ss(acc + 64, cd + (uint64_t)((ks >> 2) * 1024 + (ks & 3) * 2),
                                hd + (uint64_t)((ks >> 2) * 512 + (ks & 3) * 2), idesc_z, acc_first || ks > 0);
                 };
-                if (fast) issue_z(false);
+                if (fast && !z2) issue_z(false);
                 ok = mbar_wait(&bars[BAR_MFULL + f], (uint32_t)((hi >> 2) & 1), status);
                 if (!ok) break;
                 tc_fence_after();
@@ -355,6 +371,35 @@ __device__ __forceinline__ void body(const CUtensorMap* tmX, const CUtensorMap* 
             }
             if (!ok) s_flag[0] = 1;
         }
+    } else if (warp == 14) {
+        // ================================================== second MMA issuer (ZW, fast path)
+        if (z2 && lane == 0) {
+            const uint32_t idesc_z = idesc_bf16_f32(128, 64, false, false);   // C, h both K-major
+            const uint64_t cd = smem_desc_sw128(smem_u32(sC), 16, 1024);
+            bool ok = mbar_wait(&bars[BAR_BC], 0, status);                  // C has landed
+            for (int hi = 0; hi < HG && ok; ++hi) {
+                const int s = hi & (R - 1);
+                const int a = hi & 1;
+                const int f = hi & 3;
+                ok = mbar_wait(&bars[BAR_ALFULL + f], (uint32_t)((hi >> 2) & 1), status) &&
+                     mbar_wait(&bars[BAR_XFULL + s], (uint32_t)((hi / R) & 1), status) &&
+                     (hi < 2 || mbar_wait(&bars[BAR_ACCEMPTY + a], (uint32_t)(((hi >> 1) - 1) & 1),
+                                          status));
+                if (!ok) break;
+                tc_fence_after();
+                if (s_path[f] != 0) {
+                    const uint32_t acc = tmem + kColAcc + 128 * a;
+                    const uint64_t hd = smem_desc_sw128(smem_u32(sH + s * S::kHTile), 16, 1024);
+#pragma unroll
+                    for (int ks = 0; ks < N / 16; ++ks)
+                        mma_ss(acc + 64, cd + (uint64_t)((ks >> 2) * 1024 + (ks & 3) * 2),
+                               hd + (uint64_t)((ks >> 2) * 512 + (ks & 3) * 2), idesc_z, ks > 0);
+                }
+                mma_commit(&bars[BAR_XEMPTY + s]);
+                mma_commit(&bars[BAR_ACCFULL + a]);
+            }
+            if (!ok) s_flag[0] = 1;
+        }
     } else if (warp < 8) {
         // ================================================== mask / scale warps (0-7)
         // Warp w owns TMEM lane quarter q = w % 4 (rows 32q..32q+31) and half
@@ -363,11 +408,25 @@ __device__ __forceinline__ void body(const CUtensorMap* tmX, const CUtensorMap* 
         const int m = q * 32 + lane;               // row within the tile
         const int i = row0 + m;                    // row within the chunk
         const uint32_t lane_base = (uint32_t)(q * 32) << 16;
-        // Thread tid < KJ holds dt of token tid for the head in turn, loaded one
-        // head ahead (the first one while the prologue runs).
-        const bool tok_in = tid < KJ && tid < len;
-        const float* dt_tok = dt + (b * L + t0 + tid) * Hr;
-        float dt_next = tok_in ? dt_tok[head0 / ksplit] : 0.f;
+        // The prefix sums of dt*A are taken for four heads at a time: warp w
+        // scans head slot k = w % 4 over half sg = w / 4 of the tile's KJ
+        // columns, a lane holding kPer = KJ / 64 consecutive tokens, whose dt
+        // it loads one batch of four heads ahead (the first while the
+        // prologue runs).
+        constexpr int kPerMax = Q / 64;
+        const int per = KJ / 64;
+        const int sk = warp & 3, sg = warp >> 2;
+        const int jseg = sg * (KJ / 2) + lane * per;          // this lane's first token
+        float dnext[kPerMax];
+        auto load_dt = [&](int hb) {                          // heads hb .. hb + 3
+#pragma unroll
+            for (int e = 0; e < kPerMax; ++e) {
+                const int j = jseg + e;
+                dnext[e] = (e < per && j < len && hb + sk < HG)
+                               ? dt[(b * L + t0 + j) * Hr + (head0 + hb + sk) / ksplit] : 0.f;
+            }
+        };
+        load_dt(0);
         if (tid < HG) {
             s_Ah[tid] = A[(head0 + tid) / ksplit] * kLog2e;
             s_Dh[tid] = Dv[(head0 + tid) / ksplit];
@@ -437,33 +496,50 @@ __device__ __forceinline__ void body(const CUtensorMap* tmX, const CUtensorMap* 
             for (int hi = 0; hi < HG; ++hi) {
                 const int s = hi & (R - 1);           // x/h ring slot
                 const int f = hi & 3;                 // factor slot and skip-term x slot
-                // factor slot f is free once the epilogue of head hi - 4 has read it
-                {
-                    // inclusive prefix sums of dt*A (log2 units) of this head over the
-                    // tile's KJ columns: a shuffle scan per warp, then the warp offsets
-                    const float dt_cur = dt_next;
-                    if (hi + 1 < HG) dt_next = tok_in ? dt_tok[(head0 + hi + 1) / ksplit] : 0.f;
-                    float v = dt_cur * s_Ah[hi];
+                if ((hi & 3) == 0) {
+                    // inclusive prefix sums of dt*A (log2 units) of heads hi .. hi + 3
+                    // over the tile's KJ columns: a shuffle scan per warp segment,
+                    // then the first segment's total as the second's offset.  The
+                    // slots written are those of heads hi - 4 .. hi - 1, which every
+                    // thread has finished with once it reaches the first barrier.
+                    float dcur[kPerMax], v[kPerMax];
+#pragma unroll
+                    for (int e = 0; e < kPerMax; ++e) dcur[e] = dnext[e];
+                    if (hi + 4 < HG) load_dt(hi + 4);
+                    const float Ak = hi + sk < HG ? s_Ah[hi + sk] : 0.f;
+                    float run = 0.f;
+#pragma unroll
+                    for (int e = 0; e < kPerMax; ++e) {
+                        run += dcur[e] * Ak;              // tokens past KJ or L add 0
+                        v[e] = run;
+                    }
+                    float incl = run;
 #pragma unroll
                     for (int o = 1; o < 32; o <<= 1) {
-                        const float u = __shfl_up_sync(0xffffffffu, v, o);
-                        if (lane >= o) v += u;
+                        const float u = __shfl_up_sync(0xffffffffu, incl, o);
+                        if (lane >= o) incl += u;
                     }
-                    if (lane == 31) s_ws[warp] = v;
-                    // (the barrier that publishes the warp sums also shares the verdict
-                    // of the factor slot's wait)
-                    fail = hi >= 4 && !mbar_wait(&bars[BAR_FEMPTY + f], (uint32_t)(((hi >> 2) - 1) & 1), status);
-                    if (named_bar_or(1, 256, fail)) break;
-                    float off = 0.f;
-                    for (int w2 = 0; w2 < warp; ++w2) off += s_ws[w2];
-                    if (tid < KJ) {
-                        s_cs[tid] = v + off;
-                        s_dt[tid] = dt_cur;
-                    }
+                    if (lane == 31) s_ws[warp] = incl;
+                    named_bar_sync(1, 256);
+                    const float off = (incl - run) + (sg ? s_ws[sk] : 0.f);
+                    float* csk = s_cs + sk * Q;
+                    float* dtk = s_dt + sk * Q;
+#pragma unroll
+                    for (int e = 0; e < kPerMax; ++e)
+                        if (e < per) {
+                            csk[jseg + e] = v[e] + off;
+                            dtk[jseg + e] = dcur[e];
+                        }
                     named_bar_sync(1, 256);
                 }
-                const float* cs = s_cs;
-                const float* hdt = s_dt;
+                // factor slot f is free once the epilogue of head hi - 4 has read it
+                // (each thread waits before writing it; the barrier that publishes
+                // the factors below also shares the outcome)
+                fail = hi >= 4 && !mbar_wait(&bars[BAR_FEMPTY + f], (uint32_t)(((hi >> 2) - 1) & 1), status);
+                const float* cs = s_cs + f * Q;
+                const float* hdt = s_dt + f * Q;
+                float* beta = s_beta + f * 128;
+                float* beta2 = s_beta2 + f * 128;
                 const float cs_i = cs[i];
                 const float r = (t == 1) ? cs[127] : 0.f;
                 // the tile's decay span decides the path (the same for every thread)
@@ -475,13 +551,13 @@ __device__ __forceinline__ void body(const CUtensorMap* tmX, const CUtensorMap* 
                 const bool fast = fabsf(c_last - c_first) <= kFastSpan &&
                                   (t == 0 || r1 - cs[0] <= 0.5f * kFastSpan);
                 if (hf == 0) {
-                    if (t == 1) s_beta[m] = fast_exp2((fast ? r1 : r) - cs[m]) * hdt[m];
+                    if (t == 1) beta[m] = fast_exp2((fast ? r1 : r) - cs[m]) * hdt[m];
                     s_al[f * 128 + m] = fast_exp2(fast ? cs_i : cs_i - r);
                     s_row[f * 128 + m] = fast ? fast_exp2(cs_i - r1) : 1.f;
                 } else {
                     // fast: b_j; exact: beta of j through the end of its 32-column block
                     const int j = row0 + m;
-                    s_beta2[m] = fast_exp2((fast ? r1 : cs[row0 + (m | 31)]) - cs[j]) * hdt[j];
+                    beta2[m] = fast_exp2((fast ? r1 : cs[row0 + (m | 31)]) - cs[j]) * hdt[j];
                 }
                 if (tid == 0) s_path[f] = fast ? 1 : 0;
                 // the exact path writes the mask slot: free once the MMAs of head hi - 1
@@ -490,7 +566,8 @@ __device__ __forceinline__ void body(const CUtensorMap* tmX, const CUtensorMap* 
                 // one head ahead of the MMAs, while the epilogue of head hi - 5 is
                 // known to be done, so this barrier lags by at most one phase); both
                 // paths need the head's x rows and entering state
-                fail = (!fast && hi >= 1 &&
+                fail = fail ||
+                       (!fast && hi >= 1 &&
                         !mbar_wait(&bars[BAR_FEMPTY + ((hi - 1) & 3)],
                                    (uint32_t)(((hi - 1) >> 2) & 1), status)) ||
                        !mbar_wait(&bars[BAR_XFULL + s], (uint32_t)((hi / R) & 1), status);
@@ -499,7 +576,7 @@ __device__ __forceinline__ void body(const CUtensorMap* tmX, const CUtensorMap* 
                 if (t == 1) {
                     // x rows 0..127 *= b_j (fast path) or beta_j (exact path), row j =
                     // piece / 8; on the exact path also h *= exp(r); in place
-                    scale_pieces<4>(sX + s * kXSlot, tid, [&](int k) { return s_beta[k >> 3]; });
+                    scale_pieces<4>(sX + s * kXSlot, tid, [&](int k) { return beta[k >> 3]; });
                     if (!fast) {
                         const float er = fast_exp2(r);
                         scale_pieces<S::kHTile / 4096>(sH + s * S::kHTile, tid, [&](int) { return er; });
@@ -526,7 +603,7 @@ __device__ __forceinline__ void body(const CUtensorMap* tmX, const CUtensorMap* 
                         tmem_st16(tmem + lane_base + col_xs(f) + 16 * hf, w);
                     }
                     if (fast) {
-                        const float bm = s_beta2[m];
+                        const float bm = beta2[m];
 #pragma unroll
                         for (int u = 0; u < 4; ++u) {
                             uint32_t* e4 = reinterpret_cast<uint32_t*>(&v[u]);
@@ -562,7 +639,7 @@ __device__ __forceinline__ void body(const CUtensorMap* tmX, const CUtensorMap* 
                         if (cb < q) {
                             // entirely below the diagonal: factorised through the block's end
                             const float alpha = fast_exp2(cs_i - cs[j0 + 31]);
-                            const float4* bet = reinterpret_cast<const float4*>(s_beta2 + 32 * cb);
+                            const float4* bet = reinterpret_cast<const float4*>(beta2 + 32 * cb);
 #pragma unroll
                             for (int u = 0; u < 8; ++u) {
                                 const float4 bv = bet[u];
@@ -588,9 +665,10 @@ __device__ __forceinline__ void body(const CUtensorMap* tmX, const CUtensorMap* 
                     tmem_st16(tmem + lane_base + kColM + 16 * cb, packed);
                 }
                 // Each warp reports its share (scaled rows, mask blocks) by itself.  No
-                // block barrier is needed here: the next head's first barrier keeps
-                // its writes of the single-buffered factors and sums after every
-                // warp is done with this head's.
+                // block barrier is needed here: the factors, sums and dt of a head
+                // live in slot hi % 4, which is rewritten only after the next batch
+                // scan's first barrier, and the shared mask slot (exact path) only
+                // after the next head's factor barrier.
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars[BAR_MFULL + f]);

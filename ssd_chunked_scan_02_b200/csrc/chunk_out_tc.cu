@@ -40,7 +40,7 @@ chunk_out_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
     const int64_t bt = bx / kTiles;
     extern __shared__ uint8_t smem_raw[];
     outk::body<Q, N>(&tmX, &tmB, &tmC, &tmH, &tmY, dt, A, Dv, L, H, G, T, HG, ksplit, bt / T,
-                     bt % T, t, (int)blockIdx.y * HG, align1024(smem_raw), nullptr, 1, status);
+                     bt % T, t, (int)blockIdx.y * HG, align1024(smem_raw), nullptr, 1, true, status);
 }
 
 template <int Q, int N>

@@ -40,7 +40,7 @@ namespace {
 using namespace sm100;
 
 constexpr int kThreads = outk::kThreads;
-static_assert(walk::Roles<4>::kThreads == outk::kThreads, "one block size for both roles");
+static_assert(walk::Roles<4>::kThreads <= outk::kThreads, "one block size for both roles");
 static_assert(walk::Roles<2>::kThreads <= outk::kThreads, "one block size for both roles");
 
 template <int Q, int N, int HP>
@@ -136,7 +136,7 @@ walk_out_tc_kernel(const __grid_constant__ CUtensorMap tmXw, const __grid_consta
         const int r2 = (int)(r - b * (kTiles * nhg));
         const int t = r2 / nhg, hg = r2 - t * nhg;
         outk::body<Q, N>(&tmX, &tmB, &tmC, &tmH, &tmY, dt, A, Dv, L, H, G, T, hgs, ksplit, b, c,
-                         t, hg * hgs, smem, progress, HP, status);
+                         t, hg * hgs, smem, progress, HP, false, status);
     }
 }
 
