@@ -310,6 +310,34 @@ def test_fused_walk_output_full_forward(case):
     ssd.ssd_poll_device_status()       # raises if a bounded wait gave up
 
 
+def test_fused_flow_without_states_and_workspace_reuse():
+    """The one-launch flow with neither initial nor final states (y only),
+    then two different inputs through one workspace: the scheduling counters
+    are reset before every launch, so the second call starts clean."""
+    w = _w("fused_nostates", 8, 1100, 24, 64, 128, 1, 256, "bf16", False, seed=40)
+    inp = inputs.make_inputs(w)
+    y, f = gpu_fwd(inp, 256, want_final=False, flow=ssd.SSD_FLOW_WALK_OUTPUT_FUSED)
+    assert f is None
+    y_ref, _ = oracle_fwd(inp)
+    assert rel_err(y, y_ref) <= TOL["bf16"]
+    dims = ssd.make_dims(w.batch, w.seqlen, w.nheads, w.headdim, w.dstate, w.ngroups)
+    n = ssd.ssd_chunk_scan_fwd_workspace_size(dims, 256, torch.bfloat16,
+                                              flow=ssd.SSD_FLOW_WALK_OUTPUT_FUSED)
+    ws = torch.empty(n, device="cuda", dtype=torch.uint8)
+    for seed in (41, 42):
+        wi = _w("fused_reuse", 8, 1100, 24, 64, 128, 1, 256, "bf16", True, seed=seed)
+        inp = inputs.make_inputs(wi)
+        d = to_dev(inp)
+        y, f = ssd.ssd_chunk_scan_fwd(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], 256,
+                                      init_states=d["init"], return_final_states=True,
+                                      workspace=ws, flow=ssd.SSD_FLOW_WALK_OUTPUT_FUSED)
+        torch.cuda.synchronize()
+        y_ref, f_ref = oracle_fwd(inp)
+        assert rel_err(y.double().cpu().numpy(), y_ref) <= TOL["bf16"], seed
+        assert rel_err(f.double().cpu().numpy(), f_ref) <= TOL["bf16"], seed
+    ssd.ssd_poll_device_status()
+
+
 def test_fused_flow_taken_for_long_sequences():
     """With 8 chunks or more the forward takes the one-launch flow by itself
     (16 chunks, ragged last chunk; every element checked)."""
