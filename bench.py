@@ -19,6 +19,7 @@ import argparse
 import hashlib
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -101,12 +102,21 @@ KERNEL_SOURCES = {
 }
 
 
+def code_text(src: str) -> str:
+    """A CUDA source with its comments removed and its whitespace collapsed:
+    what a kernel's DRAM traffic can depend on."""
+    src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", " ", src)
+    return " ".join(src.split())
+
+
 def source_sha(kernel: str) -> str:
     h = hashlib.sha256()
     for f in KERNEL_SOURCES[kernel]:
         p = os.path.join(ROOT, "ssd_chunked_scan_02_b200", "csrc", f)
         if os.path.exists(p):
-            h.update(open(p, "rb").read())
+            with open(p) as fh:
+                h.update(code_text(fh.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -44,7 +44,7 @@
 // scale a head's x rows in shared memory first copy them, unscaled, to one of
 // four TMEM slots.
 //
-// Roles (448 threads):
+// Roles (480 threads, 15 warps):
 //   warps 0-7   prologue: G = C_t B^T (M = 128, N = 128 (t+1), K = dstate) is
 //               copied from TMEM: the diagonal block becomes G o causal in bf16
 //               (TMEM, the A operand of Y), the block to its left goes to
