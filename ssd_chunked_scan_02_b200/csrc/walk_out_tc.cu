@@ -13,8 +13,8 @@
 //
 // Scheduling.  Every CTA first takes a ticket (one atomic add on a counter
 // the host zeroes before the launch).  Tickets 0 .. W-1 are the walkers, one
-// per (batch, HP heads of one group: four for dstate 128 when walkers of two
-// would not leave SMs for the tiles, else two), each holding an SM to itself;
+// per (batch, HP heads of one group: four for dstate 128, two for dstate
+// 64), each holding an SM to itself;
 // tickets W and up are output tiles in chunk-major order.  A walker waits on
 // nothing outside its CTA.  An output tile waits (bounded, like every wait
 // here) only on walkers, and only for walkers whose tickets were taken before
@@ -63,12 +63,15 @@ struct Cfg {
 
 Cfg config(const Dims& v) {
     Cfg c;
-    const int64_t hpg = v.H / v.G;
-    const int64_t pairs = v.b * v.G * ((hpg + 1) / 2);
-    // walkers of two heads walk faster (4.5 against 6 us a chunk) but must
-    // leave SMs for the output tiles; four heads (dstate 128 only) halve them
-    c.hp = (v.N == 128 && pairs > 100) ? 4 : 2;
+    // walkers of two heads walk faster (4.5 against 6 us a chunk) but take
+    // twice the SMs from the output tiles; with dstate 128 (a walker of four
+    // heads fits TMEM) four heads come out ahead at every measured size
+    c.hp = (v.N == 128) ? 4 : 2;
     c.hg = outk::pick_heads_per_cta(v.H, v.G);
+    // enough output tiles to spread over the SMs: halve the heads a tile
+    // while the launch has fewer than 256 tiles
+    while (c.hg % 2 == 0 && c.hg >= 8 && v.b * v.T * (v.Q / 128) * (v.H / c.hg) < 256)
+        c.hg /= 2;
     c.ks = (c.hg % 2 == 0 && c.hg >= 8 && v.T > 2) ? 2 : 0;
     c.hg2 = c.ks ? c.hg / 2 : c.hg;
     return c;
@@ -225,8 +228,6 @@ cudaError_t launch_walk_out_tc(const void* x, const float* dt, const float* A, c
                                         k, pc, cf, s);
     SSD_WALK_OUT(256, 128, 4)
     SSD_WALK_OUT(128, 128, 4)
-    SSD_WALK_OUT(256, 128, 2)
-    SSD_WALK_OUT(128, 128, 2)
     SSD_WALK_OUT(256, 64, 2)
     SSD_WALK_OUT(128, 64, 2)
 #undef SSD_WALK_OUT

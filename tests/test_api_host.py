@@ -139,11 +139,11 @@ def test_forced_flow_workspace_and_rejections(lib):
     three = _round(4 * ns) + _round(8 * T * 24 * 4) + _round(2 * ns)
     assert ws(d, 256, ssd.SSD_FLOW_TC_THREE_KERNEL)[1] == three
     assert ws(d, 256, ssd.SSD_FLOW_SIMT)[1] == three
-    # walkers of two heads below 100 pairs: 96 walkers, then 32 + 96 counters
-    assert ws(d, 256, ssd.SSD_FLOW_WALK_OUTPUT_FUSED)[1] == _round(2 * ns) + _round((32 + 96) * 4)
-    odd = ssd.make_dims(16, 600, 10, 64, 128, 2)            # 5 heads a group: 3 walkers a group
+    # walkers of four heads (dstate 128): 48 walkers, then 32 + 48 counters
+    assert ws(d, 256, ssd.SSD_FLOW_WALK_OUTPUT_FUSED)[1] == _round(2 * ns) + _round((32 + 48) * 4)
+    odd = ssd.make_dims(16, 600, 10, 64, 128, 2)            # 5 heads a group: 2 walkers a group
     assert ws(odd, 256, ssd.SSD_FLOW_WALK_OUTPUT_FUSED)[1] == \
-        _round(16 * 3 * 10 * 64 * 128 * 2) + _round((32 + 16 * 2 * 3) * 4)
+        _round(16 * 3 * 10 * 64 * 128 * 2) + _round((32 + 16 * 2 * 2) * 4)
     n64 = ssd.make_dims(8, 2048, 24, 64, 48, 1)             # dstate 48: SIMT only
     assert ws(n64, 256, ssd.SSD_FLOW_WALK_OUTPUT_FUSED)[0] == ssd.SSD_ERR_UNSUPPORTED
     p96 = ssd.make_dims(2, 600, 4, 96, 128, 1)              # no tensor cores

@@ -281,17 +281,19 @@ def test_walk_path_full_forward_ragged_groups(case):
 
 FUSED_FWD_CASES = [
     # name,                 b,  L,    H,  P,   N,  G,  Q,  init
-    ("fused_n128_g2", 8, 900, 40, 64, 128, 2, 256, True),       # 4 chunks, last one partial
+    ("fused_n128_g2", 8, 900, 40, 64, 128, 2, 256, True),       # 4 chunks, last one partial;
+                                                                # tiles of 10, then 5 heads
     ("fused_q128_p128", 8, 1000, 24, 128, 128, 1, 128, True),   # 48 virtual heads, 8 chunks
     ("fused_p32", 8, 600, 48, 32, 128, 1, 256, False),          # headdim 32 (zero-padded)
-    ("fused_tile_heads_18", 6, 700, 36, 64, 128, 1, 256, True),  # tiles of 18 heads: a walker's
-                                                                 # four heads split between tiles
+    ("fused_tile_heads_9", 6, 700, 36, 64, 128, 1, 256, True),  # tiles of 9 heads: a walker's
+                                                                # four heads split between tiles
     ("fused_192_walkers", 48, 520, 16, 64, 128, 1, 256, True),  # more walkers than SMs
     ("fused_one_chunk", 4, 200, 8, 64, 128, 1, 256, True),      # a single (partial) chunk
-    ("fused_few_walkers", 1, 1300, 4, 64, 128, 1, 256, True),   # walkers of two heads
+    ("fused_few_walkers", 1, 1300, 4, 64, 128, 1, 256, True),   # a single walker
     ("fused_quad_phantoms", 40, 300, 6, 64, 128, 1, 256, True),  # walkers of four heads, 6 a
                                                                  # group: two phantom heads
-    ("fused_pair_phantom", 16, 600, 10, 64, 128, 2, 256, True),  # walkers of two, 5 heads a group
+    ("fused_three_phantoms", 16, 600, 10, 64, 128, 2, 256, True),  # 5 heads a group: the second
+                                                                   # walker has one real head
     ("fused_n64", 16, 1100, 12, 64, 64, 2, 128, True),          # dstate 64 (walkers of two)
 ]
 
