@@ -295,6 +295,8 @@ FUSED_FWD_CASES = [
     ("fused_three_phantoms", 16, 600, 10, 64, 128, 2, 256, True),  # 5 heads a group: the second
                                                                    # walker has one real head
     ("fused_n64", 16, 1100, 12, 64, 64, 2, 128, True),          # dstate 64 (walkers of two)
+    ("fused_tiles_halved", 2, 2300, 32, 64, 128, 1, 256, True),  # 9 chunks, few tiles: heads a
+                                                                 # tile halved 32 -> 4
 ]
 
 
