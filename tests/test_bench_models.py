@@ -58,3 +58,13 @@ def test_backward_bytes():
     reads = b * L * (2 * H * P * 2 + 2 * N * 2 + 4 * H)
     writes = b * L * (H * P * 4 + 4 * H + 2 * N * 4)
     assert bench.bwd_bytes(inputs.LAYER_130M) == reads + writes + 4 * b * H * P * N == 235929600
+
+
+def test_traffic_records_follow_code_not_comments():
+    """A recorded DRAM traffic figure stays valid while a kernel's code is
+    unchanged: the source hash ignores comments and whitespace, but not code."""
+    src = "int f(int a) {\n    // scale\n    return a * 2; /* twice */\n}\n"
+    same = "int f(int a) {   return a * 2;\n}  // reworded comment\n"
+    other = "int f(int a) {\n    return a * 3;\n}\n"
+    assert bench.code_text(src) == bench.code_text(same)
+    assert bench.code_text(src) != bench.code_text(other)
