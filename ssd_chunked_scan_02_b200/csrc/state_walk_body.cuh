@@ -56,6 +56,68 @@ namespace ssd {
 namespace walk {
 using namespace sm100;
 
+// Split forms for software pipelining: a TMEM load without its wait, the wait
+// that orders every later use of the loaded registers (they are its in/out
+// operands, so no use can be scheduled above it), a TMEM store without its
+// wait (the source registers are read when the store issues; later
+// instructions may reuse them) and the wait for all of this thread's stores.
+__device__ __forceinline__ void tmem_ld32x2_nowait(uint32_t ta, uint32_t tb, uint32_t (&ra)[32],
+                                                   uint32_t (&rb)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%64];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
+        "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%65];"
+        : "=r"(ra[0]), "=r"(ra[1]), "=r"(ra[2]), "=r"(ra[3]), "=r"(ra[4]), "=r"(ra[5]),
+          "=r"(ra[6]), "=r"(ra[7]), "=r"(ra[8]), "=r"(ra[9]), "=r"(ra[10]), "=r"(ra[11]),
+          "=r"(ra[12]), "=r"(ra[13]), "=r"(ra[14]), "=r"(ra[15]), "=r"(ra[16]), "=r"(ra[17]),
+          "=r"(ra[18]), "=r"(ra[19]), "=r"(ra[20]), "=r"(ra[21]), "=r"(ra[22]), "=r"(ra[23]),
+          "=r"(ra[24]), "=r"(ra[25]), "=r"(ra[26]), "=r"(ra[27]), "=r"(ra[28]), "=r"(ra[29]),
+          "=r"(ra[30]), "=r"(ra[31]), "=r"(rb[0]), "=r"(rb[1]), "=r"(rb[2]), "=r"(rb[3]),
+          "=r"(rb[4]), "=r"(rb[5]), "=r"(rb[6]), "=r"(rb[7]), "=r"(rb[8]), "=r"(rb[9]),
+          "=r"(rb[10]), "=r"(rb[11]), "=r"(rb[12]), "=r"(rb[13]), "=r"(rb[14]), "=r"(rb[15]),
+          "=r"(rb[16]), "=r"(rb[17]), "=r"(rb[18]), "=r"(rb[19]), "=r"(rb[20]), "=r"(rb[21]),
+          "=r"(rb[22]), "=r"(rb[23]), "=r"(rb[24]), "=r"(rb[25]), "=r"(rb[26]), "=r"(rb[27]),
+          "=r"(rb[28]), "=r"(rb[29]), "=r"(rb[30]), "=r"(rb[31])
+        : "r"(ta), "r"(tb)
+        : "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld64(uint32_t (&ra)[32], uint32_t (&rb)[32]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(ra[0]), "+r"(ra[1]), "+r"(ra[2]), "+r"(ra[3]), "+r"(ra[4]), "+r"(ra[5]),
+                   "+r"(ra[6]), "+r"(ra[7]), "+r"(ra[8]), "+r"(ra[9]), "+r"(ra[10]),
+                   "+r"(ra[11]), "+r"(ra[12]), "+r"(ra[13]), "+r"(ra[14]), "+r"(ra[15]),
+                   "+r"(ra[16]), "+r"(ra[17]), "+r"(ra[18]), "+r"(ra[19]), "+r"(ra[20]),
+                   "+r"(ra[21]), "+r"(ra[22]), "+r"(ra[23]), "+r"(ra[24]), "+r"(ra[25]),
+                   "+r"(ra[26]), "+r"(ra[27]), "+r"(ra[28]), "+r"(ra[29]), "+r"(ra[30]),
+                   "+r"(ra[31]), "+r"(rb[0]), "+r"(rb[1]), "+r"(rb[2]), "+r"(rb[3]), "+r"(rb[4]),
+                   "+r"(rb[5]), "+r"(rb[6]), "+r"(rb[7]), "+r"(rb[8]), "+r"(rb[9]), "+r"(rb[10]),
+                   "+r"(rb[11]), "+r"(rb[12]), "+r"(rb[13]), "+r"(rb[14]), "+r"(rb[15]),
+                   "+r"(rb[16]), "+r"(rb[17]), "+r"(rb[18]), "+r"(rb[19]), "+r"(rb[20]),
+                   "+r"(rb[21]), "+r"(rb[22]), "+r"(rb[23]), "+r"(rb[24]), "+r"(rb[25]),
+                   "+r"(rb[26]), "+r"(rb[27]), "+r"(rb[28]), "+r"(rb[29]), "+r"(rb[30]),
+                   "+r"(rb[31])
+                 :
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_st32_nowait(uint32_t taddr, const uint32_t (&r)[32]) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+                 "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+                 "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
+                 ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]),
+                   "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]),
+                   "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]),
+                   "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
+                   "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]),
+                   "r"(r[31])
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() {
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
 constexpr int kSub = 64;                 // tokens per ring entry
 constexpr int kPrefetch = 6;             // L2 prefetch distance, in ring entries
 
@@ -445,27 +507,28 @@ __device__ __forceinline__ void body(const CUtensorMap* tmX, const CUtensorMap* 
             for (int k = 0; k < HP; ++k) av[k] = s_a[cb * HP + k];
             named_bar_sync(2, 128);
             if (m == 0) mbar_arrive(&bars[BAR_AFREE + cb]);
-            // pass 1: h' = a h + S in TMEM (h' over h); then S is free for the next chunk
+            // pass 1: h' = a h + S in TMEM (h' over h); then S is free for the next
+            // chunk.  Per 32-column block: the update in place in the loaded
+            // registers, its store issued without a wait, then the next block's
+            // loads; one wait for all the stores at the end.
             {
                 const int nk = kTrans ? 2 * HP : N / 32;
+                uint32_t hr[32], sr[32];
+                tmem_ld32x2_nowait(tH, tS, hr, sr);
 #pragma unroll 1
                 for (int cc = 0; cc < nk; ++cc) {
+                    tmem_wait_ld64(hr, sr);
                     const int k = kTrans ? (cc >> 1) : (m >> 6);
                     float a = av[0];
 #pragma unroll
                     for (int kk = 1; kk < HP; ++kk) a = (k == kk) ? av[kk] : a;
-                    uint32_t hr[32], sr[32];
-                    tmem_ld32x2(tH + cc * 32, tS + cc * 32, hr, sr);
-                    uint32_t lo[16], hi[16];
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        lo[e] = __float_as_uint(fmaf(a, __uint_as_float(hr[e]), __uint_as_float(sr[e])));
-                        hi[e] = __float_as_uint(
-                            fmaf(a, __uint_as_float(hr[16 + e]), __uint_as_float(sr[16 + e])));
-                    }
-                    tmem_st16(tH + cc * 32, lo);
-                    tmem_st16(tH + cc * 32 + 16, hi);
+                    for (int e = 0; e < 32; ++e)
+                        hr[e] = __float_as_uint(fmaf(a, __uint_as_float(hr[e]), __uint_as_float(sr[e])));
+                    tmem_st32_nowait(tH + cc * 32, hr);
+                    if (cc + 1 < nk) tmem_ld32x2_nowait(tH + (cc + 1) * 32, tS + (cc + 1) * 32, hr, sr);
                 }
+                tmem_wait_st();
             }
             tc_fence_before();
             named_bar_sync(2, 128);
